@@ -1,0 +1,11 @@
+"""fp64 CPU oracle for LiteLA.  Test infrastructure: imported only by the tests, the
+package smoke check and the benchmark's CPU-baseline leg; never by the product path."""
+from .litela_oracle import (  # noqa: F401
+    decode_bf16,
+    unpack_qkv,
+    relu,
+    lite_la_rows,
+    lite_la_fwd,
+    lite_la_block_causal_fwd,
+    visible_key_count,
+)
