@@ -1,0 +1,442 @@
+#!/usr/bin/env python
+"""LiteLA forward benchmark on B200 (one JSON line on stdout, rank 0).
+
+Workload (default): Sana 4096px LiteLA forward, B=2, N=128*128=16384 tokens, H=70 heads of
+d=32, packed bf16 qkv drawn i.i.d. N(0,1) from seeds 4000..4059, eps=1e-15.  One step is 60
+back-to-back calls on 60 distinct input buffers (the 60 self-attention layers of the 4.8B
+model per sampling step).  Every call's input (440 MB) is larger than the 126 MB L2, so no
+flush is needed between calls.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 it runs under torch.distributed.run, one rank per GPU, each rank doing the same
+per-GPU workload (weak scaling; the calls are independent, there is no data-path
+collective).  Timing: CUDA events on the launching stream, barrier + synchronize on both
+sides, max over ranks.  `--impl reference` times the fp64 CPU oracle (the only reference
+this method has) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOADS_BENCH = {
+    # name: (B, N, H, calls per step, seed base)
+    "sana4800m_4096px_x60": (2, 128 * 128, 70, 60, 4000),
+    # one 4096px call per step on one buffer: the small case for detailed ncu captures
+    "sana4800m_4096px_x1": (2, 128 * 128, 70, 1, 4000),
+    "sana1600m_1024px": (2, 32 * 32, 70, 20, 1001),
+    "sana1600m_2048px": (2, 64 * 64, 70, 20, 1002),
+}
+D = 32
+EPS = 1e-15
+METRIC = "LiteLA fwd tokens·heads/s and µs/call at 4096px; % of HBM/FMA roofline"
+UNIT = "tokens·heads/s"
+FP32_LANES_PER_SM = 128          # B200: 4 SM sub-partitions x 32 fp32 lanes
+NUM_SMS = 148
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
+# name of each kernel the library launches per call, in launch order
+KERNELS = ("litela_reduce_simt", "litela_apply_simt")
+KERNEL_BOUND = {"litela_reduce_simt": "alu", "litela_apply_simt": "alu"}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["_source"] = "measured"
+        return d
+    d = dict(PEAKS_FALLBACK)
+    d["_source"] = "fallback"
+    return d
+
+
+def fp32_fma_peak_tflops(mhz):
+    return NUM_SMS * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during a timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid):
+        self.uuid, self.proc, self.path = gpu_uuid, None, None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or self.path is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 8:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        power = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(power) if power else None}
+
+
+def clocks_rejected(c):
+    bad = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+    if bad & set(c.get("reasons", [])):
+        return True
+    if c.get("sm_mhz") and c.get("sm_max_mhz") and c["sm_mhz"] < 0.5 * c["sm_max_mhz"] \
+            and "sw_power_cap" not in c.get("reasons", []):
+        return True
+    return False
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n and n[0]:
+            return int(n[0])
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def one_head_bits(qkv_bits, B, N, H, b, h):
+    """Packed [1, N, 3*d] bits of head h of batch b (input re-packing only)."""
+    import numpy as np
+    x = qkv_bits.reshape(B, N, 3, H, D)[b, :, :, h, :]
+    return np.ascontiguousarray(x.reshape(1, N, 3 * D))
+
+
+def oracle_head_rate(qkv_bits, B, N, H, seconds, max_heads=None):
+    """Times the fp64 oracle on whole heads (all N queries of one (batch, head)) until
+    `seconds` have passed; returns (tokens*heads per second, heads done, elapsed)."""
+    import oracle
+    heads, t0 = 0, time.perf_counter()
+    while True:
+        b, h = divmod(heads % (B * H), H)
+        oracle.lite_la_fwd(one_head_bits(qkv_bits, B, N, H, b, h), 1, N, 1, D, EPS)
+        heads += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_heads and heads >= max_heads):
+            return heads * N / el, heads, el
+
+
+def emit(line):
+    print(json.dumps(line), flush=True)
+
+
+def run_reference(args, wl):
+    """Reference arm: the fp64 oracle on the host cores, one whole head per step."""
+    import numpy as np
+    import torch
+    from linear_attention_diffusion_litela_b200.inputs import make_qkv, to_bits
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    B, N, H, calls, seed = WORKLOADS_BENCH[wl]
+    bits = to_bits(make_qkv(B, N, H, D, seed=seed, device="cpu"))
+    import oracle
+    heads = [(i // H % B, i % H) for i in range(args.warmup + args.steps)]
+    for i in range(args.warmup):
+        oracle.lite_la_fwd(one_head_bits(bits, B, N, H, *heads[i]), 1, N, 1, D, EPS)
+    times = []
+    for i in range(args.steps):
+        hb = one_head_bits(bits, B, N, H, *heads[args.warmup + i])
+        t0 = time.perf_counter()
+        oracle.lite_la_fwd(hb, 1, N, 1, D, EPS)
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * float(np.mean(times))
+    value = N / (ms / 1e3)
+    sample = "one whole (batch, head) per step: all %d queries against all %d keys" % (N, N)
+    emit({"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+          "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+          "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+          "data": "synthetic: i.i.d. N(0,1) bf16 qkv, seed %d" % seed,
+          "config": config_of(wl),
+          "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                           "sample": sample},
+          "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
+    return 0
+
+
+def config_of(wl):
+    B, N, H, calls, seed = WORKLOADS_BENCH[wl]
+    return {"workload": wl, "B": B, "N": N, "H": H, "d": D, "calls_per_step": calls,
+            "distinct_input_buffers": calls, "eps": EPS, "layout": "qkv bf16 [B,N,3*H*d], out bf16 [B,N,H*d]",
+            "l2": "inputs larger than L2 (%.0f MB per call vs 126 MB), no flush" % (B * N * 3 * H * D * 2 / 1e6)}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=list(WORKLOADS_BENCH), default="sana4800m_4096px_x60")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args, args.workload)
+
+    import ctypes
+
+    import numpy as np
+    import torch
+    import linear_attention_diffusion_litela_b200 as ll
+    from linear_attention_diffusion_litela_b200.inputs import make_qkv, to_bits
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE %d (launch N>1 with torch.distributed.run)" % (args.gpus, world))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    lib = ll.lib()
+    B, N, H, calls, seed0 = WORKLOADS_BENCH[args.workload]
+    qkv_bytes, out_bytes = B * N * 3 * H * D * 2, B * N * H * D * 2
+    free, _ = torch.cuda.mem_get_info(dev)
+    need = calls * (qkv_bytes + out_bytes) + (2 << 30)
+    if free < need:
+        raise SystemExit("not enough free GPU memory: need %.1f GB, free %.1f GB" % (need / 1e9, free / 1e9))
+    seeds = [seed0 + i for i in range(calls)] if args.workload.startswith("sana4800m") else [seed0 * 10 + i for i in range(calls)]
+    if world > 1:
+        seeds = [s + 100000 * rank for s in seeds]
+    ins = [make_qkv(B, N, H, D, seed=s, device=dev) for s in seeds]
+    outs = [torch.empty((B, N, H * D), dtype=torch.bfloat16, device=dev) for _ in range(calls)]
+    stream = torch.cuda.current_stream(dev)
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    in_p = [t.data_ptr() for t in ins]
+    out_p = [t.data_ptr() for t in outs]
+    fwd = lib.lite_la_fwd
+
+    def step():
+        for i in range(calls):
+            s = fwd(in_p[i], out_p[i], B, N, H, D, EPS, sh)
+            if s != 0:
+                raise ll.LiteLAError(s, lib.lite_la_last_error().decode())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+
+    def timed(fn, K):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        with ClockSampler(uuid) as cs:
+            e0.record(stream)
+            for _ in range(K):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+        barrier()
+        return e0.elapsed_time(e1), cs.summary()
+
+    ms_total, clocks = timed(step, args.steps)
+    rejected = None
+    if clocks_rejected(clocks):
+        rejected = clocks
+        ms_total, clocks = timed(step, args.steps)
+    ms_total = max_over_ranks(ms_total)
+    ms_step = ms_total / args.steps
+    us_call = 1e3 * ms_step / calls
+    tokens_heads = B * N * H * calls * args.steps * world
+    value = tokens_heads / (ms_total / 1e3)
+
+    # per-kernel durations: the same calls through lite_la_fwd_events (3 events per call)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(calls)]
+    for trip in evs:                      # recording once creates the underlying CUDA events
+        for e in trip:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
+    ev_handles = [(ctypes.c_void_p * 3)(*[ctypes.c_void_p(e.cuda_event) for e in trip]) for trip in evs]
+    kern_ms = {k: 0.0 for k in KERNELS}
+    nlaunch = 0
+    for _ in range(args.steps):
+        for i in range(calls):
+            s = lib.lite_la_fwd_events(in_p[i], out_p[i], B, N, H, D, EPS, sh, ev_handles[i])
+            if s != 0:
+                raise ll.LiteLAError(s, lib.lite_la_last_error().decode())
+        torch.cuda.synchronize(dev)
+        for trip in evs:
+            kern_ms[KERNELS[0]] += trip[0].elapsed_time(trip[1])
+            kern_ms[KERNELS[1]] += trip[1].elapsed_time(trip[2])
+        nlaunch += calls
+    kern_us = {k: 1e3 * v / nlaunch for k, v in kern_ms.items()}
+    E = B * N * H * D
+    flops_per_kernel = 2 * B * H * N * D * (D + 1)
+    alg_bytes = {KERNELS[0]: 4 * E, KERNELS[1]: 4 * E}
+    peaks = load_peaks()
+    dom = max(kern_us, key=kern_us.get)
+    bound = KERNEL_BOUND[dom]
+    traffic = load_traffic(dom)
+    if bound == "hbm":
+        achieved = alg_bytes[dom] / (kern_us[dom] * 1e-6) / 1e9
+        peak, unit = peaks["hbm_gbs"], "GB/s"
+        peak_note = "%s copy bandwidth" % peaks["_source"]
+    else:
+        achieved = flops_per_kernel / (kern_us[dom] * 1e-6) / 1e12
+        peak, unit = fp32_fma_peak_tflops(peaks.get("sm_max_mhz", 1965.0)), "TFLOP/s"
+        peak_note = "fp32 FMA: 148 SMs x 128 lanes x 2 x %.0f MHz max clock" % peaks.get("sm_max_mhz", 1965.0)
+    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                "traffic": traffic, "kernel": dom, "kernel_us": kern_us[dom],
+                "alg_bytes_per_launch": alg_bytes[dom], "alg_flops_per_launch": flops_per_kernel,
+                "peak_source": peak_note, "kernel_us_all": kern_us}
+    # the call as a whole against the slower of the HBM and fp32-FMA bounds
+    t_hbm = 8 * E / (peaks["hbm_gbs"] * 1e9) * 1e6
+    t_fma = 4 * B * H * N * D * (D + 1) / (fp32_fma_peak_tflops(peaks.get("sm_max_mhz", 1965.0)) * 1e12) * 1e6
+    call_roof = {"t_hbm_us": t_hbm, "t_fma_us": t_fma, "t_roof_us": max(t_hbm, t_fma),
+                 "us_per_call": us_call, "frac": max(t_hbm, t_fma) / us_call}
+    if clocks.get("sm_mhz"):
+        t_fma_clk = t_fma * peaks.get("sm_max_mhz", 1965.0) / clocks["sm_mhz"]
+        call_roof["t_fma_us_at_measured_clock"] = t_fma_clk
+        call_roof["frac_at_measured_clock"] = max(t_hbm, t_fma_clk) / us_call
+
+    # end to end: pinned host input -> device, forward, device -> pinned host output, per call
+    e2e = None
+    if args.e2e_steps > 0:
+        nbuf = 2
+        h_in = [torch.empty((B, N, 3 * H * D), dtype=torch.bfloat16, pin_memory=True) for _ in range(nbuf)]
+        h_out = [torch.empty((B, N, H * D), dtype=torch.bfloat16, pin_memory=True) for _ in range(nbuf)]
+        for j in range(nbuf):
+            h_in[j].copy_(ins[j])
+
+        def e2e_step():
+            for i in range(calls):
+                j = i % nbuf
+                ins[j].copy_(h_in[j], non_blocking=True)
+                s = fwd(in_p[j], out_p[j], B, N, H, D, EPS, sh)
+                if s != 0:
+                    raise ll.LiteLAError(s, lib.lite_la_last_error().decode())
+                h_out[j].copy_(outs[j], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        e2e_ms, _ = timed(e2e_step, args.e2e_steps)
+        e2e_ms = max_over_ranks(e2e_ms)
+        e2e = {"value": B * N * H * calls * args.e2e_steps * world / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": calls * qkv_bytes, "d2h_bytes_per_step": calls * out_bytes,
+               "ms_per_step": e2e_ms / args.e2e_steps, "steps": args.e2e_steps,
+               "how": "per call: pinned host qkv -> device copy, lite_la_fwd, device -> pinned host out copy, one stream"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        bits = to_bits(ins[0])
+        rate, heads, el = oracle_head_rate(bits, B, N, H, args.cpu_seconds)
+        cpu = {"value": rate, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+               "sample": "%d whole (batch, head) pairs of input buffer 0 (all %d queries x %d keys each), %.1f s"
+                         % (heads, N, N, el)}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "us_per_call": us_call,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic: i.i.d. N(0,1) bf16 qkv from seeded torch generators",
+                "config": config_of(args.workload), "roofline": roofline, "call_roofline": call_roof,
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": len(KERNELS) * calls * args.steps,
+                "clocks": clocks, "gpu": torch.cuda.get_device_name(dev)}
+        if world > 1:
+            line["config"]["parallelism"] = "dp%d (independent calls per rank, no collective)" % world
+        if rejected is not None:
+            line["clocks_rejected_first_run"] = rejected
+        emit(line)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def load_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when there is
+    none or the kernel sources changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(kernel)
+    if not ent or ent.get("sources_sha256") != sources_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def sources_hash():
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_attention_diffusion_litela_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,105 @@
+/*
+ * liblitela — LiteLA forward (Sana's ReLU linear self-attention) for NVIDIA B200 (sm_100a).
+ *
+ * The operation (Sana explainer "Sana: the autoencoder does more of the work than the linear
+ * attention", section "What LiteLA actually computes"; instagit page "How Linear Attention
+ * Improves Efficiency in DiT for High-Resolution Images", sections "Mathematical Foundation"
+ * and "Implementation Details"): for every (batch b, head h), with phi = ReLU applied to q and
+ * k only and V padded with a row of ones,
+ *
+ *     S    = [V ; 1] . phi(K)^T                  a (d+1) x d state, accumulated in fp32
+ *     y_n  = S . phi(q_n)                         d+1 values per query token n
+ *     out_n[r] = y_n[r] / (y_n[d] + eps)          r = 0 .. d-1
+ *
+ * which equals sum_j w_nj v_j / (sum_j w_nj + eps) with w_nj = phi(q_n).phi(k_j).
+ *
+ * Layouts (all row-major, densely packed, no padding between rows):
+ *   qkv : bf16 [B, N, 3*H*d]; one token row is [q | k | v], each head-major, i.e. element
+ *         (b, n, h, c) of q, k, v is at ((b*N + n)*3*H + {0, 1, 2}*H + h)*d + c.
+ *   out : [B, N, H*d]; element (b, n, h, c) at ((b*N + n)*H + h)*d + c; bf16 (round to
+ *         nearest even) for the plain entry points, fp32 for the *_f32out ones.
+ *
+ * Ownership: the caller owns qkv and out (device memory, at least 16-byte aligned, not
+ * overlapping).  The library owns a per-(device, stream) workspace of partial states (a few
+ * MB, see lite_la_workspace_bytes) that it allocates on first use, grows on demand (both after
+ * synchronising that stream, so the first call with a new size must not happen during graph
+ * capture) and keeps until lite_la_release_workspace().  Calls are asynchronous with respect to
+ * the host; calls on one stream are ordered by that stream, calls on different streams use
+ * different workspaces.
+ *
+ * Errors: every entry point returns a litela_status and never throws.  Argument errors are
+ * detected on the host before anything is launched.  A kernel launch failure returns
+ * LITELA_ERR_CUDA; a fault that happens later in an asynchronous kernel surfaces at the next
+ * synchronisation, as usual in CUDA.  lite_la_last_error() gives a message for the calling
+ * thread's last failure.
+ *
+ * Only d = 32 (Sana's linear_head_dim) is built; other d give LITELA_ERR_UNSUPPORTED.
+ * B, N or H equal to 0 is an empty problem: the call returns LITELA_OK and touches nothing.
+ */
+#ifndef LITELA_H_
+#define LITELA_H_
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LITELA_OK = 0,
+  LITELA_ERR_INVALID_ARGUMENT = 1, /* null pointer, negative size, misaligned or overlapping
+                                      buffers, eps < 0 or not finite, tokens_per_block < 1,
+                                      sizes whose element count overflows int64 */
+  LITELA_ERR_UNSUPPORTED = 2,      /* d != 32 */
+  LITELA_ERR_OUT_OF_MEMORY = 3,    /* workspace allocation failed */
+  LITELA_ERR_CUDA = 4              /* a CUDA runtime call or kernel launch failed */
+} litela_status;
+
+/* Non-causal LiteLA forward, bf16 output.
+ * qkv: device pointer, bf16 [B, N, 3*H*d] (layout above); out: device pointer, bf16
+ * [B, N, H*d].  eps is added to the denominator (Sana uses a tiny eps such as 1e-15).
+ * stream: the CUDA stream to run on (0 = legacy default stream). */
+litela_status lite_la_fwd(const void* qkv, void* out, int B, int N, int H, int d, float eps,
+                          cudaStream_t stream);
+
+/* Block-causal LiteLA forward, bf16 output ("Block-Linear Attention" for video: same instagit
+ * page, section "Video Generation and Constant-Memory KV Cache").  Tokens are cut into
+ * consecutive blocks of tokens_per_block tokens (the last block may be shorter); a query in
+ * block b uses the state summed over the keys/values of blocks 0..b (inclusive prefix).
+ * tokens_per_block >= N gives the non-causal result.  Other arguments as lite_la_fwd. */
+litela_status lite_la_block_causal_fwd(const void* qkv, void* out, int B, int N, int H, int d,
+                                       float eps, int tokens_per_block, cudaStream_t stream);
+
+/* The same two operations with an fp32 output buffer [B, N, H*d] (debug / accuracy mode). */
+litela_status lite_la_fwd_f32out(const void* qkv, float* out, int B, int N, int H, int d,
+                                 float eps, cudaStream_t stream);
+litela_status lite_la_block_causal_fwd_f32out(const void* qkv, float* out, int B, int N, int H,
+                                              int d, float eps, int tokens_per_block,
+                                              cudaStream_t stream);
+
+/* lite_la_fwd with phase timing: identical launches, plus cudaEventRecord of events[0] before
+ * the state-reduction kernel, events[1] between it and the apply kernel and events[2] after the
+ * apply kernel, all on `stream`.  events: host array of 3 caller-created CUDA events.  Used by
+ * the benchmark to time each kernel on its own stream. */
+litela_status lite_la_fwd_events(const void* qkv, void* out, int B, int N, int H, int d, float eps,
+                                 cudaStream_t stream, cudaEvent_t* events);
+
+/* Static description of a status code (never NULL). */
+const char* lite_la_status_string(litela_status status);
+
+/* Message describing the calling thread's most recent failure ("" if none). */
+const char* lite_la_last_error(void);
+
+/* Frees every cached workspace on every device.  Synchronises each device that holds one
+ * first, so it must not be called while another thread is capturing a CUDA graph. */
+litela_status lite_la_release_workspace(void);
+
+/* Size in bytes of the workspace a call with these arguments needs (tokens_per_block <= 0
+ * means non-causal).  Returns 0 for invalid arguments or an empty problem. */
+size_t lite_la_workspace_bytes(int B, int N, int H, int d, int tokens_per_block);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LITELA_H_ */

@@ -1,0 +1,135 @@
+"""LiteLA forward (Sana's ReLU linear self-attention) on B200: Python binding of liblitela.
+
+This module only marshals arguments to the C ABI of liblitela.so (include/litela.h); every
+step of the computation runs in the library's CUDA kernels.  torch supplies device memory
+and the current stream.  There is no fallback: if the library is missing or the tensors are
+not on a CUDA device, the calls raise.
+
+    from linear_attention_diffusion_litela_b200 import lite_la_fwd
+    out = lite_la_fwd(qkv, H=70)          # qkv: bf16 CUDA tensor [B, N, 3*H*32]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+__all__ = [
+    "LiteLAError", "lib", "lib_path", "lite_la_fwd", "lite_la_block_causal_fwd",
+    "lite_la_workspace_bytes", "lite_la_release_workspace", "STATUS", "EXPORTED_SYMBOLS",
+]
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_PKG_DIR, "liblitela.so")
+
+STATUS = {
+    0: "LITELA_OK",
+    1: "LITELA_ERR_INVALID_ARGUMENT",
+    2: "LITELA_ERR_UNSUPPORTED",
+    3: "LITELA_ERR_OUT_OF_MEMORY",
+    4: "LITELA_ERR_CUDA",
+}
+
+# name -> (restype, argtypes); mirrors include/litela.h
+_c_int, _c_float, _vp, _c_size = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+_SIGNATURES = {
+    "lite_la_fwd": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp]),
+    "lite_la_block_causal_fwd": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
+    "lite_la_fwd_f32out": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp]),
+    "lite_la_block_causal_fwd_f32out": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
+    "lite_la_fwd_events": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp, _vp]),
+    "lite_la_status_string": (ctypes.c_char_p, [_c_int]),
+    "lite_la_last_error": (ctypes.c_char_p, []),
+    "lite_la_release_workspace": (_c_int, []),
+    "lite_la_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+}
+EXPORTED_SYMBOLS = tuple(_SIGNATURES)
+
+_lib = None
+_lock = threading.Lock()
+
+
+class LiteLAError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = status
+        super().__init__("%s: %s" % (STATUS.get(status, status), message))
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded liblitela.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(lib_path):
+                raise ImportError("liblitela.so is not built; run "
+                                  "`python -m linear_attention_diffusion_litela_b200.build`")
+            h = ctypes.CDLL(lib_path)
+            for name, (res, args) in _SIGNATURES.items():
+                fn = getattr(h, name)
+                fn.restype, fn.argtypes = res, args
+            _lib = h
+    return _lib
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        msg = lib().lite_la_last_error().decode(errors="replace")
+        raise LiteLAError(status, msg)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _prepare(qkv, H: int, d: int, out, out_dtype):
+    torch = _torch()
+    if not isinstance(qkv, torch.Tensor) or not qkv.is_cuda:
+        raise TypeError("qkv must be a CUDA tensor")
+    if qkv.dtype != torch.bfloat16 or qkv.dim() != 3 or not qkv.is_contiguous():
+        raise TypeError("qkv must be a contiguous bf16 tensor [B, N, 3*H*d]")
+    B, N, W = qkv.shape
+    if W != 3 * H * d:
+        raise ValueError("qkv last dim %d != 3*H*d = %d" % (W, 3 * H * d))
+    if out is None:
+        out = torch.empty((B, N, H * d), dtype=out_dtype, device=qkv.device)
+    if out.dtype not in (torch.bfloat16, torch.float32) or not out.is_contiguous() \
+            or tuple(out.shape) != (B, N, H * d) or out.device != qkv.device:
+        raise TypeError("out must be a contiguous bf16/fp32 tensor [B, N, H*d] on qkv's device")
+    return B, N, out
+
+
+def _stream_handle(stream, device):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def lite_la_fwd(qkv, H: int, d: int = 32, eps: float = 1e-15, out=None, out_dtype=None, stream=None):
+    """Non-causal LiteLA forward; returns out [B, N, H*d] (bf16 unless out/out_dtype say fp32)."""
+    torch = _torch()
+    B, N, out = _prepare(qkv, H, d, out, out_dtype or torch.bfloat16)
+    fn = lib().lite_la_fwd if out.dtype == torch.bfloat16 else lib().lite_la_fwd_f32out
+    with torch.cuda.device(qkv.device):
+        _check(fn(qkv.data_ptr(), out.data_ptr(), B, N, H, d, eps, _stream_handle(stream, qkv.device)))
+    return out
+
+
+def lite_la_block_causal_fwd(qkv, H: int, tokens_per_block: int, d: int = 32, eps: float = 1e-15,
+                             out=None, out_dtype=None, stream=None):
+    """Block-causal LiteLA forward (a query in block b sees blocks 0..b); returns out."""
+    torch = _torch()
+    B, N, out = _prepare(qkv, H, d, out, out_dtype or torch.bfloat16)
+    fn = lib().lite_la_block_causal_fwd if out.dtype == torch.bfloat16 else lib().lite_la_block_causal_fwd_f32out
+    with torch.cuda.device(qkv.device):
+        _check(fn(qkv.data_ptr(), out.data_ptr(), B, N, H, d, eps, int(tokens_per_block),
+                  _stream_handle(stream, qkv.device)))
+    return out
+
+
+def lite_la_workspace_bytes(B: int, N: int, H: int, d: int = 32, tokens_per_block: int = 0) -> int:
+    return int(lib().lite_la_workspace_bytes(B, N, H, d, tokens_per_block))
+
+
+def lite_la_release_workspace() -> None:
+    _check(lib().lite_la_release_workspace())

@@ -1,0 +1,114 @@
+"""CPU-only checks of the C ABI: the library loads, exports every symbol include/litela.h
+declares, and its host-side logic (status strings, argument validation, workspace sizing)
+behaves as documented.  Nothing here launches a kernel."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_diffusion_litela_b200 as ll
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "litela.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from linear_attention_diffusion_litela_b200.build import build
+    build()
+    return ll.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lite_la_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_documented_entry_points():
+    names = declared_functions()
+    for required in ("lite_la_fwd", "lite_la_block_causal_fwd", "lite_la_fwd_f32out",
+                     "lite_la_block_causal_fwd_f32out", "lite_la_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert isinstance(getattr(lib, name), ctypes._CFuncPtr)
+
+
+def test_binding_covers_every_declared_symbol():
+    assert sorted(ll.EXPORTED_SYMBOLS) == declared_functions()
+
+
+def test_status_strings(lib):
+    for code, name in ll.STATUS.items():
+        assert lib.lite_la_status_string(code).decode() == name
+    assert lib.lite_la_status_string(99).decode() == "LITELA_UNKNOWN_STATUS"
+
+
+# Argument validation happens on the host, before any CUDA call.
+BAD_ARGS = [
+    # (B, N, H, d, eps, expected status)
+    (-1, 4, 1, 32, 1e-15, 1),
+    (1, -4, 1, 32, 1e-15, 1),
+    (1, 4, -1, 32, 1e-15, 1),
+    (1, 4, 1, 0, 1e-15, 1),
+    (1, 4, 1, 64, 1e-15, 2),
+    (1, 4, 1, 16, 1e-15, 2),
+    (1, 4, 1, 32, -1.0, 1),
+    (1, 4, 1, 32, float("nan"), 1),
+    (1, 4, 1, 32, float("inf"), 1),
+    (70000, 4, 1, 32, 1e-15, 1),
+]
+
+
+@pytest.mark.parametrize("B,N,H,d,eps,want", BAD_ARGS)
+def test_invalid_arguments_are_rejected_on_the_host(lib, B, N, H, d, eps, want):
+    fake_in, fake_out = ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 30)
+    assert lib.lite_la_fwd(fake_in, fake_out, B, N, H, d, eps, None) == want
+    assert lib.lite_la_last_error().decode() != ""
+    assert lib.lite_la_fwd_f32out(fake_in, fake_out, B, N, H, d, eps, None) == want
+    assert lib.lite_la_block_causal_fwd(fake_in, fake_out, B, N, H, d, eps, 16, None) == want
+
+
+def test_null_misaligned_and_overlapping_buffers_are_rejected(lib):
+    a, b = 1 << 20, 1 << 30
+    assert lib.lite_la_fwd(None, ctypes.c_void_p(b), 1, 4, 1, 32, 1e-15, None) == 1
+    assert lib.lite_la_fwd(ctypes.c_void_p(a), None, 1, 4, 1, 32, 1e-15, None) == 1
+    assert lib.lite_la_fwd(ctypes.c_void_p(a + 2), ctypes.c_void_p(b), 1, 4, 1, 32, 1e-15, None) == 1
+    assert lib.lite_la_fwd(ctypes.c_void_p(a), ctypes.c_void_p(b + 8), 1, 4, 1, 32, 1e-15, None) == 1
+    # out starts inside qkv (qkv is 4 tokens * 96 channels * 2 bytes = 768 bytes)
+    assert lib.lite_la_fwd(ctypes.c_void_p(a), ctypes.c_void_p(a + 256), 1, 4, 1, 32, 1e-15, None) == 1
+    assert "overlap" in lib.lite_la_last_error().decode()
+
+
+@pytest.mark.parametrize("T", [0, -3])
+def test_block_size_must_be_positive(lib, T):
+    a, b = 1 << 20, 1 << 30
+    assert lib.lite_la_block_causal_fwd(ctypes.c_void_p(a), ctypes.c_void_p(b), 1, 4, 1, 32, 1e-15, T, None) == 1
+
+
+@pytest.mark.parametrize("B,N,H", [(0, 4, 1), (1, 0, 1), (1, 4, 0), (0, 0, 0)])
+def test_empty_problem_is_a_no_op(lib, B, N, H):
+    # null pointers are fine for an empty problem: nothing is read or written
+    assert lib.lite_la_fwd(None, None, B, N, H, 32, 1e-15, None) == 0
+    assert lib.lite_la_block_causal_fwd(None, None, B, N, H, 32, 1e-15, 4, None) == 0
+
+
+def test_workspace_bytes(lib):
+    state = 33 * 32 * 4
+    assert ll.lite_la_workspace_bytes(0, 16, 1) == 0
+    assert ll.lite_la_workspace_bytes(1, 16, 1, d=64) == 0
+    for (B, N, H, T) in [(1, 1, 1, 0), (2, 1024, 70, 0), (2, 16384, 70, 0), (1, 16384, 70, 1024),
+                         (1, 100, 3, 7)]:
+        nblk = 1 if T <= 0 else -(-N // T)
+        got = ll.lite_la_workspace_bytes(B, N, H, 32, T)
+        # at least one partial and one final state per (batch, head, block) plus a counter
+        assert got >= B * H * nblk * 2 * state + B * H * 4
+        assert got % 4 == 0
+    # a causal block at least as long as N is the non-causal problem
+    assert ll.lite_la_workspace_bytes(2, 500, 3, 32, 500) == ll.lite_la_workspace_bytes(2, 500, 3, 32, 0)
+    assert ll.lite_la_workspace_bytes(2, 500, 3, 32, 10**6) == ll.lite_la_workspace_bytes(2, 500, 3, 32, 0)

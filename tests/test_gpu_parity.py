@@ -1,0 +1,200 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle, element by element.
+
+Tolerances (per element, o = oracle value):
+  bf16 output: |gpu - o| <= 1e-3 + 8e-3 * |o|
+  fp32 output: |gpu - o| <= 1e-5 + 1e-4 * |o|
+Small and medium shapes are compared on every output; the full-size workloads are compared
+on sampled query rows (first, last, block edges and a seeded random set), which the oracle
+evaluates one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_diffusion_litela_b200 as ll
+from linear_attention_diffusion_litela_b200.inputs import WORKLOADS, make_qkv, pack_qkv, to_bits
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+EPS = 1e-15
+TOL = {"bf16": (1e-3, 8e-3), "f32": (1e-5, 1e-4)}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from linear_attention_diffusion_litela_b200.build import build
+    build()
+    ll.lib()
+
+
+def gpu_run(qkv, H, T=None, mode="bf16"):
+    dt = torch.bfloat16 if mode == "bf16" else torch.float32
+    if T is None:
+        out = ll.lite_la_fwd(qkv, H, eps=EPS, out_dtype=dt)
+    else:
+        out = ll.lite_la_block_causal_fwd(qkv, H, T, eps=EPS, out_dtype=dt)
+    torch.cuda.synchronize()
+    B, N = qkv.shape[:2]
+    return out.view(B, N, H, 32).to(torch.float64).cpu().numpy()
+
+
+def oracle_run(qkv, H, T=None, rows=None):
+    B, N = qkv.shape[:2]
+    bits = to_bits(qkv)
+    if T is None:
+        return oracle.lite_la_fwd(bits, B, N, H, 32, EPS, rows=rows)
+    return oracle.lite_la_block_causal_fwd(bits, B, N, H, 32, EPS, T, rows=rows)
+
+
+def assert_close(got, want, mode):
+    atol, rtol = TOL[mode]
+    err = np.abs(got - want)
+    bound = atol + rtol * np.abs(want)
+    bad = err > bound
+    if bad.any():
+        i = np.unravel_index(np.argmax(err - bound), err.shape)
+        raise AssertionError("%d of %d elements out of tolerance; worst at %s: gpu=%r oracle=%r"
+                             % (bad.sum(), bad.size, i, got[i], want[i]))
+
+
+SMALL = [  # (B, N, H): several tiles, ragged tails, tiny cases
+    (1, 1, 1), (1, 2, 1), (1, 7, 3), (2, 31, 2), (1, 33, 5), (2, 300, 5), (1, 1000, 7),
+    (3, 257, 4), (1, 2049, 2),
+]
+
+
+@pytest.mark.parametrize("mode", ["bf16", "f32"])
+@pytest.mark.parametrize("B,N,H", SMALL)
+def test_small_shapes_every_element(B, N, H, mode):
+    qkv = make_qkv(B, N, H, 32, seed=B * 100003 + N * 31 + H, device="cuda")
+    assert_close(gpu_run(qkv, H, mode=mode), oracle_run(qkv, H), mode)
+
+
+@pytest.mark.parametrize("mode", ["bf16", "f32"])
+@pytest.mark.parametrize("B,N,H,T", [(1, 7, 2, 1), (2, 40, 3, 1), (1, 100, 2, 7), (2, 300, 3, 128),
+                                     (1, 1000, 4, 256), (1, 1000, 2, 300), (1, 513, 3, 512),
+                                     (2, 64, 2, 64), (1, 50, 2, 1000), (1, 2500, 2, 1024)])
+def test_block_causal_small_shapes_every_element(B, N, H, T, mode):
+    qkv = make_qkv(B, N, H, 32, seed=7 * N + T + H, device="cuda")
+    assert_close(gpu_run(qkv, H, T=T, mode=mode), oracle_run(qkv, H, T=T), mode)
+
+
+@pytest.mark.parametrize("mode", ["bf16", "f32"])
+@pytest.mark.parametrize("name", ["sana600m_512px", "sana1600m_1024px"])
+def test_small_workloads_every_element(name, mode):
+    w = WORKLOADS[name]
+    qkv = make_qkv(w["B"], w["N"], w["H"], 32, seed=1000 + list(WORKLOADS).index(name), device="cuda")
+    assert_close(gpu_run(qkv, w["H"], mode=mode), oracle_run(qkv, w["H"]), mode)
+
+
+def sample_rows(N, T=None, k=192, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = {0, 1, N - 2, N - 1}
+    if T is not None:
+        for b0 in range(0, N, T):
+            rows.update({b0, max(b0 - 1, 0), min(b0 + T - 1, N - 1)})
+    rows.update(rng.choice(N, size=min(k, N), replace=False).tolist())
+    return np.array(sorted(r for r in rows if 0 <= r < N))
+
+
+@pytest.mark.parametrize("mode", ["bf16", "f32"])
+@pytest.mark.parametrize("shift", [0.0, -1.5])
+def test_2048px_sampled(shift, mode):
+    w = WORKLOADS["sana1600m_2048px"]
+    seed = 1002 if shift == 0.0 else 3001
+    qkv = make_qkv(w["B"], w["N"], w["H"], 32, seed=seed, device="cuda", qk_shift=shift)
+    rows = sample_rows(w["N"], seed=seed)
+    got = gpu_run(qkv, w["H"], mode=mode)[:, rows]
+    assert_close(got, oracle_run(qkv, w["H"], rows=rows), mode)
+
+
+@pytest.mark.parametrize("mode", ["bf16", "f32"])
+def test_4096px_sampled(mode):
+    w = WORKLOADS["sana4800m_4096px"]
+    qkv = make_qkv(w["B"], w["N"], w["H"], 32, seed=4000, device="cuda")
+    rows = sample_rows(w["N"], k=96, seed=4)
+    got = gpu_run(qkv, w["H"], mode=mode)[:, rows]
+    assert_close(got, oracle_run(qkv, w["H"], rows=rows), mode)
+
+
+@pytest.mark.parametrize("mode", ["bf16", "f32"])
+def test_block_causal_workload_sampled(mode):
+    w = WORKLOADS["block_causal_16x1024"]
+    T = w["tokens_per_block"]
+    qkv = make_qkv(w["B"], w["N"], w["H"], 32, seed=1004, device="cuda")
+    rows = sample_rows(w["N"], T=T, k=64, seed=5)
+    got = gpu_run(qkv, w["H"], T=T, mode=mode)[:, rows]
+    assert_close(got, oracle_run(qkv, w["H"], T=T, rows=rows), mode)
+
+
+def test_hand_worked_example_padded_to_d32():
+    """The golden d=2 example embedded in channels 0..1 of a d=32 head (other channels 0)."""
+    from tests.test_golden import as_float, load_golden
+    g = load_golden()
+    q, k, v = (np.zeros((1, 3, 1, 32)) for _ in range(3))
+    q[0, :, 0, :2], k[0, :, 0, :2], v[0, :, 0, :2] = as_float(g["q"]), as_float(g["k"]), as_float(g["v"])
+    qkv = pack_qkv(q, k, v).cuda()
+    for key, T in (("out_noncausal", None), ("out_block_T1", 1), ("out_block_T2", 2)):
+        got = gpu_run(qkv, 1, T=T, mode="f32")[0, :, 0]
+        np.testing.assert_allclose(got[:, :2], as_float(g[key]), rtol=1e-6, atol=1e-7)
+        assert np.all(got[:, 2:] == 0)
+
+
+def test_bitwise_deterministic():
+    qkv = make_qkv(2, 3000, 7, 32, seed=77, device="cuda")
+    a = gpu_run(qkv, 7, mode="f32")
+    b = gpu_run(qkv, 7, mode="f32")
+    assert np.array_equal(a, b)
+    c = gpu_run(qkv, 7, T=500, mode="f32")
+    d = gpu_run(qkv, 7, T=500, mode="f32")
+    assert np.array_equal(c, d)
+
+
+def test_all_negative_query_row_is_exactly_zero_and_q_scaling_is_bitwise_invariant():
+    B, N, H = 1, 700, 3
+    qkv = make_qkv(B, N, H, 32, seed=91, device="cuda")
+    x = qkv.view(B, N, 3, H, 32)
+    x[0, 10, 0, 1] = -x[0, 10, 0, 1].abs() - 0.5
+    out = gpu_run(qkv, H, mode="f32")
+    assert np.all(out[0, 10, 1] == 0.0)
+    y = qkv.clone().view(B, N, 3, H, 32)
+    y[:, :, 0] *= 4.0
+    out2 = gpu_run(y.view(B, N, -1), H, mode="f32")
+    assert np.array_equal(out, out2)
+
+
+def test_non_default_stream_and_empty_problem():
+    qkv = make_qkv(1, 129, 2, 32, seed=5, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        out = ll.lite_la_fwd(qkv, 2, eps=EPS, out_dtype=torch.float32, stream=s)
+    s.synchronize()
+    got = out.view(1, 129, 2, 32).double().cpu().numpy()
+    assert_close(got, oracle_run(qkv, 2), "f32")
+    empty = torch.empty((1, 0, 3 * 2 * 32), dtype=torch.bfloat16, device="cuda")
+    assert ll.lite_la_fwd(empty, 2).shape == (1, 0, 64)
+
+
+def test_rejects_bad_arguments_without_launching():
+    qkv = make_qkv(1, 16, 1, 32, seed=1, device="cuda")
+    out = torch.empty((1, 16, 32), dtype=torch.bfloat16, device="cuda")
+    lib = ll.lib()
+    assert lib.lite_la_fwd(qkv.data_ptr() + 2, out.data_ptr(), 1, 15, 1, 32, EPS, None) == 1
+    assert lib.lite_la_fwd(qkv.data_ptr(), qkv.data_ptr(), 1, 16, 1, 32, EPS, None) == 1
+    assert lib.lite_la_fwd(qkv.data_ptr(), out.data_ptr(), 1, 16, 1, 16, EPS, None) == 2
+
+
+def test_workspace_allocation_failure_is_reported(monkeypatch):
+    qkv = make_qkv(1, 64, 1, 32, seed=2, device="cuda")
+    s = torch.cuda.Stream()                      # fresh stream: forces a new workspace
+    monkeypatch.setenv("LITELA_FAIL_ALLOC", "1")
+    with pytest.raises(ll.LiteLAError) as ei:
+        ll.lite_la_fwd(qkv, 1, stream=s)
+    assert ei.value.status == 3
+    monkeypatch.delenv("LITELA_FAIL_ALLOC")
+    out = ll.lite_la_fwd(qkv, 1, stream=s, out_dtype=torch.float32)
+    s.synchronize()
+    assert_close(out.view(1, 64, 1, 32).double().cpu().numpy(), oracle_run(qkv, 1), "f32")
