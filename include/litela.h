@@ -98,6 +98,27 @@ litela_status lite_la_release_workspace(void);
  * means non-causal).  Returns 0 for invalid arguments or an empty problem. */
 size_t lite_la_workspace_bytes(int B, int N, int H, int d, int tokens_per_block);
 
+/* lite_la_fwd without any allocation.  The pages describe no such call; it exists for callers
+ * that cannot let a library allocate device memory: a host that owns all of the device memory
+ * through its own pool and hands each op only its input and output buffers, or a latency-bound
+ * loop in which a first-use cudaMalloc (and the device synchronisation it may bring) is not
+ * acceptable.  Same arguments, layouts and result as lite_la_fwd (bf16 output, non-causal).
+ *
+ * Its scratch (partial states, merged states, arrival counters) is one fixed array of
+ * LITELA_NOALLOC_SCRATCH_BYTES in device memory that the library defines statically; every
+ * GPU that loads the library holds it until the process exits.  A problem whose scratch does
+ * not fit (roughly: lite_la_workspace_bytes() near or above the limit; the 4096px Sana call with
+ * B=2, N=16384, H=70 needs about 6 MB) is rejected with LITELA_ERR_INVALID_ARGUMENT and a
+ * message before anything is launched.  The first call on a device looks
+ * up that device's address of the array (once per device); make that first call before any
+ * stream capture.  The call never calls cudaMalloc or cudaFree; it clears the counters it needs
+ * with cudaMemsetAsync on `stream`.  All calls on a device share the one array and it keeps the
+ * last call's contents, so calls that can overlap on the GPU (different streams without an
+ * ordering between them) race and give wrong results: order them, e.g. on one stream. */
+#define LITELA_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+litela_status lite_la_fwd_noalloc(const void* qkv, void* out, int B, int N, int H, int d,
+                                  float eps, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

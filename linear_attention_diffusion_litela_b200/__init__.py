@@ -42,6 +42,7 @@ _SIGNATURES = {
     "lite_la_last_error": (ctypes.c_char_p, []),
     "lite_la_release_workspace": (_c_int, []),
     "lite_la_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "lite_la_fwd_noalloc": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp]),
 }
 EXPORTED_SYMBOLS = tuple(_SIGNATURES)
 

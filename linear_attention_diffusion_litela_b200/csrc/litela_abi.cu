@@ -156,10 +156,77 @@ litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float 
   return LITELA_OK;
 }
 
+// Fixed scratch of lite_la_fwd_noalloc: one array per device, defined statically so that the
+// entry point never allocates.  Host code must not use the symbol as an address; it asks the
+// runtime for each device's address once (noalloc_scratch below).
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LITELA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (looked up once per device).
+litela_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(LITELA_ERR_UNSUPPORTED, "device index above 63");
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return LITELA_OK;
+}
+
+litela_status run_noalloc(const void* qkv, __nv_bfloat16* out, int B, int N, int H, int d, float eps,
+                          cudaStream_t stream) {
+  Plan plan;
+  litela_status s = validate(qkv, out, sizeof(__nv_bfloat16), B, N, H, d, eps, 0, false, &plan);
+  if (s != LITELA_OK || plan.B == 0) return s;
+  const size_t counter_bytes = align_up(plan.counters * sizeof(unsigned), 256);
+  const size_t need = counter_bytes + plan.bytes;
+  if (need > LITELA_NOALLOC_SCRATCH_BYTES)
+    return fail(LITELA_ERR_INVALID_ARGUMENT,
+                "problem needs " + std::to_string(need) + " bytes of scratch; lite_la_fwd_noalloc has " +
+                    std::to_string((size_t)LITELA_NOALLOC_SCRATCH_BYTES));
+  void* scratch = nullptr;
+  s = noalloc_scratch(&scratch);
+  if (s != LITELA_OK) return s;
+  char* base = static_cast<char*>(scratch);
+  unsigned* counters = reinterpret_cast<unsigned*>(base);
+  float* partials = reinterpret_cast<float*>(base + counter_bytes + plan.off_partials);
+  float* states = reinterpret_cast<float*>(base + counter_bytes + plan.off_states);
+  cudaError_t e = cudaMemsetAsync(counters, 0, plan.counters * sizeof(unsigned), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(no-alloc counters)");
+  DevPlan dp{plan.B, plan.N, plan.H, plan.T, plan.nblk, plan.chunks_per_block, plan.chunk,
+             plan.tiles_per_block, eps};
+  const auto* in = static_cast<const __nv_bfloat16*>(qkv);
+  dim3 rgrid(plan.nblk * plan.chunks_per_block, H, B);
+  litela_reduce_simt<<<rgrid, kReduceThreads, 0, stream>>>(in, partials, states, counters, dp);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch litela_reduce_simt");
+  dim3 agrid(plan.nblk * plan.tiles_per_block, H, B);
+  litela_apply_simt<__nv_bfloat16><<<agrid, kApplyTile, 0, stream>>>(in, states, out, dp);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch litela_apply_simt");
+  g_last_error.clear();
+  return LITELA_OK;
+}
+
 }  // namespace
 }  // namespace litela
 
 extern "C" {
+
+litela_status lite_la_fwd_noalloc(const void* qkv, void* out, int B, int N, int H, int d, float eps,
+                                  cudaStream_t stream) {
+  return litela::run_noalloc(qkv, static_cast<__nv_bfloat16*>(out), B, N, H, d, eps, stream);
+}
+
 
 litela_status lite_la_fwd(const void* qkv, void* out, int B, int N, int H, int d, float eps,
                           cudaStream_t stream) {
