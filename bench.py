@@ -46,8 +46,8 @@ FP32_LANES_PER_SM = 128          # B200: 4 SM sub-partitions x 32 fp32 lanes
 NUM_SMS = 148
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
 # name of each kernel the library launches per call, in launch order
-KERNELS = ("litela_reduce_simt", "litela_apply_simt")
-KERNEL_BOUND = {"litela_reduce_simt": "alu", "litela_apply_simt": "alu"}
+KERNELS = ("litela_reduce_tc", "litela_apply_tc")
+KERNEL_BOUND = {"litela_reduce_tc": "hbm", "litela_apply_tc": "hbm"}
 
 
 def load_peaks():
@@ -398,7 +398,8 @@ def main():
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_step, "us_per_call": us_call,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "math": "tensor-core bf16 x bf16 products with fp32 accumulation; fp32 state applied as bf16 hi + lo",
                 "data": "synthetic: i.i.d. N(0,1) bf16 qkv from seeded torch generators",
                 "config": config_of(args.workload), "roofline": roofline, "call_roofline": call_roof,
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": len(KERNELS) * calls * args.steps,

@@ -52,7 +52,8 @@ typedef enum {
                                       sizes whose element count overflows int64 */
   LITELA_ERR_UNSUPPORTED = 2,      /* d != 32 */
   LITELA_ERR_OUT_OF_MEMORY = 3,    /* workspace allocation failed */
-  LITELA_ERR_CUDA = 4              /* a CUDA runtime call or kernel launch failed */
+  LITELA_ERR_CUDA = 4,             /* a CUDA runtime call or kernel launch failed */
+  LITELA_ERR_DEVICE_TIMEOUT = 5    /* a kernel gave up on a bounded wait (lite_la_device_status) */
 } litela_status;
 
 /* Non-causal LiteLA forward, bf16 output.
@@ -77,12 +78,29 @@ litela_status lite_la_block_causal_fwd_f32out(const void* qkv, float* out, int B
                                               int d, float eps, int tokens_per_block,
                                               cudaStream_t stream);
 
+/* The LiteLA state alone (the first contraction, and the video "KV cache" of Block-Linear
+ * Attention): for every batch b, head h and causal block k (one block when tokens_per_block <= 0
+ * or >= N) the inclusive prefix state over the tokens of blocks 0..k,
+ *     states[b][h][k][r][c] = sum_n v[n][h][r] * relu(k[n][h][c])   for r < d,
+ *     states[b][h][k][d][c] = sum_n relu(k[n][h][c])                  (the ones-pad row),
+ * fp32, layout [B, H, nblk, d+1, d] row-major, nblk = ceil(N / tokens_per_block).  states is a
+ * caller-owned device buffer (16-byte aligned, not overlapping qkv). */
+litela_status lite_la_state_fwd(const void* qkv, float* states, int B, int N, int H, int d,
+                                int tokens_per_block, cudaStream_t stream);
+
 /* lite_la_fwd with phase timing: identical launches, plus cudaEventRecord of events[0] before
  * the state-reduction kernel, events[1] between it and the apply kernel and events[2] after the
  * apply kernel, all on `stream`.  events: host array of 3 caller-created CUDA events.  Used by
  * the benchmark to time each kernel on its own stream. */
 litela_status lite_la_fwd_events(const void* qkv, void* out, int B, int N, int H, int d, float eps,
                                  cudaStream_t stream, cudaEvent_t* events);
+
+/* Synchronises `stream`, then reads and clears the error word that this library's kernels on
+ * the current device set when one of their bounded waits timed out (each wait inside the
+ * kernels gives up after about 1.5 s, records a code, frees its tensor memory and returns, so
+ * the GPU context stays usable).  Returns LITELA_ERR_DEVICE_TIMEOUT (message with the code) if
+ * a kernel of this stream's workspace or of lite_la_fwd_noalloc reported one, else LITELA_OK. */
+litela_status lite_la_device_status(cudaStream_t stream);
 
 /* Static description of a status code (never NULL). */
 const char* lite_la_status_string(litela_status status);

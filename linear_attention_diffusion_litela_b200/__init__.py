@@ -28,6 +28,7 @@ STATUS = {
     2: "LITELA_ERR_UNSUPPORTED",
     3: "LITELA_ERR_OUT_OF_MEMORY",
     4: "LITELA_ERR_CUDA",
+    5: "LITELA_ERR_DEVICE_TIMEOUT",
 }
 
 # name -> (restype, argtypes); mirrors include/litela.h
@@ -38,6 +39,8 @@ _SIGNATURES = {
     "lite_la_fwd_f32out": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp]),
     "lite_la_block_causal_fwd_f32out": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
     "lite_la_fwd_events": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp, _vp]),
+    "lite_la_device_status": (_c_int, [_vp]),
+    "lite_la_state_fwd": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "lite_la_status_string": (ctypes.c_char_p, [_c_int]),
     "lite_la_last_error": (ctypes.c_char_p, []),
     "lite_la_release_workspace": (_c_int, []),
@@ -128,8 +131,36 @@ def lite_la_block_causal_fwd(qkv, H: int, tokens_per_block: int, d: int = 32, ep
     return out
 
 
+def lite_la_state_fwd(qkv, H: int, tokens_per_block: int = 0, d: int = 32, out=None, stream=None):
+    """Per-(batch, head, block) inclusive prefix states, fp32 [B, H, nblk, d+1, d]."""
+    torch = _torch()
+    if not isinstance(qkv, torch.Tensor) or not qkv.is_cuda or qkv.dtype != torch.bfloat16 \
+            or qkv.dim() != 3 or not qkv.is_contiguous():
+        raise TypeError("qkv must be a contiguous bf16 CUDA tensor [B, N, 3*H*d]")
+    B, N, W = qkv.shape
+    if W != 3 * H * d:
+        raise ValueError("qkv last dim %d != 3*H*d = %d" % (W, 3 * H * d))
+    T = tokens_per_block if 0 < tokens_per_block < N else N
+    nblk = -(-N // T) if N > 0 else 0
+    if out is None:
+        out = torch.empty((B, H, nblk, d + 1, d), dtype=torch.float32, device=qkv.device)
+    if out.dtype != torch.float32 or not out.is_contiguous() or tuple(out.shape) != (B, H, nblk, d + 1, d):
+        raise TypeError("out must be a contiguous fp32 tensor [B, H, nblk, d+1, d]")
+    with torch.cuda.device(qkv.device):
+        _check(lib().lite_la_state_fwd(qkv.data_ptr(), out.data_ptr(), B, N, H, d, int(tokens_per_block),
+                                       _stream_handle(stream, qkv.device)))
+    return out
+
+
 def lite_la_workspace_bytes(B: int, N: int, H: int, d: int = 32, tokens_per_block: int = 0) -> int:
     return int(lib().lite_la_workspace_bytes(B, N, H, d, tokens_per_block))
+
+
+def lite_la_device_status(stream=None) -> None:
+    """Synchronises the stream and raises LiteLAError if a kernel reported a timed-out wait."""
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    _check(lib().lite_la_device_status(ctypes.c_void_p(s.cuda_stream)))
 
 
 def lite_la_release_workspace() -> None:

@@ -1,5 +1,8 @@
-// C ABI of liblitela: argument validation, per-(device, stream) workspace, kernel launches.
-// The operation, the layouts and the error behaviour are documented in include/litela.h.
+// C ABI of liblitela: argument validation, per-(device, stream) workspace, TMA descriptors and
+// kernel launches.  The operation, the layouts and the error behaviour are documented in
+// include/litela.h.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -15,7 +18,7 @@
 
 #include "../../include/litela.h"
 #include "litela_plan.h"
-#include "litela_simt.cuh"
+#include "litela_tc.cuh"
 
 namespace litela {
 namespace {
@@ -31,12 +34,79 @@ litela_status cuda_fail(cudaError_t e, const char* what) {
   return fail(LITELA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
 }
 
-// One workspace per (device, stream): partial/prefix states plus arrival counters that the
-// kernels always leave at zero.
+// ---------------------------------------------------------------------------------------
+// per-device set-up: SM count, kernel shared-memory limits, the driver's tensor-map encoder
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+};
+std::mutex g_dev_mutex;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+litela_status device_setup(int* num_sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(LITELA_ERR_UNSUPPORTED, "device index above 63");
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute(compute capability)");
+    if (major != 10 || minor != 0)
+      return fail(LITELA_ERR_UNSUPPORTED, "liblitela is built for sm_100a (B200); device is sm_" +
+                                              std::to_string(major) + std::to_string(minor));
+    if ((e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
+    if ((e = cudaFuncSetAttribute(litela_reduce_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kRedSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_apply_tc<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kApSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_apply_tc<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kApSmemBytes)) != cudaSuccess)
+      return cuda_fail(e, "cudaFuncSetAttribute(dynamic shared memory)");
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+      if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return fail(LITELA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    d.ready = true;
+  }
+  *num_sms = d.num_sms;
+  return LITELA_OK;
+}
+
+// 3-D view of the packed qkv buffer for TMA: (channel, token, batch), bf16, boxes of 64
+// channels x box_tokens tokens, 128-byte swizzle, zero fill outside the tensor.
+litela_status encode_qkv_map(const void* qkv, int B, int N, int H, int box_tokens, CUtensorMap* map) {
+  const cuuint64_t row = 3ull * H * kD;
+  const cuuint64_t dims[3] = {row, (cuuint64_t)N, (cuuint64_t)B};
+  const cuuint64_t strides[2] = {row * 2, row * 2 * (cuuint64_t)N};
+  const cuuint32_t box[3] = {64, (cuuint32_t)box_tokens, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(qkv), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LITELA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string((int)r) + ")");
+  return LITELA_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// workspace: one per (device, stream)
+
 struct Workspace {
   void* states = nullptr;
   size_t states_bytes = 0;
-  unsigned* counters = nullptr;
+  unsigned* counters = nullptr;   // word 0: device error word; counters from kCounterBase
   size_t counters_len = 0;
 };
 
@@ -56,8 +126,9 @@ litela_status get_workspace(const Plan& plan, cudaStream_t stream, Workspace** o
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   std::lock_guard<std::mutex> lock(g_ws_mutex);
   Workspace& ws = g_ws[{dev, reinterpret_cast<uintptr_t>(stream)}];
+  const size_t need_counters = kCounterBase + plan.counters;
   const bool grow_states = ws.states_bytes < plan.bytes;
-  const bool grow_counters = ws.counters_len < plan.counters;
+  const bool grow_counters = ws.counters_len < need_counters;
   if (grow_states || grow_counters) {
     if (alloc_fault_injected())
       return fail(LITELA_ERR_OUT_OF_MEMORY, "workspace allocation failed (injected by LITELA_FAIL_ALLOC)");
@@ -79,14 +150,14 @@ litela_status get_workspace(const Plan& plan, cudaStream_t stream, Workspace** o
       if (ws.counters) cudaFree(ws.counters);
       ws.counters = nullptr;
       ws.counters_len = 0;
-      e = cudaMalloc(&ws.counters, plan.counters * sizeof(unsigned));
+      e = cudaMalloc(&ws.counters, need_counters * sizeof(unsigned));
       if (e != cudaSuccess) {
         cudaGetLastError();
         return fail(LITELA_ERR_OUT_OF_MEMORY, std::string("counter cudaMalloc: ") + cudaGetErrorString(e));
       }
-      e = cudaMemset(ws.counters, 0, plan.counters * sizeof(unsigned));
+      e = cudaMemset(ws.counters, 0, need_counters * sizeof(unsigned));
       if (e != cudaSuccess) return cuda_fail(e, "cudaMemset counters");
-      ws.counters_len = plan.counters;
+      ws.counters_len = need_counters;
     }
   }
   *out = &ws;
@@ -98,11 +169,11 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   return x < y + nb && y < x + na;
 }
 
-// Host-side validation; on success fills *plan (or returns LITELA_OK with plan->B == 0 for an
-// empty problem).
-litela_status validate(const void* qkv, const void* out, size_t out_elem, int B, int N, int H,
-                       int d, float eps, int tokens_per_block, bool causal, Plan* plan) {
-  *plan = Plan{};
+// Host-side validation of the arguments (no CUDA call).  Returns LITELA_OK with *empty = true
+// for an empty problem.
+litela_status validate(const void* qkv, const void* out, size_t out_elem, int B, int N, int H, int d,
+                       float eps, int tokens_per_block, bool causal, bool* empty) {
+  *empty = false;
   if (B < 0 || N < 0 || H < 0) return fail(LITELA_ERR_INVALID_ARGUMENT, "B, N and H must be >= 0");
   if (d <= 0) return fail(LITELA_ERR_INVALID_ARGUMENT, "d must be positive");
   if (d != kD) return fail(LITELA_ERR_UNSUPPORTED, "only d = 32 is built");
@@ -110,7 +181,10 @@ litela_status validate(const void* qkv, const void* out, size_t out_elem, int B,
   if (causal && tokens_per_block < 1) return fail(LITELA_ERR_INVALID_ARGUMENT, "tokens_per_block must be >= 1");
   if (B > 65535 || H > 65535) return fail(LITELA_ERR_INVALID_ARGUMENT, "B and H must be <= 65535");
   if (N > (1 << 30)) return fail(LITELA_ERR_INVALID_ARGUMENT, "N must be <= 2^30");
-  if (B == 0 || N == 0 || H == 0) return LITELA_OK;           // empty problem
+  if (B == 0 || N == 0 || H == 0) {
+    *empty = true;
+    return LITELA_OK;
+  }
   if (qkv == nullptr || out == nullptr) return fail(LITELA_ERR_INVALID_ARGUMENT, "null qkv or out");
   if ((reinterpret_cast<uintptr_t>(qkv) & 15u) || (reinterpret_cast<uintptr_t>(out) & 15u))
     return fail(LITELA_ERR_INVALID_ARGUMENT, "qkv and out must be 16-byte aligned");
@@ -119,41 +193,88 @@ litela_status validate(const void* qkv, const void* out, size_t out_elem, int B,
   const size_t qkv_bytes = (size_t)B * N * 3 * H * d * sizeof(__nv_bfloat16);
   const size_t out_bytes = (size_t)B * N * H * d * out_elem;
   if (overlaps(qkv, qkv_bytes, out, out_bytes)) return fail(LITELA_ERR_INVALID_ARGUMENT, "out overlaps qkv");
-  make_plan(B, N, H, causal ? tokens_per_block : 0, plan);
+  return LITELA_OK;
+}
+
+// Launches the state reduction and the apply for `plan` with the given scratch.
+template <typename OutT>
+litela_status launch(const Plan& plan, const void* qkv, OutT* out, float eps, float* partials,
+                     uint8_t* images, unsigned* counters, int num_sms, cudaStream_t stream,
+                     cudaEvent_t* events) {
+  CUtensorMap map_red, map_ap;
+  litela_status s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kRedTile, &map_red);
+  if (s != LITELA_OK) return s;
+  s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kApTile, &map_ap);
+  if (s != LITELA_OK) return s;
+  TcPlan tp{plan.B, plan.N, plan.H, plan.T, plan.nblk, plan.ngroups, plan.chunks_per_block, plan.chunk,
+            plan.npairs, plan.tiles_per_block, (long long)plan.items, eps};
+  int* err = reinterpret_cast<int*>(counters);
+  cudaError_t e;
+  if (events && (e = cudaEventRecord(events[0], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  dim3 rgrid(plan.nblk * plan.chunks_per_block, plan.ngroups, plan.B);
+  litela_reduce_tc<<<rgrid, kRedThreads, kRedSmemBytes, stream>>>(map_red, partials, images, nullptr, counters,
+                                                                   err, tp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "launch litela_reduce_tc");
+  if (events && (e = cudaEventRecord(events[1], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  const long long grid = plan.items < num_sms ? plan.items : num_sms;
+  litela_apply_tc<OutT><<<(unsigned)grid, kApThreads, kApSmemBytes, stream>>>(map_ap, images, out, err, tp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "launch litela_apply_tc");
+  if (events && (e = cudaEventRecord(events[2], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  return LITELA_OK;
+}
+
+// State reduction alone, writing the fp32 prefix states to `states`.
+litela_status run_states(const void* qkv, float* states, int B, int N, int H, int d, int tokens_per_block,
+                         cudaStream_t stream) {
+  bool empty = false;
+  litela_status s = validate(qkv, states, 0, B, N, H, d, 0.f, 0, false, &empty);
+  if (s != LITELA_OK || empty) return s;
+  int num_sms = 0;
+  s = device_setup(&num_sms);
+  if (s != LITELA_OK) return s;
+  Plan plan;
+  make_plan(B, N, H, tokens_per_block, num_sms, &plan);
+  const size_t state_bytes = (size_t)B * H * plan.nblk * kStateFloats * sizeof(float);
+  const size_t qkv_bytes = (size_t)B * N * 3 * H * d * sizeof(__nv_bfloat16);
+  if (overlaps(qkv, qkv_bytes, states, state_bytes)) return fail(LITELA_ERR_INVALID_ARGUMENT, "states overlaps qkv");
+  Workspace* ws = nullptr;
+  s = get_workspace(plan, stream, &ws);
+  if (s != LITELA_OK) return s;
+  CUtensorMap map_red;
+  s = encode_qkv_map(qkv, B, N, H, kRedTile, &map_red);
+  if (s != LITELA_OK) return s;
+  TcPlan tp{plan.B, plan.N, plan.H, plan.T, plan.nblk, plan.ngroups, plan.chunks_per_block, plan.chunk,
+            plan.npairs, plan.tiles_per_block, (long long)plan.items, 0.f};
+  char* base = static_cast<char*>(ws->states);
+  dim3 rgrid(plan.nblk * plan.chunks_per_block, plan.ngroups, plan.B);
+  litela_reduce_tc<<<rgrid, kRedThreads, kRedSmemBytes, stream>>>(
+      map_red, reinterpret_cast<float*>(base + plan.off_partials), nullptr, states, ws->counters,
+      reinterpret_cast<int*>(ws->counters), tp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch litela_reduce_tc");
+  g_last_error.clear();
   return LITELA_OK;
 }
 
 template <typename OutT>
-litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float eps,
-                  int tokens_per_block, bool causal, cudaStream_t stream,
-                  cudaEvent_t* events = nullptr) {
+litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float eps, int tokens_per_block,
+                  bool causal, cudaStream_t stream, cudaEvent_t* events = nullptr) {
+  bool empty = false;
+  litela_status s = validate(qkv, out, sizeof(OutT), B, N, H, d, eps, tokens_per_block, causal, &empty);
+  if (s != LITELA_OK || empty) return s;
+  int num_sms = 0;
+  s = device_setup(&num_sms);
+  if (s != LITELA_OK) return s;
   Plan plan;
-  litela_status s = validate(qkv, out, sizeof(OutT), B, N, H, d, eps, tokens_per_block, causal, &plan);
-  if (s != LITELA_OK || plan.B == 0) return s;
+  make_plan(B, N, H, causal ? tokens_per_block : 0, num_sms, &plan);
   Workspace* ws = nullptr;
   s = get_workspace(plan, stream, &ws);
   if (s != LITELA_OK) return s;
-  DevPlan dp{plan.B, plan.N, plan.H, plan.T, plan.nblk, plan.chunks_per_block, plan.chunk,
-             plan.tiles_per_block, eps};
   char* base = static_cast<char*>(ws->states);
-  float* partials = reinterpret_cast<float*>(base + plan.off_partials);
-  float* states = reinterpret_cast<float*>(base + plan.off_states);
-  const auto* in = static_cast<const __nv_bfloat16*>(qkv);
-
-  cudaError_t e;
-  if (events && (e = cudaEventRecord(events[0], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  dim3 rgrid(plan.nblk * plan.chunks_per_block, H, B);
-  litela_reduce_simt<<<rgrid, kReduceThreads, 0, stream>>>(in, partials, states, ws->counters, dp);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "launch litela_reduce_simt");
-  if (events && (e = cudaEventRecord(events[1], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  dim3 agrid(plan.nblk * plan.tiles_per_block, H, B);
-  litela_apply_simt<OutT><<<agrid, kApplyTile, 0, stream>>>(in, states, out, dp);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "launch litela_apply_simt");
-  if (events && (e = cudaEventRecord(events[2], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  g_last_error.clear();
-  return LITELA_OK;
+  s = launch(plan, qkv, out, eps, reinterpret_cast<float*>(base + plan.off_partials),
+             reinterpret_cast<uint8_t*>(base + plan.off_images), ws->counters, num_sms, stream, events);
+  if (s == LITELA_OK) g_last_error.clear();
+  return s;
 }
 
 // Fixed scratch of lite_la_fwd_noalloc: one array per device, defined statically so that the
@@ -161,7 +282,6 @@ litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float 
 // runtime for each device's address once (noalloc_scratch below).
 static __device__ __align__(256) unsigned char g_noalloc_scratch[LITELA_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void* g_noalloc_ptr[kMaxDevices] = {};
 
@@ -184,10 +304,15 @@ litela_status noalloc_scratch(void** out) {
 
 litela_status run_noalloc(const void* qkv, __nv_bfloat16* out, int B, int N, int H, int d, float eps,
                           cudaStream_t stream) {
+  bool empty = false;
+  litela_status s = validate(qkv, out, sizeof(__nv_bfloat16), B, N, H, d, eps, 0, false, &empty);
+  if (s != LITELA_OK || empty) return s;
+  int num_sms = 0;
+  s = device_setup(&num_sms);
+  if (s != LITELA_OK) return s;
   Plan plan;
-  litela_status s = validate(qkv, out, sizeof(__nv_bfloat16), B, N, H, d, eps, 0, false, &plan);
-  if (s != LITELA_OK || plan.B == 0) return s;
-  const size_t counter_bytes = align_up(plan.counters * sizeof(unsigned), 256);
+  make_plan(B, N, H, 0, num_sms, &plan);
+  const size_t counter_bytes = align_up((kCounterBase + plan.counters) * sizeof(unsigned), 256);
   const size_t need = counter_bytes + plan.bytes;
   if (need > LITELA_NOALLOC_SCRATCH_BYTES)
     return fail(LITELA_ERR_INVALID_ARGUMENT,
@@ -198,35 +323,19 @@ litela_status run_noalloc(const void* qkv, __nv_bfloat16* out, int B, int N, int
   if (s != LITELA_OK) return s;
   char* base = static_cast<char*>(scratch);
   unsigned* counters = reinterpret_cast<unsigned*>(base);
-  float* partials = reinterpret_cast<float*>(base + counter_bytes + plan.off_partials);
-  float* states = reinterpret_cast<float*>(base + counter_bytes + plan.off_states);
-  cudaError_t e = cudaMemsetAsync(counters, 0, plan.counters * sizeof(unsigned), stream);
+  cudaError_t e = cudaMemsetAsync(counters, 0, (kCounterBase + plan.counters) * sizeof(unsigned), stream);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(no-alloc counters)");
-  DevPlan dp{plan.B, plan.N, plan.H, plan.T, plan.nblk, plan.chunks_per_block, plan.chunk,
-             plan.tiles_per_block, eps};
-  const auto* in = static_cast<const __nv_bfloat16*>(qkv);
-  dim3 rgrid(plan.nblk * plan.chunks_per_block, H, B);
-  litela_reduce_simt<<<rgrid, kReduceThreads, 0, stream>>>(in, partials, states, counters, dp);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "launch litela_reduce_simt");
-  dim3 agrid(plan.nblk * plan.tiles_per_block, H, B);
-  litela_apply_simt<__nv_bfloat16><<<agrid, kApplyTile, 0, stream>>>(in, states, out, dp);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "launch litela_apply_simt");
-  g_last_error.clear();
-  return LITELA_OK;
+  s = launch(plan, qkv, out, eps, reinterpret_cast<float*>(base + counter_bytes + plan.off_partials),
+             reinterpret_cast<uint8_t*>(base + counter_bytes + plan.off_images), counters, num_sms, stream,
+             nullptr);
+  if (s == LITELA_OK) g_last_error.clear();
+  return s;
 }
 
 }  // namespace
 }  // namespace litela
 
 extern "C" {
-
-litela_status lite_la_fwd_noalloc(const void* qkv, void* out, int B, int N, int H, int d, float eps,
-                                  cudaStream_t stream) {
-  return litela::run_noalloc(qkv, static_cast<__nv_bfloat16*>(out), B, N, H, d, eps, stream);
-}
-
 
 litela_status lite_la_fwd(const void* qkv, void* out, int B, int N, int H, int d, float eps,
                           cudaStream_t stream) {
@@ -235,8 +344,7 @@ litela_status lite_la_fwd(const void* qkv, void* out, int B, int N, int H, int d
 
 litela_status lite_la_block_causal_fwd(const void* qkv, void* out, int B, int N, int H, int d,
                                        float eps, int tokens_per_block, cudaStream_t stream) {
-  return litela::run(qkv, static_cast<__nv_bfloat16*>(out), B, N, H, d, eps, tokens_per_block, true,
-                     stream);
+  return litela::run(qkv, static_cast<__nv_bfloat16*>(out), B, N, H, d, eps, tokens_per_block, true, stream);
 }
 
 litela_status lite_la_fwd_f32out(const void* qkv, float* out, int B, int N, int H, int d, float eps,
@@ -256,6 +364,52 @@ litela_status lite_la_fwd_events(const void* qkv, void* out, int B, int N, int H
   return litela::run(qkv, static_cast<__nv_bfloat16*>(out), B, N, H, d, eps, 0, false, stream, events);
 }
 
+litela_status lite_la_state_fwd(const void* qkv, float* states, int B, int N, int H, int d,
+                                int tokens_per_block, cudaStream_t stream) {
+  return litela::run_states(qkv, states, B, N, H, d, tokens_per_block, stream);
+}
+
+litela_status lite_la_fwd_noalloc(const void* qkv, void* out, int B, int N, int H, int d, float eps,
+                                  cudaStream_t stream) {
+  return litela::run_noalloc(qkv, static_cast<__nv_bfloat16*>(out), B, N, H, d, eps, stream);
+}
+
+litela_status lite_la_device_status(cudaStream_t stream) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return litela::cuda_fail(e, "cudaGetDevice");
+  e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return litela::cuda_fail(e, "cudaStreamSynchronize");
+  unsigned* words[2] = {nullptr, nullptr};
+  {
+    std::lock_guard<std::mutex> lock(litela::g_ws_mutex);
+    auto it = litela::g_ws.find({dev, reinterpret_cast<uintptr_t>(stream)});
+    if (it != litela::g_ws.end()) words[0] = it->second.counters;
+  }
+  {
+    std::lock_guard<std::mutex> lock(litela::g_noalloc_mutex);
+    if (dev < litela::kMaxDevices) words[1] = static_cast<unsigned*>(litela::g_noalloc_ptr[dev]);
+  }
+  int code = 0;
+  for (unsigned* w : words) {
+    if (w == nullptr) continue;
+    int v = 0;
+    if ((e = cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+      return litela::cuda_fail(e, "reading the device error word");
+    if (v != 0) {
+      if (code == 0) code = v;
+      if ((e = cudaMemset(w, 0, sizeof(int))) != cudaSuccess)
+        return litela::cuda_fail(e, "clearing the device error word");
+    }
+  }
+  if (code != 0) {
+    char buf[128];
+    std::snprintf(buf, sizeof(buf), "a kernel wait timed out (code 0x%x)", code);
+    return litela::fail(LITELA_ERR_DEVICE_TIMEOUT, buf);
+  }
+  return LITELA_OK;
+}
+
 const char* lite_la_status_string(litela_status status) {
   switch (status) {
     case LITELA_OK: return "LITELA_OK";
@@ -263,6 +417,7 @@ const char* lite_la_status_string(litela_status status) {
     case LITELA_ERR_UNSUPPORTED: return "LITELA_ERR_UNSUPPORTED";
     case LITELA_ERR_OUT_OF_MEMORY: return "LITELA_ERR_OUT_OF_MEMORY";
     case LITELA_ERR_CUDA: return "LITELA_ERR_CUDA";
+    case LITELA_ERR_DEVICE_TIMEOUT: return "LITELA_ERR_DEVICE_TIMEOUT";
   }
   return "LITELA_UNKNOWN_STATUS";
 }
@@ -288,8 +443,8 @@ litela_status lite_la_release_workspace(void) {
 size_t lite_la_workspace_bytes(int B, int N, int H, int d, int tokens_per_block) {
   if (B < 0 || N < 0 || H < 0 || d != litela::kD) return 0;
   litela::Plan p;
-  if (!litela::make_plan(B, N, H, tokens_per_block, &p)) return 0;
-  return p.bytes + p.counters * sizeof(unsigned);
+  if (!litela::make_plan(B, N, H, tokens_per_block, 148, &p)) return 0;
+  return p.bytes + (litela::kCounterBase + p.counters) * sizeof(unsigned);
 }
 
 }  // extern "C"

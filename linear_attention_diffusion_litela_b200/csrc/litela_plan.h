@@ -1,6 +1,6 @@
-// Host-side partition of one LiteLA call into reduce chunks, blocks and apply tiles.
-// Plain C++ (no CUDA), so the same arithmetic is compiled into the library and can be
-// queried on a machine without a GPU.
+// Host-side partition of one LiteLA call into causal blocks, state-reduction CTAs and apply
+// work items, and the layout of the workspace.  Plain C++ (no CUDA), so the same arithmetic is
+// compiled into the library and can be queried on a machine without a GPU.
 #pragma once
 
 #include <cstddef>
@@ -12,52 +12,72 @@ constexpr int kD = 32;             // head dim (Sana's linear_head_dim)
 constexpr int kRows = kD + 1;      // state rows: d value channels + the ones (denominator) row
 constexpr int kStateFloats = kRows * kD;
 
+// state reduction: a CTA owns 4 heads (the MMA's M = 4 x 32 key channels) and one chunk of
+// tokens inside one causal block, streamed in stages of 64 tokens
+constexpr int kRedHeads = 4;
+constexpr int kRedTile = 64;
+constexpr int kRedCtasPerSm = 2;
+// apply: a work item is 2 heads x one 128-token tile inside one causal block
+constexpr int kApHeads = 2;
+constexpr int kApTile = 128;
+// one head's state in the apply MMA's B-operand layout: 80 rows (33 hi rows + 7 zero rows,
+// 33 lo rows + 7 zero rows) x 32 bf16
+constexpr int kImageRows = 80;
+constexpr int kImageLoRow = 40;
+constexpr int kImageBytes = kImageRows * kD * 2;
+// workspace word where kernels report a wait that timed out (first error wins)
+constexpr int kCounterBase = 64;   // counters start 256 bytes into their buffer
+
 struct Plan {
   int B = 0, N = 0, H = 0;
   int T = 0;                 // tokens per causal block (N when non-causal)
   int nblk = 0;              // number of blocks, ceil(N / T)
-  int chunks_per_block = 0;  // reduce CTAs per (batch, head, block)
-  int chunk = 0;             // tokens per reduce CTA (a multiple of kReduceTile)
-  int tiles_per_block = 0;   // apply CTAs per (batch, head, block)
-  int apply_tile = 0;        // tokens per apply CTA
-  // state workspace layout, in bytes from its base (each region 256-byte aligned)
-  size_t off_partials = 0, off_states = 0, bytes = 0;
-  // arrival counters, one per (batch, head); they live in a separate zero-initialised
-  // buffer that the kernels leave at zero when they finish
+  int ngroups = 0;           // reduce head groups, ceil(H / 4)
+  int chunks_per_block = 0;  // reduce CTAs per (batch, group, block)
+  int chunk = 0;             // tokens per reduce CTA (a multiple of kRedTile)
+  int npairs = 0;            // apply head pairs, ceil(H / 2)
+  int tiles_per_block = 0;   // apply tiles per (batch, pair, block)
+  int64_t items = 0;         // apply work items
+  // state workspace, in bytes from its base (each region 256-byte aligned):
+  //   partials fp32 [B][ngroups][nblk * chunks_per_block][4][33][32]
+  //   images   bf16 [B][H][nblk][kImageBytes]
+  size_t off_partials = 0, off_images = 0, bytes = 0;
+  // arrival counters, one per (batch, group); they live after kCounterBase words of a
+  // separate zero-initialised buffer that the kernels leave at zero when they finish
   size_t counters = 0;
 };
-
-constexpr int kReduceTile = 32;     // tokens staged per reduce iteration
-constexpr int kApplyTile = 256;     // tokens per apply CTA (one per thread)
-constexpr int kTargetReduceCtas = 148 * 8;
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // tokens_per_block <= 0 or >= N selects the non-causal form.  Returns false for an empty
-// problem (B, N or H == 0); sizes must already be validated as non-negative.
-inline bool make_plan(int B, int N, int H, int tokens_per_block, Plan* p) {
+// problem (B, N or H == 0); sizes must already be validated as non-negative.  num_sms is the
+// device's SM count (148 on B200).
+inline bool make_plan(int B, int N, int H, int tokens_per_block, int num_sms, Plan* p) {
   *p = Plan{};
   if (B <= 0 || N <= 0 || H <= 0) return false;
   p->B = B; p->N = N; p->H = H;
   p->T = (tokens_per_block <= 0 || tokens_per_block >= N) ? N : tokens_per_block;
   p->nblk = (N + p->T - 1) / p->T;
-  const int64_t heads = (int64_t)B * H * p->nblk;
-  int64_t want = (kTargetReduceCtas + heads - 1) / heads;           // chunks per block
-  int64_t max_chunks = (p->T + kReduceTile - 1) / kReduceTile;
+  p->ngroups = (H + kRedHeads - 1) / kRedHeads;
+  const int64_t units = (int64_t)B * p->ngroups * p->nblk;
+  const int64_t target = (int64_t)(num_sms > 0 ? num_sms : 148) * kRedCtasPerSm;
+  int64_t want = target / units;                                  // chunks per block
+  const int64_t max_chunks = (p->T + kRedTile - 1) / kRedTile;
   if (want > max_chunks) want = max_chunks;
   if (want < 1) want = 1;
   int64_t chunk = (p->T + want - 1) / want;
-  chunk = (chunk + kReduceTile - 1) / kReduceTile * kReduceTile;
+  chunk = (chunk + kRedTile - 1) / kRedTile * kRedTile;
   p->chunk = (int)chunk;
   p->chunks_per_block = (int)((p->T + chunk - 1) / chunk);
-  p->apply_tile = kApplyTile;
-  p->tiles_per_block = (p->T + kApplyTile - 1) / kApplyTile;
-  const size_t partials = (size_t)heads * p->chunks_per_block * kStateFloats * sizeof(float);
-  const size_t states = (size_t)heads * kStateFloats * sizeof(float);
+  p->npairs = (H + kApHeads - 1) / kApHeads;
+  p->tiles_per_block = (p->T + kApTile - 1) / kApTile;
+  p->items = (int64_t)B * p->npairs * p->nblk * p->tiles_per_block;
+  const size_t partials = (size_t)units * p->chunks_per_block * kRedHeads * kStateFloats * sizeof(float);
+  const size_t images = (size_t)B * H * p->nblk * kImageBytes;
   p->off_partials = 0;
-  p->off_states = align_up(partials, 256);
-  p->bytes = p->off_states + align_up(states, 256);
-  p->counters = (size_t)B * H;
+  p->off_images = align_up(partials, 256);
+  p->bytes = p->off_images + align_up(images, 256);
+  p->counters = (size_t)B * p->ngroups;
   return true;
 }
 

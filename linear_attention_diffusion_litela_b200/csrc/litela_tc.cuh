@@ -1,0 +1,529 @@
+// LiteLA forward on the 5th-generation tensor cores (tcgen05, TMEM accumulators, TMA staging).
+//
+// Method (Sana explainer "Sana: the autoencoder does more of the work than the linear
+// attention", section "What LiteLA actually computes"): phi = ReLU on q and k, V padded with a
+// row of ones, state S = [V;1] . phi(K)^T (a (d+1) x d fp32 matrix per batch and head),
+// y = S . phi(q), out = y[:d] / (y[d] + eps).  Block-causal variant (instagit page "How Linear
+// Attention Improves Efficiency in DiT for High-Resolution Images", section "Video Generation
+// and Constant-Memory KV Cache"): a query in block b uses the sum of the per-block states of
+// blocks 0..b.
+//
+// litela_reduce_tc  (one CTA = 4 heads x one chunk of tokens inside one causal block)
+//   TMA streams the chunk's k and v columns of the 4 heads (64 tokens x 128 channels each, 128B
+//   swizzle) through a 3-stage ring.  Four ReLU warps clamp k in shared memory (and zero the
+//   rows of tokens outside the chunk).  One thread issues, per 16 tokens,
+//     D[0:128, 0:128]   += phi(K)^T . V     (M = 4 heads x 32 key channels, N = 4 x 32 values)
+//     D[0:128, 128:144] += phi(K)^T . 1     (the ones pad: the denominator row)
+//   with fp32 accumulators in TMEM; only the 4 diagonal 32 x 32 blocks of the first product
+//   are used (the off-diagonal blocks pair different heads and are discarded: the tensor core
+//   has 30x more throughput than this HBM-bound pass needs).  Products of bf16 values are exact
+//   in fp32, so this is the fp32 state the method specifies.  The epilogue writes the chunk's
+//   partial states; the last CTA of a (batch, head group) to finish sums the partials in fixed
+//   order (deterministic), forms the per-block inclusive prefix, and stores each head's state
+//   as the apply's B operand: S split into bf16 hi + lo (S = hi + lo to 2^-17 relative), and,
+//   when asked, as plain fp32 (d+1) x d matrices.
+//
+// litela_apply_tc  (persistent, one CTA per SM; work item = 2 heads x 128 tokens of a block)
+//   TMA streams q tiles (128 tokens x 64 channels, 128B swizzle) through a 6-stage ring; two
+//   ReLU warps clamp them in place; one thread issues y = phi(Q) . [S_hi ; S_lo]^T per head
+//   (M = 128 tokens, N = 80, K = 32) into one of three TMEM accumulator slots; four epilogue
+//   warps read them back (thread = token), form (y_hi + y_lo)[r] / ((y_hi + y_lo)[32] + eps)
+//   and store bf16 (or fp32).
+//
+// Every mbarrier wait is bounded (sm100::mbar_wait): on a time-out the kernel records an
+// error code in the workspace's error word, stops its loops, waits (bounded) for its own TMA
+// copies, frees its TMEM and returns.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "litela_plan.h"
+#include "sm100_ptx.cuh"
+
+namespace litela {
+
+struct TcPlan {
+  int B, N, H, T, nblk, ngroups, cpb, chunk, npairs, tpb;
+  long long items;
+  float eps;
+};
+
+// error codes written to the workspace error word: 0x100 | role << 4 | stage
+enum : int {
+  kErrReduceProducer = 0x110, kErrReduceMma = 0x120, kErrReduceRelu = 0x130, kErrReduceEpi = 0x140,
+  kErrApplyProducer = 0x210, kErrApplyMma = 0x220, kErrApplyRelu = 0x230, kErrApplyEpi = 0x240,
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// ReLU of 8 packed bf16 values (IEEE maxNum with +0: negative and -0 become +0)
+__device__ __forceinline__ uint4 relu_bf16x8(uint4 w) {
+  const __nv_bfloat162 z = __float2bfloat162_rn(0.f);
+  uint32_t* u = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&u[i]);
+    x = __hmax2(x, z);
+    u[i] = *reinterpret_cast<uint32_t*>(&x);
+  }
+  return w;
+}
+
+// byte offset of element (row n, column c) in a head's state image (the apply's B operand,
+// K-major without swizzle: 8 x 8 core matrices of 128 B, K-direction stride 128 B, 8-row
+// group stride 512 B)
+__device__ __forceinline__ uint32_t image_offset(int n, int c) {
+  return (uint32_t)((n >> 3) * 512 + (c >> 3) * 128 + (n & 7) * 16 + (c & 7) * 2);
+}
+
+// ---------------------------------------------------------------------------------------
+// state reduction
+
+constexpr int kRedStages = 3;
+constexpr int kRedThreads = 192;                       // w0 TMA, w1 MMA, w2..5 ReLU + epilogue
+constexpr uint32_t kRedBoxBytes = 64 * 2 * kRedTile;   // 64 channels x 64 tokens x bf16
+constexpr uint32_t kRedStageBytes = 4 * kRedBoxBytes;  // k lo/hi channels, v lo/hi channels
+constexpr uint32_t kRedTmemCols = 256;
+constexpr uint32_t kRedSmemBytes = kRedStages * kRedStageBytes + 512 + 256 + 1024;
+
+__global__ void __launch_bounds__(kRedThreads, 1)
+litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ partials,
+                 uint8_t* __restrict__ images, float* __restrict__ states_f32, unsigned* __restrict__ counters,
+                 int* __restrict__ err, TcPlan p) {
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* stages = smem;
+  uint8_t* ones = smem + kRedStages * kRedStageBytes;                 // 16 x 16 bf16 ones
+  uint64_t* full = reinterpret_cast<uint64_t*>(ones + 512);
+  uint64_t* relu_done = full + kRedStages;
+  uint64_t* empty = relu_done + kRedStages;
+  uint64_t* done = empty + kRedStages;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* last_flag = reinterpret_cast<int*>(tmem_holder + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int x = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int blk = x / p.cpb, ch = x - blk * p.cpb;
+  const int blk_end = min((blk + 1) * p.T, p.N);
+  const int n0 = blk * p.T + ch * p.chunk;
+  const int n1 = min(n0 + p.chunk, blk_end);
+  const int ntiles = n1 > n0 ? (n1 - n0 + kRedTile - 1) / kRedTile : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRedStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&relu_done[s], 128);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < 128; i += kRedThreads) reinterpret_cast<uint32_t*>(ones)[i] = 0x3F803F80u;
+  fence_proxy_async_smem();
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, kRedTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) prefetch_tensormap(&tmap);
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_holder;
+
+  const int kx = p.H * kD + g * (kRedHeads * kD);       // first key channel of the group
+  const int vx = 2 * p.H * kD + g * (kRedHeads * kD);   // first value channel of the group
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % kRedStages;
+        if (i >= kRedStages &&
+            !mbar_wait(&empty[s], ((i / kRedStages) - 1) & 1, abort_flag, err, kErrReduceProducer | s))
+          break;
+        uint8_t* st = stages + s * kRedStageBytes;
+        const int y = n0 + i * kRedTile;
+        mbar_arrive_expect_tx(&full[s], kRedStageBytes);
+        tma_load_3d(st, &tmap, &full[s], kx, y, b);
+        tma_load_3d(st + kRedBoxBytes, &tmap, &full[s], kx + 64, y, b);
+        tma_load_3d(st + 2 * kRedBoxBytes, &tmap, &full[s], vx, y, b);
+        tma_load_3d(st + 3 * kRedBoxBytes, &tmap, &full[s], vx + 64, y, b);
+        issued = i + 1;
+      }
+      if (*abort_flag) {   // let the copies still in flight land before the CTA exits (bounded)
+        for (int i = (issued > kRedStages ? issued - kRedStages : 0); i < issued; ++i)
+          mbar_drain(&full[i % kRedStages], (i / kRedStages) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && ntiles > 0) {
+      constexpr uint32_t idesc_num = idesc_bf16_f32(128, 128, true, true);
+      constexpr uint32_t idesc_den = idesc_bf16_f32(128, 16, true, false);
+      const uint64_t ones_desc = smem_desc(smem_u32(ones), 128, 256, kSwizzleNone);
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % kRedStages;
+        if (!mbar_wait(&relu_done[s], (i / kRedStages) & 1, abort_flag, err, kErrReduceMma | s)) break;
+        tc_fence_after_sync();
+        const uint32_t kbase = smem_u32(stages + s * kRedStageBytes);
+        const uint32_t vbase = kbase + 2 * kRedBoxBytes;
+#pragma unroll
+        for (int ks = 0; ks < kRedTile / 16; ++ks) {
+          // MN-major, 128B swizzle: 8-token row groups 1024 B apart, 64-channel blocks one box apart
+          const uint64_t a = smem_desc(kbase + ks * 2048, kRedBoxBytes, 1024, kSwizzle128B);
+          const uint64_t bv = smem_desc(vbase + ks * 2048, kRedBoxBytes, 1024, kSwizzle128B);
+          const uint32_t acc = (i | ks) != 0;
+          umma_bf16(tmem, a, bv, idesc_num, acc);
+          umma_bf16(tmem + 128, a, ones_desc, idesc_den, acc);
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(done);
+    }
+  } else {
+    const int t = threadIdx.x - 64;   // 0..127
+    for (int i = 0; i < ntiles; ++i) {
+      const int s = i % kRedStages;
+      if (!mbar_wait(&full[s], (i / kRedStages) & 1, abort_flag, err, kErrReduceRelu | s)) break;
+      uint8_t* st = stages + s * kRedStageBytes;
+      const int valid = min(kRedTile, n1 - (n0 + i * kRedTile));   // tokens of this chunk in the tile
+#pragma unroll 4
+      for (int j = t; j < 1024; j += 128) {          // k: 2 boxes x 64 rows x 8 chunks of 16 B
+        uint4* c = reinterpret_cast<uint4*>(st + j * 16);
+        const int row = (j >> 3) & (kRedTile - 1);
+        *c = row < valid ? relu_bf16x8(*c) : make_uint4(0u, 0u, 0u, 0u);
+      }
+      if (valid < kRedTile) {
+        for (int j = t; j < 1024; j += 128) {
+          const int row = (j >> 3) & (kRedTile - 1);
+          if (row >= valid) *reinterpret_cast<uint4*>(st + 2 * kRedBoxBytes + j * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&relu_done[s]);
+    }
+    // epilogue: warp quarter q reads TMEM lanes 32q..32q+31 = head q's key channels c
+    const int q = warp & 3;
+    float sv[kRows];
+    bool ok = ntiles > 0;
+    if (ok) ok = mbar_wait(done, 0, abort_flag, err, kErrReduceEpi);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after_sync();
+      uint32_t r[32], zr;
+      const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      tmem_ld_x32(ta + q * 32, r);
+      tmem_ld_x1(ta + 128, zr);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(r[j]);
+      sv[32] = __uint_as_float(zr);
+    } else {
+#pragma unroll
+      for (int j = 0; j < kRows; ++j) sv[j] = 0.f;
+    }
+    const int64_t nparts = (int64_t)p.nblk * p.cpb;
+    float* dst = partials + ((((int64_t)b * p.ngroups + g) * nparts + x) * kRedHeads + q) * kStateFloats;
+#pragma unroll
+    for (int j = 0; j < kRows; ++j) dst[j * kD + lane] = sv[j];   // S[r = j][c = lane]
+  }
+
+  // teardown of the tensor memory
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kRedTmemCols);
+  }
+
+  // the last CTA of this (batch, group) to arrive merges; no CTA ever waits for another
+  __threadfence();
+  __syncthreads();
+  const unsigned cidx = kCounterBase + (unsigned)b * p.ngroups + g;
+  const unsigned nparts = (unsigned)(p.nblk * p.cpb);
+  if (threadIdx.x == 0) *last_flag = (atomicAdd(&counters[cidx], 1u) == nparts - 1u) ? 1 : 0;
+  __syncthreads();
+  if (!*last_flag) return;
+  __threadfence();
+  const float* gp = partials + ((int64_t)b * p.ngroups + g) * nparts * (kRedHeads * kStateFloats);
+  const int heads_here = min(kRedHeads, p.H - g * kRedHeads);
+  for (int e = threadIdx.x; e < kRedHeads * kStateFloats; e += kRedThreads) {
+    const int hl = e / kStateFloats, rc = e - hl * kStateFloats, r = rc >> 5, c = rc & 31;
+    float run = 0.f;
+    for (int bb = 0; bb < p.nblk; ++bb) {
+      float s = 0.f;
+      for (int k = 0; k < p.cpb; ++k)
+        s += __ldcg(gp + ((int64_t)bb * p.cpb + k) * (kRedHeads * kStateFloats) + e);
+      run += s;
+      if (hl < heads_here && states_f32 != nullptr)
+        states_f32[(((int64_t)b * p.H + g * kRedHeads + hl) * p.nblk + bb) * kStateFloats + rc] = run;
+      if (hl < heads_here && images != nullptr) {
+        uint8_t* img = images + (((int64_t)b * p.H + g * kRedHeads + hl) * p.nblk + bb) * kImageBytes;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(run);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(run - __bfloat162float(hi));
+        *reinterpret_cast<__nv_bfloat16*>(img + image_offset(r, c)) = hi;
+        *reinterpret_cast<__nv_bfloat16*>(img + image_offset(kImageLoRow + r, c)) = lo;
+      }
+    }
+  }
+  // zero rows of the images: 33..39 and 73..79 (7 + 7 rows x 32 columns)
+  const int zeros_per_image = 14 * kD;
+  for (int e = threadIdx.x; images != nullptr && e < heads_here * p.nblk * zeros_per_image; e += kRedThreads) {
+    const int im = e / zeros_per_image, k = e - im * zeros_per_image;
+    const int hl = im / p.nblk, bb = im - hl * p.nblk;
+    const int zr = k >> 5, c = k & 31;
+    const int n = zr < 7 ? kRows + zr : kImageLoRow + kRows + (zr - 7);
+    uint8_t* img = images + (((int64_t)b * p.H + g * kRedHeads + hl) * p.nblk + bb) * kImageBytes;
+    *reinterpret_cast<__nv_bfloat16*>(img + image_offset(n, c)) = __float2bfloat16_rn(0.f);
+  }
+  if (threadIdx.x == 0) counters[cidx] = 0u;
+}
+
+// ---------------------------------------------------------------------------------------
+// apply
+
+constexpr int kApStages = 6;
+constexpr int kApThreads = 256;                        // w0 TMA, w1 MMA, w2..3 ReLU, w4..7 epilogue
+constexpr uint32_t kApStageBytes = kApTile * 64 * 2;   // 128 tokens x 64 channels x bf16
+constexpr int kApAccSlots = 3;
+constexpr uint32_t kApAccCols = kApHeads * kImageRows; // 160 fp32 columns per slot
+constexpr uint32_t kApTmemCols = 512;
+constexpr uint32_t kApSbufBytes = kApHeads * kImageBytes;
+constexpr uint32_t kApSmemBytes = kApStages * kApStageBytes + 2 * kApSbufBytes + 512 + 1024;
+
+struct ApItem {
+  int b, pair, blk, tok0, tok1;
+  long long seg;
+};
+
+__device__ __forceinline__ ApItem ap_decode(long long it, const TcPlan& p) {
+  ApItem I;
+  const int tile = (int)(it % p.tpb);
+  I.seg = it / p.tpb;
+  long long r = I.seg;
+  I.blk = (int)(r % p.nblk);
+  r /= p.nblk;
+  I.pair = (int)(r % p.npairs);
+  I.b = (int)(r / p.npairs);
+  I.tok0 = I.blk * p.T + tile * kApTile;
+  I.tok1 = min(I.tok0 + kApTile, min((I.blk + 1) * p.T, p.N));
+  return I;
+}
+
+template <typename OutT>
+__device__ __forceinline__ void store_row(OutT* dst, const float* o);
+
+template <>
+__device__ __forceinline__ void store_row<__nv_bfloat16>(__nv_bfloat16* dst, const float* o) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      __nv_bfloat162 v2 = __floats2bfloat162_rn(o[i * 8 + 2 * j], o[i * 8 + 2 * j + 1]);
+      w[j] = *reinterpret_cast<uint32_t*>(&v2);
+    }
+    d4[i] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+template <>
+__device__ __forceinline__ void store_row<float>(float* dst, const float* o) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) d4[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+}
+
+template <typename OutT>
+__global__ void __launch_bounds__(kApThreads, 1)
+litela_apply_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t* __restrict__ images,
+                OutT* __restrict__ out, int* __restrict__ err, TcPlan p) {
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* qst = smem;                                            // kApStages q tiles
+  uint8_t* sbuf = smem + kApStages * kApStageBytes;               // 2 state buffers
+  uint64_t* qfull = reinterpret_cast<uint64_t*>(sbuf + 2 * kApSbufBytes);
+  uint64_t* qrelu = qfull + kApStages;
+  uint64_t* qempty = qrelu + kApStages;
+  uint64_t* sfull = qempty + kApStages;
+  uint64_t* sempty = sfull + 2;
+  uint64_t* tfull = sempty + 2;
+  uint64_t* tempty = tfull + kApAccSlots;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + kApAccSlots);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long w0 = (long long)blockIdx.x * p.items / gridDim.x;
+  const long long w1 = (long long)(blockIdx.x + 1) * p.items / gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kApStages; ++s) {
+      mbar_init(&qfull[s], 1);
+      mbar_init(&qrelu[s], 64);
+      mbar_init(&qempty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sfull[s], 1);
+      mbar_init(&sempty[s], 1);
+    }
+    for (int s = 0; s < kApAccSlots; ++s) {
+      mbar_init(&tfull[s], 1);
+      mbar_init(&tempty[s], 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, kApTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) prefetch_tensormap(&tmap);
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      long long prev = -1;
+      int seg_n = -1, seg_loaded = -1, issued = 0;
+      for (long long it = w0; it < w1; ++it) {
+        const int li = (int)(it - w0);
+        const ApItem I = ap_decode(it, p);
+        if (I.seg != prev) {
+          prev = I.seg;
+          ++seg_n;
+          const int sb = seg_n & 1;
+          if (seg_n >= 2 &&
+              !mbar_wait(&sempty[sb], ((seg_n >> 1) - 1) & 1, abort_flag, err, kErrApplyProducer | 8 | sb))
+            break;
+          const int nh = min(kApHeads, p.H - I.pair * kApHeads);
+          mbar_arrive_expect_tx(&sfull[sb], nh * kImageBytes);
+          for (int j = 0; j < nh; ++j) {
+            const uint8_t* src =
+                images + (((int64_t)I.b * p.H + I.pair * kApHeads + j) * p.nblk + I.blk) * kImageBytes;
+            bulk_load(sbuf + sb * kApSbufBytes + j * kImageBytes, src, kImageBytes, &sfull[sb]);
+          }
+          seg_loaded = seg_n;
+        }
+        const int s = li % kApStages;
+        if (li >= kApStages &&
+            !mbar_wait(&qempty[s], ((li / kApStages) - 1) & 1, abort_flag, err, kErrApplyProducer | s))
+          break;
+        mbar_arrive_expect_tx(&qfull[s], kApStageBytes);
+        tma_load_3d(qst + s * kApStageBytes, &tmap, &qfull[s], I.pair * kApHeads * kD, I.tok0, I.b);
+        issued = li + 1;
+      }
+      if (*abort_flag) {   // let the copies still in flight land before the CTA exits (bounded)
+        for (int i = (issued > kApStages ? issued - kApStages : 0); i < issued; ++i)
+          mbar_drain(&qfull[i % kApStages], (i / kApStages) & 1);
+        for (int k = (seg_loaded > 0 ? seg_loaded - 1 : 0); k <= seg_loaded; ++k)
+          mbar_drain(&sfull[k & 1], (k >> 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, kImageRows, false, false);
+      long long prev = -1;
+      int seg_n = -1, sb = 0;
+      for (long long it = w0; it < w1; ++it) {
+        const int li = (int)(it - w0);
+        const ApItem I = ap_decode(it, p);
+        if (I.seg != prev) {
+          prev = I.seg;
+          ++seg_n;
+          sb = seg_n & 1;
+          if (!mbar_wait(&sfull[sb], (seg_n >> 1) & 1, abort_flag, err, kErrApplyMma | 8 | sb)) break;
+        }
+        const int s = li % kApStages, a = li % kApAccSlots;
+        if (!mbar_wait(&qrelu[s], (li / kApStages) & 1, abort_flag, err, kErrApplyMma | s)) break;
+        if (li >= kApAccSlots &&
+            !mbar_wait(&tempty[a], ((li / kApAccSlots) - 1) & 1, abort_flag, err, kErrApplyMma | 12 | a))
+          break;
+        tc_fence_after_sync();
+        const int nh = min(kApHeads, p.H - I.pair * kApHeads);
+        const uint32_t qaddr = smem_u32(qst + s * kApStageBytes);
+        const uint32_t saddr = smem_u32(sbuf + sb * kApSbufBytes);
+        for (int j = 0; j < nh; ++j) {
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks) {
+            // A: K-major 128B swizzle, 8-token groups 1024 B apart; head j's 32 channels at +64j B
+            const uint64_t ad = smem_desc(qaddr + j * 64 + ks * 32, 16, 1024, kSwizzle128B);
+            // B: K-major no swizzle, K-direction core matrices 128 B apart, row groups 512 B apart
+            const uint64_t bd = smem_desc(saddr + j * kImageBytes + ks * 256, 128, 512, kSwizzleNone);
+            umma_bf16(tmem + a * kApAccCols + j * kImageRows, ad, bd, idesc, ks);
+          }
+        }
+        umma_commit(&qempty[s]);
+        umma_commit(&tfull[a]);
+        const bool seg_ends = (it + 1 >= w1) || (ap_decode(it + 1, p).seg != I.seg);
+        if (seg_ends) umma_commit(&sempty[sb]);
+      }
+    }
+  } else if (warp < 4) {
+    const int t = threadIdx.x - 64;   // 0..63
+    for (long long it = w0; it < w1; ++it) {
+      const int li = (int)(it - w0);
+      const int s = li % kApStages;
+      if (!mbar_wait(&qfull[s], (li / kApStages) & 1, abort_flag, err, kErrApplyRelu | s)) break;
+      uint8_t* st = qst + s * kApStageBytes;
+#pragma unroll 4
+      for (int j = t; j < (int)(kApStageBytes / 16); j += 64) {
+        uint4* c = reinterpret_cast<uint4*>(st + j * 16);
+        *c = relu_bf16x8(*c);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&qrelu[s]);
+    }
+  } else {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    for (long long it = w0; it < w1; ++it) {
+      const int li = (int)(it - w0);
+      const int a = li % kApAccSlots;
+      const ApItem I = ap_decode(it, p);
+      bool ok = mbar_wait(&tfull[a], (li / kApAccSlots) & 1, abort_flag, err, kErrApplyEpi | a);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after_sync();
+      const int nh = min(kApHeads, p.H - I.pair * kApHeads);
+      const int n = I.tok0 + row;
+      const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + a * kApAccCols;
+      for (int j = 0; j < nh; ++j) {
+        uint32_t v[kImageRows];
+#pragma unroll
+        for (int k = 0; k < kImageRows / 16; ++k) tmem_ld_x16(ta + j * kImageRows + k * 16, v + k * 16);
+        tmem_wait_ld();
+        if (j == nh - 1) {
+          tc_fence_before_sync();
+          mbar_arrive(&tempty[a]);
+        }
+        if (n < I.tok1) {
+          const float den = (__uint_as_float(v[kD]) + __uint_as_float(v[kImageLoRow + kD])) + p.eps;
+          const float inv = 1.0f / den;
+          float o[kD];
+#pragma unroll
+          for (int r = 0; r < kD; ++r)
+            o[r] = (__uint_as_float(v[r]) + __uint_as_float(v[kImageLoRow + r])) * inv;
+          store_row<OutT>(out + (((int64_t)I.b * p.N + n) * p.H + I.pair * kApHeads + j) * kD, o);
+        }
+      }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kApTmemCols);
+  }
+}
+
+}  // namespace litela

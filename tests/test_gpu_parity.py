@@ -37,6 +37,7 @@ def gpu_run(qkv, H, T=None, mode="bf16"):
     else:
         out = ll.lite_la_block_causal_fwd(qkv, H, T, eps=EPS, out_dtype=dt)
     torch.cuda.synchronize()
+    ll.lite_la_device_status()
     B, N = qkv.shape[:2]
     return out.view(B, N, H, 32).to(torch.float64).cpu().numpy()
 
@@ -198,3 +199,35 @@ def test_workspace_allocation_failure_is_reported(monkeypatch):
     out = ll.lite_la_fwd(qkv, 1, stream=s, out_dtype=torch.float32)
     s.synchronize()
     assert_close(out.view(1, 64, 1, 32).double().cpu().numpy(), oracle_run(qkv, 1), "f32")
+
+
+def state_reference(bits, B, N, H, T):
+    """[V;1]^T . relu(K) per (batch, head), summed over blocks 0..k (fp64, from the decoded
+    bf16 inputs): the state the pages define, used to check lite_la_state_fwd."""
+    x = oracle.decode_bf16(bits).reshape(B, N, 3 * H * 32)
+    _, k, v = oracle.unpack_qkv(x, H, 32)
+    T = T if 0 < T < N else N
+    nblk = -(-N // T)
+    out = np.zeros((B, H, nblk, 33, 32))
+    for b in range(B):
+        for h in range(H):
+            run = np.zeros((33, 32))
+            for blk in range(nblk):
+                kk = np.maximum(k[b, blk * T:(blk + 1) * T, h], 0.0)
+                vv = np.concatenate([v[b, blk * T:(blk + 1) * T, h], np.ones((kk.shape[0], 1))], axis=1)
+                run = run + vv.T @ kk
+                out[b, h, blk] = run
+    return out
+
+
+@pytest.mark.parametrize("B,N,H,T", [(1, 1, 1, 0), (1, 65, 3, 0), (2, 1000, 5, 0), (1, 300, 4, 128),
+                                     (2, 100, 2, 7), (1, 4096, 70, 1024)])
+def test_state_fwd_matches_padded_state_definition(B, N, H, T):
+    qkv = make_qkv(B, N, H, 32, seed=3 * N + H + T, device="cuda")
+    st = ll.lite_la_state_fwd(qkv, H, T)
+    ll.lite_la_device_status()
+    ref = state_reference(to_bits(qkv), B, N, H, T)
+    got = st.double().cpu().numpy()
+    # fp32 sums of exact bf16 products: relative error ~ sqrt(N) * 2^-24 of the magnitudes
+    scale = np.abs(ref).max(axis=(-1, -2), keepdims=True) + 1e-30
+    assert np.all(np.abs(got - ref) <= 1e-5 * scale + 1e-6)
