@@ -67,9 +67,9 @@ litela_status device_setup(int* num_sms) {
     if ((e = cudaFuncSetAttribute(litela_reduce_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kRedSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_apply_tc<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)kApSmemBytes)) != cudaSuccess ||
+                                  (int)ApplyCfg<__nv_bfloat16>::kSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_apply_tc<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)kApSmemBytes)) != cudaSuccess)
+                                  (int)ApplyCfg<float>::kSmemBytes)) != cudaSuccess)
       return cuda_fail(e, "cudaFuncSetAttribute(dynamic shared memory)");
     if (g_encode == nullptr) {
       void* fn = nullptr;
@@ -100,14 +100,32 @@ litela_status encode_qkv_map(const void* qkv, int B, int N, int H, int box_token
   return LITELA_OK;
 }
 
+// 3-D view of the output [B, N, H*d] for TMA stores: (channel, token, batch), boxes of
+// 128 bytes of channels x kApTile tokens, 128-byte swizzle.
+template <typename OutT>
+litela_status encode_out_map(OutT* out, int B, int N, int H, CUtensorMap* map) {
+  const CUtensorMapDataType dt =
+      sizeof(OutT) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const cuuint64_t row = (cuuint64_t)H * kD;
+  const cuuint64_t dims[3] = {row, (cuuint64_t)N, (cuuint64_t)B};
+  const cuuint64_t strides[2] = {row * sizeof(OutT), row * sizeof(OutT) * (cuuint64_t)N};
+  const cuuint32_t box[3] = {(cuuint32_t)(128 / sizeof(OutT)), (cuuint32_t)kApTile, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, dt, 3, static_cast<void*>(out), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(LITELA_ERR_CUDA, "cuTensorMapEncodeTiled(out) failed (" + std::to_string((int)r) + ")");
+  return LITELA_OK;
+}
+
 // ---------------------------------------------------------------------------------------
 // workspace: one per (device, stream)
 
 struct Workspace {
-  void* states = nullptr;
-  size_t states_bytes = 0;
-  unsigned* counters = nullptr;   // word 0: device error word; counters from kCounterBase
-  size_t counters_len = 0;
+  void* partials = nullptr;
+  size_t partials_bytes = 0;
+  int* err = nullptr;   // kErrWords words; word 0 is the kernels' error word
 };
 
 std::mutex g_ws_mutex;
@@ -126,38 +144,33 @@ litela_status get_workspace(const Plan& plan, cudaStream_t stream, Workspace** o
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   std::lock_guard<std::mutex> lock(g_ws_mutex);
   Workspace& ws = g_ws[{dev, reinterpret_cast<uintptr_t>(stream)}];
-  const size_t need_counters = kCounterBase + plan.counters;
-  const bool grow_states = ws.states_bytes < plan.bytes;
-  const bool grow_counters = ws.counters_len < need_counters;
-  if (grow_states || grow_counters) {
+  const bool grow = ws.partials_bytes < plan.bytes || ws.err == nullptr;
+  if (grow) {
     if (alloc_fault_injected())
       return fail(LITELA_ERR_OUT_OF_MEMORY, "workspace allocation failed (injected by LITELA_FAIL_ALLOC)");
-    // kernels of earlier calls on this stream may still use the old buffers
+    // kernels of earlier calls on this stream may still use the old buffer
     e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize before workspace growth");
-    if (grow_states) {
-      if (ws.states) cudaFree(ws.states);
-      ws.states = nullptr;
-      ws.states_bytes = 0;
-      e = cudaMalloc(&ws.states, plan.bytes);
+    if (ws.err == nullptr) {
+      e = cudaMalloc(&ws.err, kErrWords * sizeof(int));
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        ws.err = nullptr;
+        return fail(LITELA_ERR_OUT_OF_MEMORY, std::string("error-word cudaMalloc: ") + cudaGetErrorString(e));
+      }
+      e = cudaMemset(ws.err, 0, kErrWords * sizeof(int));
+      if (e != cudaSuccess) return cuda_fail(e, "cudaMemset error word");
+    }
+    if (ws.partials_bytes < plan.bytes) {
+      if (ws.partials) cudaFree(ws.partials);
+      ws.partials = nullptr;
+      ws.partials_bytes = 0;
+      e = cudaMalloc(&ws.partials, plan.bytes);
       if (e != cudaSuccess) {
         cudaGetLastError();
         return fail(LITELA_ERR_OUT_OF_MEMORY, std::string("workspace cudaMalloc: ") + cudaGetErrorString(e));
       }
-      ws.states_bytes = plan.bytes;
-    }
-    if (grow_counters) {
-      if (ws.counters) cudaFree(ws.counters);
-      ws.counters = nullptr;
-      ws.counters_len = 0;
-      e = cudaMalloc(&ws.counters, need_counters * sizeof(unsigned));
-      if (e != cudaSuccess) {
-        cudaGetLastError();
-        return fail(LITELA_ERR_OUT_OF_MEMORY, std::string("counter cudaMalloc: ") + cudaGetErrorString(e));
-      }
-      e = cudaMemset(ws.counters, 0, need_counters * sizeof(unsigned));
-      if (e != cudaSuccess) return cuda_fail(e, "cudaMemset counters");
-      ws.counters_len = need_counters;
+      ws.partials_bytes = plan.bytes;
     }
   }
   *out = &ws;
@@ -196,29 +209,54 @@ litela_status validate(const void* qkv, const void* out, size_t out_elem, int B,
   return LITELA_OK;
 }
 
-// Launches the state reduction and the apply for `plan` with the given scratch.
+TcPlan tc_plan(const Plan& plan, float eps) {
+  return TcPlan{plan.B,       plan.N,      plan.H,     plan.T, plan.nblk, plan.ngroups, plan.chunks_per_block,
+                plan.chunk,   plan.npairs, plan.tiles_per_block, (long long)plan.items, eps};
+}
+
+litela_status launch_reduce(const Plan& plan, const void* qkv, float* partials, int* err, cudaStream_t stream) {
+  CUtensorMap map;
+  litela_status s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kRedTile, &map);
+  if (s != LITELA_OK) return s;
+  dim3 grid(plan.nblk * plan.chunks_per_block, plan.ngroups, plan.B);
+  litela_reduce_tc<<<grid, kRedThreads, kRedSmemBytes, stream>>>(map, partials, err, tc_plan(plan, 0.f));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "launch litela_reduce_tc");
+  return LITELA_OK;
+}
+
+// Launches the state reduction and the apply for `plan` with the given scratch.  The apply is
+// a programmatic dependent of the reduction (its prologue and q prefetch overlap the
+// reduction's end) unless phase events are requested, in which case the two run in plain
+// stream order with an event between them.
 template <typename OutT>
-litela_status launch(const Plan& plan, const void* qkv, OutT* out, float eps, float* partials,
-                     uint8_t* images, unsigned* counters, int num_sms, cudaStream_t stream,
-                     cudaEvent_t* events) {
-  CUtensorMap map_red, map_ap;
-  litela_status s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kRedTile, &map_red);
+litela_status launch(const Plan& plan, const void* qkv, OutT* out, float eps, float* partials, int* err,
+                     int num_sms, cudaStream_t stream, cudaEvent_t* events) {
+  CUtensorMap map_q, map_out;
+  litela_status s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kApTile, &map_q);
   if (s != LITELA_OK) return s;
-  s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kApTile, &map_ap);
+  s = encode_out_map(out, plan.B, plan.N, plan.H, &map_out);
   if (s != LITELA_OK) return s;
-  TcPlan tp{plan.B, plan.N, plan.H, plan.T, plan.nblk, plan.ngroups, plan.chunks_per_block, plan.chunk,
-            plan.npairs, plan.tiles_per_block, (long long)plan.items, eps};
-  int* err = reinterpret_cast<int*>(counters);
   cudaError_t e;
   if (events && (e = cudaEventRecord(events[0], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  dim3 rgrid(plan.nblk * plan.chunks_per_block, plan.ngroups, plan.B);
-  litela_reduce_tc<<<rgrid, kRedThreads, kRedSmemBytes, stream>>>(map_red, partials, images, nullptr, counters,
-                                                                   err, tp);
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "launch litela_reduce_tc");
+  s = launch_reduce(plan, qkv, partials, err, stream);
+  if (s != LITELA_OK) return s;
   if (events && (e = cudaEventRecord(events[1], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  const TcPlan tp = tc_plan(plan, eps);
   const long long grid = plan.items < num_sms ? plan.items : num_sms;
-  litela_apply_tc<OutT><<<(unsigned)grid, kApThreads, kApSmemBytes, stream>>>(map_ap, images, out, err, tp);
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "launch litela_apply_tc");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kApThreads);
+  cfg.dynamicSmemBytes = ApplyCfg<OutT>::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = events ? 0 : 1;
+  e = cudaLaunchKernelEx(&cfg, litela_apply_tc<OutT>, map_q, map_out, static_cast<const float*>(partials), out, err,
+                         tp);
+  if (e != cudaSuccess) return cuda_fail(e, "launch litela_apply_tc");
   if (events && (e = cudaEventRecord(events[2], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   return LITELA_OK;
 }
@@ -240,18 +278,12 @@ litela_status run_states(const void* qkv, float* states, int B, int N, int H, in
   Workspace* ws = nullptr;
   s = get_workspace(plan, stream, &ws);
   if (s != LITELA_OK) return s;
-  CUtensorMap map_red;
-  s = encode_qkv_map(qkv, B, N, H, kRedTile, &map_red);
+  float* partials = static_cast<float*>(ws->partials);
+  s = launch_reduce(plan, qkv, partials, ws->err, stream);
   if (s != LITELA_OK) return s;
-  TcPlan tp{plan.B, plan.N, plan.H, plan.T, plan.nblk, plan.ngroups, plan.chunks_per_block, plan.chunk,
-            plan.npairs, plan.tiles_per_block, (long long)plan.items, 0.f};
-  char* base = static_cast<char*>(ws->states);
-  dim3 rgrid(plan.nblk * plan.chunks_per_block, plan.ngroups, plan.B);
-  litela_reduce_tc<<<rgrid, kRedThreads, kRedSmemBytes, stream>>>(
-      map_red, reinterpret_cast<float*>(base + plan.off_partials), nullptr, states, ws->counters,
-      reinterpret_cast<int*>(ws->counters), tp);
+  litela_state_merge<<<dim3(H, B), 256, 0, stream>>>(partials, states, tc_plan(plan, 0.f));
   cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "launch litela_reduce_tc");
+  if (e != cudaSuccess) return cuda_fail(e, "launch litela_state_merge");
   g_last_error.clear();
   return LITELA_OK;
 }
@@ -270,9 +302,7 @@ litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float 
   Workspace* ws = nullptr;
   s = get_workspace(plan, stream, &ws);
   if (s != LITELA_OK) return s;
-  char* base = static_cast<char*>(ws->states);
-  s = launch(plan, qkv, out, eps, reinterpret_cast<float*>(base + plan.off_partials),
-             reinterpret_cast<uint8_t*>(base + plan.off_images), ws->counters, num_sms, stream, events);
+  s = launch(plan, qkv, out, eps, static_cast<float*>(ws->partials), ws->err, num_sms, stream, events);
   if (s == LITELA_OK) g_last_error.clear();
   return s;
 }
@@ -312,8 +342,8 @@ litela_status run_noalloc(const void* qkv, __nv_bfloat16* out, int B, int N, int
   if (s != LITELA_OK) return s;
   Plan plan;
   make_plan(B, N, H, 0, num_sms, &plan);
-  const size_t counter_bytes = align_up((kCounterBase + plan.counters) * sizeof(unsigned), 256);
-  const size_t need = counter_bytes + plan.bytes;
+  const size_t err_bytes = align_up(kErrWords * sizeof(int), 256);
+  const size_t need = err_bytes + plan.bytes;
   if (need > LITELA_NOALLOC_SCRATCH_BYTES)
     return fail(LITELA_ERR_INVALID_ARGUMENT,
                 "problem needs " + std::to_string(need) + " bytes of scratch; lite_la_fwd_noalloc has " +
@@ -322,12 +352,8 @@ litela_status run_noalloc(const void* qkv, __nv_bfloat16* out, int B, int N, int
   s = noalloc_scratch(&scratch);
   if (s != LITELA_OK) return s;
   char* base = static_cast<char*>(scratch);
-  unsigned* counters = reinterpret_cast<unsigned*>(base);
-  cudaError_t e = cudaMemsetAsync(counters, 0, (kCounterBase + plan.counters) * sizeof(unsigned), stream);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(no-alloc counters)");
-  s = launch(plan, qkv, out, eps, reinterpret_cast<float*>(base + counter_bytes + plan.off_partials),
-             reinterpret_cast<uint8_t*>(base + counter_bytes + plan.off_images), counters, num_sms, stream,
-             nullptr);
+  s = launch(plan, qkv, out, eps, reinterpret_cast<float*>(base + err_bytes), reinterpret_cast<int*>(base), num_sms,
+             stream, nullptr);
   if (s == LITELA_OK) g_last_error.clear();
   return s;
 }
@@ -380,18 +406,18 @@ litela_status lite_la_device_status(cudaStream_t stream) {
   if (e != cudaSuccess) return litela::cuda_fail(e, "cudaGetDevice");
   e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) return litela::cuda_fail(e, "cudaStreamSynchronize");
-  unsigned* words[2] = {nullptr, nullptr};
+  int* words[2] = {nullptr, nullptr};
   {
     std::lock_guard<std::mutex> lock(litela::g_ws_mutex);
     auto it = litela::g_ws.find({dev, reinterpret_cast<uintptr_t>(stream)});
-    if (it != litela::g_ws.end()) words[0] = it->second.counters;
+    if (it != litela::g_ws.end()) words[0] = it->second.err;
   }
   {
     std::lock_guard<std::mutex> lock(litela::g_noalloc_mutex);
-    if (dev < litela::kMaxDevices) words[1] = static_cast<unsigned*>(litela::g_noalloc_ptr[dev]);
+    if (dev < litela::kMaxDevices) words[1] = static_cast<int*>(litela::g_noalloc_ptr[dev]);
   }
   int code = 0;
-  for (unsigned* w : words) {
+  for (int* w : words) {
     if (w == nullptr) continue;
     int v = 0;
     if ((e = cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
@@ -432,8 +458,8 @@ litela_status lite_la_release_workspace(void) {
   for (auto& kv : litela::g_ws) {
     if (cudaSetDevice(kv.first.first) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
       s = litela::fail(LITELA_ERR_CUDA, "device synchronisation before workspace release failed");
-    if (kv.second.states) cudaFree(kv.second.states);
-    if (kv.second.counters) cudaFree(kv.second.counters);
+    if (kv.second.partials) cudaFree(kv.second.partials);
+    if (kv.second.err) cudaFree(kv.second.err);
   }
   litela::g_ws.clear();
   cudaSetDevice(cur);
@@ -444,7 +470,7 @@ size_t lite_la_workspace_bytes(int B, int N, int H, int d, int tokens_per_block)
   if (B < 0 || N < 0 || H < 0 || d != litela::kD) return 0;
   litela::Plan p;
   if (!litela::make_plan(B, N, H, tokens_per_block, 148, &p)) return 0;
-  return p.bytes + (litela::kCounterBase + p.counters) * sizeof(unsigned);
+  return p.bytes + litela::kErrWords * sizeof(int);
 }
 
 }  // extern "C"

@@ -20,13 +20,13 @@ constexpr int kRedCtasPerSm = 2;
 // apply: a work item is 2 heads x one 128-token tile inside one causal block
 constexpr int kApHeads = 2;
 constexpr int kApTile = 128;
-// one head's state in the apply MMA's B-operand layout: 80 rows (33 hi rows + 7 zero rows,
-// 33 lo rows + 7 zero rows) x 32 bf16
+// one head's state in the apply MMA's B-operand layout (in shared memory): 80 rows (33 hi rows
+// + 7 zero rows, 33 lo rows + 7 zero rows) x 32 bf16
 constexpr int kImageRows = 80;
 constexpr int kImageLoRow = 40;
 constexpr int kImageBytes = kImageRows * kD * 2;
-// workspace word where kernels report a wait that timed out (first error wins)
-constexpr int kCounterBase = 64;   // counters start 256 bytes into their buffer
+// the kernels' error word (a bounded wait that timed out) lives in its own small buffer
+constexpr int kErrWords = 64;
 
 struct Plan {
   int B = 0, N = 0, H = 0;
@@ -38,13 +38,8 @@ struct Plan {
   int npairs = 0;            // apply head pairs, ceil(H / 2)
   int tiles_per_block = 0;   // apply tiles per (batch, pair, block)
   int64_t items = 0;         // apply work items
-  // state workspace, in bytes from its base (each region 256-byte aligned):
-  //   partials fp32 [B][ngroups][nblk * chunks_per_block][4][33][32]
-  //   images   bf16 [B][H][nblk][kImageBytes]
-  size_t off_partials = 0, off_images = 0, bytes = 0;
-  // arrival counters, one per (batch, group); they live after kCounterBase words of a
-  // separate zero-initialised buffer that the kernels leave at zero when they finish
-  size_t counters = 0;
+  // workspace: partial states fp32 [B][ngroups][nblk * chunks_per_block][4][33][32]
+  size_t bytes = 0;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -73,11 +68,7 @@ inline bool make_plan(int B, int N, int H, int tokens_per_block, int num_sms, Pl
   p->tiles_per_block = (p->T + kApTile - 1) / kApTile;
   p->items = (int64_t)B * p->npairs * p->nblk * p->tiles_per_block;
   const size_t partials = (size_t)units * p->chunks_per_block * kRedHeads * kStateFloats * sizeof(float);
-  const size_t images = (size_t)B * H * p->nblk * kImageBytes;
-  p->off_partials = 0;
-  p->off_images = align_up(partials, 256);
-  p->bytes = p->off_images + align_up(images, 256);
-  p->counters = (size_t)B * p->ngroups;
+  p->bytes = align_up(partials, 256);
   return true;
 }
 

@@ -18,17 +18,20 @@
 //   are used (the off-diagonal blocks pair different heads and are discarded: the tensor core
 //   has 30x more throughput than this HBM-bound pass needs).  Products of bf16 values are exact
 //   in fp32, so this is the fp32 state the method specifies.  The epilogue writes the chunk's
-//   partial states; the last CTA of a (batch, head group) to finish sums the partials in fixed
-//   order (deterministic), forms the per-block inclusive prefix, and stores each head's state
-//   as the apply's B operand: S split into bf16 hi + lo (S = hi + lo to 2^-17 relative), and,
-//   when asked, as plain fp32 (d+1) x d matrices.
+//   partial states [4][33][32] to the workspace; nothing else (no atomics, no merge tail).
 //
 // litela_apply_tc  (persistent, one CTA per SM; work item = 2 heads x 128 tokens of a block)
-//   TMA streams q tiles (128 tokens x 64 channels, 128B swizzle) through a 6-stage ring; two
-//   ReLU warps clamp them in place; one thread issues y = phi(Q) . [S_hi ; S_lo]^T per head
-//   (M = 128 tokens, N = 80, K = 32) into one of three TMEM accumulator slots; four epilogue
-//   warps read them back (thread = token), form (y_hi + y_lo)[r] / ((y_hi + y_lo)[32] + eps)
-//   and store bf16 (or fp32).
+//   Two merge warps sum the partial states of the CTA's heads in fixed order (deterministic;
+//   for the block-causal form a running inclusive prefix over blocks) and write each head's
+//   state into shared memory as the MMA's B operand, split into bf16 hi + lo (S = hi + lo to
+//   2^-17 relative).  TMA streams q tiles (128 tokens x 64 channels, 128B swizzle) through a
+//   6-stage ring; two ReLU warps clamp them in place; one thread issues
+//   y = phi(Q) . [S_hi ; S_lo]^T per head (M = 128 tokens, N = 80, K = 32) into one of three
+//   TMEM accumulator slots; four epilogue warps read them back (thread = token), form
+//   (y_hi + y_lo)[r] / ((y_hi + y_lo)[32] + eps), stage the tile in shared memory and store it
+//   with one TMA store (partial tiles inside a causal block are stored row by row).  The
+//   kernel is launched as a programmatic dependent of the reduction: everything but the merge
+//   warps starts while the reduction drains.
 //
 // Every mbarrier wait is bounded (sm100::mbar_wait): on a time-out the kernel records an
 // error code in the workspace's error word, stops its loops, waits (bounded) for its own TMA
@@ -54,6 +57,7 @@ struct TcPlan {
 enum : int {
   kErrReduceProducer = 0x110, kErrReduceMma = 0x120, kErrReduceRelu = 0x130, kErrReduceEpi = 0x140,
   kErrApplyProducer = 0x210, kErrApplyMma = 0x220, kErrApplyRelu = 0x230, kErrApplyEpi = 0x240,
+  kErrApplyMerge = 0x250,
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -92,7 +96,6 @@ constexpr uint32_t kRedSmemBytes = kRedStages * kRedStageBytes + 512 + 256 + 102
 
 __global__ void __launch_bounds__(kRedThreads, 1)
 litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ partials,
-                 uint8_t* __restrict__ images, float* __restrict__ states_f32, unsigned* __restrict__ counters,
                  int* __restrict__ err, TcPlan p) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
@@ -105,7 +108,10 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
   uint64_t* done = empty + kRedStages;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  int* last_flag = reinterpret_cast<int*>(tmem_holder + 2);
+
+  // the apply kernel (launched as a programmatic dependent) may start its prologue now; it
+  // waits for this grid to finish before it reads the partial states
+  pdl_launch_dependents();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int x = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -234,68 +240,60 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
     for (int j = 0; j < kRows; ++j) dst[j * kD + lane] = sv[j];   // S[r = j][c = lane]
   }
 
-  // teardown of the tensor memory
   tc_fence_before_sync();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after_sync();
     tmem_dealloc(tmem, kRedTmemCols);
   }
+}
 
-  // the last CTA of this (batch, group) to arrive merges; no CTA ever waits for another
-  __threadfence();
-  __syncthreads();
-  const unsigned cidx = kCounterBase + (unsigned)b * p.ngroups + g;
-  const unsigned nparts = (unsigned)(p.nblk * p.cpb);
-  if (threadIdx.x == 0) *last_flag = (atomicAdd(&counters[cidx], 1u) == nparts - 1u) ? 1 : 0;
-  __syncthreads();
-  if (!*last_flag) return;
-  __threadfence();
-  const float* gp = partials + ((int64_t)b * p.ngroups + g) * nparts * (kRedHeads * kStateFloats);
-  const int heads_here = min(kRedHeads, p.H - g * kRedHeads);
-  for (int e = threadIdx.x; e < kRedHeads * kStateFloats; e += kRedThreads) {
-    const int hl = e / kStateFloats, rc = e - hl * kStateFloats, r = rc >> 5, c = rc & 31;
+// address of partial `part` (block * cpb + chunk) of head h of batch b
+__device__ __forceinline__ const float* partial_ptr(const float* partials, const TcPlan& p, int b, int h,
+                                                    int part) {
+  const int g = h / kRedHeads, hl = h - g * kRedHeads;
+  return partials + ((((int64_t)b * p.ngroups + g) * ((int64_t)p.nblk * p.cpb) + part) * kRedHeads + hl) *
+                        kStateFloats;
+}
+
+// lite_la_state_fwd only: fp32 inclusive prefix states [B][H][nblk][33][32] from the partials.
+// grid (H, B), 256 threads.
+__global__ void __launch_bounds__(256)
+litela_state_merge(const float* __restrict__ partials, float* __restrict__ states, TcPlan p) {
+  const int h = blockIdx.x, b = blockIdx.y;
+  for (int e = threadIdx.x; e < kStateFloats; e += 256) {
     float run = 0.f;
-    for (int bb = 0; bb < p.nblk; ++bb) {
+    for (int blk = 0; blk < p.nblk; ++blk) {
       float s = 0.f;
-      for (int k = 0; k < p.cpb; ++k)
-        s += __ldcg(gp + ((int64_t)bb * p.cpb + k) * (kRedHeads * kStateFloats) + e);
+      for (int c = 0; c < p.cpb; ++c) s += partial_ptr(partials, p, b, h, blk * p.cpb + c)[e];
       run += s;
-      if (hl < heads_here && states_f32 != nullptr)
-        states_f32[(((int64_t)b * p.H + g * kRedHeads + hl) * p.nblk + bb) * kStateFloats + rc] = run;
-      if (hl < heads_here && images != nullptr) {
-        uint8_t* img = images + (((int64_t)b * p.H + g * kRedHeads + hl) * p.nblk + bb) * kImageBytes;
-        const __nv_bfloat16 hi = __float2bfloat16_rn(run);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(run - __bfloat162float(hi));
-        *reinterpret_cast<__nv_bfloat16*>(img + image_offset(r, c)) = hi;
-        *reinterpret_cast<__nv_bfloat16*>(img + image_offset(kImageLoRow + r, c)) = lo;
-      }
+      states[(((int64_t)b * p.H + h) * p.nblk + blk) * kStateFloats + e] = run;
     }
   }
-  // zero rows of the images: 33..39 and 73..79 (7 + 7 rows x 32 columns)
-  const int zeros_per_image = 14 * kD;
-  for (int e = threadIdx.x; images != nullptr && e < heads_here * p.nblk * zeros_per_image; e += kRedThreads) {
-    const int im = e / zeros_per_image, k = e - im * zeros_per_image;
-    const int hl = im / p.nblk, bb = im - hl * p.nblk;
-    const int zr = k >> 5, c = k & 31;
-    const int n = zr < 7 ? kRows + zr : kImageLoRow + kRows + (zr - 7);
-    uint8_t* img = images + (((int64_t)b * p.H + g * kRedHeads + hl) * p.nblk + bb) * kImageBytes;
-    *reinterpret_cast<__nv_bfloat16*>(img + image_offset(n, c)) = __float2bfloat16_rn(0.f);
-  }
-  if (threadIdx.x == 0) counters[cidx] = 0u;
 }
 
 // ---------------------------------------------------------------------------------------
 // apply
 
 constexpr int kApStages = 6;
-constexpr int kApThreads = 256;                        // w0 TMA, w1 MMA, w2..3 ReLU, w4..7 epilogue
+constexpr int kApThreads = 320;   // w0 TMA, w1 MMA, w2..3 ReLU, w4..7 epilogue, w8..9 state merge
 constexpr uint32_t kApStageBytes = kApTile * 64 * 2;   // 128 tokens x 64 channels x bf16
 constexpr int kApAccSlots = 3;
 constexpr uint32_t kApAccCols = kApHeads * kImageRows; // 160 fp32 columns per slot
 constexpr uint32_t kApTmemCols = 512;
 constexpr uint32_t kApSbufBytes = kApHeads * kImageBytes;
-constexpr uint32_t kApSmemBytes = kApStages * kApStageBytes + 2 * kApSbufBytes + 512 + 1024;
+constexpr uint32_t kOutBoxBytes = kApTile * 128;       // one 128B-swizzled box: 128 rows x 128 B
+constexpr int kApMergeThreads = 64;
+constexpr int kApMergePerThread = kApHeads * kStateFloats / kApMergeThreads;   // 33
+
+template <typename OutT>
+struct ApplyCfg {
+  static constexpr int kOutBoxes = (int)sizeof(OutT) / 2;          // boxes per item (64 channels)
+  static constexpr int kBoxChannels = 128 / (int)sizeof(OutT);     // channels per box
+  static constexpr uint32_t kOutSlotBytes = kOutBoxes * kOutBoxBytes;
+  static constexpr uint32_t kSmemBytes =
+      kApStages * kApStageBytes + 2 * kApSbufBytes + 2 * kOutSlotBytes + 512 + 1024;
+};
 
 struct ApItem {
   int b, pair, blk, tok0, tok1;
@@ -316,40 +314,38 @@ __device__ __forceinline__ ApItem ap_decode(long long it, const TcPlan& p) {
   return I;
 }
 
-template <typename OutT>
-__device__ __forceinline__ void store_row(OutT* dst, const float* o);
-
-template <>
-__device__ __forceinline__ void store_row<__nv_bfloat16>(__nv_bfloat16* dst, const float* o) {
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
+__device__ __forceinline__ void pack_out(__nv_bfloat16*, const float* o, uint4* w) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    uint32_t w[4];
+    uint32_t u[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       __nv_bfloat162 v2 = __floats2bfloat162_rn(o[i * 8 + 2 * j], o[i * 8 + 2 * j + 1]);
-      w[j] = *reinterpret_cast<uint32_t*>(&v2);
+      u[j] = *reinterpret_cast<uint32_t*>(&v2);
     }
-    d4[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    w[i] = make_uint4(u[0], u[1], u[2], u[3]);
   }
 }
 
-template <>
-__device__ __forceinline__ void store_row<float>(float* dst, const float* o) {
-  float4* d4 = reinterpret_cast<float4*>(dst);
+__device__ __forceinline__ void pack_out(float*, const float* o, uint4* w) {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) d4[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+  for (int i = 0; i < 8; ++i)
+    w[i] = make_uint4(__float_as_uint(o[4 * i]), __float_as_uint(o[4 * i + 1]), __float_as_uint(o[4 * i + 2]),
+                      __float_as_uint(o[4 * i + 3]));
 }
 
 template <typename OutT>
 __global__ void __launch_bounds__(kApThreads, 1)
-litela_apply_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t* __restrict__ images,
-                OutT* __restrict__ out, int* __restrict__ err, TcPlan p) {
+litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_out,
+                const float* __restrict__ partials, OutT* __restrict__ out, int* __restrict__ err, TcPlan p) {
   using namespace sm100;
+  using Cfg = ApplyCfg<OutT>;
+  constexpr int kChunksPerHead = kD * (int)sizeof(OutT) / 16;   // 16-byte chunks of one head's row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* qst = smem;                                            // kApStages q tiles
-  uint8_t* sbuf = smem + kApStages * kApStageBytes;               // 2 state buffers
+  uint8_t* qst = smem;                                              // kApStages q tiles
+  uint8_t* obuf = qst + kApStages * kApStageBytes;                  // 2 output staging slots
+  uint8_t* sbuf = obuf + 2 * Cfg::kOutSlotBytes;                    // 2 state buffers
   uint64_t* qfull = reinterpret_cast<uint64_t*>(sbuf + 2 * kApSbufBytes);
   uint64_t* qrelu = qfull + kApStages;
   uint64_t* qempty = qrelu + kApStages;
@@ -371,7 +367,7 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t* __restr
       mbar_init(&qempty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&sfull[s], 1);
+      mbar_init(&sfull[s], kApMergeThreads);
       mbar_init(&sempty[s], 1);
     }
     for (int s = 0; s < kApAccSlots; ++s) {
@@ -385,51 +381,37 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t* __restr
     tmem_alloc(tmem_holder, kApTmemCols);
     tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) prefetch_tensormap(&tmap);
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmap_q);
+    prefetch_tensormap(&tmap_out);
+  }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_holder;
 
   if (warp == 0) {
+    // ---- producer: q tiles
     if (lane == 0) {
-      long long prev = -1;
-      int seg_n = -1, seg_loaded = -1, issued = 0;
+      int issued = 0;
       for (long long it = w0; it < w1; ++it) {
         const int li = (int)(it - w0);
         const ApItem I = ap_decode(it, p);
-        if (I.seg != prev) {
-          prev = I.seg;
-          ++seg_n;
-          const int sb = seg_n & 1;
-          if (seg_n >= 2 &&
-              !mbar_wait(&sempty[sb], ((seg_n >> 1) - 1) & 1, abort_flag, err, kErrApplyProducer | 8 | sb))
-            break;
-          const int nh = min(kApHeads, p.H - I.pair * kApHeads);
-          mbar_arrive_expect_tx(&sfull[sb], nh * kImageBytes);
-          for (int j = 0; j < nh; ++j) {
-            const uint8_t* src =
-                images + (((int64_t)I.b * p.H + I.pair * kApHeads + j) * p.nblk + I.blk) * kImageBytes;
-            bulk_load(sbuf + sb * kApSbufBytes + j * kImageBytes, src, kImageBytes, &sfull[sb]);
-          }
-          seg_loaded = seg_n;
-        }
         const int s = li % kApStages;
         if (li >= kApStages &&
             !mbar_wait(&qempty[s], ((li / kApStages) - 1) & 1, abort_flag, err, kErrApplyProducer | s))
           break;
         mbar_arrive_expect_tx(&qfull[s], kApStageBytes);
-        tma_load_3d(qst + s * kApStageBytes, &tmap, &qfull[s], I.pair * kApHeads * kD, I.tok0, I.b);
+        tma_load_3d(qst + s * kApStageBytes, &tmap_q, &qfull[s], I.pair * kApHeads * kD, I.tok0, I.b);
         issued = li + 1;
       }
       if (*abort_flag) {   // let the copies still in flight land before the CTA exits (bounded)
         for (int i = (issued > kApStages ? issued - kApStages : 0); i < issued; ++i)
           mbar_drain(&qfull[i % kApStages], (i / kApStages) & 1);
-        for (int k = (seg_loaded > 0 ? seg_loaded - 1 : 0); k <= seg_loaded; ++k)
-          mbar_drain(&sfull[k & 1], (k >> 1) & 1);
       }
     }
   } else if (warp == 1) {
+    // ---- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, kImageRows, false, false);
       long long prev = -1;
@@ -469,6 +451,7 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t* __restr
       }
     }
   } else if (warp < 4) {
+    // ---- ReLU of the q tiles in place
     const int t = threadIdx.x - 64;   // 0..63
     for (long long it = w0; it < w1; ++it) {
       const int li = (int)(it - w0);
@@ -483,18 +466,28 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t* __restr
       fence_proxy_async_smem();
       mbar_arrive(&qrelu[s]);
     }
-  } else {
+  } else if (warp < 8) {
+    // ---- epilogue: TMEM -> normalise -> staged TMA store (or row stores for partial tiles)
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    const bool leader = (warp == 4 && lane == 0);
+    int nstaged = 0;   // staged items so far: item k uses slot k % 2 and bulk group k
     for (long long it = w0; it < w1; ++it) {
       const int li = (int)(it - w0);
       const int a = li % kApAccSlots;
       const ApItem I = ap_decode(it, p);
-      bool ok = mbar_wait(&tfull[a], (li / kApAccSlots) & 1, abort_flag, err, kErrApplyEpi | a);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      const bool ok = mbar_wait(&tfull[a], (li / kApAccSlots) & 1, abort_flag, err, kErrApplyEpi | a);
+      if (bar_any(1, 128, !ok)) break;
       tc_fence_after_sync();
       const int nh = min(kApHeads, p.H - I.pair * kApHeads);
       const int n = I.tok0 + row;
+      const bool staged = (I.tok1 - I.tok0 == kApTile) || (I.tok1 == p.N);
+      uint8_t* slot = obuf + (nstaged & 1) * Cfg::kOutSlotBytes;
+      if (staged) {
+        if (leader) bulk_wait_group_read<1>();   // the store that last used this slot has read it
+        bar_sync(2, 128);
+        ++nstaged;
+      }
       const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + a * kApAccCols;
       for (int j = 0; j < nh; ++j) {
         uint32_t v[kImageRows];
@@ -505,16 +498,102 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap, const uint8_t* __restr
           tc_fence_before_sync();
           mbar_arrive(&tempty[a]);
         }
-        if (n < I.tok1) {
-          const float den = (__uint_as_float(v[kD]) + __uint_as_float(v[kImageLoRow + kD])) + p.eps;
-          const float inv = 1.0f / den;
-          float o[kD];
+        const float den = (__uint_as_float(v[kD]) + __uint_as_float(v[kImageLoRow + kD])) + p.eps;
+        const float inv = 1.0f / den;
+        float o[kD];
 #pragma unroll
-          for (int r = 0; r < kD; ++r)
-            o[r] = (__uint_as_float(v[r]) + __uint_as_float(v[kImageLoRow + r])) * inv;
-          store_row<OutT>(out + (((int64_t)I.b * p.N + n) * p.H + I.pair * kApHeads + j) * kD, o);
+        for (int r = 0; r < kD; ++r) o[r] = (__uint_as_float(v[r]) + __uint_as_float(v[kImageLoRow + r])) * inv;
+        uint4 w[kChunksPerHead];
+        pack_out(static_cast<OutT*>(nullptr), o, w);
+        if (staged) {
+          // row `row` of the tile; 16-byte chunk k of the row lands in box k/8 at chunk
+          // (k%8) ^ (row%8): the 128B swizzle the TMA store expects
+#pragma unroll
+          for (int k = 0; k < kChunksPerHead; ++k) {
+            const int ck = j * kChunksPerHead + k;
+            uint8_t* box = slot + (ck >> 3) * kOutBoxBytes;
+            *reinterpret_cast<uint4*>(box + row * 128 + (((ck & 7) ^ (row & 7)) << 4)) = w[k];
+          }
+        } else if (n < I.tok1) {
+          uint4* dst = reinterpret_cast<uint4*>(out + (((int64_t)I.b * p.N + n) * p.H + I.pair * kApHeads + j) * kD);
+#pragma unroll
+          for (int k = 0; k < kChunksPerHead; ++k) dst[k] = w[k];
         }
       }
+      if (staged) {
+        fence_proxy_async_smem();
+        bar_sync(2, 128);
+        if (leader) {
+          const int x0 = I.pair * kApHeads * kD;
+#pragma unroll
+          for (int bx = 0; bx < Cfg::kOutBoxes; ++bx)
+            if (x0 + bx * Cfg::kBoxChannels < p.H * kD)
+              tma_store_3d(&tmap_out, slot + bx * kOutBoxBytes, x0 + bx * Cfg::kBoxChannels, I.tok0, I.b);
+          bulk_commit_group();
+        }
+      }
+    }
+    if (leader) bulk_wait_group<0>();
+  } else {
+    // ---- state merge: partial states -> running (prefix) sum -> bf16 hi/lo B operand
+    const int t = threadIdx.x - 256;   // 0..63
+    for (int e = t; e < 2 * kApHeads * 14 * kD; e += kApMergeThreads) {   // zero rows, both buffers
+      const int bufhead = e / (14 * kD), k = e - bufhead * (14 * kD);
+      const int zr = k >> 5, c = k & 31;
+      const int nrow = zr < 7 ? kRows + zr : kImageLoRow + kRows + (zr - 7);
+      *reinterpret_cast<__nv_bfloat16*>(sbuf + bufhead * kImageBytes + image_offset(nrow, c)) =
+          __float2bfloat16_rn(0.f);
+    }
+    pdl_wait_primary();   // the partial states are written by the preceding reduction grid
+    float run[kApMergePerThread];
+    int prev_b = -1, prev_pair = -1, prev_blk = -1, seg_n = -1;
+    long long prev = -1;
+    for (long long it = w0; it < w1; ++it) {
+      const ApItem I = ap_decode(it, p);
+      if (I.seg == prev) continue;
+      prev = I.seg;
+      ++seg_n;
+      const int sb = seg_n & 1;
+      const bool cont = (I.b == prev_b && I.pair == prev_pair && I.blk == prev_blk + 1);
+      if (!cont) {
+#pragma unroll
+        for (int i = 0; i < kApMergePerThread; ++i) run[i] = 0.f;
+      }
+      const int nh = min(kApHeads, p.H - I.pair * kApHeads);
+      for (int bb = cont ? I.blk : 0; bb <= I.blk; ++bb) {
+        for (int c = 0; c < p.cpb; ++c) {
+          float v[kApMergePerThread];
+#pragma unroll
+          for (int i = 0; i < kApMergePerThread; ++i) {
+            const int e = t + kApMergeThreads * i;
+            const int j = e >= kStateFloats ? 1 : 0;
+            v[i] = j < nh ? __ldcg(partial_ptr(partials, p, I.b, I.pair * kApHeads + j, bb * p.cpb + c) +
+                                   (e - j * kStateFloats))
+                          : 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < kApMergePerThread; ++i) run[i] += v[i];
+        }
+      }
+      prev_b = I.b;
+      prev_pair = I.pair;
+      prev_blk = I.blk;
+      if (seg_n >= 2 &&
+          !mbar_wait(&sempty[sb], ((seg_n >> 1) - 1) & 1, abort_flag, err, kErrApplyMerge | sb))
+        break;
+      uint8_t* buf = sbuf + sb * kApSbufBytes;
+#pragma unroll
+      for (int i = 0; i < kApMergePerThread; ++i) {
+        const int e = t + kApMergeThreads * i;
+        const int j = e >= kStateFloats ? 1 : 0;
+        const int rc = e - j * kStateFloats, r = rc >> 5, c = rc & 31;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(run[i]);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(run[i] - __bfloat162float(hi));
+        *reinterpret_cast<__nv_bfloat16*>(buf + j * kImageBytes + image_offset(r, c)) = hi;
+        *reinterpret_cast<__nv_bfloat16*>(buf + j * kImageBytes + image_offset(kImageLoRow + r, c)) = lo;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&sfull[sb]);
     }
   }
 

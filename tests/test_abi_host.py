@@ -106,8 +106,8 @@ def test_workspace_bytes(lib):
                          (1, 100, 3, 7)]:
         nblk = 1 if T <= 0 else -(-N // T)
         got = ll.lite_la_workspace_bytes(B, N, H, 32, T)
-        # at least one partial and one final state per (batch, head, block) plus a counter
-        assert got >= B * H * nblk * 2 * state + B * H * 4
+        # at least one partial state per (batch, head, block)
+        assert got >= B * H * nblk * state
         assert got % 4 == 0
     # a causal block at least as long as N is the non-causal problem
     assert ll.lite_la_workspace_bytes(2, 500, 3, 32, 500) == ll.lite_la_workspace_bytes(2, 500, 3, 32, 0)
