@@ -45,7 +45,9 @@ UNIT = "tokens·heads/s"
 FP32_LANES_PER_SM = 128          # B200: 4 SM sub-partitions x 32 fp32 lanes
 NUM_SMS = 148
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
-# name of each kernel the library launches per call, in launch order
+# the kernels the library launches per call, in launch order, and the two phases that
+# lite_la_fwd_events times (the state reduction with its scan, then the apply)
+LAUNCHES_PER_CALL = 3   # litela_reduce_tc, litela_state_scan, litela_apply_tc
 KERNELS = ("litela_reduce_tc", "litela_apply_tc")
 KERNEL_BOUND = {"litela_reduce_tc": "hbm", "litela_apply_tc": "hbm"}
 
@@ -349,7 +351,9 @@ def main():
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": traffic, "kernel": dom, "kernel_us": kern_us[dom],
                 "alg_bytes_per_launch": alg_bytes[dom], "alg_flops_per_launch": flops_per_kernel,
-                "peak_source": peak_note, "kernel_us_all": kern_us}
+                "peak_source": peak_note, "kernel_us_all": kern_us,
+                "timing": "phase events on the launching stream: litela_reduce_tc includes the small "
+                          "litela_state_scan that follows it"}
     # the call as a whole against the slower of the HBM and fp32-FMA bounds
     t_hbm = 8 * E / (peaks["hbm_gbs"] * 1e9) * 1e6
     t_fma = 4 * B * H * N * D * (D + 1) / (fp32_fma_peak_tflops(peaks.get("sm_max_mhz", 1965.0)) * 1e12) * 1e6
@@ -402,7 +406,7 @@ def main():
                 "math": "tensor-core bf16 x bf16 products with fp32 accumulation; fp32 state applied as bf16 hi + lo",
                 "data": "synthetic: i.i.d. N(0,1) bf16 qkv from seeded torch generators",
                 "config": config_of(args.workload), "roofline": roofline, "call_roofline": call_roof,
-                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": len(KERNELS) * calls * args.steps,
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": LAUNCHES_PER_CALL * calls * args.steps,
                 "clocks": clocks, "gpu": torch.cuda.get_device_name(dev)}
         if world > 1:
             line["config"]["parallelism"] = "dp%d (independent calls per rank, no collective)" % world

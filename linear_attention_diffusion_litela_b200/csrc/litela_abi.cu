@@ -210,8 +210,8 @@ litela_status validate(const void* qkv, const void* out, size_t out_elem, int B,
 }
 
 TcPlan tc_plan(const Plan& plan, float eps) {
-  return TcPlan{plan.B,       plan.N,      plan.H,     plan.T, plan.nblk, plan.ngroups, plan.chunks_per_block,
-                plan.chunk,   plan.npairs, plan.tiles_per_block, (long long)plan.items, eps};
+  return TcPlan{plan.B,     plan.N,      plan.H,     plan.T, plan.nblk, plan.ngroups, plan.chunks_per_block,
+                plan.chunk, plan.nquads, plan.tiles_per_block, (long long)plan.units, eps};
 }
 
 litela_status launch_reduce(const Plan& plan, const void* qkv, float* partials, int* err, cudaStream_t stream) {
@@ -225,37 +225,62 @@ litela_status launch_reduce(const Plan& plan, const void* qkv, float* partials, 
   return LITELA_OK;
 }
 
-// Launches the state reduction and the apply for `plan` with the given scratch.  The apply is
-// a programmatic dependent of the reduction (its prologue and q prefetch overlap the
-// reduction's end) unless phase events are requested, in which case the two run in plain
-// stream order with an event between them.
-template <typename OutT>
-litela_status launch(const Plan& plan, const void* qkv, OutT* out, float eps, float* partials, int* err,
-                     int num_sms, cudaStream_t stream, cudaEvent_t* events) {
-  CUtensorMap map_q, map_out;
-  litela_status s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kApTile, &map_q);
-  if (s != LITELA_OK) return s;
-  s = encode_out_map(out, plan.B, plan.N, plan.H, &map_out);
-  if (s != LITELA_OK) return s;
-  cudaError_t e;
-  if (events && (e = cudaEventRecord(events[0], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  s = launch_reduce(plan, qkv, partials, err, stream);
-  if (s != LITELA_OK) return s;
-  if (events && (e = cudaEventRecord(events[1], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  const TcPlan tp = tc_plan(plan, eps);
-  const long long grid = plan.items < num_sms ? plan.items : num_sms;
+// Launches kernel `k` with `args` as a programmatic dependent of the previous kernel in the
+// stream (its prologue overlaps the previous kernel's end) unless `pdl` is false.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool pdl,
+                      Args... args) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(kApThreads);
-  cfg.dynamicSmemBytes = ApplyCfg<OutT>::kSmemBytes;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = events ? 0 : 1;
-  e = cudaLaunchKernelEx(&cfg, litela_apply_tc<OutT>, map_q, map_out, static_cast<const float*>(partials), out, err,
-                         tp);
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k, static_cast<KArgs>(args)...);
+}
+
+litela_status launch_scan(const Plan& plan, const float* partials, uint8_t* images, float* states,
+                          cudaStream_t stream, bool pdl) {
+  cudaError_t e = launch_ex(litela_state_scan, dim3(kScanBlocks, plan.H, plan.B), dim3(kScanThreads), 0, stream, pdl,
+                            partials, images, states, tc_plan(plan, 0.f));
+  if (e != cudaSuccess) return cuda_fail(e, "launch litela_state_scan");
+  return LITELA_OK;
+}
+
+// Launches the state reduction, the scan and the apply for `plan` with the given scratch.  The
+// scan and the apply are programmatic dependents (their prologues overlap the preceding
+// kernel's end) unless phase events are requested, in which case the kernels run in plain
+// stream order with events between the reduction (with the scan) and the apply.
+template <typename OutT>
+litela_status launch(const Plan& plan, const void* qkv, OutT* out, float eps, float* partials, uint8_t* images,
+                     int* err, int num_sms, cudaStream_t stream, cudaEvent_t* events) {
+  CUtensorMap map_q, map_out;
+  litela_status s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kApTile, &map_q);
+  if (s != LITELA_OK) return s;
+  s = encode_out_map(out, plan.B, plan.N, plan.H, &map_out);
+  if (s != LITELA_OK) return s;
+  const bool pdl = events == nullptr;
+  cudaError_t e;
+  if (events && (e = cudaEventRecord(events[0], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  s = launch_reduce(plan, qkv, partials, err, stream);
+  if (s != LITELA_OK) return s;
+  s = launch_scan(plan, partials, images, nullptr, stream, pdl);
+  if (s != LITELA_OK) return s;
+  if (events && (e = cudaEventRecord(events[1], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  // CTAs: a multiple of the head quads when that keeps at least 7/8 of the SMs busy (all quads
+  // then advance through the same token rows together), else one per SM
+  long long grid = num_sms;
+  if (plan.nquads <= num_sms) {
+    const long long even = (long long)(num_sms / plan.nquads) * plan.nquads;
+    if (8 * even >= 7LL * num_sms) grid = even;
+  }
+  if (grid > plan.units) grid = plan.units;
+  e = launch_ex(litela_apply_tc<OutT>, dim3((unsigned)grid), dim3(kApThreads), ApplyCfg<OutT>::kSmemBytes, stream,
+                pdl, map_q, map_out, static_cast<const uint8_t*>(images), out, err, tc_plan(plan, eps));
   if (e != cudaSuccess) return cuda_fail(e, "launch litela_apply_tc");
   if (events && (e = cudaEventRecord(events[2], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   return LITELA_OK;
@@ -281,9 +306,8 @@ litela_status run_states(const void* qkv, float* states, int B, int N, int H, in
   float* partials = static_cast<float*>(ws->partials);
   s = launch_reduce(plan, qkv, partials, ws->err, stream);
   if (s != LITELA_OK) return s;
-  litela_state_merge<<<dim3(H, B), 256, 0, stream>>>(partials, states, tc_plan(plan, 0.f));
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "launch litela_state_merge");
+  s = launch_scan(plan, partials, nullptr, states, stream, true);
+  if (s != LITELA_OK) return s;
   g_last_error.clear();
   return LITELA_OK;
 }
@@ -302,7 +326,9 @@ litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float 
   Workspace* ws = nullptr;
   s = get_workspace(plan, stream, &ws);
   if (s != LITELA_OK) return s;
-  s = launch(plan, qkv, out, eps, static_cast<float*>(ws->partials), ws->err, num_sms, stream, events);
+  char* base = static_cast<char*>(ws->partials);
+  s = launch(plan, qkv, out, eps, reinterpret_cast<float*>(base), reinterpret_cast<uint8_t*>(base + plan.off_images),
+             ws->err, num_sms, stream, events);
   if (s == LITELA_OK) g_last_error.clear();
   return s;
 }
@@ -352,7 +378,8 @@ litela_status run_noalloc(const void* qkv, __nv_bfloat16* out, int B, int N, int
   s = noalloc_scratch(&scratch);
   if (s != LITELA_OK) return s;
   char* base = static_cast<char*>(scratch);
-  s = launch(plan, qkv, out, eps, reinterpret_cast<float*>(base + err_bytes), reinterpret_cast<int*>(base), num_sms,
+  s = launch(plan, qkv, out, eps, reinterpret_cast<float*>(base + err_bytes),
+             reinterpret_cast<uint8_t*>(base + err_bytes + plan.off_images), reinterpret_cast<int*>(base), num_sms,
              stream, nullptr);
   if (s == LITELA_OK) g_last_error.clear();
   return s;

@@ -17,7 +17,9 @@ constexpr int kStateFloats = kRows * kD;
 constexpr int kRedHeads = 4;
 constexpr int kRedTile = 64;
 constexpr int kRedCtasPerSm = 2;
-// apply: a work item is 2 heads x one 128-token tile inside one causal block
+// apply: a work unit is 4 heads (256-byte q and output rows) x one 128-token tile inside one
+// causal block; the MMA and the accumulators work on one head pair at a time
+constexpr int kApUnitHeads = 4;
 constexpr int kApHeads = 2;
 constexpr int kApTile = 128;
 // one head's state in the apply MMA's B-operand layout (in shared memory): 80 rows (33 hi rows
@@ -35,11 +37,13 @@ struct Plan {
   int ngroups = 0;           // reduce head groups, ceil(H / 4)
   int chunks_per_block = 0;  // reduce CTAs per (batch, group, block)
   int chunk = 0;             // tokens per reduce CTA (a multiple of kRedTile)
-  int npairs = 0;            // apply head pairs, ceil(H / 2)
-  int tiles_per_block = 0;   // apply tiles per (batch, pair, block)
-  int64_t items = 0;         // apply work items
-  // workspace: partial states fp32 [B][ngroups][nblk * chunks_per_block][4][33][32]
-  size_t bytes = 0;
+  int nquads = 0;            // apply head quads, ceil(H / 4)
+  int tiles_per_block = 0;   // apply tiles per (batch, quad, block)
+  int64_t units = 0;         // apply work units
+  // workspace, in bytes from its base (each region 256-byte aligned):
+  //   partial states fp32 [B][ngroups][nblk * chunks_per_block][4][33][32]
+  //   state images (the apply's B operand) bf16 [B][H][nblk][kImageBytes]
+  size_t off_images = 0, bytes = 0;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -64,11 +68,13 @@ inline bool make_plan(int B, int N, int H, int tokens_per_block, int num_sms, Pl
   chunk = (chunk + kRedTile - 1) / kRedTile * kRedTile;
   p->chunk = (int)chunk;
   p->chunks_per_block = (int)((p->T + chunk - 1) / chunk);
-  p->npairs = (H + kApHeads - 1) / kApHeads;
+  p->nquads = (H + kApUnitHeads - 1) / kApUnitHeads;
   p->tiles_per_block = (p->T + kApTile - 1) / kApTile;
-  p->items = (int64_t)B * p->npairs * p->nblk * p->tiles_per_block;
+  p->units = (int64_t)B * p->nquads * p->nblk * p->tiles_per_block;
   const size_t partials = (size_t)units * p->chunks_per_block * kRedHeads * kStateFloats * sizeof(float);
-  p->bytes = align_up(partials, 256);
+  const size_t images = (size_t)B * H * p->nblk * kImageBytes;
+  p->off_images = align_up(partials, 256);
+  p->bytes = p->off_images + align_up(images, 256);
   return true;
 }
 

@@ -20,18 +20,21 @@
 //   in fp32, so this is the fp32 state the method specifies.  The epilogue writes the chunk's
 //   partial states [4][33][32] to the workspace; nothing else (no atomics, no merge tail).
 //
-// litela_apply_tc  (persistent, one CTA per SM; work item = 2 heads x 128 tokens of a block)
-//   Two merge warps sum the partial states of the CTA's heads in fixed order (deterministic;
-//   for the block-causal form a running inclusive prefix over blocks) and write each head's
-//   state into shared memory as the MMA's B operand, split into bf16 hi + lo (S = hi + lo to
-//   2^-17 relative).  TMA streams q tiles (128 tokens x 64 channels, 128B swizzle) through a
-//   6-stage ring; two ReLU warps clamp them in place; one thread issues
-//   y = phi(Q) . [S_hi ; S_lo]^T per head (M = 128 tokens, N = 80, K = 32) into one of three
-//   TMEM accumulator slots; four epilogue warps read them back (thread = token), form
-//   (y_hi + y_lo)[r] / ((y_hi + y_lo)[32] + eps), stage the tile in shared memory and store it
-//   with one TMA store (partial tiles inside a causal block are stored row by row).  The
-//   kernel is launched as a programmatic dependent of the reduction: everything but the merge
-//   warps starts while the reduction drains.
+// litela_state_scan  sums the partial states in fixed order into per-block prefix states.
+//
+// litela_apply_tc  (persistent, one CTA per SM; work unit = 4 heads x 128 tokens of a block)
+//   Units span 4 heads so that every q row read and every output row written is a 256-byte
+//   run: on B200, 128-byte runs at these row strides reach only about half the HBM bandwidth.
+//   The producer bulk-copies each segment's state images (litela_state_scan's output: the
+//   MMA's B operand, S split into bf16 hi + lo) into shared memory and streams q tiles
+//   (128 tokens x 128 channels as two 128B-swizzled boxes) through a ring with TMA; two ReLU
+//   warps clamp them in place; one thread issues
+//   y = phi(Q) . [S_hi ; S_lo]^T per head (M = 128 tokens, N = 80, K = 32), one head pair at a
+//   time into one of three TMEM accumulator slots; four epilogue warps read them back
+//   (thread = token), form (y_hi + y_lo)[r] / ((y_hi + y_lo)[32] + eps), stage the unit's
+//   output tile in shared memory and store it with TMA (partial tiles inside a causal block
+//   are stored row by row).  The kernel is launched as a programmatic dependent of the scan:
+//   its set-up and first q loads overlap the end of the preceding grids.
 //
 // Every mbarrier wait is bounded (sm100::mbar_wait): on a time-out the kernel records an
 // error code in the workspace's error word, stops its loops, waits (bounded) for its own TMA
@@ -48,8 +51,8 @@
 namespace litela {
 
 struct TcPlan {
-  int B, N, H, T, nblk, ngroups, cpb, chunk, npairs, tpb;
-  long long items;
+  int B, N, H, T, nblk, ngroups, cpb, chunk, nquads, tpb;
+  long long units;
   float eps;
 };
 
@@ -256,62 +259,142 @@ __device__ __forceinline__ const float* partial_ptr(const float* partials, const
                         kStateFloats;
 }
 
-// lite_la_state_fwd only: fp32 inclusive prefix states [B][H][nblk][33][32] from the partials.
-// grid (H, B), 256 threads.
-__global__ void __launch_bounds__(256)
-litela_state_merge(const float* __restrict__ partials, float* __restrict__ states, TcPlan p) {
-  const int h = blockIdx.x, b = blockIdx.y;
-  for (int e = threadIdx.x; e < kStateFloats; e += 256) {
-    float run = 0.f;
-    for (int blk = 0; blk < p.nblk; ++blk) {
-      float s = 0.f;
-      for (int c = 0; c < p.cpb; ++c) s += partial_ptr(partials, p, b, h, blk * p.cpb + c)[e];
-      run += s;
-      states[(((int64_t)b * p.H + h) * p.nblk + blk) * kStateFloats + e] = run;
+// litela_state_scan: partial states -> per-(batch, head, block) inclusive prefix states, summed in
+// fixed order (deterministic).  Writes each one as the apply's B-operand image (bf16 hi rows
+// 0..32, lo rows 40..72, zero rows in between and after; S = hi + lo to 2^-17 relative) and,
+// when `states` is not null, as fp32 [B][H][nblk][33][32].  One thread per state element, all
+// of its partial loads in flight at once.  grid (kScanBlocks, H, B), kScanThreads threads;
+// launched as a programmatic dependent of the reduction.
+constexpr int kScanThreads = 128;
+constexpr int kScanZeros = 14 * kD;   // zero elements of one image
+constexpr int kScanBlocks = (kStateFloats + kScanZeros + kScanThreads - 1) / kScanThreads;
+
+__global__ void __launch_bounds__(kScanThreads)
+litela_state_scan(const float* __restrict__ partials, uint8_t* __restrict__ images, float* __restrict__ states,
+                  TcPlan p) {
+  using namespace sm100;
+  pdl_launch_dependents();
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int e = blockIdx.x * kScanThreads + threadIdx.x;
+  uint8_t* img0 = images + ((int64_t)b * p.H + h) * p.nblk * kImageBytes;
+  if (e >= kStateFloats) {
+    const int k = e - kStateFloats;
+    if (k >= kScanZeros || images == nullptr) return;
+    const int zr = k >> 5, c = k & 31;
+    const int nrow = zr < 7 ? kRows + zr : kImageLoRow + kRows + (zr - 7);
+    for (int blk = 0; blk < p.nblk; ++blk)
+      *reinterpret_cast<__nv_bfloat16*>(img0 + (int64_t)blk * kImageBytes + image_offset(nrow, c)) =
+          __float2bfloat16_rn(0.f);
+    return;
+  }
+  pdl_wait_primary();   // partials come from the reduction grid
+  const int r = e >> 5, c = e & 31;
+  const int g = h / kRedHeads, hl = h - g * kRedHeads;
+  const int64_t nparts = (int64_t)p.nblk * p.cpb;
+  const float* src = partials + ((((int64_t)b * p.ngroups + g) * nparts) * kRedHeads + hl) * kStateFloats + e;
+  const int64_t pstride = (int64_t)kRedHeads * kStateFloats;
+  float run = 0.f;
+  for (int blk = 0; blk < p.nblk; ++blk) {
+    float sum = 0.f;
+    int k = 0;
+    for (; k + 8 <= p.cpb; k += 8) {
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = __ldcg(src + ((int64_t)blk * p.cpb + k + i) * pstride);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sum += v[i];
     }
+    for (; k < p.cpb; ++k) sum += __ldcg(src + ((int64_t)blk * p.cpb + k) * pstride);
+    run += sum;
+    if (images != nullptr) {
+      uint8_t* img = img0 + (int64_t)blk * kImageBytes;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(run);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(run - __bfloat162float(hi));
+      *reinterpret_cast<__nv_bfloat16*>(img + image_offset(r, c)) = hi;
+      *reinterpret_cast<__nv_bfloat16*>(img + image_offset(kImageLoRow + r, c)) = lo;
+    }
+    if (states != nullptr) states[(((int64_t)b * p.H + h) * p.nblk + blk) * kStateFloats + e] = run;
   }
 }
 
 // ---------------------------------------------------------------------------------------
 // apply
 
-constexpr int kApStages = 6;
-constexpr int kApThreads = 320;   // w0 TMA, w1 MMA, w2..3 ReLU, w4..7 epilogue, w8..9 state merge
-constexpr uint32_t kApStageBytes = kApTile * 64 * 2;   // 128 tokens x 64 channels x bf16
+constexpr int kApThreads = 256;   // w0 TMA, w1 MMA, w2..3 ReLU, w4..7 epilogue
+constexpr uint32_t kQBoxBytes = kApTile * 128;         // 128 tokens x 64 channels x bf16 (one pair)
 constexpr int kApAccSlots = 3;
-constexpr uint32_t kApAccCols = kApHeads * kImageRows; // 160 fp32 columns per slot
+constexpr uint32_t kApAccCols = kApHeads * kImageRows; // 160 fp32 columns per slot (one pair)
 constexpr uint32_t kApTmemCols = 512;
-constexpr uint32_t kApSbufBytes = kApHeads * kImageBytes;
+constexpr uint32_t kApSbufBytes = kApUnitHeads * kImageBytes;
 constexpr uint32_t kOutBoxBytes = kApTile * 128;       // one 128B-swizzled box: 128 rows x 128 B
-constexpr int kApMergeThreads = 64;
-constexpr int kApMergePerThread = kApHeads * kStateFloats / kApMergeThreads;   // 33
+constexpr int kApReluThreads = 64;
 
 template <typename OutT>
 struct ApplyCfg {
-  static constexpr int kOutBoxes = (int)sizeof(OutT) / 2;          // boxes per item (64 channels)
-  static constexpr int kBoxChannels = 128 / (int)sizeof(OutT);     // channels per box
+  static constexpr int kQStages = sizeof(OutT) == 2 ? 3 : 2;
+  static constexpr int kOutSlots = sizeof(OutT) == 2 ? 2 : 1;
+  static constexpr int kBoxChannels = 128 / (int)sizeof(OutT);     // output channels per box
+  static constexpr int kOutBoxes = kApUnitHeads * kD / kBoxChannels;
+  static constexpr uint32_t kQStageBytes = 2 * kQBoxBytes;
   static constexpr uint32_t kOutSlotBytes = kOutBoxes * kOutBoxBytes;
   static constexpr uint32_t kSmemBytes =
-      kApStages * kApStageBytes + 2 * kApSbufBytes + 2 * kOutSlotBytes + 512 + 1024;
+      kQStages * kQStageBytes + kOutSlots * kOutSlotBytes + 2 * kApSbufBytes + 512 + 1024;
 };
 
-struct ApItem {
-  int b, pair, blk, tok0, tok1;
+struct ApUnit {
+  int b, quad, blk, tok0, tok1;
   long long seg;
 };
 
-__device__ __forceinline__ ApItem ap_decode(long long it, const TcPlan& p) {
-  ApItem I;
-  const int tile = (int)(it % p.tpb);
-  I.seg = it / p.tpb;
-  long long r = I.seg;
-  I.blk = (int)(r % p.nblk);
+// Work assignment.  When the CTAs can be split evenly over the head quads (gridDim.x a multiple
+// of nquads), CTA c owns quad c % nquads and a contiguous share (c / nquads) of that quad's
+// units in (batch, block, tile) order: all quads then advance through the same token rows at
+// the same time, so together the CTAs read and write whole q / output rows (DRAM locality),
+// and each CTA changes state only at batch / block boundaries.  Otherwise CTA c takes a
+// contiguous range of units in (batch, quad, block, tile) order.
+struct ApRange {
+  long long u0, u1;   // local unit range
+  int quad;           // fixed quad, or -1 for the general order
+};
+
+__device__ __forceinline__ ApRange ap_range(const TcPlan& p) {
+  ApRange R;
+  if (gridDim.x % p.nquads == 0) {
+    const int per = gridDim.x / p.nquads, r = blockIdx.x / p.nquads;
+    const long long L = (long long)p.B * p.nblk * p.tpb;
+    R.quad = blockIdx.x % p.nquads;
+    R.u0 = (long long)r * L / per;
+    R.u1 = (long long)(r + 1) * L / per;
+  } else {
+    R.quad = -1;
+    R.u0 = (long long)blockIdx.x * p.units / gridDim.x;
+    R.u1 = (long long)(blockIdx.x + 1) * p.units / gridDim.x;
+  }
+  return R;
+}
+
+__device__ __forceinline__ ApUnit ap_decode(long long u, const ApRange& R, const TcPlan& p) {
+  ApUnit U;
+  const int tile = (int)(u % p.tpb);
+  long long r = u / p.tpb;
+  U.blk = (int)(r % p.nblk);
   r /= p.nblk;
-  I.pair = (int)(r % p.npairs);
-  I.b = (int)(r / p.npairs);
-  I.tok0 = I.blk * p.T + tile * kApTile;
-  I.tok1 = min(I.tok0 + kApTile, min((I.blk + 1) * p.T, p.N));
-  return I;
+  if (R.quad >= 0) {
+    U.quad = R.quad;
+    U.b = (int)r;
+  } else {
+    U.quad = (int)(r % p.nquads);
+    U.b = (int)(r / p.nquads);
+  }
+  U.seg = ((long long)U.b * p.nquads + U.quad) * p.nblk + U.blk;
+  U.tok0 = U.blk * p.T + tile * kApTile;
+  U.tok1 = min(U.tok0 + kApTile, min((U.blk + 1) * p.T, p.N));
+  return U;
+}
+
+// heads of pair h (0 or 1) of a unit
+__device__ __forceinline__ int pair_heads(const TcPlan& p, int quad, int h) {
+  return max(0, min(kApHeads, p.H - quad * kApUnitHeads - h * kApHeads));
 }
 
 __device__ __forceinline__ void pack_out(__nv_bfloat16*, const float* o, uint4* w) {
@@ -337,19 +420,20 @@ __device__ __forceinline__ void pack_out(float*, const float* o, uint4* w) {
 template <typename OutT>
 __global__ void __launch_bounds__(kApThreads, 1)
 litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_out,
-                const float* __restrict__ partials, OutT* __restrict__ out, int* __restrict__ err, TcPlan p) {
+                const uint8_t* __restrict__ images, OutT* __restrict__ out, int* __restrict__ err, TcPlan p) {
   using namespace sm100;
   using Cfg = ApplyCfg<OutT>;
+  constexpr int kQStages = Cfg::kQStages;
   constexpr int kChunksPerHead = kD * (int)sizeof(OutT) / 16;   // 16-byte chunks of one head's row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* qst = smem;                                              // kApStages q tiles
-  uint8_t* obuf = qst + kApStages * kApStageBytes;                  // 2 output staging slots
-  uint8_t* sbuf = obuf + 2 * Cfg::kOutSlotBytes;                    // 2 state buffers
+  uint8_t* qst = smem;                                              // q tiles (2 boxes per stage)
+  uint8_t* obuf = qst + kQStages * Cfg::kQStageBytes;               // output staging slots
+  uint8_t* sbuf = obuf + Cfg::kOutSlots * Cfg::kOutSlotBytes;       // 2 state buffers (4 heads each)
   uint64_t* qfull = reinterpret_cast<uint64_t*>(sbuf + 2 * kApSbufBytes);
-  uint64_t* qrelu = qfull + kApStages;
-  uint64_t* qempty = qrelu + kApStages;
-  uint64_t* sfull = qempty + kApStages;
+  uint64_t* qrelu = qfull + kQStages;
+  uint64_t* qempty = qrelu + kQStages;
+  uint64_t* sfull = qempty + kQStages;
   uint64_t* sempty = sfull + 2;
   uint64_t* tfull = sempty + 2;
   uint64_t* tempty = tfull + kApAccSlots;
@@ -357,17 +441,17 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long w0 = (long long)blockIdx.x * p.items / gridDim.x;
-  const long long w1 = (long long)(blockIdx.x + 1) * p.items / gridDim.x;
+  const ApRange R = ap_range(p);
+  const long long u0 = R.u0, u1 = R.u1;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kApStages; ++s) {
+    for (int s = 0; s < kQStages; ++s) {
       mbar_init(&qfull[s], 1);
-      mbar_init(&qrelu[s], 64);
+      mbar_init(&qrelu[s], kApReluThreads);
       mbar_init(&qempty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&sfull[s], kApMergeThreads);
+      mbar_init(&sfull[s], 1);
       mbar_init(&sempty[s], 1);
     }
     for (int s = 0; s < kApAccSlots; ++s) {
@@ -391,210 +475,205 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
   const uint32_t tmem = *tmem_holder;
 
   if (warp == 0) {
-    // ---- producer: q tiles
+    // ---- producer: q tiles, 128 tokens x (2 pairs x 64 channels) per unit, and the state
+    // images of each segment (bulk copies of the scan kernel's output)
     if (lane == 0) {
-      int issued = 0;
-      for (long long it = w0; it < w1; ++it) {
-        const int li = (int)(it - w0);
-        const ApItem I = ap_decode(it, p);
-        const int s = li % kApStages;
-        if (li >= kApStages &&
-            !mbar_wait(&qempty[s], ((li / kApStages) - 1) & 1, abort_flag, err, kErrApplyProducer | s))
-          break;
-        mbar_arrive_expect_tx(&qfull[s], kApStageBytes);
-        tma_load_3d(qst + s * kApStageBytes, &tmap_q, &qfull[s], I.pair * kApHeads * kD, I.tok0, I.b);
-        issued = li + 1;
+      auto load_q = [&](long long u) {
+        const int lu = (int)(u - u0);
+        const ApUnit U = ap_decode(u, R, p);
+        const int s = lu % kQStages;
+        const int np = pair_heads(p, U.quad, 1) > 0 ? 2 : 1;
+        mbar_arrive_expect_tx(&qfull[s], np * kQBoxBytes);
+        for (int h = 0; h < np; ++h)
+          tma_load_3d(qst + s * Cfg::kQStageBytes + h * kQBoxBytes, &tmap_q, &qfull[s],
+                      U.quad * kApUnitHeads * kD + h * kApHeads * kD, U.tok0, U.b);
+      };
+      // q does not depend on the preceding grids: fill the ring before waiting for them
+      const long long pre = (u1 - u0) < kQStages ? (u1 - u0) : kQStages;
+      for (long long u = u0; u < u0 + pre; ++u) load_q(u);
+      int issued = (int)pre, seg_loaded = -1;
+      pdl_wait_primary();   // the state images are written by the preceding scan grid
+      long long prev = -1;
+      int seg_n = -1;
+      for (long long u = u0; u < u1; ++u) {
+        const int lu = (int)(u - u0);
+        const ApUnit U = ap_decode(u, R, p);
+        if (U.seg != prev) {
+          prev = U.seg;
+          ++seg_n;
+          const int sb = seg_n & 1;
+          if (seg_n >= 2 &&
+              !mbar_wait(&sempty[sb], ((seg_n >> 1) - 1) & 1, abort_flag, err, kErrApplyProducer | 8 | sb))
+            break;
+          const int nh = min(kApUnitHeads, p.H - U.quad * kApUnitHeads);
+          mbar_arrive_expect_tx(&sfull[sb], nh * kImageBytes);
+          for (int j = 0; j < nh; ++j) {
+            const uint8_t* src =
+                images + (((int64_t)U.b * p.H + U.quad * kApUnitHeads + j) * p.nblk + U.blk) * kImageBytes;
+            bulk_load(sbuf + sb * kApSbufBytes + j * kImageBytes, src, kImageBytes, &sfull[sb]);
+          }
+          seg_loaded = seg_n;
+        }
+        if (lu < pre) continue;
+        const int s = lu % kQStages;
+        if (!mbar_wait(&qempty[s], ((lu / kQStages) - 1) & 1, abort_flag, err, kErrApplyProducer | s)) break;
+        load_q(u);
+        issued = lu + 1;
       }
       if (*abort_flag) {   // let the copies still in flight land before the CTA exits (bounded)
-        for (int i = (issued > kApStages ? issued - kApStages : 0); i < issued; ++i)
-          mbar_drain(&qfull[i % kApStages], (i / kApStages) & 1);
+        for (int i = (issued > kQStages ? issued - kQStages : 0); i < issued; ++i)
+          mbar_drain(&qfull[i % kQStages], (i / kQStages) & 1);
+        for (int k = (seg_loaded > 0 ? seg_loaded - 1 : 0); k <= seg_loaded; ++k)
+          mbar_drain(&sfull[k & 1], (k >> 1) & 1);
       }
     }
   } else if (warp == 1) {
-    // ---- MMA issuer
+    // ---- MMA issuer: one head pair at a time into TMEM slot (pair counter) % 3
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, kImageRows, false, false);
       long long prev = -1;
-      int seg_n = -1, sb = 0;
-      for (long long it = w0; it < w1; ++it) {
-        const int li = (int)(it - w0);
-        const ApItem I = ap_decode(it, p);
-        if (I.seg != prev) {
-          prev = I.seg;
+      int seg_n = -1, sb = 0, pn = 0;
+      bool stop = false;
+      for (long long u = u0; u < u1 && !stop; ++u) {
+        const int lu = (int)(u - u0);
+        const ApUnit U = ap_decode(u, R, p);
+        if (U.seg != prev) {
+          prev = U.seg;
           ++seg_n;
           sb = seg_n & 1;
           if (!mbar_wait(&sfull[sb], (seg_n >> 1) & 1, abort_flag, err, kErrApplyMma | 8 | sb)) break;
         }
-        const int s = li % kApStages, a = li % kApAccSlots;
-        if (!mbar_wait(&qrelu[s], (li / kApStages) & 1, abort_flag, err, kErrApplyMma | s)) break;
-        if (li >= kApAccSlots &&
-            !mbar_wait(&tempty[a], ((li / kApAccSlots) - 1) & 1, abort_flag, err, kErrApplyMma | 12 | a))
-          break;
-        tc_fence_after_sync();
-        const int nh = min(kApHeads, p.H - I.pair * kApHeads);
-        const uint32_t qaddr = smem_u32(qst + s * kApStageBytes);
+        const int s = lu % kQStages;
+        if (!mbar_wait(&qrelu[s], (lu / kQStages) & 1, abort_flag, err, kErrApplyMma | s)) break;
+        const uint32_t qaddr = smem_u32(qst + s * Cfg::kQStageBytes);
         const uint32_t saddr = smem_u32(sbuf + sb * kApSbufBytes);
-        for (int j = 0; j < nh; ++j) {
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            // A: K-major 128B swizzle, 8-token groups 1024 B apart; head j's 32 channels at +64j B
-            const uint64_t ad = smem_desc(qaddr + j * 64 + ks * 32, 16, 1024, kSwizzle128B);
-            // B: K-major no swizzle, K-direction core matrices 128 B apart, row groups 512 B apart
-            const uint64_t bd = smem_desc(saddr + j * kImageBytes + ks * 256, 128, 512, kSwizzleNone);
-            umma_bf16(tmem + a * kApAccCols + j * kImageRows, ad, bd, idesc, ks);
+        for (int h = 0; h < 2; ++h) {
+          const int nh = pair_heads(p, U.quad, h);
+          if (nh == 0) break;
+          const int a = pn % kApAccSlots;
+          if (pn >= kApAccSlots &&
+              !mbar_wait(&tempty[a], ((pn / kApAccSlots) - 1) & 1, abort_flag, err, kErrApplyMma | 12 | a)) {
+            stop = true;
+            break;
           }
+          tc_fence_after_sync();
+          for (int j = 0; j < nh; ++j) {
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks) {
+              // A: K-major 128B swizzle, 8-token groups 1024 B apart; head j's 32 channels at +64j B
+              const uint64_t ad = smem_desc(qaddr + h * kQBoxBytes + j * 64 + ks * 32, 16, 1024, kSwizzle128B);
+              // B: K-major no swizzle, K-direction core matrices 128 B apart, row groups 512 B apart
+              const uint64_t bd =
+                  smem_desc(saddr + (h * kApHeads + j) * kImageBytes + ks * 256, 128, 512, kSwizzleNone);
+              umma_bf16(tmem + a * kApAccCols + j * kImageRows, ad, bd, idesc, ks);
+            }
+          }
+          umma_commit(&tfull[a]);
+          ++pn;
         }
+        if (stop) break;
         umma_commit(&qempty[s]);
-        umma_commit(&tfull[a]);
-        const bool seg_ends = (it + 1 >= w1) || (ap_decode(it + 1, p).seg != I.seg);
+        const bool seg_ends = (u + 1 >= u1) || (ap_decode(u + 1, R, p).seg != U.seg);
         if (seg_ends) umma_commit(&sempty[sb]);
       }
     }
   } else if (warp < 4) {
     // ---- ReLU of the q tiles in place
     const int t = threadIdx.x - 64;   // 0..63
-    for (long long it = w0; it < w1; ++it) {
-      const int li = (int)(it - w0);
-      const int s = li % kApStages;
-      if (!mbar_wait(&qfull[s], (li / kApStages) & 1, abort_flag, err, kErrApplyRelu | s)) break;
-      uint8_t* st = qst + s * kApStageBytes;
+    for (long long u = u0; u < u1; ++u) {
+      const int lu = (int)(u - u0);
+      const int s = lu % kQStages;
+      if (!mbar_wait(&qfull[s], (lu / kQStages) & 1, abort_flag, err, kErrApplyRelu | s)) break;
+      const ApUnit U = ap_decode(u, R, p);
+      const int nchunks = (pair_heads(p, U.quad, 1) > 0 ? 2 : 1) * (int)(kQBoxBytes / 16);
+      uint8_t* st = qst + s * Cfg::kQStageBytes;
 #pragma unroll 4
-      for (int j = t; j < (int)(kApStageBytes / 16); j += 64) {
+      for (int j = t; j < nchunks; j += kApReluThreads) {
         uint4* c = reinterpret_cast<uint4*>(st + j * 16);
         *c = relu_bf16x8(*c);
       }
       fence_proxy_async_smem();
       mbar_arrive(&qrelu[s]);
     }
-  } else if (warp < 8) {
+  } else {
     // ---- epilogue: TMEM -> normalise -> staged TMA store (or row stores for partial tiles)
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const bool leader = (warp == 4 && lane == 0);
-    int nstaged = 0;   // staged items so far: item k uses slot k % 2 and bulk group k
-    for (long long it = w0; it < w1; ++it) {
-      const int li = (int)(it - w0);
-      const int a = li % kApAccSlots;
-      const ApItem I = ap_decode(it, p);
-      const bool ok = mbar_wait(&tfull[a], (li / kApAccSlots) & 1, abort_flag, err, kErrApplyEpi | a);
-      if (bar_any(1, 128, !ok)) break;
-      tc_fence_after_sync();
-      const int nh = min(kApHeads, p.H - I.pair * kApHeads);
-      const int n = I.tok0 + row;
-      const bool staged = (I.tok1 - I.tok0 == kApTile) || (I.tok1 == p.N);
-      uint8_t* slot = obuf + (nstaged & 1) * Cfg::kOutSlotBytes;
+    int nstaged = 0, pn = 0;
+    bool stop = false;
+    for (long long u = u0; u < u1 && !stop; ++u) {
+      const ApUnit U = ap_decode(u, R, p);
+      const int n = U.tok0 + row;
+      const bool staged = (U.tok1 - U.tok0 == kApTile) || (U.tok1 == p.N);
+      uint8_t* slot = obuf + (nstaged % Cfg::kOutSlots) * Cfg::kOutSlotBytes;
       if (staged) {
-        if (leader) bulk_wait_group_read<1>();   // the store that last used this slot has read it
+        if (leader) bulk_wait_group_read<Cfg::kOutSlots - 1>();   // the store that last used this slot has read it
         bar_sync(2, 128);
         ++nstaged;
       }
-      const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + a * kApAccCols;
-      for (int j = 0; j < nh; ++j) {
-        uint32_t v[kImageRows];
-#pragma unroll
-        for (int k = 0; k < kImageRows / 16; ++k) tmem_ld_x16(ta + j * kImageRows + k * 16, v + k * 16);
-        tmem_wait_ld();
-        if (j == nh - 1) {
-          tc_fence_before_sync();
-          mbar_arrive(&tempty[a]);
+      for (int h = 0; h < 2; ++h) {
+        const int nh = pair_heads(p, U.quad, h);
+        if (nh == 0) break;
+        const int a = pn % kApAccSlots;
+        const bool ok = mbar_wait(&tfull[a], (pn / kApAccSlots) & 1, abort_flag, err, kErrApplyEpi | a);
+        if (bar_any(1, 128, !ok)) {
+          stop = true;
+          break;
         }
-        const float den = (__uint_as_float(v[kD]) + __uint_as_float(v[kImageLoRow + kD])) + p.eps;
-        const float inv = 1.0f / den;
-        float o[kD];
+        tc_fence_after_sync();
+        const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16) + a * kApAccCols;
+        for (int j = 0; j < nh; ++j) {
+          uint32_t v[kImageRows];
 #pragma unroll
-        for (int r = 0; r < kD; ++r) o[r] = (__uint_as_float(v[r]) + __uint_as_float(v[kImageLoRow + r])) * inv;
-        uint4 w[kChunksPerHead];
-        pack_out(static_cast<OutT*>(nullptr), o, w);
-        if (staged) {
-          // row `row` of the tile; 16-byte chunk k of the row lands in box k/8 at chunk
-          // (k%8) ^ (row%8): the 128B swizzle the TMA store expects
-#pragma unroll
-          for (int k = 0; k < kChunksPerHead; ++k) {
-            const int ck = j * kChunksPerHead + k;
-            uint8_t* box = slot + (ck >> 3) * kOutBoxBytes;
-            *reinterpret_cast<uint4*>(box + row * 128 + (((ck & 7) ^ (row & 7)) << 4)) = w[k];
+          for (int k = 0; k < kImageRows / 16; ++k) tmem_ld_x16(ta + j * kImageRows + k * 16, v + k * 16);
+          tmem_wait_ld();
+          if (j == nh - 1) {
+            tc_fence_before_sync();
+            mbar_arrive(&tempty[a]);
           }
-        } else if (n < I.tok1) {
-          uint4* dst = reinterpret_cast<uint4*>(out + (((int64_t)I.b * p.N + n) * p.H + I.pair * kApHeads + j) * kD);
+          const float den = (__uint_as_float(v[kD]) + __uint_as_float(v[kImageLoRow + kD])) + p.eps;
+          const float inv = 1.0f / den;
+          float o[kD];
 #pragma unroll
-          for (int k = 0; k < kChunksPerHead; ++k) dst[k] = w[k];
+          for (int r = 0; r < kD; ++r)
+            o[r] = (__uint_as_float(v[r]) + __uint_as_float(v[kImageLoRow + r])) * inv;
+          uint4 w[kChunksPerHead];
+          pack_out(static_cast<OutT*>(nullptr), o, w);
+          const int hu = h * kApHeads + j;   // head within the unit
+          if (staged) {
+            // 16-byte chunk ck of the unit's output row lands in box ck/8 at chunk
+            // (ck%8) ^ (row%8): the 128B swizzle the TMA store expects
+#pragma unroll
+            for (int k = 0; k < kChunksPerHead; ++k) {
+              const int ck = hu * kChunksPerHead + k;
+              uint8_t* box = slot + (ck >> 3) * kOutBoxBytes;
+              *reinterpret_cast<uint4*>(box + row * 128 + (((ck & 7) ^ (row & 7)) << 4)) = w[k];
+            }
+          } else if (n < U.tok1) {
+            uint4* dst = reinterpret_cast<uint4*>(
+                out + (((int64_t)U.b * p.N + n) * p.H + U.quad * kApUnitHeads + hu) * kD);
+#pragma unroll
+            for (int k = 0; k < kChunksPerHead; ++k) dst[k] = w[k];
+          }
         }
+        ++pn;
       }
+      if (stop) break;
       if (staged) {
         fence_proxy_async_smem();
         bar_sync(2, 128);
         if (leader) {
-          const int x0 = I.pair * kApHeads * kD;
+          const int x0 = U.quad * kApUnitHeads * kD;
 #pragma unroll
           for (int bx = 0; bx < Cfg::kOutBoxes; ++bx)
             if (x0 + bx * Cfg::kBoxChannels < p.H * kD)
-              tma_store_3d(&tmap_out, slot + bx * kOutBoxBytes, x0 + bx * Cfg::kBoxChannels, I.tok0, I.b);
+              tma_store_3d(&tmap_out, slot + bx * kOutBoxBytes, x0 + bx * Cfg::kBoxChannels, U.tok0, U.b);
           bulk_commit_group();
         }
       }
     }
     if (leader) bulk_wait_group<0>();
-  } else {
-    // ---- state merge: partial states -> running (prefix) sum -> bf16 hi/lo B operand
-    const int t = threadIdx.x - 256;   // 0..63
-    for (int e = t; e < 2 * kApHeads * 14 * kD; e += kApMergeThreads) {   // zero rows, both buffers
-      const int bufhead = e / (14 * kD), k = e - bufhead * (14 * kD);
-      const int zr = k >> 5, c = k & 31;
-      const int nrow = zr < 7 ? kRows + zr : kImageLoRow + kRows + (zr - 7);
-      *reinterpret_cast<__nv_bfloat16*>(sbuf + bufhead * kImageBytes + image_offset(nrow, c)) =
-          __float2bfloat16_rn(0.f);
-    }
-    pdl_wait_primary();   // the partial states are written by the preceding reduction grid
-    float run[kApMergePerThread];
-    int prev_b = -1, prev_pair = -1, prev_blk = -1, seg_n = -1;
-    long long prev = -1;
-    for (long long it = w0; it < w1; ++it) {
-      const ApItem I = ap_decode(it, p);
-      if (I.seg == prev) continue;
-      prev = I.seg;
-      ++seg_n;
-      const int sb = seg_n & 1;
-      const bool cont = (I.b == prev_b && I.pair == prev_pair && I.blk == prev_blk + 1);
-      if (!cont) {
-#pragma unroll
-        for (int i = 0; i < kApMergePerThread; ++i) run[i] = 0.f;
-      }
-      const int nh = min(kApHeads, p.H - I.pair * kApHeads);
-      for (int bb = cont ? I.blk : 0; bb <= I.blk; ++bb) {
-        for (int c = 0; c < p.cpb; ++c) {
-          float v[kApMergePerThread];
-#pragma unroll
-          for (int i = 0; i < kApMergePerThread; ++i) {
-            const int e = t + kApMergeThreads * i;
-            const int j = e >= kStateFloats ? 1 : 0;
-            v[i] = j < nh ? __ldcg(partial_ptr(partials, p, I.b, I.pair * kApHeads + j, bb * p.cpb + c) +
-                                   (e - j * kStateFloats))
-                          : 0.f;
-          }
-#pragma unroll
-          for (int i = 0; i < kApMergePerThread; ++i) run[i] += v[i];
-        }
-      }
-      prev_b = I.b;
-      prev_pair = I.pair;
-      prev_blk = I.blk;
-      if (seg_n >= 2 &&
-          !mbar_wait(&sempty[sb], ((seg_n >> 1) - 1) & 1, abort_flag, err, kErrApplyMerge | sb))
-        break;
-      uint8_t* buf = sbuf + sb * kApSbufBytes;
-#pragma unroll
-      for (int i = 0; i < kApMergePerThread; ++i) {
-        const int e = t + kApMergeThreads * i;
-        const int j = e >= kStateFloats ? 1 : 0;
-        const int rc = e - j * kStateFloats, r = rc >> 5, c = rc & 31;
-        const __nv_bfloat16 hi = __float2bfloat16_rn(run[i]);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(run[i] - __bfloat162float(hi));
-        *reinterpret_cast<__nv_bfloat16*>(buf + j * kImageBytes + image_offset(r, c)) = hi;
-        *reinterpret_cast<__nv_bfloat16*>(buf + j * kImageBytes + image_offset(kImageLoRow + r, c)) = lo;
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&sfull[sb]);
-    }
   }
 
   tc_fence_before_sync();
