@@ -231,11 +231,11 @@ def main():
     import numpy as np
     import torch
     import linear_attention_diffusion_litela_b200 as ll
+    from linear_attention_diffusion_litela_b200.dist import aggregate_rate, rank_seeds, world_info
+    from linear_attention_diffusion_litela_b200.dist import max_over_ranks as _max_over_ranks
     from linear_attention_diffusion_litela_b200.inputs import make_qkv, to_bits
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local_rank = world_info()
     if world != args.gpus:
         raise SystemExit("--gpus %d but WORLD_SIZE %d (launch N>1 with torch.distributed.run)" % (args.gpus, world))
     if not torch.cuda.is_available():
@@ -253,11 +253,7 @@ def main():
             dist.barrier()
 
     def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return _max_over_ranks(x, device=dev)
 
     lib = ll.lib()
     B, N, H, calls, seed0 = WORKLOADS_BENCH[args.workload]
@@ -267,8 +263,7 @@ def main():
     if free < need:
         raise SystemExit("not enough free GPU memory: need %.1f GB, free %.1f GB" % (need / 1e9, free / 1e9))
     seeds = [seed0 + i for i in range(calls)] if args.workload.startswith("sana4800m") else [seed0 * 10 + i for i in range(calls)]
-    if world > 1:
-        seeds = [s + 100000 * rank for s in seeds]
+    seeds = rank_seeds(seeds, rank)
     ins = [make_qkv(B, N, H, D, seed=s, device=dev) for s in seeds]
     outs = [torch.empty((B, N, H * D), dtype=torch.bfloat16, device=dev) for _ in range(calls)]
     stream = torch.cuda.current_stream(dev)
@@ -310,8 +305,7 @@ def main():
     ms_total = max_over_ranks(ms_total)
     ms_step = ms_total / args.steps
     us_call = 1e3 * ms_step / calls
-    tokens_heads = B * N * H * calls * args.steps * world
-    value = tokens_heads / (ms_total / 1e3)
+    value = aggregate_rate(B * N * H * calls * args.steps, world, ms_total)
 
     # per-kernel durations: the same calls through lite_la_fwd_events (3 events per call)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(calls)]
@@ -386,7 +380,7 @@ def main():
         torch.cuda.synchronize(dev)
         e2e_ms, _ = timed(e2e_step, args.e2e_steps)
         e2e_ms = max_over_ranks(e2e_ms)
-        e2e = {"value": B * N * H * calls * args.e2e_steps * world / (e2e_ms / 1e3), "unit": UNIT,
+        e2e = {"value": aggregate_rate(B * N * H * calls * args.e2e_steps, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": calls * qkv_bytes, "d2h_bytes_per_step": calls * out_bytes,
                "ms_per_step": e2e_ms / args.e2e_steps, "steps": args.e2e_steps,
                "how": "per call: pinned host qkv -> device copy, lite_la_fwd, device -> pinned host out copy, one stream"}

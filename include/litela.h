@@ -102,6 +102,12 @@ litela_status lite_la_fwd_events(const void* qkv, void* out, int B, int N, int H
  * a kernel of this stream's workspace or of lite_la_fwd_noalloc reported one, else LITELA_OK. */
 litela_status lite_la_device_status(cudaStream_t stream);
 
+/* Self-test of that error path: launches on `stream` one thread that waits on a barrier nothing
+ * ever completes; after the wait limit (about 1.5 s) it records its code and returns.  The next
+ * lite_la_device_status(stream) then returns LITELA_ERR_DEVICE_TIMEOUT, and the stream and the
+ * context remain usable.  Nothing faults and nothing hangs. */
+litela_status lite_la_selftest_timeout(cudaStream_t stream);
+
 /* Static description of a status code (never NULL). */
 const char* lite_la_status_string(litela_status status);
 

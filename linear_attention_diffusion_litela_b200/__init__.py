@@ -40,6 +40,7 @@ _SIGNATURES = {
     "lite_la_block_causal_fwd_f32out": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
     "lite_la_fwd_events": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp, _vp]),
     "lite_la_device_status": (_c_int, [_vp]),
+    "lite_la_selftest_timeout": (_c_int, [_vp]),
     "lite_la_state_fwd": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
     "lite_la_status_string": (ctypes.c_char_p, [_c_int]),
     "lite_la_last_error": (ctypes.c_char_p, []),

@@ -427,6 +427,18 @@ litela_status lite_la_fwd_noalloc(const void* qkv, void* out, int B, int N, int 
   return litela::run_noalloc(qkv, static_cast<__nv_bfloat16*>(out), B, N, H, d, eps, stream);
 }
 
+litela_status lite_la_selftest_timeout(cudaStream_t stream) {
+  litela::Plan plan;
+  litela::make_plan(1, 1, 1, 0, 148, &plan);
+  litela::Workspace* ws = nullptr;
+  litela_status s = litela::get_workspace(plan, stream, &ws);
+  if (s != LITELA_OK) return s;
+  litela::litela_selftest_timeout<<<1, 32, 0, stream>>>(ws->err);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return litela::cuda_fail(e, "launch litela_selftest_timeout");
+  return LITELA_OK;
+}
+
 litela_status lite_la_device_status(cudaStream_t stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

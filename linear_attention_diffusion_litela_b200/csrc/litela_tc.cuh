@@ -61,7 +61,23 @@ enum : int {
   kErrReduceProducer = 0x110, kErrReduceMma = 0x120, kErrReduceRelu = 0x130, kErrReduceEpi = 0x140,
   kErrApplyProducer = 0x210, kErrApplyMma = 0x220, kErrApplyRelu = 0x230, kErrApplyEpi = 0x240,
   kErrApplyMerge = 0x250,
+  kErrSelfTest = 0x3f0,
 };
+
+// Self-test of the bounded-wait error path: one thread waits on an mbarrier that nothing ever
+// arrives on; after the wait limit it records kErrSelfTest in *err and the kernel returns.
+__global__ void litela_selftest_timeout(int* err) {
+  using namespace sm100;
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, err, kErrSelfTest);
+}
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -293,27 +309,33 @@ litela_state_scan(const float* __restrict__ partials, uint8_t* __restrict__ imag
   const int64_t nparts = (int64_t)p.nblk * p.cpb;
   const float* src = partials + ((((int64_t)b * p.ngroups + g) * nparts) * kRedHeads + hl) * kStateFloats + e;
   const int64_t pstride = (int64_t)kRedHeads * kStateFloats;
-  float run = 0.f;
-  for (int blk = 0; blk < p.nblk; ++blk) {
-    float sum = 0.f;
-    int k = 0;
-    for (; k + 8 <= p.cpb; k += 8) {
-      float v[8];
+  // the partials of up to 8 consecutive parts (blocks x chunks, in order) are loaded together,
+  // then summed in order: one round trip to L2 per 8 parts
+  const int nparts_i = p.nblk * p.cpb;
+  float run = 0.f, sum = 0.f;
+  for (int k0 = 0; k0 < nparts_i; k0 += 8) {
+    float v[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = __ldcg(src + ((int64_t)blk * p.cpb + k + i) * pstride);
+    for (int i = 0; i < 8; ++i) v[i] = (k0 + i < nparts_i) ? __ldcg(src + (int64_t)(k0 + i) * pstride) : 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) sum += v[i];
+    for (int i = 0; i < 8; ++i) {
+      const int k = k0 + i;
+      if (k >= nparts_i) break;
+      sum += v[i];
+      if ((k + 1) % p.cpb == 0) {   // last chunk of block k / cpb: extend the prefix
+        const int blk = k / p.cpb;
+        run += sum;
+        sum = 0.f;
+        if (images != nullptr) {
+          uint8_t* img = img0 + (int64_t)blk * kImageBytes;
+          const __nv_bfloat16 hi = __float2bfloat16_rn(run);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(run - __bfloat162float(hi));
+          *reinterpret_cast<__nv_bfloat16*>(img + image_offset(r, c)) = hi;
+          *reinterpret_cast<__nv_bfloat16*>(img + image_offset(kImageLoRow + r, c)) = lo;
+        }
+        if (states != nullptr) states[(((int64_t)b * p.H + h) * p.nblk + blk) * kStateFloats + e] = run;
+      }
     }
-    for (; k < p.cpb; ++k) sum += __ldcg(src + ((int64_t)blk * p.cpb + k) * pstride);
-    run += sum;
-    if (images != nullptr) {
-      uint8_t* img = img0 + (int64_t)blk * kImageBytes;
-      const __nv_bfloat16 hi = __float2bfloat16_rn(run);
-      const __nv_bfloat16 lo = __float2bfloat16_rn(run - __bfloat162float(hi));
-      *reinterpret_cast<__nv_bfloat16*>(img + image_offset(r, c)) = hi;
-      *reinterpret_cast<__nv_bfloat16*>(img + image_offset(kImageLoRow + r, c)) = lo;
-    }
-    if (states != nullptr) states[(((int64_t)b * p.H + h) * p.nblk + blk) * kStateFloats + e] = run;
   }
 }
 
@@ -331,14 +353,17 @@ constexpr int kApReluThreads = 64;
 
 template <typename OutT>
 struct ApplyCfg {
-  static constexpr int kQStages = sizeof(OutT) == 2 ? 3 : 2;
+  // shared memory split (bf16 output: 4 q stages, 2 output slots, 1 state buffer = 213 KB;
+  // fp32 output: 2 q stages, 1 output slot, 2 state buffers)
+  static constexpr int kQStages = sizeof(OutT) == 2 ? 4 : 2;
   static constexpr int kOutSlots = sizeof(OutT) == 2 ? 2 : 1;
+  static constexpr int kSBufs = sizeof(OutT) == 2 ? 1 : 2;
   static constexpr int kBoxChannels = 128 / (int)sizeof(OutT);     // output channels per box
   static constexpr int kOutBoxes = kApUnitHeads * kD / kBoxChannels;
   static constexpr uint32_t kQStageBytes = 2 * kQBoxBytes;
   static constexpr uint32_t kOutSlotBytes = kOutBoxes * kOutBoxBytes;
   static constexpr uint32_t kSmemBytes =
-      kQStages * kQStageBytes + kOutSlots * kOutSlotBytes + 2 * kApSbufBytes + 512 + 1024;
+      kQStages * kQStageBytes + kOutSlots * kOutSlotBytes + kSBufs * kApSbufBytes + 512 + 1024;
 };
 
 struct ApUnit {
@@ -424,18 +449,19 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
   using namespace sm100;
   using Cfg = ApplyCfg<OutT>;
   constexpr int kQStages = Cfg::kQStages;
+  constexpr int kSBufs = Cfg::kSBufs;
   constexpr int kChunksPerHead = kD * (int)sizeof(OutT) / 16;   // 16-byte chunks of one head's row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* qst = smem;                                              // q tiles (2 boxes per stage)
   uint8_t* obuf = qst + kQStages * Cfg::kQStageBytes;               // output staging slots
-  uint8_t* sbuf = obuf + Cfg::kOutSlots * Cfg::kOutSlotBytes;       // 2 state buffers (4 heads each)
-  uint64_t* qfull = reinterpret_cast<uint64_t*>(sbuf + 2 * kApSbufBytes);
+  uint8_t* sbuf = obuf + Cfg::kOutSlots * Cfg::kOutSlotBytes;       // state buffers (4 heads each)
+  uint64_t* qfull = reinterpret_cast<uint64_t*>(sbuf + kSBufs * kApSbufBytes);
   uint64_t* qrelu = qfull + kQStages;
   uint64_t* qempty = qrelu + kQStages;
   uint64_t* sfull = qempty + kQStages;
-  uint64_t* sempty = sfull + 2;
-  uint64_t* tfull = sempty + 2;
+  uint64_t* sempty = sfull + kSBufs;
+  uint64_t* tfull = sempty + kSBufs;
   uint64_t* tempty = tfull + kApAccSlots;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + kApAccSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -450,7 +476,7 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       mbar_init(&qrelu[s], kApReluThreads);
       mbar_init(&qempty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kSBufs; ++s) {
       mbar_init(&sfull[s], 1);
       mbar_init(&sempty[s], 1);
     }
@@ -498,12 +524,18 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       for (long long u = u0; u < u1; ++u) {
         const int lu = (int)(u - u0);
         const ApUnit U = ap_decode(u, R, p);
+        if (lu >= pre) {   // q first: it does not wait for the state buffer to free up
+          const int s = lu % kQStages;
+          if (!mbar_wait(&qempty[s], ((lu / kQStages) - 1) & 1, abort_flag, err, kErrApplyProducer | s)) break;
+          load_q(u);
+          issued = lu + 1;
+        }
         if (U.seg != prev) {
           prev = U.seg;
           ++seg_n;
-          const int sb = seg_n & 1;
-          if (seg_n >= 2 &&
-              !mbar_wait(&sempty[sb], ((seg_n >> 1) - 1) & 1, abort_flag, err, kErrApplyProducer | 8 | sb))
+          const int sb = seg_n % kSBufs;
+          if (seg_n >= kSBufs && !mbar_wait(&sempty[sb], ((seg_n / kSBufs) - 1) & 1, abort_flag, err,
+                                            kErrApplyProducer | 8 | sb))
             break;
           const int nh = min(kApUnitHeads, p.H - U.quad * kApUnitHeads);
           mbar_arrive_expect_tx(&sfull[sb], nh * kImageBytes);
@@ -514,17 +546,12 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
           }
           seg_loaded = seg_n;
         }
-        if (lu < pre) continue;
-        const int s = lu % kQStages;
-        if (!mbar_wait(&qempty[s], ((lu / kQStages) - 1) & 1, abort_flag, err, kErrApplyProducer | s)) break;
-        load_q(u);
-        issued = lu + 1;
       }
       if (*abort_flag) {   // let the copies still in flight land before the CTA exits (bounded)
         for (int i = (issued > kQStages ? issued - kQStages : 0); i < issued; ++i)
           mbar_drain(&qfull[i % kQStages], (i / kQStages) & 1);
-        for (int k = (seg_loaded > 0 ? seg_loaded - 1 : 0); k <= seg_loaded; ++k)
-          mbar_drain(&sfull[k & 1], (k >> 1) & 1);
+        for (int k = (seg_loaded >= kSBufs ? seg_loaded - kSBufs + 1 : 0); k <= seg_loaded; ++k)
+          mbar_drain(&sfull[k % kSBufs], (k / kSBufs) & 1);
       }
     }
   } else if (warp == 1) {
@@ -540,8 +567,8 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         if (U.seg != prev) {
           prev = U.seg;
           ++seg_n;
-          sb = seg_n & 1;
-          if (!mbar_wait(&sfull[sb], (seg_n >> 1) & 1, abort_flag, err, kErrApplyMma | 8 | sb)) break;
+          sb = seg_n % kSBufs;
+          if (!mbar_wait(&sfull[sb], (seg_n / kSBufs) & 1, abort_flag, err, kErrApplyMma | 8 | sb)) break;
         }
         const int s = lu % kQStages;
         if (!mbar_wait(&qrelu[s], (lu / kQStages) & 1, abort_flag, err, kErrApplyMma | s)) break;

@@ -7,6 +7,8 @@ Small and medium shapes are compared on every output; the full-size workloads ar
 on sampled query rows (first, last, block edges and a seeded random set), which the oracle
 evaluates one by one.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -231,3 +233,21 @@ def test_state_fwd_matches_padded_state_definition(B, N, H, T):
     # fp32 sums of exact bf16 products: relative error ~ sqrt(N) * 2^-24 of the magnitudes
     scale = np.abs(ref).max(axis=(-1, -2), keepdims=True) + 1e-30
     assert np.all(np.abs(got - ref) <= 1e-5 * scale + 1e-6)
+
+
+def test_bounded_wait_timeout_is_reported_and_the_context_stays_usable():
+    """A kernel whose barrier never completes gives up after its wait limit, records an error
+    code that lite_la_device_status turns into LITELA_ERR_DEVICE_TIMEOUT, and the stream keeps
+    working (nothing faults, nothing hangs)."""
+    s = torch.cuda.Stream()
+    lib = ll.lib()
+    assert lib.lite_la_selftest_timeout(ctypes.c_void_p(s.cuda_stream)) == 0
+    with pytest.raises(ll.LiteLAError) as ei:
+        ll.lite_la_device_status(s)
+    assert ei.value.status == 5 and "0x3f0" in str(ei.value)
+    ll.lite_la_device_status(s)                       # the error word was cleared
+    qkv = make_qkv(1, 300, 3, 32, seed=9, device="cuda")
+    out = ll.lite_la_fwd(qkv, 3, eps=EPS, out_dtype=torch.float32, stream=s)
+    s.synchronize()
+    ll.lite_la_device_status(s)
+    assert_close(out.view(1, 300, 3, 32).double().cpu().numpy(), oracle_run(qkv, 3), "f32")
