@@ -214,16 +214,6 @@ TcPlan tc_plan(const Plan& plan, float eps) {
                 plan.chunk, plan.nquads, plan.tiles_per_block, (long long)plan.units, eps};
 }
 
-litela_status launch_reduce(const Plan& plan, const void* qkv, float* partials, int* err, cudaStream_t stream) {
-  CUtensorMap map;
-  litela_status s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kRedTile, &map);
-  if (s != LITELA_OK) return s;
-  dim3 grid(plan.nblk * plan.chunks_per_block, plan.ngroups, plan.B);
-  litela_reduce_tc<<<grid, kRedThreads, kRedSmemBytes, stream>>>(map, partials, err, tc_plan(plan, 0.f));
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "launch litela_reduce_tc");
-  return LITELA_OK;
-}
 
 // Launches kernel `k` with `args` as a programmatic dependent of the previous kernel in the
 // stream (its prologue overlaps the previous kernel's end) unless `pdl` is false.
@@ -243,9 +233,23 @@ cudaError_t launch_ex(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, c
   return cudaLaunchKernelEx(&cfg, k, static_cast<KArgs>(args)...);
 }
 
-litela_status launch_scan(const Plan& plan, const float* partials, uint8_t* images, float* states,
+litela_status launch_reduce(const Plan& plan, const void* qkv, float* partials, int* err, cudaStream_t stream,
+                            bool pdl) {
+  CUtensorMap map;
+  litela_status s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kRedTile, &map);
+  if (s != LITELA_OK) return s;
+  cudaError_t e = launch_ex(litela_reduce_tc, dim3(plan.nblk * plan.chunks_per_block, plan.ngroups, plan.B),
+                            dim3(kRedThreads), kRedSmemBytes, stream, pdl, map, partials, err, tc_plan(plan, 0.f));
+  if (e != cudaSuccess) return cuda_fail(e, "launch litela_reduce_tc");
+  return LITELA_OK;
+}
+
+litela_status launch_scan(const Plan& plan, const float* partials, uint8_t* images, float* states, int num_sms,
                           cudaStream_t stream, bool pdl) {
-  cudaError_t e = launch_ex(litela_state_scan, dim3(kScanBlocks, plan.H, plan.B), dim3(kScanThreads), 0, stream, pdl,
+  const int64_t work = ((int64_t)plan.B * plan.H * kStateFloats + kScanElems - 1) / kScanElems;
+  int64_t grid = (work + kScanThreads - 1) / kScanThreads;
+  if (grid > num_sms) grid = num_sms;
+  cudaError_t e = launch_ex(litela_state_scan, dim3((unsigned)grid), dim3(kScanThreads), 0, stream, pdl,
                             partials, images, states, tc_plan(plan, 0.f));
   if (e != cudaSuccess) return cuda_fail(e, "launch litela_state_scan");
   return LITELA_OK;
@@ -266,9 +270,9 @@ litela_status launch(const Plan& plan, const void* qkv, OutT* out, float eps, fl
   const bool pdl = events == nullptr;
   cudaError_t e;
   if (events && (e = cudaEventRecord(events[0], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  s = launch_reduce(plan, qkv, partials, err, stream);
+  s = launch_reduce(plan, qkv, partials, err, stream, pdl);
   if (s != LITELA_OK) return s;
-  s = launch_scan(plan, partials, images, nullptr, stream, pdl);
+  s = launch_scan(plan, partials, images, nullptr, num_sms, stream, pdl);
   if (s != LITELA_OK) return s;
   if (events && (e = cudaEventRecord(events[1], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   // CTAs: a multiple of the head quads when that keeps at least 7/8 of the SMs busy (all quads
@@ -304,9 +308,9 @@ litela_status run_states(const void* qkv, float* states, int B, int N, int H, in
   s = get_workspace(plan, stream, &ws);
   if (s != LITELA_OK) return s;
   float* partials = static_cast<float*>(ws->partials);
-  s = launch_reduce(plan, qkv, partials, ws->err, stream);
+  s = launch_reduce(plan, qkv, partials, ws->err, stream, true);
   if (s != LITELA_OK) return s;
-  s = launch_scan(plan, partials, nullptr, states, stream, true);
+  s = launch_scan(plan, partials, nullptr, states, num_sms, stream, true);
   if (s != LITELA_OK) return s;
   g_last_error.clear();
   return LITELA_OK;

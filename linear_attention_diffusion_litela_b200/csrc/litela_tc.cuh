@@ -22,6 +22,10 @@
 //
 // litela_state_scan  sums the partial states in fixed order into per-block prefix states.
 //
+// The kernels of a call, and consecutive calls, are chained with programmatic dependent launch:
+// each kernel starts its private set-up while its predecessor drains and waits for it
+// (griddepcontrol.wait) before touching global memory that the predecessor may still use.
+//
 // litela_apply_tc  (persistent, one CTA per SM; work unit = 4 heads x 128 tokens of a block)
 //   Units span 4 heads so that every q row read and every output row written is a 256-byte
 //   run: on B200, 128-byte runs at these row strides reach only about half the HBM bandwidth.
@@ -161,6 +165,9 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_holder;
+  // launched as a programmatic dependent of the previous kernel in the stream: everything
+  // above is private set-up; qkv and the workspace are touched only after that kernel is done
+  pdl_wait_primary();
 
   const int kx = p.H * kD + g * (kRedHeads * kD);       // first key channel of the group
   const int vx = 2 * p.H * kD + g * (kRedHeads * kD);   // first value channel of the group
@@ -278,62 +285,82 @@ __device__ __forceinline__ const float* partial_ptr(const float* partials, const
 // litela_state_scan: partial states -> per-(batch, head, block) inclusive prefix states, summed in
 // fixed order (deterministic).  Writes each one as the apply's B-operand image (bf16 hi rows
 // 0..32, lo rows 40..72, zero rows in between and after; S = hi + lo to 2^-17 relative) and,
-// when `states` is not null, as fp32 [B][H][nblk][33][32].  One thread per state element, all
-// of its partial loads in flight at once.  grid (kScanBlocks, H, B), kScanThreads threads;
-// launched as a programmatic dependent of the reduction.
-constexpr int kScanThreads = 128;
+// when `states` is not null, as fp32 [B][H][nblk][33][32].  Grid-stride over the state elements
+// with at most one small CTA per SM: its CTAs launch early as a programmatic dependent of the
+// reduction and must leave registers on each SM for the apply's CTAs to land while they wait.
+// Each thread keeps 2 elements x 8 partial loads in flight per round.
+constexpr int kScanThreads = 256;
 constexpr int kScanZeros = 14 * kD;   // zero elements of one image
-constexpr int kScanBlocks = (kStateFloats + kScanZeros + kScanThreads - 1) / kScanThreads;
+constexpr int kScanElems = 2;         // state elements per thread and round
 
 __global__ void __launch_bounds__(kScanThreads)
 litela_state_scan(const float* __restrict__ partials, uint8_t* __restrict__ images, float* __restrict__ states,
                   TcPlan p) {
   using namespace sm100;
   pdl_launch_dependents();
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int e = blockIdx.x * kScanThreads + threadIdx.x;
-  uint8_t* img0 = images + ((int64_t)b * p.H + h) * p.nblk * kImageBytes;
-  if (e >= kStateFloats) {
-    const int k = e - kStateFloats;
-    if (k >= kScanZeros || images == nullptr) return;
-    const int zr = k >> 5, c = k & 31;
-    const int nrow = zr < 7 ? kRows + zr : kImageLoRow + kRows + (zr - 7);
-    for (int blk = 0; blk < p.nblk; ++blk)
-      *reinterpret_cast<__nv_bfloat16*>(img0 + (int64_t)blk * kImageBytes + image_offset(nrow, c)) =
-          __float2bfloat16_rn(0.f);
-    return;
+  const int64_t stride = (int64_t)gridDim.x * kScanThreads;
+  const int64_t tid = (int64_t)blockIdx.x * kScanThreads + threadIdx.x;
+  // the partials come from the reduction grid; the images may be read by the previous call's
+  // apply until that grid (which waited for it) is done
+  pdl_wait_primary();
+  if (images != nullptr) {   // zero rows of every image
+    const int64_t nz = (int64_t)p.B * p.H * p.nblk * kScanZeros;
+    for (int64_t i = tid; i < nz; i += stride) {
+      const int64_t im = i / kScanZeros;
+      const int k = (int)(i - im * kScanZeros);
+      const int zr = k >> 5, c = k & 31;
+      const int nrow = zr < 7 ? kRows + zr : kImageLoRow + kRows + (zr - 7);
+      *reinterpret_cast<__nv_bfloat16*>(images + im * kImageBytes + image_offset(nrow, c)) = __float2bfloat16_rn(0.f);
+    }
   }
-  pdl_wait_primary();   // partials come from the reduction grid
-  const int r = e >> 5, c = e & 31;
-  const int g = h / kRedHeads, hl = h - g * kRedHeads;
-  const int64_t nparts = (int64_t)p.nblk * p.cpb;
-  const float* src = partials + ((((int64_t)b * p.ngroups + g) * nparts) * kRedHeads + hl) * kStateFloats + e;
+  const int nparts = p.nblk * p.cpb;
   const int64_t pstride = (int64_t)kRedHeads * kStateFloats;
-  // the partials of up to 8 consecutive parts (blocks x chunks, in order) are loaded together,
-  // then summed in order: one round trip to L2 per 8 parts
-  const int nparts_i = p.nblk * p.cpb;
-  float run = 0.f, sum = 0.f;
-  for (int k0 = 0; k0 < nparts_i; k0 += 8) {
-    float v[8];
+  const int64_t total = (int64_t)p.B * p.H * kStateFloats;
+  constexpr int kE = kScanElems;
+  for (int64_t base = tid; base < total; base += kE * stride) {
+    const float* src[kE]; int64_t bh[kE]; int e[kE]; bool ok[kE];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = (k0 + i < nparts_i) ? __ldcg(src + (int64_t)(k0 + i) * pstride) : 0.f;
+    for (int j = 0; j < kE; ++j) {
+      const int64_t i = base + j * stride;
+      ok[j] = i < total;
+      bh[j] = ok[j] ? i / kStateFloats : 0;
+      e[j] = ok[j] ? (int)(i - bh[j] * kStateFloats) : 0;
+      const int b = (int)(bh[j] / p.H), h = (int)(bh[j] - (int64_t)b * p.H);
+      const int g = h / kRedHeads, hl = h - g * kRedHeads;
+      src[j] = partials + ((((int64_t)b * p.ngroups + g) * nparts) * kRedHeads + hl) * kStateFloats + e[j];
+    }
+    float run[kE], sum[kE];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int k = k0 + i;
-      if (k >= nparts_i) break;
-      sum += v[i];
-      if ((k + 1) % p.cpb == 0) {   // last chunk of block k / cpb: extend the prefix
+    for (int j = 0; j < kE; ++j) run[j] = sum[j] = 0.f;
+    for (int k0 = 0; k0 < nparts; k0 += 8) {
+      float v[kE][8];
+#pragma unroll
+      for (int j = 0; j < kE; ++j)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[j][i] = (ok[j] && k0 + i < nparts) ? __ldcg(src[j] + (int64_t)(k0 + i) * pstride) : 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int k = k0 + i;
+        if (k >= nparts) break;
+        const bool block_end = (k + 1) % p.cpb == 0;   // last chunk of block k / cpb
         const int blk = k / p.cpb;
-        run += sum;
-        sum = 0.f;
-        if (images != nullptr) {
-          uint8_t* img = img0 + (int64_t)blk * kImageBytes;
-          const __nv_bfloat16 hi = __float2bfloat16_rn(run);
-          const __nv_bfloat16 lo = __float2bfloat16_rn(run - __bfloat162float(hi));
-          *reinterpret_cast<__nv_bfloat16*>(img + image_offset(r, c)) = hi;
-          *reinterpret_cast<__nv_bfloat16*>(img + image_offset(kImageLoRow + r, c)) = lo;
+#pragma unroll
+        for (int j = 0; j < kE; ++j) {
+          sum[j] += v[j][i];
+          if (block_end && ok[j]) {   // extend the prefix and store it
+            run[j] += sum[j];
+            sum[j] = 0.f;
+            const int r = e[j] >> 5, c = e[j] & 31;
+            if (images != nullptr) {
+              uint8_t* img = images + (bh[j] * p.nblk + blk) * kImageBytes;
+              const __nv_bfloat16 hi = __float2bfloat16_rn(run[j]);
+              const __nv_bfloat16 lo = __float2bfloat16_rn(run[j] - __bfloat162float(hi));
+              *reinterpret_cast<__nv_bfloat16*>(img + image_offset(r, c)) = hi;
+              *reinterpret_cast<__nv_bfloat16*>(img + image_offset(kImageLoRow + r, c)) = lo;
+            }
+            if (states != nullptr) states[(bh[j] * p.nblk + blk) * kStateFloats + e[j]] = run[j];
+          }
         }
-        if (states != nullptr) states[(((int64_t)b * p.H + h) * p.nblk + blk) * kStateFloats + e] = run;
       }
     }
   }
@@ -470,6 +497,7 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
   const ApRange R = ap_range(p);
   const long long u0 = R.u0, u1 = R.u1;
 
+  pdl_launch_dependents();   // the next kernel waits for this grid before touching memory
   if (threadIdx.x == 0) {
     for (int s = 0; s < kQStages; ++s) {
       mbar_init(&qfull[s], 1);
