@@ -358,23 +358,41 @@ def main():
         call_roof["t_fma_us_at_measured_clock"] = t_fma_clk
         call_roof["frac_at_measured_clock"] = max(t_hbm, t_fma_clk) / us_call
 
-    # end to end: pinned host input -> device, forward, device -> pinned host output, per call
+    # end to end: pinned host input -> device, forward, device -> pinned host output, per call.
+    # The copies run on their own streams so that the next call's upload and the previous
+    # call's download overlap this call's kernels (PCIe is full duplex); events order them.
     e2e = None
     if args.e2e_steps > 0:
-        nbuf = 2
+        nbuf = 3
         h_in = [torch.empty((B, N, 3 * H * D), dtype=torch.bfloat16, pin_memory=True) for _ in range(nbuf)]
         h_out = [torch.empty((B, N, H * D), dtype=torch.bfloat16, pin_memory=True) for _ in range(nbuf)]
         for j in range(nbuf):
             h_in[j].copy_(ins[j])
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_up = [torch.cuda.Event() for _ in range(nbuf)]
+        ev_fwd = [torch.cuda.Event() for _ in range(nbuf)]
+        ev_down = [torch.cuda.Event() for _ in range(nbuf)]
+        for j in range(nbuf):
+            ev_down[j].record(down)
 
         def e2e_step():
             for i in range(calls):
                 j = i % nbuf
-                ins[j].copy_(h_in[j], non_blocking=True)
+                with torch.cuda.stream(up):
+                    up.wait_event(ev_fwd[j])          # the forward that last read ins[j] is done
+                    ins[j].copy_(h_in[j], non_blocking=True)
+                    ev_up[j].record(up)
+                stream.wait_event(ev_up[j])
+                stream.wait_event(ev_down[j])         # outs[j] has been downloaded
                 s = fwd(in_p[j], out_p[j], B, N, H, D, EPS, sh)
                 if s != 0:
                     raise ll.LiteLAError(s, lib.lite_la_last_error().decode())
-                h_out[j].copy_(outs[j], non_blocking=True)
+                ev_fwd[j].record(stream)
+                with torch.cuda.stream(down):
+                    down.wait_event(ev_fwd[j])
+                    h_out[j].copy_(outs[j], non_blocking=True)
+                    ev_down[j].record(down)
+            stream.wait_stream(down)                  # the step ends when the last result is on the host
 
         e2e_step()
         torch.cuda.synchronize(dev)
@@ -383,7 +401,8 @@ def main():
         e2e = {"value": aggregate_rate(B * N * H * calls * args.e2e_steps, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": calls * qkv_bytes, "d2h_bytes_per_step": calls * out_bytes,
                "ms_per_step": e2e_ms / args.e2e_steps, "steps": args.e2e_steps,
-               "how": "per call: pinned host qkv -> device copy, lite_la_fwd, device -> pinned host out copy, one stream"}
+               "how": "per call: pinned host qkv -> device copy (upload stream), lite_la_fwd (compute stream), "
+                      "device -> pinned host out copy (download stream); 3 buffers in rotation, events order them"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
