@@ -251,3 +251,48 @@ def test_bounded_wait_timeout_is_reported_and_the_context_stays_usable():
     s.synchronize()
     ll.lite_la_device_status(s)
     assert_close(out.view(1, 300, 3, 32).double().cpu().numpy(), oracle_run(qkv, 3), "f32")
+
+
+@pytest.mark.parametrize("mode", ["bf16", "f32"])
+def test_more_head_quads_than_sms(mode):
+    """H = 600 gives 150 head quads (more than the 148 SMs): the apply takes the general,
+    non quad-major work order."""
+    B, N, H = 1, 96, 600
+    qkv = make_qkv(B, N, H, 32, seed=600, device="cuda")
+    assert_close(gpu_run(qkv, H, mode=mode), oracle_run(qkv, H), mode)
+
+
+def test_interleaved_shapes_reuse_and_grow_the_workspace():
+    """Calls of different sizes back to back on one stream (the workspace grows while earlier
+    kernels may still be queued), without synchronising in between."""
+    shapes = [(1, 200, 3), (2, 3000, 9), (1, 50, 2), (2, 4100, 17), (1, 700, 5)]
+    qkvs = [make_qkv(B, N, H, 32, seed=B + N + H, device="cuda") for B, N, H in shapes]
+    outs = [ll.lite_la_fwd(q, H, eps=EPS, out_dtype=torch.float32) for q, (B, N, H) in zip(qkvs, shapes)]
+    outs += [ll.lite_la_block_causal_fwd(q, H, 128, eps=EPS, out_dtype=torch.float32)
+             for q, (B, N, H) in zip(qkvs, shapes)]
+    torch.cuda.synchronize()
+    ll.lite_la_device_status()
+    for i, (q, (B, N, H)) in enumerate(zip(qkvs, shapes)):
+        rows = sample_rows(N, T=128, k=64, seed=i)
+        got = outs[i].view(B, N, H, 32).double().cpu().numpy()[:, rows]
+        assert_close(got, oracle_run(q, H, rows=rows), "f32")
+        got_c = outs[len(shapes) + i].view(B, N, H, 32).double().cpu().numpy()[:, rows]
+        assert_close(got_c, oracle_run(q, H, T=128, rows=rows), "f32")
+
+
+def test_eps_zero_and_a_head_with_only_negative_keys():
+    B, N, H = 2, 500, 6
+    qkv = make_qkv(B, N, H, 32, seed=31, device="cuda")
+    x = qkv.view(B, N, 3, H, 32)
+    x[1, :, 1, 4] = -x[1, :, 1, 4].abs() - 0.125          # batch 1, head 4: every key < 0
+    out = ll.lite_la_fwd(qkv, H, eps=0.0, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ll.lite_la_device_status()
+    got = out.view(B, N, H, 32).double().cpu().numpy()
+    bits = to_bits(qkv)
+    want = oracle.lite_la_fwd(bits, B, N, H, 32, 0.0)
+    dead = np.zeros(want.shape, dtype=bool)
+    dead[1, :, 4] = True                                   # 0 / 0 there: undefined, checked below
+    assert_close(got[~dead].reshape(-1), want[~dead].reshape(-1), "f32")
+    with_eps = gpu_run(qkv, H, mode="f32")                 # with eps the dead head is exactly 0
+    assert np.all(with_eps[1, :, 4] == 0.0)
