@@ -45,11 +45,15 @@ UNIT = "tokens·heads/s"
 FP32_LANES_PER_SM = 128          # B200: 4 SM sub-partitions x 32 fp32 lanes
 NUM_SMS = 148
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
-# the kernels the library launches per call, in launch order, and the two phases that
-# lite_la_fwd_events times (the state reduction with its scan, then the apply)
-LAUNCHES_PER_CALL = 3   # litela_reduce_tc, litela_state_scan, litela_apply_tc
-KERNELS = ("litela_reduce_tc", "litela_apply_tc")
-KERNEL_BOUND = {"litela_reduce_tc": "hbm", "litela_apply_tc": "hbm"}
+# The library runs a non-causal call as one fused kernel when B * ceil(H/4) fits the SMs
+# (lite_la_kernels_per_call == 1), else as three (reduction, scan, apply); lite_la_fwd_events
+# brackets the phases.  Per path: the timed phases and their algorithmic bytes (in units of
+# E = B*N*H*d elements).
+PATHS = {
+    1: {"phases": ("litela_fused_tc",), "alg_bytes_E": {"litela_fused_tc": 8}},
+    3: {"phases": ("litela_reduce_tc", "litela_apply_tc"),
+        "alg_bytes_E": {"litela_reduce_tc": 4, "litela_apply_tc": 4}},
+}
 
 
 def load_peaks():
@@ -314,7 +318,9 @@ def main():
             e.record(stream)
     torch.cuda.synchronize(dev)
     ev_handles = [(ctypes.c_void_p * 3)(*[ctypes.c_void_p(e.cuda_event) for e in trip]) for trip in evs]
-    kern_ms = {k: 0.0 for k in KERNELS}
+    nk = int(lib.lite_la_kernels_per_call(B, N, H, D, 0))
+    phases = PATHS[nk]["phases"]
+    kern_ms = {k: 0.0 for k in phases}
     nlaunch = 0
     for _ in range(args.steps):
         for i in range(calls):
@@ -323,31 +329,29 @@ def main():
                 raise ll.LiteLAError(s, lib.lite_la_last_error().decode())
         torch.cuda.synchronize(dev)
         for trip in evs:
-            kern_ms[KERNELS[0]] += trip[0].elapsed_time(trip[1])
-            kern_ms[KERNELS[1]] += trip[1].elapsed_time(trip[2])
+            if nk == 1:
+                kern_ms[phases[0]] += trip[0].elapsed_time(trip[2])
+            else:
+                kern_ms[phases[0]] += trip[0].elapsed_time(trip[1])
+                kern_ms[phases[1]] += trip[1].elapsed_time(trip[2])
         nlaunch += calls
     kern_us = {k: 1e3 * v / nlaunch for k, v in kern_ms.items()}
     E = B * N * H * D
-    flops_per_kernel = 2 * B * H * N * D * (D + 1)
-    alg_bytes = {KERNELS[0]: 4 * E, KERNELS[1]: 4 * E}
+    flops_per_call = 4 * B * H * N * D * (D + 1)
+    alg_bytes = {k: PATHS[nk]["alg_bytes_E"][k] * E for k in phases}
     peaks = load_peaks()
     dom = max(kern_us, key=kern_us.get)
-    bound = KERNEL_BOUND[dom]
     traffic = load_traffic(dom)
-    if bound == "hbm":
-        achieved = alg_bytes[dom] / (kern_us[dom] * 1e-6) / 1e9
-        peak, unit = peaks["hbm_gbs"], "GB/s"
-        peak_note = "%s copy bandwidth" % peaks["_source"]
-    else:
-        achieved = flops_per_kernel / (kern_us[dom] * 1e-6) / 1e12
-        peak, unit = fp32_fma_peak_tflops(peaks.get("sm_max_mhz", 1965.0)), "TFLOP/s"
-        peak_note = "fp32 FMA: 148 SMs x 128 lanes x 2 x %.0f MHz max clock" % peaks.get("sm_max_mhz", 1965.0)
-    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+    achieved = alg_bytes[dom] / (kern_us[dom] * 1e-6) / 1e9
+    peak, unit = peaks["hbm_gbs"], "GB/s"
+    peak_note = "%s copy bandwidth" % peaks["_source"]
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": traffic, "kernel": dom, "kernel_us": kern_us[dom],
-                "alg_bytes_per_launch": alg_bytes[dom], "alg_flops_per_launch": flops_per_kernel,
+                "alg_bytes_per_launch": alg_bytes[dom],
+                "alg_flops_per_launch": flops_per_call * alg_bytes[dom] // (8 * E),
                 "peak_source": peak_note, "kernel_us_all": kern_us,
-                "timing": "phase events on the launching stream: litela_reduce_tc includes the small "
-                          "litela_state_scan that follows it"}
+                "timing": "CUDA events on the launching stream around each phase (lite_la_fwd_events; "
+                          "no programmatic overlap with the neighbouring kernels)"}
     # the call as a whole against the slower of the HBM and fp32-FMA bounds
     t_hbm = 8 * E / (peaks["hbm_gbs"] * 1e9) * 1e6
     t_fma = 4 * B * H * N * D * (D + 1) / (fp32_fma_peak_tflops(peaks.get("sm_max_mhz", 1965.0)) * 1e12) * 1e6
@@ -419,7 +423,7 @@ def main():
                 "math": "tensor-core bf16 x bf16 products with fp32 accumulation; fp32 state applied as bf16 hi + lo",
                 "data": "synthetic: i.i.d. N(0,1) bf16 qkv from seeded torch generators",
                 "config": config_of(args.workload), "roofline": roofline, "call_roofline": call_roof,
-                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": LAUNCHES_PER_CALL * calls * args.steps,
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": nk * calls * args.steps,
                 "clocks": clocks, "gpu": torch.cuda.get_device_name(dev)}
         if world > 1:
             line["config"]["parallelism"] = "dp%d (independent calls per rank, no collective)" % world

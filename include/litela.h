@@ -88,10 +88,11 @@ litela_status lite_la_block_causal_fwd_f32out(const void* qkv, float* out, int B
 litela_status lite_la_state_fwd(const void* qkv, float* states, int B, int N, int H, int d,
                                 int tokens_per_block, cudaStream_t stream);
 
-/* lite_la_fwd with phase timing: identical launches, plus cudaEventRecord of events[0] before
- * the state-reduction kernel, events[1] between it and the apply kernel and events[2] after the
- * apply kernel, all on `stream`.  events: host array of 3 caller-created CUDA events.  Used by
- * the benchmark to time each kernel on its own stream. */
+/* lite_la_fwd with phase timing: the same kernels (without programmatic overlap between them),
+ * plus cudaEventRecord of events[0] before the first kernel, events[1] after the state phase
+ * (reduction + scan) and events[2] after the apply, all on `stream`; on the fused single-kernel
+ * path events[1] and events[2] are both recorded after the kernel.  events: host array of 3
+ * caller-created CUDA events.  Used by the benchmark to time the kernels on their stream. */
 litela_status lite_la_fwd_events(const void* qkv, void* out, int B, int N, int H, int d, float eps,
                                  cudaStream_t stream, cudaEvent_t* events);
 
@@ -121,6 +122,11 @@ litela_status lite_la_release_workspace(void);
 /* Size in bytes of the workspace a call with these arguments needs (tokens_per_block <= 0
  * means non-causal).  Returns 0 for invalid arguments or an empty problem. */
 size_t lite_la_workspace_bytes(int B, int N, int H, int d, int tokens_per_block);
+
+/* Number of kernels one call with these arguments launches on the current device: 1 when the
+ * non-causal call fits the fused single-kernel path (B * ceil(H/4) <= SM count), 3 otherwise
+ * (state reduction, prefix scan, apply); 0 for an empty or invalid problem. */
+int lite_la_kernels_per_call(int B, int N, int H, int d, int tokens_per_block);
 
 /* lite_la_fwd without any allocation.  The pages describe no such call; it exists for callers
  * that cannot let a library allocate device memory: a host that owns all of the device memory

@@ -47,6 +47,7 @@ _SIGNATURES = {
     "lite_la_release_workspace": (_c_int, []),
     "lite_la_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "lite_la_fwd_noalloc": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp]),
+    "lite_la_kernels_per_call": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int]),
 }
 EXPORTED_SYMBOLS = tuple(_SIGNATURES)
 

@@ -18,6 +18,7 @@
 
 #include "../../include/litela.h"
 #include "litela_plan.h"
+#include "litela_fused.cuh"
 #include "litela_tc.cuh"
 
 namespace litela {
@@ -69,7 +70,11 @@ litela_status device_setup(int* num_sms) {
         (e = cudaFuncSetAttribute(litela_apply_tc<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)ApplyCfg<__nv_bfloat16>::kSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_apply_tc<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)ApplyCfg<float>::kSmemBytes)) != cudaSuccess)
+                                  (int)ApplyCfg<float>::kSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_fused_tc<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)FusedCfg<__nv_bfloat16>::kSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_fused_tc<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)FusedCfg<float>::kSmemBytes)) != cudaSuccess)
       return cuda_fail(e, "cudaFuncSetAttribute(dynamic shared memory)");
     if (g_encode == nullptr) {
       void* fn = nullptr;
@@ -123,10 +128,14 @@ litela_status encode_out_map(OutT* out, int B, int N, int H, CUtensorMap* map) {
 // workspace: one per (device, stream)
 
 struct Workspace {
-  void* partials = nullptr;
+  void* partials = nullptr;   // partial states (and, for the three-kernel path, state images)
   size_t partials_bytes = 0;
-  int* err = nullptr;   // kErrWords words; word 0 is the kernels' error word
+  int* err = nullptr;         // control words: error word, then the fused kernel's counters
+  size_t ctl_words = 0;
 };
+
+// bytes of partial-state workspace a call with `plan` uses
+size_t work_bytes(const Plan& plan) { return plan.fused ? plan.fused_bytes : plan.bytes; }
 
 std::mutex g_ws_mutex;
 std::map<std::pair<int, uintptr_t>, Workspace> g_ws;
@@ -138,39 +147,49 @@ bool alloc_fault_injected() {
   return v != nullptr && v[0] == '1';
 }
 
-litela_status get_workspace(const Plan& plan, cudaStream_t stream, Workspace** out) {
+litela_status get_workspace(const Plan& plan, cudaStream_t stream, Workspace** out, bool states_only = false) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   std::lock_guard<std::mutex> lock(g_ws_mutex);
   Workspace& ws = g_ws[{dev, reinterpret_cast<uintptr_t>(stream)}];
-  const bool grow = ws.partials_bytes < plan.bytes || ws.err == nullptr;
-  if (grow) {
+  const size_t need = states_only ? plan.bytes : work_bytes(plan);
+  const size_t need_ctl = kCounterBase + plan.counters;
+  if (ws.partials_bytes < need || ws.ctl_words < need_ctl) {
     if (alloc_fault_injected())
       return fail(LITELA_ERR_OUT_OF_MEMORY, "workspace allocation failed (injected by LITELA_FAIL_ALLOC)");
-    // kernels of earlier calls on this stream may still use the old buffer
+    // kernels of earlier calls on this stream may still use the old buffers
     e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize before workspace growth");
-    if (ws.err == nullptr) {
-      e = cudaMalloc(&ws.err, kErrWords * sizeof(int));
+    if (ws.ctl_words < need_ctl) {
+      int keep = 0;   // a pending error code survives the growth
+      if (ws.err) {
+        cudaMemcpy(&keep, ws.err, sizeof(int), cudaMemcpyDeviceToHost);
+        cudaFree(ws.err);
+      }
+      ws.err = nullptr;
+      ws.ctl_words = 0;
+      e = cudaMalloc(&ws.err, need_ctl * sizeof(int));
       if (e != cudaSuccess) {
         cudaGetLastError();
         ws.err = nullptr;
-        return fail(LITELA_ERR_OUT_OF_MEMORY, std::string("error-word cudaMalloc: ") + cudaGetErrorString(e));
+        return fail(LITELA_ERR_OUT_OF_MEMORY, std::string("control-word cudaMalloc: ") + cudaGetErrorString(e));
       }
-      e = cudaMemset(ws.err, 0, kErrWords * sizeof(int));
-      if (e != cudaSuccess) return cuda_fail(e, "cudaMemset error word");
+      e = cudaMemset(ws.err, 0, need_ctl * sizeof(int));
+      if (e == cudaSuccess && keep != 0) e = cudaMemcpy(ws.err, &keep, sizeof(int), cudaMemcpyHostToDevice);
+      if (e != cudaSuccess) return cuda_fail(e, "initialising control words");
+      ws.ctl_words = need_ctl;
     }
-    if (ws.partials_bytes < plan.bytes) {
+    if (ws.partials_bytes < need) {
       if (ws.partials) cudaFree(ws.partials);
       ws.partials = nullptr;
       ws.partials_bytes = 0;
-      e = cudaMalloc(&ws.partials, plan.bytes);
+      e = cudaMalloc(&ws.partials, need);
       if (e != cudaSuccess) {
         cudaGetLastError();
         return fail(LITELA_ERR_OUT_OF_MEMORY, std::string("workspace cudaMalloc: ") + cudaGetErrorString(e));
       }
-      ws.partials_bytes = plan.bytes;
+      ws.partials_bytes = need;
     }
   }
   *out = &ws;
@@ -255,6 +274,32 @@ litela_status launch_scan(const Plan& plan, const float* partials, uint8_t* imag
   return LITELA_OK;
 }
 
+// Launches the fused single kernel (non-causal path) for `plan` with the given scratch; phase
+// events, if requested, bracket it (events[1] is recorded with events[2], after the kernel).
+template <typename OutT>
+litela_status launch_fused(const Plan& plan, const void* qkv, OutT* out, float eps, float* partials, int* ctl,
+                           cudaStream_t stream, cudaEvent_t* events) {
+  CUtensorMap map_kv, map_q, map_out;
+  litela_status s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kRedTile, &map_kv);
+  if (s != LITELA_OK) return s;
+  s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kApTile, &map_q);
+  if (s != LITELA_OK) return s;
+  s = encode_out_map(out, plan.B, plan.N, plan.H, &map_out);
+  if (s != LITELA_OK) return s;
+  cudaError_t e;
+  if (events && (e = cudaEventRecord(events[0], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  const FusedPlan fp{plan.B, plan.N, plan.H, plan.nquads, plan.fused_cpb, plan.fused_chunk, plan.fused_ntiles, eps};
+  const unsigned grid = (unsigned)(plan.B * plan.nquads * plan.fused_cpb);
+  e = launch_ex(litela_fused_tc<OutT>, dim3(grid), dim3(kFuThreads), FusedCfg<OutT>::kSmemBytes, stream,
+                events == nullptr, map_kv, map_q, map_out, partials, reinterpret_cast<unsigned*>(ctl + kCounterBase),
+                out, ctl, fp);
+  if (e != cudaSuccess) return cuda_fail(e, "launch litela_fused_tc");
+  if (events && ((e = cudaEventRecord(events[1], stream)) != cudaSuccess ||
+                 (e = cudaEventRecord(events[2], stream)) != cudaSuccess))
+    return cuda_fail(e, "cudaEventRecord");
+  return LITELA_OK;
+}
+
 // Launches the state reduction, the scan and the apply for `plan` with the given scratch.  The
 // scan and the apply are programmatic dependents (their prologues overlap the preceding
 // kernel's end) unless phase events are requested, in which case the kernels run in plain
@@ -305,7 +350,7 @@ litela_status run_states(const void* qkv, float* states, int B, int N, int H, in
   const size_t qkv_bytes = (size_t)B * N * 3 * H * d * sizeof(__nv_bfloat16);
   if (overlaps(qkv, qkv_bytes, states, state_bytes)) return fail(LITELA_ERR_INVALID_ARGUMENT, "states overlaps qkv");
   Workspace* ws = nullptr;
-  s = get_workspace(plan, stream, &ws);
+  s = get_workspace(plan, stream, &ws, true);
   if (s != LITELA_OK) return s;
   float* partials = static_cast<float*>(ws->partials);
   s = launch_reduce(plan, qkv, partials, ws->err, stream, true);
@@ -331,8 +376,11 @@ litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float 
   s = get_workspace(plan, stream, &ws);
   if (s != LITELA_OK) return s;
   char* base = static_cast<char*>(ws->partials);
-  s = launch(plan, qkv, out, eps, reinterpret_cast<float*>(base), reinterpret_cast<uint8_t*>(base + plan.off_images),
-             ws->err, num_sms, stream, events);
+  if (plan.fused)
+    s = launch_fused(plan, qkv, out, eps, reinterpret_cast<float*>(base), ws->err, stream, events);
+  else
+    s = launch(plan, qkv, out, eps, reinterpret_cast<float*>(base), reinterpret_cast<uint8_t*>(base + plan.off_images),
+               ws->err, num_sms, stream, events);
   if (s == LITELA_OK) g_last_error.clear();
   return s;
 }
@@ -372,8 +420,8 @@ litela_status run_noalloc(const void* qkv, __nv_bfloat16* out, int B, int N, int
   if (s != LITELA_OK) return s;
   Plan plan;
   make_plan(B, N, H, 0, num_sms, &plan);
-  const size_t err_bytes = align_up(kErrWords * sizeof(int), 256);
-  const size_t need = err_bytes + plan.bytes;
+  const size_t err_bytes = align_up((kCounterBase + plan.counters) * sizeof(int), 256);
+  const size_t need = err_bytes + work_bytes(plan);
   if (need > LITELA_NOALLOC_SCRATCH_BYTES)
     return fail(LITELA_ERR_INVALID_ARGUMENT,
                 "problem needs " + std::to_string(need) + " bytes of scratch; lite_la_fwd_noalloc has " +
@@ -382,6 +430,15 @@ litela_status run_noalloc(const void* qkv, __nv_bfloat16* out, int B, int N, int
   s = noalloc_scratch(&scratch);
   if (s != LITELA_OK) return s;
   char* base = static_cast<char*>(scratch);
+  if (plan.fused) {
+    // the sibling counters must start at zero (the kernel leaves them so; an aborted call might not)
+    cudaError_t e = cudaMemsetAsync(base + kCounterBase * sizeof(int), 0, plan.counters * sizeof(unsigned), stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(no-alloc counters)");
+    s = launch_fused(plan, qkv, out, eps, reinterpret_cast<float*>(base + err_bytes), reinterpret_cast<int*>(base),
+                     stream, nullptr);
+    if (s == LITELA_OK) g_last_error.clear();
+    return s;
+  }
   s = launch(plan, qkv, out, eps, reinterpret_cast<float*>(base + err_bytes),
              reinterpret_cast<uint8_t*>(base + err_bytes + plan.off_images), reinterpret_cast<int*>(base), num_sms,
              stream, nullptr);
@@ -431,6 +488,18 @@ litela_status lite_la_fwd_noalloc(const void* qkv, void* out, int B, int N, int 
   return litela::run_noalloc(qkv, static_cast<__nv_bfloat16*>(out), B, N, H, d, eps, stream);
 }
 
+int lite_la_kernels_per_call(int B, int N, int H, int d, int tokens_per_block) {
+  if (B <= 0 || N <= 0 || H <= 0 || d != litela::kD) return 0;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  litela::Plan p;
+  litela::make_plan(B, N, H, tokens_per_block, sms, &p);
+  return p.fused ? 1 : 3;
+}
+
 litela_status lite_la_selftest_timeout(cudaStream_t stream) {
   litela::Plan plan;
   litela::make_plan(1, 1, 1, 0, 148, &plan);
@@ -450,10 +519,15 @@ litela_status lite_la_device_status(cudaStream_t stream) {
   e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) return litela::cuda_fail(e, "cudaStreamSynchronize");
   int* words[2] = {nullptr, nullptr};
+  int* words_ws0 = nullptr;
+  size_t ctl_words_ws = 0;
   {
     std::lock_guard<std::mutex> lock(litela::g_ws_mutex);
     auto it = litela::g_ws.find({dev, reinterpret_cast<uintptr_t>(stream)});
-    if (it != litela::g_ws.end()) words[0] = it->second.err;
+    if (it != litela::g_ws.end()) {
+      words[0] = words_ws0 = it->second.err;
+      ctl_words_ws = it->second.ctl_words;
+    }
   }
   {
     std::lock_guard<std::mutex> lock(litela::g_noalloc_mutex);
@@ -469,6 +543,12 @@ litela_status lite_la_device_status(cudaStream_t stream) {
       if (code == 0) code = v;
       if ((e = cudaMemset(w, 0, sizeof(int))) != cudaSuccess)
         return litela::cuda_fail(e, "clearing the device error word");
+      // an aborted fused call may have left sibling counters set: clear them too
+      size_t words = 0;
+      if (w == words_ws0) words = ctl_words_ws;
+      if (words > (size_t)litela::kCounterBase &&
+          (e = cudaMemset(w + litela::kCounterBase, 0, (words - litela::kCounterBase) * sizeof(int))) != cudaSuccess)
+        return litela::cuda_fail(e, "clearing the counters");
     }
   }
   if (code != 0) {
@@ -513,7 +593,7 @@ size_t lite_la_workspace_bytes(int B, int N, int H, int d, int tokens_per_block)
   if (B < 0 || N < 0 || H < 0 || d != litela::kD) return 0;
   litela::Plan p;
   if (!litela::make_plan(B, N, H, tokens_per_block, 148, &p)) return 0;
-  return p.bytes + litela::kErrWords * sizeof(int);
+  return litela::work_bytes(p) + (litela::kCounterBase + p.counters) * sizeof(int);
 }
 
 }  // extern "C"

@@ -1,0 +1,473 @@
+// LiteLA forward (non-causal) as one persistent kernel: state reduction, merge and apply of
+// one head quad per CTA group, with no kernel boundary in between.
+//
+// Method: see litela_tc.cuh.  CTA (b, q, r), r < cpb, of grid B x nquads x cpb:
+//   phase 1  reduces chunk r of batch b's tokens for quad q's 4 heads exactly as
+//            litela_reduce_tc does (TMA k|v boxes, ReLU in shared memory, two tcgen05 MMAs per
+//            16 tokens into TMEM) and writes the partial state [4][33][32] to the workspace;
+//   merge    waits until the cpb sibling CTAs of (b, q) have written their partials (an
+//            arrival counter; every wait is bounded), bulk-copies the cpb partials into shared
+//            memory, sums them in fixed order r = 0..cpb-1 (deterministic) and writes the
+//            quad's state as the MMA's B operand (bf16 hi + lo, as litela_state_scan does);
+//   phase 2  applies the state to tiles [r*ntiles/cpb, (r+1)*ntiles/cpb) of batch b's tokens
+//            exactly as litela_apply_tc does (its q prefetch overlaps the merge).
+// The only cross-CTA dependency is among the cpb siblings, which finish phase 1 at about the
+// same time.  The grid has at most one CTA per SM (its shared memory admits no second one) and
+// at most as many CTAs as SMs, so siblings are co-resident unless other kernels hold SMs, in
+// which case the waits end in a recorded time-out instead of a hang.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "litela_plan.h"
+#include "litela_tc.cuh"
+#include "sm100_ptx.cuh"
+
+namespace litela {
+
+struct FusedPlan {
+  int B, N, H, nquads, cpb, chunk, ntiles;
+  float eps;
+};
+
+enum : int { kErrFusedSibling = 0x410, kErrFusedMerge = 0x420, kErrFusedP1 = 0x430 };
+
+constexpr int kFuThreads = 256;     // w0 TMA, w1 MMA, w2..5 phase-1 ReLU/epilogue; phase 2: w2..3 ReLU,
+                                    // w4..7 merge then epilogue
+constexpr int kFuStages1 = 6;       // phase-1 ring of k|v stages (32 KB each)
+constexpr uint32_t kFuTmemCols = 512;
+
+template <typename OutT>
+struct FusedCfg {
+  using A = ApplyCfg<OutT>;
+  static constexpr uint32_t kPhase1Bytes = kFuStages1 * kRedStageBytes + 512;   // + the ones tile
+  static constexpr uint32_t kPhase2Bytes = A::kQStages * A::kQStageBytes + A::kOutSlots * A::kOutSlotBytes + kApSbufBytes;
+  static constexpr uint32_t kBodyBytes = kPhase1Bytes > kPhase2Bytes ? kPhase1Bytes : kPhase2Bytes;
+  static constexpr uint32_t kSmemBytes = kBodyBytes + 512 + 1024;
+  // merge batches are bulk-copied into the (still idle) output staging region
+  static constexpr int kMergeBatch = (int)(A::kOutSlots * A::kOutSlotBytes / (kRedHeads * kStateFloats * 4));
+};
+
+template <typename OutT>
+__global__ void __launch_bounds__(kFuThreads, 1)
+litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant__ CUtensorMap tmap_q,
+                const __grid_constant__ CUtensorMap tmap_out, float* __restrict__ partials,
+                unsigned* __restrict__ counters, OutT* __restrict__ out, int* __restrict__ err, FusedPlan p) {
+  using namespace sm100;
+  using Cfg = FusedCfg<OutT>;
+  using A = typename Cfg::A;
+  constexpr int kQStages = A::kQStages;
+  constexpr int kChunksPerHead = kD * (int)sizeof(OutT) / 16;
+  constexpr uint32_t kPartBytes = kRedHeads * kStateFloats * 4;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  // phase 1 layout
+  uint8_t* stages = smem;
+  uint8_t* ones = smem + kFuStages1 * kRedStageBytes;
+  // phase 2 layout (reuses the same bytes once phase 1 is over)
+  uint8_t* qst = smem;
+  uint8_t* obuf = qst + kQStages * A::kQStageBytes;
+  uint8_t* sbuf = obuf + A::kOutSlots * A::kOutSlotBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBodyBytes);
+  uint64_t* full = bars;                        // phase 1
+  uint64_t* relu_done = full + kFuStages1;
+  uint64_t* empty = relu_done + kFuStages1;
+  uint64_t* done = empty + kFuStages1;
+  uint64_t* qfull = done + 1;                   // phase 2
+  uint64_t* qrelu = qfull + kQStages;
+  uint64_t* qempty = qrelu + kQStages;
+  uint64_t* sfull = qempty + kQStages;
+  uint64_t* tfull = sfull + 1;
+  uint64_t* tempty = tfull + kApAccSlots;
+  uint64_t* merge_bar = tempty + kApAccSlots;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(merge_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q = blockIdx.x % p.nquads;
+  const int br = blockIdx.x / p.nquads;
+  const int r = br % p.cpb, b = br / p.cpb;
+  const int cidx = b * p.nquads + q;
+  // phase 1: chunk r of batch b's tokens
+  const int n0 = r * p.chunk, n1 = min(n0 + p.chunk, p.N);
+  const int ntiles1 = n1 > n0 ? (n1 - n0 + kRedTile - 1) / kRedTile : 0;
+  // phase 2: tiles [t0, t1) of batch b
+  const int t0 = (int)((long long)r * p.ntiles / p.cpb), t1 = (int)((long long)(r + 1) * p.ntiles / p.cpb);
+  const int nunits = t1 - t0;
+
+  pdl_launch_dependents();   // the next kernel waits for this grid before touching memory
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kFuStages1; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&relu_done[s], 128);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(&qfull[s], 1);
+      mbar_init(&qrelu[s], kApReluThreads);
+      mbar_init(&qempty[s], 1);
+    }
+    mbar_init(sfull, 1);
+    for (int s = 0; s < kApAccSlots; ++s) {
+      mbar_init(&tfull[s], 1);
+      mbar_init(&tempty[s], 128);
+    }
+    mbar_init(merge_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < 128; i += kFuThreads) reinterpret_cast<uint32_t*>(ones)[i] = 0x3F803F80u;
+  fence_proxy_async_smem();
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, kFuTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmap_kv);
+    prefetch_tensormap(&tmap_q);
+    prefetch_tensormap(&tmap_out);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_holder;
+  // private set-up above; global memory only after the previous kernel in the stream is done
+  pdl_wait_primary();
+
+  // =============================== phase 1: state reduction ===============================
+  const int kx = p.H * kD + q * (kRedHeads * kD), vx = 2 * p.H * kD + q * (kRedHeads * kD);
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < ntiles1; ++i) {
+        const int s = i % kFuStages1;
+        if (i >= kFuStages1 &&
+            !mbar_wait(&empty[s], ((i / kFuStages1) - 1) & 1, abort_flag, err, kErrFusedP1 | s))
+          break;
+        uint8_t* st = stages + s * kRedStageBytes;
+        const int y = n0 + i * kRedTile;
+        mbar_arrive_expect_tx(&full[s], kRedStageBytes);
+        tma_load_3d(st, &tmap_kv, &full[s], kx, y, b);
+        tma_load_3d(st + kRedBoxBytes, &tmap_kv, &full[s], kx + 64, y, b);
+        tma_load_3d(st + 2 * kRedBoxBytes, &tmap_kv, &full[s], vx, y, b);
+        tma_load_3d(st + 3 * kRedBoxBytes, &tmap_kv, &full[s], vx + 64, y, b);
+        issued = i + 1;
+      }
+      if (*abort_flag) {
+        for (int i = (issued > kFuStages1 ? issued - kFuStages1 : 0); i < issued; ++i)
+          mbar_drain(&full[i % kFuStages1], (i / kFuStages1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && ntiles1 > 0) {
+      constexpr uint32_t idesc_num = idesc_bf16_f32(128, 128, true, true);
+      constexpr uint32_t idesc_den = idesc_bf16_f32(128, 16, true, false);
+      const uint64_t ones_desc = smem_desc(smem_u32(ones), 128, 256, kSwizzleNone);
+      for (int i = 0; i < ntiles1; ++i) {
+        const int s = i % kFuStages1;
+        if (!mbar_wait(&relu_done[s], (i / kFuStages1) & 1, abort_flag, err, kErrFusedP1 | 8 | s)) break;
+        tc_fence_after_sync();
+        const uint32_t kbase = smem_u32(stages + s * kRedStageBytes);
+        const uint32_t vbase = kbase + 2 * kRedBoxBytes;
+#pragma unroll
+        for (int ks = 0; ks < kRedTile / 16; ++ks) {
+          const uint64_t a = smem_desc(kbase + ks * 2048, kRedBoxBytes, 1024, kSwizzle128B);
+          const uint64_t bv = smem_desc(vbase + ks * 2048, kRedBoxBytes, 1024, kSwizzle128B);
+          const uint32_t acc = (i | ks) != 0;
+          umma_bf16(tmem, a, bv, idesc_num, acc);
+          umma_bf16(tmem + 128, a, ones_desc, idesc_den, acc);
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(done);
+    }
+  } else if (warp < 6) {
+    const int t = threadIdx.x - 64;   // 0..127
+    for (int i = 0; i < ntiles1; ++i) {
+      const int s = i % kFuStages1;
+      if (!mbar_wait(&full[s], (i / kFuStages1) & 1, abort_flag, err, kErrFusedP1 | 12)) break;
+      uint8_t* st = stages + s * kRedStageBytes;
+      const int valid = min(kRedTile, n1 - (n0 + i * kRedTile));
+#pragma unroll 4
+      for (int j = t; j < 1024; j += 128) {
+        uint4* c = reinterpret_cast<uint4*>(st + j * 16);
+        const int row = (j >> 3) & (kRedTile - 1);
+        *c = row < valid ? relu_bf16x8(*c) : make_uint4(0u, 0u, 0u, 0u);
+      }
+      if (valid < kRedTile) {
+        for (int j = t; j < 1024; j += 128) {
+          const int row = (j >> 3) & (kRedTile - 1);
+          if (row >= valid) *reinterpret_cast<uint4*>(st + 2 * kRedBoxBytes + j * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&relu_done[s]);
+    }
+    const int hq = warp & 3;
+    float sv[kRows];
+    bool ok = ntiles1 > 0;
+    if (ok) ok = mbar_wait(done, 0, abort_flag, err, kErrFusedP1 | 13);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after_sync();
+      uint32_t rr[32], zr;
+      const uint32_t ta = tmem + (static_cast<uint32_t>(hq * 32) << 16);
+      tmem_ld_x32(ta + hq * 32, rr);
+      tmem_ld_x1(ta + 128, zr);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(rr[j]);
+      sv[32] = __uint_as_float(zr);
+    } else {
+#pragma unroll
+      for (int j = 0; j < kRows; ++j) sv[j] = 0.f;
+    }
+    float* dst = partials + (((int64_t)cidx * p.cpb + r) * kRedHeads + hq) * kStateFloats;
+#pragma unroll
+    for (int j = 0; j < kRows; ++j) dst[j * kD + lane] = sv[j];
+  }
+  // phase 1 is over for this CTA: every MMA completed (the epilogue waited for `done`), every
+  // TMEM read completed, the partial is written
+  tc_fence_before_sync();
+  __threadfence();
+  __syncthreads();
+  tc_fence_after_sync();
+  if (threadIdx.x == 0) atomicAdd(&counters[2 * cidx], 1u);   // arrival of this sibling
+
+  // =============================== phase 2: merge + apply ================================
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int lu = 0; lu < nunits; ++lu) {
+        const int s = lu % kQStages;
+        if (lu >= kQStages &&
+            !mbar_wait(&qempty[s], ((lu / kQStages) - 1) & 1, abort_flag, err, kErrApplyProducer | s))
+          break;
+        const int np = pair_heads_h(p.H, q, 1) > 0 ? 2 : 1;
+        mbar_arrive_expect_tx(&qfull[s], np * kQBoxBytes);
+        for (int h = 0; h < np; ++h)
+          tma_load_3d(qst + s * A::kQStageBytes + h * kQBoxBytes, &tmap_q, &qfull[s],
+                      q * kApUnitHeads * kD + h * kApHeads * kD, (t0 + lu) * kApTile, b);
+        issued = lu + 1;
+      }
+      if (*abort_flag) {
+        for (int i = (issued > kQStages ? issued - kQStages : 0); i < issued; ++i)
+          mbar_drain(&qfull[i % kQStages], (i / kQStages) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && mbar_wait(sfull, 0, abort_flag, err, kErrApplyMma | 8)) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, kImageRows, false, false);
+      const uint32_t saddr = smem_u32(sbuf);
+      int pn = 0;
+      bool stop = false;
+      for (int lu = 0; lu < nunits && !stop; ++lu) {
+        const int s = lu % kQStages;
+        if (!mbar_wait(&qrelu[s], (lu / kQStages) & 1, abort_flag, err, kErrApplyMma | s)) break;
+        const uint32_t qaddr = smem_u32(qst + s * A::kQStageBytes);
+        for (int h = 0; h < 2; ++h) {
+          const int nh = pair_heads_h(p.H, q, h);
+          if (nh == 0) break;
+          const int a = pn % kApAccSlots;
+          if (pn >= kApAccSlots &&
+              !mbar_wait(&tempty[a], ((pn / kApAccSlots) - 1) & 1, abort_flag, err, kErrApplyMma | 12 | a)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after_sync();
+          for (int j = 0; j < nh; ++j) {
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks) {
+              const uint64_t ad = smem_desc(qaddr + h * kQBoxBytes + j * 64 + ks * 32, 16, 1024, kSwizzle128B);
+              const uint64_t bd = smem_desc(saddr + (h * kApHeads + j) * kImageBytes + ks * 256, 128, 512, kSwizzleNone);
+              umma_bf16(tmem + a * kApAccCols + j * kImageRows, ad, bd, idesc, ks);
+            }
+          }
+          umma_commit(&tfull[a]);
+          ++pn;
+        }
+        if (stop) break;
+        umma_commit(&qempty[s]);
+      }
+    }
+  } else if (warp < 4) {
+    const int t = threadIdx.x - 64;   // 0..63
+    const int nchunks = (pair_heads_h(p.H, q, 1) > 0 ? 2 : 1) * (int)(kQBoxBytes / 16);
+    for (int lu = 0; lu < nunits; ++lu) {
+      const int s = lu % kQStages;
+      if (!mbar_wait(&qfull[s], (lu / kQStages) & 1, abort_flag, err, kErrApplyRelu | s)) break;
+      uint8_t* st = qst + s * A::kQStageBytes;
+#pragma unroll 4
+      for (int j = t; j < nchunks; j += kApReluThreads) {
+        uint4* c = reinterpret_cast<uint4*>(st + j * 16);
+        *c = relu_bf16x8(*c);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&qrelu[s]);
+    }
+  } else if (warp < 8) {
+    const int et = threadIdx.x - 128;   // 0..127
+    const bool leader = (et == 0);
+    // ---- merge: wait for the siblings, sum their partials in fixed order, build the B operand
+    bool ok = true;
+    if (leader) {
+      const uint64_t tstart = globaltimer_ns();
+      volatile unsigned* arr = counters + 2 * cidx;
+      while (*arr < (unsigned)p.cpb) {
+        if (*abort_flag) { ok = false; break; }
+        if (globaltimer_ns() - tstart > kWaitLimitNs) {
+          *abort_flag = 1;
+          atomicCAS(err, 0, kErrFusedSibling);
+          ok = false;
+          break;
+        }
+        __nanosleep(256);
+      }
+      __threadfence();   // acquire: the siblings' partial writes precede their arrivals
+    }
+    if (bar_any(1, 128, !ok)) ok = false;
+    const int heads = min(kApUnitHeads, p.H - q * kApUnitHeads);
+    constexpr int kUnits = kRedHeads * kRows * (kD / 8);   // (head, row, 8-column chunk)
+    constexpr int kUPT = (kUnits + 127) / 128;
+    float sum[kUPT][8];
+#pragma unroll
+    for (int k = 0; k < kUPT; ++k)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sum[k][i] = 0.f;
+    const uint8_t* gsrc = reinterpret_cast<const uint8_t*>(partials) + (int64_t)cidx * p.cpb * kPartBytes;
+    int batch = 0;
+    for (int k0 = 0; ok && k0 < p.cpb; k0 += Cfg::kMergeBatch, ++batch) {
+      const int nb = min(Cfg::kMergeBatch, p.cpb - k0);
+      if (leader) {
+        fence_proxy_async_global();
+        mbar_arrive_expect_tx(merge_bar, nb * kPartBytes);
+        for (int i = 0; i < nb; ++i) bulk_load(obuf + i * kPartBytes, gsrc + (int64_t)(k0 + i) * kPartBytes, kPartBytes, merge_bar);
+      }
+      const bool got = mbar_wait(merge_bar, batch & 1, abort_flag, err, kErrFusedMerge);
+      if (bar_any(1, 128, !got)) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int k = 0; k < kUPT; ++k) {
+        const int u = et + k * 128;
+        if (u >= kUnits) break;
+        const int hl = u / (kRows * 4), rcc = u - hl * (kRows * 4), rr = rcc >> 2, cc = rcc & 3;
+        for (int i = 0; i < nb; ++i) {
+          const float4* src = reinterpret_cast<const float4*>(obuf + i * kPartBytes) + (hl * kStateFloats + rr * kD + cc * 8) / 4;
+          const float4 x0 = src[0], x1 = src[1];
+          sum[k][0] += x0.x; sum[k][1] += x0.y; sum[k][2] += x0.z; sum[k][3] += x0.w;
+          sum[k][4] += x1.x; sum[k][5] += x1.y; sum[k][6] += x1.z; sum[k][7] += x1.w;
+        }
+      }
+      bar_sync(2, 128);   // the batch buffer is refilled next
+    }
+    if (ok) {
+#pragma unroll
+      for (int k = 0; k < kUPT; ++k) {
+        const int u = et + k * 128;
+        if (u >= kUnits) break;
+        const int hl = u / (kRows * 4), rcc = u - hl * (kRows * 4), rr = rcc >> 2, cc = rcc & 3;
+        float hi[8], lo[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float v = hl < heads ? sum[k][j] : 0.f;
+          hi[j] = __bfloat162float(__float2bfloat16_rn(v));
+          lo[j] = v - hi[j];
+        }
+        uint8_t* img = sbuf + hl * kImageBytes;
+        *reinterpret_cast<uint4*>(img + image_offset(rr, cc * 8)) = pack_bf16x8(hi);
+        *reinterpret_cast<uint4*>(img + image_offset(kImageLoRow + rr, cc * 8)) = pack_bf16x8(lo);
+      }
+      for (int i = et; i < kRedHeads * 14 * 4; i += 128) {   // zero rows 33..39, 73..79
+        const int hl = i / 56, k = i - hl * 56, zr = k >> 2, cc = k & 3;
+        const int nrow = zr < 7 ? kRows + zr : kImageLoRow + kRows + (zr - 7);
+        *reinterpret_cast<uint4*>(sbuf + hl * kImageBytes + image_offset(nrow, cc * 8)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      fence_proxy_async_smem();
+    }
+    bar_sync(2, 128);
+    if (leader && ok) {
+      mbar_arrive(sfull);
+      // departure of this sibling; the last one resets both counters for the next call
+      if (atomicAdd(&counters[2 * cidx + 1], 1u) == (unsigned)p.cpb - 1u) {
+        counters[2 * cidx] = 0u;
+        counters[2 * cidx + 1] = 0u;
+      }
+    }
+    // ---- epilogue (as litela_apply_tc; the merge buffer was the output staging region)
+    const int hq = warp & 3;
+    const int row = hq * 32 + lane;
+    int nstaged = 0, pn = 0;
+    for (int lu = 0; ok && lu < nunits; ++lu) {
+      const int tok0 = (t0 + lu) * kApTile;   // the last tile is clipped to N by the TMA store
+      uint8_t* slot = obuf + (nstaged % A::kOutSlots) * A::kOutSlotBytes;
+      if (leader) bulk_wait_group_read<A::kOutSlots - 1>();
+      bar_sync(2, 128);
+      ++nstaged;
+      bool stop = false;
+      for (int h = 0; h < 2; ++h) {
+        const int nh = pair_heads_h(p.H, q, h);
+        if (nh == 0) break;
+        const int a = pn % kApAccSlots;
+        const bool okw = mbar_wait(&tfull[a], (pn / kApAccSlots) & 1, abort_flag, err, kErrApplyEpi | a);
+        if (bar_any(1, 128, !okw)) {
+          stop = true;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t ta = tmem + (static_cast<uint32_t>(hq * 32) << 16) + a * kApAccCols;
+        for (int j = 0; j < nh; ++j) {
+          uint32_t v[kImageRows];
+#pragma unroll
+          for (int k = 0; k < kImageRows / 16; ++k) tmem_ld_x16(ta + j * kImageRows + k * 16, v + k * 16);
+          tmem_wait_ld();
+          if (j == nh - 1) {
+            tc_fence_before_sync();
+            mbar_arrive(&tempty[a]);
+          }
+          const float den = (__uint_as_float(v[kD]) + __uint_as_float(v[kImageLoRow + kD])) + p.eps;
+          const float inv = 1.0f / den;
+          float o[kD];
+#pragma unroll
+          for (int rr2 = 0; rr2 < kD; ++rr2)
+            o[rr2] = (__uint_as_float(v[rr2]) + __uint_as_float(v[kImageLoRow + rr2])) * inv;
+          uint4 w[kChunksPerHead];
+          pack_out(static_cast<OutT*>(nullptr), o, w);
+          const int hu = h * kApHeads + j;
+#pragma unroll
+          for (int k = 0; k < kChunksPerHead; ++k) {
+            const int ck = hu * kChunksPerHead + k;
+            uint8_t* box = slot + (ck >> 3) * kOutBoxBytes;
+            *reinterpret_cast<uint4*>(box + row * 128 + (((ck & 7) ^ (row & 7)) << 4)) = w[k];
+          }
+        }
+        ++pn;
+      }
+      if (stop) break;
+      fence_proxy_async_smem();
+      bar_sync(2, 128);
+      if (leader) {
+        const int x0 = q * kApUnitHeads * kD;
+#pragma unroll
+        for (int bx = 0; bx < A::kOutBoxes; ++bx)
+          if (x0 + bx * A::kBoxChannels < p.H * kD)
+            tma_store_3d(&tmap_out, slot + bx * kOutBoxBytes, x0 + bx * A::kBoxChannels, tok0, b);
+        bulk_commit_group();
+      }
+    }
+    if (leader) bulk_wait_group<0>();
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kFuTmemCols);
+  }
+}
+
+}  // namespace litela

@@ -27,8 +27,10 @@ constexpr int kApTile = 128;
 constexpr int kImageRows = 80;
 constexpr int kImageLoRow = 40;
 constexpr int kImageBytes = kImageRows * kD * 2;
-// the kernels' error word (a bounded wait that timed out) lives in its own small buffer
+// small zero-initialised control buffer: word 0 is the kernels' error word (a bounded wait that
+// timed out); the fused kernel's sibling counters start at word kCounterBase
 constexpr int kErrWords = 64;
+constexpr int kCounterBase = kErrWords;
 
 struct Plan {
   int B = 0, N = 0, H = 0;
@@ -44,6 +46,11 @@ struct Plan {
   //   partial states fp32 [B][ngroups][nblk * chunks_per_block][4][33][32]
   //   state images (the apply's B operand) bf16 [B][H][nblk][kImageBytes]
   size_t off_images = 0, bytes = 0;
+  // fused single-kernel path (non-causal, B * nquads <= SMs): CTA (b, quad, r), r < fused_cpb;
+  // workspace = fused partials [B][nquads][fused_cpb][4][33][32]; counters 2 per (b, quad)
+  bool fused = false;
+  int fused_cpb = 0, fused_chunk = 0, fused_ntiles = 0;
+  size_t fused_bytes = 0, counters = 0;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -75,6 +82,20 @@ inline bool make_plan(int B, int N, int H, int tokens_per_block, int num_sms, Pl
   const size_t images = (size_t)B * H * p->nblk * kImageBytes;
   p->off_images = align_up(partials, 256);
   p->bytes = p->off_images + align_up(images, 256);
+  const int sms = num_sms > 0 ? num_sms : 148;
+  if (p->nblk == 1 && (int64_t)B * p->nquads <= sms) {
+    p->fused = true;
+    p->fused_ntiles = (N + kApTile - 1) / kApTile;
+    int cpb = sms / (B * p->nquads);
+    if (cpb > p->fused_ntiles) cpb = p->fused_ntiles;
+    if (cpb < 1) cpb = 1;
+    int64_t chunk = ((int64_t)N + cpb - 1) / cpb;
+    chunk = (chunk + kRedTile - 1) / kRedTile * kRedTile;
+    p->fused_cpb = cpb;
+    p->fused_chunk = (int)chunk;
+    p->fused_bytes = align_up((size_t)B * p->nquads * cpb * kRedHeads * kStateFloats * sizeof(float), 256);
+    p->counters = (size_t)2 * B * p->nquads;
+  }
   return true;
 }
 

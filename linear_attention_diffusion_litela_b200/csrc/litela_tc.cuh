@@ -445,8 +445,20 @@ __device__ __forceinline__ ApUnit ap_decode(long long u, const ApRange& R, const
 }
 
 // heads of pair h (0 or 1) of a unit
-__device__ __forceinline__ int pair_heads(const TcPlan& p, int quad, int h) {
-  return max(0, min(kApHeads, p.H - quad * kApUnitHeads - h * kApHeads));
+__device__ __forceinline__ int pair_heads_h(int H, int quad, int h) {
+  return max(0, min(kApHeads, H - quad * kApUnitHeads - h * kApHeads));
+}
+__device__ __forceinline__ int pair_heads(const TcPlan& p, int quad, int h) { return pair_heads_h(p.H, quad, h); }
+
+// 8 floats -> 8 packed bf16 (round to nearest even)
+__device__ __forceinline__ uint4 pack_bf16x8(const float* x) {
+  uint32_t u[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 v2 = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    u[i] = *reinterpret_cast<uint32_t*>(&v2);
+  }
+  return make_uint4(u[0], u[1], u[2], u[3]);
 }
 
 __device__ __forceinline__ void pack_out(__nv_bfloat16*, const float* o, uint4* w) {

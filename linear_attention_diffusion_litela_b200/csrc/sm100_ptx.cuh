@@ -28,6 +28,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// orders generic-proxy global writes (made visible to this thread by an acquire) before
+// this thread's later async-proxy (bulk copy) reads of the same memory
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------------------
 // mbarriers
 
