@@ -71,6 +71,24 @@ litela_status lite_la_fwd(const void* qkv, void* out, int B, int N, int H, int d
 litela_status lite_la_block_causal_fwd(const void* qkv, void* out, int B, int N, int H, int d,
                                        float eps, int tokens_per_block, cudaStream_t stream);
 
+/* Block-causal LiteLA over one chunk of a longer sequence, carrying the state across chunks
+ * (the "constant-memory KV cache" of Block-Linear Attention: same instagit page, section "Video
+ * Generation and Constant-Memory KV Cache").  state_in: device fp32 [B, H, d+1, d], the prefix
+ * state of every token of the earlier chunks (rows r < d: sum of v_r * relu(k); row d: sum of
+ * relu(k)), or NULL for none; it is added to the state of every block of this chunk.
+ * state_out: device fp32 [B, H, d+1, d], receives state_in plus the state of all of this chunk's
+ * tokens (the state_in of the next chunk), or NULL.  state_out may be state_in (updated in
+ * place); neither may overlap qkv or out; both 16-byte aligned.  With chunk lengths that are
+ * multiples of tokens_per_block, chaining chunks gives exactly the block-causal result of the
+ * whole sequence.  Other arguments as lite_la_block_causal_fwd. */
+litela_status lite_la_block_causal_fwd_carry(const void* qkv, void* out, int B, int N, int H, int d,
+                                             float eps, int tokens_per_block, const float* state_in,
+                                             float* state_out, cudaStream_t stream);
+litela_status lite_la_block_causal_fwd_carry_f32out(const void* qkv, float* out, int B, int N, int H,
+                                                    int d, float eps, int tokens_per_block,
+                                                    const float* state_in, float* state_out,
+                                                    cudaStream_t stream);
+
 /* The same two operations with an fp32 output buffer [B, N, H*d] (debug / accuracy mode). */
 litela_status lite_la_fwd_f32out(const void* qkv, float* out, int B, int N, int H, int d,
                                  float eps, cudaStream_t stream);

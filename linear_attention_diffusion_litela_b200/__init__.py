@@ -39,6 +39,8 @@ _SIGNATURES = {
     "lite_la_fwd_f32out": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp]),
     "lite_la_block_causal_fwd_f32out": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
     "lite_la_fwd_events": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp, _vp]),
+    "lite_la_block_causal_fwd_carry": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp, _vp, _vp]),
+    "lite_la_block_causal_fwd_carry_f32out": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp, _vp, _vp]),
     "lite_la_device_status": (_c_int, [_vp]),
     "lite_la_selftest_timeout": (_c_int, [_vp]),
     "lite_la_state_fwd": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _vp]),
@@ -131,6 +133,30 @@ def lite_la_block_causal_fwd(qkv, H: int, tokens_per_block: int, d: int = 32, ep
         _check(fn(qkv.data_ptr(), out.data_ptr(), B, N, H, d, eps, int(tokens_per_block),
                   _stream_handle(stream, qkv.device)))
     return out
+
+
+def lite_la_block_causal_fwd_carry(qkv, H: int, tokens_per_block: int, state_in=None, state_out=None,
+                                   d: int = 32, eps: float = 1e-15, out=None, out_dtype=None, stream=None):
+    """Block-causal LiteLA of one chunk with the state of earlier chunks carried in (state_in,
+    fp32 [B, H, d+1, d] or None) and the state after this chunk written to state_out (allocated
+    when None; may be state_in).  Returns (out, state_out)."""
+    torch = _torch()
+    B, N, out = _prepare(qkv, H, d, out, out_dtype or torch.bfloat16)
+    shape = (B, H, d + 1, d)
+    for t in (state_in,):
+        if t is not None and (t.dtype != torch.float32 or tuple(t.shape) != shape or not t.is_contiguous()
+                              or t.device != qkv.device):
+            raise TypeError("state_in must be a contiguous fp32 tensor [B, H, d+1, d] on qkv's device")
+    if state_out is None:
+        state_out = torch.empty(shape, dtype=torch.float32, device=qkv.device)
+    elif state_out.dtype != torch.float32 or tuple(state_out.shape) != shape or not state_out.is_contiguous():
+        raise TypeError("state_out must be a contiguous fp32 tensor [B, H, d+1, d]")
+    fn = lib().lite_la_block_causal_fwd_carry if out.dtype == torch.bfloat16 else lib().lite_la_block_causal_fwd_carry_f32out
+    with torch.cuda.device(qkv.device):
+        _check(fn(qkv.data_ptr(), out.data_ptr(), B, N, H, d, eps, int(tokens_per_block),
+                  None if state_in is None else state_in.data_ptr(), state_out.data_ptr(),
+                  _stream_handle(stream, qkv.device)))
+    return out, state_out
 
 
 def lite_la_state_fwd(qkv, H: int, tokens_per_block: int = 0, d: int = 32, out=None, stream=None):

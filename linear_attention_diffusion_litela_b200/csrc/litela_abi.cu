@@ -130,8 +130,9 @@ litela_status encode_out_map(OutT* out, int B, int N, int H, CUtensorMap* map) {
 struct Workspace {
   void* partials = nullptr;   // partial states (and, for the three-kernel path, state images)
   size_t partials_bytes = 0;
-  int* err = nullptr;         // control words: error word, then the fused kernel's counters
+  int* err = nullptr;         // control words: error word, then the fused kernel's two counter sets
   size_t ctl_words = 0;
+  unsigned long long calls = 0;   // fused calls so far: their parity selects the counter set
 };
 
 // bytes of partial-state workspace a call with `plan` uses
@@ -264,12 +265,13 @@ litela_status launch_reduce(const Plan& plan, const void* qkv, float* partials, 
 }
 
 litela_status launch_scan(const Plan& plan, const float* partials, uint8_t* images, float* states, int num_sms,
-                          cudaStream_t stream, bool pdl) {
+                          cudaStream_t stream, bool pdl, const float* state_in = nullptr,
+                          float* state_out = nullptr) {
   const int64_t work = ((int64_t)plan.B * plan.H * kStateFloats + kScanElems - 1) / kScanElems;
   int64_t grid = (work + kScanThreads - 1) / kScanThreads;
   if (grid > num_sms) grid = num_sms;
   cudaError_t e = launch_ex(litela_state_scan, dim3((unsigned)grid), dim3(kScanThreads), 0, stream, pdl,
-                            partials, images, states, tc_plan(plan, 0.f));
+                            partials, images, states, state_in, state_out, tc_plan(plan, 0.f));
   if (e != cudaSuccess) return cuda_fail(e, "launch litela_state_scan");
   return LITELA_OK;
 }
@@ -278,7 +280,8 @@ litela_status launch_scan(const Plan& plan, const float* partials, uint8_t* imag
 // events, if requested, bracket it (events[1] is recorded with events[2], after the kernel).
 template <typename OutT>
 litela_status launch_fused(const Plan& plan, const void* qkv, OutT* out, float eps, float* partials, int* ctl,
-                           cudaStream_t stream, cudaEvent_t* events) {
+                           size_t ctl_words, unsigned long long call_index, cudaStream_t stream,
+                           cudaEvent_t* events) {
   CUtensorMap map_kv, map_q, map_out;
   litela_status s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kRedTile, &map_kv);
   if (s != LITELA_OK) return s;
@@ -288,7 +291,10 @@ litela_status launch_fused(const Plan& plan, const void* qkv, OutT* out, float e
   if (s != LITELA_OK) return s;
   cudaError_t e;
   if (events && (e = cudaEventRecord(events[0], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  const FusedPlan fp{plan.B, plan.N, plan.H, plan.nquads, plan.fused_cpb, plan.fused_chunk, plan.fused_ntiles, eps};
+  // two counter sets of (ctl_words - kCounterBase) / 2 words each; calls alternate between them
+  const int set_words = (int)((ctl_words - kCounterBase) / 2);
+  const FusedPlan fp{plan.B,           plan.N,    plan.H, plan.nquads, plan.fused_cpb, plan.fused_chunk,
+                     plan.fused_ntiles, (int)(call_index & 1), set_words, eps};
   const unsigned grid = (unsigned)(plan.B * plan.nquads * plan.fused_cpb);
   e = launch_ex(litela_fused_tc<OutT>, dim3(grid), dim3(kFuThreads), FusedCfg<OutT>::kSmemBytes, stream,
                 events == nullptr, map_kv, map_q, map_out, partials, reinterpret_cast<unsigned*>(ctl + kCounterBase),
@@ -306,7 +312,8 @@ litela_status launch_fused(const Plan& plan, const void* qkv, OutT* out, float e
 // stream order with events between the reduction (with the scan) and the apply.
 template <typename OutT>
 litela_status launch(const Plan& plan, const void* qkv, OutT* out, float eps, float* partials, uint8_t* images,
-                     int* err, int num_sms, cudaStream_t stream, cudaEvent_t* events) {
+                     int* err, int num_sms, cudaStream_t stream, cudaEvent_t* events,
+                     const float* state_in = nullptr, float* state_out = nullptr) {
   CUtensorMap map_q, map_out;
   litela_status s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kApTile, &map_q);
   if (s != LITELA_OK) return s;
@@ -317,7 +324,7 @@ litela_status launch(const Plan& plan, const void* qkv, OutT* out, float eps, fl
   if (events && (e = cudaEventRecord(events[0], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   s = launch_reduce(plan, qkv, partials, err, stream, pdl);
   if (s != LITELA_OK) return s;
-  s = launch_scan(plan, partials, images, nullptr, num_sms, stream, pdl);
+  s = launch_scan(plan, partials, images, nullptr, num_sms, stream, pdl, state_in, state_out);
   if (s != LITELA_OK) return s;
   if (events && (e = cudaEventRecord(events[1], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   // CTAs: a multiple of the head quads when that keeps at least 7/8 of the SMs busy (all quads
@@ -363,7 +370,8 @@ litela_status run_states(const void* qkv, float* states, int B, int N, int H, in
 
 template <typename OutT>
 litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float eps, int tokens_per_block,
-                  bool causal, cudaStream_t stream, cudaEvent_t* events = nullptr) {
+                  bool causal, cudaStream_t stream, cudaEvent_t* events = nullptr, bool carry = false,
+                  const float* state_in = nullptr, float* state_out = nullptr) {
   bool empty = false;
   litela_status s = validate(qkv, out, sizeof(OutT), B, N, H, d, eps, tokens_per_block, causal, &empty);
   if (s != LITELA_OK || empty) return s;
@@ -372,12 +380,29 @@ litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float 
   if (s != LITELA_OK) return s;
   Plan plan;
   make_plan(B, N, H, causal ? tokens_per_block : 0, num_sms, &plan);
+  if (carry) {   // the carried state enters through the scan: use the three-kernel path
+    plan.fused = false;
+    plan.counters = 0;
+    const size_t sbytes = (size_t)B * H * kStateFloats * sizeof(float);
+    const size_t qkv_bytes = (size_t)B * N * 3 * H * d * sizeof(__nv_bfloat16);
+    const size_t out_bytes = (size_t)B * N * H * d * sizeof(OutT);
+    if ((state_in && (reinterpret_cast<uintptr_t>(state_in) & 15u)) ||
+        (state_out && (reinterpret_cast<uintptr_t>(state_out) & 15u)))
+      return fail(LITELA_ERR_INVALID_ARGUMENT, "state_in and state_out must be 16-byte aligned");
+    if ((state_in && (overlaps(state_in, sbytes, qkv, qkv_bytes) || overlaps(state_in, sbytes, out, out_bytes))) ||
+        (state_out && (overlaps(state_out, sbytes, qkv, qkv_bytes) || overlaps(state_out, sbytes, out, out_bytes))))
+      return fail(LITELA_ERR_INVALID_ARGUMENT, "a state buffer overlaps qkv or out");
+  }
   Workspace* ws = nullptr;
   s = get_workspace(plan, stream, &ws);
   if (s != LITELA_OK) return s;
   char* base = static_cast<char*>(ws->partials);
-  if (plan.fused)
-    s = launch_fused(plan, qkv, out, eps, reinterpret_cast<float*>(base), ws->err, stream, events);
+  if (carry)
+    s = launch(plan, qkv, out, eps, reinterpret_cast<float*>(base), reinterpret_cast<uint8_t*>(base + plan.off_images),
+               ws->err, num_sms, stream, events, state_in, state_out);
+  else if (plan.fused)
+    s = launch_fused(plan, qkv, out, eps, reinterpret_cast<float*>(base), ws->err, ws->ctl_words, ws->calls++, stream,
+                     events);
   else
     s = launch(plan, qkv, out, eps, reinterpret_cast<float*>(base), reinterpret_cast<uint8_t*>(base + plan.off_images),
                ws->err, num_sms, stream, events);
@@ -431,11 +456,11 @@ litela_status run_noalloc(const void* qkv, __nv_bfloat16* out, int B, int N, int
   if (s != LITELA_OK) return s;
   char* base = static_cast<char*>(scratch);
   if (plan.fused) {
-    // the sibling counters must start at zero (the kernel leaves them so; an aborted call might not)
+    // the counters must start at zero: cleared here every call (no state survives between calls)
     cudaError_t e = cudaMemsetAsync(base + kCounterBase * sizeof(int), 0, plan.counters * sizeof(unsigned), stream);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(no-alloc counters)");
     s = launch_fused(plan, qkv, out, eps, reinterpret_cast<float*>(base + err_bytes), reinterpret_cast<int*>(base),
-                     stream, nullptr);
+                     kCounterBase + plan.counters, 0, stream, nullptr);
     if (s == LITELA_OK) g_last_error.clear();
     return s;
   }
@@ -469,6 +494,19 @@ litela_status lite_la_fwd_f32out(const void* qkv, float* out, int B, int N, int 
 litela_status lite_la_block_causal_fwd_f32out(const void* qkv, float* out, int B, int N, int H, int d,
                                               float eps, int tokens_per_block, cudaStream_t stream) {
   return litela::run(qkv, out, B, N, H, d, eps, tokens_per_block, true, stream);
+}
+
+litela_status lite_la_block_causal_fwd_carry(const void* qkv, void* out, int B, int N, int H, int d, float eps,
+                                             int tokens_per_block, const float* state_in, float* state_out,
+                                             cudaStream_t stream) {
+  return litela::run(qkv, static_cast<__nv_bfloat16*>(out), B, N, H, d, eps, tokens_per_block, true, stream, nullptr,
+                     true, state_in, state_out);
+}
+
+litela_status lite_la_block_causal_fwd_carry_f32out(const void* qkv, float* out, int B, int N, int H, int d,
+                                                    float eps, int tokens_per_block, const float* state_in,
+                                                    float* state_out, cudaStream_t stream) {
+  return litela::run(qkv, out, B, N, H, d, eps, tokens_per_block, true, stream, nullptr, true, state_in, state_out);
 }
 
 litela_status lite_la_fwd_events(const void* qkv, void* out, int B, int N, int H, int d, float eps,

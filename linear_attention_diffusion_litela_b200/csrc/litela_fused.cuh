@@ -11,6 +11,9 @@
 //            quad's state as the MMA's B operand (bf16 hi + lo, as litela_state_scan does);
 //   phase 2  applies the state to tiles [r*ntiles/cpb, (r+1)*ntiles/cpb) of batch b's tokens
 //            exactly as litela_apply_tc does (its q prefetch overlaps the merge).
+// The arrival counters come in two sets used by alternate calls: a call zeroes the set its
+// predecessor used (after waiting for it), so a set is clean whenever it is used, even after a
+// call that gave up on a wait.
 // The only cross-CTA dependency is among the cpb siblings, which finish phase 1 at about the
 // same time.  The grid has at most one CTA per SM (its shared memory admits no second one) and
 // at most as many CTAs as SMs, so siblings are co-resident unless other kernels hold SMs, in
@@ -29,6 +32,8 @@ namespace litela {
 
 struct FusedPlan {
   int B, N, H, nquads, cpb, chunk, ntiles;
+  int parity;          // which of the two counter sets this call uses (calls alternate)
+  int counter_words;   // capacity of one counter set
   float eps;
 };
 
@@ -90,6 +95,8 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
   const int br = blockIdx.x / p.nquads;
   const int r = br % p.cpb, b = br / p.cpb;
   const int cidx = b * p.nquads + q;
+  unsigned* my_counters = counters + (size_t)p.parity * p.counter_words;
+  unsigned* old_counters = counters + (size_t)(p.parity ^ 1) * p.counter_words;
   // phase 1: chunk r of batch b's tokens
   const int n0 = r * p.chunk, n1 = min(n0 + p.chunk, p.N);
   const int ntiles1 = n1 > n0 ? (n1 - n0 + kRedTile - 1) / kRedTile : 0;
@@ -136,6 +143,8 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
   const uint32_t tmem = *tmem_holder;
   // private set-up above; global memory only after the previous kernel in the stream is done
   pdl_wait_primary();
+  for (int i = blockIdx.x * kFuThreads + threadIdx.x; i < p.counter_words; i += gridDim.x * kFuThreads)
+    old_counters[i] = 0u;   // the previous call's set: clean for the call after this one
 
   // =============================== phase 1: state reduction ===============================
   const int kx = p.H * kD + q * (kRedHeads * kD), vx = 2 * p.H * kD + q * (kRedHeads * kD);
@@ -235,7 +244,7 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
   __threadfence();
   __syncthreads();
   tc_fence_after_sync();
-  if (threadIdx.x == 0) atomicAdd(&counters[2 * cidx], 1u);   // arrival of this sibling
+  if (threadIdx.x == 0) atomicAdd(&my_counters[cidx], 1u);   // arrival of this sibling
 
   // =============================== phase 2: merge + apply ================================
   if (warp == 0) {
@@ -315,7 +324,7 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
     bool ok = true;
     if (leader) {
       const uint64_t tstart = globaltimer_ns();
-      volatile unsigned* arr = counters + 2 * cidx;
+      volatile unsigned* arr = my_counters + cidx;
       while (*arr < (unsigned)p.cpb) {
         if (*abort_flag) { ok = false; break; }
         if (globaltimer_ns() - tstart > kWaitLimitNs) {
@@ -390,14 +399,7 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
       fence_proxy_async_smem();
     }
     bar_sync(2, 128);
-    if (leader && ok) {
-      mbar_arrive(sfull);
-      // departure of this sibling; the last one resets both counters for the next call
-      if (atomicAdd(&counters[2 * cidx + 1], 1u) == (unsigned)p.cpb - 1u) {
-        counters[2 * cidx] = 0u;
-        counters[2 * cidx + 1] = 0u;
-      }
-    }
+    if (leader && ok) mbar_arrive(sfull);
     // ---- epilogue (as litela_apply_tc; the merge buffer was the output staging region)
     const int hq = warp & 3;
     const int row = hq * 32 + lane;

@@ -47,7 +47,8 @@ struct Plan {
   //   state images (the apply's B operand) bf16 [B][H][nblk][kImageBytes]
   size_t off_images = 0, bytes = 0;
   // fused single-kernel path (non-causal, B * nquads <= SMs): CTA (b, quad, r), r < fused_cpb;
-  // workspace = fused partials [B][nquads][fused_cpb][4][33][32]; counters 2 per (b, quad)
+  // workspace = fused partials [B][nquads][fused_cpb][4][33][32]; two sets of B * nquads
+  // arrival counters (calls alternate between them)
   bool fused = false;
   int fused_cpb = 0, fused_chunk = 0, fused_ntiles = 0;
   size_t fused_bytes = 0, counters = 0;
@@ -94,7 +95,7 @@ inline bool make_plan(int B, int N, int H, int tokens_per_block, int num_sms, Pl
     p->fused_cpb = cpb;
     p->fused_chunk = (int)chunk;
     p->fused_bytes = align_up((size_t)B * p->nquads * cpb * kRedHeads * kStateFloats * sizeof(float), 256);
-    p->counters = (size_t)2 * B * p->nquads;
+    p->counters = (size_t)2 * B * p->nquads;   // both sets
   }
   return true;
 }

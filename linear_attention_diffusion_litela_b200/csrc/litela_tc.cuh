@@ -285,7 +285,9 @@ __device__ __forceinline__ const float* partial_ptr(const float* partials, const
 // litela_state_scan: partial states -> per-(batch, head, block) inclusive prefix states, summed in
 // fixed order (deterministic).  Writes each one as the apply's B-operand image (bf16 hi rows
 // 0..32, lo rows 40..72, zero rows in between and after; S = hi + lo to 2^-17 relative) and,
-// when `states` is not null, as fp32 [B][H][nblk][33][32].  Grid-stride over the state elements
+// when `states` is not null, as fp32 [B][H][nblk][33][32].  `state_in` (fp32 [B][H][33][32], may be
+// null) is a state carried from earlier chunks of the sequence and starts every prefix;
+// `state_out` (may be null, may alias state_in) receives the final prefix.  Grid-stride over the state elements
 // with at most one small CTA per SM: its CTAs launch early as a programmatic dependent of the
 // reduction and must leave registers on each SM for the apply's CTAs to land while they wait.
 // Each thread keeps 2 elements x 8 partial loads in flight per round.
@@ -295,7 +297,7 @@ constexpr int kScanElems = 2;         // state elements per thread and round
 
 __global__ void __launch_bounds__(kScanThreads)
 litela_state_scan(const float* __restrict__ partials, uint8_t* __restrict__ images, float* __restrict__ states,
-                  TcPlan p) {
+                  const float* __restrict__ state_in, float* __restrict__ state_out, TcPlan p) {
   using namespace sm100;
   pdl_launch_dependents();
   const int64_t stride = (int64_t)gridDim.x * kScanThreads;
@@ -331,7 +333,10 @@ litela_state_scan(const float* __restrict__ partials, uint8_t* __restrict__ imag
     }
     float run[kE], sum[kE];
 #pragma unroll
-    for (int j = 0; j < kE; ++j) run[j] = sum[j] = 0.f;
+    for (int j = 0; j < kE; ++j) {   // the carried state of earlier chunks starts every prefix
+      run[j] = (state_in != nullptr && ok[j]) ? state_in[bh[j] * kStateFloats + e[j]] : 0.f;
+      sum[j] = 0.f;
+    }
     for (int k0 = 0; k0 < nparts; k0 += 8) {
       float v[kE][8];
 #pragma unroll
@@ -362,6 +367,11 @@ litela_state_scan(const float* __restrict__ partials, uint8_t* __restrict__ imag
           }
         }
       }
+    }
+    if (state_out != nullptr) {
+#pragma unroll
+      for (int j = 0; j < kE; ++j)
+        if (ok[j]) state_out[bh[j] * kStateFloats + e[j]] = run[j];
     }
   }
 }

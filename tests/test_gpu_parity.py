@@ -296,3 +296,44 @@ def test_eps_zero_and_a_head_with_only_negative_keys():
     assert_close(got[~dead].reshape(-1), want[~dead].reshape(-1), "f32")
     with_eps = gpu_run(qkv, H, mode="f32")                 # with eps the dead head is exactly 0
     assert np.all(with_eps[1, :, 4] == 0.0)
+
+
+@pytest.mark.parametrize("mode", ["bf16", "f32"])
+@pytest.mark.parametrize("B,H,T,chunks", [(1, 3, 128, [256, 384, 100]), (2, 5, 64, [64, 64, 128, 7]),
+                                          (1, 70, 1024, [4096, 4096])])
+def test_state_carry_over_chunks_equals_the_whole_sequence(B, H, T, chunks, mode):
+    """Chunked block-causal calls that carry the state (chunk lengths multiples of T) give the
+    block-causal result of the whole sequence, and the final carried state is the state of all
+    tokens."""
+    N = sum(chunks)
+    dt = torch.bfloat16 if mode == "bf16" else torch.float32
+    qkv = make_qkv(B, N, H, 32, seed=17 * N + H + T, device="cuda")
+    state, outs, n0 = None, [], 0
+    for i, c in enumerate(chunks):
+        part = qkv[:, n0:n0 + c].contiguous()
+        # alternate between a fresh output state and updating the carried state in place
+        out, state = ll.lite_la_block_causal_fwd_carry(part, H, T, state_in=state,
+                                                       state_out=state if (i % 2 and state is not None) else None,
+                                                       eps=EPS, out_dtype=dt)
+        outs.append(out)
+        n0 += c
+    torch.cuda.synchronize()
+    ll.lite_la_device_status()
+    got = torch.cat(outs, dim=1).view(B, N, H, 32).double().cpu().numpy()
+    rows = np.arange(N) if N <= 2048 else sample_rows(N, T=T, k=96, seed=3)
+    assert_close(got[:, rows], oracle_run(qkv, H, T=T, rows=rows), mode)
+    full = state_reference(to_bits(qkv), B, N, H, 0)[:, :, 0]
+    scale = np.abs(full).max(axis=(-1, -2), keepdims=True) + 1e-30
+    assert np.all(np.abs(state.double().cpu().numpy() - full) <= 1e-5 * scale + 1e-6)
+
+
+def test_state_carry_without_state_in_is_the_plain_block_causal_call():
+    B, N, H, T = 1, 700, 4, 128
+    qkv = make_qkv(B, N, H, 32, seed=77, device="cuda")
+    out, st = ll.lite_la_block_causal_fwd_carry(qkv, H, T, eps=EPS, out_dtype=torch.float32)
+    ref = ll.lite_la_block_causal_fwd(qkv, H, T, eps=EPS, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)                      # same kernels, same order: bitwise
+    full = ll.lite_la_state_fwd(qkv, H, 0)
+    torch.cuda.synchronize()
+    assert torch.allclose(st, full[:, :, 0], rtol=1e-6, atol=1e-5)
