@@ -31,12 +31,15 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 WORKLOADS_BENCH = {
-    # name: (B, N, H, calls per step, seed base)
-    "sana4800m_4096px_x60": (2, 128 * 128, 70, 60, 4000),
+    # name: (B, N, H, calls per step, seed base, tokens per causal block or 0)
+    "sana4800m_4096px_x60": (2, 128 * 128, 70, 60, 4000, 0),
     # one 4096px call per step on one buffer: the small case for detailed ncu captures
-    "sana4800m_4096px_x1": (2, 128 * 128, 70, 1, 4000),
-    "sana1600m_1024px": (2, 32 * 32, 70, 20, 1001),
-    "sana1600m_2048px": (2, 64 * 64, 70, 20, 1002),
+    "sana4800m_4096px_x1": (2, 128 * 128, 70, 1, 4000, 0),
+    "sana1600m_1024px": (2, 32 * 32, 70, 20, 1001, 0),
+    "sana1600m_2048px": (2, 64 * 64, 70, 20, 1002, 0),
+    # video-style block-causal call: 16 blocks of 1024 tokens, 20 distinct buffers per step
+    "block_causal_16x1024": (1, 16 * 1024, 70, 20, 1004, 1024),
+    "block_causal_16x1024_x1": (1, 16 * 1024, 70, 1, 1004, 1024),
 }
 D = 32
 EPS = 1e-15
@@ -51,8 +54,8 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
 # E = B*N*H*d elements).
 PATHS = {
     1: {"phases": ("litela_fused_tc",), "alg_bytes_E": {"litela_fused_tc": 8}},
-    3: {"phases": ("litela_reduce_tc", "litela_apply_tc"),
-        "alg_bytes_E": {"litela_reduce_tc": 4, "litela_apply_tc": 4}},
+    3: {"phases": ("litela_reduce_tc+litela_state_scan", "litela_apply_tc"),
+        "alg_bytes_E": {"litela_reduce_tc+litela_state_scan": 4, "litela_apply_tc": 4}},
 }
 
 
@@ -137,6 +140,39 @@ def clocks_rejected(c):
     return False
 
 
+def measure_ffma_peak(ll, dev, stream, seconds):
+    """fp32 FMA peak of this GPU: the FMA loop of liblitela_ffma_peak on every SM (4 CTAs of
+    512 threads per SM), sized to run about `seconds`, timed with CUDA events on `stream`, with
+    the clocks it ran at."""
+    import ctypes
+    import torch
+    h = ll.ffma_peak_lib()
+    props = torch.cuda.get_device_properties(dev)
+    blocks, threads = props.multi_processor_count * 4, 512
+    sink = torch.empty(blocks * threads, dtype=torch.float32, device=dev)
+    sh = ctypes.c_void_p(stream.cuda_stream)
+
+    def run(iters):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        if h.litela_ffma_launch(sink.data_ptr(), blocks, threads, iters, sh) != 0:
+            raise RuntimeError("litela_ffma_launch failed")
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1)
+
+    iters = 2000
+    ms = run(iters)
+    iters = max(iters, int(iters * seconds * 1e3 / max(ms, 1e-3)))
+    uuid = "GPU-" + str(props.uuid)
+    with ClockSampler(uuid) as cs:
+        ms = run(iters)
+    flops = h.litela_ffma_flops(blocks, threads, iters)
+    return {"tflops": flops / (ms * 1e-3) / 1e12, "seconds": ms * 1e-3, "blocks": blocks, "threads": threads,
+            "clocks": cs.summary(), "how": "8 independent fp32 FMA chains per thread, 2048 threads per SM, "
+                                           "CUDA events on the launching stream"}
+
+
 def cpu_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -155,14 +191,21 @@ def one_head_bits(qkv_bits, B, N, H, b, h):
     return np.ascontiguousarray(x.reshape(1, N, 3 * D))
 
 
-def oracle_head_rate(qkv_bits, B, N, H, seconds, max_heads=None):
+def oracle_head(oracle, head_bits, N, T):
+    """The oracle on one whole (batch, head): non-causal when T == 0."""
+    if T:
+        return oracle.lite_la_block_causal_fwd(head_bits, 1, N, 1, D, EPS, T)
+    return oracle.lite_la_fwd(head_bits, 1, N, 1, D, EPS)
+
+
+def oracle_head_rate(qkv_bits, B, N, H, T, seconds, max_heads=None):
     """Times the fp64 oracle on whole heads (all N queries of one (batch, head)) until
     `seconds` have passed; returns (tokens*heads per second, heads done, elapsed)."""
     import oracle
     heads, t0 = 0, time.perf_counter()
     while True:
         b, h = divmod(heads % (B * H), H)
-        oracle.lite_la_fwd(one_head_bits(qkv_bits, B, N, H, b, h), 1, N, 1, D, EPS)
+        oracle_head(oracle, one_head_bits(qkv_bits, B, N, H, b, h), N, T)
         heads += 1
         el = time.perf_counter() - t0
         if el >= seconds or (max_heads and heads >= max_heads):
@@ -181,21 +224,22 @@ def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    B, N, H, calls, seed = WORKLOADS_BENCH[wl]
+    B, N, H, calls, seed, T = WORKLOADS_BENCH[wl]
     bits = to_bits(make_qkv(B, N, H, D, seed=seed, device="cpu"))
     import oracle
     heads = [(i // H % B, i % H) for i in range(args.warmup + args.steps)]
     for i in range(args.warmup):
-        oracle.lite_la_fwd(one_head_bits(bits, B, N, H, *heads[i]), 1, N, 1, D, EPS)
+        oracle_head(oracle, one_head_bits(bits, B, N, H, *heads[i]), N, T)
     times = []
     for i in range(args.steps):
         hb = one_head_bits(bits, B, N, H, *heads[args.warmup + i])
         t0 = time.perf_counter()
-        oracle.lite_la_fwd(hb, 1, N, 1, D, EPS)
+        oracle_head(oracle, hb, N, T)
         times.append(time.perf_counter() - t0)
     ms = 1e3 * float(np.mean(times))
     value = N / (ms / 1e3)
-    sample = "one whole (batch, head) per step: all %d queries against all %d keys" % (N, N)
+    sample = ("one whole (batch, head) per step: all %d queries against all %d keys" % (N, N) if not T else
+              "one whole (batch, head) per step: %d queries, blocks of %d tokens" % (N, T))
     emit({"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
           "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -208,8 +252,8 @@ def run_reference(args, wl):
 
 
 def config_of(wl):
-    B, N, H, calls, seed = WORKLOADS_BENCH[wl]
-    return {"workload": wl, "B": B, "N": N, "H": H, "d": D, "calls_per_step": calls,
+    B, N, H, calls, seed, T = WORKLOADS_BENCH[wl]
+    return {"workload": wl, "B": B, "N": N, "H": H, "d": D, "tokens_per_block": T or None, "calls_per_step": calls,
             "distinct_input_buffers": calls, "eps": EPS, "layout": "qkv bf16 [B,N,3*H*d], out bf16 [B,N,H*d]",
             "l2": "inputs larger than L2 (%.0f MB per call vs 126 MB), no flush" % (B * N * 3 * H * D * 2 / 1e6)}
 
@@ -224,6 +268,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ffma-seconds", type=float, default=2.0,
+                    help="duration of the fp32 FMA peak measurement (0 skips it)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -260,7 +306,7 @@ def main():
         return _max_over_ranks(x, device=dev)
 
     lib = ll.lib()
-    B, N, H, calls, seed0 = WORKLOADS_BENCH[args.workload]
+    B, N, H, calls, seed0, T = WORKLOADS_BENCH[args.workload]
     qkv_bytes, out_bytes = B * N * 3 * H * D * 2, B * N * H * D * 2
     free, _ = torch.cuda.mem_get_info(dev)
     need = calls * (qkv_bytes + out_bytes) + (2 << 30)
@@ -274,7 +320,14 @@ def main():
     sh = ctypes.c_void_p(stream.cuda_stream)
     in_p = [t.data_ptr() for t in ins]
     out_p = [t.data_ptr() for t in outs]
-    fwd = lib.lite_la_fwd
+    if T:
+        def fwd(qkv, out, B, N, H, d, eps, stream):
+            return lib.lite_la_block_causal_fwd(qkv, out, B, N, H, d, eps, T, stream)
+
+        def fwd_events(qkv, out, B, N, H, d, eps, stream, evs):
+            return lib.lite_la_block_causal_fwd_events(qkv, out, B, N, H, d, eps, T, stream, evs)
+    else:
+        fwd, fwd_events = lib.lite_la_fwd, lib.lite_la_fwd_events
 
     def step():
         for i in range(calls):
@@ -318,13 +371,13 @@ def main():
             e.record(stream)
     torch.cuda.synchronize(dev)
     ev_handles = [(ctypes.c_void_p * 3)(*[ctypes.c_void_p(e.cuda_event) for e in trip]) for trip in evs]
-    nk = int(lib.lite_la_kernels_per_call(B, N, H, D, 0))
+    nk = int(lib.lite_la_kernels_per_call(B, N, H, D, T))
     phases = PATHS[nk]["phases"]
     kern_ms = {k: 0.0 for k in phases}
     nlaunch = 0
     for _ in range(args.steps):
         for i in range(calls):
-            s = lib.lite_la_fwd_events(in_p[i], out_p[i], B, N, H, D, EPS, sh, ev_handles[i])
+            s = fwd_events(in_p[i], out_p[i], B, N, H, D, EPS, sh, ev_handles[i])
             if s != 0:
                 raise ll.LiteLAError(s, lib.lite_la_last_error().decode())
         torch.cuda.synchronize(dev)
@@ -336,12 +389,18 @@ def main():
                 kern_ms[phases[1]] += trip[1].elapsed_time(trip[2])
         nlaunch += calls
     kern_us = {k: 1e3 * v / nlaunch for k, v in kern_ms.items()}
+    kern_us_isolated = dict(kern_us)
+    if nk == 1:
+        # one kernel per call: its average launch duration over the timed region is the period
+        # of the back-to-back calls (launches overlap only through programmatic dependent launch:
+        # a kernel's set-up runs while its predecessor drains, its memory traffic after it)
+        kern_us = {phases[0]: us_call}
     E = B * N * H * D
     flops_per_call = 4 * B * H * N * D * (D + 1)
     alg_bytes = {k: PATHS[nk]["alg_bytes_E"][k] * E for k in phases}
     peaks = load_peaks()
     dom = max(kern_us, key=kern_us.get)
-    traffic = load_traffic(dom)
+    traffic = load_traffic(dom, B, N, H, T)
     achieved = alg_bytes[dom] / (kern_us[dom] * 1e-6) / 1e9
     peak, unit = peaks["hbm_gbs"], "GB/s"
     peak_note = "%s copy bandwidth" % peaks["_source"]
@@ -349,9 +408,12 @@ def main():
                 "traffic": traffic, "kernel": dom, "kernel_us": kern_us[dom],
                 "alg_bytes_per_launch": alg_bytes[dom],
                 "alg_flops_per_launch": flops_per_call * alg_bytes[dom] // (8 * E),
-                "peak_source": peak_note, "kernel_us_all": kern_us,
-                "timing": "CUDA events on the launching stream around each phase (lite_la_fwd_events; "
-                          "no programmatic overlap with the neighbouring kernels)"}
+                "peak_source": peak_note, "kernel_us_all": kern_us, "kernel_us_isolated": kern_us_isolated,
+                "timing": ("average launch duration over the timed region: CUDA events around the back-to-back "
+                           "calls on the launching stream, / launches" if nk == 1 else
+                           "CUDA events on the launching stream around each phase (phase-timed entry points; "
+                           "no programmatic overlap with the neighbouring kernels)")
+                          + "; kernel_us_isolated: each call alone between events"}
     # the call as a whole against the slower of the HBM and fp32-FMA bounds
     t_hbm = 8 * E / (peaks["hbm_gbs"] * 1e9) * 1e6
     t_fma = 4 * B * H * N * D * (D + 1) / (fp32_fma_peak_tflops(peaks.get("sm_max_mhz", 1965.0)) * 1e12) * 1e6
@@ -361,6 +423,12 @@ def main():
         t_fma_clk = t_fma * peaks.get("sm_max_mhz", 1965.0) / clocks["sm_mhz"]
         call_roof["t_fma_us_at_measured_clock"] = t_fma_clk
         call_roof["frac_at_measured_clock"] = max(t_hbm, t_fma_clk) / us_call
+    if args.ffma_seconds > 0:
+        ffma = measure_ffma_peak(ll, dev, stream, args.ffma_seconds)
+        t_fma_meas = 4 * B * H * N * D * (D + 1) / (ffma["tflops"] * 1e12) * 1e6
+        call_roof["ffma_peak_measured"] = ffma
+        call_roof["t_fma_us_measured_peak"] = t_fma_meas
+        call_roof["frac_vs_measured_fma_peak"] = max(t_hbm, t_fma_meas) / us_call
 
     # end to end: pinned host input -> device, forward, device -> pinned host output, per call.
     # The copies run on their own streams so that the next call's upload and the previous
@@ -411,7 +479,7 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         bits = to_bits(ins[0])
-        rate, heads, el = oracle_head_rate(bits, B, N, H, args.cpu_seconds)
+        rate, heads, el = oracle_head_rate(bits, B, N, H, T, args.cpu_seconds)
         cpu = {"value": rate, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": "%d whole (batch, head) pairs of input buffer 0 (all %d queries x %d keys each), %.1f s"
                          % (heads, N, N, el)}
@@ -436,18 +504,23 @@ def main():
     return 0
 
 
-def load_traffic(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, or None when there is
-    none or the kernel sources changed since it was taken."""
+def load_traffic(kernel, B, N, H, T):
+    """DRAM bytes per launch of `kernel` (a phase name may join several kernels with '+') on a
+    call of this shape, from the committed ncu summaries; None when there is none or the kernel
+    sources changed since it was taken."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
-    ent = d.get(kernel)
-    if not ent or ent.get("sources_sha256") != sources_hash():
-        return None
-    return ent.get("dram_bytes_per_launch")
+    h = sources_hash()
+    total = 0
+    for k in kernel.split("+"):
+        ent = [e for e in d.get("entries", []) if e["kernel"] == k and [e["B"], e["N"], e["H"], e["T"]] == [B, N, H, T]]
+        if not ent or ent[0].get("sources_sha256") != h:
+            return None
+        total += ent[0]["dram_bytes_per_launch"]
+    return total
 
 
 def sources_hash():

@@ -114,6 +114,14 @@ litela_status lite_la_state_fwd(const void* qkv, float* states, int B, int N, in
 litela_status lite_la_fwd_events(const void* qkv, void* out, int B, int N, int H, int d, float eps,
                                  cudaStream_t stream, cudaEvent_t* events);
 
+/* lite_la_block_causal_fwd with the phase timing of lite_la_fwd_events: events[0] before the
+ * reduction, events[1] after the prefix scan, events[2] after the apply (tokens_per_block >= N
+ * is the non-causal call and takes its path).  Arguments are validated as for
+ * lite_la_block_causal_fwd. */
+litela_status lite_la_block_causal_fwd_events(const void* qkv, void* out, int B, int N, int H, int d,
+                                              float eps, int tokens_per_block, cudaStream_t stream,
+                                              cudaEvent_t* events);
+
 /* Synchronises `stream`, then reads and clears the error word that this library's kernels on
  * the current device set when one of their bounded waits timed out (each wait inside the
  * kernels gives up after about 1.5 s, records a code, frees its tensor memory and returns, so

@@ -39,6 +39,8 @@ _SIGNATURES = {
     "lite_la_fwd_f32out": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp]),
     "lite_la_block_causal_fwd_f32out": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
     "lite_la_fwd_events": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp, _vp]),
+    "lite_la_block_causal_fwd_events": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int,
+                                                 _vp, _vp]),
     "lite_la_block_causal_fwd_carry": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp, _vp, _vp]),
     "lite_la_block_causal_fwd_carry_f32out": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp, _vp, _vp]),
     "lite_la_device_status": (_c_int, [_vp]),
@@ -77,6 +79,27 @@ def lib() -> ctypes.CDLL:
                 fn.restype, fn.argtypes = res, args
             _lib = h
     return _lib
+
+
+ffma_lib_path = os.path.join(_PKG_DIR, "liblitela_ffma_peak.so")
+_ffma_lib = None
+
+
+def ffma_peak_lib() -> ctypes.CDLL:
+    """The benchmark's fp32 FMA-peak microbenchmark (include/litela_ffma_peak.h)."""
+    global _ffma_lib
+    with _lock:
+        if _ffma_lib is None:
+            if not os.path.exists(ffma_lib_path):
+                raise ImportError("liblitela_ffma_peak.so is not built; run "
+                                  "`python -m linear_attention_diffusion_litela_b200.build`")
+            h = ctypes.CDLL(ffma_lib_path)
+            h.litela_ffma_flops.restype = ctypes.c_longlong
+            h.litela_ffma_flops.argtypes = [_c_int, _c_int, ctypes.c_longlong]
+            h.litela_ffma_launch.restype = _c_int
+            h.litela_ffma_launch.argtypes = [_vp, _c_int, _c_int, ctypes.c_longlong, _vp]
+            _ffma_lib = h
+    return _ffma_lib
 
 
 def _check(status: int) -> None:

@@ -516,6 +516,13 @@ litela_status lite_la_fwd_events(const void* qkv, void* out, int B, int N, int H
   return litela::run(qkv, static_cast<__nv_bfloat16*>(out), B, N, H, d, eps, 0, false, stream, events);
 }
 
+litela_status lite_la_block_causal_fwd_events(const void* qkv, void* out, int B, int N, int H, int d, float eps,
+                                              int tokens_per_block, cudaStream_t stream, cudaEvent_t* events) {
+  if (events == nullptr || !events[0] || !events[1] || !events[2])
+    return litela::fail(LITELA_ERR_INVALID_ARGUMENT, "events must point to 3 CUDA events");
+  return litela::run(qkv, static_cast<__nv_bfloat16*>(out), B, N, H, d, eps, tokens_per_block, true, stream, events);
+}
+
 litela_status lite_la_state_fwd(const void* qkv, float* states, int B, int N, int H, int d,
                                 int tokens_per_block, cudaStream_t stream) {
   return litela::run_states(qkv, states, B, N, H, d, tokens_per_block, stream);

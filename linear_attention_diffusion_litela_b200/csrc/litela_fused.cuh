@@ -51,8 +51,10 @@ struct FusedCfg {
   static constexpr uint32_t kPhase2Bytes = A::kQStages * A::kQStageBytes + A::kOutSlots * A::kOutSlotBytes + kApSbufBytes;
   static constexpr uint32_t kBodyBytes = kPhase1Bytes > kPhase2Bytes ? kPhase1Bytes : kPhase2Bytes;
   static constexpr uint32_t kSmemBytes = kBodyBytes + 512 + 1024;
-  // merge batches are bulk-copied into the (still idle) output staging region
-  static constexpr int kMergeBatch = (int)(A::kOutSlots * A::kOutSlotBytes / (kRedHeads * kStateFloats * 4));
+  // merge batches are bulk-copied into the last q stage and the output staging region, which
+  // are contiguous and idle until the state is ready (the last stage's first q load waits)
+  static constexpr uint32_t kMergeBufBytes = A::kQStageBytes + A::kOutSlots * A::kOutSlotBytes;
+  static constexpr int kMergeBatch = (int)(kMergeBufBytes / (kRedHeads * kStateFloats * 4));
 };
 
 template <typename OutT>
@@ -75,6 +77,7 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
   uint8_t* qst = smem;
   uint8_t* obuf = qst + kQStages * A::kQStageBytes;
   uint8_t* sbuf = obuf + A::kOutSlots * A::kOutSlotBytes;
+  uint8_t* mbuf = qst + (kQStages - 1) * A::kQStageBytes;   // merge buffer: last q stage + staging
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBodyBytes);
   uint64_t* full = bars;                        // phase 1
   uint64_t* relu_done = full + kFuStages1;
@@ -255,6 +258,8 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
         if (lu >= kQStages &&
             !mbar_wait(&qempty[s], ((lu / kQStages) - 1) & 1, abort_flag, err, kErrApplyProducer | s))
           break;
+        // the last stage is the merge buffer until the state is ready
+        if (lu == kQStages - 1 && !mbar_wait(sfull, 0, abort_flag, err, kErrApplyProducer | 8)) break;
         const int np = pair_heads_h(p.H, q, 1) > 0 ? 2 : 1;
         mbar_arrive_expect_tx(&qfull[s], np * kQBoxBytes);
         for (int h = 0; h < np; ++h)
@@ -353,7 +358,7 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
       if (leader) {
         fence_proxy_async_global();
         mbar_arrive_expect_tx(merge_bar, nb * kPartBytes);
-        for (int i = 0; i < nb; ++i) bulk_load(obuf + i * kPartBytes, gsrc + (int64_t)(k0 + i) * kPartBytes, kPartBytes, merge_bar);
+        for (int i = 0; i < nb; ++i) bulk_load(mbuf + i * kPartBytes, gsrc + (int64_t)(k0 + i) * kPartBytes, kPartBytes, merge_bar);
       }
       const bool got = mbar_wait(merge_bar, batch & 1, abort_flag, err, kErrFusedMerge);
       if (bar_any(1, 128, !got)) {
@@ -366,7 +371,7 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
         if (u >= kUnits) break;
         const int hl = u / (kRows * 4), rcc = u - hl * (kRows * 4), rr = rcc >> 2, cc = rcc & 3;
         for (int i = 0; i < nb; ++i) {
-          const float4* src = reinterpret_cast<const float4*>(obuf + i * kPartBytes) + (hl * kStateFloats + rr * kD + cc * 8) / 4;
+          const float4* src = reinterpret_cast<const float4*>(mbuf + i * kPartBytes) + (hl * kStateFloats + rr * kD + cc * 8) / 4;
           const float4 x0 = src[0], x1 = src[1];
           sum[k][0] += x0.x; sum[k][1] += x0.y; sum[k][2] += x0.z; sum[k][3] += x0.w;
           sum[k][4] += x1.x; sum[k][5] += x1.y; sum[k][6] += x1.z; sum[k][7] += x1.w;
@@ -400,7 +405,7 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
     }
     bar_sync(2, 128);
     if (leader && ok) mbar_arrive(sfull);
-    // ---- epilogue (as litela_apply_tc; the merge buffer was the output staging region)
+    // ---- epilogue (as litela_apply_tc; the merge buffer overlapped the output staging region)
     const int hq = warp & 3;
     const int row = hq * 32 + lane;
     int nstaged = 0, pn = 0;

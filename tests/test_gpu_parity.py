@@ -337,3 +337,32 @@ def test_state_carry_without_state_in_is_the_plain_block_causal_call():
     full = ll.lite_la_state_fwd(qkv, H, 0)
     torch.cuda.synchronize()
     assert torch.allclose(st, full[:, :, 0], rtol=1e-6, atol=1e-5)
+
+
+@pytest.mark.parametrize("B,N,H,T", [(2, 3000, 9, 0), (2, 1000, 600, 0), (1, 4000, 7, 512), (2, 700, 5, 700)])
+def test_phase_timed_calls_give_the_plain_calls_result(B, N, H, T):
+    """lite_la_fwd_events / lite_la_block_causal_fwd_events run the same kernels with events
+    between the phases: bitwise the plain call's output, events complete and in order."""
+    lib = ll.lib()
+    qkv = make_qkv(B, N, H, 32, seed=9000 + N + H, device="cuda")
+    want = ll.lite_la_fwd(qkv, H, eps=EPS) if T == 0 else ll.lite_la_block_causal_fwd(qkv, H, T, eps=EPS)
+    out = torch.empty_like(want)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    stream = torch.cuda.current_stream()
+    for e in evs:
+        e.record(stream)
+    torch.cuda.synchronize()
+    handles = (ctypes.c_void_p * 3)(*[ctypes.c_void_p(e.cuda_event) for e in evs])
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    if T == 0:
+        s = lib.lite_la_fwd_events(qkv.data_ptr(), out.data_ptr(), B, N, H, 32, EPS, sh, handles)
+    else:
+        s = lib.lite_la_block_causal_fwd_events(qkv.data_ptr(), out.data_ptr(), B, N, H, 32, EPS, T, sh, handles)
+    assert s == 0, lib.lite_la_last_error().decode()
+    torch.cuda.synchronize()
+    ll.lite_la_device_status()
+    assert torch.equal(out, want)
+    assert evs[0].elapsed_time(evs[1]) >= 0.0 and evs[1].elapsed_time(evs[2]) >= 0.0
+    assert evs[0].elapsed_time(evs[2]) > 0.0
+    null = (ctypes.c_void_p * 3)(None, None, None)
+    assert lib.lite_la_fwd_events(qkv.data_ptr(), out.data_ptr(), B, N, H, 32, EPS, sh, null) == 1
