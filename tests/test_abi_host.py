@@ -112,3 +112,22 @@ def test_workspace_bytes(lib):
     # a causal block at least as long as N is the non-causal problem
     assert ll.lite_la_workspace_bytes(2, 500, 3, 32, 500) == ll.lite_la_workspace_bytes(2, 500, 3, 32, 0)
     assert ll.lite_la_workspace_bytes(2, 500, 3, 32, 10**6) == ll.lite_la_workspace_bytes(2, 500, 3, 32, 0)
+
+
+def test_ffma_peak_library_exports_its_header_and_counts_flops():
+    from linear_attention_diffusion_litela_b200.build import build
+    build()
+    text = open(os.path.join(ROOT, "include", "litela_ffma_peak.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = sorted(set(re.findall(r"\b(litela_ffma_\w+)\s*\(", text)))
+    assert names == ["litela_ffma_flops", "litela_ffma_launch"]
+    h = ll.ffma_peak_lib()
+    for n in names:
+        assert hasattr(h, n)
+    # 2 FLOPs per multiply-add, 8 chains x 16 unrolled rounds per iteration per thread
+    assert h.litela_ffma_flops(148, 512, 10) == 2 * 148 * 512 * 10 * 128
+    assert h.litela_ffma_flops(0, 512, 10) == 0
+    # invalid launch arguments are rejected before anything is launched
+    assert h.litela_ffma_launch(None, 1, 32, 1, None) == 1
+    assert h.litela_ffma_launch(ctypes.c_void_p(1 << 20), 1, 48, 1, None) == 1
+    assert h.litela_ffma_launch(ctypes.c_void_p(1 << 20), 1, 1024, 1, None) == 1
