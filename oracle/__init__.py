@@ -9,3 +9,8 @@ from .litela_oracle import (  # noqa: F401
     lite_la_block_causal_fwd,
     visible_key_count,
 )
+from .litela_bwd_oracle import (  # noqa: F401
+    lite_la_bwd_head,
+    lite_la_bwd,
+    lite_la_block_causal_bwd,
+)

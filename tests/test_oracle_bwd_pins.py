@@ -1,0 +1,173 @@
+"""Pins for the fp64 backward oracle (oracle/litela_bwd_oracle.py), independent of its own
+formulas: central finite differences of the pinned forward oracle, PyTorch autograd of the
+quadratic form, closed-form identities that follow from the forward's homogeneity and
+linearity, the ReLU masks, and the block-causal special cases.  CPU only."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_diffusion_litela_b200.inputs import to_bits
+
+def bits_of(a):
+    """bf16 bit patterns of a float32 array (round to nearest even)."""
+    return to_bits(torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16))
+
+
+D = 32
+
+
+def away_from_kinks(rng, shape, lo=0.05):
+    """Gaussian values with |x| >= lo, so relu is differentiable within a small step."""
+    x = rng.standard_normal(shape)
+    return np.where(np.abs(x) < lo, np.sign(x + 1e-300) * lo, x)
+
+
+def loss(q, k, v, g, eps, T):
+    N = q.shape[0]
+    nv = None if T is None else oracle.visible_key_count(np.arange(N), N, T)
+    return float((oracle.lite_la_rows(q, k, v, eps, nv) * g).sum())
+
+
+def finite_difference(q, k, v, g, eps, T, h=1e-6):
+    grads = []
+    for which in range(3):
+        x = [q.copy(), k.copy(), v.copy()]
+        out = np.zeros_like(x[which])
+        for idx in np.ndindex(*out.shape):
+            xp = [a.copy() for a in x]
+            xm = [a.copy() for a in x]
+            xp[which][idx] += h
+            xm[which][idx] -= h
+            out[idx] = (loss(*xp, g, eps, T) - loss(*xm, g, eps, T)) / (2 * h)
+        grads.append(out)
+    return grads
+
+
+@pytest.mark.parametrize("N,T,eps", [(1, None, 1e-15), (5, None, 1e-15), (6, None, 0.3), (7, 2, 1e-15),
+                                     (6, 1, 0.2), (5, 3, 1e-15)])
+def test_matches_central_finite_differences_of_the_forward_oracle(N, T, eps):
+    rng = np.random.default_rng(100 + N + (T or 0))
+    q, k, v, g = (away_from_kinks(rng, (N, D)) for _ in range(4))
+    dq, dk, dv = oracle.lite_la_bwd_head(q, k, v, g, eps, T)
+    fq, fk, fv = finite_difference(q, k, v, g, eps, T)
+    # relative to the gradient's overall size: a tensor whose true gradient is eps-small (the
+    # queries and keys when N = 1) is checked to be that small
+    scale = max(np.abs(f).max() for f in (fq, fk, fv))
+    for got, want in ((dq, fq), (dk, fk), (dv, fv)):
+        assert np.abs(got - want).max() <= 1e-6 * scale
+
+
+@pytest.mark.parametrize("T", [None, 3])
+def test_matches_torch_autograd_of_the_quadratic_form(T):
+    rng = np.random.default_rng(7)
+    N, eps = 11, 1e-3
+    q, k, v, g = (rng.standard_normal((N, D)) for _ in range(4))
+    tq, tk, tv = (torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (q, k, v))
+    w = torch.relu(tq) @ torch.relu(tk).T
+    if T is not None:
+        i = torch.arange(N)[:, None]
+        j = torch.arange(N)[None, :]
+        w = torch.where(j // T <= i // T, w, torch.zeros_like(w))
+    out = (w @ tv) / (w.sum(1, keepdim=True) + eps)
+    (out * torch.tensor(g)).sum().backward()
+    dq, dk, dv = oracle.lite_la_bwd_head(q, k, v, g, eps, T)
+    np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=1e-11, atol=1e-12)
+
+
+def forward_parts(q, k, v, eps, T=None):
+    """num_i and den_i (eps included) of the quadratic form, for the identities below."""
+    N = q.shape[0]
+    w = np.maximum(q, 0) @ np.maximum(k, 0).T
+    if T is not None:
+        w = np.where(np.arange(N)[None, :] // T <= np.arange(N)[:, None] // T, w, 0.0)
+    return w @ v, w.sum(1) + eps
+
+
+@pytest.mark.parametrize("T", [None, 4])
+def test_homogeneity_and_linearity_identities(T):
+    """out is unchanged (up to eps) by scaling one query or all keys, affine in V:
+      q_i . dq_i          = eps * (dout_i . num_i) / den_i^2
+      sum_j k_j . dk_j    = eps * sum_i (dout_i . num_i) / den_i^2
+      sum_j dv_j          = sum_i dout_i * (den_i - eps) / den_i
+      sum_j v_j . dv_j    = sum_i dout_i . out_i
+    With a large eps every one of them is far from 0 and tests its eps term."""
+    rng = np.random.default_rng(11)
+    N, eps = 20, 0.7
+    q, k, v, g = (rng.standard_normal((N, D)) for _ in range(4))
+    dq, dk, dv = oracle.lite_la_bwd_head(q, k, v, g, eps, T)
+    num, den = forward_parts(q, k, v, eps, T)
+    e = eps * (g * num).sum(1) / den ** 2
+    np.testing.assert_allclose((q * dq).sum(1), e, rtol=1e-10, atol=1e-13)
+    np.testing.assert_allclose((k * dk).sum(), e.sum(), rtol=1e-10)
+    np.testing.assert_allclose(dv.sum(0), (g * ((den - eps) / den)[:, None]).sum(0), rtol=1e-10, atol=1e-13)
+    np.testing.assert_allclose((v * dv).sum(), (g * num / den[:, None]).sum(), rtol=1e-10)
+
+
+def test_relu_masks_and_a_query_that_sees_nothing():
+    rng = np.random.default_rng(12)
+    N = 9
+    q, k, v, g = (rng.standard_normal((N, D)) for _ in range(4))
+    q[4] = -np.abs(q[4])                       # relu(q_4) = 0: out_4 = 0 whatever the keys
+    dq, dk, dv = oracle.lite_la_bwd_head(q, k, v, g, 1e-15)
+    assert np.all(dq[q <= 0] == 0.0) and np.all(dk[k <= 0] == 0.0)
+    assert np.all(dq[4] == 0.0)
+    g2 = g.copy()
+    g2[4] = 100.0 * rng.standard_normal(D)      # that row's incoming gradient reaches nothing
+    dq2, dk2, dv2 = oracle.lite_la_bwd_head(q, k, v, g2, 1e-15)
+    np.testing.assert_allclose(dk2, dk, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(dv2, dv, rtol=1e-12, atol=1e-15)
+    np.testing.assert_array_equal(np.delete(dq2, 4, 0), np.delete(dq, 4, 0))
+
+
+def test_block_causal_special_cases():
+    rng = np.random.default_rng(13)
+    N, eps = 10, 1e-15
+    q, k, v, g = (rng.standard_normal((N, D)) for _ in range(4))
+    full = oracle.lite_la_bwd_head(q, k, v, g, eps)
+    for T in (N, N + 5):                       # one block: the non-causal gradient
+        for a, b in zip(oracle.lite_la_bwd_head(q, k, v, g, eps, T), full):
+            np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-15)
+    # token-causal (T = 1): the last key is seen by the last query only, so
+    # dv_{N-1} = w_{N-1,N-1} dout_{N-1} / den_{N-1}
+    dq, dk, dv = oracle.lite_la_bwd_head(q, k, v, g, eps, 1)
+    num, den = forward_parts(q, k, v, eps, 1)
+    w_last = np.maximum(q[-1], 0) @ np.maximum(k[-1], 0)
+    np.testing.assert_allclose(dv[-1], w_last * g[-1] / den[-1], rtol=1e-12, atol=1e-15)
+    # keys of the last block get gradient only from queries of the last block
+    T = 4
+    g_early = g.copy()
+    g_early[8:] = 0.0
+    _, dk_e, dv_e = oracle.lite_la_bwd_head(q, k, v, g_early, eps, T)
+    assert np.all(dk_e[8:] == 0.0) and np.all(dv_e[8:] == 0.0)
+
+
+def test_rows_select_the_full_result_and_packed_entry_points_agree():
+    rng = np.random.default_rng(14)
+    B, N, H = 2, 13, 3
+    qkv = rng.standard_normal((B, N, 3 * H * D)).astype(np.float32)
+    dout = rng.standard_normal((B, N, H * D)).astype(np.float32)
+    qb, gb = bits_of(qkv), bits_of(dout)
+    x = oracle.decode_bf16(qb)
+    q, k, v = oracle.unpack_qkv(x, H, D)
+    g = oracle.decode_bf16(gb).reshape(B, N, H, D)
+    rows = np.array([0, 5, 12])
+    for T in (None, 4):
+        if T is None:
+            dq, dk, dv = oracle.lite_la_bwd(qb, gb, B, N, H, D, 1e-15)
+            sq, sk, sv = oracle.lite_la_bwd(qb, gb, B, N, H, D, 1e-15, rows=rows, heads=[(1, 2)])
+        else:
+            dq, dk, dv = oracle.lite_la_block_causal_bwd(qb, gb, B, N, H, D, 1e-15, T)
+            sq, sk, sv = oracle.lite_la_block_causal_bwd(qb, gb, B, N, H, D, 1e-15, T, rows=rows, heads=[(1, 2)])
+        for b in range(B):
+            for h in range(H):
+                ref = oracle.lite_la_bwd_head(q[b, :, h], k[b, :, h], v[b, :, h], g[b, :, h], 1e-15, T)
+                for got, want in zip((dq, dk, dv), ref):
+                    np.testing.assert_array_equal(got[b, :, h], want)
+        for full, samp in ((dq, sq), (dk, sk), (dv, sv)):
+            np.testing.assert_allclose(samp[1, :, 2], full[1, rows, 2], rtol=1e-13, atol=1e-16)
+            assert np.isnan(samp[0]).all()
+    with pytest.raises(ValueError):
+        oracle.lite_la_block_causal_bwd(qb, gb, B, N, H, D, 1e-15, 0)
