@@ -135,6 +135,49 @@ litela_status lite_la_device_status(cudaStream_t stream);
  * context remain usable.  Nothing faults and nothing hangs. */
 litela_status lite_la_selftest_timeout(cudaStream_t stream);
 
+/* ---- backward -------------------------------------------------------------------------
+ *
+ * Gradients of L = sum over all outputs of dout * out with respect to q, k and v, for the
+ * forward of lite_la_fwd (non-causal) or lite_la_block_causal_fwd.  The pages print only the
+ * forward (Sana explainer, "What LiteLA actually computes"); Sana trains through it, and these
+ * are its derivatives by the chain rule, per (batch, head), with S the state a query uses
+ * (block-causal: the prefix state of its block), den = (S relu(q))[d] + eps, g = dout:
+ *     dq = relu'(q) * (S[0:d]^T g / den + h * S[d]),   h = -(g . out) / den
+ *     dS = sum over the queries that use S of [g / den ; h] relu(q)^T
+ *          (block-causal: block b's own state gets the sum of dS over blocks b .. last)
+ *     dk = relu'(k) * (dS[0:d]^T v + dS[d]),   dv = dS[0:d] relu(k)
+ * relu'(x) = 1 for x > 0, else 0.  eps is a constant; the ones row that pads v has no gradient.
+ *
+ * qkv  : the forward's input, bf16 [B, N, 3*H*d] (layout as above).
+ * dout : the incoming gradient, bf16 [B, N, H*d] (the layout of out).
+ * dqkv : the result, [B, N, 3*H*d] in qkv's layout (dq | dk | dv per token row); bf16 (round to
+ *        nearest even) for the plain entry points, fp32 for the *_f32out ones.  Every element is
+ *        written.
+ * All three are caller-owned device buffers, 16-byte aligned; dqkv must not overlap qkv or dout
+ * (LITELA_ERR_INVALID_ARGUMENT).  Other arguments, the workspace, streams, status codes and
+ * asynchrony as for the forward entry points.  The forward's output is not needed: the
+ * backward recomputes the state (minimal HBM traffic 18 bytes per (token, head, channel):
+ * k, v read for the state, q and dout read, k and v read again, dq, dk, dv written). */
+litela_status lite_la_bwd(const void* qkv, const void* dout, void* dqkv, int B, int N, int H, int d, float eps,
+                          cudaStream_t stream);
+litela_status lite_la_block_causal_bwd(const void* qkv, const void* dout, void* dqkv, int B, int N, int H, int d,
+                                       float eps, int tokens_per_block, cudaStream_t stream);
+litela_status lite_la_bwd_f32out(const void* qkv, const void* dout, float* dqkv, int B, int N, int H, int d,
+                                 float eps, cudaStream_t stream);
+litela_status lite_la_block_causal_bwd_f32out(const void* qkv, const void* dout, float* dqkv, int B, int N, int H,
+                                              int d, float eps, int tokens_per_block, cudaStream_t stream);
+
+/* The backward (bf16 dqkv) with phase timing: events[0] before its first kernel, events[1]
+ * after the state (reduction + scan), events[2] after the dq kernel, events[3] after the
+ * dk/dv kernels; tokens_per_block <= 0 is the non-causal call.  events: host array of 4
+ * caller-created CUDA events.  The kernels run without programmatic overlap. */
+litela_status lite_la_bwd_events(const void* qkv, const void* dout, void* dqkv, int B, int N, int H, int d,
+                                 float eps, int tokens_per_block, cudaStream_t stream, cudaEvent_t* events);
+
+/* Size in bytes of the workspace a backward call with these arguments needs (tokens_per_block
+ * <= 0 means non-causal; a 148-SM device).  0 for invalid arguments or an empty problem. */
+size_t lite_la_bwd_workspace_bytes(int B, int N, int H, int d, int tokens_per_block);
+
 /* Static description of a status code (never NULL). */
 const char* lite_la_status_string(litela_status status);
 

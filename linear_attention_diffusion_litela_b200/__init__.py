@@ -15,7 +15,7 @@ import os
 import threading
 
 __all__ = [
-    "LiteLAError", "lib", "lib_path", "lite_la_fwd", "lite_la_block_causal_fwd",
+    "LiteLAError", "lib", "lib_path", "lite_la_fwd", "lite_la_block_causal_fwd", "lite_la_bwd",
     "lite_la_workspace_bytes", "lite_la_release_workspace", "STATUS", "EXPORTED_SYMBOLS",
 ]
 
@@ -52,6 +52,13 @@ _SIGNATURES = {
     "lite_la_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "lite_la_fwd_noalloc": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp]),
     "lite_la_kernels_per_call": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "lite_la_bwd": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp]),
+    "lite_la_block_causal_bwd": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
+    "lite_la_bwd_f32out": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp]),
+    "lite_la_block_causal_bwd_f32out": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int,
+                                                 _vp]),
+    "lite_la_bwd_events": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp, _vp]),
+    "lite_la_bwd_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
 }
 EXPORTED_SYMBOLS = tuple(_SIGNATURES)
 
@@ -201,6 +208,32 @@ def lite_la_state_fwd(qkv, H: int, tokens_per_block: int = 0, d: int = 32, out=N
         _check(lib().lite_la_state_fwd(qkv.data_ptr(), out.data_ptr(), B, N, H, d, int(tokens_per_block),
                                        _stream_handle(stream, qkv.device)))
     return out
+
+
+def lite_la_bwd(qkv, dout, H: int, tokens_per_block: int = 0, d: int = 32, eps: float = 1e-15, dqkv=None,
+                out_dtype=None, stream=None):
+    """Gradients (dq | dk | dv, in qkv's layout [B, N, 3*H*d]) of sum(dout * out) for the LiteLA
+    forward of qkv (block-causal when tokens_per_block > 0).  dout: bf16 [B, N, H*d]; the
+    result is bf16 unless dqkv/out_dtype say fp32."""
+    torch = _torch()
+    B, N, _ = _prepare(qkv, H, d, dout, torch.bfloat16)
+    if dout.dtype != torch.bfloat16:
+        raise TypeError("dout must be a contiguous bf16 tensor [B, N, H*d]")
+    if dqkv is None:
+        dqkv = torch.empty((B, N, 3 * H * d), dtype=out_dtype or torch.bfloat16, device=qkv.device)
+    if dqkv.dtype not in (torch.bfloat16, torch.float32) or not dqkv.is_contiguous() \
+            or tuple(dqkv.shape) != (B, N, 3 * H * d) or dqkv.device != qkv.device:
+        raise TypeError("dqkv must be a contiguous bf16/fp32 tensor [B, N, 3*H*d] on qkv's device")
+    f32 = dqkv.dtype == torch.float32
+    sh = _stream_handle(stream, qkv.device)
+    with torch.cuda.device(qkv.device):
+        if tokens_per_block > 0:
+            fn = lib().lite_la_block_causal_bwd_f32out if f32 else lib().lite_la_block_causal_bwd
+            _check(fn(qkv.data_ptr(), dout.data_ptr(), dqkv.data_ptr(), B, N, H, d, eps, int(tokens_per_block), sh))
+        else:
+            fn = lib().lite_la_bwd_f32out if f32 else lib().lite_la_bwd
+            _check(fn(qkv.data_ptr(), dout.data_ptr(), dqkv.data_ptr(), B, N, H, d, eps, sh))
+    return dqkv
 
 
 def lite_la_workspace_bytes(B: int, N: int, H: int, d: int = 32, tokens_per_block: int = 0) -> int:

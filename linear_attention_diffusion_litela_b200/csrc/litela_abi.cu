@@ -18,6 +18,7 @@
 
 #include "../../include/litela.h"
 #include "litela_plan.h"
+#include "litela_bwd.cuh"
 #include "litela_fused.cuh"
 #include "litela_tc.cuh"
 
@@ -74,7 +75,15 @@ litela_status device_setup(int* num_sms) {
         (e = cudaFuncSetAttribute(litela_fused_tc<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)FusedCfg<__nv_bfloat16>::kSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_fused_tc<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)FusedCfg<float>::kSmemBytes)) != cudaSuccess)
+                                  (int)FusedCfg<float>::kSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_bwd_q_tc<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kBqSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_bwd_q_tc<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kBqSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_bwd_kv_tc<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kBkSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_bwd_kv_tc<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kBkSmemBytes)) != cudaSuccess)
       return cuda_fail(e, "cudaFuncSetAttribute(dynamic shared memory)");
     if (g_encode == nullptr) {
       void* fn = nullptr;
@@ -148,13 +157,13 @@ bool alloc_fault_injected() {
   return v != nullptr && v[0] == '1';
 }
 
-litela_status get_workspace(const Plan& plan, cudaStream_t stream, Workspace** out, bool states_only = false) {
+// `need`: bytes of partial-state workspace the call uses (work_bytes(plan) for a forward call)
+litela_status get_workspace(const Plan& plan, cudaStream_t stream, Workspace** out, size_t need) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   std::lock_guard<std::mutex> lock(g_ws_mutex);
   Workspace& ws = g_ws[{dev, reinterpret_cast<uintptr_t>(stream)}];
-  const size_t need = states_only ? plan.bytes : work_bytes(plan);
   const size_t need_ctl = kCounterBase + plan.counters;
   if (ws.partials_bytes < need || ws.ctl_words < need_ctl) {
     if (alloc_fault_injected())
@@ -266,12 +275,15 @@ litela_status launch_reduce(const Plan& plan, const void* qkv, float* partials, 
 
 litela_status launch_scan(const Plan& plan, const float* partials, uint8_t* images, float* states, int num_sms,
                           cudaStream_t stream, bool pdl, const float* state_in = nullptr,
-                          float* state_out = nullptr) {
+                          float* state_out = nullptr, uint8_t* images_t = nullptr, bool reverse = false,
+                          int chunks_per_block = 0) {
   const int64_t work = ((int64_t)plan.B * plan.H * kStateFloats + kScanElems - 1) / kScanElems;
   int64_t grid = (work + kScanThreads - 1) / kScanThreads;
   if (grid > num_sms) grid = num_sms;
+  TcPlan tp = tc_plan(plan, 0.f);
+  if (chunks_per_block > 0) tp.cpb = chunks_per_block;   // partials of another chunking (the backward's)
   cudaError_t e = launch_ex(litela_state_scan, dim3((unsigned)grid), dim3(kScanThreads), 0, stream, pdl,
-                            partials, images, states, state_in, state_out, tc_plan(plan, 0.f));
+                            partials, images, images_t, states, state_in, state_out, reverse, tp);
   if (e != cudaSuccess) return cuda_fail(e, "launch litela_state_scan");
   return LITELA_OK;
 }
@@ -357,7 +369,7 @@ litela_status run_states(const void* qkv, float* states, int B, int N, int H, in
   const size_t qkv_bytes = (size_t)B * N * 3 * H * d * sizeof(__nv_bfloat16);
   if (overlaps(qkv, qkv_bytes, states, state_bytes)) return fail(LITELA_ERR_INVALID_ARGUMENT, "states overlaps qkv");
   Workspace* ws = nullptr;
-  s = get_workspace(plan, stream, &ws, true);
+  s = get_workspace(plan, stream, &ws, plan.bytes);
   if (s != LITELA_OK) return s;
   float* partials = static_cast<float*>(ws->partials);
   s = launch_reduce(plan, qkv, partials, ws->err, stream, true);
@@ -394,7 +406,7 @@ litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float 
       return fail(LITELA_ERR_INVALID_ARGUMENT, "a state buffer overlaps qkv or out");
   }
   Workspace* ws = nullptr;
-  s = get_workspace(plan, stream, &ws);
+  s = get_workspace(plan, stream, &ws, work_bytes(plan));
   if (s != LITELA_OK) return s;
   char* base = static_cast<char*>(ws->partials);
   if (carry)
@@ -408,6 +420,74 @@ litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float 
                ws->err, num_sms, stream, events);
   if (s == LITELA_OK) g_last_error.clear();
   return s;
+}
+
+// ---------------------------------------------------------------------------------------
+// backward
+
+// Five kernels: reduction and scan (S, S images, S^T images), dq + partial dS, reverse scan
+// (dS images), dk + dv.  Chained with programmatic dependent launch unless phase events are
+// requested: then events[0] precedes the reduction, events[1] follows the scan, events[2] the
+// dq kernel and events[3] the dk/dv kernel (after the reverse scan).
+template <typename OutT>
+litela_status run_bwd(const void* qkv, const void* dout, OutT* dqkv, int B, int N, int H, int d, float eps,
+                      int tokens_per_block, bool causal, cudaStream_t stream, cudaEvent_t* events = nullptr) {
+  bool empty = false;
+  // qkv and dout as the forward's qkv and out
+  litela_status s = validate(qkv, dout, sizeof(__nv_bfloat16), B, N, H, d, eps, tokens_per_block, causal, &empty);
+  if (s != LITELA_OK || empty) return s;
+  if (dqkv == nullptr) return fail(LITELA_ERR_INVALID_ARGUMENT, "null dqkv");
+  if (reinterpret_cast<uintptr_t>(dqkv) & 15u) return fail(LITELA_ERR_INVALID_ARGUMENT, "dqkv must be 16-byte aligned");
+  const size_t qkv_bytes = (size_t)B * N * 3 * H * d * sizeof(__nv_bfloat16);
+  const size_t dout_bytes = (size_t)B * N * H * d * sizeof(__nv_bfloat16);
+  const size_t dqkv_bytes = (size_t)B * N * 3 * H * d * sizeof(OutT);
+  if (overlaps(dqkv, dqkv_bytes, qkv, qkv_bytes) || overlaps(dqkv, dqkv_bytes, dout, dout_bytes))
+    return fail(LITELA_ERR_INVALID_ARGUMENT, "dqkv overlaps qkv or dout");
+  int num_sms = 0;
+  s = device_setup(&num_sms);
+  if (s != LITELA_OK) return s;
+  Plan plan;
+  make_plan(B, N, H, causal ? tokens_per_block : 0, num_sms, &plan);
+  make_bwd_plan(num_sms, &plan);
+  Workspace* ws = nullptr;
+  s = get_workspace(plan, stream, &ws, plan.bwd_bytes);
+  if (s != LITELA_OK) return s;
+  char* base = static_cast<char*>(ws->partials);
+  float* partials = reinterpret_cast<float*>(base);
+  uint8_t* images = reinterpret_cast<uint8_t*>(base + plan.off_images);
+  uint8_t* images_t = reinterpret_cast<uint8_t*>(base + plan.off_images_t);
+  float* dpartials = reinterpret_cast<float*>(base + plan.off_dpartials);
+  uint8_t* dimages = reinterpret_cast<uint8_t*>(base + plan.off_dimages);
+  uint8_t* dimages_t = reinterpret_cast<uint8_t*>(base + plan.off_dimages_t);
+  CUtensorMap map_qkv, map_g;
+  s = encode_qkv_map(qkv, B, N, H, kApTile, &map_qkv);
+  if (s != LITELA_OK) return s;
+  s = encode_out_map(static_cast<__nv_bfloat16*>(const_cast<void*>(dout)), B, N, H, &map_g);
+  if (s != LITELA_OK) return s;
+  const bool pdl = events == nullptr;
+  const BwdPlan bp{B, N, H, plan.T, plan.nblk, plan.nquads, plan.bwd_cpb, plan.bwd_chunk, eps};
+  const dim3 grid((unsigned)(plan.nblk * plan.bwd_cpb), (unsigned)plan.nquads, (unsigned)B);
+  cudaError_t e;
+  if (events && (e = cudaEventRecord(events[0], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  s = launch_reduce(plan, qkv, partials, ws->err, stream, pdl);
+  if (s != LITELA_OK) return s;
+  s = launch_scan(plan, partials, images, nullptr, num_sms, stream, pdl, nullptr, nullptr, images_t, false);
+  if (s != LITELA_OK) return s;
+  if (events && (e = cudaEventRecord(events[1], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  e = launch_ex(litela_bwd_q_tc<OutT>, grid, dim3(kBwThreads), kBqSmemBytes, stream, pdl, map_qkv, map_g,
+                static_cast<const uint8_t*>(images), static_cast<const uint8_t*>(images_t), dpartials, dqkv, ws->err,
+                bp);
+  if (e != cudaSuccess) return cuda_fail(e, "launch litela_bwd_q_tc");
+  if (events && (e = cudaEventRecord(events[2], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  s = launch_scan(plan, dpartials, dimages, nullptr, num_sms, stream, pdl, nullptr, nullptr, dimages_t, true,
+                  plan.bwd_cpb);
+  if (s != LITELA_OK) return s;
+  e = launch_ex(litela_bwd_kv_tc<OutT>, grid, dim3(kBwThreads), kBkSmemBytes, stream, pdl, map_qkv,
+                static_cast<const uint8_t*>(dimages), static_cast<const uint8_t*>(dimages_t), dqkv, ws->err, bp);
+  if (e != cudaSuccess) return cuda_fail(e, "launch litela_bwd_kv_tc");
+  if (events && (e = cudaEventRecord(events[3], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  g_last_error.clear();
+  return LITELA_OK;
 }
 
 // Fixed scratch of lite_la_fwd_noalloc: one array per device, defined statically so that the
@@ -533,6 +613,43 @@ litela_status lite_la_fwd_noalloc(const void* qkv, void* out, int B, int N, int 
   return litela::run_noalloc(qkv, static_cast<__nv_bfloat16*>(out), B, N, H, d, eps, stream);
 }
 
+litela_status lite_la_bwd(const void* qkv, const void* dout, void* dqkv, int B, int N, int H, int d, float eps,
+                          cudaStream_t stream) {
+  return litela::run_bwd(qkv, dout, static_cast<__nv_bfloat16*>(dqkv), B, N, H, d, eps, 0, false, stream);
+}
+
+litela_status lite_la_block_causal_bwd(const void* qkv, const void* dout, void* dqkv, int B, int N, int H, int d,
+                                       float eps, int tokens_per_block, cudaStream_t stream) {
+  return litela::run_bwd(qkv, dout, static_cast<__nv_bfloat16*>(dqkv), B, N, H, d, eps, tokens_per_block, true,
+                         stream);
+}
+
+litela_status lite_la_bwd_f32out(const void* qkv, const void* dout, float* dqkv, int B, int N, int H, int d,
+                                 float eps, cudaStream_t stream) {
+  return litela::run_bwd(qkv, dout, dqkv, B, N, H, d, eps, 0, false, stream);
+}
+
+litela_status lite_la_block_causal_bwd_f32out(const void* qkv, const void* dout, float* dqkv, int B, int N, int H,
+                                              int d, float eps, int tokens_per_block, cudaStream_t stream) {
+  return litela::run_bwd(qkv, dout, dqkv, B, N, H, d, eps, tokens_per_block, true, stream);
+}
+
+litela_status lite_la_bwd_events(const void* qkv, const void* dout, void* dqkv, int B, int N, int H, int d,
+                                 float eps, int tokens_per_block, cudaStream_t stream, cudaEvent_t* events) {
+  if (events == nullptr || !events[0] || !events[1] || !events[2] || !events[3])
+    return litela::fail(LITELA_ERR_INVALID_ARGUMENT, "events must point to 4 CUDA events");
+  return litela::run_bwd(qkv, dout, static_cast<__nv_bfloat16*>(dqkv), B, N, H, d, eps, tokens_per_block,
+                         tokens_per_block > 0, stream, events);
+}
+
+size_t lite_la_bwd_workspace_bytes(int B, int N, int H, int d, int tokens_per_block) {
+  if (B < 0 || N < 0 || H < 0 || d != litela::kD) return 0;
+  litela::Plan p;
+  if (!litela::make_plan(B, N, H, tokens_per_block, 148, &p)) return 0;
+  litela::make_bwd_plan(148, &p);
+  return p.bwd_bytes + (litela::kCounterBase + p.counters) * sizeof(int);
+}
+
 int lite_la_kernels_per_call(int B, int N, int H, int d, int tokens_per_block) {
   if (B <= 0 || N <= 0 || H <= 0 || d != litela::kD) return 0;
   int dev = 0, sms = 148;
@@ -549,7 +666,7 @@ litela_status lite_la_selftest_timeout(cudaStream_t stream) {
   litela::Plan plan;
   litela::make_plan(1, 1, 1, 0, 148, &plan);
   litela::Workspace* ws = nullptr;
-  litela_status s = litela::get_workspace(plan, stream, &ws);
+  litela_status s = litela::get_workspace(plan, stream, &ws, litela::work_bytes(plan));
   if (s != LITELA_OK) return s;
   litela::litela_selftest_timeout<<<1, 32, 0, stream>>>(ws->err);
   cudaError_t e = cudaGetLastError();

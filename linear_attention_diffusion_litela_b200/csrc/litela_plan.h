@@ -27,6 +27,10 @@ constexpr int kApTile = 128;
 constexpr int kImageRows = 80;
 constexpr int kImageLoRow = 40;
 constexpr int kImageBytes = kImageRows * kD * 2;
+// the transposed image of a state's first d rows (rows c: hi 0..31, lo 32..63; K = r, 32 wide),
+// the B operand of the backward's products with S[0:d]^T
+constexpr int kImageTRows = 2 * kD;
+constexpr int kImageTBytes = kImageTRows * kD * 2;
 // small zero-initialised control buffer: word 0 is the kernels' error word (a bounded wait that
 // timed out); the fused kernel's sibling counters start at word kCounterBase
 constexpr int kErrWords = 64;
@@ -52,6 +56,12 @@ struct Plan {
   bool fused = false;
   int fused_cpb = 0, fused_chunk = 0, fused_ntiles = 0;
   size_t fused_bytes = 0, counters = 0;
+  // backward (make_bwd_plan): the forward's reduction and scan (partials, images above), then
+  //   S^T images bf16 [B][H][nblk][kImageTBytes]                       at off_images_t
+  //   dS partials fp32 [B][nquads][nblk * bwd_cpb][4][33][32]           at off_dpartials
+  //   dS images [B][H][nblk][kImageBytes], dS^T images (kImageTBytes)   at off_dimages, off_dimages_t
+  int bwd_cpb = 0, bwd_chunk = 0;   // CTAs per (batch, quad, block); tokens per CTA (multiple of 128)
+  size_t off_images_t = 0, off_dpartials = 0, off_dimages = 0, off_dimages_t = 0, bwd_bytes = 0;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -98,6 +108,28 @@ inline bool make_plan(int B, int N, int H, int tokens_per_block, int num_sms, Pl
     p->counters = (size_t)2 * B * p->nquads;   // both sets
   }
   return true;
+}
+
+// Adds the backward's partition and workspace layout to a plan made by make_plan: one CTA per
+// (batch, head quad, block, chunk of the block), about one CTA per SM in total.
+inline void make_bwd_plan(int num_sms, Plan* p) {
+  const int sms = num_sms > 0 ? num_sms : 148;
+  const int64_t segs = (int64_t)p->B * p->nquads * p->nblk;
+  int64_t want = sms / segs;
+  if (want > p->tiles_per_block) want = p->tiles_per_block;
+  if (want < 1) want = 1;
+  int64_t chunk = (p->T + want - 1) / want;
+  chunk = (chunk + kApTile - 1) / kApTile * kApTile;
+  p->bwd_chunk = (int)chunk;
+  p->bwd_cpb = (int)((p->T + chunk - 1) / chunk);
+  const size_t img_t = (size_t)p->B * p->H * p->nblk * kImageTBytes;
+  const size_t img = (size_t)p->B * p->H * p->nblk * kImageBytes;
+  const size_t dpart = (size_t)segs * p->bwd_cpb * kRedHeads * kStateFloats * sizeof(float);
+  p->off_images_t = align_up(p->bytes, 256);
+  p->off_dpartials = p->off_images_t + align_up(img_t, 256);
+  p->off_dimages = p->off_dpartials + align_up(dpart, 256);
+  p->off_dimages_t = p->off_dimages + align_up(img, 256);
+  p->bwd_bytes = p->off_dimages_t + align_up(img_t, 256);
 }
 
 }  // namespace litela

@@ -132,10 +132,6 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
-  // the apply kernel (launched as a programmatic dependent) may start its prologue now; it
-  // waits for this grid to finish before it reads the partial states
-  pdl_launch_dependents();
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int x = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int blk = x / p.cpb, ch = x - blk * p.cpb;
@@ -168,6 +164,10 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
   // launched as a programmatic dependent of the previous kernel in the stream: everything
   // above is private set-up; qkv and the workspace are touched only after that kernel is done
   pdl_wait_primary();
+  // Only now may the next kernels launch.  This kernel opens a call, and the later kernels of
+  // the call read their inputs (q, the incoming gradient) before their own waits: releasing
+  // them after this wait means that whatever produced those inputs upstream has finished.
+  pdl_launch_dependents();
 
   const int kx = p.H * kD + g * (kRedHeads * kD);       // first key channel of the group
   const int vx = 2 * p.H * kD + g * (kRedHeads * kD);   // first value channel of the group
@@ -284,8 +284,11 @@ __device__ __forceinline__ const float* partial_ptr(const float* partials, const
 
 // litela_state_scan: partial states -> per-(batch, head, block) inclusive prefix states, summed in
 // fixed order (deterministic).  Writes each one as the apply's B-operand image (bf16 hi rows
-// 0..32, lo rows 40..72, zero rows in between and after; S = hi + lo to 2^-17 relative) and,
-// when `states` is not null, as fp32 [B][H][nblk][33][32].  `state_in` (fp32 [B][H][33][32], may be
+// 0..32, lo rows 40..72, zero rows in between and after; S = hi + lo to 2^-17 relative), when
+// `images_t` is not null also as the transposed image of its first 32 rows (rows c: hi 0..31,
+// lo 32..63, K = r; the B operand of products with S[0:32]^T), and, when `states` is not null,
+// as fp32 [B][H][nblk][33][32].  With `reverse` the blocks are visited last to first, giving
+// the inclusive SUFFIX sums over blocks (the gradient of a prefix-summed state).  `state_in` (fp32 [B][H][33][32], may be
 // null) is a state carried from earlier chunks of the sequence and starts every prefix;
 // `state_out` (may be null, may alias state_in) receives the final prefix.  Grid-stride over the state elements
 // with at most one small CTA per SM: its CTAs launch early as a programmatic dependent of the
@@ -296,8 +299,9 @@ constexpr int kScanZeros = 14 * kD;   // zero elements of one image
 constexpr int kScanElems = 2;         // state elements per thread and round
 
 __global__ void __launch_bounds__(kScanThreads)
-litela_state_scan(const float* __restrict__ partials, uint8_t* __restrict__ images, float* __restrict__ states,
-                  const float* __restrict__ state_in, float* __restrict__ state_out, TcPlan p) {
+litela_state_scan(const float* __restrict__ partials, uint8_t* __restrict__ images, uint8_t* __restrict__ images_t,
+                  float* __restrict__ states, const float* __restrict__ state_in, float* __restrict__ state_out,
+                  bool reverse, TcPlan p) {
   using namespace sm100;
   pdl_launch_dependents();
   const int64_t stride = (int64_t)gridDim.x * kScanThreads;
@@ -342,12 +346,16 @@ litela_state_scan(const float* __restrict__ partials, uint8_t* __restrict__ imag
 #pragma unroll
       for (int j = 0; j < kE; ++j)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[j][i] = (ok[j] && k0 + i < nparts) ? __ldcg(src[j] + (int64_t)(k0 + i) * pstride) : 0.f;
+        for (int i = 0; i < 8; ++i) {
+          const int k = reverse ? nparts - 1 - (k0 + i) : k0 + i;
+          v[j][i] = (ok[j] && k0 + i < nparts) ? __ldcg(src[j] + (int64_t)k * pstride) : 0.f;
+        }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int k = k0 + i;
-        if (k >= nparts) break;
-        const bool block_end = (k + 1) % p.cpb == 0;   // last chunk of block k / cpb
+        if (k0 + i >= nparts) break;
+        const int k = reverse ? nparts - 1 - (k0 + i) : k0 + i;
+        // last chunk of block k / cpb in visiting order
+        const bool block_end = reverse ? (k % p.cpb == 0) : ((k + 1) % p.cpb == 0);
         const int blk = k / p.cpb;
 #pragma unroll
         for (int j = 0; j < kE; ++j) {
@@ -362,6 +370,11 @@ litela_state_scan(const float* __restrict__ partials, uint8_t* __restrict__ imag
               const __nv_bfloat16 lo = __float2bfloat16_rn(run[j] - __bfloat162float(hi));
               *reinterpret_cast<__nv_bfloat16*>(img + image_offset(r, c)) = hi;
               *reinterpret_cast<__nv_bfloat16*>(img + image_offset(kImageLoRow + r, c)) = lo;
+              if (images_t != nullptr && r < kD) {
+                uint8_t* imt = images_t + (bh[j] * p.nblk + blk) * kImageTBytes;
+                *reinterpret_cast<__nv_bfloat16*>(imt + image_offset(c, r)) = hi;
+                *reinterpret_cast<__nv_bfloat16*>(imt + image_offset(kD + c, r)) = lo;
+              }
             }
             if (states != nullptr) states[(bh[j] * p.nblk + blk) * kStateFloats + e[j]] = run[j];
           }

@@ -28,6 +28,18 @@ what the CUDA path takes.  Readings (also listed in the design doc): relu'(x) = 1 for
 otherwise (0 at x = 0, as PyTorch's ReLU backward); eps is a constant; the ones row that pads
 v is a constant and gets no gradient.
 
+Error magnitudes (magnitudes=True).  A gradient element is a sum of terms of both signs and
+may cancel to far below the size of its terms (for N = 1, dq is exactly eps-small), so a
+floating-point evaluation of it errs in proportion to its terms, not to itself.  With
+magnitudes=True each function also returns, per element, the same sums taken over absolute
+values, with |dL/dden_i| replaced by the bound sum_r |dout_ir| (sum_j w_ij |v_jr|) / den_i^2 of
+its own terms:
+    M(dq_i) = sum_j (|dL/dnum_i| . |v_j| + B_i) relu(k_j)
+    M(dk_j) = sum_i (|dL/dnum_i| . |v_j| + B_i) relu(q_i)
+    M(dv_j) = sum_i w_ij |dL/dnum_i|
+These bound what any route that reassociates the sums (such as the state route) adds up, so
+a computed gradient is compared with tolerance rtol * |g| + atol * M.
+
 Parity status: lite_la_bwd_head, lite_la_bwd and lite_la_block_causal_bwd are pinned by
 tests/test_oracle_bwd_pins.py (central finite differences of the pinned forward oracle,
 PyTorch autograd of the quadratic form, closed-form identities from homogeneity and
@@ -51,12 +63,14 @@ def _weights(pq_rows, pk, n_visible):
 
 
 def lite_la_bwd_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, dout: np.ndarray, eps: float,
-                     tokens_per_block: int | None = None, rows=None, chunk: int = 1024):
+                     tokens_per_block: int | None = None, rows=None, chunk: int = 1024,
+                     magnitudes: bool = False):
     """Gradients of L = sum(dout * out) for ONE (batch, head).
 
     q, k, v, dout: [N, d] float64 (raw q and k; relu is applied here).  rows: token indices
     whose gradients are returned (None = all N); every query contributes to dk and dv.
-    Returns (dq, dk, dv), each [len(rows), d] float64.
+    Returns (dq, dk, dv), each [len(rows), d] float64, followed by their error magnitudes
+    (mq, mk, mv) when `magnitudes` is set.
     """
     N, d = q.shape
     T = None if tokens_per_block is None else int(tokens_per_block)
@@ -64,8 +78,10 @@ def lite_la_bwd_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, dout: np.ndarr
     pq, pk = relu(q), relu(k)
     v_rows = v[rows]
 
+    av = np.abs(v)
     # dq for the selected queries: sum over the keys each one sees
     dq = np.zeros((rows.size, d))
+    mq = np.zeros((rows.size, d))
     for s in range(0, rows.size, chunk):
         r = rows[s:s + chunk]
         nv = None if T is None else visible_key_count(r, N, T)
@@ -78,10 +94,19 @@ def lite_la_bwd_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, dout: np.ndarr
         if mask is not None:
             dw = np.where(mask, dw, 0.0)
         dq[s:s + chunk] = (dw @ pk) * (q[r] > 0)
+        if magnitudes:
+            bnd = (np.abs(dout[r]) * (w @ av)).sum(axis=1) / den ** 2
+            aw = np.abs(dnum) @ av.T + bnd[:, None]
+            if mask is not None:
+                aw = np.where(mask, aw, 0.0)
+            mq[s:s + chunk] = aw @ pk
 
     # dk and dv for the selected keys: sum over every query that sees them
     dkt = np.zeros((rows.size, d))
     dv = np.zeros((rows.size, d))
+    mk = np.zeros((rows.size, d))
+    mv = np.zeros((rows.size, d))
+    av_rows = av[rows]
     for s in range(0, N, chunk):
         i = np.arange(s, min(s + chunk, N), dtype=np.int64)
         nv = None if T is None else visible_key_count(i, N, T)
@@ -96,38 +121,49 @@ def lite_la_bwd_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, dout: np.ndarr
             dw_sel = np.where(mask[:, rows], dw_sel, 0.0)
         dv += w_sel.T @ dnum
         dkt += dw_sel.T @ pq[i]
+        if magnitudes:
+            bnd = (np.abs(dout[i]) * (w @ av)).sum(axis=1) / den ** 2
+            aw_sel = np.abs(dnum) @ av_rows.T + bnd[:, None]
+            if mask is not None:
+                aw_sel = np.where(mask[:, rows], aw_sel, 0.0)
+            mv += w_sel.T @ np.abs(dnum)
+            mk += aw_sel.T @ pq[i]
     dk = dkt * (k[rows] > 0)
+    if magnitudes:
+        return dq, dk, dv, mq, mk, mv
     return dq, dk, dv
 
 
-def _backward(qkv_bits, dout_bits, B, N, H, d, eps, tokens_per_block, rows, heads, chunk):
+def _backward(qkv_bits, dout_bits, B, N, H, d, eps, tokens_per_block, rows, heads, chunk, magnitudes=False):
     x = decode_bf16(np.asarray(qkv_bits).reshape(B, N, 3 * H * d))
     g = decode_bf16(np.asarray(dout_bits).reshape(B, N, H, d))
     q, k, v = unpack_qkv(x, H, d)
     rows = np.arange(N, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
     heads = [(b, h) for b in range(B) for h in range(H)] if heads is None else list(heads)
-    dq = np.full((B, rows.size, H, d), np.nan)
-    dk = np.full_like(dq, np.nan)
-    dv = np.full_like(dq, np.nan)
+    res = [np.full((B, rows.size, H, d), np.nan) for _ in range(6 if magnitudes else 3)]
     for (b, h) in heads:
-        gq, gk, gv = lite_la_bwd_head(np.ascontiguousarray(q[b, :, h]), np.ascontiguousarray(k[b, :, h]),
-                                      np.ascontiguousarray(v[b, :, h]), np.ascontiguousarray(g[b, :, h]),
-                                      eps, tokens_per_block, rows, chunk)
-        dq[b, :, h], dk[b, :, h], dv[b, :, h] = gq, gk, gv
-    return dq, dk, dv
+        got = lite_la_bwd_head(np.ascontiguousarray(q[b, :, h]), np.ascontiguousarray(k[b, :, h]),
+                               np.ascontiguousarray(v[b, :, h]), np.ascontiguousarray(g[b, :, h]),
+                               eps, tokens_per_block, rows, chunk, magnitudes)
+        for dst, src in zip(res, got):
+            dst[b, :, h] = src
+    return tuple(res)
 
 
 def lite_la_bwd(qkv_bits, dout_bits, B: int, N: int, H: int, d: int, eps: float,
-                rows=None, heads=None, chunk: int = 1024):
+                rows=None, heads=None, chunk: int = 1024, magnitudes: bool = False):
     """Non-causal LiteLA backward on packed bf16 qkv bits [B, N, 3*H*d] and bf16 dout bits
-    [B, N, H*d].  Returns float64 (dq, dk, dv), each [B, len(rows), H, d]; rows selects token
-    indices (None = all), heads a list of (b, h) to evaluate (None = all; the others are NaN)."""
-    return _backward(qkv_bits, dout_bits, B, N, H, d, eps, None, rows, heads, chunk)
+    [B, N, H*d].  Returns float64 (dq, dk, dv), each [B, len(rows), H, d] (then their error
+    magnitudes when `magnitudes` is set); rows selects token indices (None = all), heads a list
+    of (b, h) to evaluate (None = all; the others are NaN)."""
+    return _backward(qkv_bits, dout_bits, B, N, H, d, eps, None, rows, heads, chunk, magnitudes)
 
 
 def lite_la_block_causal_bwd(qkv_bits, dout_bits, B: int, N: int, H: int, d: int, eps: float,
-                             tokens_per_block: int, rows=None, heads=None, chunk: int = 1024):
+                             tokens_per_block: int, rows=None, heads=None, chunk: int = 1024,
+                             magnitudes: bool = False):
     """Block-causal LiteLA backward: query i sees the keys of blocks 0..floor(i/T)."""
     if int(tokens_per_block) <= 0:
         raise ValueError("tokens_per_block must be positive")
-    return _backward(qkv_bits, dout_bits, B, N, H, d, eps, int(tokens_per_block), rows, heads, chunk)
+    return _backward(qkv_bits, dout_bits, B, N, H, d, eps, int(tokens_per_block), rows, heads, chunk,
+                     magnitudes)

@@ -131,3 +131,37 @@ def test_ffma_peak_library_exports_its_header_and_counts_flops():
     assert h.litela_ffma_launch(None, 1, 32, 1, None) == 1
     assert h.litela_ffma_launch(ctypes.c_void_p(1 << 20), 1, 48, 1, None) == 1
     assert h.litela_ffma_launch(ctypes.c_void_p(1 << 20), 1, 1024, 1, None) == 1
+
+
+def test_backward_arguments_are_validated_on_the_host(lib):
+    a, g, o = ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 24), ctypes.c_void_p(1 << 30)
+    # qkv is 4 tokens x 96 channels x 2 bytes = 768 bytes, dout 256 bytes
+    for B, N, H, d, eps, want in BAD_ARGS:
+        assert lib.lite_la_bwd(a, g, o, B, N, H, d, eps, None) == want
+        assert lib.lite_la_bwd_f32out(a, g, o, B, N, H, d, eps, None) == want
+        assert lib.lite_la_block_causal_bwd(a, g, o, B, N, H, d, eps, 16, None) == want
+    assert lib.lite_la_bwd(None, g, o, 1, 4, 1, 32, 1e-15, None) == 1
+    assert lib.lite_la_bwd(a, None, o, 1, 4, 1, 32, 1e-15, None) == 1
+    assert lib.lite_la_bwd(a, g, None, 1, 4, 1, 32, 1e-15, None) == 1
+    assert lib.lite_la_bwd(a, g, ctypes.c_void_p((1 << 30) + 4), 1, 4, 1, 32, 1e-15, None) == 1
+    # dqkv overlapping qkv or dout
+    assert lib.lite_la_bwd(a, g, ctypes.c_void_p((1 << 20) + 512), 1, 4, 1, 32, 1e-15, None) == 1
+    assert "overlap" in lib.lite_la_last_error().decode()
+    assert lib.lite_la_bwd(a, g, ctypes.c_void_p((1 << 24) - 512), 1, 4, 1, 32, 1e-15, None) == 1
+    assert lib.lite_la_block_causal_bwd(a, g, o, 1, 4, 1, 32, 1e-15, 0, None) == 1
+    # an empty problem is a no-op; events are required for the timed variant
+    assert lib.lite_la_bwd(None, None, None, 0, 4, 1, 32, 1e-15, None) == 0
+    null = (ctypes.c_void_p * 4)(None, None, None, None)
+    assert lib.lite_la_bwd_events(a, g, o, 1, 4, 1, 32, 1e-15, 0, None, null) == 1
+
+
+def test_backward_workspace_bytes(lib):
+    state = 33 * 32 * 4
+    assert ll.lib().lite_la_bwd_workspace_bytes(0, 16, 1, 32, 0) == 0
+    assert ll.lib().lite_la_bwd_workspace_bytes(1, 16, 1, 64, 0) == 0
+    for (B, N, H, T) in [(1, 1, 1, 0), (2, 16384, 70, 0), (1, 16384, 70, 1024), (1, 100, 3, 7)]:
+        nblk = 1 if T <= 0 else -(-N // T)
+        got = ll.lib().lite_la_bwd_workspace_bytes(B, N, H, 32, T)
+        # the forward's partials, S images (5120 B) and S^T images (4096 B), dS partials and images
+        assert got >= B * H * nblk * (2 * state + 2 * (5120 + 4096))
+        assert got >= ll.lite_la_workspace_bytes(B, N, H, 32, T) - 64 * 4

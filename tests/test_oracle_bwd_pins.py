@@ -171,3 +171,25 @@ def test_rows_select_the_full_result_and_packed_entry_points_agree():
             assert np.isnan(samp[0]).all()
     with pytest.raises(ValueError):
         oracle.lite_la_block_causal_bwd(qb, gb, B, N, H, D, 1e-15, 0)
+
+
+@pytest.mark.parametrize("T", [None, 3])
+def test_error_magnitudes_bound_the_gradients(T):
+    """M >= |gradient| elementwise, with equality for dv when dout and v are non-negative (then
+    no term of dv = sum_i w_ij dout_i / den_i is negative); flipping signs of v or dout entries
+    leaves M unchanged."""
+    rng = np.random.default_rng(15)
+    N, eps = 12, 1e-15
+    q, k, v, g = (rng.standard_normal((N, D)) for _ in range(4))
+    dq, dk, dv, mq, mk, mv = oracle.lite_la_bwd_head(q, k, v, g, eps, T, magnitudes=True)
+    for grad, mag in ((dq, mq), (dk, mk), (dv, mv)):
+        assert np.all(mag >= np.abs(grad) * (1 - 1e-12))
+    flip = np.where(rng.random((N, D)) < 0.5, -1.0, 1.0)
+    _, _, _, mq2, mk2, mv2 = oracle.lite_la_bwd_head(q, k, v * flip, g * flip[::-1], eps, T, magnitudes=True)
+    for a, b in ((mq, mq2), (mk, mk2), (mv, mv2)):
+        np.testing.assert_allclose(a, b, rtol=1e-12)
+    _, _, dvp, _, _, mvp = oracle.lite_la_bwd_head(q, k, np.abs(v), np.abs(g), eps, T, magnitudes=True)
+    np.testing.assert_allclose(mvp, dvp, rtol=1e-12)
+    # for N = 1 dq is eps-small while its magnitude is not
+    dq1, _, _, mq1, _, _ = oracle.lite_la_bwd_head(q[:1], k[:1], v[:1], g[:1], eps, None, magnitudes=True)
+    assert np.abs(dq1).max() < 1e-12 * mq1.max()
