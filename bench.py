@@ -44,6 +44,7 @@ WORKLOADS_BENCH = {
 D = 32
 EPS = 1e-15
 METRIC = "LiteLA fwd tokens·heads/s and µs/call at 4096px; % of HBM/FMA roofline"
+METRIC_BWD = "LiteLA bwd tokens·heads/s and µs/call at 4096px; % of HBM roofline"
 UNIT = "tokens·heads/s"
 FP32_LANES_PER_SM = 128          # B200: 4 SM sub-partitions x 32 fp32 lanes
 NUM_SMS = 148
@@ -53,6 +54,11 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
 # brackets the phases.  Per path: the timed phases and their algorithmic bytes (in units of
 # E = B*N*H*d elements).
 PATHS = {
+    # backward (--direction bwd): five kernels in three timed phases; 18 bytes per element
+    # (k, v read for the state; q, dout read and dq written; k, v read and dk, dv written)
+    5: {"phases": ("litela_reduce_tc+litela_state_scan", "litela_bwd_q_tc", "litela_state_scan+litela_bwd_kv_tc"),
+        "alg_bytes_E": {"litela_reduce_tc+litela_state_scan": 4, "litela_bwd_q_tc": 6,
+                        "litela_state_scan+litela_bwd_kv_tc": 8}},
     1: {"phases": ("litela_fused_tc",), "alg_bytes_E": {"litela_fused_tc": 8}},
     3: {"phases": ("litela_reduce_tc+litela_state_scan", "litela_apply_tc"),
         "alg_bytes_E": {"litela_reduce_tc+litela_state_scan": 4, "litela_apply_tc": 4}},
@@ -191,21 +197,33 @@ def one_head_bits(qkv_bits, B, N, H, b, h):
     return np.ascontiguousarray(x.reshape(1, N, 3 * D))
 
 
-def oracle_head(oracle, head_bits, N, T):
-    """The oracle on one whole (batch, head): non-causal when T == 0."""
+def oracle_head(oracle, head_bits, N, T, dout_bits=None):
+    """The oracle on one whole (batch, head): non-causal when T == 0; the backward (all N
+    tokens' dq, dk, dv) when dout_bits [1, N, d] is given."""
+    if dout_bits is not None:
+        if T:
+            return oracle.lite_la_block_causal_bwd(head_bits, dout_bits, 1, N, 1, D, EPS, T)
+        return oracle.lite_la_bwd(head_bits, dout_bits, 1, N, 1, D, EPS)
     if T:
         return oracle.lite_la_block_causal_fwd(head_bits, 1, N, 1, D, EPS, T)
     return oracle.lite_la_fwd(head_bits, 1, N, 1, D, EPS)
 
 
-def oracle_head_rate(qkv_bits, B, N, H, T, seconds, max_heads=None):
+def one_head_dout_bits(dout_bits, B, N, H, b, h):
+    """[1, N, d] bits of head h of batch b of an incoming gradient [B, N, H*d]."""
+    import numpy as np
+    return np.ascontiguousarray(dout_bits.reshape(B, N, H, D)[b, :, h, :].reshape(1, N, D))
+
+
+def oracle_head_rate(qkv_bits, B, N, H, T, seconds, max_heads=None, dout_bits=None):
     """Times the fp64 oracle on whole heads (all N queries of one (batch, head)) until
     `seconds` have passed; returns (tokens*heads per second, heads done, elapsed)."""
     import oracle
     heads, t0 = 0, time.perf_counter()
     while True:
         b, h = divmod(heads % (B * H), H)
-        oracle_head(oracle, one_head_bits(qkv_bits, B, N, H, b, h), N, T)
+        g = None if dout_bits is None else one_head_dout_bits(dout_bits, B, N, H, b, h)
+        oracle_head(oracle, one_head_bits(qkv_bits, B, N, H, b, h), N, T, g)
         heads += 1
         el = time.perf_counter() - t0
         if el >= seconds or (max_heads and heads >= max_heads):
@@ -226,34 +244,50 @@ def run_reference(args, wl):
         return 0
     B, N, H, calls, seed, T = WORKLOADS_BENCH[wl]
     bits = to_bits(make_qkv(B, N, H, D, seed=seed, device="cpu"))
+    bwd = args.direction == "bwd"
+    gbits = to_bits(make_dout(B, N, H, seed + 500, "cpu")) if bwd else None
     import oracle
     heads = [(i // H % B, i % H) for i in range(args.warmup + args.steps)]
+
+    def head_dout(b, h):
+        return None if gbits is None else one_head_dout_bits(gbits, B, N, H, b, h)
+
     for i in range(args.warmup):
-        oracle_head(oracle, one_head_bits(bits, B, N, H, *heads[i]), N, T)
+        oracle_head(oracle, one_head_bits(bits, B, N, H, *heads[i]), N, T, head_dout(*heads[i]))
     times = []
     for i in range(args.steps):
         hb = one_head_bits(bits, B, N, H, *heads[args.warmup + i])
+        gb = head_dout(*heads[args.warmup + i])
         t0 = time.perf_counter()
-        oracle_head(oracle, hb, N, T)
+        oracle_head(oracle, hb, N, T, gb)
         times.append(time.perf_counter() - t0)
     ms = 1e3 * float(np.mean(times))
     value = N / (ms / 1e3)
     sample = ("one whole (batch, head) per step: all %d queries against all %d keys" % (N, N) if not T else
               "one whole (batch, head) per step: %d queries, blocks of %d tokens" % (N, T))
-    emit({"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+    emit({"impl": "reference", "metric": METRIC_BWD if bwd else METRIC, "value": value, "unit": UNIT,
           "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
           "data": "synthetic: i.i.d. N(0,1) bf16 qkv, seed %d" % seed,
-          "config": config_of(wl),
+          "config": config_of(wl, args.direction),
           "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                            "sample": sample},
           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
     return 0
 
 
-def config_of(wl):
+def make_dout(B, N, H, seed, device):
+    """Incoming gradient for the backward: bf16 [B, N, H*d], i.i.d. N(0,1) from a seeded generator."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return torch.randn((B, N, H * D), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+
+def config_of(wl, direction="fwd"):
     B, N, H, calls, seed, T = WORKLOADS_BENCH[wl]
-    return {"workload": wl, "B": B, "N": N, "H": H, "d": D, "tokens_per_block": T or None, "calls_per_step": calls,
+    return {"workload": wl + ("_bwd" if direction == "bwd" else ""), "direction": direction,
+            "B": B, "N": N, "H": H, "d": D, "tokens_per_block": T or None, "calls_per_step": calls,
             "distinct_input_buffers": calls, "eps": EPS, "layout": "qkv bf16 [B,N,3*H*d], out bf16 [B,N,H*d]",
             "l2": "inputs larger than L2 (%.0f MB per call vs 126 MB), no flush" % (B * N * 3 * H * D * 2 / 1e6)}
 
@@ -270,6 +304,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ffma-seconds", type=float, default=2.0,
                     help="duration of the fp32 FMA peak measurement (0 skips it)")
+    ap.add_argument("--direction", choices=["fwd", "bwd"], default="fwd",
+                    help="bwd times the backward (dq, dk, dv of a seeded incoming gradient)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -307,20 +343,35 @@ def main():
 
     lib = ll.lib()
     B, N, H, calls, seed0, T = WORKLOADS_BENCH[args.workload]
+    bwd = args.direction == "bwd"
     qkv_bytes, out_bytes = B * N * 3 * H * D * 2, B * N * H * D * 2
     free, _ = torch.cuda.mem_get_info(dev)
-    need = calls * (qkv_bytes + out_bytes) + (2 << 30)
+    need = calls * (qkv_bytes + out_bytes + (qkv_bytes if bwd else 0)) + (2 << 30)
     if free < need:
         raise SystemExit("not enough free GPU memory: need %.1f GB, free %.1f GB" % (need / 1e9, free / 1e9))
     seeds = [seed0 + i for i in range(calls)] if args.workload.startswith("sana4800m") else [seed0 * 10 + i for i in range(calls)]
     seeds = rank_seeds(seeds, rank)
     ins = [make_qkv(B, N, H, D, seed=s, device=dev) for s in seeds]
     outs = [torch.empty((B, N, H * D), dtype=torch.bfloat16, device=dev) for _ in range(calls)]
+    if bwd:   # the backward reads an incoming gradient (in `outs`) and writes dqkv
+        outs = [make_dout(B, N, H, s + 500, dev) for s in seeds]
+        grads = [torch.empty((B, N, 3 * H * D), dtype=torch.bfloat16, device=dev) for _ in range(calls)]
+        grad_p = [t.data_ptr() for t in grads]
     stream = torch.cuda.current_stream(dev)
     sh = ctypes.c_void_p(stream.cuda_stream)
     in_p = [t.data_ptr() for t in ins]
     out_p = [t.data_ptr() for t in outs]
-    if T:
+    if bwd:   # fwd(i, ...) runs call i: here the backward of buffer i
+        dq_of = {p_: g_ for p_, g_ in zip(in_p, grad_p)}
+
+        def fwd(qkv, out, B, N, H, d, eps, stream):
+            if T:
+                return lib.lite_la_block_causal_bwd(qkv, out, dq_of[qkv], B, N, H, d, eps, T, stream)
+            return lib.lite_la_bwd(qkv, out, dq_of[qkv], B, N, H, d, eps, stream)
+
+        def fwd_events(qkv, out, B, N, H, d, eps, stream, evs):
+            return lib.lite_la_bwd_events(qkv, out, dq_of[qkv], B, N, H, d, eps, T, stream, evs)
+    elif T:
         def fwd(qkv, out, B, N, H, d, eps, stream):
             return lib.lite_la_block_causal_fwd(qkv, out, B, N, H, d, eps, T, stream)
 
@@ -364,14 +415,16 @@ def main():
     us_call = 1e3 * ms_step / calls
     value = aggregate_rate(B * N * H * calls * args.steps, world, ms_total)
 
-    # per-kernel durations: the same calls through lite_la_fwd_events (3 events per call)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(calls)]
+    # per-kernel durations: the same calls through the phase-timed entry points (3 events per
+    # forward call, 4 per backward call)
+    nev = 4 if bwd else 3
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(calls)]
     for trip in evs:                      # recording once creates the underlying CUDA events
         for e in trip:
             e.record(stream)
     torch.cuda.synchronize(dev)
-    ev_handles = [(ctypes.c_void_p * 3)(*[ctypes.c_void_p(e.cuda_event) for e in trip]) for trip in evs]
-    nk = int(lib.lite_la_kernels_per_call(B, N, H, D, T))
+    ev_handles = [(ctypes.c_void_p * nev)(*[ctypes.c_void_p(e.cuda_event) for e in trip]) for trip in evs]
+    nk = 5 if bwd else int(lib.lite_la_kernels_per_call(B, N, H, D, T))
     phases = PATHS[nk]["phases"]
     kern_ms = {k: 0.0 for k in phases}
     nlaunch = 0
@@ -385,8 +438,8 @@ def main():
             if nk == 1:
                 kern_ms[phases[0]] += trip[0].elapsed_time(trip[2])
             else:
-                kern_ms[phases[0]] += trip[0].elapsed_time(trip[1])
-                kern_ms[phases[1]] += trip[1].elapsed_time(trip[2])
+                for k in range(len(phases)):
+                    kern_ms[phases[k]] += trip[k].elapsed_time(trip[k + 1])
         nlaunch += calls
     kern_us = {k: 1e3 * v / nlaunch for k, v in kern_ms.items()}
     kern_us_isolated = dict(kern_us)
@@ -396,7 +449,10 @@ def main():
         # a kernel's set-up runs while its predecessor drains, its memory traffic after it)
         kern_us = {phases[0]: us_call}
     E = B * N * H * D
-    flops_per_call = 4 * B * H * N * D * (D + 1)
+    # algorithmic FLOPs (2 per multiply-add): forward, the state (d+1) and the apply (d+1) per
+    # element; backward, the state (d+1), y (d+1), S^T g (d), dS (d+1), dk (d), dv (d)
+    flops_per_call = 2 * E * ((D + 1) + (D + 1) + D + (D + 1) + D + D) if bwd else 4 * B * H * N * D * (D + 1)
+    call_bytes_E = 18 if bwd else 8
     alg_bytes = {k: PATHS[nk]["alg_bytes_E"][k] * E for k in phases}
     peaks = load_peaks()
     dom = max(kern_us, key=kern_us.get)
@@ -407,7 +463,7 @@ def main():
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": traffic, "kernel": dom, "kernel_us": kern_us[dom],
                 "alg_bytes_per_launch": alg_bytes[dom],
-                "alg_flops_per_launch": flops_per_call * alg_bytes[dom] // (8 * E),
+                "alg_flops_per_launch": flops_per_call * alg_bytes[dom] // (call_bytes_E * E),
                 "peak_source": peak_note, "kernel_us_all": kern_us, "kernel_us_isolated": kern_us_isolated,
                 "timing": ("average launch duration over the timed region: CUDA events around the back-to-back "
                            "calls on the launching stream, / launches" if nk == 1 else
@@ -415,8 +471,8 @@ def main():
                            "no programmatic overlap with the neighbouring kernels)")
                           + "; kernel_us_isolated: each call alone between events"}
     # the call as a whole against the slower of the HBM and fp32-FMA bounds
-    t_hbm = 8 * E / (peaks["hbm_gbs"] * 1e9) * 1e6
-    t_fma = 4 * B * H * N * D * (D + 1) / (fp32_fma_peak_tflops(peaks.get("sm_max_mhz", 1965.0)) * 1e12) * 1e6
+    t_hbm = call_bytes_E * E / (peaks["hbm_gbs"] * 1e9) * 1e6
+    t_fma = flops_per_call / (fp32_fma_peak_tflops(peaks.get("sm_max_mhz", 1965.0)) * 1e12) * 1e6
     call_roof = {"t_hbm_us": t_hbm, "t_fma_us": t_fma, "t_roof_us": max(t_hbm, t_fma),
                  "us_per_call": us_call, "frac": max(t_hbm, t_fma) / us_call}
     if clocks.get("sm_mhz"):
@@ -425,7 +481,7 @@ def main():
         call_roof["frac_at_measured_clock"] = max(t_hbm, t_fma_clk) / us_call
     if args.ffma_seconds > 0:
         ffma = measure_ffma_peak(ll, dev, stream, args.ffma_seconds)
-        t_fma_meas = 4 * B * H * N * D * (D + 1) / (ffma["tflops"] * 1e12) * 1e6
+        t_fma_meas = flops_per_call / (ffma["tflops"] * 1e12) * 1e6
         call_roof["ffma_peak_measured"] = ffma
         call_roof["t_fma_us_measured_peak"] = t_fma_meas
         call_roof["frac_vs_measured_fma_peak"] = max(t_hbm, t_fma_meas) / us_call
@@ -440,6 +496,12 @@ def main():
         h_out = [torch.empty((B, N, H * D), dtype=torch.bfloat16, pin_memory=True) for _ in range(nbuf)]
         for j in range(nbuf):
             h_in[j].copy_(ins[j])
+        if bwd:   # the backward uploads qkv and dout, and downloads dqkv
+            h_g = [torch.empty((B, N, H * D), dtype=torch.bfloat16, pin_memory=True) for _ in range(nbuf)]
+            h_out = [torch.empty((B, N, 3 * H * D), dtype=torch.bfloat16, pin_memory=True) for _ in range(nbuf)]
+            for j in range(nbuf):
+                h_g[j].copy_(outs[j])
+        results = grads if bwd else outs
         up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         ev_up = [torch.cuda.Event() for _ in range(nbuf)]
         ev_fwd = [torch.cuda.Event() for _ in range(nbuf)]
@@ -453,6 +515,8 @@ def main():
                 with torch.cuda.stream(up):
                     up.wait_event(ev_fwd[j])          # the forward that last read ins[j] is done
                     ins[j].copy_(h_in[j], non_blocking=True)
+                    if bwd:
+                        outs[j].copy_(h_g[j], non_blocking=True)
                     ev_up[j].record(up)
                 stream.wait_event(ev_up[j])
                 stream.wait_event(ev_down[j])         # outs[j] has been downloaded
@@ -462,7 +526,7 @@ def main():
                 ev_fwd[j].record(stream)
                 with torch.cuda.stream(down):
                     down.wait_event(ev_fwd[j])
-                    h_out[j].copy_(outs[j], non_blocking=True)
+                    h_out[j].copy_(results[j], non_blocking=True)
                     ev_down[j].record(down)
             stream.wait_stream(down)                  # the step ends when the last result is on the host
 
@@ -471,26 +535,33 @@ def main():
         e2e_ms, _ = timed(e2e_step, args.e2e_steps)
         e2e_ms = max_over_ranks(e2e_ms)
         e2e = {"value": aggregate_rate(B * N * H * calls * args.e2e_steps, world, e2e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": calls * qkv_bytes, "d2h_bytes_per_step": calls * out_bytes,
+               "h2d_bytes_per_step": calls * (qkv_bytes + (out_bytes if bwd else 0)),
+               "d2h_bytes_per_step": calls * (qkv_bytes if bwd else out_bytes),
                "ms_per_step": e2e_ms / args.e2e_steps, "steps": args.e2e_steps,
-               "how": "per call: pinned host qkv -> device copy (upload stream), lite_la_fwd (compute stream), "
-                      "device -> pinned host out copy (download stream); 3 buffers in rotation, events order them"}
+               "how": ("per call: pinned host qkv and dout -> device (upload stream), lite_la_bwd (compute stream), "
+                       "dqkv -> pinned host (download stream)" if bwd else
+                       "per call: pinned host qkv -> device copy (upload stream), lite_la_fwd (compute stream), "
+                       "device -> pinned host out copy (download stream)")
+                      + "; 3 buffers in rotation, events order them"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         bits = to_bits(ins[0])
-        rate, heads, el = oracle_head_rate(bits, B, N, H, T, args.cpu_seconds)
+        gbits = to_bits(outs[0]) if bwd else None
+        rate, heads, el = oracle_head_rate(bits, B, N, H, T, args.cpu_seconds, dout_bits=gbits)
         cpu = {"value": rate, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-               "sample": "%d whole (batch, head) pairs of input buffer 0 (all %d queries x %d keys each), %.1f s"
-                         % (heads, N, N, el)}
+               "sample": "%d whole (batch, head) pairs of input buffer 0 (%s, all %d tokens), %.1f s"
+                         % (heads, "dq, dk, dv" if bwd else "all queries x all keys", N, el)}
 
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        line = {"metric": METRIC_BWD if bwd else METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_step, "us_per_call": us_call,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "math": "tensor-core bf16 x bf16 products with fp32 accumulation; fp32 state applied as bf16 hi + lo",
                 "data": "synthetic: i.i.d. N(0,1) bf16 qkv from seeded torch generators",
-                "config": config_of(args.workload), "roofline": roofline, "call_roofline": call_roof,
+                "config": config_of(args.workload, args.direction), "roofline": roofline,
+                "call_roofline": call_roof,
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": nk * calls * args.steps,
                 "clocks": clocks, "gpu": torch.cuda.get_device_name(dev)}
         if world > 1:

@@ -482,7 +482,13 @@ litela_status run_bwd(const void* qkv, const void* dout, OutT* dqkv, int B, int 
   s = launch_scan(plan, dpartials, dimages, nullptr, num_sms, stream, pdl, nullptr, nullptr, dimages_t, true,
                   plan.bwd_cpb);
   if (s != LITELA_OK) return s;
-  e = launch_ex(litela_bwd_kv_tc<OutT>, grid, dim3(kBwThreads), kBkSmemBytes, stream, pdl, map_qkv,
+  // TMA stores of dk, dv (bf16 output; the fp32 output is written row by row and never uses it)
+  CUtensorMap map_dqkv = map_qkv;
+  if (sizeof(OutT) == 2) {
+    s = encode_qkv_map(dqkv, B, N, H, kApTile, &map_dqkv);
+    if (s != LITELA_OK) return s;
+  }
+  e = launch_ex(litela_bwd_kv_tc<OutT>, grid, dim3(kBwThreads), kBkSmemBytes, stream, pdl, map_qkv, map_dqkv,
                 static_cast<const uint8_t*>(dimages), static_cast<const uint8_t*>(dimages_t), dqkv, ws->err, bp);
   if (e != cudaSuccess) return cuda_fail(e, "launch litela_bwd_kv_tc");
   if (events && (e = cudaEventRecord(events[3], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");

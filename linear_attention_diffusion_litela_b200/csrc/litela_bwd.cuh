@@ -55,14 +55,20 @@ enum : int {
   kErrBwdKvProducer = 0x610, kErrBwdKvMma = 0x620, kErrBwdKvRelu = 0x630, kErrBwdKvEpi = 0x640,
 };
 
-constexpr int kBwThreads = 256;   // w0 TMA, w1 MMA, w2..3 ReLU, w4..7 epilogue
+// w0 TMA, w1 MMA, w2..3 ReLU, w4..11 epilogue in two groups of 4 warps (group g takes the heads
+// j with j % 2 == g; each group covers all 128 TMEM lanes)
+constexpr int kBwThreads = 384;
+constexpr int kBwEpiThreads = 256;
 constexpr int kBwStages = 2;
 constexpr uint32_t kBwBoxBytes = kApTile * 128;        // 128 tokens x 64 channels (one head pair)
 constexpr uint32_t kBwTileBytes = 2 * kBwBoxBytes;     // 4 heads
 constexpr uint32_t kBwStageBytes = 2 * kBwTileBytes;   // two tensors: (q, dout) or (k, v)
 constexpr uint32_t kBwHBytes = (kApTile / 16) * 512;   // 16 columns x 128 tokens, K-major
 constexpr uint32_t kBwImgBytes = kApUnitHeads * (kImageBytes + kImageTBytes);
-constexpr uint32_t kBwSlotCols = 144;                   // TMEM columns per head: 80 + 64
+// TMEM: two accumulator slots (slot g serves epilogue group g) of 144 columns: the products with
+// an S (or dS) image (N = 80: hi rows 0..39, lo rows 40..79) and with an S^T image (N = 64: hi
+// columns 0..31, lo 32..63); the epilogue adds the hi and lo halves.
+constexpr uint32_t kBwSlotCols = kImageRows + kImageTRows;
 constexpr uint32_t kBwDsCol = 2 * kBwSlotCols;          // dS^T accumulator (128 columns)
 constexpr uint32_t kBwDhCol = kBwDsCol + 128;           // its ones-row part (16 columns)
 constexpr uint32_t kBwTmemCols = 512;
@@ -71,11 +77,13 @@ constexpr uint32_t kBqOffGlo = kBwStages * kBwStageBytes;
 constexpr uint32_t kBqOffH = kBqOffGlo + kBwTileBytes;
 constexpr uint32_t kBqOffImg = kBqOffH + kBwHBytes;
 constexpr uint32_t kBqOffBars = kBqOffImg + kBwImgBytes;
-constexpr uint32_t kBqSmemBytes = kBqOffBars + 256 + 1024;
+constexpr uint32_t kBqOffZ = kBqOffBars + 256;            // ones rows S[d] in fp32, [4][32]
+constexpr uint32_t kBqSmemBytes = kBqOffZ + 512 + 1024;
 // litela_bwd_kv_tc shared memory
 constexpr uint32_t kBkOffImg = kBwStages * kBwStageBytes;
 constexpr uint32_t kBkOffBars = kBkOffImg + kBwImgBytes;
-constexpr uint32_t kBkSmemBytes = kBkOffBars + 256 + 1024;
+constexpr uint32_t kBkOffZ = kBkOffBars + 256;            // ones rows dS[d] in fp32, [4][32]
+constexpr uint32_t kBkSmemBytes = kBkOffZ + 512 + 1024;
 
 // byte offset of bf16 element (token t, channel ch of the 4 heads) in a tile of two 128B-swizzled
 // TMA boxes (64 channels x 128 tokens each)
@@ -100,6 +108,22 @@ __device__ __forceinline__ void unpack_bf16x8(uint4 w, float* x) {
 
 __device__ __forceinline__ float bf16_at(const uint8_t* p) {
   return __uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(p)) << 16);
+}
+
+// true for element e (0..7) of 8 packed bf16 values that are not +0 (for values that went
+// through ReLU: the element is > 0)
+__device__ __forceinline__ bool bf16_nonzero(uint4 w, int e) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+  return ((e & 1) ? (u[e >> 1] >> 16) : (u[e >> 1] & 0xFFFFu)) != 0u;
+}
+
+// fp32 copies (hi + lo) of the ones rows (row d) of the nh state images at `img`, into zf[j][c]
+// (epilogue threads et = 0..127)
+__device__ __forceinline__ void ones_rows_fp32(const uint8_t* img, int nh, float* zf, int et) {
+  const int j = et >> 5, c = et & 31;
+  if (j < nh)
+    zf[et] = bf16_at(img + j * kImageBytes + image_offset(kD, c)) +
+             bf16_at(img + j * kImageBytes + image_offset(kImageLoRow + kD, c));
 }
 
 // stores 32 values of one head's row to global memory (bf16: 4 x 16 B, fp32: 8 x 16 B)
@@ -150,7 +174,7 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
   uint64_t* qrelu = qfull + kBwStages;
   uint64_t* qempty = qrelu + kBwStages;
   uint64_t* sfull = qempty + kBwStages;
-  uint64_t* tfull = sfull + 1;
+  uint64_t* tfull = sfull + 1;                 // one per TMEM slot
   uint64_t* tempty = tfull + 2;
   uint64_t* gready = tempty + 2;
   uint64_t* gfree = gready + 1;
@@ -176,7 +200,7 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 128);
     }
-    mbar_init(gready, 128);
+    mbar_init(gready, kBwEpiThreads);
     mbar_init(gfree, 1);
     mbar_init(dsfull, 1);
     *abort_flag = 0;
@@ -245,41 +269,13 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       constexpr uint32_t idesc_t = idesc_bf16_f32(128, kImageTRows, false, false);
       constexpr uint32_t idesc_ds = idesc_bf16_f32(128, 128, true, true);
       constexpr uint32_t idesc_dh = idesc_bf16_f32(128, 16, true, false);
-      int hc = 0;
-      bool stop = false;
-      for (int i = 0; i < sp.ntiles && !stop; ++i) {
+      const uint32_t la = smem_u32(glo), ha = smem_u32(hbuf);
+      // the dS product of tile i, once its epilogue has written g/den (hi over the g tile, lo
+      // into glo) and h
+      auto ds_product = [&](int i) {
         const int s = i % kBwStages;
-        if (!mbar_wait(&qrelu[s], (i / kBwStages) & 1, abort_flag, err, kErrBwdQMma | s)) break;
         tc_fence_after_sync();
         const uint32_t qa = smem_u32(qtile(s)), ga = smem_u32(gtile(s));
-        for (int j = 0; j < sp.nh; ++j, ++hc) {
-          const int a = hc & 1;
-          if (hc >= 2 && !mbar_wait(&tempty[a], ((hc >> 1) - 1) & 1, abort_flag, err, kErrBwdQMma | 4 | a)) {
-            stop = true;
-            break;
-          }
-          tc_fence_after_sync();
-          const uint32_t off = (j >> 1) * kBwBoxBytes + (j & 1) * 64;   // head j's 32 channels
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            // y = q~ . S^T: A K-major 128B swizzle (8-token groups 1024 B apart), B = S image
-            umma_bf16(tmem + a * kBwSlotCols, smem_desc(qa + off + ks * 32, 16, 1024, kSwizzle128B),
-                      smem_desc(smem_u32(simg + j * kImageBytes) + ks * 256, 128, 512, kSwizzleNone), idesc_y, ks);
-          }
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            // T = g . S[0:d]: A = the raw dout tile, B = the S^T image
-            umma_bf16(tmem + a * kBwSlotCols + kImageRows, smem_desc(ga + off + ks * 32, 16, 1024, kSwizzle128B),
-                      smem_desc(smem_u32(stimg + j * kImageTBytes) + ks * 256, 128, 512, kSwizzleNone), idesc_t,
-                      ks);
-          }
-          umma_commit(&tfull[a]);
-        }
-        if (stop) break;
-        // the epilogue has written g/den (hi over the g tile, lo into glo) and h for this tile
-        if (!mbar_wait(gready, i & 1, abort_flag, err, kErrBwdQMma | 12)) break;
-        tc_fence_after_sync();
-        const uint32_t la = smem_u32(glo), ha = smem_u32(hbuf);
 #pragma unroll
         for (int ks = 0; ks < kApTile / 16; ++ks) {
           // dS^T[c][r] += sum over 16 tokens of q~[t][c] (g/den)[t][r]: A = q~ MN-major (M = 4 heads
@@ -293,6 +289,57 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         }
         umma_commit(&qempty[s]);
         umma_commit(gfree);
+      };
+      // The head products of tile i need tile i's ReLU; the dS product of tile i needs tile i's
+      // epilogue (gready).  Issue whichever becomes ready first, the dS product preferred (it
+      // releases the stage for the next load and glo for the next epilogue).  The heads of
+      // tile i are not issued before the dS product of tile i - 2: their TMEM slots are freed by
+      // the epilogue of tile i - 1, which waits for that product.
+      int use[2] = {0, 0};
+      int hnext = 0, dnext = 0;
+      bool stop = false;
+      uint64_t t_idle = globaltimer_ns();
+      while (dnext < sp.ntiles && !stop) {
+        if (dnext < hnext && mbar_test(gready, dnext & 1)) {
+          ds_product(dnext++);
+          t_idle = globaltimer_ns();
+          continue;
+        }
+        if (!(hnext < sp.ntiles && hnext <= dnext + 1 && mbar_test(&qrelu[hnext % kBwStages], (hnext / kBwStages) & 1))) {
+          if (*abort_flag) break;
+          if (globaltimer_ns() - t_idle > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicCAS(err, 0, kErrBwdQMma | 12);
+            break;
+          }
+          continue;
+        }
+        const int i = hnext++;
+        const int s = i % kBwStages;
+        tc_fence_after_sync();
+        const uint32_t qa = smem_u32(qtile(s)), ga = smem_u32(gtile(s));
+        for (int j = 0; j < sp.nh; ++j) {
+          const int a = j & 1;   // the slot of epilogue group j % 2
+          if (use[a] > 0 && !mbar_wait(&tempty[a], (use[a] - 1) & 1, abort_flag, err, kErrBwdQMma | 4 | a)) {
+            stop = true;
+            break;
+          }
+          ++use[a];
+          tc_fence_after_sync();
+          const uint32_t off = (j >> 1) * kBwBoxBytes + (j & 1) * 64;   // head j's 32 channels
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks) {
+            // y = q~ . S^T: A K-major 128B swizzle (8-token groups 1024 B apart), B = S image
+            umma_bf16(tmem + a * kBwSlotCols, smem_desc(qa + off + ks * 32, 16, 1024, kSwizzle128B),
+                      smem_desc(smem_u32(simg + j * kImageBytes) + ks * 256, 128, 512, kSwizzleNone), idesc_y, ks);
+            // T = g . S[0:d]: A = the raw dout tile, B = the S^T image
+            umma_bf16(tmem + a * kBwSlotCols + kImageRows, smem_desc(ga + off + ks * 32, 16, 1024, kSwizzle128B),
+                      smem_desc(smem_u32(stimg + j * kImageTBytes) + ks * 256, 128, 512, kSwizzleNone), idesc_t,
+                      ks);
+          }
+          umma_commit(&tfull[a]);
+        }
+        t_idle = globaltimer_ns();
       }
       umma_commit(dsfull);
     }
@@ -304,7 +351,7 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       const int s = i % kBwStages;
       if (!mbar_wait(&qfull[s], (i / kBwStages) & 1, abort_flag, err, kErrBwdQRelu | s)) break;
       uint8_t* st = qtile(s);
-#pragma unroll 4
+#pragma unroll 8
       for (int j = t; j < nchunks; j += kApReluThreads) {
         uint4* c = reinterpret_cast<uint4*>(st + j * 16);
         *c = relu_bf16x8(*c);
@@ -313,89 +360,110 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       mbar_arrive(&qrelu[s]);
     }
   } else {
-    // epilogue: thread = token row of the tile (TMEM lane)
-    const int wq = warp & 3, row = wq * 32 + lane;
+    // epilogue: group g takes heads g, g + 2 through TMEM slot g; thread = token row (TMEM lane)
+    const int g = (warp - 4) >> 2, wq = warp & 3, row = wq * 32 + lane;
+    const int gbar = 1 + 2 * g;   // the group's named barrier (1 or 3)
+    float* zf = reinterpret_cast<float*>(smem + kBqOffZ);
     bool ok = sp.ntiles > 0 && mbar_wait(sfull, 0, abort_flag, err, kErrBwdQEpi | 8);
-    int hc = 0;
+    if (ok && threadIdx.x < 256) ones_rows_fp32(simg, sp.nh, zf, threadIdx.x - 128);
+    bar_sync(2, kBwEpiThreads);
+    int use = 0;
     for (int i = 0; ok && i < sp.ntiles; ++i) {
       const int s = i % kBwStages;
       const int tok = sp.n0 + i * kApTile + row;
       const bool valid = tok < sp.n1;
       // the tile's TMA data (this thread reads dout and q~ from it; the stage cannot be refilled
-      // before this epilogue releases it), and the previous tile's dS product has read glo, hbuf
+      // before this epilogue releases it)
       if (!mbar_wait(&qfull[s], (i / kBwStages) & 1, abort_flag, err, kErrBwdQEpi | 14)) ok = false;
-      if (ok && i > 0 && !mbar_wait(gfree, (i - 1) & 1, abort_flag, err, kErrBwdQEpi | 12)) ok = false;
-      if (bar_any(1, 128, !ok)) {
+      if (bar_any(gbar, 128, !ok)) {
         ok = false;
         break;
       }
-      for (int j = 0; j < sp.nh; ++j, ++hc) {
-        const int a = hc & 1;
-        const bool okw = mbar_wait(&tfull[a], (hc >> 1) & 1, abort_flag, err, kErrBwdQEpi | a);
-        if (bar_any(1, 128, !okw)) {
+      bool first = true;
+      for (int j = g; j < sp.nh; j += 2) {
+        const bool okw = mbar_wait(&tfull[g], use & 1, abort_flag, err, kErrBwdQEpi | g);
+        ++use;
+        if (bar_any(gbar, 128, !okw)) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
-        const uint32_t ta = tmem + (static_cast<uint32_t>(wq * 32) << 16) + a * kBwSlotCols;
-        float o[kD], den;
+        const uint32_t ta = tmem + (static_cast<uint32_t>(wq * 32) << 16) + g * kBwSlotCols;
+        uint8_t* gt = gtile(s);
+        const uint8_t* qt = qtile(s);
+        // g (raw dout) of this token and head, from shared memory
+        uint4 gw[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) gw[k] = *reinterpret_cast<const uint4*>(gt + sw_offset(row, j * kD + k * 8));
+        // den and h = -(g . out) / den = -(g . y[0:d]) / den^2
+        float inv, h;
         {
           uint32_t v[kImageRows];
 #pragma unroll
           for (int k = 0; k < kImageRows / 16; ++k) tmem_ld_x16(ta + k * 16, v + k * 16);
           tmem_wait_ld();
-          den = (__uint_as_float(v[kD]) + __uint_as_float(v[kImageLoRow + kD])) + p.eps;
-          const float inv = 1.0f / den;
+          inv = 1.0f / ((__uint_as_float(v[kD]) + __uint_as_float(v[kImageLoRow + kD])) + p.eps);
+          float dot = 0.f;
 #pragma unroll
-          for (int r = 0; r < kD; ++r) o[r] = (__uint_as_float(v[r]) + __uint_as_float(v[kImageLoRow + r])) * inv;
+          for (int k = 0; k < 4; ++k) {
+            float g8[8];
+            unpack_bf16x8(gw[k], g8);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dot = fmaf(g8[e], __uint_as_float(v[8 * k + e]) + __uint_as_float(v[kImageLoRow + 8 * k + e]), dot);
+          }
+          h = -dot * inv * inv;
         }
-        const float inv = 1.0f / den;
-        // g (raw dout) of this token and head, from shared memory; h = -(g . out) / den
-        float g[kD];
-        uint8_t* gt = gtile(s);
-        const uint8_t* qt = qtile(s);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          unpack_bf16x8(*reinterpret_cast<const uint4*>(gt + sw_offset(row, j * kD + k * 8)), g + 8 * k);
-        float dot = 0.f;
-#pragma unroll
-        for (int r = 0; r < kD; ++r) dot = fmaf(g[r], o[r], dot);
-        const float h = -dot * inv;
         uint32_t tv[kImageTRows];
 #pragma unroll
         for (int k = 0; k < kImageTRows / 16; ++k) tmem_ld_x16(ta + kImageRows + k * 16, tv + k * 16);
         tmem_wait_ld();
         tc_fence_before_sync();
-        mbar_arrive(&tempty[a]);
-        // dq = relu'(q) * (S[0:d]^T g / den + h S[d]); S[d] (the ones row) from the S image
-        const uint8_t* im = simg + j * kImageBytes;
+        mbar_arrive(&tempty[g]);
+        // dq = relu'(q) * (S[0:d]^T g / den + h S[d]); relu(q) > 0 <=> its bf16 bits are not 0
+        const float4* z4 = reinterpret_cast<const float4*>(zf + j * kD);
         float dq[kD];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          float qr[8];
-          unpack_bf16x8(*reinterpret_cast<const uint4*>(qt + sw_offset(row, j * kD + k * 8)), qr);
+          const uint4 qw = *reinterpret_cast<const uint4*>(qt + sw_offset(row, j * kD + k * 8));
+          const float4 za = z4[2 * k], zb = z4[2 * k + 1];
+          const float z[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int c = 8 * k + e;
-            const float z = bf16_at(im + image_offset(kD, c)) + bf16_at(im + image_offset(kImageLoRow + kD, c));
             const float t = (__uint_as_float(tv[c]) + __uint_as_float(tv[kD + c])) * inv;
-            dq[c] = qr[e] > 0.f ? fmaf(z, h, t) : 0.f;
+            dq[c] = bf16_nonzero(qw, e) ? fmaf(z[e], h, t) : 0.f;
           }
         }
         if (valid) store_row32(dqkv + ((int64_t)b * p.N + tok) * (3 * p.H * kD) + (quad * kApUnitHeads + j) * kD, dq);
+        // the previous tile's dS product has read glo and hbuf (the columns of other heads of
+        // the g tile are not touched below)
+        if (first && i > 0) {
+          const bool okg = mbar_wait(gfree, (i - 1) & 1, abort_flag, err, kErrBwdQEpi | 12);
+          if (bar_any(gbar, 128, !okg)) {
+            ok = false;
+            break;
+          }
+        }
+        first = false;
         // operands of the dS product: g/den over the g tile (hi) and into glo (lo); h hi / lo
-        float ghi[8], glo8[8];
+        const float sc = valid ? inv : 0.f;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
+          const uint32_t gu[4] = {gw[k].x, gw[k].y, gw[k].z, gw[k].w};
+          uint32_t hw[4], lw[4];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float x = valid ? g[8 * k + e] * inv : 0.f;
-            ghi[e] = __bfloat162float(__float2bfloat16_rn(x));
-            glo8[e] = x - ghi[e];
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float x0 = __uint_as_float(gu[e2] << 16) * sc, x1 = __uint_as_float(gu[e2] & 0xFFFF0000u) * sc;
+            __nv_bfloat162 hp = __floats2bfloat162_rn(x0, x1);
+            const uint32_t hu = *reinterpret_cast<uint32_t*>(&hp);
+            __nv_bfloat162 lp = __floats2bfloat162_rn(x0 - __uint_as_float(hu << 16), x1 - __uint_as_float(hu & 0xFFFF0000u));
+            hw[e2] = hu;
+            lw[e2] = *reinterpret_cast<uint32_t*>(&lp);
           }
           const uint32_t off = sw_offset(row, j * kD + k * 8);
-          *reinterpret_cast<uint4*>(gt + off) = pack_bf16x8(ghi);
-          *reinterpret_cast<uint4*>(glo + off) = pack_bf16x8(glo8);
+          *reinterpret_cast<uint4*>(gt + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(glo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
         const float hv = valid ? h : 0.f;
         const __nv_bfloat16 hh = __float2bfloat16_rn(hv);
@@ -404,30 +472,38 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         *reinterpret_cast<__nv_bfloat16*>(hbuf + h_offset(kApUnitHeads + j, row)) = hl;
       }
       if (!ok) break;
+      // a group without heads in this quad (nh == 1) skips to here and still takes part
       fence_proxy_async_smem();
       mbar_arrive(gready);
     }
-    // the CTA's partial dS: warp quarter wq holds head wq's query channels (TMEM lanes)
-    float sv[kRows];
+    // the CTA's partial dS (group 0): warp quarter wq holds head wq's query channels (TMEM lanes)
+    if (g == 0) {
+      float sv[kRows];
 #pragma unroll
-    for (int r = 0; r < kRows; ++r) sv[r] = 0.f;
-    if (ok && sp.ntiles > 0) ok = mbar_wait(dsfull, 0, abort_flag, err, kErrBwdQEpi | 13);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok && sp.ntiles > 0 && wq < sp.nh) {
-      tc_fence_after_sync();
-      uint32_t rr[32], hh[16];
-      const uint32_t ta = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-      tmem_ld_x32(ta + kBwDsCol + wq * 32, rr);
-      tmem_ld_x16(ta + kBwDhCol, hh);
-      tmem_wait_ld();
+      for (int r = 0; r < kRows; ++r) sv[r] = 0.f;
+      if (ok && sp.ntiles > 0) ok = mbar_wait(dsfull, 0, abort_flag, err, kErrBwdQEpi | 13);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok && sp.ntiles > 0 && wq < sp.nh) {
+        tc_fence_after_sync();
+        uint32_t rr[32], hh[16];
+        const uint32_t ta = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+        tmem_ld_x32(ta + kBwDsCol + wq * 32, rr);
+        tmem_ld_x16(ta + kBwDhCol, hh);
+        tmem_wait_ld();
 #pragma unroll
-      for (int r = 0; r < kD; ++r) sv[r] = __uint_as_float(rr[r]);
-      sv[kD] = __uint_as_float(hh[wq]) + __uint_as_float(hh[kApUnitHeads + wq]);
+        for (int r = 0; r < kD; ++r) sv[r] = __uint_as_float(rr[r]);
+        // columns wq and 4 + wq of the ones-row part (selected without dynamic register indexing)
+        float zsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          if (c == wq || c == kApUnitHeads + wq) zsum += __uint_as_float(hh[c]);
+        sv[kD] = zsum;
+      }
+      const int64_t nparts = (int64_t)p.nblk * p.cpb;
+      float* dst = dpartials + ((((int64_t)b * p.nquads + quad) * nparts + blockIdx.x) * kRedHeads + wq) * kStateFloats;
+#pragma unroll
+      for (int r = 0; r < kRows; ++r) dst[r * kD + lane] = sv[r];   // dS[r][c = lane]
     }
-    const int64_t nparts = (int64_t)p.nblk * p.cpb;
-    float* dst = dpartials + ((((int64_t)b * p.nquads + quad) * nparts + blockIdx.x) * kRedHeads + wq) * kStateFloats;
-#pragma unroll
-    for (int r = 0; r < kRows; ++r) dst[r * kD + lane] = sv[r];   // dS[r][c = lane]
   }
 
   tc_fence_before_sync();
@@ -443,8 +519,9 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
 
 template <typename OutT>
 __global__ void __launch_bounds__(kBwThreads, 1)
-litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const uint8_t* __restrict__ dimages,
-                 const uint8_t* __restrict__ dimages_t, OutT* __restrict__ dqkv, int* __restrict__ err, BwdPlan p) {
+litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant__ CUtensorMap tmap_dqkv,
+                 const uint8_t* __restrict__ dimages, const uint8_t* __restrict__ dimages_t, OutT* __restrict__ dqkv,
+                 int* __restrict__ err, BwdPlan p) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -452,9 +529,9 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const uint8_t* __r
   uint8_t* dtimg = dimg + kApUnitHeads * kImageBytes;
   uint64_t* kvfull = reinterpret_cast<uint64_t*>(smem + kBkOffBars);
   uint64_t* krelu = kvfull + kBwStages;
-  uint64_t* kvempty = krelu + kBwStages;   // the MMAs' commit + the 128 epilogue threads
+  uint64_t* kvempty = krelu + kBwStages;   // the MMAs' commit + the epilogue's storing thread
   uint64_t* sfull = kvempty + kBwStages;
-  uint64_t* tfull = sfull + 1;
+  uint64_t* tfull = sfull + 1;             // one per TMEM slot
   uint64_t* tempty = tfull + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -470,7 +547,7 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const uint8_t* __r
     for (int s = 0; s < kBwStages; ++s) {
       mbar_init(&kvfull[s], 1);
       mbar_init(&krelu[s], kApReluThreads);
-      mbar_init(&kvempty[s], 1 + 128);
+      mbar_init(&kvempty[s], 2);
     }
     mbar_init(sfull, 1);
     for (int a = 0; a < 2; ++a) {
@@ -484,7 +561,10 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const uint8_t* __r
     tmem_alloc(tmem_holder, kBwTmemCols);
     tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) prefetch_tensormap(&tmap_kv);
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmap_kv);
+    prefetch_tensormap(&tmap_dqkv);
+  }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -532,19 +612,20 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const uint8_t* __r
     if (lane == 0 && sp.ntiles > 0 && mbar_wait(sfull, 0, abort_flag, err, kErrBwdKvMma | 8)) {
       constexpr uint32_t idesc_k = idesc_bf16_f32(128, kImageTRows, false, false);
       constexpr uint32_t idesc_v = idesc_bf16_f32(128, kImageRows, false, false);
-      int hc = 0;
+      int use[2] = {0, 0};
       bool stop = false;
       for (int i = 0; i < sp.ntiles && !stop; ++i) {
         const int s = i % kBwStages;
         if (!mbar_wait(&krelu[s], (i / kBwStages) & 1, abort_flag, err, kErrBwdKvMma | s)) break;
         tc_fence_after_sync();
         const uint32_t ka = smem_u32(ktile(s)), va = smem_u32(vtile(s));
-        for (int j = 0; j < sp.nh; ++j, ++hc) {
-          const int a = hc & 1;
-          if (hc >= 2 && !mbar_wait(&tempty[a], ((hc >> 1) - 1) & 1, abort_flag, err, kErrBwdKvMma | 4 | a)) {
+        for (int j = 0; j < sp.nh; ++j) {
+          const int a = j & 1;
+          if (use[a] > 0 && !mbar_wait(&tempty[a], (use[a] - 1) & 1, abort_flag, err, kErrBwdKvMma | 4 | a)) {
             stop = true;
             break;
           }
+          ++use[a];
           tc_fence_after_sync();
           const uint32_t off = (j >> 1) * kBwBoxBytes + (j & 1) * 64;
 #pragma unroll
@@ -552,9 +633,6 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const uint8_t* __r
             // dk~ (before the ones row) = v . dS[0:d]: A = v (K-major), B = the dS^T image
             umma_bf16(tmem + a * kBwSlotCols, smem_desc(va + off + ks * 32, 16, 1024, kSwizzle128B),
                       smem_desc(smem_u32(dtimg + j * kImageTBytes) + ks * 256, 128, 512, kSwizzleNone), idesc_k, ks);
-          }
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
             // dv = k~ . dS^T: A = k~ (K-major), B = the dS image (rows r)
             umma_bf16(tmem + a * kBwSlotCols + kImageTRows, smem_desc(ka + off + ks * 32, 16, 1024, kSwizzle128B),
                       smem_desc(smem_u32(dimg + j * kImageBytes) + ks * 256, 128, 512, kSwizzleNone), idesc_v, ks);
@@ -572,7 +650,7 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const uint8_t* __r
       const int s = i % kBwStages;
       if (!mbar_wait(&kvfull[s], (i / kBwStages) & 1, abort_flag, err, kErrBwdKvRelu | s)) break;
       uint8_t* st = ktile(s);
-#pragma unroll 4
+#pragma unroll 8
       for (int j = t; j < nchunks; j += kApReluThreads) {
         uint4* c = reinterpret_cast<uint4*>(st + j * 16);
         *c = relu_bf16x8(*c);
@@ -581,65 +659,108 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const uint8_t* __r
       mbar_arrive(&krelu[s]);
     }
   } else {
-    const int wq = warp & 3, row = wq * 32 + lane;
+    // epilogue: group g takes heads g, g + 2 through TMEM slot g; thread = token row (TMEM lane)
+    const int g = (warp - 4) >> 2, wq = warp & 3, row = wq * 32 + lane;
+    const int gbar = 1 + 2 * g;
+    float* zf = reinterpret_cast<float*>(smem + kBkOffZ);
     bool ok = sp.ntiles > 0 && mbar_wait(sfull, 0, abort_flag, err, kErrBwdKvEpi | 8);
-    int hc = 0;
+    if (ok && threadIdx.x < 256) ones_rows_fp32(dimg, sp.nh, zf, threadIdx.x - 128);
+    bar_sync(2, kBwEpiThreads);
+    // bf16 results of a whole tile are written over the k and v tiles they came from (each
+    // head's columns once its products are done and its mask is read) and stored with TMA:
+    // when the quad's heads fill whole boxes and the tile is whole or ends at N (a TMA store is
+    // clipped only at N).  Otherwise each thread stores its row.
+    const bool stage_ok = sizeof(OutT) == 2 && (sp.nh % 2) == 0;
+    const bool storer = threadIdx.x == 128;
+    int use = 0;
     for (int i = 0; ok && i < sp.ntiles; ++i) {
       const int s = i % kBwStages;
-      const int tok = sp.n0 + i * kApTile + row;
+      const int tok0 = sp.n0 + i * kApTile, tok = tok0 + row;
       const bool valid = tok < sp.n1;
-      const uint8_t* kt = ktile(s);
-      // the tile's TMA data (k~ is read here; the stage is refilled only after this thread's
-      // arrival on kvempty)
+      const bool staged = stage_ok && (tok0 + kApTile <= sp.n1 || sp.n1 == p.N);
+      uint8_t* kt = ktile(s);
+      uint8_t* vt = vtile(s);
+      // the tile's TMA data (k~ is read here; the stage is refilled only after its release)
       if (!mbar_wait(&kvfull[s], (i / kBwStages) & 1, abort_flag, err, kErrBwdKvEpi | 14)) ok = false;
-      if (bar_any(1, 128, !ok)) {
+      if (bar_any(2, kBwEpiThreads, !ok)) {
         ok = false;
         break;
       }
-      for (int j = 0; j < sp.nh; ++j, ++hc) {
-        const int a = hc & 1;
-        const bool okw = mbar_wait(&tfull[a], (hc >> 1) & 1, abort_flag, err, kErrBwdKvEpi | a);
-        if (bar_any(1, 128, !okw)) {
+      for (int j = g; j < sp.nh; j += 2) {
+        const bool okw = mbar_wait(&tfull[g], use & 1, abort_flag, err, kErrBwdKvEpi | g);
+        ++use;
+        if (bar_any(gbar, 128, !okw)) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
-        const uint32_t ta = tmem + (static_cast<uint32_t>(wq * 32) << 16) + a * kBwSlotCols;
-        const uint8_t* im = dimg + j * kImageBytes;
+        const uint32_t ta = tmem + (static_cast<uint32_t>(wq * 32) << 16) + g * kBwSlotCols;
+        const float4* z4 = reinterpret_cast<const float4*>(zf + j * kD);
+        const int64_t rowbase = ((int64_t)b * p.N + tok) * (3 * p.H * kD) + (quad * kApUnitHeads + j) * kD;
         float x[kD];
         {
           uint32_t v[kImageTRows];
 #pragma unroll
           for (int k = 0; k < kImageTRows / 16; ++k) tmem_ld_x16(ta + k * 16, v + k * 16);
           tmem_wait_ld();
-          float kr[kD];
+          // dk = relu'(k) * (v . dS[0:d] + dS[d]); relu(k) > 0 <=> its bf16 bits are not 0
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            unpack_bf16x8(*reinterpret_cast<const uint4*>(kt + sw_offset(row, j * kD + k * 8)), kr + 8 * k);
+          for (int k = 0; k < 4; ++k) {
+            const uint4 kw = *reinterpret_cast<const uint4*>(kt + sw_offset(row, j * kD + k * 8));
+            const float4 za = z4[2 * k], zb = z4[2 * k + 1];
+            const float z[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
 #pragma unroll
-          for (int c = 0; c < kD; ++c) {
-            const float z = bf16_at(im + image_offset(kD, c)) + bf16_at(im + image_offset(kImageLoRow + kD, c));
-            const float t = (__uint_as_float(v[c]) + __uint_as_float(v[kD + c])) + z;
-            x[c] = kr[c] > 0.f ? t : 0.f;
+            for (int e = 0; e < 8; ++e) {
+              const int c = 8 * k + e;
+              const float t = (__uint_as_float(v[c]) + __uint_as_float(v[kD + c])) + z[e];
+              x[c] = bf16_nonzero(kw, e) ? t : 0.f;
+            }
           }
         }
-        const int64_t rowbase = ((int64_t)b * p.N + tok) * (3 * p.H * kD) + (quad * kApUnitHeads + j) * kD;
-        if (valid) store_row32(dqkv + rowbase + p.H * kD, x);
+        if (staged) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<uint4*>(kt + sw_offset(row, j * kD + k * 8)) = pack_bf16x8(x + 8 * k);
+        } else if (valid) {
+          store_row32(dqkv + rowbase + p.H * kD, x);
+        }
         {
           uint32_t v[kImageRows];
 #pragma unroll
           for (int k = 0; k < kImageRows / 16; ++k) tmem_ld_x16(ta + kImageTRows + k * 16, v + k * 16);
           tmem_wait_ld();
+          tc_fence_before_sync();
+          mbar_arrive(&tempty[g]);
 #pragma unroll
           for (int r = 0; r < kD; ++r) x[r] = __uint_as_float(v[r]) + __uint_as_float(v[kImageLoRow + r]);
         }
-        tc_fence_before_sync();
-        mbar_arrive(&tempty[a]);
-        if (valid) store_row32(dqkv + rowbase + 2 * p.H * kD, x);
+        if (staged) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<uint4*>(vt + sw_offset(row, j * kD + k * 8)) = pack_bf16x8(x + 8 * k);
+        } else if (valid) {
+          store_row32(dqkv + rowbase + 2 * p.H * kD, x);
+        }
       }
-      if (!ok) break;
-      mbar_arrive(&kvempty[s]);   // this thread no longer reads the k tile
+      fence_proxy_async_smem();
+      if (bar_any(2, kBwEpiThreads, !ok)) {   // every epilogue thread has written its rows
+        ok = false;
+        break;
+      }
+      if (storer) {
+        if (staged) {
+          for (int h = 0; h < sp.np; ++h) {
+            const int x0 = quad * kApUnitHeads * kD + h * kApHeads * kD;
+            tma_store_3d(&tmap_dqkv, kt + h * kBwBoxBytes, p.H * kD + x0, tok0, b);
+            tma_store_3d(&tmap_dqkv, vt + h * kBwBoxBytes, 2 * p.H * kD + x0, tok0, b);
+          }
+          bulk_commit_group();
+          bulk_wait_group_read<0>();   // the stage may be refilled once the stores have read it
+        }
+        mbar_arrive(&kvempty[s]);
+      }
     }
+    if (storer) bulk_wait_group<0>();
   }
 
   tc_fence_before_sync();
