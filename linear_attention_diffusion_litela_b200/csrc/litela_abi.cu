@@ -101,14 +101,18 @@ litela_status device_setup(int* num_sms) {
 
 // 3-D view of the packed qkv buffer for TMA: (channel, token, batch), bf16, boxes of 64
 // channels x box_tokens tokens, 128-byte swizzle, zero fill outside the tensor.
-litela_status encode_qkv_map(const void* qkv, int B, int N, int H, int box_tokens, CUtensorMap* map) {
+// box_channels = 32 gives boxes of one head's 32 channels with 64-byte swizzle (the backward's
+// dq stores).
+litela_status encode_qkv_map(const void* qkv, int B, int N, int H, int box_tokens, CUtensorMap* map,
+                             int box_channels = 64) {
   const cuuint64_t row = 3ull * H * kD;
   const cuuint64_t dims[3] = {row, (cuuint64_t)N, (cuuint64_t)B};
   const cuuint64_t strides[2] = {row * 2, row * 2 * (cuuint64_t)N};
-  const cuuint32_t box[3] = {64, (cuuint32_t)box_tokens, 1};
+  const cuuint32_t box[3] = {(cuuint32_t)box_channels, (cuuint32_t)box_tokens, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(qkv), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        box_channels == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(LITELA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string((int)r) + ")");
   return LITELA_OK;
@@ -276,14 +280,14 @@ litela_status launch_reduce(const Plan& plan, const void* qkv, float* partials, 
 litela_status launch_scan(const Plan& plan, const float* partials, uint8_t* images, float* states, int num_sms,
                           cudaStream_t stream, bool pdl, const float* state_in = nullptr,
                           float* state_out = nullptr, uint8_t* images_t = nullptr, bool reverse = false,
-                          int chunks_per_block = 0) {
+                          int chunks_per_block = 0, bool rows64 = false, float* zrows = nullptr) {
   const int64_t work = ((int64_t)plan.B * plan.H * kStateFloats + kScanElems - 1) / kScanElems;
   int64_t grid = (work + kScanThreads - 1) / kScanThreads;
   if (grid > num_sms) grid = num_sms;
   TcPlan tp = tc_plan(plan, 0.f);
   if (chunks_per_block > 0) tp.cpb = chunks_per_block;   // partials of another chunking (the backward's)
   cudaError_t e = launch_ex(litela_state_scan, dim3((unsigned)grid), dim3(kScanThreads), 0, stream, pdl,
-                            partials, images, images_t, states, state_in, state_out, reverse, tp);
+                            partials, images, images_t, states, state_in, state_out, reverse, rows64, zrows, tp);
   if (e != cudaSuccess) return cuda_fail(e, "launch litela_state_scan");
   return LITELA_OK;
 }
@@ -459,11 +463,21 @@ litela_status run_bwd(const void* qkv, const void* dout, OutT* dqkv, int B, int 
   float* dpartials = reinterpret_cast<float*>(base + plan.off_dpartials);
   uint8_t* dimages = reinterpret_cast<uint8_t*>(base + plan.off_dimages);
   uint8_t* dimages_t = reinterpret_cast<uint8_t*>(base + plan.off_dimages_t);
+  float* dzrows = reinterpret_cast<float*>(base + plan.off_dzrows);
   CUtensorMap map_qkv, map_g;
   s = encode_qkv_map(qkv, B, N, H, kApTile, &map_qkv);
   if (s != LITELA_OK) return s;
   s = encode_out_map(static_cast<__nv_bfloat16*>(const_cast<void*>(dout)), B, N, H, &map_g);
   if (s != LITELA_OK) return s;
+  // TMA stores of dq (one head per box) and of dk, dv (head pairs) for bf16 output; the fp32
+  // output is written row by row and never uses these maps
+  CUtensorMap map_dq = map_qkv, map_dqkv = map_qkv;
+  if (sizeof(OutT) == 2) {
+    s = encode_qkv_map(dqkv, B, N, H, kApTile, &map_dq, 32);
+    if (s != LITELA_OK) return s;
+    s = encode_qkv_map(dqkv, B, N, H, kApTile, &map_dqkv);
+    if (s != LITELA_OK) return s;
+  }
   const bool pdl = events == nullptr;
   const BwdPlan bp{B, N, H, plan.T, plan.nblk, plan.nquads, plan.bwd_cpb, plan.bwd_chunk, eps};
   const dim3 grid((unsigned)(plan.nblk * plan.bwd_cpb), (unsigned)plan.nquads, (unsigned)B);
@@ -474,22 +488,17 @@ litela_status run_bwd(const void* qkv, const void* dout, OutT* dqkv, int B, int 
   s = launch_scan(plan, partials, images, nullptr, num_sms, stream, pdl, nullptr, nullptr, images_t, false);
   if (s != LITELA_OK) return s;
   if (events && (e = cudaEventRecord(events[1], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  e = launch_ex(litela_bwd_q_tc<OutT>, grid, dim3(kBwThreads), kBqSmemBytes, stream, pdl, map_qkv, map_g,
+  e = launch_ex(litela_bwd_q_tc<OutT>, grid, dim3(kBwThreads), kBqSmemBytes, stream, pdl, map_qkv, map_g, map_dq,
                 static_cast<const uint8_t*>(images), static_cast<const uint8_t*>(images_t), dpartials, dqkv, ws->err,
                 bp);
   if (e != cudaSuccess) return cuda_fail(e, "launch litela_bwd_q_tc");
   if (events && (e = cudaEventRecord(events[2], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   s = launch_scan(plan, dpartials, dimages, nullptr, num_sms, stream, pdl, nullptr, nullptr, dimages_t, true,
-                  plan.bwd_cpb);
+                  plan.bwd_cpb, true, dzrows);
   if (s != LITELA_OK) return s;
-  // TMA stores of dk, dv (bf16 output; the fp32 output is written row by row and never uses it)
-  CUtensorMap map_dqkv = map_qkv;
-  if (sizeof(OutT) == 2) {
-    s = encode_qkv_map(dqkv, B, N, H, kApTile, &map_dqkv);
-    if (s != LITELA_OK) return s;
-  }
   e = launch_ex(litela_bwd_kv_tc<OutT>, grid, dim3(kBwThreads), kBkSmemBytes, stream, pdl, map_qkv, map_dqkv,
-                static_cast<const uint8_t*>(dimages), static_cast<const uint8_t*>(dimages_t), dqkv, ws->err, bp);
+                static_cast<const uint8_t*>(dimages), static_cast<const uint8_t*>(dimages_t),
+                static_cast<const float*>(dzrows), dqkv, ws->err, bp);
   if (e != cudaSuccess) return cuda_fail(e, "launch litela_bwd_kv_tc");
   if (events && (e = cudaEventRecord(events[3], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   g_last_error.clear();

@@ -78,17 +78,31 @@ constexpr uint32_t kBqOffH = kBqOffGlo + kBwTileBytes;
 constexpr uint32_t kBqOffImg = kBqOffH + kBwHBytes;
 constexpr uint32_t kBqOffBars = kBqOffImg + kBwImgBytes;
 constexpr uint32_t kBqOffZ = kBqOffBars + 256;            // ones rows S[d] in fp32, [4][32]
-constexpr uint32_t kBqSmemBytes = kBqOffZ + 512 + 1024;
-// litela_bwd_kv_tc shared memory
-constexpr uint32_t kBkOffImg = kBwStages * kBwStageBytes;
-constexpr uint32_t kBkOffBars = kBkOffImg + kBwImgBytes;
-constexpr uint32_t kBkOffZ = kBkOffBars + 256;            // ones rows dS[d] in fp32, [4][32]
-constexpr uint32_t kBkSmemBytes = kBkOffZ + 512 + 1024;
+constexpr uint32_t kDqBoxBytes = kApTile * 64;            // one head's dq: 128 tokens x 32 channels
+constexpr uint32_t kBqOffDq = (kBqOffZ + 512 + 1023) / 1024 * 1024;   // a staging box per group
+constexpr uint32_t kBqSmemBytes = kBqOffDq + 2 * kDqBoxBytes + 1024;
+// litela_bwd_kv_tc: 3 stages; the dS images hold rows 0..31 only (hi rows 0..31, lo rows 32..63)
+// and the ones row dS[d] comes in fp32
+constexpr int kBkStages = 3;
+constexpr uint32_t kBkSlotCols = 2 * kImageTRows;          // dk~ (hi | lo) + dv (hi | lo)
+constexpr uint32_t kBkOffImg = kBkStages * kBwStageBytes;
+constexpr uint32_t kBkOffZ = kBkOffImg + kApUnitHeads * 2 * kImageTBytes;   // [4][32] fp32
+constexpr uint32_t kBkOffBars = kBkOffZ + 512;
+constexpr uint32_t kBkSmemBytes = kBkOffBars + 256 + 1024;
+
+static_assert(kBqSmemBytes <= 232448 && kBkSmemBytes <= 232448, "shared memory above the 227 KB per-block limit");
+static_assert(2 * kBwSlotCols + 128 + 16 <= kBwTmemCols && 2 * kBkSlotCols <= kBwTmemCols, "TMEM columns");
 
 // byte offset of bf16 element (token t, channel ch of the 4 heads) in a tile of two 128B-swizzled
 // TMA boxes (64 channels x 128 tokens each)
 __device__ __forceinline__ uint32_t sw_offset(int t, int ch) {
   return (uint32_t)((ch >> 6) * kBwBoxBytes + t * 128 + ((((ch >> 3) & 7) ^ (t & 7)) << 4) + (ch & 7) * 2);
+}
+
+// byte offset of bf16 element (token t, channel c < 32) in a 64B-swizzled TMA box of 32 channels
+// x 128 tokens (16-byte chunk c/8 of row t sits at chunk (c/8) ^ ((t/2) & 3))
+__device__ __forceinline__ uint32_t sw64_offset(int t, int c) {
+  return (uint32_t)(t * 64 + ((((c >> 3) & 3) ^ ((t >> 1) & 3)) << 4) + (c & 7) * 2);
 }
 
 // byte offset of element (column j, token t) in the 16-column K-major tile of the h values
@@ -161,7 +175,8 @@ __device__ __forceinline__ BwSpan bw_span(const BwdPlan& p) {
 template <typename OutT>
 __global__ void __launch_bounds__(kBwThreads, 1)
 litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_g,
-                const uint8_t* __restrict__ images, const uint8_t* __restrict__ images_t,
+                const __grid_constant__ CUtensorMap tmap_dq, const uint8_t* __restrict__ images,
+                const uint8_t* __restrict__ images_t,
                 float* __restrict__ dpartials, OutT* __restrict__ dqkv, int* __restrict__ err, BwdPlan p) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
@@ -217,6 +232,7 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmap_q);
     prefetch_tensormap(&tmap_g);
+    prefetch_tensormap(&tmap_dq);
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -364,14 +380,19 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     const int g = (warp - 4) >> 2, wq = warp & 3, row = wq * 32 + lane;
     const int gbar = 1 + 2 * g;   // the group's named barrier (1 or 3)
     float* zf = reinterpret_cast<float*>(smem + kBqOffZ);
+    // bf16 dq of a whole tile (or of the tile that ends at N) is staged in the group's box and
+    // stored with TMA by the group's first thread; otherwise each thread stores its row
+    uint8_t* dqbuf = smem + kBqOffDq + g * kDqBoxBytes;
+    const bool storer = lane == 0 && wq == 0;
     bool ok = sp.ntiles > 0 && mbar_wait(sfull, 0, abort_flag, err, kErrBwdQEpi | 8);
     if (ok && threadIdx.x < 256) ones_rows_fp32(simg, sp.nh, zf, threadIdx.x - 128);
     bar_sync(2, kBwEpiThreads);
     int use = 0;
     for (int i = 0; ok && i < sp.ntiles; ++i) {
       const int s = i % kBwStages;
-      const int tok = sp.n0 + i * kApTile + row;
+      const int tok0 = sp.n0 + i * kApTile, tok = tok0 + row;
       const bool valid = tok < sp.n1;
+      const bool staged = sizeof(OutT) == 2 && (tok0 + kApTile <= sp.n1 || sp.n1 == p.N);
       // the tile's TMA data (this thread reads dout and q~ from it; the stage cannot be refilled
       // before this epilogue releases it)
       if (!mbar_wait(&qfull[s], (i / kBwStages) & 1, abort_flag, err, kErrBwdQEpi | 14)) ok = false;
@@ -383,6 +404,7 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       for (int j = g; j < sp.nh; j += 2) {
         const bool okw = mbar_wait(&tfull[g], use & 1, abort_flag, err, kErrBwdQEpi | g);
         ++use;
+        if (storer) bulk_wait_group_read<0>();   // the group's previous dq store has read its box
         if (bar_any(gbar, 128, !okw)) {
           ok = false;
           break;
@@ -435,7 +457,18 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
             dq[c] = bf16_nonzero(qw, e) ? fmaf(z[e], h, t) : 0.f;
           }
         }
-        if (valid) store_row32(dqkv + ((int64_t)b * p.N + tok) * (3 * p.H * kD) + (quad * kApUnitHeads + j) * kD, dq);
+        if (staged) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) *reinterpret_cast<uint4*>(dqbuf + sw64_offset(row, 8 * k)) = pack_bf16x8(dq + 8 * k);
+          fence_proxy_async_smem();
+          bar_sync(gbar, 128);
+          if (storer) {
+            tma_store_3d(&tmap_dq, dqbuf, (quad * kApUnitHeads + j) * kD, tok0, b);
+            bulk_commit_group();
+          }
+        } else if (valid) {
+          store_row32(dqkv + ((int64_t)b * p.N + tok) * (3 * p.H * kD) + (quad * kApUnitHeads + j) * kD, dq);
+        }
         // the previous tile's dS product has read glo and hbuf (the columns of other heads of
         // the g tile are not touched below)
         if (first && i > 0) {
@@ -476,6 +509,7 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       fence_proxy_async_smem();
       mbar_arrive(gready);
     }
+    if (storer) bulk_wait_group<0>();
     // the CTA's partial dS (group 0): warp quarter wq holds head wq's query channels (TMEM lanes)
     if (g == 0) {
       float sv[kRows];
@@ -520,17 +554,18 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
 template <typename OutT>
 __global__ void __launch_bounds__(kBwThreads, 1)
 litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant__ CUtensorMap tmap_dqkv,
-                 const uint8_t* __restrict__ dimages, const uint8_t* __restrict__ dimages_t, OutT* __restrict__ dqkv,
-                 int* __restrict__ err, BwdPlan p) {
+                 const uint8_t* __restrict__ dimages, const uint8_t* __restrict__ dimages_t,
+                 const float* __restrict__ dzrows, OutT* __restrict__ dqkv, int* __restrict__ err, BwdPlan p) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* dimg = smem + kBkOffImg;   // 4 dS images, then 4 dS^T images
-  uint8_t* dtimg = dimg + kApUnitHeads * kImageBytes;
+  uint8_t* dimg = smem + kBkOffImg;   // 4 dS images (rows r), then 4 dS^T images (rows c)
+  uint8_t* dtimg = dimg + kApUnitHeads * kImageTBytes;
+  float* zf = reinterpret_cast<float*>(smem + kBkOffZ);   // dS[d] of the 4 heads
   uint64_t* kvfull = reinterpret_cast<uint64_t*>(smem + kBkOffBars);
-  uint64_t* krelu = kvfull + kBwStages;
-  uint64_t* kvempty = krelu + kBwStages;   // the MMAs' commit + the epilogue's storing thread
-  uint64_t* sfull = kvempty + kBwStages;
+  uint64_t* krelu = kvfull + kBkStages;
+  uint64_t* kvempty = krelu + kBkStages;   // the MMAs' commit + the epilogue's storing thread
+  uint64_t* sfull = kvempty + kBkStages;
   uint64_t* tfull = sfull + 1;             // one per TMEM slot
   uint64_t* tempty = tfull + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
@@ -544,7 +579,7 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
 
   pdl_launch_dependents();
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kBwStages; ++s) {
+    for (int s = 0; s < kBkStages; ++s) {
       mbar_init(&kvfull[s], 1);
       mbar_init(&krelu[s], kApReluThreads);
       mbar_init(&kvempty[s], 2);
@@ -573,7 +608,7 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
   if (warp == 0) {
     if (lane == 0) {
       auto load = [&](int i) {
-        const int s = i % kBwStages;
+        const int s = i % kBkStages;
         const int y = sp.n0 + i * kApTile;
         mbar_arrive_expect_tx(&kvfull[s], 2 * sp.np * kBwBoxBytes);
         for (int h = 0; h < sp.np; ++h) {
@@ -582,41 +617,41 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
           tma_load_3d(vtile(s) + h * kBwBoxBytes, &tmap_kv, &kvfull[s], 2 * p.H * kD + x, y, b);
         }
       };
-      const int pre = sp.ntiles < kBwStages ? sp.ntiles : kBwStages;
+      const int pre = sp.ntiles < kBkStages ? sp.ntiles : kBkStages;
       for (int i = 0; i < pre; ++i) load(i);   // inputs: see litela_bwd_q_tc
       int issued = pre;
       bool images_loaded = false;
       pdl_wait_primary();   // the dS images come from the preceding scan
       if (sp.ntiles > 0) {
-        mbar_arrive_expect_tx(sfull, sp.nh * (kImageBytes + kImageTBytes));
+        mbar_arrive_expect_tx(sfull, sp.nh * (2 * kImageTBytes + kD * 4));
         for (int j = 0; j < sp.nh; ++j) {
           const int64_t im = ((int64_t)b * p.H + quad * kApUnitHeads + j) * p.nblk + sp.blk;
-          bulk_load(dimg + j * kImageBytes, dimages + im * kImageBytes, kImageBytes, sfull);
+          bulk_load(dimg + j * kImageTBytes, dimages + im * kImageTBytes, kImageTBytes, sfull);
           bulk_load(dtimg + j * kImageTBytes, dimages_t + im * kImageTBytes, kImageTBytes, sfull);
+          bulk_load(zf + j * kD, dzrows + im * kD, kD * 4, sfull);
         }
         images_loaded = true;
       }
       for (int i = pre; i < sp.ntiles; ++i) {
-        const int s = i % kBwStages;
-        if (!mbar_wait(&kvempty[s], ((i / kBwStages) - 1) & 1, abort_flag, err, kErrBwdKvProducer | s)) break;
+        const int s = i % kBkStages;
+        if (!mbar_wait(&kvempty[s], ((i / kBkStages) - 1) & 1, abort_flag, err, kErrBwdKvProducer | s)) break;
         load(i);
         issued = i + 1;
       }
       if (*abort_flag) {
-        for (int i = (issued > kBwStages ? issued - kBwStages : 0); i < issued; ++i)
-          mbar_drain(&kvfull[i % kBwStages], (i / kBwStages) & 1);
+        for (int i = (issued > kBkStages ? issued - kBkStages : 0); i < issued; ++i)
+          mbar_drain(&kvfull[i % kBkStages], (i / kBkStages) & 1);
         if (images_loaded) mbar_drain(sfull, 0);
       }
     }
   } else if (warp == 1) {
     if (lane == 0 && sp.ntiles > 0 && mbar_wait(sfull, 0, abort_flag, err, kErrBwdKvMma | 8)) {
-      constexpr uint32_t idesc_k = idesc_bf16_f32(128, kImageTRows, false, false);
-      constexpr uint32_t idesc_v = idesc_bf16_f32(128, kImageRows, false, false);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, kImageTRows, false, false);
       int use[2] = {0, 0};
       bool stop = false;
       for (int i = 0; i < sp.ntiles && !stop; ++i) {
-        const int s = i % kBwStages;
-        if (!mbar_wait(&krelu[s], (i / kBwStages) & 1, abort_flag, err, kErrBwdKvMma | s)) break;
+        const int s = i % kBkStages;
+        if (!mbar_wait(&krelu[s], (i / kBkStages) & 1, abort_flag, err, kErrBwdKvMma | s)) break;
         tc_fence_after_sync();
         const uint32_t ka = smem_u32(ktile(s)), va = smem_u32(vtile(s));
         for (int j = 0; j < sp.nh; ++j) {
@@ -631,11 +666,11 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
 #pragma unroll
           for (int ks = 0; ks < 2; ++ks) {
             // dk~ (before the ones row) = v . dS[0:d]: A = v (K-major), B = the dS^T image
-            umma_bf16(tmem + a * kBwSlotCols, smem_desc(va + off + ks * 32, 16, 1024, kSwizzle128B),
-                      smem_desc(smem_u32(dtimg + j * kImageTBytes) + ks * 256, 128, 512, kSwizzleNone), idesc_k, ks);
-            // dv = k~ . dS^T: A = k~ (K-major), B = the dS image (rows r)
-            umma_bf16(tmem + a * kBwSlotCols + kImageTRows, smem_desc(ka + off + ks * 32, 16, 1024, kSwizzle128B),
-                      smem_desc(smem_u32(dimg + j * kImageBytes) + ks * 256, 128, 512, kSwizzleNone), idesc_v, ks);
+            umma_bf16(tmem + a * kBkSlotCols, smem_desc(va + off + ks * 32, 16, 1024, kSwizzle128B),
+                      smem_desc(smem_u32(dtimg + j * kImageTBytes) + ks * 256, 128, 512, kSwizzleNone), idesc, ks);
+            // dv = k~ . dS[0:d]^T: A = k~ (K-major), B = the dS image (rows r)
+            umma_bf16(tmem + a * kBkSlotCols + kImageTRows, smem_desc(ka + off + ks * 32, 16, 1024, kSwizzle128B),
+                      smem_desc(smem_u32(dimg + j * kImageTBytes) + ks * 256, 128, 512, kSwizzleNone), idesc, ks);
           }
           umma_commit(&tfull[a]);
         }
@@ -647,8 +682,8 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
     const int t = threadIdx.x - 64;
     const int nchunks = sp.np * (int)(kBwBoxBytes / 16);
     for (int i = 0; i < sp.ntiles; ++i) {
-      const int s = i % kBwStages;
-      if (!mbar_wait(&kvfull[s], (i / kBwStages) & 1, abort_flag, err, kErrBwdKvRelu | s)) break;
+      const int s = i % kBkStages;
+      if (!mbar_wait(&kvfull[s], (i / kBkStages) & 1, abort_flag, err, kErrBwdKvRelu | s)) break;
       uint8_t* st = ktile(s);
 #pragma unroll 8
       for (int j = t; j < nchunks; j += kApReluThreads) {
@@ -662,10 +697,7 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
     // epilogue: group g takes heads g, g + 2 through TMEM slot g; thread = token row (TMEM lane)
     const int g = (warp - 4) >> 2, wq = warp & 3, row = wq * 32 + lane;
     const int gbar = 1 + 2 * g;
-    float* zf = reinterpret_cast<float*>(smem + kBkOffZ);
     bool ok = sp.ntiles > 0 && mbar_wait(sfull, 0, abort_flag, err, kErrBwdKvEpi | 8);
-    if (ok && threadIdx.x < 256) ones_rows_fp32(dimg, sp.nh, zf, threadIdx.x - 128);
-    bar_sync(2, kBwEpiThreads);
     // bf16 results of a whole tile are written over the k and v tiles they came from (each
     // head's columns once its products are done and its mask is read) and stored with TMA:
     // when the quad's heads fill whole boxes and the tile is whole or ends at N (a TMA store is
@@ -674,14 +706,14 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
     const bool storer = threadIdx.x == 128;
     int use = 0;
     for (int i = 0; ok && i < sp.ntiles; ++i) {
-      const int s = i % kBwStages;
+      const int s = i % kBkStages;
       const int tok0 = sp.n0 + i * kApTile, tok = tok0 + row;
       const bool valid = tok < sp.n1;
       const bool staged = stage_ok && (tok0 + kApTile <= sp.n1 || sp.n1 == p.N);
       uint8_t* kt = ktile(s);
       uint8_t* vt = vtile(s);
       // the tile's TMA data (k~ is read here; the stage is refilled only after its release)
-      if (!mbar_wait(&kvfull[s], (i / kBwStages) & 1, abort_flag, err, kErrBwdKvEpi | 14)) ok = false;
+      if (!mbar_wait(&kvfull[s], (i / kBkStages) & 1, abort_flag, err, kErrBwdKvEpi | 14)) ok = false;
       if (bar_any(2, kBwEpiThreads, !ok)) {
         ok = false;
         break;
@@ -694,7 +726,7 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
           break;
         }
         tc_fence_after_sync();
-        const uint32_t ta = tmem + (static_cast<uint32_t>(wq * 32) << 16) + g * kBwSlotCols;
+        const uint32_t ta = tmem + (static_cast<uint32_t>(wq * 32) << 16) + g * kBkSlotCols;
         const float4* z4 = reinterpret_cast<const float4*>(zf + j * kD);
         const int64_t rowbase = ((int64_t)b * p.N + tok) * (3 * p.H * kD) + (quad * kApUnitHeads + j) * kD;
         float x[kD];
@@ -725,14 +757,14 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
           store_row32(dqkv + rowbase + p.H * kD, x);
         }
         {
-          uint32_t v[kImageRows];
+          uint32_t v[kImageTRows];
 #pragma unroll
-          for (int k = 0; k < kImageRows / 16; ++k) tmem_ld_x16(ta + kImageTRows + k * 16, v + k * 16);
+          for (int k = 0; k < kImageTRows / 16; ++k) tmem_ld_x16(ta + kImageTRows + k * 16, v + k * 16);
           tmem_wait_ld();
           tc_fence_before_sync();
           mbar_arrive(&tempty[g]);
 #pragma unroll
-          for (int r = 0; r < kD; ++r) x[r] = __uint_as_float(v[r]) + __uint_as_float(v[kImageLoRow + r]);
+          for (int r = 0; r < kD; ++r) x[r] = __uint_as_float(v[r]) + __uint_as_float(v[kD + r]);
         }
         if (staged) {
 #pragma unroll

@@ -59,9 +59,10 @@ struct Plan {
   // backward (make_bwd_plan): the forward's reduction and scan (partials, images above), then
   //   S^T images bf16 [B][H][nblk][kImageTBytes]                       at off_images_t
   //   dS partials fp32 [B][nquads][nblk * bwd_cpb][4][33][32]           at off_dpartials
-  //   dS images [B][H][nblk][kImageBytes], dS^T images (kImageTBytes)   at off_dimages, off_dimages_t
+  //   dS images, rows 0..d-1 [B][H][nblk][kImageTBytes], dS^T images (the same size) and the
+  //   ones rows dS[d] fp32 [B][H][nblk][d]                  at off_dimages, off_dimages_t, off_dzrows
   int bwd_cpb = 0, bwd_chunk = 0;   // CTAs per (batch, quad, block); tokens per CTA (multiple of 128)
-  size_t off_images_t = 0, off_dpartials = 0, off_dimages = 0, off_dimages_t = 0, bwd_bytes = 0;
+  size_t off_images_t = 0, off_dpartials = 0, off_dimages = 0, off_dimages_t = 0, off_dzrows = 0, bwd_bytes = 0;
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -123,13 +124,14 @@ inline void make_bwd_plan(int num_sms, Plan* p) {
   p->bwd_chunk = (int)chunk;
   p->bwd_cpb = (int)((p->T + chunk - 1) / chunk);
   const size_t img_t = (size_t)p->B * p->H * p->nblk * kImageTBytes;
-  const size_t img = (size_t)p->B * p->H * p->nblk * kImageBytes;
+  const size_t zrows = (size_t)p->B * p->H * p->nblk * kD * sizeof(float);
   const size_t dpart = (size_t)segs * p->bwd_cpb * kRedHeads * kStateFloats * sizeof(float);
   p->off_images_t = align_up(p->bytes, 256);
   p->off_dpartials = p->off_images_t + align_up(img_t, 256);
   p->off_dimages = p->off_dpartials + align_up(dpart, 256);
-  p->off_dimages_t = p->off_dimages + align_up(img, 256);
-  p->bwd_bytes = p->off_dimages_t + align_up(img_t, 256);
+  p->off_dimages_t = p->off_dimages + align_up(img_t, 256);
+  p->off_dzrows = p->off_dimages_t + align_up(img_t, 256);
+  p->bwd_bytes = p->off_dzrows + align_up(zrows, 256);
 }
 
 }  // namespace litela

@@ -288,7 +288,9 @@ __device__ __forceinline__ const float* partial_ptr(const float* partials, const
 // `images_t` is not null also as the transposed image of its first 32 rows (rows c: hi 0..31,
 // lo 32..63, K = r; the B operand of products with S[0:32]^T), and, when `states` is not null,
 // as fp32 [B][H][nblk][33][32].  With `reverse` the blocks are visited last to first, giving
-// the inclusive SUFFIX sums over blocks (the gradient of a prefix-summed state).  `state_in` (fp32 [B][H][33][32], may be
+// the inclusive SUFFIX sums over blocks (the gradient of a prefix-summed state).  With `rows64`
+// the images hold only rows 0..31 (hi rows 0..31, lo rows 32..63: kImageTBytes each, no zero
+// rows) and row 32 goes to `zrows` in fp32 ([B][H][nblk][32]).  `state_in` (fp32 [B][H][33][32], may be
 // null) is a state carried from earlier chunks of the sequence and starts every prefix;
 // `state_out` (may be null, may alias state_in) receives the final prefix.  Grid-stride over the state elements
 // with at most one small CTA per SM: its CTAs launch early as a programmatic dependent of the
@@ -301,7 +303,7 @@ constexpr int kScanElems = 2;         // state elements per thread and round
 __global__ void __launch_bounds__(kScanThreads)
 litela_state_scan(const float* __restrict__ partials, uint8_t* __restrict__ images, uint8_t* __restrict__ images_t,
                   float* __restrict__ states, const float* __restrict__ state_in, float* __restrict__ state_out,
-                  bool reverse, TcPlan p) {
+                  bool reverse, bool rows64, float* __restrict__ zrows, TcPlan p) {
   using namespace sm100;
   pdl_launch_dependents();
   const int64_t stride = (int64_t)gridDim.x * kScanThreads;
@@ -309,7 +311,7 @@ litela_state_scan(const float* __restrict__ partials, uint8_t* __restrict__ imag
   // the partials come from the reduction grid; the images may be read by the previous call's
   // apply until that grid (which waited for it) is done
   pdl_wait_primary();
-  if (images != nullptr) {   // zero rows of every image
+  if (images != nullptr && !rows64) {   // zero rows of every image
     const int64_t nz = (int64_t)p.B * p.H * p.nblk * kScanZeros;
     for (int64_t i = tid; i < nz; i += stride) {
       const int64_t im = i / kScanZeros;
@@ -364,17 +366,24 @@ litela_state_scan(const float* __restrict__ partials, uint8_t* __restrict__ imag
             run[j] += sum[j];
             sum[j] = 0.f;
             const int r = e[j] >> 5, c = e[j] & 31;
-            if (images != nullptr) {
-              uint8_t* img = images + (bh[j] * p.nblk + blk) * kImageBytes;
-              const __nv_bfloat16 hi = __float2bfloat16_rn(run[j]);
-              const __nv_bfloat16 lo = __float2bfloat16_rn(run[j] - __bfloat162float(hi));
+            const __nv_bfloat16 hi = __float2bfloat16_rn(run[j]);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(run[j] - __bfloat162float(hi));
+            const int64_t im = bh[j] * p.nblk + blk;
+            if (images != nullptr && !rows64) {
+              uint8_t* img = images + im * kImageBytes;
               *reinterpret_cast<__nv_bfloat16*>(img + image_offset(r, c)) = hi;
               *reinterpret_cast<__nv_bfloat16*>(img + image_offset(kImageLoRow + r, c)) = lo;
-              if (images_t != nullptr && r < kD) {
-                uint8_t* imt = images_t + (bh[j] * p.nblk + blk) * kImageTBytes;
-                *reinterpret_cast<__nv_bfloat16*>(imt + image_offset(c, r)) = hi;
-                *reinterpret_cast<__nv_bfloat16*>(imt + image_offset(kD + c, r)) = lo;
-              }
+            }
+            if (images != nullptr && rows64 && r < kD) {
+              uint8_t* img = images + im * kImageTBytes;
+              *reinterpret_cast<__nv_bfloat16*>(img + image_offset(r, c)) = hi;
+              *reinterpret_cast<__nv_bfloat16*>(img + image_offset(kD + r, c)) = lo;
+            }
+            if (zrows != nullptr && r == kD) zrows[im * kD + c] = run[j];
+            if (images_t != nullptr && r < kD) {
+              uint8_t* imt = images_t + im * kImageTBytes;
+              *reinterpret_cast<__nv_bfloat16*>(imt + image_offset(c, r)) = hi;
+              *reinterpret_cast<__nv_bfloat16*>(imt + image_offset(kD + c, r)) = lo;
             }
             if (states != nullptr) states[(bh[j] * p.nblk + blk) * kStateFloats + e[j]] = run[j];
           }
