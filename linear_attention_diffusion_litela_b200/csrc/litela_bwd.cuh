@@ -186,8 +186,8 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
   uint8_t* simg = smem + kBqOffImg;   // 4 S images, then 4 S^T images
   uint8_t* stimg = simg + kApUnitHeads * kImageBytes;
   uint64_t* qfull = reinterpret_cast<uint64_t*>(smem + kBqOffBars);
-  uint64_t* qrelu = qfull + kBwStages;
-  uint64_t* qempty = qrelu + kBwStages;
+  uint64_t* qrelu = qfull + kBwStages;        // [stage][box]: ReLU done for head pair `box`
+  uint64_t* qempty = qrelu + 2 * kBwStages;
   uint64_t* sfull = qempty + kBwStages;
   uint64_t* tfull = sfull + 1;                 // one per TMEM slot
   uint64_t* tempty = tfull + 2;
@@ -207,7 +207,8 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
   if (threadIdx.x == 0) {
     for (int s = 0; s < kBwStages; ++s) {
       mbar_init(&qfull[s], 1);
-      mbar_init(&qrelu[s], kApReluThreads);
+      mbar_init(&qrelu[2 * s], kApReluThreads);
+      mbar_init(&qrelu[2 * s + 1], kApReluThreads);
       mbar_init(&qempty[s], 1);
     }
     mbar_init(sfull, 1);
@@ -321,7 +322,8 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
           t_idle = globaltimer_ns();
           continue;
         }
-        if (!(hnext < sp.ntiles && hnext <= dnext + 1 && mbar_test(&qrelu[hnext % kBwStages], (hnext / kBwStages) & 1))) {
+        if (!(hnext < sp.ntiles && hnext <= dnext + 1 &&
+              mbar_test(&qrelu[2 * (hnext % kBwStages)], (hnext / kBwStages) & 1))) {
           if (*abort_flag) break;
           if (globaltimer_ns() - t_idle > kWaitLimitNs) {
             *abort_flag = 1;
@@ -336,6 +338,10 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         const uint32_t qa = smem_u32(qtile(s)), ga = smem_u32(gtile(s));
         for (int j = 0; j < sp.nh; ++j) {
           const int a = j & 1;   // the slot of epilogue group j % 2
+          if (j == kApHeads && !mbar_wait(&qrelu[2 * s + 1], (i / kBwStages) & 1, abort_flag, err, kErrBwdQMma | 3)) {
+            stop = true;
+            break;
+          }
           if (use[a] > 0 && !mbar_wait(&tempty[a], (use[a] - 1) & 1, abort_flag, err, kErrBwdQMma | 4 | a)) {
             stop = true;
             break;
@@ -360,20 +366,22 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       umma_commit(dsfull);
     }
   } else if (warp < 4) {
-    // ReLU of the q tiles in place (the raw dout tile is not touched)
+    // ReLU of the q tiles in place (the raw dout tile is not touched), one head-pair box at a
+    // time so that the first pair's products can start early
     const int t = threadIdx.x - 64;
-    const int nchunks = sp.np * (int)(kBwBoxBytes / 16);
     for (int i = 0; i < sp.ntiles; ++i) {
       const int s = i % kBwStages;
       if (!mbar_wait(&qfull[s], (i / kBwStages) & 1, abort_flag, err, kErrBwdQRelu | s)) break;
-      uint8_t* st = qtile(s);
+      for (int h = 0; h < sp.np; ++h) {
+        uint8_t* st = qtile(s) + h * kBwBoxBytes;
 #pragma unroll 8
-      for (int j = t; j < nchunks; j += kApReluThreads) {
-        uint4* c = reinterpret_cast<uint4*>(st + j * 16);
-        *c = relu_bf16x8(*c);
+        for (int j = t; j < (int)(kBwBoxBytes / 16); j += kApReluThreads) {
+          uint4* c = reinterpret_cast<uint4*>(st + j * 16);
+          *c = relu_bf16x8(*c);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&qrelu[2 * s + h]);
       }
-      fence_proxy_async_smem();
-      mbar_arrive(&qrelu[s]);
     }
   } else {
     // epilogue: group g takes heads g, g + 2 through TMEM slot g; thread = token row (TMEM lane)
@@ -563,8 +571,8 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
   uint8_t* dtimg = dimg + kApUnitHeads * kImageTBytes;
   float* zf = reinterpret_cast<float*>(smem + kBkOffZ);   // dS[d] of the 4 heads
   uint64_t* kvfull = reinterpret_cast<uint64_t*>(smem + kBkOffBars);
-  uint64_t* krelu = kvfull + kBkStages;
-  uint64_t* kvempty = krelu + kBkStages;   // the MMAs' commit + the epilogue's storing thread
+  uint64_t* krelu = kvfull + kBkStages;        // [stage][box]: ReLU done for head pair `box`
+  uint64_t* kvempty = krelu + 2 * kBkStages;   // the MMAs' commit + the epilogue's storing thread
   uint64_t* sfull = kvempty + kBkStages;
   uint64_t* tfull = sfull + 1;             // one per TMEM slot
   uint64_t* tempty = tfull + 2;
@@ -581,7 +589,8 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
   if (threadIdx.x == 0) {
     for (int s = 0; s < kBkStages; ++s) {
       mbar_init(&kvfull[s], 1);
-      mbar_init(&krelu[s], kApReluThreads);
+      mbar_init(&krelu[2 * s], kApReluThreads);
+      mbar_init(&krelu[2 * s + 1], kApReluThreads);
       mbar_init(&kvempty[s], 2);
     }
     mbar_init(sfull, 1);
@@ -651,11 +660,15 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
       bool stop = false;
       for (int i = 0; i < sp.ntiles && !stop; ++i) {
         const int s = i % kBkStages;
-        if (!mbar_wait(&krelu[s], (i / kBkStages) & 1, abort_flag, err, kErrBwdKvMma | s)) break;
+        if (!mbar_wait(&krelu[2 * s], (i / kBkStages) & 1, abort_flag, err, kErrBwdKvMma | s)) break;
         tc_fence_after_sync();
         const uint32_t ka = smem_u32(ktile(s)), va = smem_u32(vtile(s));
         for (int j = 0; j < sp.nh; ++j) {
           const int a = j & 1;
+          if (j == kApHeads && !mbar_wait(&krelu[2 * s + 1], (i / kBkStages) & 1, abort_flag, err, kErrBwdKvMma | 3)) {
+            stop = true;
+            break;
+          }
           if (use[a] > 0 && !mbar_wait(&tempty[a], (use[a] - 1) & 1, abort_flag, err, kErrBwdKvMma | 4 | a)) {
             stop = true;
             break;
@@ -679,19 +692,21 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
       }
     }
   } else if (warp < 4) {
+    // ReLU of the k tiles in place, one head-pair box at a time
     const int t = threadIdx.x - 64;
-    const int nchunks = sp.np * (int)(kBwBoxBytes / 16);
     for (int i = 0; i < sp.ntiles; ++i) {
       const int s = i % kBkStages;
       if (!mbar_wait(&kvfull[s], (i / kBkStages) & 1, abort_flag, err, kErrBwdKvRelu | s)) break;
-      uint8_t* st = ktile(s);
+      for (int h = 0; h < sp.np; ++h) {
+        uint8_t* st = ktile(s) + h * kBwBoxBytes;
 #pragma unroll 8
-      for (int j = t; j < nchunks; j += kApReluThreads) {
-        uint4* c = reinterpret_cast<uint4*>(st + j * 16);
-        *c = relu_bf16x8(*c);
+        for (int j = t; j < (int)(kBwBoxBytes / 16); j += kApReluThreads) {
+          uint4* c = reinterpret_cast<uint4*>(st + j * 16);
+          *c = relu_bf16x8(*c);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&krelu[2 * s + h]);
       }
-      fence_proxy_async_smem();
-      mbar_arrive(&krelu[s]);
     }
   } else {
     // epilogue: group g takes heads g, g + 2 through TMEM slot g; thread = token row (TMEM lane)
@@ -704,6 +719,7 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
     // clipped only at N).  Otherwise each thread stores its row.
     const bool stage_ok = sizeof(OutT) == 2 && (sp.nh % 2) == 0;
     const bool storer = threadIdx.x == 128;
+    int pending = -1;   // (storer) stage whose TMA stores may still be reading it
     int use = 0;
     for (int i = 0; ok && i < sp.ntiles; ++i) {
       const int s = i % kBkStages;
@@ -780,6 +796,8 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
         break;
       }
       if (storer) {
+        // a stage is released (kvempty) once the stores out of it have read it; that wait is
+        // deferred by one tile so that the epilogue goes on with the next tile meanwhile
         if (staged) {
           for (int h = 0; h < sp.np; ++h) {
             const int x0 = quad * kApUnitHeads * kD + h * kApHeads * kD;
@@ -787,12 +805,25 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
             tma_store_3d(&tmap_dqkv, vt + h * kBwBoxBytes, 2 * p.H * kD + x0, tok0, b);
           }
           bulk_commit_group();
-          bulk_wait_group_read<0>();   // the stage may be refilled once the stores have read it
+          if (pending >= 0) {
+            bulk_wait_group_read<1>();
+            mbar_arrive(&kvempty[pending]);
+          }
+          pending = s;
+        } else {
+          if (pending >= 0) {
+            bulk_wait_group_read<0>();
+            mbar_arrive(&kvempty[pending]);
+            pending = -1;
+          }
+          mbar_arrive(&kvempty[s]);
         }
-        mbar_arrive(&kvempty[s]);
       }
     }
-    if (storer) bulk_wait_group<0>();
+    if (storer) {
+      bulk_wait_group<0>();
+      if (pending >= 0) mbar_arrive(&kvempty[pending]);
+    }
   }
 
   tc_fence_before_sync();
