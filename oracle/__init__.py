@@ -14,3 +14,8 @@ from .litela_bwd_oracle import (  # noqa: F401
     lite_la_bwd,
     lite_la_block_causal_bwd,
 )
+from .litela_elu_oracle import (  # noqa: F401
+    phi_elu1,
+    elu1_rows,
+    elu1_fwd,
+)
