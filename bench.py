@@ -197,9 +197,11 @@ def one_head_bits(qkv_bits, B, N, H, b, h):
     return np.ascontiguousarray(x.reshape(1, N, 3 * D))
 
 
-def oracle_head(oracle, head_bits, N, T, dout_bits=None):
+def oracle_head(oracle, head_bits, N, T, dout_bits=None, variant="litela"):
     """The oracle on one whole (batch, head): non-causal when T == 0; the backward (all N
-    tokens' dq, dk, dv) when dout_bits [1, N, d] is given."""
+    tokens' dq, dk, dv) when dout_bits [1, N, d] is given; the ELU+1 forward for elu1."""
+    if variant == "elu1":
+        return oracle.elu1_fwd(head_bits, 1, N, 1, D, 1e-6, T or None)
     if dout_bits is not None:
         if T:
             return oracle.lite_la_block_causal_bwd(head_bits, dout_bits, 1, N, 1, D, EPS, T)
@@ -215,7 +217,7 @@ def one_head_dout_bits(dout_bits, B, N, H, b, h):
     return np.ascontiguousarray(dout_bits.reshape(B, N, H, D)[b, :, h, :].reshape(1, N, D))
 
 
-def oracle_head_rate(qkv_bits, B, N, H, T, seconds, max_heads=None, dout_bits=None):
+def oracle_head_rate(qkv_bits, B, N, H, T, seconds, max_heads=None, dout_bits=None, variant="litela"):
     """Times the fp64 oracle on whole heads (all N queries of one (batch, head)) until
     `seconds` have passed; returns (tokens*heads per second, heads done, elapsed)."""
     import oracle
@@ -223,7 +225,7 @@ def oracle_head_rate(qkv_bits, B, N, H, T, seconds, max_heads=None, dout_bits=No
     while True:
         b, h = divmod(heads % (B * H), H)
         g = None if dout_bits is None else one_head_dout_bits(dout_bits, B, N, H, b, h)
-        oracle_head(oracle, one_head_bits(qkv_bits, B, N, H, b, h), N, T, g)
+        oracle_head(oracle, one_head_bits(qkv_bits, B, N, H, b, h), N, T, g, variant)
         heads += 1
         el = time.perf_counter() - t0
         if el >= seconds or (max_heads and heads >= max_heads):
@@ -253,13 +255,13 @@ def run_reference(args, wl):
         return None if gbits is None else one_head_dout_bits(gbits, B, N, H, b, h)
 
     for i in range(args.warmup):
-        oracle_head(oracle, one_head_bits(bits, B, N, H, *heads[i]), N, T, head_dout(*heads[i]))
+        oracle_head(oracle, one_head_bits(bits, B, N, H, *heads[i]), N, T, head_dout(*heads[i]), args.variant)
     times = []
     for i in range(args.steps):
         hb = one_head_bits(bits, B, N, H, *heads[args.warmup + i])
         gb = head_dout(*heads[args.warmup + i])
         t0 = time.perf_counter()
-        oracle_head(oracle, hb, N, T, gb)
+        oracle_head(oracle, hb, N, T, gb, args.variant)
         times.append(time.perf_counter() - t0)
     ms = 1e3 * float(np.mean(times))
     value = N / (ms / 1e3)
@@ -269,7 +271,7 @@ def run_reference(args, wl):
           "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
           "data": "synthetic: i.i.d. N(0,1) bf16 qkv, seed %d" % seed,
-          "config": config_of(wl, args.direction),
+          "config": config_of(wl, args.direction, args.variant),
           "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                            "sample": sample},
           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
@@ -284,9 +286,10 @@ def make_dout(B, N, H, seed, device):
     return torch.randn((B, N, H * D), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
 
 
-def config_of(wl, direction="fwd"):
+def config_of(wl, direction="fwd", variant="litela"):
     B, N, H, calls, seed, T = WORKLOADS_BENCH[wl]
-    return {"workload": wl + ("_bwd" if direction == "bwd" else ""), "direction": direction,
+    return {"workload": wl + ("_bwd" if direction == "bwd" else "") + ("_elu1" if variant == "elu1" else ""),
+            "direction": direction, "feature_map": "relu" if variant == "litela" else "elu+1 (clamp 1e-6)",
             "B": B, "N": N, "H": H, "d": D, "tokens_per_block": T or None, "calls_per_step": calls,
             "distinct_input_buffers": calls, "eps": EPS, "layout": "qkv bf16 [B,N,3*H*d], out bf16 [B,N,H*d]",
             "l2": "inputs larger than L2 (%.0f MB per call vs 126 MB), no flush" % (B * N * 3 * H * D * 2 / 1e6)}
@@ -306,6 +309,8 @@ def main():
                     help="duration of the fp32 FMA peak measurement (0 skips it)")
     ap.add_argument("--direction", choices=["fwd", "bwd"], default="fwd",
                     help="bwd times the backward (dq, dk, dv of a seeded incoming gradient)")
+    ap.add_argument("--variant", choices=["litela", "elu1"], default="litela",
+                    help="elu1 times the ELU+1 feature-map variant of the forward (clamp 1e-6)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -361,7 +366,16 @@ def main():
     sh = ctypes.c_void_p(stream.cuda_stream)
     in_p = [t.data_ptr() for t in ins]
     out_p = [t.data_ptr() for t in outs]
-    if bwd:   # fwd(i, ...) runs call i: here the backward of buffer i
+    if args.variant == "elu1":
+        if bwd:
+            raise SystemExit("--variant elu1 has no backward")
+
+        def fwd(qkv, out, B, N, H, d, eps, stream):
+            return lib.lite_la_elu1_fwd(qkv, out, B, N, H, d, 1e-6, T, stream)
+
+        def fwd_events(qkv, out, B, N, H, d, eps, stream, evs):
+            return lib.lite_la_elu1_fwd_events(qkv, out, B, N, H, d, 1e-6, T, stream, evs)
+    elif bwd:   # fwd(i, ...) runs call i: here the backward of buffer i
         dq_of = {p_: g_ for p_, g_ in zip(in_p, grad_p)}
 
         def fwd(qkv, out, B, N, H, d, eps, stream):
@@ -424,7 +438,7 @@ def main():
             e.record(stream)
     torch.cuda.synchronize(dev)
     ev_handles = [(ctypes.c_void_p * nev)(*[ctypes.c_void_p(e.cuda_event) for e in trip]) for trip in evs]
-    nk = 5 if bwd else int(lib.lite_la_kernels_per_call(B, N, H, D, T))
+    nk = 5 if bwd else (3 if args.variant == "elu1" else int(lib.lite_la_kernels_per_call(B, N, H, D, T)))
     phases = PATHS[nk]["phases"]
     kern_ms = {k: 0.0 for k in phases}
     nlaunch = 0
@@ -548,7 +562,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         bits = to_bits(ins[0])
         gbits = to_bits(outs[0]) if bwd else None
-        rate, heads, el = oracle_head_rate(bits, B, N, H, T, args.cpu_seconds, dout_bits=gbits)
+        rate, heads, el = oracle_head_rate(bits, B, N, H, T, args.cpu_seconds, dout_bits=gbits, variant=args.variant)
         cpu = {"value": rate, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": "%d whole (batch, head) pairs of input buffer 0 (%s, all %d tokens), %.1f s"
                          % (heads, "dq, dk, dv" if bwd else "all queries x all keys", N, el)}
@@ -560,7 +574,7 @@ def main():
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "math": "tensor-core bf16 x bf16 products with fp32 accumulation; fp32 state applied as bf16 hi + lo",
                 "data": "synthetic: i.i.d. N(0,1) bf16 qkv from seeded torch generators",
-                "config": config_of(args.workload, args.direction), "roofline": roofline,
+                "config": config_of(args.workload, args.direction, args.variant), "roofline": roofline,
                 "call_roofline": call_roof,
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": nk * calls * args.steps,
                 "clocks": clocks, "gpu": torch.cuda.get_device_name(dev)}

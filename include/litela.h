@@ -135,6 +135,26 @@ litela_status lite_la_device_status(cudaStream_t stream);
  * context remain usable.  Nothing faults and nothing hangs. */
 litela_status lite_la_selftest_timeout(cudaStream_t stream);
 
+/* ---- ELU + 1 variant ------------------------------------------------------------------
+ *
+ * Kernelised linear attention as the Sana tutorial page (aifetchly) writes its linear-attention
+ * block: phi(x) = ELU(x) + 1 (exp(x) for x <= 0, x + 1 above; alpha = 1) on q and k, phi(q)
+ * scaled by 1/sqrt(d), the same state S = [V;1] . phi(K)^T, and the denominator clamped from
+ * below instead of adding eps:
+ *     out_n[r] = y_n[r] / max(y_n[d], clamp_min),   y_n = S . (phi(q_n) / sqrt(d)).
+ * Sana's LiteLA is the ReLU form above; this variant is provided beside it.  tokens_per_block
+ * > 0 gives the block-causal form, <= 0 the non-causal one.  clamp_min (the page uses 1e-6)
+ * must be finite and >= 0.  Layouts, buffers, streams and status codes as for lite_la_fwd
+ * (bf16 output; fp32 for the _f32out form). */
+litela_status lite_la_elu1_fwd(const void* qkv, void* out, int B, int N, int H, int d, float clamp_min,
+                               int tokens_per_block, cudaStream_t stream);
+litela_status lite_la_elu1_fwd_f32out(const void* qkv, float* out, int B, int N, int H, int d, float clamp_min,
+                                      int tokens_per_block, cudaStream_t stream);
+/* lite_la_elu1_fwd with the phase timing of lite_la_fwd_events (three kernels: events[0]
+ * before the reduction, events[1] after the scan, events[2] after the apply). */
+litela_status lite_la_elu1_fwd_events(const void* qkv, void* out, int B, int N, int H, int d, float clamp_min,
+                                      int tokens_per_block, cudaStream_t stream, cudaEvent_t* events);
+
 /* ---- backward -------------------------------------------------------------------------
  *
  * Gradients of L = sum over all outputs of dout * out with respect to q, k and v, for the

@@ -52,6 +52,9 @@ _SIGNATURES = {
     "lite_la_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "lite_la_fwd_noalloc": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp]),
     "lite_la_kernels_per_call": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "lite_la_elu1_fwd": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
+    "lite_la_elu1_fwd_f32out": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
+    "lite_la_elu1_fwd_events": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp, _vp]),
     "lite_la_bwd": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp]),
     "lite_la_block_causal_bwd": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
     "lite_la_bwd_f32out": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp]),
@@ -207,6 +210,19 @@ def lite_la_state_fwd(qkv, H: int, tokens_per_block: int = 0, d: int = 32, out=N
     with torch.cuda.device(qkv.device):
         _check(lib().lite_la_state_fwd(qkv.data_ptr(), out.data_ptr(), B, N, H, d, int(tokens_per_block),
                                        _stream_handle(stream, qkv.device)))
+    return out
+
+
+def lite_la_elu1_fwd(qkv, H: int, tokens_per_block: int = 0, d: int = 32, clamp_min: float = 1e-6, out=None,
+                     out_dtype=None, stream=None):
+    """The ELU+1 variant (phi = ELU + 1, phi(q) / sqrt(d), denominator clamped at clamp_min);
+    block-causal when tokens_per_block > 0.  Returns out [B, N, H*d]."""
+    torch = _torch()
+    B, N, out = _prepare(qkv, H, d, out, out_dtype or torch.bfloat16)
+    fn = lib().lite_la_elu1_fwd if out.dtype == torch.bfloat16 else lib().lite_la_elu1_fwd_f32out
+    with torch.cuda.device(qkv.device):
+        _check(fn(qkv.data_ptr(), out.data_ptr(), B, N, H, d, clamp_min, int(tokens_per_block),
+                  _stream_handle(stream, qkv.device)))
     return out
 
 

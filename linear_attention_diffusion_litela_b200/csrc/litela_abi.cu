@@ -66,8 +66,14 @@ litela_status device_setup(int* num_sms) {
                                               std::to_string(major) + std::to_string(minor));
     if ((e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
       return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
-    if ((e = cudaFuncSetAttribute(litela_reduce_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)kRedSmemBytes)) != cudaSuccess ||
+    if ((e = cudaFuncSetAttribute(litela_reduce_tc<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)RedCfg<0>::kSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_reduce_tc<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)RedCfg<1>::kSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_apply_tc<__nv_bfloat16, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)ApplyCfg<__nv_bfloat16, 1>::kSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_apply_tc<float, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)ApplyCfg<float, 1>::kSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_apply_tc<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)ApplyCfg<__nv_bfloat16>::kSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_apply_tc<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -266,13 +272,15 @@ cudaError_t launch_ex(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, c
   return cudaLaunchKernelEx(&cfg, k, static_cast<KArgs>(args)...);
 }
 
+template <int kMap = 0>
 litela_status launch_reduce(const Plan& plan, const void* qkv, float* partials, int* err, cudaStream_t stream,
                             bool pdl) {
   CUtensorMap map;
   litela_status s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kRedTile, &map);
   if (s != LITELA_OK) return s;
-  cudaError_t e = launch_ex(litela_reduce_tc, dim3(plan.nblk * plan.chunks_per_block, plan.ngroups, plan.B),
-                            dim3(kRedThreads), kRedSmemBytes, stream, pdl, map, partials, err, tc_plan(plan, 0.f));
+  cudaError_t e = launch_ex(litela_reduce_tc<kMap>, dim3(plan.nblk * plan.chunks_per_block, plan.ngroups, plan.B),
+                            dim3(kRedThreads), RedCfg<kMap>::kSmemBytes, stream, pdl, map, partials, err,
+                            tc_plan(plan, 0.f));
   if (e != cudaSuccess) return cuda_fail(e, "launch litela_reduce_tc");
   return LITELA_OK;
 }
@@ -326,7 +334,7 @@ litela_status launch_fused(const Plan& plan, const void* qkv, OutT* out, float e
 // scan and the apply are programmatic dependents (their prologues overlap the preceding
 // kernel's end) unless phase events are requested, in which case the kernels run in plain
 // stream order with events between the reduction (with the scan) and the apply.
-template <typename OutT>
+template <typename OutT, int kMap = 0>
 litela_status launch(const Plan& plan, const void* qkv, OutT* out, float eps, float* partials, uint8_t* images,
                      int* err, int num_sms, cudaStream_t stream, cudaEvent_t* events,
                      const float* state_in = nullptr, float* state_out = nullptr) {
@@ -338,7 +346,7 @@ litela_status launch(const Plan& plan, const void* qkv, OutT* out, float eps, fl
   const bool pdl = events == nullptr;
   cudaError_t e;
   if (events && (e = cudaEventRecord(events[0], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  s = launch_reduce(plan, qkv, partials, err, stream, pdl);
+  s = launch_reduce<kMap>(plan, qkv, partials, err, stream, pdl);
   if (s != LITELA_OK) return s;
   s = launch_scan(plan, partials, images, nullptr, num_sms, stream, pdl, state_in, state_out);
   if (s != LITELA_OK) return s;
@@ -351,8 +359,9 @@ litela_status launch(const Plan& plan, const void* qkv, OutT* out, float eps, fl
     if (8 * even >= 7LL * num_sms) grid = even;
   }
   if (grid > plan.units) grid = plan.units;
-  e = launch_ex(litela_apply_tc<OutT>, dim3((unsigned)grid), dim3(kApThreads), ApplyCfg<OutT>::kSmemBytes, stream,
-                pdl, map_q, map_out, static_cast<const uint8_t*>(images), out, err, tc_plan(plan, eps));
+  e = launch_ex(litela_apply_tc<OutT, kMap>, dim3((unsigned)grid), dim3(kApThreads),
+                ApplyCfg<OutT, kMap>::kSmemBytes, stream, pdl, map_q, map_out, static_cast<const uint8_t*>(images), out,
+                err, tc_plan(plan, eps));
   if (e != cudaSuccess) return cuda_fail(e, "launch litela_apply_tc");
   if (events && (e = cudaEventRecord(events[2], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   return LITELA_OK;
@@ -384,7 +393,9 @@ litela_status run_states(const void* qkv, float* states, int B, int N, int H, in
   return LITELA_OK;
 }
 
-template <typename OutT>
+// kMap 0: LiteLA (ReLU, + eps); kMap 1: the ELU + 1 variant (eps is the denominator's clamp),
+// always on the three-kernel path.
+template <typename OutT, int kMap = 0>
 litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float eps, int tokens_per_block,
                   bool causal, cudaStream_t stream, cudaEvent_t* events = nullptr, bool carry = false,
                   const float* state_in = nullptr, float* state_out = nullptr) {
@@ -396,9 +407,11 @@ litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float 
   if (s != LITELA_OK) return s;
   Plan plan;
   make_plan(B, N, H, causal ? tokens_per_block : 0, num_sms, &plan);
-  if (carry) {   // the carried state enters through the scan: use the three-kernel path
+  if (carry || kMap != 0) {   // the carried state enters through the scan: the three-kernel path
     plan.fused = false;
     plan.counters = 0;
+  }
+  if (carry) {
     const size_t sbytes = (size_t)B * H * kStateFloats * sizeof(float);
     const size_t qkv_bytes = (size_t)B * N * 3 * H * d * sizeof(__nv_bfloat16);
     const size_t out_bytes = (size_t)B * N * H * d * sizeof(OutT);
@@ -414,14 +427,15 @@ litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float 
   if (s != LITELA_OK) return s;
   char* base = static_cast<char*>(ws->partials);
   if (carry)
-    s = launch(plan, qkv, out, eps, reinterpret_cast<float*>(base), reinterpret_cast<uint8_t*>(base + plan.off_images),
-               ws->err, num_sms, stream, events, state_in, state_out);
+    s = launch<OutT, kMap>(plan, qkv, out, eps, reinterpret_cast<float*>(base),
+                           reinterpret_cast<uint8_t*>(base + plan.off_images), ws->err, num_sms, stream, events,
+                           state_in, state_out);
   else if (plan.fused)
     s = launch_fused(plan, qkv, out, eps, reinterpret_cast<float*>(base), ws->err, ws->ctl_words, ws->calls++, stream,
                      events);
   else
-    s = launch(plan, qkv, out, eps, reinterpret_cast<float*>(base), reinterpret_cast<uint8_t*>(base + plan.off_images),
-               ws->err, num_sms, stream, events);
+    s = launch<OutT, kMap>(plan, qkv, out, eps, reinterpret_cast<float*>(base),
+                           reinterpret_cast<uint8_t*>(base + plan.off_images), ws->err, num_sms, stream, events);
   if (s == LITELA_OK) g_last_error.clear();
   return s;
 }
@@ -626,6 +640,25 @@ litela_status lite_la_state_fwd(const void* qkv, float* states, int B, int N, in
 litela_status lite_la_fwd_noalloc(const void* qkv, void* out, int B, int N, int H, int d, float eps,
                                   cudaStream_t stream) {
   return litela::run_noalloc(qkv, static_cast<__nv_bfloat16*>(out), B, N, H, d, eps, stream);
+}
+
+litela_status lite_la_elu1_fwd(const void* qkv, void* out, int B, int N, int H, int d, float clamp_min,
+                               int tokens_per_block, cudaStream_t stream) {
+  return litela::run<__nv_bfloat16, 1>(qkv, static_cast<__nv_bfloat16*>(out), B, N, H, d, clamp_min,
+                                       tokens_per_block, tokens_per_block > 0, stream);
+}
+
+litela_status lite_la_elu1_fwd_events(const void* qkv, void* out, int B, int N, int H, int d, float clamp_min,
+                                      int tokens_per_block, cudaStream_t stream, cudaEvent_t* events) {
+  if (events == nullptr || !events[0] || !events[1] || !events[2])
+    return litela::fail(LITELA_ERR_INVALID_ARGUMENT, "events must point to 3 CUDA events");
+  return litela::run<__nv_bfloat16, 1>(qkv, static_cast<__nv_bfloat16*>(out), B, N, H, d, clamp_min,
+                                       tokens_per_block, tokens_per_block > 0, stream, events);
+}
+
+litela_status lite_la_elu1_fwd_f32out(const void* qkv, float* out, int B, int N, int H, int d, float clamp_min,
+                                      int tokens_per_block, cudaStream_t stream) {
+  return litela::run<float, 1>(qkv, out, B, N, H, d, clamp_min, tokens_per_block, tokens_per_block > 0, stream);
 }
 
 litela_status lite_la_bwd(const void* qkv, const void* dout, void* dqkv, int B, int N, int H, int d, float eps,

@@ -117,14 +117,46 @@ constexpr uint32_t kRedStageBytes = 4 * kRedBoxBytes;  // k lo/hi channels, v lo
 constexpr uint32_t kRedTmemCols = 256;
 constexpr uint32_t kRedSmemBytes = kRedStages * kRedStageBytes + 512 + 256 + 1024;
 
+// Feature maps.  kMap 0: phi = ReLU (LiteLA), exact in bf16.  kMap 1: phi = ELU + 1 (the Sana
+// tutorial page's linear-attention block: exp(x) for x <= 0, x + 1 above), formed in fp32 and
+// entered into the tensor cores as a bf16 hi + lo pair (the lo halves in an extra buffer).
+template <int kMap>
+struct RedCfg {
+  static constexpr uint32_t kStageBytes = (kMap ? 6 : 4) * kRedBoxBytes;   // + phi(k) lo boxes
+  static constexpr uint32_t kSmemBytes = kRedStages * kStageBytes + 512 + 256 + 1024;
+};
+
+__device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : expf(x); }
+constexpr float kInvSqrtD = 0.17677669529663687f;   // 1 / sqrt(32): the variant's scale of phi(q)
+
+// phi = ELU + 1 of 8 packed bf16 values, times `scale`, as bf16 hi and lo (hi + lo equals the
+// fp32 value to 2^-17 relative)
+__device__ __forceinline__ void phi_elu1_hilo(uint4 w, float scale, uint4& hi, uint4& lo) {
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float x0 = phi_elu1(__uint_as_float(u[i] << 16)) * scale;
+    const float x1 = phi_elu1(__uint_as_float(u[i] & 0xFFFF0000u)) * scale;
+    __nv_bfloat162 hp = __floats2bfloat162_rn(x0, x1);
+    h[i] = *reinterpret_cast<uint32_t*>(&hp);
+    __nv_bfloat162 lp = __floats2bfloat162_rn(x0 - __uint_as_float(h[i] << 16), x1 - __uint_as_float(h[i] & 0xFFFF0000u));
+    l[i] = *reinterpret_cast<uint32_t*>(&lp);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+template <int kMap>
 __global__ void __launch_bounds__(kRedThreads, 1)
 litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ partials,
                  int* __restrict__ err, TcPlan p) {
   using namespace sm100;
+  constexpr uint32_t kStageBytes = RedCfg<kMap>::kStageBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* stages = smem;
-  uint8_t* ones = smem + kRedStages * kRedStageBytes;                 // 16 x 16 bf16 ones
+  uint8_t* ones = smem + kRedStages * kStageBytes;                 // 16 x 16 bf16 ones
   uint64_t* full = reinterpret_cast<uint64_t*>(ones + 512);
   uint64_t* relu_done = full + kRedStages;
   uint64_t* empty = relu_done + kRedStages;
@@ -180,7 +212,7 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
         if (i >= kRedStages &&
             !mbar_wait(&empty[s], ((i / kRedStages) - 1) & 1, abort_flag, err, kErrReduceProducer | s))
           break;
-        uint8_t* st = stages + s * kRedStageBytes;
+        uint8_t* st = stages + s * kStageBytes;
         const int y = n0 + i * kRedTile;
         mbar_arrive_expect_tx(&full[s], kRedStageBytes);
         tma_load_3d(st, &tmap, &full[s], kx, y, b);
@@ -203,7 +235,7 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
         const int s = i % kRedStages;
         if (!mbar_wait(&relu_done[s], (i / kRedStages) & 1, abort_flag, err, kErrReduceMma | s)) break;
         tc_fence_after_sync();
-        const uint32_t kbase = smem_u32(stages + s * kRedStageBytes);
+        const uint32_t kbase = smem_u32(stages + s * kStageBytes);
         const uint32_t vbase = kbase + 2 * kRedBoxBytes;
 #pragma unroll
         for (int ks = 0; ks < kRedTile / 16; ++ks) {
@@ -213,6 +245,11 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
           const uint32_t acc = (i | ks) != 0;
           umma_bf16(tmem, a, bv, idesc_num, acc);
           umma_bf16(tmem + 128, a, ones_desc, idesc_den, acc);
+          if (kMap) {   // the lo halves of phi(k)
+            const uint64_t al = smem_desc(kbase + 4 * kRedBoxBytes + ks * 2048, kRedBoxBytes, 1024, kSwizzle128B);
+            umma_bf16(tmem, al, bv, idesc_num, 1u);
+            umma_bf16(tmem + 128, al, ones_desc, idesc_den, 1u);
+          }
         }
         umma_commit(&empty[s]);
       }
@@ -223,13 +260,20 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
     for (int i = 0; i < ntiles; ++i) {
       const int s = i % kRedStages;
       if (!mbar_wait(&full[s], (i / kRedStages) & 1, abort_flag, err, kErrReduceRelu | s)) break;
-      uint8_t* st = stages + s * kRedStageBytes;
+      uint8_t* st = stages + s * kStageBytes;
       const int valid = min(kRedTile, n1 - (n0 + i * kRedTile));   // tokens of this chunk in the tile
 #pragma unroll 4
       for (int j = t; j < 1024; j += 128) {          // k: 2 boxes x 64 rows x 8 chunks of 16 B
         uint4* c = reinterpret_cast<uint4*>(st + j * 16);
         const int row = (j >> 3) & (kRedTile - 1);
-        *c = row < valid ? relu_bf16x8(*c) : make_uint4(0u, 0u, 0u, 0u);
+        if (kMap == 0) {
+          *c = row < valid ? relu_bf16x8(*c) : make_uint4(0u, 0u, 0u, 0u);
+        } else {
+          uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
+          if (row < valid) phi_elu1_hilo(*c, 1.0f, hi, lo);
+          *c = hi;
+          *reinterpret_cast<uint4*>(st + 4 * kRedBoxBytes + j * 16) = lo;
+        }
       }
       if (valid < kRedTile) {
         for (int j = t; j < 1024; j += 128) {
@@ -410,16 +454,17 @@ constexpr uint32_t kApSbufBytes = kApUnitHeads * kImageBytes;
 constexpr uint32_t kOutBoxBytes = kApTile * 128;       // one 128B-swizzled box: 128 rows x 128 B
 constexpr int kApReluThreads = 64;
 
-template <typename OutT>
+template <typename OutT, int kMap = 0>
 struct ApplyCfg {
   // shared memory split (bf16 output: 4 q stages, 2 output slots, 1 state buffer = 213 KB;
-  // fp32 output: 2 q stages, 1 output slot, 2 state buffers)
-  static constexpr int kQStages = sizeof(OutT) == 2 ? 4 : 2;
+  // fp32 output: 2 q stages, 1 output slot, 2 state buffers; ELU + 1: 2 q stages of twice the
+  // size (phi(q) hi and lo), 1 state buffer)
+  static constexpr int kQStages = kMap ? 2 : (sizeof(OutT) == 2 ? 4 : 2);
   static constexpr int kOutSlots = sizeof(OutT) == 2 ? 2 : 1;
-  static constexpr int kSBufs = sizeof(OutT) == 2 ? 1 : 2;
+  static constexpr int kSBufs = kMap ? 1 : (sizeof(OutT) == 2 ? 1 : 2);
   static constexpr int kBoxChannels = 128 / (int)sizeof(OutT);     // output channels per box
   static constexpr int kOutBoxes = kApUnitHeads * kD / kBoxChannels;
-  static constexpr uint32_t kQStageBytes = 2 * kQBoxBytes;
+  static constexpr uint32_t kQStageBytes = (kMap ? 4 : 2) * kQBoxBytes;
   static constexpr uint32_t kOutSlotBytes = kOutBoxes * kOutBoxBytes;
   static constexpr uint32_t kSmemBytes =
       kQStages * kQStageBytes + kOutSlots * kOutSlotBytes + kSBufs * kApSbufBytes + 512 + 1024;
@@ -513,12 +558,12 @@ __device__ __forceinline__ void pack_out(float*, const float* o, uint4* w) {
                       __float_as_uint(o[4 * i + 3]));
 }
 
-template <typename OutT>
+template <typename OutT, int kMap = 0>
 __global__ void __launch_bounds__(kApThreads, 1)
 litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_out,
                 const uint8_t* __restrict__ images, OutT* __restrict__ out, int* __restrict__ err, TcPlan p) {
   using namespace sm100;
-  using Cfg = ApplyCfg<OutT>;
+  using Cfg = ApplyCfg<OutT, kMap>;
   constexpr int kQStages = Cfg::kQStages;
   constexpr int kSBufs = Cfg::kSBufs;
   constexpr int kChunksPerHead = kD * (int)sizeof(OutT) / 16;   // 16-byte chunks of one head's row
@@ -665,6 +710,11 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
               const uint64_t bd =
                   smem_desc(saddr + (h * kApHeads + j) * kImageBytes + ks * 256, 128, 512, kSwizzleNone);
               umma_bf16(tmem + a * kApAccCols + j * kImageRows, ad, bd, idesc, ks);
+              if (kMap) {   // the lo halves of phi(q)
+                const uint64_t al =
+                    smem_desc(qaddr + 2 * kQBoxBytes + h * kQBoxBytes + j * 64 + ks * 32, 16, 1024, kSwizzle128B);
+                umma_bf16(tmem + a * kApAccCols + j * kImageRows, al, bd, idesc, 1u);
+              }
             }
           }
           umma_commit(&tfull[a]);
@@ -689,7 +739,14 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
 #pragma unroll 4
       for (int j = t; j < nchunks; j += kApReluThreads) {
         uint4* c = reinterpret_cast<uint4*>(st + j * 16);
-        *c = relu_bf16x8(*c);
+        if (kMap == 0) {
+          *c = relu_bf16x8(*c);
+        } else {   // phi(q) / sqrt(d): hi in place, lo two boxes further
+          uint4 hi, lo;
+          phi_elu1_hilo(*c, kInvSqrtD, hi, lo);
+          *c = hi;
+          *reinterpret_cast<uint4*>(st + 2 * kQBoxBytes + j * 16) = lo;
+        }
       }
       fence_proxy_async_smem();
       mbar_arrive(&qrelu[s]);
@@ -731,7 +788,9 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
             tc_fence_before_sync();
             mbar_arrive(&tempty[a]);
           }
-          const float den = (__uint_as_float(v[kD]) + __uint_as_float(v[kImageLoRow + kD])) + p.eps;
+          // LiteLA adds eps to the denominator; the ELU + 1 variant clamps it from below (p.eps)
+          const float y_d = __uint_as_float(v[kD]) + __uint_as_float(v[kImageLoRow + kD]);
+          const float den = kMap ? fmaxf(y_d, p.eps) : y_d + p.eps;
           const float inv = 1.0f / den;
           float o[kD];
 #pragma unroll
