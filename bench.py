@@ -286,9 +286,10 @@ def make_dout(B, N, H, seed, device):
     return torch.randn((B, N, H * D), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
 
 
-def config_of(wl, direction="fwd", variant="litela"):
+def config_of(wl, direction="fwd", variant="litela", from_state=False):
     B, N, H, calls, seed, T = WORKLOADS_BENCH[wl]
-    return {"workload": wl + ("_bwd" if direction == "bwd" else "") + ("_elu1" if variant == "elu1" else ""),
+    return {"workload": wl + ("_bwd" if direction == "bwd" else "") + ("_elu1" if variant == "elu1" else "")
+            + ("_from_state" if from_state else ""),
             "direction": direction, "feature_map": "relu" if variant == "litela" else "elu+1 (clamp 1e-6)",
             "B": B, "N": N, "H": H, "d": D, "tokens_per_block": T or None, "calls_per_step": calls,
             "distinct_input_buffers": calls, "eps": EPS, "layout": "qkv bf16 [B,N,3*H*d], out bf16 [B,N,H*d]",
@@ -309,6 +310,9 @@ def main():
                     help="duration of the fp32 FMA peak measurement (0 skips it)")
     ap.add_argument("--direction", choices=["fwd", "bwd"], default="fwd",
                     help="bwd times the backward (dq, dk, dv of a seeded incoming gradient)")
+    ap.add_argument("--bwd-from-state", action="store_true",
+                    help="with --direction bwd: the backward given the forward's saved states "
+                         "(lite_la_bwd_from_state; the states are made once before timing)")
     ap.add_argument("--variant", choices=["litela", "elu1"], default="litela",
                     help="elu1 times the ELU+1 feature-map variant of the forward (clamp 1e-6)")
     args = ap.parse_args()
@@ -377,11 +381,23 @@ def main():
             return lib.lite_la_elu1_fwd_events(qkv, out, B, N, H, d, 1e-6, T, stream, evs)
     elif bwd:   # fwd(i, ...) runs call i: here the backward of buffer i
         dq_of = {p_: g_ for p_, g_ in zip(in_p, grad_p)}
+        if args.bwd_from_state:   # the forward's states of every buffer, made before timing
+            nblk = -(-N // T) if T else 1
+            st_bufs = [torch.empty((B, H, nblk, D + 1, D), dtype=torch.float32, device=dev) for _ in range(calls)]
+            tmp = torch.empty((B, N, H * D), dtype=torch.bfloat16, device=dev)
+            for p_, st in zip(in_p, st_bufs):
+                if lib.lite_la_fwd_save_state(p_, tmp.data_ptr(), st.data_ptr(), B, N, H, D, EPS, T, sh) != 0:
+                    raise ll.LiteLAError(1, lib.lite_la_last_error().decode())
+            torch.cuda.synchronize(dev)
+            st_of = {p_: st.data_ptr() for p_, st in zip(in_p, st_bufs)}
 
-        def fwd(qkv, out, B, N, H, d, eps, stream):
-            if T:
-                return lib.lite_la_block_causal_bwd(qkv, out, dq_of[qkv], B, N, H, d, eps, T, stream)
-            return lib.lite_la_bwd(qkv, out, dq_of[qkv], B, N, H, d, eps, stream)
+            def fwd(qkv, out, B, N, H, d, eps, stream):
+                return lib.lite_la_bwd_from_state(qkv, out, st_of[qkv], dq_of[qkv], B, N, H, d, eps, T, stream)
+        else:
+            def fwd(qkv, out, B, N, H, d, eps, stream):
+                if T:
+                    return lib.lite_la_block_causal_bwd(qkv, out, dq_of[qkv], B, N, H, d, eps, T, stream)
+                return lib.lite_la_bwd(qkv, out, dq_of[qkv], B, N, H, d, eps, stream)
 
         def fwd_events(qkv, out, B, N, H, d, eps, stream, evs):
             return lib.lite_la_bwd_events(qkv, out, dq_of[qkv], B, N, H, d, eps, T, stream, evs)
@@ -483,7 +499,9 @@ def main():
                            "calls on the launching stream, / launches" if nk == 1 else
                            "CUDA events on the launching stream around each phase (phase-timed entry points; "
                            "no programmatic overlap with the neighbouring kernels)")
-                          + "; kernel_us_isolated: each call alone between events"}
+                          + "; kernel_us_isolated: each call alone between events"
+                          + ("; phases timed on the recomputing backward (the same dq and dk/dv kernels)"
+                             if bwd and args.bwd_from_state else "")}
     # the call as a whole against the slower of the HBM and fp32-FMA bounds
     t_hbm = call_bytes_E * E / (peaks["hbm_gbs"] * 1e9) * 1e6
     t_fma = flops_per_call / (fp32_fma_peak_tflops(peaks.get("sm_max_mhz", 1965.0)) * 1e12) * 1e6
@@ -574,7 +592,8 @@ def main():
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "math": "tensor-core bf16 x bf16 products with fp32 accumulation; fp32 state applied as bf16 hi + lo",
                 "data": "synthetic: i.i.d. N(0,1) bf16 qkv from seeded torch generators",
-                "config": config_of(args.workload, args.direction, args.variant), "roofline": roofline,
+                "config": config_of(args.workload, args.direction, args.variant, args.bwd_from_state),
+                "roofline": roofline,
                 "call_roofline": call_roof,
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": nk * calls * args.steps,
                 "clocks": clocks, "gpu": torch.cuda.get_device_name(dev)}

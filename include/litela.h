@@ -187,6 +187,20 @@ litela_status lite_la_bwd_f32out(const void* qkv, const void* dout, float* dqkv,
 litela_status lite_la_block_causal_bwd_f32out(const void* qkv, const void* dout, float* dqkv, int B, int N, int H,
                                               int d, float eps, int tokens_per_block, cudaStream_t stream);
 
+/* The forward and the backward with the state carried between them.  lite_la_fwd_save_state
+ * is lite_la_fwd (tokens_per_block <= 0) or lite_la_block_causal_fwd (> 0), bitwise the same
+ * output, that also writes the states its queries use, fp32 [B, H, nblk, d+1, d] (the layout of
+ * lite_la_state_fwd: the per-block inclusive prefix states; nblk = 1 when non-causal) into the
+ * caller's buffer `states` (16-byte aligned, not overlapping qkv or out).
+ * lite_la_bwd_from_state is lite_la_bwd / lite_la_block_causal_bwd (bf16 dqkv) given those
+ * states: it skips recomputing them (a reduction over k and v and a scan), which saves 4 of the
+ * 18 bytes of HBM traffic per (token, head, channel).  `states` must hold the states of the same
+ * qkv and tokens_per_block (not checked); other arguments as for lite_la_bwd. */
+litela_status lite_la_fwd_save_state(const void* qkv, void* out, float* states, int B, int N, int H, int d,
+                                     float eps, int tokens_per_block, cudaStream_t stream);
+litela_status lite_la_bwd_from_state(const void* qkv, const void* dout, const float* states, void* dqkv, int B, int N,
+                                     int H, int d, float eps, int tokens_per_block, cudaStream_t stream);
+
 /* The backward (bf16 dqkv) with phase timing: events[0] before its first kernel, events[1]
  * after the state (reduction + scan), events[2] after the dq kernel, events[3] after the
  * dk/dv kernels; tokens_per_block <= 0 is the non-causal call.  events: host array of 4

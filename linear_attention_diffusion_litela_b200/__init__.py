@@ -62,6 +62,8 @@ _SIGNATURES = {
                                                  _vp]),
     "lite_la_bwd_events": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp, _vp]),
     "lite_la_bwd_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "lite_la_fwd_save_state": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
+    "lite_la_bwd_from_state": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
 }
 EXPORTED_SYMBOLS = tuple(_SIGNATURES)
 
@@ -249,6 +251,36 @@ def lite_la_bwd(qkv, dout, H: int, tokens_per_block: int = 0, d: int = 32, eps: 
         else:
             fn = lib().lite_la_bwd_f32out if f32 else lib().lite_la_bwd
             _check(fn(qkv.data_ptr(), dout.data_ptr(), dqkv.data_ptr(), B, N, H, d, eps, sh))
+    return dqkv
+
+
+def lite_la_fwd_save_state(qkv, H: int, tokens_per_block: int = 0, d: int = 32, eps: float = 1e-15, stream=None):
+    """Forward (bf16 out) that also returns the states its queries use, fp32 [B, H, nblk, d+1, d],
+    for lite_la_bwd_from_state.  Returns (out, states)."""
+    torch = _torch()
+    B, N, out = _prepare(qkv, H, d, None, torch.bfloat16)
+    T = tokens_per_block if 0 < tokens_per_block < N else N
+    nblk = -(-N // T) if N > 0 else 0
+    states = torch.empty((B, H, nblk, d + 1, d), dtype=torch.float32, device=qkv.device)
+    with torch.cuda.device(qkv.device):
+        _check(lib().lite_la_fwd_save_state(qkv.data_ptr(), out.data_ptr(), states.data_ptr(), B, N, H, d, eps,
+                                            int(tokens_per_block), _stream_handle(stream, qkv.device)))
+    return out, states
+
+
+def lite_la_bwd_from_state(qkv, dout, states, H: int, tokens_per_block: int = 0, d: int = 32, eps: float = 1e-15,
+                           stream=None):
+    """lite_la_bwd (bf16 dqkv) given the forward's states from lite_la_fwd_save_state."""
+    torch = _torch()
+    B, N, _ = _prepare(qkv, H, d, dout, torch.bfloat16)
+    if dout.dtype != torch.bfloat16:
+        raise TypeError("dout must be a contiguous bf16 tensor [B, N, H*d]")
+    if states.dtype != torch.float32 or not states.is_contiguous() or states.device != qkv.device:
+        raise TypeError("states must be a contiguous fp32 tensor on qkv's device")
+    dqkv = torch.empty((B, N, 3 * H * d), dtype=torch.bfloat16, device=qkv.device)
+    with torch.cuda.device(qkv.device):
+        _check(lib().lite_la_bwd_from_state(qkv.data_ptr(), dout.data_ptr(), states.data_ptr(), dqkv.data_ptr(), B, N,
+                                            H, d, eps, int(tokens_per_block), _stream_handle(stream, qkv.device)))
     return dqkv
 
 

@@ -279,7 +279,7 @@ litela_status launch_reduce(const Plan& plan, const void* qkv, float* partials, 
   litela_status s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kRedTile, &map);
   if (s != LITELA_OK) return s;
   cudaError_t e = launch_ex(litela_reduce_tc<kMap>, dim3(plan.nblk * plan.chunks_per_block, plan.ngroups, plan.B),
-                            dim3(kRedThreads), RedCfg<kMap>::kSmemBytes, stream, pdl, map, partials, err,
+                            dim3(RedCfg<kMap>::kThreads), RedCfg<kMap>::kSmemBytes, stream, pdl, map, partials, err,
                             tc_plan(plan, 0.f));
   if (e != cudaSuccess) return cuda_fail(e, "launch litela_reduce_tc");
   return LITELA_OK;
@@ -305,7 +305,7 @@ litela_status launch_scan(const Plan& plan, const float* partials, uint8_t* imag
 template <typename OutT>
 litela_status launch_fused(const Plan& plan, const void* qkv, OutT* out, float eps, float* partials, int* ctl,
                            size_t ctl_words, unsigned long long call_index, cudaStream_t stream,
-                           cudaEvent_t* events) {
+                           cudaEvent_t* events, float* states = nullptr) {
   CUtensorMap map_kv, map_q, map_out;
   litela_status s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kRedTile, &map_kv);
   if (s != LITELA_OK) return s;
@@ -318,7 +318,7 @@ litela_status launch_fused(const Plan& plan, const void* qkv, OutT* out, float e
   // two counter sets of (ctl_words - kCounterBase) / 2 words each; calls alternate between them
   const int set_words = (int)((ctl_words - kCounterBase) / 2);
   const FusedPlan fp{plan.B,           plan.N,    plan.H, plan.nquads, plan.fused_cpb, plan.fused_chunk,
-                     plan.fused_ntiles, (int)(call_index & 1), set_words, eps};
+                     plan.fused_ntiles, (int)(call_index & 1), set_words, eps, states};
   const unsigned grid = (unsigned)(plan.B * plan.nquads * plan.fused_cpb);
   e = launch_ex(litela_fused_tc<OutT>, dim3(grid), dim3(kFuThreads), FusedCfg<OutT>::kSmemBytes, stream,
                 events == nullptr, map_kv, map_q, map_out, partials, reinterpret_cast<unsigned*>(ctl + kCounterBase),
@@ -337,7 +337,7 @@ litela_status launch_fused(const Plan& plan, const void* qkv, OutT* out, float e
 template <typename OutT, int kMap = 0>
 litela_status launch(const Plan& plan, const void* qkv, OutT* out, float eps, float* partials, uint8_t* images,
                      int* err, int num_sms, cudaStream_t stream, cudaEvent_t* events,
-                     const float* state_in = nullptr, float* state_out = nullptr) {
+                     const float* state_in = nullptr, float* state_out = nullptr, float* states = nullptr) {
   CUtensorMap map_q, map_out;
   litela_status s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kApTile, &map_q);
   if (s != LITELA_OK) return s;
@@ -348,7 +348,7 @@ litela_status launch(const Plan& plan, const void* qkv, OutT* out, float eps, fl
   if (events && (e = cudaEventRecord(events[0], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   s = launch_reduce<kMap>(plan, qkv, partials, err, stream, pdl);
   if (s != LITELA_OK) return s;
-  s = launch_scan(plan, partials, images, nullptr, num_sms, stream, pdl, state_in, state_out);
+  s = launch_scan(plan, partials, images, states, num_sms, stream, pdl, state_in, state_out);
   if (s != LITELA_OK) return s;
   if (events && (e = cudaEventRecord(events[1], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   // CTAs: a multiple of the head quads when that keeps at least 7/8 of the SMs busy (all quads
@@ -359,7 +359,7 @@ litela_status launch(const Plan& plan, const void* qkv, OutT* out, float eps, fl
     if (8 * even >= 7LL * num_sms) grid = even;
   }
   if (grid > plan.units) grid = plan.units;
-  e = launch_ex(litela_apply_tc<OutT, kMap>, dim3((unsigned)grid), dim3(kApThreads),
+  e = launch_ex(litela_apply_tc<OutT, kMap>, dim3((unsigned)grid), dim3(ApplyCfg<OutT, kMap>::kThreads),
                 ApplyCfg<OutT, kMap>::kSmemBytes, stream, pdl, map_q, map_out, static_cast<const uint8_t*>(images), out,
                 err, tc_plan(plan, eps));
   if (e != cudaSuccess) return cuda_fail(e, "launch litela_apply_tc");
@@ -398,10 +398,20 @@ litela_status run_states(const void* qkv, float* states, int B, int N, int H, in
 template <typename OutT, int kMap = 0>
 litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float eps, int tokens_per_block,
                   bool causal, cudaStream_t stream, cudaEvent_t* events = nullptr, bool carry = false,
-                  const float* state_in = nullptr, float* state_out = nullptr) {
+                  const float* state_in = nullptr, float* state_out = nullptr, float* save_states = nullptr) {
   bool empty = false;
   litela_status s = validate(qkv, out, sizeof(OutT), B, N, H, d, eps, tokens_per_block, causal, &empty);
   if (s != LITELA_OK || empty) return s;
+  if (save_states != nullptr) {   // the states the queries use, fp32 [B][H][nblk][33][32]
+    const int nb = (!causal || tokens_per_block >= N) ? 1 : (N + tokens_per_block - 1) / tokens_per_block;
+    const size_t sbytes = (size_t)B * H * nb * kStateFloats * sizeof(float);
+    const size_t qkv_bytes = (size_t)B * N * 3 * H * d * sizeof(__nv_bfloat16);
+    const size_t out_bytes = (size_t)B * N * H * d * sizeof(OutT);
+    if (reinterpret_cast<uintptr_t>(save_states) & 15u)
+      return fail(LITELA_ERR_INVALID_ARGUMENT, "states must be 16-byte aligned");
+    if (overlaps(save_states, sbytes, qkv, qkv_bytes) || overlaps(save_states, sbytes, out, out_bytes))
+      return fail(LITELA_ERR_INVALID_ARGUMENT, "states overlaps qkv or out");
+  }
   int num_sms = 0;
   s = device_setup(&num_sms);
   if (s != LITELA_OK) return s;
@@ -432,10 +442,11 @@ litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float 
                            state_in, state_out);
   else if (plan.fused)
     s = launch_fused(plan, qkv, out, eps, reinterpret_cast<float*>(base), ws->err, ws->ctl_words, ws->calls++, stream,
-                     events);
+                     events, save_states);
   else
     s = launch<OutT, kMap>(plan, qkv, out, eps, reinterpret_cast<float*>(base),
-                           reinterpret_cast<uint8_t*>(base + plan.off_images), ws->err, num_sms, stream, events);
+                           reinterpret_cast<uint8_t*>(base + plan.off_images), ws->err, num_sms, stream, events,
+                           nullptr, nullptr, save_states);
   if (s == LITELA_OK) g_last_error.clear();
   return s;
 }
@@ -447,9 +458,12 @@ litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float 
 // (dS images), dk + dv.  Chained with programmatic dependent launch unless phase events are
 // requested: then events[0] precedes the reduction, events[1] follows the scan, events[2] the
 // dq kernel and events[3] the dk/dv kernel (after the reverse scan).
+// states_in (optional): the forward's states, fp32 [B][H][nblk][33][32] (lite_la_fwd_save_state);
+// the reduction and the scan are then replaced by their conversion into images.
 template <typename OutT>
 litela_status run_bwd(const void* qkv, const void* dout, OutT* dqkv, int B, int N, int H, int d, float eps,
-                      int tokens_per_block, bool causal, cudaStream_t stream, cudaEvent_t* events = nullptr) {
+                      int tokens_per_block, bool causal, cudaStream_t stream, cudaEvent_t* events = nullptr,
+                      const float* states_in = nullptr) {
   bool empty = false;
   // qkv and dout as the forward's qkv and out
   litela_status s = validate(qkv, dout, sizeof(__nv_bfloat16), B, N, H, d, eps, tokens_per_block, causal, &empty);
@@ -461,6 +475,13 @@ litela_status run_bwd(const void* qkv, const void* dout, OutT* dqkv, int B, int 
   const size_t dqkv_bytes = (size_t)B * N * 3 * H * d * sizeof(OutT);
   if (overlaps(dqkv, dqkv_bytes, qkv, qkv_bytes) || overlaps(dqkv, dqkv_bytes, dout, dout_bytes))
     return fail(LITELA_ERR_INVALID_ARGUMENT, "dqkv overlaps qkv or dout");
+  if (states_in != nullptr) {
+    if (reinterpret_cast<uintptr_t>(states_in) & 15u)
+      return fail(LITELA_ERR_INVALID_ARGUMENT, "states must be 16-byte aligned");
+    const int nb = (!causal || tokens_per_block >= N) ? 1 : (N + tokens_per_block - 1) / tokens_per_block;
+    if (overlaps(states_in, (size_t)B * H * nb * kStateFloats * sizeof(float), dqkv, dqkv_bytes))
+      return fail(LITELA_ERR_INVALID_ARGUMENT, "states overlaps dqkv");
+  }
   int num_sms = 0;
   s = device_setup(&num_sms);
   if (s != LITELA_OK) return s;
@@ -497,10 +518,19 @@ litela_status run_bwd(const void* qkv, const void* dout, OutT* dqkv, int B, int 
   const dim3 grid((unsigned)(plan.nblk * plan.bwd_cpb), (unsigned)plan.nquads, (unsigned)B);
   cudaError_t e;
   if (events && (e = cudaEventRecord(events[0], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  s = launch_reduce(plan, qkv, partials, ws->err, stream, pdl);
-  if (s != LITELA_OK) return s;
-  s = launch_scan(plan, partials, images, nullptr, num_sms, stream, pdl, nullptr, nullptr, images_t, false);
-  if (s != LITELA_OK) return s;
+  if (states_in == nullptr) {
+    s = launch_reduce(plan, qkv, partials, ws->err, stream, pdl);
+    if (s != LITELA_OK) return s;
+    s = launch_scan(plan, partials, images, nullptr, num_sms, stream, pdl, nullptr, nullptr, images_t, false);
+    if (s != LITELA_OK) return s;
+  } else {
+    const long long nst = (long long)B * H * plan.nblk;
+    long long grid = (nst * kStateFloats + kScanThreads - 1) / kScanThreads;
+    if (grid > num_sms) grid = num_sms;
+    e = launch_ex(litela_state_images, dim3((unsigned)grid), dim3(kScanThreads), 0, stream, pdl, states_in, images,
+                  images_t, nst);
+    if (e != cudaSuccess) return cuda_fail(e, "launch litela_state_images");
+  }
   if (events && (e = cudaEventRecord(events[1], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   e = launch_ex(litela_bwd_q_tc<OutT>, grid, dim3(kBwThreads), kBqSmemBytes, stream, pdl, map_qkv, map_g, map_dq,
                 static_cast<const uint8_t*>(images), static_cast<const uint8_t*>(images_t), dpartials, dqkv, ws->err,
@@ -670,6 +700,22 @@ litela_status lite_la_block_causal_bwd(const void* qkv, const void* dout, void* 
                                        float eps, int tokens_per_block, cudaStream_t stream) {
   return litela::run_bwd(qkv, dout, static_cast<__nv_bfloat16*>(dqkv), B, N, H, d, eps, tokens_per_block, true,
                          stream);
+}
+
+litela_status lite_la_fwd_save_state(const void* qkv, void* out, float* states, int B, int N, int H, int d,
+                                     float eps, int tokens_per_block, cudaStream_t stream) {
+  if (states == nullptr && B > 0 && N > 0 && H > 0)
+    return litela::fail(LITELA_ERR_INVALID_ARGUMENT, "null states");
+  return litela::run(qkv, static_cast<__nv_bfloat16*>(out), B, N, H, d, eps, tokens_per_block, tokens_per_block > 0,
+                     stream, nullptr, false, nullptr, nullptr, states);
+}
+
+litela_status lite_la_bwd_from_state(const void* qkv, const void* dout, const float* states, void* dqkv, int B, int N,
+                                     int H, int d, float eps, int tokens_per_block, cudaStream_t stream) {
+  if (states == nullptr && B > 0 && N > 0 && H > 0)
+    return litela::fail(LITELA_ERR_INVALID_ARGUMENT, "null states");
+  return litela::run_bwd(qkv, dout, static_cast<__nv_bfloat16*>(dqkv), B, N, H, d, eps, tokens_per_block,
+                         tokens_per_block > 0, stream, nullptr, states);
 }
 
 litela_status lite_la_bwd_f32out(const void* qkv, const void* dout, float* dqkv, int B, int N, int H, int d,

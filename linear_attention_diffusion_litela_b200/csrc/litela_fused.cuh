@@ -35,6 +35,7 @@ struct FusedPlan {
   int parity;          // which of the two counter sets this call uses (calls alternate)
   int counter_words;   // capacity of one counter set
   float eps;
+  float* states;       // when not null: the merged states, fp32 [B][H][33][32] (sibling 0 writes)
 };
 
 enum : int { kErrFusedSibling = 0x410, kErrFusedMerge = 0x420, kErrFusedP1 = 0x430 };
@@ -395,6 +396,12 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
         uint8_t* img = sbuf + hl * kImageBytes;
         *reinterpret_cast<uint4*>(img + image_offset(rr, cc * 8)) = pack_bf16x8(hi);
         *reinterpret_cast<uint4*>(img + image_offset(kImageLoRow + rr, cc * 8)) = pack_bf16x8(lo);
+        if (p.states != nullptr && r == 0 && hl < heads) {
+          float4* dst = reinterpret_cast<float4*>(
+              p.states + ((int64_t)b * p.H + q * kApUnitHeads + hl) * kStateFloats + rr * kD + cc * 8);
+          dst[0] = make_float4(sum[k][0], sum[k][1], sum[k][2], sum[k][3]);
+          dst[1] = make_float4(sum[k][4], sum[k][5], sum[k][6], sum[k][7]);
+        }
       }
       for (int i = et; i < kRedHeads * 14 * 4; i += 128) {   // zero rows 33..39, 73..79
         const int hl = i / 56, k = i - hl * 56, zr = k >> 2, cc = k & 3;

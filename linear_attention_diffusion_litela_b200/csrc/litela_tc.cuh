@@ -124,9 +124,15 @@ template <int kMap>
 struct RedCfg {
   static constexpr uint32_t kStageBytes = (kMap ? 6 : 4) * kRedBoxBytes;   // + phi(k) lo boxes
   static constexpr uint32_t kSmemBytes = kRedStages * kStageBytes + 512 + 256 + 1024;
+  // warps: 0 TMA, 1 MMA, 2.. feature map (4 for ReLU, 8 for ELU + 1); warps 2..5 also read the
+  // accumulators at the end
+  static constexpr int kMapWarps = kMap ? 8 : 4;
+  static constexpr int kThreads = 32 * (2 + kMapWarps);
 };
 
-__device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : expf(x); }
+// exp by the hardware approximation (__expf, ~2^-21 relative error here): far inside the
+// tolerance of a bf16 or fp32 result, and cheap enough for an elementwise pass over q and k
+__device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : __expf(x); }
 constexpr float kInvSqrtD = 0.17677669529663687f;   // 1 / sqrt(32): the variant's scale of phi(q)
 
 // phi = ELU + 1 of 8 packed bf16 values, times `scale`, as bf16 hi and lo (hi + lo equals the
@@ -148,7 +154,7 @@ __device__ __forceinline__ void phi_elu1_hilo(uint4 w, float scale, uint4& hi, u
 }
 
 template <int kMap>
-__global__ void __launch_bounds__(kRedThreads, 1)
+__global__ void __launch_bounds__(RedCfg<kMap>::kThreads, 1)
 litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ partials,
                  int* __restrict__ err, TcPlan p) {
   using namespace sm100;
@@ -175,7 +181,7 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
   if (threadIdx.x == 0) {
     for (int s = 0; s < kRedStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&relu_done[s], 128);
+      mbar_init(&relu_done[s], 32 * RedCfg<kMap>::kMapWarps);
       mbar_init(&empty[s], 1);
     }
     mbar_init(done, 1);
@@ -256,14 +262,15 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
       umma_commit(done);
     }
   } else {
-    const int t = threadIdx.x - 64;   // 0..127
+    constexpr int kMapThreads = 32 * RedCfg<kMap>::kMapWarps;
+    const int t = threadIdx.x - 64;
     for (int i = 0; i < ntiles; ++i) {
       const int s = i % kRedStages;
       if (!mbar_wait(&full[s], (i / kRedStages) & 1, abort_flag, err, kErrReduceRelu | s)) break;
       uint8_t* st = stages + s * kStageBytes;
       const int valid = min(kRedTile, n1 - (n0 + i * kRedTile));   // tokens of this chunk in the tile
 #pragma unroll 4
-      for (int j = t; j < 1024; j += 128) {          // k: 2 boxes x 64 rows x 8 chunks of 16 B
+      for (int j = t; j < 1024; j += kMapThreads) {   // k: 2 boxes x 64 rows x 8 chunks of 16 B
         uint4* c = reinterpret_cast<uint4*>(st + j * 16);
         const int row = (j >> 3) & (kRedTile - 1);
         if (kMap == 0) {
@@ -276,7 +283,7 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
         }
       }
       if (valid < kRedTile) {
-        for (int j = t; j < 1024; j += 128) {
+        for (int j = t; j < 1024; j += kMapThreads) {
           const int row = (j >> 3) & (kRedTile - 1);
           if (row >= valid) *reinterpret_cast<uint4*>(st + 2 * kRedBoxBytes + j * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
@@ -284,7 +291,8 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
       fence_proxy_async_smem();
       mbar_arrive(&relu_done[s]);
     }
-    // epilogue: warp quarter q reads TMEM lanes 32q..32q+31 = head q's key channels c
+    // epilogue (warps 2..5): warp quarter q reads TMEM lanes 32q..32q+31 = head q's key channels c
+    if (warp < 6) {
     const int q = warp & 3;
     float sv[kRows];
     bool ok = ntiles > 0;
@@ -308,6 +316,7 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
     float* dst = partials + ((((int64_t)b * p.ngroups + g) * nparts + x) * kRedHeads + q) * kStateFloats;
 #pragma unroll
     for (int j = 0; j < kRows; ++j) dst[j * kD + lane] = sv[j];   // S[r = j][c = lane]
+    }
   }
 
   tc_fence_before_sync();
@@ -442,6 +451,41 @@ litela_state_scan(const float* __restrict__ partials, uint8_t* __restrict__ imag
   }
 }
 
+// litela_state_images: fp32 states [n][33][32] (n = B * H * nblk, already the states the
+// queries use) -> the apply's B-operand images (bf16 hi rows 0..32, lo rows 40..72, zero rows)
+// and, when images_t is not null, the transposed images of rows 0..31.  Used by the backward
+// when the forward's states are supplied instead of recomputed.
+__global__ void __launch_bounds__(kScanThreads)
+litela_state_images(const float* __restrict__ states, uint8_t* __restrict__ images, uint8_t* __restrict__ images_t,
+                    long long n) {
+  using namespace sm100;
+  pdl_launch_dependents();
+  pdl_wait_primary();
+  const int64_t stride = (int64_t)gridDim.x * kScanThreads;
+  const int64_t tid = (int64_t)blockIdx.x * kScanThreads + threadIdx.x;
+  for (int64_t i = tid; i < n * kScanZeros; i += stride) {   // zero rows 33..39 and 73..79
+    const int64_t im = i / kScanZeros;
+    const int k = (int)(i - im * kScanZeros), zr = k >> 5, c = k & 31;
+    const int nrow = zr < 7 ? kRows + zr : kImageLoRow + kRows + (zr - 7);
+    *reinterpret_cast<__nv_bfloat16*>(images + im * kImageBytes + image_offset(nrow, c)) = __float2bfloat16_rn(0.f);
+  }
+  for (int64_t i = tid; i < n * kStateFloats; i += stride) {
+    const int64_t im = i / kStateFloats;
+    const int e = (int)(i - im * kStateFloats), r = e >> 5, c = e & 31;
+    const float v = states[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+    uint8_t* img = images + im * kImageBytes;
+    *reinterpret_cast<__nv_bfloat16*>(img + image_offset(r, c)) = hi;
+    *reinterpret_cast<__nv_bfloat16*>(img + image_offset(kImageLoRow + r, c)) = lo;
+    if (images_t != nullptr && r < kD) {
+      uint8_t* imt = images_t + im * kImageTBytes;
+      *reinterpret_cast<__nv_bfloat16*>(imt + image_offset(c, r)) = hi;
+      *reinterpret_cast<__nv_bfloat16*>(imt + image_offset(kD + c, r)) = lo;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------------------
 // apply
 
@@ -462,6 +506,10 @@ struct ApplyCfg {
   static constexpr int kQStages = kMap ? 2 : (sizeof(OutT) == 2 ? 4 : 2);
   static constexpr int kOutSlots = sizeof(OutT) == 2 ? 2 : 1;
   static constexpr int kSBufs = kMap ? 1 : (sizeof(OutT) == 2 ? 1 : 2);
+  // warps: 0 TMA, 1 MMA, 2.. feature map (2 warps for ReLU, 6 for ELU + 1), then 4 epilogue warps
+  static constexpr int kMapWarps = kMap ? 6 : 2;
+  static constexpr int kThreads = 32 * (2 + kMapWarps + 4);
+  static constexpr int kEpiWarp0 = 2 + kMapWarps;
   static constexpr int kBoxChannels = 128 / (int)sizeof(OutT);     // output channels per box
   static constexpr int kOutBoxes = kApUnitHeads * kD / kBoxChannels;
   static constexpr uint32_t kQStageBytes = (kMap ? 4 : 2) * kQBoxBytes;
@@ -559,7 +607,7 @@ __device__ __forceinline__ void pack_out(float*, const float* o, uint4* w) {
 }
 
 template <typename OutT, int kMap = 0>
-__global__ void __launch_bounds__(kApThreads, 1)
+__global__ void __launch_bounds__(ApplyCfg<OutT, kMap>::kThreads, 1)
 litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_out,
                 const uint8_t* __restrict__ images, OutT* __restrict__ out, int* __restrict__ err, TcPlan p) {
   using namespace sm100;
@@ -590,7 +638,7 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
   if (threadIdx.x == 0) {
     for (int s = 0; s < kQStages; ++s) {
       mbar_init(&qfull[s], 1);
-      mbar_init(&qrelu[s], kApReluThreads);
+      mbar_init(&qrelu[s], 32 * Cfg::kMapWarps);
       mbar_init(&qempty[s], 1);
     }
     for (int s = 0; s < kSBufs; ++s) {
@@ -726,9 +774,9 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         if (seg_ends) umma_commit(&sempty[sb]);
       }
     }
-  } else if (warp < 4) {
-    // ---- ReLU of the q tiles in place
-    const int t = threadIdx.x - 64;   // 0..63
+  } else if (warp < Cfg::kEpiWarp0) {
+    // ---- feature map of the q tiles in place (ReLU; or ELU + 1 with its lo halves)
+    const int t = threadIdx.x - 64;
     for (long long u = u0; u < u1; ++u) {
       const int lu = (int)(u - u0);
       const int s = lu % kQStages;
@@ -737,7 +785,7 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       const int nchunks = (pair_heads(p, U.quad, 1) > 0 ? 2 : 1) * (int)(kQBoxBytes / 16);
       uint8_t* st = qst + s * Cfg::kQStageBytes;
 #pragma unroll 4
-      for (int j = t; j < nchunks; j += kApReluThreads) {
+      for (int j = t; j < nchunks; j += 32 * Cfg::kMapWarps) {
         uint4* c = reinterpret_cast<uint4*>(st + j * 16);
         if (kMap == 0) {
           *c = relu_bf16x8(*c);
@@ -755,7 +803,7 @@ litela_apply_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     // ---- epilogue: TMEM -> normalise -> staged TMA store (or row stores for partial tiles)
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    const bool leader = (warp == 4 && lane == 0);
+    const bool leader = (warp == Cfg::kEpiWarp0 && lane == 0);
     int nstaged = 0, pn = 0;
     bool stop = false;
     for (long long u = u0; u < u1 && !stop; ++u) {

@@ -166,3 +166,13 @@ def test_backward_workspace_bytes(lib):
         # images (4096 B each) and dS ones rows (128 B)
         assert got >= B * H * nblk * (2 * state + 5120 + 3 * 4096 + 128)
         assert got >= ll.lite_la_workspace_bytes(B, N, H, 32, T) - 64 * 4
+
+
+def test_saved_state_entry_points_validate_on_the_host(lib):
+    a, g, o, st = (ctypes.c_void_p(1 << k) for k in (20, 24, 30, 34))
+    assert lib.lite_la_fwd_save_state(a, o, None, 1, 4, 1, 32, 1e-15, 0, None) == 1
+    assert lib.lite_la_fwd_save_state(a, o, ctypes.c_void_p((1 << 34) + 4), 1, 4, 1, 32, 1e-15, 0, None) == 1
+    assert lib.lite_la_bwd_from_state(a, g, None, o, 1, 4, 1, 32, 1e-15, 0, None) == 1
+    assert lib.lite_la_bwd_from_state(a, g, ctypes.c_void_p((1 << 34) + 8), o, 1, 4, 1, 32, 1e-15, 0, None) == 1
+    assert lib.lite_la_fwd_save_state(None, None, None, 0, 4, 1, 32, 1e-15, 0, None) == 0
+    assert lib.lite_la_bwd_from_state(a, g, st, o, 1, 4, 1, 64, 1e-15, 0, None) == 2

@@ -214,3 +214,27 @@ def test_zz_report_worst_errors():
     """Prints the largest error beyond the output rounding seen above, in units of M."""
     for k in sorted(WORST):
         print("worst excess error / M  %-5s %-3s %.3g" % (k[0], k[1], WORST[k]))
+
+
+@pytest.mark.parametrize("B,N,H,T", [(2, 1500, 9, 0), (1, 700, 600, 0), (1, 2000, 5, 256), (2, 300, 3, 1)])
+def test_forward_saves_the_state_and_the_backward_uses_it(B, N, H, T):
+    """lite_la_fwd_save_state: bitwise the plain forward's output, states equal to their
+    definition; lite_la_bwd_from_state: the backward within tolerance of the oracle."""
+    from tests.test_gpu_parity import state_reference
+    qkv = make_qkv(B, N, H, D, seed=7950 + N + H + T, device="cuda")
+    dout = make_dout(B, N, H, seed=7951 + N)
+    out, states = ll.lite_la_fwd_save_state(qkv, H, tokens_per_block=T, eps=EPS)
+    plain = ll.lite_la_fwd(qkv, H, eps=EPS) if T == 0 else ll.lite_la_block_causal_fwd(qkv, H, T, eps=EPS)
+    torch.cuda.synchronize()
+    assert torch.equal(out, plain)
+    want_states = state_reference(to_bits(qkv), B, N, H, T)
+    got_states = states.double().cpu().numpy()
+    err = np.abs(got_states - want_states)
+    assert np.all(err <= 1e-6 * (np.abs(want_states) + 1.0) * max(1.0, np.sqrt(N)))
+    dqkv = ll.lite_la_bwd_from_state(qkv, dout, states, H, tokens_per_block=T, eps=EPS)
+    torch.cuda.synchronize()
+    ll.lite_la_device_status()
+    x = dqkv.view(B, N, 3, H, D).to(torch.float64).cpu().numpy()
+    want = oracle_bwd(qkv, dout, H, T or None)
+    for i, name in enumerate(("dq", "dk", "dv")):
+        assert_grad_close(x[:, :, i], want[i], want[3 + i], "bf16", name)
