@@ -82,6 +82,10 @@ litela_status device_setup(int* num_sms) {
                                   (int)FusedCfg<__nv_bfloat16>::kSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_fused_tc<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)FusedCfg<float>::kSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_fused_tc<__nv_bfloat16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)FusedCfg<__nv_bfloat16, true>::kSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_fused_tc<float, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)FusedCfg<float, true>::kSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_bwd_q_tc<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kBqSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_bwd_q_tc<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -317,12 +321,19 @@ litela_status launch_fused(const Plan& plan, const void* qkv, OutT* out, float e
   if (events && (e = cudaEventRecord(events[0], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   // two counter sets of (ctl_words - kCounterBase) / 2 words each; calls alternate between them
   const int set_words = (int)((ctl_words - kCounterBase) / 2);
-  const FusedPlan fp{plan.B,           plan.N,    plan.H, plan.nquads, plan.fused_cpb, plan.fused_chunk,
-                     plan.fused_ntiles, (int)(call_index & 1), set_words, eps, states};
+  float* totals = plan.fused_causal ? reinterpret_cast<float*>(reinterpret_cast<char*>(partials) + plan.fused_off_totals)
+                                    : nullptr;
+  const FusedPlan fp{plan.B,   plan.N,    plan.H,     plan.nquads,      plan.fused_cpb, plan.fused_chunk,
+                     plan.fused_ntiles, (int)(call_index & 1), set_words, eps, states, plan.T, plan.nblk,
+                     plan.fused_bpc, totals};
   const unsigned grid = (unsigned)(plan.B * plan.nquads * plan.fused_cpb);
-  e = launch_ex(litela_fused_tc<OutT>, dim3(grid), dim3(kFuThreads), FusedCfg<OutT>::kSmemBytes, stream,
-                events == nullptr, map_kv, map_q, map_out, partials, reinterpret_cast<unsigned*>(ctl + kCounterBase),
-                out, ctl, fp);
+  unsigned* counters = reinterpret_cast<unsigned*>(ctl + kCounterBase);
+  if (plan.fused_causal)
+    e = launch_ex(litela_fused_tc<OutT, true>, dim3(grid), dim3(kFuThreads), FusedCfg<OutT, true>::kSmemBytes, stream,
+                  events == nullptr, map_kv, map_q, map_out, partials, counters, out, ctl, fp);
+  else
+    e = launch_ex(litela_fused_tc<OutT, false>, dim3(grid), dim3(kFuThreads), FusedCfg<OutT>::kSmemBytes, stream,
+                  events == nullptr, map_kv, map_q, map_out, partials, counters, out, ctl, fp);
   if (e != cudaSuccess) return cuda_fail(e, "launch litela_fused_tc");
   if (events && ((e = cudaEventRecord(events[1], stream)) != cudaSuccess ||
                  (e = cudaEventRecord(events[2], stream)) != cudaSuccess))
@@ -418,7 +429,7 @@ litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float 
   Plan plan;
   make_plan(B, N, H, causal ? tokens_per_block : 0, num_sms, &plan);
   if (carry || kMap != 0) {   // the carried state enters through the scan: the three-kernel path
-    plan.fused = false;
+    plan.fused = plan.fused_causal = false;
     plan.counters = 0;
   }
   if (carry) {

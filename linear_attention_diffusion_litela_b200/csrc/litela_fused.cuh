@@ -14,6 +14,12 @@
 // The arrival counters come in two sets used by alternate calls: a call zeroes the set its
 // predecessor used (after waiting for it), so a set is clean whenever it is used, even after a
 // call that gave up on a wait.
+// Block-causal form (kCausal): each CTA owns whole causal blocks [b0, b1) (at most two; the
+// block size is a multiple of 128 tokens).  Phase 1 reduces each of its blocks into its own TMEM
+// accumulator and writes the block states and their sum (the CTA's total); sibling r then waits
+// only for siblings 0..r-1, forms the prefix state of each of its blocks in fixed order (the
+// totals of siblings 0..r-1, then its own blocks one by one) and applies each block's prefix to
+// that block's tiles.
 // The only cross-CTA dependency is among the cpb siblings, which finish phase 1 at about the
 // same time.  The grid has at most one CTA per SM (its shared memory admits no second one) and
 // at most as many CTAs as SMs, so siblings are co-resident unless other kernels hold SMs, in
@@ -35,7 +41,11 @@ struct FusedPlan {
   int parity;          // which of the two counter sets this call uses (calls alternate)
   int counter_words;   // capacity of one counter set
   float eps;
-  float* states;       // when not null: the merged states, fp32 [B][H][33][32] (sibling 0 writes)
+  float* states;       // when not null: the states the queries use, fp32 [B][H][nblk][33][32]
+  // block-causal form: block size, number of blocks, blocks per CTA; the CTA totals (fp32
+  // [B][nquads][cpb][4][33][32]; the block states go to `partials`, [B][nquads][nblk][4][33][32])
+  int T, nblk, bpc;
+  float* totals;
 };
 
 enum : int { kErrFusedSibling = 0x410, kErrFusedMerge = 0x420, kErrFusedP1 = 0x430 };
@@ -45,11 +55,15 @@ constexpr int kFuThreads = 256;     // w0 TMA, w1 MMA, w2..5 phase-1 ReLU/epilog
 constexpr int kFuStages1 = 6;       // phase-1 ring of k|v stages (32 KB each)
 constexpr uint32_t kFuTmemCols = 512;
 
-template <typename OutT>
+template <typename OutT, bool kCausal = false>
 struct FusedCfg {
   using A = ApplyCfg<OutT>;
+  // the block-causal form keeps two state images (its blocks) and, for bf16 output, one q stage less
+  static constexpr int kQStages = (kCausal && sizeof(OutT) == 2) ? A::kQStages - 1 : A::kQStages;
+  static constexpr int kSBufs = kCausal ? 2 : 1;
   static constexpr uint32_t kPhase1Bytes = kFuStages1 * kRedStageBytes + 512;   // + the ones tile
-  static constexpr uint32_t kPhase2Bytes = A::kQStages * A::kQStageBytes + A::kOutSlots * A::kOutSlotBytes + kApSbufBytes;
+  static constexpr uint32_t kPhase2Bytes =
+      kQStages * A::kQStageBytes + A::kOutSlots * A::kOutSlotBytes + kSBufs * kApSbufBytes;
   static constexpr uint32_t kBodyBytes = kPhase1Bytes > kPhase2Bytes ? kPhase1Bytes : kPhase2Bytes;
   static constexpr uint32_t kSmemBytes = kBodyBytes + 512 + 1024;
   // merge batches are bulk-copied into the last q stage and the output staging region, which
@@ -58,15 +72,15 @@ struct FusedCfg {
   static constexpr int kMergeBatch = (int)(kMergeBufBytes / (kRedHeads * kStateFloats * 4));
 };
 
-template <typename OutT>
+template <typename OutT, bool kCausal = false>
 __global__ void __launch_bounds__(kFuThreads, 1)
 litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant__ CUtensorMap tmap_q,
                 const __grid_constant__ CUtensorMap tmap_out, float* __restrict__ partials,
                 unsigned* __restrict__ counters, OutT* __restrict__ out, int* __restrict__ err, FusedPlan p) {
   using namespace sm100;
-  using Cfg = FusedCfg<OutT>;
+  using Cfg = FusedCfg<OutT, kCausal>;
   using A = typename Cfg::A;
-  constexpr int kQStages = A::kQStages;
+  constexpr int kQStages = Cfg::kQStages;
   constexpr int kChunksPerHead = kD * (int)sizeof(OutT) / 16;
   constexpr uint32_t kPartBytes = kRedHeads * kStateFloats * 4;
   extern __shared__ uint8_t smem_raw[];
@@ -101,11 +115,16 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
   const int cidx = b * p.nquads + q;
   unsigned* my_counters = counters + (size_t)p.parity * p.counter_words;
   unsigned* old_counters = counters + (size_t)(p.parity ^ 1) * p.counter_words;
-  // phase 1: chunk r of batch b's tokens
-  const int n0 = r * p.chunk, n1 = min(n0 + p.chunk, p.N);
+  // phase 1: chunk r of batch b's tokens (block-causal: blocks [blk0, blk0 + nlb))
+  const int blk0 = kCausal ? r * p.bpc : 0;
+  const int nlb = kCausal ? max(0, min(blk0 + p.bpc, p.nblk) - blk0) : 1;
+  const int n0 = kCausal ? blk0 * p.T : r * p.chunk;
+  const int n1 = kCausal ? min((blk0 + nlb) * p.T, p.N) : min(n0 + p.chunk, p.N);
   const int ntiles1 = n1 > n0 ? (n1 - n0 + kRedTile - 1) / kRedTile : 0;
-  // phase 2: tiles [t0, t1) of batch b
-  const int t0 = (int)((long long)r * p.ntiles / p.cpb), t1 = (int)((long long)(r + 1) * p.ntiles / p.cpb);
+  // phase 2: tiles [t0, t1) of batch b (block-causal: the tiles of the same blocks)
+  const int t0 = kCausal ? n0 / kApTile : (int)((long long)r * p.ntiles / p.cpb);
+  const int t1 = kCausal ? (n1 > n0 ? (n1 + kApTile - 1) / kApTile : t0)
+                         : (int)((long long)(r + 1) * p.ntiles / p.cpb);
   const int nunits = t1 - t0;
 
   pdl_launch_dependents();   // the next kernel waits for this grid before touching memory
@@ -179,19 +198,23 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
       constexpr uint32_t idesc_num = idesc_bf16_f32(128, 128, true, true);
       constexpr uint32_t idesc_den = idesc_bf16_f32(128, 16, true, false);
       const uint64_t ones_desc = smem_desc(smem_u32(ones), 128, 256, kSwizzleNone);
+      const int tpb = kCausal ? p.T / kRedTile : 1;   // tiles per causal block
       for (int i = 0; i < ntiles1; ++i) {
         const int s = i % kFuStages1;
         if (!mbar_wait(&relu_done[s], (i / kFuStages1) & 1, abort_flag, err, kErrFusedP1 | 8 | s)) break;
         tc_fence_after_sync();
         const uint32_t kbase = smem_u32(stages + s * kRedStageBytes);
         const uint32_t vbase = kbase + 2 * kRedBoxBytes;
+        // block-causal: local block i / tpb accumulates in its own 256-column TMEM region
+        const uint32_t dacc = tmem + (kCausal ? (uint32_t)(i / tpb) * 256u : 0u);
+        const bool first = kCausal ? (i % tpb) == 0 : i == 0;
 #pragma unroll
         for (int ks = 0; ks < kRedTile / 16; ++ks) {
           const uint64_t a = smem_desc(kbase + ks * 2048, kRedBoxBytes, 1024, kSwizzle128B);
           const uint64_t bv = smem_desc(vbase + ks * 2048, kRedBoxBytes, 1024, kSwizzle128B);
-          const uint32_t acc = (i | ks) != 0;
-          umma_bf16(tmem, a, bv, idesc_num, acc);
-          umma_bf16(tmem + 128, a, ones_desc, idesc_den, acc);
+          const uint32_t acc = (!first || ks != 0) ? 1u : 0u;
+          umma_bf16(dacc, a, bv, idesc_num, acc);
+          umma_bf16(dacc + 128, a, ones_desc, idesc_den, acc);
         }
         umma_commit(&empty[s]);
       }
@@ -220,27 +243,41 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
       mbar_arrive(&relu_done[s]);
     }
     const int hq = warp & 3;
-    float sv[kRows];
+    float sv[kRows], tot[kRows];
+#pragma unroll
+    for (int j = 0; j < kRows; ++j) tot[j] = 0.f;
     bool ok = ntiles1 > 0;
     if (ok) ok = mbar_wait(done, 0, abort_flag, err, kErrFusedP1 | 13);
     ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
-      tc_fence_after_sync();
-      uint32_t rr[32], zr;
-      const uint32_t ta = tmem + (static_cast<uint32_t>(hq * 32) << 16);
-      tmem_ld_x32(ta + hq * 32, rr);
-      tmem_ld_x1(ta + 128, zr);
-      tmem_wait_ld();
+    for (int lb = 0; lb < nlb; ++lb) {   // non-causal: the one accumulator
+      if (ok) {
+        tc_fence_after_sync();
+        uint32_t rr[32], zr;
+        const uint32_t ta = tmem + (static_cast<uint32_t>(hq * 32) << 16) + (uint32_t)lb * 256u;
+        tmem_ld_x32(ta + hq * 32, rr);
+        tmem_ld_x1(ta + 128, zr);
+        tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(rr[j]);
-      sv[32] = __uint_as_float(zr);
-    } else {
+        for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(rr[j]);
+        sv[32] = __uint_as_float(zr);
+      } else {
 #pragma unroll
-      for (int j = 0; j < kRows; ++j) sv[j] = 0.f;
+        for (int j = 0; j < kRows; ++j) sv[j] = 0.f;
+      }
+      // non-causal: this sibling's partial; block-causal: the state of block blk0 + lb
+      float* dst = partials + (((int64_t)cidx * (kCausal ? p.nblk : p.cpb) + (kCausal ? blk0 + lb : r)) * kRedHeads + hq) *
+                                  kStateFloats;
+#pragma unroll
+      for (int j = 0; j < kRows; ++j) {
+        dst[j * kD + lane] = sv[j];
+        tot[j] += sv[j];
+      }
     }
-    float* dst = partials + (((int64_t)cidx * p.cpb + r) * kRedHeads + hq) * kStateFloats;
+    if (kCausal) {   // the sum of this CTA's blocks, for the siblings after it
+      float* dst = p.totals + (((int64_t)cidx * p.cpb + r) * kRedHeads + hq) * kStateFloats;
 #pragma unroll
-    for (int j = 0; j < kRows; ++j) dst[j * kD + lane] = sv[j];
+      for (int j = 0; j < kRows; ++j) dst[j * kD + lane] = tot[j];
+    }
   }
   // phase 1 is over for this CTA: every MMA completed (the epilogue waited for `done`), every
   // TMEM read completed, the partial is written
@@ -248,7 +285,10 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
   __threadfence();
   __syncthreads();
   tc_fence_after_sync();
-  if (threadIdx.x == 0) atomicAdd(&my_counters[cidx], 1u);   // arrival of this sibling
+  if (threadIdx.x == 0) {   // arrival of this sibling (block-causal: its own flag)
+    if (kCausal) atomicExch(&my_counters[cidx * p.cpb + r], 1u);
+    else atomicAdd(&my_counters[cidx], 1u);
+  }
 
   // =============================== phase 2: merge + apply ================================
   if (warp == 0) {
@@ -283,6 +323,8 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
         const int s = lu % kQStages;
         if (!mbar_wait(&qrelu[s], (lu / kQStages) & 1, abort_flag, err, kErrApplyMma | s)) break;
         const uint32_t qaddr = smem_u32(qst + s * A::kQStageBytes);
+        // block-causal: the image of the tile's block
+        const uint32_t iaddr = saddr + (kCausal ? (uint32_t)(((t0 + lu) * kApTile - n0) / p.T) * kApSbufBytes : 0u);
         for (int h = 0; h < 2; ++h) {
           const int nh = pair_heads_h(p.H, q, h);
           if (nh == 0) break;
@@ -297,7 +339,7 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
 #pragma unroll
             for (int ks = 0; ks < 2; ++ks) {
               const uint64_t ad = smem_desc(qaddr + h * kQBoxBytes + j * 64 + ks * 32, 16, 1024, kSwizzle128B);
-              const uint64_t bd = smem_desc(saddr + (h * kApHeads + j) * kImageBytes + ks * 256, 128, 512, kSwizzleNone);
+              const uint64_t bd = smem_desc(iaddr + (h * kApHeads + j) * kImageBytes + ks * 256, 128, 512, kSwizzleNone);
               umma_bf16(tmem + a * kApAccCols + j * kImageRows, ad, bd, idesc, ks);
             }
           }
@@ -326,20 +368,24 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
   } else if (warp < 8) {
     const int et = threadIdx.x - 128;   // 0..127
     const bool leader = (et == 0);
-    // ---- merge: wait for the siblings, sum their partials in fixed order, build the B operand
+    // ---- merge: wait for the siblings, sum their partials in fixed order, build the B operand.
+    // Non-causal: all cpb siblings' partials, then one image.  Block-causal: the totals of
+    // siblings 0..r-1, then this CTA's block states one by one, an image after each.
     bool ok = true;
     if (leader) {
       const uint64_t tstart = globaltimer_ns();
-      volatile unsigned* arr = my_counters + cidx;
-      while (*arr < (unsigned)p.cpb) {
-        if (*abort_flag) { ok = false; break; }
-        if (globaltimer_ns() - tstart > kWaitLimitNs) {
-          *abort_flag = 1;
-          atomicCAS(err, 0, kErrFusedSibling);
-          ok = false;
-          break;
+      for (int w = 0; ok && w < (kCausal ? r : 1); ++w) {
+        volatile unsigned* arr = my_counters + (kCausal ? cidx * p.cpb + w : cidx);
+        while (kCausal ? *arr == 0u : *arr < (unsigned)p.cpb) {
+          if (*abort_flag) { ok = false; break; }
+          if (globaltimer_ns() - tstart > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicCAS(err, 0, kErrFusedSibling);
+            ok = false;
+            break;
+          }
+          __nanosleep(256);
         }
-        __nanosleep(256);
       }
       __threadfence();   // acquire: the siblings' partial writes precede their arrivals
     }
@@ -352,35 +398,8 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
     for (int k = 0; k < kUPT; ++k)
 #pragma unroll
       for (int i = 0; i < 8; ++i) sum[k][i] = 0.f;
-    const uint8_t* gsrc = reinterpret_cast<const uint8_t*>(partials) + (int64_t)cidx * p.cpb * kPartBytes;
-    int batch = 0;
-    for (int k0 = 0; ok && k0 < p.cpb; k0 += Cfg::kMergeBatch, ++batch) {
-      const int nb = min(Cfg::kMergeBatch, p.cpb - k0);
-      if (leader) {
-        fence_proxy_async_global();
-        mbar_arrive_expect_tx(merge_bar, nb * kPartBytes);
-        for (int i = 0; i < nb; ++i) bulk_load(mbuf + i * kPartBytes, gsrc + (int64_t)(k0 + i) * kPartBytes, kPartBytes, merge_bar);
-      }
-      const bool got = mbar_wait(merge_bar, batch & 1, abort_flag, err, kErrFusedMerge);
-      if (bar_any(1, 128, !got)) {
-        ok = false;
-        break;
-      }
-#pragma unroll
-      for (int k = 0; k < kUPT; ++k) {
-        const int u = et + k * 128;
-        if (u >= kUnits) break;
-        const int hl = u / (kRows * 4), rcc = u - hl * (kRows * 4), rr = rcc >> 2, cc = rcc & 3;
-        for (int i = 0; i < nb; ++i) {
-          const float4* src = reinterpret_cast<const float4*>(mbuf + i * kPartBytes) + (hl * kStateFloats + rr * kD + cc * 8) / 4;
-          const float4 x0 = src[0], x1 = src[1];
-          sum[k][0] += x0.x; sum[k][1] += x0.y; sum[k][2] += x0.z; sum[k][3] += x0.w;
-          sum[k][4] += x1.x; sum[k][5] += x1.y; sum[k][6] += x1.z; sum[k][7] += x1.w;
-        }
-      }
-      bar_sync(2, 128);   // the batch buffer is refilled next
-    }
-    if (ok) {
+    // the image (and, when requested, the fp32 state) of the running sums, for image slot `slot`
+    auto emit = [&](int slot) {
 #pragma unroll
       for (int k = 0; k < kUPT; ++k) {
         const int u = et + k * 128;
@@ -393,12 +412,12 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
           hi[j] = __bfloat162float(__float2bfloat16_rn(v));
           lo[j] = v - hi[j];
         }
-        uint8_t* img = sbuf + hl * kImageBytes;
+        uint8_t* img = sbuf + slot * kApSbufBytes + hl * kImageBytes;
         *reinterpret_cast<uint4*>(img + image_offset(rr, cc * 8)) = pack_bf16x8(hi);
         *reinterpret_cast<uint4*>(img + image_offset(kImageLoRow + rr, cc * 8)) = pack_bf16x8(lo);
-        if (p.states != nullptr && r == 0 && hl < heads) {
-          float4* dst = reinterpret_cast<float4*>(
-              p.states + ((int64_t)b * p.H + q * kApUnitHeads + hl) * kStateFloats + rr * kD + cc * 8);
+        if (p.states != nullptr && (kCausal || r == 0) && hl < heads) {
+          const int64_t st = ((int64_t)b * p.H + q * kApUnitHeads + hl) * (kCausal ? p.nblk : 1) + (kCausal ? blk0 + slot : 0);
+          float4* dst = reinterpret_cast<float4*>(p.states + st * kStateFloats + rr * kD + cc * 8);
           dst[0] = make_float4(sum[k][0], sum[k][1], sum[k][2], sum[k][3]);
           dst[1] = make_float4(sum[k][4], sum[k][5], sum[k][6], sum[k][7]);
         }
@@ -406,10 +425,47 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
       for (int i = et; i < kRedHeads * 14 * 4; i += 128) {   // zero rows 33..39, 73..79
         const int hl = i / 56, k = i - hl * 56, zr = k >> 2, cc = k & 3;
         const int nrow = zr < 7 ? kRows + zr : kImageLoRow + kRows + (zr - 7);
-        *reinterpret_cast<uint4*>(sbuf + hl * kImageBytes + image_offset(nrow, cc * 8)) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(sbuf + slot * kApSbufBytes + hl * kImageBytes + image_offset(nrow, cc * 8)) =
+            make_uint4(0u, 0u, 0u, 0u);
       }
-      fence_proxy_async_smem();
+    };
+    // source k of the merge (global memory)
+    const int nsrc = kCausal ? r + nlb : p.cpb;
+    auto source = [&](int k) -> const uint8_t* {
+      if (!kCausal) return reinterpret_cast<const uint8_t*>(partials) + ((int64_t)cidx * p.cpb + k) * kPartBytes;
+      if (k < r) return reinterpret_cast<const uint8_t*>(p.totals) + ((int64_t)cidx * p.cpb + k) * kPartBytes;
+      return reinterpret_cast<const uint8_t*>(partials) + ((int64_t)cidx * p.nblk + blk0 + (k - r)) * kPartBytes;
+    };
+    int batch = 0;
+    for (int k0 = 0; ok && k0 < nsrc; k0 += Cfg::kMergeBatch, ++batch) {
+      const int nb = min(Cfg::kMergeBatch, nsrc - k0);
+      if (leader) {
+        fence_proxy_async_global();
+        mbar_arrive_expect_tx(merge_bar, nb * kPartBytes);
+        for (int i = 0; i < nb; ++i) bulk_load(mbuf + i * kPartBytes, source(k0 + i), kPartBytes, merge_bar);
+      }
+      const bool got = mbar_wait(merge_bar, batch & 1, abort_flag, err, kErrFusedMerge);
+      if (bar_any(1, 128, !got)) {
+        ok = false;
+        break;
+      }
+      for (int i = 0; i < nb; ++i) {
+#pragma unroll
+        for (int k = 0; k < kUPT; ++k) {
+          const int u = et + k * 128;
+          if (u >= kUnits) break;
+          const int hl = u / (kRows * 4), rcc = u - hl * (kRows * 4), rr = rcc >> 2, cc = rcc & 3;
+          const float4* src = reinterpret_cast<const float4*>(mbuf + i * kPartBytes) + (hl * kStateFloats + rr * kD + cc * 8) / 4;
+          const float4 x0 = src[0], x1 = src[1];
+          sum[k][0] += x0.x; sum[k][1] += x0.y; sum[k][2] += x0.z; sum[k][3] += x0.w;
+          sum[k][4] += x1.x; sum[k][5] += x1.y; sum[k][6] += x1.z; sum[k][7] += x1.w;
+        }
+        if (kCausal && k0 + i >= r) emit(k0 + i - r);   // the prefix state of block blk0 + (k - r)
+      }
+      bar_sync(2, 128);   // the batch buffer is refilled next
     }
+    if (ok && !kCausal) emit(0);
+    if (ok) fence_proxy_async_smem();
     bar_sync(2, 128);
     if (leader && ok) mbar_arrive(sfull);
     // ---- epilogue (as litela_apply_tc; the merge buffer overlapped the output staging region)

@@ -56,6 +56,12 @@ struct Plan {
   bool fused = false;
   int fused_cpb = 0, fused_chunk = 0, fused_ntiles = 0;
   size_t fused_bytes = 0, counters = 0;
+  // block-causal fused path (fused_causal): CTA (b, quad, r) owns blocks [r * fused_bpc, ...),
+  // at most 2; workspace = block states [B][nquads][nblk][4][33][32], then the CTA totals
+  // [B][nquads][fused_cpb][4][33][32] at fused_off_totals; counters = 2 sets of one flag per CTA
+  bool fused_causal = false;
+  int fused_bpc = 0;
+  size_t fused_off_totals = 0;
   // backward (make_bwd_plan): the forward's reduction and scan (partials, images above), then
   //   S^T images bf16 [B][H][nblk][kImageTBytes]                       at off_images_t
   //   dS partials fp32 [B][nquads][nblk * bwd_cpb][4][33][32]           at off_dpartials
@@ -107,6 +113,21 @@ inline bool make_plan(int B, int N, int H, int tokens_per_block, int num_sms, Pl
     p->fused_chunk = (int)chunk;
     p->fused_bytes = align_up((size_t)B * p->nquads * cpb * kRedHeads * kStateFloats * sizeof(float), 256);
     p->counters = (size_t)2 * B * p->nquads;   // both sets
+  } else if (p->nblk > 1 && p->T % kApTile == 0 && (int64_t)B * p->nquads <= sms) {
+    int cpb = sms / (B * p->nquads);
+    if (cpb > p->nblk) cpb = p->nblk;
+    const int bpc = (p->nblk + cpb - 1) / cpb;
+    if (bpc <= 2) {   // each CTA keeps the images of its blocks in shared memory
+      cpb = (p->nblk + bpc - 1) / bpc;
+      p->fused = p->fused_causal = true;
+      p->fused_cpb = cpb;
+      p->fused_bpc = bpc;
+      p->fused_ntiles = (N + kApTile - 1) / kApTile;
+      const size_t part = (size_t)kRedHeads * kStateFloats * sizeof(float);
+      p->fused_off_totals = align_up((size_t)B * p->nquads * p->nblk * part, 256);
+      p->fused_bytes = p->fused_off_totals + align_up((size_t)B * p->nquads * cpb * part, 256);
+      p->counters = (size_t)2 * B * p->nquads * cpb;   // both sets
+    }
   }
   return true;
 }

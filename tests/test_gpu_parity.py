@@ -333,7 +333,9 @@ def test_state_carry_without_state_in_is_the_plain_block_causal_call():
     out, st = ll.lite_la_block_causal_fwd_carry(qkv, H, T, eps=EPS, out_dtype=torch.float32)
     ref = ll.lite_la_block_causal_fwd(qkv, H, T, eps=EPS, out_dtype=torch.float32)
     torch.cuda.synchronize()
-    assert torch.equal(out, ref)                      # same kernels, same order: bitwise
+    # the plain call may take the fused block-causal kernel, which sums the block states in
+    # another (fixed) order than the carry path's scan: equal to fp32 rounding, not bitwise
+    assert torch.allclose(out, ref, rtol=1e-5, atol=1e-6)
     full = ll.lite_la_state_fwd(qkv, H, 0)
     torch.cuda.synchronize()
     assert torch.allclose(st, full[:, :, 0], rtol=1e-6, atol=1e-5)
