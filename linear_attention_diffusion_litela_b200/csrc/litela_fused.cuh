@@ -109,23 +109,9 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q = blockIdx.x % p.nquads;
-  const int br = blockIdx.x / p.nquads;
-  const int r = br % p.cpb, b = br / p.cpb;
-  const int cidx = b * p.nquads + q;
   unsigned* my_counters = counters + (size_t)p.parity * p.counter_words;
   unsigned* old_counters = counters + (size_t)(p.parity ^ 1) * p.counter_words;
-  // phase 1: chunk r of batch b's tokens (block-causal: blocks [blk0, blk0 + nlb))
-  const int blk0 = kCausal ? r * p.bpc : 0;
-  const int nlb = kCausal ? max(0, min(blk0 + p.bpc, p.nblk) - blk0) : 1;
-  const int n0 = kCausal ? blk0 * p.T : r * p.chunk;
-  const int n1 = kCausal ? min((blk0 + nlb) * p.T, p.N) : min(n0 + p.chunk, p.N);
-  const int ntiles1 = n1 > n0 ? (n1 - n0 + kRedTile - 1) / kRedTile : 0;
-  // phase 2: tiles [t0, t1) of batch b (block-causal: the tiles of the same blocks)
-  const int t0 = kCausal ? n0 / kApTile : (int)((long long)r * p.ntiles / p.cpb);
-  const int t1 = kCausal ? (n1 > n0 ? (n1 + kApTile - 1) / kApTile : t0)
-                         : (int)((long long)(r + 1) * p.ntiles / p.cpb);
-  const int nunits = t1 - t0;
+  int* ticket_slot = reinterpret_cast<int*>(tmem_holder + 2);
 
   pdl_launch_dependents();   // the next kernel waits for this grid before touching memory
   if (threadIdx.x == 0) {
@@ -166,8 +152,28 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
   const uint32_t tmem = *tmem_holder;
   // private set-up above; global memory only after the previous kernel in the stream is done
   pdl_wait_primary();
+  // The CTA's role (batch, quad, sibling) comes from a ticket taken in arrival order, siblings
+  // on consecutive tickets: whatever subset of the grid is resident (other kernels may hold SMs),
+  // it holds whole sibling groups before any later CTA, so every wait below can be satisfied.
+  if (threadIdx.x == 0) *ticket_slot = (int)atomicAdd(&my_counters[p.counter_words - 1], 1u);
   for (int i = blockIdx.x * kFuThreads + threadIdx.x; i < p.counter_words; i += gridDim.x * kFuThreads)
     old_counters[i] = 0u;   // the previous call's set: clean for the call after this one
+  __syncthreads();
+  const int ticket = *ticket_slot;
+  const int r = ticket % p.cpb, qb = ticket / p.cpb;
+  const int q = qb % p.nquads, b = qb / p.nquads;
+  const int cidx = b * p.nquads + q;
+  // phase 1: chunk r of batch b's tokens (block-causal: blocks [blk0, blk0 + nlb))
+  const int blk0 = kCausal ? r * p.bpc : 0;
+  const int nlb = kCausal ? max(0, min(blk0 + p.bpc, p.nblk) - blk0) : 1;
+  const int n0 = kCausal ? blk0 * p.T : r * p.chunk;
+  const int n1 = kCausal ? min((blk0 + nlb) * p.T, p.N) : min(n0 + p.chunk, p.N);
+  const int ntiles1 = n1 > n0 ? (n1 - n0 + kRedTile - 1) / kRedTile : 0;
+  // phase 2: tiles [t0, t1) of batch b (block-causal: the tiles of the same blocks)
+  const int t0 = kCausal ? n0 / kApTile : (int)((long long)r * p.ntiles / p.cpb);
+  const int t1 = kCausal ? (n1 > n0 ? (n1 + kApTile - 1) / kApTile : t0)
+                         : (int)((long long)(r + 1) * p.ntiles / p.cpb);
+  const int nunits = t1 - t0;
 
   // =============================== phase 1: state reduction ===============================
   const int kx = p.H * kD + q * (kRedHeads * kD), vx = 2 * p.H * kD + q * (kRedHeads * kD);

@@ -52,7 +52,7 @@ struct Plan {
   size_t off_images = 0, bytes = 0;
   // fused single-kernel path (non-causal, B * nquads <= SMs): CTA (b, quad, r), r < fused_cpb;
   // workspace = fused partials [B][nquads][fused_cpb][4][33][32]; two sets of B * nquads
-  // arrival counters (calls alternate between them)
+  // arrival counters and a ticket counter (calls alternate between the sets)
   bool fused = false;
   int fused_cpb = 0, fused_chunk = 0, fused_ntiles = 0;
   size_t fused_bytes = 0, counters = 0;
@@ -112,7 +112,7 @@ inline bool make_plan(int B, int N, int H, int tokens_per_block, int num_sms, Pl
     p->fused_cpb = cpb;
     p->fused_chunk = (int)chunk;
     p->fused_bytes = align_up((size_t)B * p->nquads * cpb * kRedHeads * kStateFloats * sizeof(float), 256);
-    p->counters = (size_t)2 * B * p->nquads;   // both sets
+    p->counters = (size_t)2 * (B * p->nquads + 1);   // both sets; the last word of a set: the ticket
   } else if (p->nblk > 1 && p->T % kApTile == 0 && (int64_t)B * p->nquads <= sms) {
     int cpb = sms / (B * p->nquads);
     if (cpb > p->nblk) cpb = p->nblk;
@@ -126,7 +126,7 @@ inline bool make_plan(int B, int N, int H, int tokens_per_block, int num_sms, Pl
       const size_t part = (size_t)kRedHeads * kStateFloats * sizeof(float);
       p->fused_off_totals = align_up((size_t)B * p->nquads * p->nblk * part, 256);
       p->fused_bytes = p->fused_off_totals + align_up((size_t)B * p->nquads * cpb * part, 256);
-      p->counters = (size_t)2 * B * p->nquads * cpb;   // both sets
+      p->counters = (size_t)2 * ((size_t)B * p->nquads * cpb + 1);   // both sets, each with its ticket word
     }
   }
   return true;

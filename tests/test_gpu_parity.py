@@ -368,3 +368,28 @@ def test_phase_timed_calls_give_the_plain_calls_result(B, N, H, T):
     assert evs[0].elapsed_time(evs[2]) > 0.0
     null = (ctypes.c_void_p * 3)(None, None, None)
     assert lib.lite_la_fwd_events(qkv.data_ptr(), out.data_ptr(), B, N, H, 32, EPS, sh, null) == 1
+
+
+@pytest.mark.parametrize("T", [0, 1024])
+def test_concurrent_fused_calls_on_two_streams(T):
+    """Two fused calls at once on two streams: each grid alone fills the SMs, so only part of
+    each can be resident; CTAs take their roles by ticket in arrival order, so both complete.
+    The results equal the single-stream ones bitwise and no wait times out."""
+    B, N, H = (2, 8192, 70) if T == 0 else (1, 16384, 70)
+    xa = make_qkv(B, N, H, 32, seed=6100 + T, device="cuda")
+    xb = make_qkv(B, N, H, 32, seed=6200 + T, device="cuda")
+    run = (lambda x, **kw: ll.lite_la_fwd(x, H, eps=EPS, **kw)) if T == 0 else \
+        (lambda x, **kw: ll.lite_la_block_causal_fwd(x, H, T, eps=EPS, **kw))
+    assert ll.lib().lite_la_kernels_per_call(B, N, H, 32, T) == 1
+    ra, rb = run(xa), run(xb)
+    torch.cuda.synchronize()
+    sa, sb = torch.cuda.Stream(), torch.cuda.Stream()
+    for _ in range(5):
+        with torch.cuda.stream(sa):
+            oa = run(xa, stream=sa)
+        with torch.cuda.stream(sb):
+            ob = run(xb, stream=sb)
+        torch.cuda.synchronize()
+        ll.lite_la_device_status(sa)
+        ll.lite_la_device_status(sb)
+        assert torch.equal(oa, ra) and torch.equal(ob, rb)
