@@ -486,7 +486,7 @@ def main():
     alg_bytes = {k: PATHS[nk]["alg_bytes_E"][k] * E for k in phases}
     peaks = load_peaks()
     dom = max(kern_us, key=kern_us.get)
-    traffic = load_traffic(dom, B, N, H, T)
+    traffic = load_traffic(dom, B, N, H, T, "bwd" if bwd else ("elu1_fwd" if args.variant == "elu1" else "fwd"))
     achieved = alg_bytes[dom] / (kern_us[dom] * 1e-6) / 1e9
     peak, unit = peaks["hbm_gbs"], "GB/s"
     peak_note = "%s copy bandwidth" % peaks["_source"]
@@ -608,10 +608,10 @@ def main():
     return 0
 
 
-def load_traffic(kernel, B, N, H, T):
+def load_traffic(kernel, B, N, H, T, call="fwd"):
     """DRAM bytes per launch of `kernel` (a phase name may join several kernels with '+') on a
-    call of this shape, from the committed ncu summaries; None when there is none or the kernel
-    sources changed since it was taken."""
+    call of this kind ("fwd", "bwd", "elu1_fwd") and shape, from the committed ncu summaries;
+    None when there is none or the kernel sources changed since it was taken."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
@@ -620,7 +620,8 @@ def load_traffic(kernel, B, N, H, T):
     h = sources_hash()
     total = 0
     for k in kernel.split("+"):
-        ent = [e for e in d.get("entries", []) if e["kernel"] == k and [e["B"], e["N"], e["H"], e["T"]] == [B, N, H, T]]
+        ent = [e for e in d.get("entries", []) if e["kernel"] == k and e.get("call", "fwd") == call
+               and [e["B"], e["N"], e["H"], e["T"]] == [B, N, H, T]]
         if not ent or ent[0].get("sources_sha256") != h:
             return None
         total += ent[0]["dram_bytes_per_launch"]

@@ -153,9 +153,8 @@ litela_status encode_out_map(OutT* out, int B, int N, int H, CUtensorMap* map) {
 struct Workspace {
   void* partials = nullptr;   // partial states (and, for the three-kernel path, state images)
   size_t partials_bytes = 0;
-  int* err = nullptr;         // control words: error word, then the fused kernel's two counter sets
+  int* err = nullptr;         // control words: error word, then the fused kernel's counters
   size_t ctl_words = 0;
-  unsigned long long calls = 0;   // fused calls so far: their parity selects the counter set
 };
 
 // bytes of partial-state workspace a call with `plan` uses
@@ -308,7 +307,7 @@ litela_status launch_scan(const Plan& plan, const float* partials, uint8_t* imag
 // events, if requested, bracket it (events[1] is recorded with events[2], after the kernel).
 template <typename OutT>
 litela_status launch_fused(const Plan& plan, const void* qkv, OutT* out, float eps, float* partials, int* ctl,
-                           size_t ctl_words, unsigned long long call_index, cudaStream_t stream,
+                           size_t ctl_words, cudaStream_t stream,
                            cudaEvent_t* events, float* states = nullptr) {
   CUtensorMap map_kv, map_q, map_out;
   litela_status s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kRedTile, &map_kv);
@@ -319,12 +318,12 @@ litela_status launch_fused(const Plan& plan, const void* qkv, OutT* out, float e
   if (s != LITELA_OK) return s;
   cudaError_t e;
   if (events && (e = cudaEventRecord(events[0], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  // two counter sets of (ctl_words - kCounterBase) / 2 words each; calls alternate between them
-  const int set_words = (int)((ctl_words - kCounterBase) / 2);
+  // the fused kernel's control words: every word after kCounterBase (the last two: finish, ticket)
+  const int set_words = (int)(ctl_words - kCounterBase);
   float* totals = plan.fused_causal ? reinterpret_cast<float*>(reinterpret_cast<char*>(partials) + plan.fused_off_totals)
                                     : nullptr;
   const FusedPlan fp{plan.B,   plan.N,    plan.H,     plan.nquads,      plan.fused_cpb, plan.fused_chunk,
-                     plan.fused_ntiles, (int)(call_index & 1), set_words, eps, states, plan.T, plan.nblk,
+                     plan.fused_ntiles, set_words, eps, states, plan.T, plan.nblk,
                      plan.fused_bpc, totals};
   const unsigned grid = (unsigned)(plan.B * plan.nquads * plan.fused_cpb);
   unsigned* counters = reinterpret_cast<unsigned*>(ctl + kCounterBase);
@@ -452,7 +451,7 @@ litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float 
                            reinterpret_cast<uint8_t*>(base + plan.off_images), ws->err, num_sms, stream, events,
                            state_in, state_out);
   else if (plan.fused)
-    s = launch_fused(plan, qkv, out, eps, reinterpret_cast<float*>(base), ws->err, ws->ctl_words, ws->calls++, stream,
+    s = launch_fused(plan, qkv, out, eps, reinterpret_cast<float*>(base), ws->err, ws->ctl_words, stream,
                      events, save_states);
   else
     s = launch<OutT, kMap>(plan, qkv, out, eps, reinterpret_cast<float*>(base),
@@ -610,7 +609,7 @@ litela_status run_noalloc(const void* qkv, __nv_bfloat16* out, int B, int N, int
     cudaError_t e = cudaMemsetAsync(base + kCounterBase * sizeof(int), 0, plan.counters * sizeof(unsigned), stream);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(no-alloc counters)");
     s = launch_fused(plan, qkv, out, eps, reinterpret_cast<float*>(base + err_bytes), reinterpret_cast<int*>(base),
-                     kCounterBase + plan.counters, 0, stream, nullptr);
+                     kCounterBase + plan.counters, stream, nullptr);
     if (s == LITELA_OK) g_last_error.clear();
     return s;
   }
@@ -810,7 +809,8 @@ litela_status lite_la_device_status(cudaStream_t stream) {
       if (code == 0) code = v;
       if ((e = cudaMemset(w, 0, sizeof(int))) != cudaSuccess)
         return litela::cuda_fail(e, "clearing the device error word");
-      // an aborted fused call may have left sibling counters set: clear them too
+      // the fused kernel's last CTA leaves its counters clean even after a time-out; clear them
+      // anyway, in case a call ended without reaching that point
       size_t words = 0;
       if (w == words_ws0) words = ctl_words_ws;
       if (words > (size_t)litela::kCounterBase &&

@@ -11,9 +11,12 @@
 //            quad's state as the MMA's B operand (bf16 hi + lo, as litela_state_scan does);
 //   phase 2  applies the state to tiles [r*ntiles/cpb, (r+1)*ntiles/cpb) of batch b's tokens
 //            exactly as litela_apply_tc does (its q prefetch overlaps the merge).
-// The arrival counters come in two sets used by alternate calls: a call zeroes the set its
-// predecessor used (after waiting for it), so a set is clean whenever it is used, even after a
-// call that gave up on a wait.
+// Cross-CTA control words (one set per stream's workspace): the arrival counters, a finish
+// counter and a ticket counter.  The arrival and finish counters are touched only after the
+// previous kernel in the stream has completed (the programmatic-launch wait), and the CTA that
+// counts itself out last zeroes them; the ticket counter is reset by the CTA that takes the
+// last ticket, before the grid releases the next kernels.  So every call, eager or replayed
+// from a captured graph, finds them clean.
 // Block-causal form (kCausal): each CTA owns whole causal blocks [b0, b1) (at most two; the
 // block size is a multiple of 128 tokens).  Phase 1 reduces each of its blocks into its own TMEM
 // accumulator and writes the block states and their sum (the CTA's total); sibling r then waits
@@ -38,8 +41,7 @@ namespace litela {
 
 struct FusedPlan {
   int B, N, H, nquads, cpb, chunk, ntiles;
-  int parity;          // which of the two counter sets this call uses (calls alternate)
-  int counter_words;   // capacity of one counter set
+  int counter_words;   // control words: arrival counters, then the finish and ticket counters
   float eps;
   float* states;       // when not null: the states the queries use, fp32 [B][H][nblk][33][32]
   // block-causal form: block size, number of blocks, blocks per CTA; the CTA totals (fp32
@@ -48,7 +50,7 @@ struct FusedPlan {
   float* totals;
 };
 
-enum : int { kErrFusedSibling = 0x410, kErrFusedMerge = 0x420, kErrFusedP1 = 0x430 };
+enum : int { kErrFusedSibling = 0x410, kErrFusedMerge = 0x420, kErrFusedP1 = 0x430, kErrFusedTicket = 0x440 };
 
 constexpr int kFuThreads = 256;     // w0 TMA, w1 MMA, w2..5 phase-1 ReLU/epilogue; phase 2: w2..3 ReLU,
                                     // w4..7 merge then epilogue
@@ -105,16 +107,24 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
   uint64_t* tfull = sfull + 1;
   uint64_t* tempty = tfull + kApAccSlots;
   uint64_t* merge_bar = tempty + kApAccSlots;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(merge_bar + 1);
+  uint64_t* wait_done = merge_bar + 1;          // the merge leader's sibling wait is over
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(wait_done + 1);
+  // mbarriers above, then tmem_holder, abort flag and ticket: in the 512 bytes after the body
+  static_assert((3 * kFuStages1 + 1 + 3 * kQStages + 1 + 2 * kApAccSlots + 2) * 8 + 3 * 4 <= 512,
+                "fused kernel: barrier area");
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  unsigned* my_counters = counters + (size_t)p.parity * p.counter_words;
-  unsigned* old_counters = counters + (size_t)(p.parity ^ 1) * p.counter_words;
+  unsigned* my_counters = counters;
   int* ticket_slot = reinterpret_cast<int*>(tmem_holder + 2);
 
-  pdl_launch_dependents();   // the next kernel waits for this grid before touching memory
   if (threadIdx.x == 0) {
+    // The CTA's role (batch, quad, sibling) comes from a ticket taken in arrival order, siblings
+    // on consecutive tickets: whatever subset of the grid is resident (other kernels may hold
+    // SMs), it holds whole sibling groups before any later CTA, so every wait can be satisfied.
+    // Taken before the programmatic-launch wait: a call releases the next kernels only after all
+    // its CTAs hold tickets, and the last one to take a ticket resets the counter first.
+    const unsigned tk = atomicAdd(&my_counters[p.counter_words - 1], 1u);
     for (int s = 0; s < kFuStages1; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&relu_done[s], 128);
@@ -132,7 +142,13 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
       mbar_init(&tempty[s], 128);
     }
     mbar_init(merge_bar, 1);
+    mbar_init(wait_done, 1);
     *abort_flag = 0;
+    if (tk == gridDim.x - 1) {
+      my_counters[p.counter_words - 1] = 0u;
+      __threadfence();
+    }
+    *ticket_slot = (int)tk;
     fence_mbar_init();
   }
   for (int i = threadIdx.x; i < 128; i += kFuThreads) reinterpret_cast<uint32_t*>(ones)[i] = 0x3F803F80u;
@@ -150,16 +166,37 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_holder;
-  // private set-up above; global memory only after the previous kernel in the stream is done
+  // the next kernel may launch once every CTA of this grid holds its ticket; it waits for this
+  // grid to complete before it touches memory
+  pdl_launch_dependents();
+  // private set-up above (and the ticket); global memory only after the previous kernel in the
+  // stream is done
+  // Every CTA counts itself out of the arrival and finish counters once, after its last access
+  // to them: thread 0 makes the CTA's arrival after phase 1 and, once it has issued its last q
+  // load and the merge leader's wait on the siblings is over, counts out; the CTA that counts
+  // out last zeroes them for the next call, all but the ticket counter, which the next call
+  // may already be using.  (No round trip lies on the merge leader's path or at exit.)
+  constexpr int kCounter = 0;
+  auto count_out = [&]() {
+    if (atomicAdd(&my_counters[p.counter_words - 2], 1u) == gridDim.x - 1)
+      for (int i = 0; i < p.counter_words - 1; ++i) my_counters[i] = 0u;
+  };
+  auto leave = [&]() {
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+      tc_fence_after_sync();
+      tmem_dealloc(tmem, kFuTmemCols);
+    }
+  };
   pdl_wait_primary();
-  // The CTA's role (batch, quad, sibling) comes from a ticket taken in arrival order, siblings
-  // on consecutive tickets: whatever subset of the grid is resident (other kernels may hold SMs),
-  // it holds whole sibling groups before any later CTA, so every wait below can be satisfied.
-  if (threadIdx.x == 0) *ticket_slot = (int)atomicAdd(&my_counters[p.counter_words - 1], 1u);
-  for (int i = blockIdx.x * kFuThreads + threadIdx.x; i < p.counter_words; i += gridDim.x * kFuThreads)
-    old_counters[i] = 0u;   // the previous call's set: clean for the call after this one
-  __syncthreads();
   const int ticket = *ticket_slot;
+  if (ticket < 0 || ticket >= (int)gridDim.x) {   // control words not clean: record it, do nothing
+    if (threadIdx.x == 0) atomicCAS(err, 0, kErrFusedTicket);
+    if (threadIdx.x == kCounter) count_out();
+    leave();
+    return;
+  }
   const int r = ticket % p.cpb, qb = ticket / p.cpb;
   const int q = qb % p.nquads, b = qb / p.nquads;
   const int cidx = b * p.nquads + q;
@@ -291,14 +328,14 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
   __threadfence();
   __syncthreads();
   tc_fence_after_sync();
-  if (threadIdx.x == 0) {   // arrival of this sibling (block-causal: its own flag)
-    if (kCausal) atomicExch(&my_counters[cidx * p.cpb + r], 1u);
-    else atomicAdd(&my_counters[cidx], 1u);
-  }
 
   // =============================== phase 2: merge + apply ================================
   if (warp == 0) {
-    if (lane == 0) {
+    if (lane == kCounter) {
+      // arrival of this sibling (block-causal: its own flag), released by the fence and the
+      // barrier after phase 1
+      if (kCausal) atomicExch(&my_counters[cidx * p.cpb + r], 1u);
+      else atomicAdd(&my_counters[cidx], 1u);
       int issued = 0;
       for (int lu = 0; lu < nunits; ++lu) {
         const int s = lu % kQStages;
@@ -318,6 +355,12 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
         for (int i = (issued > kQStages ? issued - kQStages : 0); i < issued; ++i)
           mbar_drain(&qfull[i % kQStages], (i / kQStages) & 1);
       }
+      // the count-out, ordered after the arrival and, through wait_done (the leader always
+      // signals it, its own wait being bounded), after the leader's reads of the siblings'
+      // arrivals
+      mbar_drain(wait_done, 0);
+      __threadfence();
+      count_out();
     }
   } else if (warp == 1) {
     if (lane == 0 && mbar_wait(sfull, 0, abort_flag, err, kErrApplyMma | 8)) {
@@ -394,6 +437,7 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
         }
       }
       __threadfence();   // acquire: the siblings' partial writes precede their arrivals
+      mbar_arrive(wait_done);
     }
     if (bar_any(1, 128, !ok)) ok = false;
     const int heads = min(kApUnitHeads, p.H - q * kApUnitHeads);
@@ -538,12 +582,7 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
     if (leader) bulk_wait_group<0>();
   }
 
-  tc_fence_before_sync();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after_sync();
-    tmem_dealloc(tmem, kFuTmemCols);
-  }
+  leave();
 }
 
 }  // namespace litela

@@ -51,14 +51,15 @@ struct Plan {
   //   state images (the apply's B operand) bf16 [B][H][nblk][kImageBytes]
   size_t off_images = 0, bytes = 0;
   // fused single-kernel path (non-causal, B * nquads <= SMs): CTA (b, quad, r), r < fused_cpb;
-  // workspace = fused partials [B][nquads][fused_cpb][4][33][32]; two sets of B * nquads
-  // arrival counters and a ticket counter (calls alternate between the sets)
+  // workspace = fused partials [B][nquads][fused_cpb][4][33][32]; control words: B * nquads
+  // arrival counters, a finish counter and a ticket counter
   bool fused = false;
   int fused_cpb = 0, fused_chunk = 0, fused_ntiles = 0;
   size_t fused_bytes = 0, counters = 0;
   // block-causal fused path (fused_causal): CTA (b, quad, r) owns blocks [r * fused_bpc, ...),
   // at most 2; workspace = block states [B][nquads][nblk][4][33][32], then the CTA totals
-  // [B][nquads][fused_cpb][4][33][32] at fused_off_totals; counters = 2 sets of one flag per CTA
+  // [B][nquads][fused_cpb][4][33][32] at fused_off_totals; control words: an arrival flag per
+  // CTA, the finish and ticket counters
   bool fused_causal = false;
   int fused_bpc = 0;
   size_t fused_off_totals = 0;
@@ -112,7 +113,7 @@ inline bool make_plan(int B, int N, int H, int tokens_per_block, int num_sms, Pl
     p->fused_cpb = cpb;
     p->fused_chunk = (int)chunk;
     p->fused_bytes = align_up((size_t)B * p->nquads * cpb * kRedHeads * kStateFloats * sizeof(float), 256);
-    p->counters = (size_t)2 * (B * p->nquads + 1);   // both sets; the last word of a set: the ticket
+    p->counters = (size_t)B * p->nquads + 2;   // an arrival counter per quad; finish, ticket
   } else if (p->nblk > 1 && p->T % kApTile == 0 && (int64_t)B * p->nquads <= sms) {
     int cpb = sms / (B * p->nquads);
     if (cpb > p->nblk) cpb = p->nblk;
@@ -126,7 +127,7 @@ inline bool make_plan(int B, int N, int H, int tokens_per_block, int num_sms, Pl
       const size_t part = (size_t)kRedHeads * kStateFloats * sizeof(float);
       p->fused_off_totals = align_up((size_t)B * p->nquads * p->nblk * part, 256);
       p->fused_bytes = p->fused_off_totals + align_up((size_t)B * p->nquads * cpb * part, 256);
-      p->counters = (size_t)2 * ((size_t)B * p->nquads * cpb + 1);   // both sets, each with its ticket word
+      p->counters = (size_t)B * p->nquads * cpb + 2;   // an arrival flag per CTA; finish, ticket
     }
   }
   return true;

@@ -459,8 +459,10 @@ __global__ void __launch_bounds__(kScanThreads)
 litela_state_images(const float* __restrict__ states, uint8_t* __restrict__ images, uint8_t* __restrict__ images_t,
                     long long n) {
   using namespace sm100;
-  pdl_launch_dependents();
   pdl_wait_primary();
+  // This kernel opens a call; the kernels after it read the call's inputs before their own
+  // waits, so they are released only once whatever came before in the stream has finished.
+  pdl_launch_dependents();
   const int64_t stride = (int64_t)gridDim.x * kScanThreads;
   const int64_t tid = (int64_t)blockIdx.x * kScanThreads + threadIdx.x;
   for (int64_t i = tid; i < n * kScanZeros; i += stride) {   // zero rows 33..39 and 73..79

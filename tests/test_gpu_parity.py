@@ -393,3 +393,38 @@ def test_concurrent_fused_calls_on_two_streams(T):
         ll.lite_la_device_status(sa)
         ll.lite_la_device_status(sb)
         assert torch.equal(oa, ra) and torch.equal(ob, rb)
+
+
+@pytest.mark.parametrize("T", [0, 1024])
+def test_fused_call_replayed_from_a_captured_graph(T):
+    """One fused call captured into a CUDA graph and replayed several times, interleaved with
+    eager calls on the same stream: the kernel's control words are left clean by the last CTA
+    of every call, so each replay and each eager call gives the eager result bitwise."""
+    B, N, H = (2, 8192, 70) if T == 0 else (1, 16384, 70)
+    x = make_qkv(B, N, H, 32, seed=6300 + T, device="cuda")
+    run = (lambda **kw: ll.lite_la_fwd(x, H, eps=EPS, **kw)) if T == 0 else \
+        (lambda **kw: ll.lite_la_block_causal_fwd(x, H, T, eps=EPS, **kw))
+    assert ll.lib().lite_la_kernels_per_call(B, N, H, 32, T) == 1
+    ref = run()
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    og = torch.empty_like(ref)
+    oe = torch.empty_like(ref)
+    with torch.cuda.stream(s):
+        run(out=og, stream=s)          # the stream's workspace exists before the capture
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        run(out=og, stream=s)
+    for _ in range(4):
+        og.zero_()
+        oe.zero_()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(s):
+            g.replay()
+            run(out=oe, stream=s)
+            g.replay()
+        s.synchronize()
+        ll.lite_la_device_status(s)
+        assert torch.equal(og, ref) and torch.equal(oe, ref)
+    del g
