@@ -513,7 +513,16 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
         *reinterpret_cast<__nv_bfloat16*>(hbuf + h_offset(kApUnitHeads + j, row)) = hl;
       }
       if (!ok) break;
-      // a group without heads in this quad (nh == 1) skips to here and still takes part
+      // a group without heads in this quad (nh == 1) skips to here and still takes part; it
+      // too waits for the previous tile's dS product first, so that its arrival cannot run a
+      // tile ahead and complete this tile's phase before the other group has written g/den
+      if (first && i > 0) {
+        const bool okg = mbar_wait(gfree, (i - 1) & 1, abort_flag, err, kErrBwdQEpi | 15);
+        if (bar_any(gbar, 128, !okg)) {
+          ok = false;
+          break;
+        }
+      }
       fence_proxy_async_smem();
       mbar_arrive(gready);
     }

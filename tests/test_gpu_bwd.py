@@ -154,12 +154,25 @@ def test_bwd_block_causal_workload_sampled():
     full_size_check(qkv, dout, H, T, heads, sampled(N, T, seed=2), "bf16")
 
 
-def test_bwd_is_bitwise_deterministic_and_matches_the_phase_timed_call():
-    B, N, H = 2, 3000, 9
+@pytest.mark.parametrize("H,T", [(9, 0), (7, 0), (5, 1024)])
+def test_bwd_many_tiles_per_cta_with_a_lone_last_head(H, T):
+    """An odd head count leaves the last head pair (and, for H % 4 == 1, the last quad) with one
+    head, so one epilogue group of the CTA has no head; with many tiles per CTA that group must
+    still keep step with the other.  Sampled rows of the lone head and two others."""
+    B, N = 2, 16384
+    qkv = make_qkv(B, N, H, D, seed=7650 + H + T, device="cuda")
+    dout = make_dout(B, N, H, seed=7660 + H + T)
+    heads = [(0, 0), (1, H - 2), (0, H - 1), (1, H - 1)]
+    full_size_check(qkv, dout, H, T or None, heads, sampled(N, T or None, seed=3), "bf16")
+
+
+@pytest.mark.parametrize("H,T", [(9, 0), (8, 0), (5, 512)])
+def test_bwd_is_bitwise_deterministic_and_matches_the_phase_timed_call(H, T):
+    B, N = 2, 3000
     qkv = make_qkv(B, N, H, D, seed=7700, device="cuda")
     dout = make_dout(B, N, H, seed=7701)
-    a = ll.lite_la_bwd(qkv, dout, H)
-    b = ll.lite_la_bwd(qkv, dout, H)
+    a = ll.lite_la_bwd(qkv, dout, H, tokens_per_block=T)
+    b = ll.lite_la_bwd(qkv, dout, H, tokens_per_block=T)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     stream = torch.cuda.current_stream()
     for e in evs:
@@ -167,7 +180,7 @@ def test_bwd_is_bitwise_deterministic_and_matches_the_phase_timed_call():
     torch.cuda.synchronize()
     c = torch.empty_like(a)
     handles = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in evs])
-    s = ll.lib().lite_la_bwd_events(qkv.data_ptr(), dout.data_ptr(), c.data_ptr(), B, N, H, D, EPS, 0,
+    s = ll.lib().lite_la_bwd_events(qkv.data_ptr(), dout.data_ptr(), c.data_ptr(), B, N, H, D, EPS, T,
                                     ctypes.c_void_p(stream.cuda_stream), handles)
     assert s == 0, ll.lib().lite_la_last_error().decode()
     torch.cuda.synchronize()
