@@ -25,7 +25,9 @@
  * synchronising that stream, so the first call with a new size must not happen during graph
  * capture) and keeps until lite_la_release_workspace().  Calls are asynchronous with respect to
  * the host; calls on one stream are ordered by that stream, calls on different streams use
- * different workspaces.
+ * different workspaces.  Once a stream's workspace has the size a call needs, the call may be
+ * captured into a CUDA graph on that stream: every call leaves the workspace's control words
+ * as it found them, so the graph may be replayed any number of times, between eager calls.
  *
  * Errors: every entry point returns a litela_status and never throws.  Argument errors are
  * detected on the host before anything is launched.  A kernel launch failure returns
