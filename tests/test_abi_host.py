@@ -176,3 +176,19 @@ def test_saved_state_entry_points_validate_on_the_host(lib):
     assert lib.lite_la_bwd_from_state(a, g, ctypes.c_void_p((1 << 34) + 8), o, 1, 4, 1, 32, 1e-15, 0, None) == 1
     assert lib.lite_la_fwd_save_state(None, None, None, 0, 4, 1, 32, 1e-15, 0, None) == 0
     assert lib.lite_la_bwd_from_state(a, g, st, o, 1, 4, 1, 64, 1e-15, 0, None) == 2
+
+
+def test_elu1_entry_points_validate_on_the_host(lib):
+    """The ELU+1 variant shares the forward's checks: clamp_min takes eps's place (finite, >= 0);
+    tokens_per_block <= 0 selects the non-causal form rather than being an error."""
+    a, o = ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 30)
+    for B, N, H, d, clamp, want in BAD_ARGS:
+        assert lib.lite_la_elu1_fwd(a, o, B, N, H, d, clamp, 0, None) == want
+        assert lib.lite_la_elu1_fwd_f32out(a, o, B, N, H, d, clamp, 16, None) == want
+    assert lib.lite_la_elu1_fwd(None, o, 1, 4, 1, 32, 1e-6, 0, None) == 1
+    assert lib.lite_la_elu1_fwd(a, ctypes.c_void_p((1 << 30) + 8), 1, 4, 1, 32, 1e-6, 0, None) == 1
+    assert lib.lite_la_elu1_fwd(a, ctypes.c_void_p((1 << 20) + 256), 1, 4, 1, 32, 1e-6, 0, None) == 1
+    assert "overlap" in lib.lite_la_last_error().decode()
+    assert lib.lite_la_elu1_fwd(None, None, 0, 4, 1, 32, 1e-6, 0, None) == 0
+    null = (ctypes.c_void_p * 3)(None, None, None)
+    assert lib.lite_la_elu1_fwd_events(a, o, 1, 4, 1, 32, 1e-6, 0, None, null) == 1
