@@ -284,6 +284,44 @@ def lite_la_bwd_from_state(qkv, dout, states, H: int, tokens_per_block: int = 0,
     return dqkv
 
 
+_AUTOGRAD_FN = None
+
+
+def _autograd_fn():
+    """The torch.autograd.Function behind lite_la (built on first use: torch is imported lazily)."""
+    global _AUTOGRAD_FN
+    if _AUTOGRAD_FN is None:
+        torch = _torch()
+
+        class LiteLAFunction(torch.autograd.Function):
+            @staticmethod
+            def forward(ctx, qkv, H, tokens_per_block, d, eps):
+                out, states = lite_la_fwd_save_state(qkv, H, tokens_per_block, d, eps)
+                ctx.save_for_backward(qkv, states)
+                ctx.args = (H, tokens_per_block, d, eps)
+                return out
+
+            @staticmethod
+            def backward(ctx, grad_out):
+                qkv, states = ctx.saved_tensors
+                H, tokens_per_block, d, eps = ctx.args
+                if grad_out.dtype != torch.bfloat16 or not grad_out.is_contiguous():
+                    grad_out = grad_out.to(torch.bfloat16).contiguous()
+                dqkv = lite_la_bwd_from_state(qkv, grad_out, states, H, tokens_per_block, d, eps)
+                return dqkv, None, None, None, None
+
+        _AUTOGRAD_FN = LiteLAFunction
+    return _AUTOGRAD_FN
+
+
+def lite_la(qkv, H: int, tokens_per_block: int = 0, d: int = 32, eps: float = 1e-15):
+    """LiteLA forward (block-causal when tokens_per_block > 0) that torch autograd can
+    differentiate: returns out bf16 [B, N, H*d].  The forward keeps the fp32 states its queries
+    use (lite_la_fwd_save_state); the backward hands them with the incoming gradient (as bf16)
+    to lite_la_bwd_from_state and returns d(qkv) in qkv's layout."""
+    return _autograd_fn().apply(qkv, H, int(tokens_per_block), d, eps)
+
+
 def lite_la_workspace_bytes(B: int, N: int, H: int, d: int = 32, tokens_per_block: int = 0) -> int:
     return int(lib().lite_la_workspace_bytes(B, N, H, d, tokens_per_block))
 

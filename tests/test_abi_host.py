@@ -192,3 +192,10 @@ def test_elu1_entry_points_validate_on_the_host(lib):
     assert lib.lite_la_elu1_fwd(None, None, 0, 4, 1, 32, 1e-6, 0, None) == 0
     null = (ctypes.c_void_p * 3)(None, None, None)
     assert lib.lite_la_elu1_fwd_events(a, o, 1, 4, 1, 32, 1e-6, 0, None, null) == 1
+
+
+def test_autograd_entry_point_rejects_host_tensors():
+    import torch
+    qkv = torch.zeros((1, 4, 96), dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        ll.lite_la(qkv, 1)

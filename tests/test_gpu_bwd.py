@@ -251,3 +251,21 @@ def test_forward_saves_the_state_and_the_backward_uses_it(B, N, H, T):
     want = oracle_bwd(qkv, dout, H, T or None)
     for i, name in enumerate(("dq", "dk", "dv")):
         assert_grad_close(x[:, :, i], want[i], want[3 + i], "bf16", name)
+
+
+@pytest.mark.parametrize("T", [0, 128])
+def test_autograd_function_matches_the_oracle(T):
+    """lite_la as a torch.autograd.Function: gradients of a downstream fp32 loss reach qkv
+    through the saved-state backward and match the oracle's."""
+    B, N, H = 2, 300, 3
+    qkv = make_qkv(B, N, H, D, seed=7900 + T, device="cuda").requires_grad_(True)
+    dout = make_dout(B, N, H, seed=7901 + T)
+    out = ll.lite_la(qkv, H, tokens_per_block=T, eps=EPS)
+    assert out.dtype == torch.bfloat16 and out.requires_grad
+    (out.float() * dout.float()).sum().backward()
+    torch.cuda.synchronize()
+    ll.lite_la_device_status()
+    got = qkv.grad.view(B, N, 3, H, D).to(torch.float64).cpu().numpy()
+    want = oracle_bwd(qkv.detach(), dout, H, T or None)
+    for i, name in enumerate(("dq", "dk", "dv")):
+        assert_grad_close(got[:, :, i], want[i], want[3 + i], "bf16", name)
