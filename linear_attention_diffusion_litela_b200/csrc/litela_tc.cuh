@@ -123,7 +123,10 @@ constexpr uint32_t kRedSmemBytes = kRedStages * kRedStageBytes + 512 + 256 + 102
 template <int kMap>
 struct RedCfg {
   static constexpr uint32_t kStageBytes = (kMap ? 6 : 4) * kRedBoxBytes;   // + phi(k) lo boxes
-  static constexpr uint32_t kSmemBytes = kRedStages * kStageBytes + 512 + 256 + 1024;
+  // ring depth: two CTAs per SM either way (the grid is one wave of two CTAs per SM), so the
+  // ELU + 1 form, with 48 KB stages, keeps two of them
+  static constexpr int kStages = kMap ? 2 : kRedStages;
+  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 512 + 256 + 1024;
   // warps: 0 TMA, 1 MMA, 2.. feature map (4 for ReLU, 8 for ELU + 1); warps 2..5 also read the
   // accumulators at the end
   static constexpr int kMapWarps = kMap ? 8 : 4;
@@ -159,14 +162,15 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
                  int* __restrict__ err, TcPlan p) {
   using namespace sm100;
   constexpr uint32_t kStageBytes = RedCfg<kMap>::kStageBytes;
+  constexpr int kStages = RedCfg<kMap>::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* stages = smem;
-  uint8_t* ones = smem + kRedStages * kStageBytes;                 // 16 x 16 bf16 ones
+  uint8_t* ones = smem + kStages * kStageBytes;                 // 16 x 16 bf16 ones
   uint64_t* full = reinterpret_cast<uint64_t*>(ones + 512);
-  uint64_t* relu_done = full + kRedStages;
-  uint64_t* empty = relu_done + kRedStages;
-  uint64_t* done = empty + kRedStages;
+  uint64_t* relu_done = full + kStages;
+  uint64_t* empty = relu_done + kStages;
+  uint64_t* done = empty + kStages;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -179,7 +183,7 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
   const int ntiles = n1 > n0 ? (n1 - n0 + kRedTile - 1) / kRedTile : 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kRedStages; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&relu_done[s], 32 * RedCfg<kMap>::kMapWarps);
       mbar_init(&empty[s], 1);
@@ -214,9 +218,9 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
     if (lane == 0) {
       int issued = 0;
       for (int i = 0; i < ntiles; ++i) {
-        const int s = i % kRedStages;
-        if (i >= kRedStages &&
-            !mbar_wait(&empty[s], ((i / kRedStages) - 1) & 1, abort_flag, err, kErrReduceProducer | s))
+        const int s = i % kStages;
+        if (i >= kStages &&
+            !mbar_wait(&empty[s], ((i / kStages) - 1) & 1, abort_flag, err, kErrReduceProducer | s))
           break;
         uint8_t* st = stages + s * kStageBytes;
         const int y = n0 + i * kRedTile;
@@ -228,8 +232,8 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
         issued = i + 1;
       }
       if (*abort_flag) {   // let the copies still in flight land before the CTA exits (bounded)
-        for (int i = (issued > kRedStages ? issued - kRedStages : 0); i < issued; ++i)
-          mbar_drain(&full[i % kRedStages], (i / kRedStages) & 1);
+        for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
+          mbar_drain(&full[i % kStages], (i / kStages) & 1);
       }
     }
   } else if (warp == 1) {
@@ -238,8 +242,8 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
       constexpr uint32_t idesc_den = idesc_bf16_f32(128, 16, true, false);
       const uint64_t ones_desc = smem_desc(smem_u32(ones), 128, 256, kSwizzleNone);
       for (int i = 0; i < ntiles; ++i) {
-        const int s = i % kRedStages;
-        if (!mbar_wait(&relu_done[s], (i / kRedStages) & 1, abort_flag, err, kErrReduceMma | s)) break;
+        const int s = i % kStages;
+        if (!mbar_wait(&relu_done[s], (i / kStages) & 1, abort_flag, err, kErrReduceMma | s)) break;
         tc_fence_after_sync();
         const uint32_t kbase = smem_u32(stages + s * kStageBytes);
         const uint32_t vbase = kbase + 2 * kRedBoxBytes;
@@ -265,8 +269,8 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
     constexpr int kMapThreads = 32 * RedCfg<kMap>::kMapWarps;
     const int t = threadIdx.x - 64;
     for (int i = 0; i < ntiles; ++i) {
-      const int s = i % kRedStages;
-      if (!mbar_wait(&full[s], (i / kRedStages) & 1, abort_flag, err, kErrReduceRelu | s)) break;
+      const int s = i % kStages;
+      if (!mbar_wait(&full[s], (i / kStages) & 1, abort_flag, err, kErrReduceRelu | s)) break;
       uint8_t* st = stages + s * kStageBytes;
       const int valid = min(kRedTile, n1 - (n0 + i * kRedTile));   // tokens of this chunk in the tile
 #pragma unroll 4
@@ -509,7 +513,7 @@ struct ApplyCfg {
   static constexpr int kOutSlots = sizeof(OutT) == 2 ? 2 : 1;
   static constexpr int kSBufs = kMap ? 1 : (sizeof(OutT) == 2 ? 1 : 2);
   // warps: 0 TMA, 1 MMA, 2.. feature map (2 warps for ReLU, 6 for ELU + 1), then 4 epilogue warps
-  static constexpr int kMapWarps = kMap ? 6 : 2;
+  static constexpr int kMapWarps = kMap ? 8 : 2;
   static constexpr int kThreads = 32 * (2 + kMapWarps + 4);
   static constexpr int kEpiWarp0 = 2 + kMapWarps;
   static constexpr int kBoxChannels = 128 / (int)sizeof(OutT);     // output channels per box
