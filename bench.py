@@ -632,22 +632,30 @@ def load_traffic(kernel, B, N, H, T, call="fwd"):
         return None
     with open(p) as f:
         d = json.load(f)
-    h = sources_hash()
     total = 0
     for k in kernel.split("+"):
         ent = [e for e in d.get("entries", []) if e["kernel"] == k and e.get("call", "fwd") == call
                and [e["B"], e["N"], e["H"], e["T"]] == [B, N, H, T]]
-        if not ent or ent[0].get("sources_sha256") != h:
+        if not ent or ent[0].get("sources_sha256") != sources_hash(ent[0].get("sources")):
             return None
         total += ent[0]["dram_bytes_per_launch"]
     return total
 
 
-def sources_hash():
+# the kernel sources each profiled kernel is built from (the ABI file sets its launch shape)
+KERNEL_SOURCES = {
+    "fwd": ["litela_abi.cu", "litela_fused.cuh", "litela_plan.h", "litela_tc.cuh", "sm100_ptx.cuh"],
+    "elu1_fwd": ["litela_abi.cu", "litela_plan.h", "litela_tc.cuh", "sm100_ptx.cuh"],
+    "bwd": ["litela_abi.cu", "litela_bwd.cuh", "litela_plan.h", "litela_tc.cuh", "sm100_ptx.cuh"],
+}
+
+
+def sources_hash(files=None):
+    """sha256 over the named kernel source files (all of csrc/ when None)."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_attention_diffusion_litela_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(files if files is not None else os.listdir(csrc)):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()
