@@ -228,9 +228,11 @@ litela_status lite_la_release_workspace(void);
  * means non-causal).  Returns 0 for invalid arguments or an empty problem. */
 size_t lite_la_workspace_bytes(int B, int N, int H, int d, int tokens_per_block);
 
-/* Number of kernels one call with these arguments launches on the current device: 1 when the
- * non-causal call fits the fused single-kernel path (B * ceil(H/4) <= SM count), 3 otherwise
- * (state reduction, prefix scan, apply); 0 for an empty or invalid problem. */
+/* Number of kernels one forward call with these arguments launches on the current device: 1
+ * when it takes the fused single kernel (B * ceil(H/4) <= SM count; block-causal calls also need
+ * a block size that is a multiple of 128 tokens and at most two blocks per CTA), 3 otherwise
+ * (state reduction, prefix scan, apply); 0 for an empty or invalid problem.  The streaming-carry
+ * and ELU+1 forms always take the three-kernel path. */
 int lite_la_kernels_per_call(int B, int N, int H, int d, int tokens_per_block);
 
 /* lite_la_fwd without any allocation.  The pages describe no such call; it exists for callers
