@@ -240,6 +240,32 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_holder;
 
+  // The dS product of tile i (issued by warp 0's lane 1, beside the head products of warp 1,
+  // so that neither kind of product queues behind the other)
+  constexpr uint32_t idesc_ds = idesc_bf16_f32(128, 128, true, true);
+  constexpr uint32_t idesc_dh = idesc_bf16_f32(128, 16, true, false);
+  const uint32_t la = smem_u32(glo), ha = smem_u32(hbuf);
+  // the dS product of tile i, once its epilogue has written g/den (hi over the g tile, lo
+  // into glo) and h
+  auto ds_product = [&](int i) {
+    const int s = i % kBwStages;
+    tc_fence_after_sync();
+    const uint32_t qa = smem_u32(qtile(s)), ga = smem_u32(gtile(s));
+#pragma unroll
+    for (int ks = 0; ks < kApTile / 16; ++ks) {
+      // dS^T[c][r] += sum over 16 tokens of q~[t][c] (g/den)[t][r]: A = q~ MN-major (M = 4 heads
+      // x 32 channels, the two boxes kBwBoxBytes apart), B = g/den MN-major, hi then lo
+      const uint64_t ad = smem_desc(qa + ks * 2048, kBwBoxBytes, 1024, kSwizzle128B);
+      const uint32_t acc = (i | ks) != 0;
+      umma_bf16(tmem + kBwDsCol, ad, smem_desc(ga + ks * 2048, kBwBoxBytes, 1024, kSwizzle128B), idesc_ds, acc);
+      umma_bf16(tmem + kBwDsCol, ad, smem_desc(la + ks * 2048, kBwBoxBytes, 1024, kSwizzle128B), idesc_ds, 1u);
+      // the ones row: sum of q~[t][c] h[t] (h hi in column j, lo in column 4 + j)
+      umma_bf16(tmem + kBwDhCol, ad, smem_desc(ha + ks * 512, 128, 256, kSwizzleNone), idesc_dh, acc);
+    }
+    umma_commit(&qempty[s]);
+    umma_commit(gfree);
+  };
+
   if (warp == 0) {
     if (lane == 0) {
       auto load = [&](int i) {
@@ -279,61 +305,27 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
           mbar_drain(&qfull[i % kBwStages], (i / kBwStages) & 1);
         if (images_loaded) mbar_drain(sfull, 0);
       }
+    } else if (lane == 1) {
+      // the dS product of each tile once both epilogue groups have written its g/den and h
+      // (gready); it frees the stage (qempty) and glo / hbuf (gfree).  dsfull follows the last.
+      int i = 0;
+      for (; i < sp.ntiles; ++i) {
+        if (!mbar_wait(gready, i & 1, abort_flag, err, kErrBwdQMma | 13)) break;
+        ds_product(i);
+      }
+      if (sp.ntiles > 0 && i == sp.ntiles) umma_commit(dsfull);
     }
   } else if (warp == 1) {
     if (lane == 0 && sp.ntiles > 0 && mbar_wait(sfull, 0, abort_flag, err, kErrBwdQMma | 8)) {
       constexpr uint32_t idesc_y = idesc_bf16_f32(128, kImageRows, false, false);
       constexpr uint32_t idesc_t = idesc_bf16_f32(128, kImageTRows, false, false);
-      constexpr uint32_t idesc_ds = idesc_bf16_f32(128, 128, true, true);
-      constexpr uint32_t idesc_dh = idesc_bf16_f32(128, 16, true, false);
-      const uint32_t la = smem_u32(glo), ha = smem_u32(hbuf);
-      // the dS product of tile i, once its epilogue has written g/den (hi over the g tile, lo
-      // into glo) and h
-      auto ds_product = [&](int i) {
-        const int s = i % kBwStages;
-        tc_fence_after_sync();
-        const uint32_t qa = smem_u32(qtile(s)), ga = smem_u32(gtile(s));
-#pragma unroll
-        for (int ks = 0; ks < kApTile / 16; ++ks) {
-          // dS^T[c][r] += sum over 16 tokens of q~[t][c] (g/den)[t][r]: A = q~ MN-major (M = 4 heads
-          // x 32 channels, the two boxes kBwBoxBytes apart), B = g/den MN-major, hi then lo
-          const uint64_t ad = smem_desc(qa + ks * 2048, kBwBoxBytes, 1024, kSwizzle128B);
-          const uint32_t acc = (i | ks) != 0;
-          umma_bf16(tmem + kBwDsCol, ad, smem_desc(ga + ks * 2048, kBwBoxBytes, 1024, kSwizzle128B), idesc_ds, acc);
-          umma_bf16(tmem + kBwDsCol, ad, smem_desc(la + ks * 2048, kBwBoxBytes, 1024, kSwizzle128B), idesc_ds, 1u);
-          // the ones row: sum of q~[t][c] h[t] (h hi in column j, lo in column 4 + j)
-          umma_bf16(tmem + kBwDhCol, ad, smem_desc(ha + ks * 512, 128, 256, kSwizzleNone), idesc_dh, acc);
-        }
-        umma_commit(&qempty[s]);
-        umma_commit(gfree);
-      };
-      // The head products of tile i need tile i's ReLU; the dS product of tile i needs tile i's
-      // epilogue (gready).  Issue whichever becomes ready first, the dS product preferred (it
-      // releases the stage for the next load and glo for the next epilogue).  The heads of
-      // tile i are not issued before the dS product of tile i - 2: their TMEM slots are freed by
-      // the epilogue of tile i - 1, which waits for that product.
+      // The head products of tile i, once tile i's ReLU is done; each waits for its TMEM slot,
+      // which the epilogue frees before it waits for any dS product (issued by another thread).
       int use[2] = {0, 0};
-      int hnext = 0, dnext = 0;
       bool stop = false;
-      uint64_t t_idle = globaltimer_ns();
-      while (dnext < sp.ntiles && !stop) {
-        if (dnext < hnext && mbar_test(gready, dnext & 1)) {
-          ds_product(dnext++);
-          t_idle = globaltimer_ns();
-          continue;
-        }
-        if (!(hnext < sp.ntiles && hnext <= dnext + 1 &&
-              mbar_test(&qrelu[2 * (hnext % kBwStages)], (hnext / kBwStages) & 1))) {
-          if (*abort_flag) break;
-          if (globaltimer_ns() - t_idle > kWaitLimitNs) {
-            *abort_flag = 1;
-            atomicCAS(err, 0, kErrBwdQMma | 12);
-            break;
-          }
-          continue;
-        }
-        const int i = hnext++;
+      for (int i = 0; i < sp.ntiles && !stop; ++i) {
         const int s = i % kBwStages;
+        if (!mbar_wait(&qrelu[2 * s], (i / kBwStages) & 1, abort_flag, err, kErrBwdQMma | 12)) break;
         tc_fence_after_sync();
         const uint32_t qa = smem_u32(qtile(s)), ga = smem_u32(gtile(s));
         for (int j = 0; j < sp.nh; ++j) {
@@ -361,9 +353,7 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
           }
           umma_commit(&tfull[a]);
         }
-        t_idle = globaltimer_ns();
       }
-      umma_commit(dsfull);
     }
   } else if (warp < 4) {
     // ReLU of the q tiles in place (the raw dout tile is not touched), one head-pair box at a
