@@ -55,8 +55,9 @@ enum : int {
   kErrBwdKvProducer = 0x610, kErrBwdKvMma = 0x620, kErrBwdKvRelu = 0x630, kErrBwdKvEpi = 0x640,
 };
 
-// w0 TMA, w1 MMA, w2..3 ReLU, w4..11 epilogue in two groups of 4 warps (group g takes the heads
-// j with j % 2 == g; each group covers all 128 TMEM lanes)
+// w0 TMA (lane 0; in the dq kernel lane 1 issues the dS products), w1 MMA, w2..3 ReLU,
+// w4..11 epilogue in two groups of 4 warps (group g takes the heads j with j % 2 == g; each
+// group covers all 128 TMEM lanes)
 constexpr int kBwThreads = 384;
 constexpr int kBwEpiThreads = 256;
 constexpr int kBwStages = 2;
