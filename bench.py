@@ -497,7 +497,11 @@ def main():
     # algorithmic FLOPs (2 per multiply-add): forward, the state (d+1) and the apply (d+1) per
     # element; backward, the state (d+1), y (d+1), S^T g (d), dS (d+1), dk (d), dv (d)
     flops_per_call = 2 * E * ((D + 1) + (D + 1) + D + (D + 1) + D + D) if bwd else 4 * B * H * N * D * (D + 1)
-    call_bytes_E = 18 if bwd else 8
+    phase_bytes_E = 18 if bwd else 8   # the phases are timed on the recomputing call
+    # the call itself: the saved-state backward skips the state (k and v read, d+1 MACs per
+    # element), 14 bytes per element instead of 18
+    call_bytes_E = (14 if args.bwd_from_state else 18) if bwd else 8
+    call_flops = flops_per_call - (2 * E * (D + 1) if bwd and args.bwd_from_state else 0)
     alg_bytes = {k: PATHS[nk]["alg_bytes_E"][k] * E for k in phases}
     peaks = load_peaks()
     dom = max(kern_us, key=kern_us.get)
@@ -508,7 +512,7 @@ def main():
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": traffic, "kernel": dom, "kernel_us": kern_us[dom],
                 "alg_bytes_per_launch": alg_bytes[dom],
-                "alg_flops_per_launch": flops_per_call * alg_bytes[dom] // (call_bytes_E * E),
+                "alg_flops_per_launch": flops_per_call * alg_bytes[dom] // (phase_bytes_E * E),
                 "peak_source": peak_note, "kernel_us_all": kern_us, "kernel_us_isolated": kern_us_isolated,
                 "timing": ("average launch duration over the timed region: CUDA events around the back-to-back "
                            "calls on the launching stream, / launches" if nk == 1 else
@@ -519,7 +523,7 @@ def main():
                              if bwd and args.bwd_from_state else "")}
     # the call as a whole against the slower of the HBM and fp32-FMA bounds
     t_hbm = call_bytes_E * E / (peaks["hbm_gbs"] * 1e9) * 1e6
-    t_fma = flops_per_call / (fp32_fma_peak_tflops(peaks.get("sm_max_mhz", 1965.0)) * 1e12) * 1e6
+    t_fma = call_flops / (fp32_fma_peak_tflops(peaks.get("sm_max_mhz", 1965.0)) * 1e12) * 1e6
     call_roof = {"t_hbm_us": t_hbm, "t_fma_us": t_fma, "t_roof_us": max(t_hbm, t_fma),
                  "us_per_call": us_call, "frac": max(t_hbm, t_fma) / us_call}
     if clocks.get("sm_mhz"):
@@ -528,7 +532,7 @@ def main():
         call_roof["frac_at_measured_clock"] = max(t_hbm, t_fma_clk) / us_call
     if args.ffma_seconds > 0:
         ffma = measure_ffma_peak(ll, dev, stream, args.ffma_seconds)
-        t_fma_meas = flops_per_call / (ffma["tflops"] * 1e12) * 1e6
+        t_fma_meas = call_flops / (ffma["tflops"] * 1e12) * 1e6
         call_roof["ffma_peak_measured"] = ffma
         call_roof["t_fma_us_measured_peak"] = t_fma_meas
         call_roof["frac_vs_measured_fma_peak"] = max(t_hbm, t_fma_meas) / us_call
@@ -610,7 +614,10 @@ def main():
                 "config": config_of(args.workload, args.direction, args.variant, args.bwd_from_state),
                 "roofline": roofline,
                 "call_roofline": call_roof,
-                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": nk * calls * args.steps,
+                "cpu_baseline": cpu, "e2e": e2e,
+                # kernels the timed calls launch: the saved-state backward runs the state images,
+                # the dq kernel, the reverse scan and the dk/dv kernel (4), not the 5 of `nk`
+                "gpu_launches": (4 if bwd and args.bwd_from_state else nk) * calls * args.steps,
                 "clocks": clocks, "gpu": torch.cuda.get_device_name(dev)}
         if world > 1:
             line["config"]["parallelism"] = "dp%d (independent calls per rank, no collective)" % world
