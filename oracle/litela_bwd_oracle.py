@@ -24,7 +24,7 @@ for the scalar L = sum_i dout_i . out_i (dout is the incoming gradient):
     dL/dk_j   = relu'(k_j) * sum_i dL/dw_ij relu(q_i)
 
 It forms one weight per (query, key) pair and never the (d+1) x d state; the state route is
-what the CUDA path takes.  Readings (also listed in the design doc): relu'(x) = 1 for x > 0 and 0
+what the CUDA path takes.  Readings where the pages are silent: relu'(x) = 1 for x > 0 and 0
 otherwise (0 at x = 0, as PyTorch's ReLU backward); eps is a constant; the ones row that pads
 v is a constant and gets no gradient.
 
@@ -43,7 +43,9 @@ a computed gradient is compared with tolerance rtol * |g| + atol * M.
 Parity status: lite_la_bwd_head, lite_la_bwd and lite_la_block_causal_bwd are pinned by
 tests/test_oracle_bwd_pins.py (central finite differences of the pinned forward oracle,
 PyTorch autograd of the quadratic form, closed-form identities from homogeneity and
-linearity, ReLU masks and block-causal special cases).
+linearity, ReLU masks and block-causal special cases); the error magnitudes are pinned from
+both sides by the sums of the absolute values of every chain-rule term, written out per
+(query, key) pair in exact rational arithmetic on tiny inputs.
 """
 from __future__ import annotations
 

@@ -14,8 +14,8 @@ the numerator by the denominator clamped from below at 1e-6 instead of adding an
     w_ij  = (phi(q_i) / sqrt(d)) . phi(k_j)       (j over the keys query i sees)
     out_i = (sum_j w_ij v_j) / max(sum_j w_ij, clamp_min)
 
-Block-causal masking is the same as for LiteLA (oracle/litela_oracle.py).  Readings (also in
-the design doc): ELU's alpha is 1 (PyTorch's default); inputs are the exactly decoded bf16 values.
+Block-causal masking is the same as for LiteLA (oracle/litela_oracle.py).  Readings where the
+page is silent: ELU's alpha is 1 (PyTorch's default); inputs are the exactly decoded bf16 values.
 
 Parity status: phi_elu1 and elu1_fwd are pinned by tests/test_oracle_elu_pins.py (closed
 forms of phi, the context route evaluated independently, invariants, the clamp branch).

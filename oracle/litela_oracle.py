@@ -28,7 +28,7 @@ block b sees exactly the keys/values of blocks 0..b (inclusive; a ragged last bl
 allowed).  The oracle is the same quadratic form with the key set restricted to that
 prefix.
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   * phi is ReLU on q and k only; v is not passed through phi.
   * eps is ADDED to the denominator, never used as a clamp; no 1/sqrt(d) scale.
   * bf16 inputs are decoded exactly (bits << 16 -> float32 -> float64).

@@ -193,3 +193,127 @@ def test_error_magnitudes_bound_the_gradients(T):
     # for N = 1 dq is eps-small while its magnitude is not
     dq1, _, _, mq1, _, _ = oracle.lite_la_bwd_head(q[:1], k[:1], v[:1], g[:1], eps, None, magnitudes=True)
     assert np.abs(dq1).max() < 1e-12 * mq1.max()
+
+
+# ---------------------------------------------------------------------------------------------
+# The error magnitudes, pinned from above: every chain-rule term written out per (query, key)
+# pair in exact rational arithmetic.
+
+def _explicit_terms(q, k, v, g, eps, T):
+    """The gradients of L = sum_i dout_i . out_i expanded into elementary products, with
+    exact Fractions on tiny inputs.  With out_i = num_i / den_i, num_i = sum_j w_ij v_j,
+    den_i = sum_j w_ij + eps and w_ij = relu(q_i) . relu(k_j) (j visible to i):
+
+        dq_ic = sum_j relu(k_jc) [ sum_r g_ir v_jr / den_i  -  sum_r sum_j' g_ir w_ij' v_j'r / den_i^2 ]
+        dk_jc = sum_i relu(q_ic) [ the same bracket ]          (i that see j)
+        dv_jr = sum_i w_ij g_ir / den_i
+
+    (the masks relu'(q), relu'(k) left off, as in the magnitudes).  Each product above is one
+    term; w_ij and den_i are sums of non-negative terms and enter as they are.  Returns the
+    signed sums (the gradients before the ReLU masks) and the sums of the terms' absolute
+    values (what any reassociation of these sums adds up)."""
+    from fractions import Fraction as F
+    N, d = len(q), len(q[0])
+    fr = lambda a: [[F(x) for x in row] for row in a]
+    q, k, v, g = fr(q), fr(k), fr(v), fr(g)
+    eps = F(eps)
+    rq = [[max(x, F(0)) for x in row] for row in q]
+    rk = [[max(x, F(0)) for x in row] for row in k]
+    vis = lambda i, j: T is None or j // T <= i // T
+    w = [[sum(rq[i][c] * rk[j][c] for c in range(d)) if vis(i, j) else F(0) for j in range(N)] for i in range(N)]
+    den = [sum(w[i]) + eps for i in range(N)]
+    zero = lambda: [[F(0)] * d for _ in range(N)]
+    dq, dk, dv, aq, ak, av = zero(), zero(), zero(), zero(), zero(), zero()
+    for i in range(N):
+        for j in range(N):
+            if not vis(i, j):
+                continue
+            # the bracket of pair (i, j): its terms, each with its sign
+            terms = [g[i][r] * v[j][r] / den[i] for r in range(d)]
+            terms += [-(g[i][r] * w[i][jj] * v[jj][r]) / den[i] ** 2 for r in range(d) for jj in range(N) if vis(i, jj)]
+            s, a = sum(terms), sum(abs(t) for t in terms)
+            for c in range(d):
+                dq[i][c] += rk[j][c] * s
+                aq[i][c] += rk[j][c] * a
+                dk[j][c] += rq[i][c] * s
+                ak[j][c] += rq[i][c] * a
+            for r in range(d):
+                t = w[i][j] * g[i][r] / den[i]
+                dv[j][r] += t
+                av[j][r] += abs(t)
+    as_np = lambda a: np.array([[float(x) for x in row] for row in a])
+    return tuple(as_np(a) for a in (dq, dk, dv, aq, ak, av))
+
+
+def _dyadic(rng, shape, scale=8):
+    """Small values exactly representable in binary (multiples of 1/scale), some negative."""
+    return rng.integers(-2 * scale, 2 * scale + 1, size=shape) / scale
+
+
+def _check_magnitudes(got, explicit, masks):
+    """The oracle's (dq, dk, dv, mq, mk, mv) against the explicit term sums, to 1e-12."""
+    dq, dk, dv, mq, mk, mv = got
+    eq, ek, ev, aq, ak, av = explicit
+    mask_q, mask_k = masks
+    ok = True
+    # the signed sums cancel (dq is eps-small for N = 1): they are compared relative to their
+    # own terms' magnitudes; the magnitudes relative to themselves
+    for x, want, size in ((dq, eq * mask_q, aq), (dk, ek * mask_k, ak), (dv, ev, av),
+                          (mq, aq, aq), (mk, ak, ak), (mv, av, av)):
+        ok &= bool(np.all(np.abs(x - want) <= 1e-12 * size + 1e-300))
+    return ok
+
+
+MAG_CASES = [(1, 2, None, 1e-15), (3, 3, None, 1e-15), (4, 4, None, 0.25), (5, 2, 2, 1e-15),
+             (6, 3, 2, 0.5), (6, 4, None, 1e-15), (5, 4, 3, 1e-15)]
+
+
+@pytest.mark.parametrize("N,d,T,eps", MAG_CASES)
+def test_error_magnitudes_equal_the_explicit_term_sums(N, d, T, eps):
+    """M(dq), M(dk) and M(dv) equal, to 1e-12, the sums of the absolute values of every term of
+    the chain rule written out pair by pair in exact rational arithmetic (and the signed sums
+    of the same terms reproduce the gradients, so the term list is the gradient's own).  This
+    bounds the magnitudes from above as well as from below: a magnitude counted twice, or a
+    term missing its 1/den, fails here."""
+    rng = np.random.default_rng(900 + 10 * N + d + (T or 0))
+    q, k, v, g = (_dyadic(rng, (N, d)) for _ in range(4))
+    got = oracle.lite_la_bwd_head(q, k, v, g, eps, T, magnitudes=True)
+    explicit = _explicit_terms(q, k, v, g, eps, T)
+    assert _check_magnitudes(got, explicit, ((q > 0).astype(float), (k > 0).astype(float)))
+
+
+def _planted(src_old, src_new):
+    """A copy of the backward oracle module with one slip planted in its source text."""
+    import importlib.util
+    import types
+    spec = importlib.util.find_spec("oracle.litela_bwd_oracle")
+    src = open(spec.origin).read()
+    assert src.count(src_old) >= 1, src_old
+    mod = types.ModuleType("planted_bwd_oracle")
+    mod.__dict__["__package__"] = "oracle"
+    exec(compile(src.replace(src_old, src_new), spec.origin, "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("old,new", [
+    ("mq[s:s + chunk] = aw @ pk", "mq[s:s + chunk] = 2 * (aw @ pk)"),            # M(dq) doubled
+    ("mk += aw_sel.T @ pq[i]", "mk += 2 * (aw_sel.T @ pq[i])"),                  # M(dk) doubled
+    ("/ den ** 2\n            aw = ", "/ den\n            aw = "),                # bnd without one 1/den (dq side)
+    ("/ den ** 2\n            aw_sel", "/ den\n            aw_sel"),              # the same on the dk side
+    ("aw = np.abs(dnum) @ av.T + bnd[:, None]", "aw = np.abs(dnum) @ av.T"),    # the denominator's terms dropped
+    ("mv += w_sel.T @ np.abs(dnum)", "mv += w_sel.T @ np.abs(dout[i])"),       # M(dv) without 1/den
+])
+def test_a_planted_magnitude_slip_fails_the_explicit_pin(old, new):
+    """Each slip, planted in a copy of the oracle's source, fails the explicit-term pin on at
+    least one of the cases above (the pin is sensitive to it)."""
+    mod = _planted(old, new)
+    caught = False
+    for N, d, T, eps in MAG_CASES:
+        rng = np.random.default_rng(900 + 10 * N + d + (T or 0))
+        q, k, v, g = (_dyadic(rng, (N, d)) for _ in range(4))
+        got = mod.lite_la_bwd_head(q, k, v, g, eps, T, magnitudes=True)
+        explicit = _explicit_terms(q, k, v, g, eps, T)
+        if not _check_magnitudes(got, explicit, ((q > 0).astype(float), (k > 0).astype(float))):
+            caught = True
+            break
+    assert caught
