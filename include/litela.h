@@ -128,7 +128,12 @@ litela_status lite_la_block_causal_fwd_events(const void* qkv, void* out, int B,
  * the current device set when one of their bounded waits timed out (each wait inside the
  * kernels gives up after about 1.5 s, records a code, frees its tensor memory and returns, so
  * the GPU context stays usable).  Returns LITELA_ERR_DEVICE_TIMEOUT (message with the code) if
- * a kernel of this stream's workspace or of lite_la_fwd_noalloc reported one, else LITELA_OK. */
+ * a kernel of this stream's workspace or of lite_la_fwd_noalloc reported one, else LITELA_OK.
+ * This stream's workspace has an error word of its own; lite_la_fwd_noalloc's word is one per
+ * device, shared by every stream.  That word is therefore read reliably only once every stream
+ * that issued lite_la_fwd_noalloc calls has been synchronised (a call still running on another
+ * stream can set it after the read), and a time-out it holds may come from another stream's
+ * call; it is reported, and cleared, by whichever stream asks first. */
 litela_status lite_la_device_status(cudaStream_t stream);
 
 /* Self-test of that error path: launches on `stream` one thread that waits on a barrier nothing
@@ -244,9 +249,12 @@ int lite_la_kernels_per_call(int B, int N, int H, int d, int tokens_per_block);
  * Its scratch (partial states, merged states, arrival counters) is one fixed array of
  * LITELA_NOALLOC_SCRATCH_BYTES in device memory that the library defines statically; every
  * GPU that loads the library holds it until the process exits.  A problem whose scratch does
- * not fit (roughly: lite_la_workspace_bytes() near or above the limit; the 4096px Sana call with
- * B=2, N=16384, H=70 needs about 6 MB) is rejected with LITELA_ERR_INVALID_ARGUMENT and a
- * message before anything is launched.  The first call on a device looks
+ * not fit (lite_la_workspace_bytes() plus a few hundred bytes of control words above the limit)
+ * is rejected with LITELA_ERR_INVALID_ARGUMENT and a message before anything is launched.  The
+ * 4096px Sana call (B=2, N=16384, H=70) takes the single fused kernel and needs about 2.4 MB
+ * (its sibling partial states); calls with more than 148 head quads (B * ceil(H/4)) take the
+ * three-kernel path, whose partial states and state images need more (B=8, N=512, H=80: about
+ * 6 MB).  The first call on a device looks
  * up that device's address of the array (once per device); make that first call before any
  * stream capture.  The call never calls cudaMalloc or cudaFree; it clears the counters it needs
  * with cudaMemsetAsync on `stream`.  All calls on a device share the one array and it keeps the
