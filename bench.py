@@ -39,10 +39,17 @@ WORKLOADS_BENCH = {
     "sana600m_512px": (1, 16 * 16, 36, 64, 1000, 0),
     "sana1600m_1024px": (2, 32 * 32, 70, 20, 1001, 0),
     "sana1600m_2048px": (2, 64 * 64, 70, 20, 1002, 0),
+    # the 2048px shape with q and k shifted by -1.5 before the bf16 cast (mostly negative:
+    # sparse ReLU, tiny denominators)
+    "sana1600m_2048px_mostly_negative": (2, 64 * 64, 70, 20, 3001, 0),
     # video-style block-causal call: 16 blocks of 1024 tokens, 20 distinct buffers per step
     "block_causal_16x1024": (1, 16 * 1024, 70, 20, 1004, 1024),
     "block_causal_16x1024_x1": (1, 16 * 1024, 70, 1, 1004, 1024),
 }
+QK_SHIFT = {"sana1600m_2048px_mostly_negative": -1.5}
+# the configs timed beside the headline in the default run (the `workloads` record)
+RECORD_WORKLOADS = ("sana600m_512px", "sana1600m_1024px", "sana1600m_2048px", "sana1600m_2048px_mostly_negative",
+                    "block_causal_16x1024")
 D = 32
 EPS = 1e-15
 METRIC = "LiteLA fwd tokens·heads/s and µs/call at 4096px; % of HBM/FMA roofline"
@@ -234,6 +241,76 @@ def oracle_head_rate(qkv_bits, B, N, H, T, seconds, max_heads=None, dout_bits=No
             return heads * N / el, heads, el
 
 
+def workload_seeds(wl, calls):
+    """Seeds of a workload's distinct input buffers (the 4096px ones are 4000 + i)."""
+    seed0 = WORKLOADS_BENCH[wl][4]
+    return [seed0 + i for i in range(calls)] if wl.startswith("sana4800m") else [seed0 * 10 + i for i in range(calls)]
+
+
+def call_bounds_us(B, N, H, peaks, ffma_tflops=None):
+    """The workload definition's roofline of one forward call: 8 bytes per (token, head,
+    channel) at the copy bandwidth, and 4*B*H*N*d*(d+1) FLOPs at the fp32 FMA peak (from the
+    unit counts at the maximum clock, and as measured when given)."""
+    E = B * N * H * D
+    t_hbm = 8 * E / (peaks["hbm_gbs"] * 1e9) * 1e6
+    flops = 4 * B * H * N * D * (D + 1)
+    t_fma = flops / (fp32_fma_peak_tflops(peaks.get("sm_max_mhz", 1965.0)) * 1e12) * 1e6
+    t_fma_meas = flops / (ffma_tflops * 1e12) * 1e6 if ffma_tflops else None
+    return t_hbm, t_fma, t_fma_meas
+
+
+def time_record_workload(ll, lib, dev, stream, wl, peaks, ffma_tflops=None, reps=5, min_ms=25.0):
+    """One entry of the `workloads` record: the workload's calls on its distinct buffers,
+    back to back, timed with CUDA events on the launching stream; `reps` repetitions of K
+    steps (K sized so one repetition lasts at least `min_ms`), median reported."""
+    import ctypes
+    import torch
+    from linear_attention_diffusion_litela_b200.inputs import make_qkv
+    B, N, H, calls, _seed0, T = WORKLOADS_BENCH[wl]
+    ins = [make_qkv(B, N, H, D, seed=s, device=dev, qk_shift=QK_SHIFT.get(wl, 0.0)) for s in workload_seeds(wl, calls)]
+    outs = [torch.empty((B, N, H * D), dtype=torch.bfloat16, device=dev) for _ in range(calls)]
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    in_p, out_p = [t.data_ptr() for t in ins], [t.data_ptr() for t in outs]
+
+    def step():
+        for i in range(calls):
+            s = (lib.lite_la_block_causal_fwd(in_p[i], out_p[i], B, N, H, D, EPS, T, sh) if T else
+                 lib.lite_la_fwd(in_p[i], out_p[i], B, N, H, D, EPS, sh))
+            if s != 0:
+                raise ll.LiteLAError(s, lib.lite_la_last_error().decode())
+
+    def run(K):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(K):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1)
+
+    run(3)                                   # warm-up
+    K = max(3, int(min_ms / max(run(3) / 3, 1e-3)) + 1)
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    with ClockSampler(uuid) as cs:
+        us = [1e3 * run(K) / (K * calls) for _ in range(reps)]
+    clocks = cs.summary()
+    ll.lite_la_device_status(stream)
+    del ins, outs
+    us_call = statistics.median(us)
+    t_hbm, t_fma, t_fma_meas = call_bounds_us(B, N, H, peaks, ffma_tflops)
+    rec = {"workload": wl, "B": B, "N": N, "H": H, "tokens_per_block": T or None,
+           "qk_shift": QK_SHIFT.get(wl), "calls_per_step": calls, "steps_per_rep": K, "reps": reps,
+           "us_per_call": us_call, "us_per_call_reps": us, "tokens_heads_per_s": B * N * H / (us_call * 1e-6),
+           "kernels_per_call": int(lib.lite_la_kernels_per_call(B, N, H, D, T)),
+           "t_hbm_us": t_hbm, "hbm_frac": t_hbm / us_call, "t_fma_us": t_fma,
+           "t_roof_us": max(t_hbm, t_fma), "roof_frac": max(t_hbm, t_fma) / us_call,
+           "l2": l2_note(B, N, H, calls), "clocks": clocks}
+    if t_fma_meas:
+        rec["frac_vs_measured_fma_peak"] = max(t_hbm, t_fma_meas) / us_call
+    return rec
+
+
 def emit(line):
     print(json.dumps(line), flush=True)
 
@@ -247,7 +324,7 @@ def run_reference(args, wl):
     if rank != 0:
         return 0
     B, N, H, calls, seed, T = WORKLOADS_BENCH[wl]
-    bits = to_bits(make_qkv(B, N, H, D, seed=seed, device="cpu"))
+    bits = to_bits(make_qkv(B, N, H, D, seed=seed, device="cpu", qk_shift=QK_SHIFT.get(wl, 0.0)))
     bwd = args.direction == "bwd"
     gbits = to_bits(make_dout(B, N, H, seed + 500, "cpu")) if bwd else None
     import oracle
@@ -329,6 +406,8 @@ def main():
                          "(lite_la_bwd_from_state; the states are made once before timing)")
     ap.add_argument("--variant", choices=["litela", "elu1"], default="litela",
                     help="elu1 times the ELU+1 feature-map variant of the forward (clamp 1e-6)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the `workloads` record (the other configs, timed after the headline)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -372,9 +451,8 @@ def main():
     need = calls * (qkv_bytes + out_bytes + (qkv_bytes if bwd else 0)) + (2 << 30)
     if free < need:
         raise SystemExit("not enough free GPU memory: need %.1f GB, free %.1f GB" % (need / 1e9, free / 1e9))
-    seeds = [seed0 + i for i in range(calls)] if args.workload.startswith("sana4800m") else [seed0 * 10 + i for i in range(calls)]
-    seeds = rank_seeds(seeds, rank)
-    ins = [make_qkv(B, N, H, D, seed=s, device=dev) for s in seeds]
+    seeds = rank_seeds(workload_seeds(args.workload, calls), rank)
+    ins = [make_qkv(B, N, H, D, seed=s, device=dev, qk_shift=QK_SHIFT.get(args.workload, 0.0)) for s in seeds]
     outs = [torch.empty((B, N, H * D), dtype=torch.bfloat16, device=dev) for _ in range(calls)]
     if bwd:   # the backward reads an incoming gradient (in `outs`) and writes dqkv
         outs = [make_dout(B, N, H, s + 500, dev) for s in seeds]
@@ -604,6 +682,14 @@ def main():
                "sample": "%d whole (batch, head) pairs of input buffer 0 (%s, all %d tokens), %.1f s"
                          % (heads, "dq, dk, dv" if bwd else "all queries x all keys", N, el)}
 
+    # the other configs, timed in the same run on the same GPU (single-GPU runs of the
+    # headline only: a few seconds in all)
+    records = None
+    if (rank == 0 and world == 1 and not args.no_workloads and not bwd and args.variant == "litela"
+            and args.workload == "sana4800m_4096px_x60"):
+        ffma_t = call_roof.get("ffma_peak_measured", {}).get("tflops")
+        records = [time_record_workload(ll, lib, dev, stream, w, peaks, ffma_t) for w in RECORD_WORKLOADS]
+
     if rank == 0:
         line = {"metric": METRIC_BWD if bwd else METRIC, "value": value, "unit": UNIT, "n_gpus": world,
                 "steps": args.steps,
@@ -623,6 +709,8 @@ def main():
             line["config"]["parallelism"] = "dp%d (independent calls per rank, no collective)" % world
         if rejected is not None:
             line["clocks_rejected_first_run"] = rejected
+        if records is not None:
+            line["workloads"] = records
         emit(line)
     if dist is not None:
         dist.barrier()

@@ -92,3 +92,20 @@ def test_reference_arm_prints_its_line_on_the_host_cores():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
     assert line["config"]["workload"] == "sana600m_512px"
+
+
+def test_the_workloads_record_covers_every_other_config_with_its_bounds():
+    """The default run times the other configs of the workload definition beside the headline:
+    512px, 1024px, 2048px (and its mostly-negative input) and the block-causal call; each bound
+    follows from the unit counts (8 bytes per element at the copy peak; 4*B*H*N*d*(d+1) FLOPs at
+    148 SMs x 128 lanes x 2 x the clock)."""
+    assert set(bench.RECORD_WORKLOADS) == {"sana600m_512px", "sana1600m_1024px", "sana1600m_2048px",
+                                           "sana1600m_2048px_mostly_negative", "block_causal_16x1024"}
+    assert bench.QK_SHIFT["sana1600m_2048px_mostly_negative"] == -1.5
+    peaks = {"hbm_gbs": 6543.4, "sm_max_mhz": 1965.0}
+    t_hbm, t_fma, t_meas = bench.call_bounds_us(2, 16384, 70, peaks, 71.48)
+    assert abs(t_hbm - 89.74) < 0.01 and abs(t_fma - 130.14) < 0.01 and abs(t_meas - 135.54) < 0.01
+    t_hbm, t_fma, t_meas = bench.call_bounds_us(2, 1024, 70, peaks)
+    assert abs(t_hbm - 5.61) < 0.01 and abs(t_fma - 8.13) < 0.01 and t_meas is None
+    assert bench.workload_seeds("sana4800m_4096px_x60", 3) == [4000, 4001, 4002]
+    assert bench.workload_seeds("sana1600m_2048px_mostly_negative", 2) == [30010, 30011]
