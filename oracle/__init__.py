@@ -19,3 +19,7 @@ from .litela_elu_oracle import (  # noqa: F401
     elu1_rows,
     elu1_fwd,
 )
+from .litela_oproj_oracle import (  # noqa: F401
+    linear,
+    lite_la_oproj,
+)
