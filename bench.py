@@ -199,6 +199,16 @@ def cpu_threads():
     return os.cpu_count() or 1
 
 
+def single_thread_rate(fn, seconds):
+    """fn(seconds) with numpy's BLAS limited to one thread (None if that cannot be set)."""
+    try:
+        from threadpoolctl import threadpool_limits
+    except ImportError:
+        return None
+    with threadpool_limits(limits=1):
+        return fn(seconds)
+
+
 def one_head_bits(qkv_bits, B, N, H, b, h):
     """Packed [1, N, 3*d] bits of head h of batch b (input re-packing only)."""
     import numpy as np
@@ -325,6 +335,8 @@ def run_reference(args, wl):
         return 0
     B, N, H, calls, seed, T = WORKLOADS_BENCH[wl]
     bits = to_bits(make_qkv(B, N, H, D, seed=seed, device="cpu", qk_shift=QK_SHIFT.get(wl, 0.0)))
+    if args.variant == "fused_oproj":
+        return run_reference_oproj(args, wl, bits)
     bwd = args.direction == "bwd"
     gbits = to_bits(make_dout(B, N, H, seed + 500, "cpu")) if bwd else None
     import oracle
@@ -353,6 +365,39 @@ def run_reference(args, wl):
           "config": config_of(wl, args.direction, args.variant),
           "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                            "sample": sample},
+          "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
+    return 0
+
+
+def run_reference_oproj(args, wl, bits):
+    """Reference arm of --variant fused_oproj: the fp64 oracle of LiteLA + projection, 16 query
+    rows of batch 0 per step (all heads against all keys, then the projection)."""
+    import numpy as np
+    import oracle
+    from linear_attention_diffusion_litela_b200.inputs import to_bits
+    B, N, H, calls, seed, T = WORKLOADS_BENCH[wl]
+    C = H * D
+    w, b = make_proj_weight(C, C, seed + 7000, "cpu")
+    wbits, bias = to_bits(w), b.numpy()
+    bits0 = np.ascontiguousarray(bits.reshape(B, N, 3 * C)[:1])
+    times = []
+    for i in range(args.warmup + args.steps):
+        rows = (i + np.arange(16) * 1021) % N
+        t0 = time.perf_counter()
+        oracle.lite_la_oproj(bits0, wbits, 1, N, H, D, C, EPS, bias, T or None, rows=rows)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    ms = 1e3 * float(np.mean(times))
+    value = 16 * H / (ms / 1e3)
+    cfg = config_of(wl)
+    cfg.update({"workload": wl + "_fused_oproj", "variant": "fused_oproj", "C_out": C})
+    emit({"impl": "reference", "metric": METRIC_OPROJ, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+          "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+          "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+          "data": "synthetic: i.i.d. N(0,1) bf16 qkv, seed %d; seeded projection weight" % seed, "config": cfg,
+          "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                           "sample": "16 query rows of batch 0 per step: all %d heads against all %d keys, then "
+                                     "the %d x %d projection" % (H, N, C, C)},
           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
     return 0
 
@@ -404,8 +449,9 @@ def main():
     ap.add_argument("--bwd-from-state", action="store_true",
                     help="with --direction bwd: the backward given the forward's saved states "
                          "(lite_la_bwd_from_state; the states are made once before timing)")
-    ap.add_argument("--variant", choices=["litela", "elu1"], default="litela",
-                    help="elu1 times the ELU+1 feature-map variant of the forward (clamp 1e-6)")
+    ap.add_argument("--variant", choices=["litela", "elu1", "fused_oproj"], default="litela",
+                    help="elu1 times the ELU+1 feature-map variant of the forward (clamp 1e-6); fused_oproj "
+                         "LiteLA with the output projection fused (and the unfused chain beside it)")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the `workloads` record (the other configs, timed after the headline)")
     args = ap.parse_args()
@@ -413,6 +459,10 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args, args.workload)
+    if args.variant == "fused_oproj":
+        if args.direction == "bwd":
+            ap.error("--variant fused_oproj has no backward")
+        return main_oproj(args)
 
     import ctypes
 
@@ -678,9 +728,16 @@ def main():
         bits = to_bits(ins[0])
         gbits = to_bits(outs[0]) if bwd else None
         rate, heads, el = oracle_head_rate(bits, B, N, H, T, args.cpu_seconds, dout_bits=gbits, variant=args.variant)
+        what = "dq, dk, dv" if bwd else "all queries x all keys"
         cpu = {"value": rate, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                "sample": "%d whole (batch, head) pairs of input buffer 0 (%s, all %d tokens), %.1f s"
-                         % (heads, "dq, dk, dv" if bwd else "all queries x all keys", N, el)}
+                         % (heads, what, N, el)}
+        single = single_thread_rate(lambda sec: oracle_head_rate(bits, B, N, H, T, sec, dout_bits=gbits,
+                                                                 variant=args.variant), args.cpu_seconds / 2)
+        if single is not None:
+            r1, h1, e1 = single
+            cpu["single_thread"] = {"value": r1, "unit": UNIT, "cores": 1,
+                                    "sample": "%d whole (batch, head) pairs, %s, %.1f s" % (h1, what, e1)}
 
     # the other configs, timed in the same run on the same GPU (single-GPU runs of the
     # headline only: a few seconds in all)
@@ -711,6 +768,263 @@ def main():
             line["clocks_rejected_first_run"] = rejected
         if records is not None:
             line["workloads"] = records
+        emit(line)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+METRIC_OPROJ = "LiteLA fwd + output projection tokens·heads/s and µs/call at 4096px; % of tensor roofline"
+PEAKS_BF16_FALLBACK = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def make_proj_weight(C_out, C_in, seed, device):
+    """Synthetic projection weight (nn.Linear-like U(-1/sqrt(C_in), 1/sqrt(C_in)), bf16) and bias
+    (N(0, 0.02), fp32), from a seeded generator: Sana's trained weights are not available."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    w = ((torch.rand((C_out, C_in), generator=g, device=device) * 2 - 1) / C_in ** 0.5).to(torch.bfloat16)
+    b = torch.randn((C_out,), generator=g, device=device) * 0.02
+    return w, b
+
+
+def oracle_oproj_rate(qkv_bits, w_bits, bias, B, N, H, T, seconds):
+    """The fp64 oracle of LiteLA + projection on batches of 16 query rows of batch 0 (each row:
+    all heads against all keys, then the projection) until `seconds` have passed; returns
+    (tokens*heads per second, rows done, elapsed)."""
+    import numpy as np
+    import oracle
+    C = H * D
+    rows_done, t0, r0 = 0, time.perf_counter(), 0
+    bits0 = np.ascontiguousarray(qkv_bits.reshape(B, N, 3 * C)[:1])
+    while True:
+        rows = (r0 + np.arange(16) * 1021) % N
+        oracle.lite_la_oproj(bits0, w_bits, 1, N, H, D, C, EPS, bias, T or None, rows=rows)
+        rows_done += rows.size
+        r0 += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            return rows_done * H / el, rows_done, el
+
+
+def main_oproj(args):
+    """--variant fused_oproj: one step is `calls` back-to-back calls of LiteLA + output
+    projection (each layer its own qkv buffer and its own 2240 x 2240 weight and bias),
+    timed as the fused call (lite_la_fwd_oproj) and, in the same run, as the unfused chain
+    (lite_la_fwd, then lite_la_out_proj on its output)."""
+    import ctypes
+    import numpy as np
+    import torch
+    import linear_attention_diffusion_litela_b200 as ll
+    from linear_attention_diffusion_litela_b200.dist import aggregate_rate, rank_seeds, world_info
+    from linear_attention_diffusion_litela_b200.dist import max_over_ranks as _max_over_ranks
+    from linear_attention_diffusion_litela_b200.inputs import make_qkv, to_bits
+
+    world, rank, local_rank = world_info()
+    if world != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE %d (launch N>1 with torch.distributed.run)" % (args.gpus, world))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    lib = ll.lib()
+    B, N, H, calls, _seed0, T = WORKLOADS_BENCH[args.workload]
+    C = H * D
+    E = B * N * H * D
+    seeds = rank_seeds(workload_seeds(args.workload, calls), rank)
+    free, _ = torch.cuda.mem_get_info(dev)
+    need = calls * (6 * E + 2 * B * N * C + 2 * C * C) + 2 * E + (2 << 30)
+    if free < need:
+        raise SystemExit("not enough free GPU memory: need %.1f GB, free %.1f GB" % (need / 1e9, free / 1e9))
+    ins = [make_qkv(B, N, H, D, seed=s, device=dev, qk_shift=QK_SHIFT.get(args.workload, 0.0)) for s in seeds]
+    wts = [make_proj_weight(C, C, s + 7000, dev) for s in seeds]
+    ys = [torch.empty((B, N, C), dtype=torch.bfloat16, device=dev) for _ in range(calls)]
+    xbuf = torch.empty((B, N, C), dtype=torch.bfloat16, device=dev)    # the unfused chain's attention output
+    stream = torch.cuda.current_stream(dev)
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    in_p, y_p = [t.data_ptr() for t in ins], [t.data_ptr() for t in ys]
+    w_p, b_p = [w.data_ptr() for w, _ in wts], [b.data_ptr() for _, b in wts]
+
+    def call_fused(i, qkv_ptr=None, y_ptr=None):
+        s = lib.lite_la_fwd_oproj(qkv_ptr or in_p[i], w_p[i], b_p[i], y_ptr or y_p[i], B, N, H, D, C, EPS, T, sh)
+        if s != 0:
+            raise ll.LiteLAError(s, lib.lite_la_last_error().decode())
+
+    def call_unfused(i):
+        s = (lib.lite_la_block_causal_fwd(in_p[i], xbuf.data_ptr(), B, N, H, D, EPS, T, sh) if T else
+             lib.lite_la_fwd(in_p[i], xbuf.data_ptr(), B, N, H, D, EPS, sh))
+        if s == 0:
+            s = lib.lite_la_out_proj(xbuf.data_ptr(), w_p[i], b_p[i], y_p[i], B, N, C, C, sh)
+        if s != 0:
+            raise ll.LiteLAError(s, lib.lite_la_last_error().decode())
+
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+
+    def timed(fn, K):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        with ClockSampler(uuid) as cs:
+            e0.record(stream)
+            for _ in range(K):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+        barrier()
+        return e0.elapsed_time(e1), cs.summary()
+
+    def step_fused():
+        for i in range(calls):
+            call_fused(i)
+
+    def step_unfused():
+        for i in range(calls):
+            call_unfused(i)
+
+    for _ in range(args.warmup):
+        step_fused()
+        step_unfused()
+    torch.cuda.synchronize(dev)
+    ll.lite_la_device_status(stream)
+    ms_total, clocks = timed(step_fused, args.steps)
+    rejected = None
+    if _max_over_ranks(1.0 if clocks_rejected(clocks) else 0.0, device=dev) > 0.0:
+        rejected = clocks
+        ms_total, clocks = timed(step_fused, args.steps)
+    ms_total = _max_over_ranks(ms_total, device=dev)
+    ms_unf, clocks_unf = timed(step_unfused, args.steps)
+    ms_unf = _max_over_ranks(ms_unf, device=dev)
+    ll.lite_la_device_status(stream)
+    ms_step = ms_total / args.steps
+    us_call = 1e3 * ms_step / calls
+    us_unf = 1e3 * ms_unf / (args.steps * calls)
+    value = aggregate_rate(B * N * H * calls * args.steps, world, ms_total)
+
+    # phases of the fused call: the state (reduction + scan) and the apply + projection kernel
+    nev = 3
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(calls)]
+    for trip in evs:
+        for e in trip:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
+    ev_h = [(ctypes.c_void_p * nev)(*[ctypes.c_void_p(e.cuda_event) for e in trip]) for trip in evs]
+    ph = {"litela_reduce_tc+litela_state_scan": 0.0, "litela_oproj_tc": 0.0}
+    for _ in range(args.steps):
+        for i in range(calls):
+            s = lib.lite_la_fwd_oproj_events(in_p[i], w_p[i], b_p[i], y_p[i], B, N, H, D, C, EPS, T, sh, ev_h[i])
+            if s != 0:
+                raise ll.LiteLAError(s, lib.lite_la_last_error().decode())
+        torch.cuda.synchronize(dev)
+        for trip in evs:
+            ph["litela_reduce_tc+litela_state_scan"] += trip[0].elapsed_time(trip[1])
+            ph["litela_oproj_tc"] += trip[1].elapsed_time(trip[2])
+    ph_us = {k: 1e3 * v / (args.steps * calls) for k, v in ph.items()}
+    peaks = load_peaks()
+    bf16_sust = peaks.get("bf16_tflops_sustained") or PEAKS_BF16_FALLBACK["bf16_tflops_sustained"]
+    bf16_src = "measured" if peaks.get("bf16_tflops_sustained") else "fallback"
+    gemm_flops = 2 * B * N * C * C
+    apply_flops = 2 * E * (D + 1)
+    k_flops = gemm_flops + apply_flops
+    achieved = k_flops / (ph_us["litela_oproj_tc"] * 1e-6) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": bf16_sust, "unit": "TFLOP/s",
+                "frac": achieved / bf16_sust, "traffic": None, "kernel": "litela_oproj_tc",
+                "kernel_us": ph_us["litela_oproj_tc"], "alg_flops_per_launch": k_flops,
+                "alg_bytes_per_launch": 2 * E + 2 * C * C + 2 * B * N * C,
+                "peak_source": "%s sustained dense bf16 (cuBLAS) throughput" % bf16_src, "kernel_us_all": ph_us,
+                "timing": "CUDA events on the launching stream around each phase (phase-timed entry point; no "
+                          "programmatic overlap with the neighbouring kernels)"}
+    t_tensor = k_flops / (bf16_sust * 1e12) * 1e6
+    t_hbm = (4 * E + 2 * E + 2 * C * C + 2 * B * N * C) / (peaks["hbm_gbs"] * 1e9) * 1e6
+    call_roof = {"t_tensor_us": t_tensor, "t_hbm_us": t_hbm, "t_roof_us": max(t_tensor, t_hbm),
+                 "us_per_call": us_call, "frac": max(t_tensor, t_hbm) / us_call,
+                 "how": "the projection GEMM's FLOPs (2 B N C^2) plus the apply's at the sustained bf16 peak, "
+                        "against k, v, q read once, W read once and y written once at the copy bandwidth"}
+
+    e2e = None
+    if args.e2e_steps > 0:
+        nbuf = 3
+        h_in = [torch.empty((B, N, 3 * C), dtype=torch.bfloat16, pin_memory=True) for _ in range(nbuf)]
+        h_out = [torch.empty((B, N, C), dtype=torch.bfloat16, pin_memory=True) for _ in range(nbuf)]
+        for j in range(nbuf):
+            h_in[j].copy_(ins[j])
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_up = [torch.cuda.Event() for _ in range(nbuf)]
+        ev_fw = [torch.cuda.Event() for _ in range(nbuf)]
+        ev_dn = [torch.cuda.Event() for _ in range(nbuf)]
+        for j in range(nbuf):
+            ev_dn[j].record(down)
+
+        def e2e_step():
+            for i in range(calls):
+                j = i % nbuf
+                with torch.cuda.stream(up):
+                    up.wait_event(ev_fw[j])
+                    ins[j].copy_(h_in[j], non_blocking=True)
+                    ev_up[j].record(up)
+                stream.wait_event(ev_up[j])
+                stream.wait_event(ev_dn[j])
+                s = lib.lite_la_fwd_oproj(in_p[j], w_p[i], b_p[i], y_p[j], B, N, H, D, C, EPS, T, sh)
+                if s != 0:
+                    raise ll.LiteLAError(s, lib.lite_la_last_error().decode())
+                ev_fw[j].record(stream)
+                with torch.cuda.stream(down):
+                    down.wait_event(ev_fw[j])
+                    h_out[j].copy_(ys[j], non_blocking=True)
+                    ev_dn[j].record(down)
+            stream.wait_stream(down)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        e2e_ms, _ = timed(e2e_step, args.e2e_steps)
+        e2e_ms = _max_over_ranks(e2e_ms, device=dev)
+        e2e = {"value": aggregate_rate(B * N * H * calls * args.e2e_steps, world, e2e_ms), "unit": UNIT,
+               "h2d_bytes_per_step": calls * 6 * E, "d2h_bytes_per_step": calls * 2 * B * N * C,
+               "ms_per_step": e2e_ms / args.e2e_steps, "steps": args.e2e_steps,
+               "how": "per call: pinned host qkv -> device (upload stream), lite_la_fwd_oproj (compute stream, the "
+                      "layer's resident weight), y -> pinned host (download stream); 3 buffers in rotation"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, nrows, el = oracle_oproj_rate(to_bits(ins[0]), to_bits(wts[0][0]), wts[0][1].cpu().numpy(), B, N, H, T,
+                                            args.cpu_seconds)
+        cpu = {"value": rate, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+               "sample": "%d query rows of batch 0 of input buffer 0 (all %d heads against all %d keys, then the "
+                         "%d x %d projection), %.1f s" % (nrows, H, N, C, C, el)}
+
+    if rank == 0:
+        cfg = config_of(args.workload)
+        cfg.update({"workload": args.workload + "_fused_oproj", "variant": "fused_oproj", "C_out": C,
+                    "weights": "%d distinct %d x %d bf16 weights and fp32 biases, one per layer (synthetic, seeded)"
+                               % (calls, C, C),
+                    "layout": "qkv bf16 [B,N,3*H*d], W bf16 [C_out, H*d], bias fp32 [C_out], y bf16 [B,N,C_out]"})
+        line = {"metric": METRIC_OPROJ, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "us_per_call": us_call,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "math": "tensor-core bf16 x bf16 products with fp32 accumulation; LiteLA's output rounded to bf16 "
+                        "inside the GEMM's operand prologue",
+                "data": "synthetic: i.i.d. N(0,1) bf16 qkv and seeded nn.Linear-like weights",
+                "config": cfg, "roofline": roofline, "call_roofline": call_roof,
+                "unfused_chain": {"us_per_call": us_unf, "speedup_fused": us_unf / us_call, "clocks": clocks_unf,
+                                  "how": "lite_la_fwd then lite_la_out_proj (this library's tcgen05 GEMM, the same "
+                                         "tiles) on the same buffers, back to back"},
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * calls * args.steps,
+                "clocks": clocks, "gpu": torch.cuda.get_device_name(dev)}
+        if world > 1:
+            line["config"]["parallelism"] = "dp%d (independent calls per rank, no collective)" % world
+        if rejected is not None:
+            line["clocks_rejected_first_run"] = rejected
         emit(line)
     if dist is not None:
         dist.barrier()

@@ -240,6 +240,40 @@ size_t lite_la_workspace_bytes(int B, int N, int H, int d, int tokens_per_block)
  * and ELU+1 forms always take the three-kernel path. */
 int lite_la_kernels_per_call(int B, int N, int H, int d, int tokens_per_block);
 
+/* ---- LiteLA with the output projection fused ---------------------------------------------
+ *
+ * In Sana's block, LiteLA's output feeds the attention's output projection (Sana explainer,
+ * "What LiteLA actually computes"; the FLOP ledger of "Two levers" counts qkv + out proj as
+ * 4 N d^2 multiply-adds per layer).  The projection is read as a linear layer in PyTorch's
+ * convention, y = x W^T (+ b).
+ *
+ * lite_la_fwd_oproj computes y = LiteLA(qkv) W^T + bias without writing LiteLA's output x to
+ * memory: the apply (S . relu(q), normalised) runs in the projection GEMM's operand prologue
+ * and x is rounded to bf16 there, as lite_la_fwd's output would be.
+ *   qkv  : device, bf16 [B, N, 3*H*d] (layout above); d must be 32.
+ *   w_o  : device, bf16 [C_out, H*d], row-major (nn.Linear's weight), 16-byte aligned.
+ *   bias : device, fp32 [C_out], or NULL for none.
+ *   y    : device, bf16 [B, N, C_out], 16-byte aligned, not overlapping any input.
+ *   C_out: a multiple of 8 (16-byte rows), >= 0.  tokens_per_block <= 0 (or >= N): non-causal;
+ *          otherwise block-causal, and then it must be a multiple of 128 (LITELA_ERR_UNSUPPORTED
+ *          otherwise).
+ * Three kernels: the state reduction, the prefix scan (the state images, in this stream's
+ * workspace) and the fused apply + projection GEMM (tcgen05, tiles of 128 tokens x 224 output
+ * columns).  Errors, workspace and asynchrony as for lite_la_fwd.
+ * lite_la_fwd_oproj_events brackets the phases: events[0] before the reduction, events[1]
+ * after the scan, events[2] after the projection kernel (no programmatic overlap then).
+ *
+ * lite_la_out_proj is the projection alone, y = x W^T (+ bias), on a bf16 [B, N, C_in] input x
+ * (e.g. lite_la_fwd's output: the unfused chain), with the same GEMM kernel and tiles.  C_in and
+ * C_out must be multiples of 8; x, w_o and y 16-byte aligned; y must not overlap the inputs. */
+litela_status lite_la_fwd_oproj(const void* qkv, const void* w_o, const float* bias, void* y, int B, int N, int H,
+                                int d, int C_out, float eps, int tokens_per_block, cudaStream_t stream);
+litela_status lite_la_fwd_oproj_events(const void* qkv, const void* w_o, const float* bias, void* y, int B, int N,
+                                       int H, int d, int C_out, float eps, int tokens_per_block, cudaStream_t stream,
+                                       cudaEvent_t* events);
+litela_status lite_la_out_proj(const void* x, const void* w_o, const float* bias, void* y, int B, int N, int C_in,
+                               int C_out, cudaStream_t stream);
+
 /* lite_la_fwd without any allocation.  The pages describe no such call; it exists for callers
  * that cannot let a library allocate device memory: a host that owns all of the device memory
  * through its own pool and hands each op only its input and output buffers, or a latency-bound

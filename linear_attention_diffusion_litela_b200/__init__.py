@@ -16,6 +16,7 @@ import threading
 
 __all__ = [
     "LiteLAError", "lib", "lib_path", "lite_la_fwd", "lite_la_block_causal_fwd", "lite_la_bwd",
+    "lite_la_fwd_oproj", "lite_la_out_proj",
     "lite_la_workspace_bytes", "lite_la_release_workspace", "STATUS", "EXPORTED_SYMBOLS",
 ]
 
@@ -64,6 +65,10 @@ _SIGNATURES = {
     "lite_la_bwd_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "lite_la_fwd_save_state": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
     "lite_la_bwd_from_state": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
+    "lite_la_fwd_oproj": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
+    "lite_la_fwd_oproj_events": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
+                                          _c_int, _vp, _vp]),
+    "lite_la_out_proj": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _vp]),
 }
 EXPORTED_SYMBOLS = tuple(_SIGNATURES)
 
@@ -324,6 +329,62 @@ def lite_la(qkv, H: int, tokens_per_block: int = 0, d: int = 32, eps: float = 1e
 
 def lite_la_workspace_bytes(B: int, N: int, H: int, d: int = 32, tokens_per_block: int = 0) -> int:
     return int(lib().lite_la_workspace_bytes(B, N, H, d, tokens_per_block))
+
+
+def _check_weight(w, bias, C_in, device):
+    torch = _torch()
+    if not isinstance(w, torch.Tensor) or w.dtype != torch.bfloat16 or w.dim() != 2 or not w.is_contiguous() \
+            or w.shape[1] != C_in or w.device != device:
+        raise TypeError("w_o must be a contiguous bf16 tensor [C_out, %d] on the input's device" % C_in)
+    if bias is not None and (bias.dtype != torch.float32 or tuple(bias.shape) != (w.shape[0],)
+                             or not bias.is_contiguous() or bias.device != device):
+        raise TypeError("bias must be a contiguous fp32 tensor [C_out] on the input's device")
+    return int(w.shape[0])
+
+
+def _proj_out(out, B, N, C_out, device):
+    torch = _torch()
+    if out is None:
+        return torch.empty((B, N, C_out), dtype=torch.bfloat16, device=device)
+    if out.dtype != torch.bfloat16 or not out.is_contiguous() or tuple(out.shape) != (B, N, C_out) \
+            or out.device != device:
+        raise TypeError("out must be a contiguous bf16 tensor [B, N, C_out] on the input's device")
+    return out
+
+
+def lite_la_fwd_oproj(qkv, H: int, w_o, bias=None, tokens_per_block: int = 0, d: int = 32, eps: float = 1e-15,
+                      out=None, stream=None):
+    """LiteLA followed by the output projection, y = LiteLA(qkv) w_o^T (+ bias), in one pass
+    whose apply runs inside the projection GEMM (LiteLA's output never goes to memory).
+    w_o: bf16 [C_out, H*d]; bias: fp32 [C_out] or None; returns y bf16 [B, N, C_out]."""
+    torch = _torch()
+    if not isinstance(qkv, torch.Tensor) or not qkv.is_cuda or qkv.dtype != torch.bfloat16 or qkv.dim() != 3 \
+            or not qkv.is_contiguous() or qkv.shape[2] != 3 * H * d:
+        raise TypeError("qkv must be a contiguous bf16 CUDA tensor [B, N, 3*H*d]")
+    B, N = int(qkv.shape[0]), int(qkv.shape[1])
+    C_out = _check_weight(w_o, bias, H * d, qkv.device)
+    out = _proj_out(out, B, N, C_out, qkv.device)
+    with torch.cuda.device(qkv.device):
+        _check(lib().lite_la_fwd_oproj(qkv.data_ptr(), w_o.data_ptr(), bias.data_ptr() if bias is not None else None,
+                                       out.data_ptr(), B, N, H, d, C_out, eps, int(tokens_per_block),
+                                       _stream_handle(stream, qkv.device)))
+    return out
+
+
+def lite_la_out_proj(x, w_o, bias=None, out=None, stream=None):
+    """The projection alone, y = x w_o^T (+ bias), on a bf16 [B, N, C_in] input (e.g.
+    lite_la_fwd's output: the unfused chain), with the same GEMM kernel."""
+    torch = _torch()
+    if not isinstance(x, torch.Tensor) or not x.is_cuda or x.dtype != torch.bfloat16 or x.dim() != 3 \
+            or not x.is_contiguous():
+        raise TypeError("x must be a contiguous bf16 CUDA tensor [B, N, C_in]")
+    B, N, C_in = x.shape
+    C_out = _check_weight(w_o, bias, C_in, x.device)
+    out = _proj_out(out, B, N, C_out, x.device)
+    with torch.cuda.device(x.device):
+        _check(lib().lite_la_out_proj(x.data_ptr(), w_o.data_ptr(), bias.data_ptr() if bias is not None else None,
+                                      out.data_ptr(), B, N, C_in, C_out, _stream_handle(stream, x.device)))
+    return out
 
 
 def lite_la_device_status(stream=None) -> None:

@@ -20,6 +20,7 @@
 #include "litela_plan.h"
 #include "litela_bwd.cuh"
 #include "litela_fused.cuh"
+#include "litela_oproj.cuh"
 #include "litela_tc.cuh"
 
 namespace litela {
@@ -93,7 +94,11 @@ litela_status device_setup(int* num_sms) {
         (e = cudaFuncSetAttribute(litela_bwd_kv_tc<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kBkSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_bwd_kv_tc<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)kBkSmemBytes)) != cudaSuccess)
+                                  (int)kBkSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_oproj_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kOpSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_oproj_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kOpSmemBytes)) != cudaSuccess)
       return cuda_fail(e, "cudaFuncSetAttribute(dynamic shared memory)");
     if (g_encode == nullptr) {
       void* fn = nullptr;
@@ -144,6 +149,34 @@ litela_status encode_out_map(OutT* out, int B, int N, int H, CUtensorMap* map) {
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(LITELA_ERR_CUDA, "cuTensorMapEncodeTiled(out) failed (" + std::to_string((int)r) + ")");
+  return LITELA_OK;
+}
+
+// 3-D view of a bf16 [B, N, C] activation (the output projection's plain input): (channel,
+// token, batch), boxes of 64 channels x 128 tokens, 128-byte swizzle, zero fill outside.
+litela_status encode_rows_map(const void* x, int B, int N, int C, CUtensorMap* map) {
+  const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)N, (cuuint64_t)B};
+  const cuuint64_t strides[2] = {(cuuint64_t)C * 2, (cuuint64_t)C * 2 * (cuuint64_t)N};
+  const cuuint32_t box[3] = {(cuuint32_t)kOpK, (cuuint32_t)kOpTileM, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LITELA_ERR_CUDA, "cuTensorMapEncodeTiled(input) failed (" + std::to_string((int)r) + ")");
+  return LITELA_OK;
+}
+
+// 2-D view of the projection weight W [C_out, C_in] bf16: (input channel, output channel), boxes
+// of 64 input channels x 224 output channels, 128-byte swizzle, zero fill outside.
+litela_status encode_weight_map(const void* w, int C_out, int C_in, CUtensorMap* map) {
+  const cuuint64_t dims[2] = {(cuuint64_t)C_in, (cuuint64_t)C_out};
+  const cuuint64_t strides[1] = {(cuuint64_t)C_in * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kOpK, (cuuint32_t)kOpTileN};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LITELA_ERR_CUDA, "cuTensorMapEncodeTiled(weight) failed (" + std::to_string((int)r) + ")");
   return LITELA_OK;
 }
 
@@ -559,6 +592,123 @@ litela_status run_bwd(const void* qkv, const void* dout, OutT* dqkv, int B, int 
   return LITELA_OK;
 }
 
+// ---------------------------------------------------------------------------------------
+// output projection: LiteLA with the apply in the projection GEMM's prologue, and the plain
+// projection (the unfused chain's second step)
+
+// Validation shared by both: sizes, then (unless the problem is empty) the weight, bias and
+// output buffers (host-side, no CUDA call).
+litela_status validate_proj(const void* w, const float* bias, const void* y, int C_in, int C_out, bool empty) {
+  if (C_out < 0 || C_in < 0) return fail(LITELA_ERR_INVALID_ARGUMENT, "C_in and C_out must be >= 0");
+  if (C_out % 8 != 0 || C_in % 8 != 0)
+    return fail(LITELA_ERR_INVALID_ARGUMENT, "C_in and C_out must be multiples of 8 (16-byte rows)");
+  if (C_out > (1 << 24) || C_in > (1 << 24)) return fail(LITELA_ERR_INVALID_ARGUMENT, "C_in and C_out must be <= 2^24");
+  if (C_out == 0 || empty) return LITELA_OK;
+  if (w == nullptr || y == nullptr) return fail(LITELA_ERR_INVALID_ARGUMENT, "null weight or output");
+  if ((reinterpret_cast<uintptr_t>(w) & 15u) || (reinterpret_cast<uintptr_t>(y) & 15u))
+    return fail(LITELA_ERR_INVALID_ARGUMENT, "weight and output must be 16-byte aligned");
+  if (bias != nullptr && (reinterpret_cast<uintptr_t>(bias) & 3u))
+    return fail(LITELA_ERR_INVALID_ARGUMENT, "bias must be 4-byte aligned");
+  return LITELA_OK;
+}
+
+OprojPlan oproj_plan(int B, int N, int H, int C_in, int C_out, int T, int nblk, float eps) {
+  OprojPlan p{};
+  p.B = B; p.N = N; p.H = H; p.C_in = C_in; p.C_out = C_out; p.T = T; p.nblk = nblk; p.eps = eps;
+  p.ntn = (C_out + kOpTileN - 1) / kOpTileN;
+  p.ntt = (N + kOpTileM - 1) / kOpTileM;
+  p.nsteps = (C_in + kOpK - 1) / kOpK;
+  p.ntiles = (long long)B * p.ntt * p.ntn;
+  return p;
+}
+
+// LiteLA (non-causal, or block-causal with a block size that is a multiple of 128 tokens), then
+// y = x W^T (+ bias): the state reduction, the prefix scan (the state images) and the fused
+// apply + projection kernel.  events (optional): [0] before the reduction, [1] after the scan,
+// [2] after the projection kernel (then no programmatic overlap).
+litela_status run_oproj(const void* qkv, const void* w, const float* bias, __nv_bfloat16* y, int B, int N, int H, int d,
+                        int C_out, float eps, int tokens_per_block, cudaStream_t stream, cudaEvent_t* events) {
+  const bool causal = tokens_per_block > 0;
+  bool empty = false;
+  litela_status s = validate(qkv, y, 0, B, N, H, d, eps, tokens_per_block, causal, &empty);
+  if (s != LITELA_OK) return s;
+  s = validate_proj(w, bias, y, H * d, C_out, empty);
+  if (s != LITELA_OK || empty || C_out == 0) return s;
+  if (causal && tokens_per_block < N && tokens_per_block % kOpTileM != 0)
+    return fail(LITELA_ERR_UNSUPPORTED, "the fused projection needs tokens_per_block to be a multiple of 128 (or >= N)");
+  const size_t qkv_bytes = (size_t)B * N * 3 * H * d * 2, y_bytes = (size_t)B * N * C_out * 2;
+  const size_t w_bytes = (size_t)C_out * H * d * 2;
+  if (overlaps(y, y_bytes, qkv, qkv_bytes) || overlaps(y, y_bytes, w, w_bytes) ||
+      (bias && overlaps(y, y_bytes, bias, (size_t)C_out * 4)))
+    return fail(LITELA_ERR_INVALID_ARGUMENT, "the output overlaps an input");
+  int num_sms = 0;
+  s = device_setup(&num_sms);
+  if (s != LITELA_OK) return s;
+  Plan plan;
+  make_plan(B, N, H, causal ? tokens_per_block : 0, num_sms, &plan);
+  plan.fused = plan.fused_causal = false;   // the state images go through the workspace
+  plan.counters = 0;
+  Workspace* ws = nullptr;
+  s = get_workspace(plan, stream, &ws, plan.bytes);
+  if (s != LITELA_OK) return s;
+  char* base = static_cast<char*>(ws->partials);
+  float* partials = reinterpret_cast<float*>(base);
+  uint8_t* images = reinterpret_cast<uint8_t*>(base + plan.off_images);
+  CUtensorMap map_q, map_w;
+  if ((s = encode_qkv_map(qkv, B, N, H, kOpTileM, &map_q)) != LITELA_OK) return s;
+  if ((s = encode_weight_map(w, C_out, H * d, &map_w)) != LITELA_OK) return s;
+  const bool pdl = events == nullptr;
+  cudaError_t e;
+  if (events && (e = cudaEventRecord(events[0], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  if ((s = launch_reduce(plan, qkv, partials, ws->err, stream, pdl)) != LITELA_OK) return s;
+  if ((s = launch_scan(plan, partials, images, nullptr, num_sms, stream, pdl)) != LITELA_OK) return s;
+  if (events && (e = cudaEventRecord(events[1], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  const OprojPlan op = oproj_plan(B, N, H, H * d, C_out, plan.T, plan.nblk, eps);
+  const unsigned grid = (unsigned)(op.ntiles < num_sms ? op.ntiles : num_sms);
+  e = launch_ex(litela_oproj_tc<true>, dim3(grid), dim3(kOpThreads), kOpSmemBytes, stream, pdl, map_q, map_w,
+                static_cast<const uint8_t*>(images), bias, y, ws->err, op);
+  if (e != cudaSuccess) return cuda_fail(e, "launch litela_oproj_tc");
+  if (events && (e = cudaEventRecord(events[2], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  g_last_error.clear();
+  return LITELA_OK;
+}
+
+// y = x W^T (+ bias) on a bf16 [B, N, C_in] input: the same kernel with the input loaded by TMA.
+litela_status run_linear(const void* x, const void* w, const float* bias, __nv_bfloat16* y, int B, int N, int C_in,
+                         int C_out, cudaStream_t stream) {
+  if (B < 0 || N < 0) return fail(LITELA_ERR_INVALID_ARGUMENT, "B and N must be >= 0");
+  if (B > 65535 || N > (1 << 30)) return fail(LITELA_ERR_INVALID_ARGUMENT, "B must be <= 65535 and N <= 2^30");
+  litela_status s = validate_proj(w, bias, y, C_in, C_out, B == 0 || N == 0);
+  if (s != LITELA_OK) return s;
+  if (B == 0 || N == 0 || C_out == 0) return LITELA_OK;
+  if (C_in == 0) return fail(LITELA_ERR_INVALID_ARGUMENT, "C_in must be positive");
+  if (x == nullptr || (reinterpret_cast<uintptr_t>(x) & 15u))
+    return fail(LITELA_ERR_INVALID_ARGUMENT, "the input must be non-null and 16-byte aligned");
+  const size_t x_bytes = (size_t)B * N * C_in * 2, y_bytes = (size_t)B * N * C_out * 2;
+  if (overlaps(y, y_bytes, x, x_bytes) || overlaps(y, y_bytes, w, (size_t)C_out * C_in * 2) ||
+      (bias && overlaps(y, y_bytes, bias, (size_t)C_out * 4)))
+    return fail(LITELA_ERR_INVALID_ARGUMENT, "the output overlaps an input");
+  int num_sms = 0;
+  s = device_setup(&num_sms);
+  if (s != LITELA_OK) return s;
+  Plan plan;
+  make_plan(1, 1, 1, 0, num_sms, &plan);   // only for the error word of this stream's workspace
+  plan.counters = 0;
+  Workspace* ws = nullptr;
+  s = get_workspace(plan, stream, &ws, 0);
+  if (s != LITELA_OK) return s;
+  CUtensorMap map_x, map_w;
+  if ((s = encode_rows_map(x, B, N, C_in, &map_x)) != LITELA_OK) return s;
+  if ((s = encode_weight_map(w, C_out, C_in, &map_w)) != LITELA_OK) return s;
+  const OprojPlan op = oproj_plan(B, N, 0, C_in, C_out, N, 1, 0.f);
+  const unsigned grid = (unsigned)(op.ntiles < num_sms ? op.ntiles : num_sms);
+  cudaError_t e = launch_ex(litela_oproj_tc<false>, dim3(grid), dim3(kOpThreads), kOpSmemBytes, stream, true, map_x,
+                            map_w, static_cast<const uint8_t*>(nullptr), bias, y, ws->err, op);
+  if (e != cudaSuccess) return cuda_fail(e, "launch litela_oproj_tc");
+  g_last_error.clear();
+  return LITELA_OK;
+}
+
 // Fixed scratch of lite_la_fwd_noalloc: one array per device, defined statically so that the
 // entry point never allocates.  Host code must not use the symbol as an address; it asks the
 // runtime for each device's address once (noalloc_scratch below).
@@ -680,6 +830,26 @@ litela_status lite_la_state_fwd(const void* qkv, float* states, int B, int N, in
 litela_status lite_la_fwd_noalloc(const void* qkv, void* out, int B, int N, int H, int d, float eps,
                                   cudaStream_t stream) {
   return litela::run_noalloc(qkv, static_cast<__nv_bfloat16*>(out), B, N, H, d, eps, stream);
+}
+
+litela_status lite_la_fwd_oproj(const void* qkv, const void* w_o, const float* bias, void* y, int B, int N, int H,
+                                int d, int C_out, float eps, int tokens_per_block, cudaStream_t stream) {
+  return litela::run_oproj(qkv, w_o, bias, static_cast<__nv_bfloat16*>(y), B, N, H, d, C_out, eps, tokens_per_block,
+                           stream, nullptr);
+}
+
+litela_status lite_la_fwd_oproj_events(const void* qkv, const void* w_o, const float* bias, void* y, int B, int N,
+                                       int H, int d, int C_out, float eps, int tokens_per_block, cudaStream_t stream,
+                                       cudaEvent_t* events) {
+  if (events == nullptr || !events[0] || !events[1] || !events[2])
+    return litela::fail(LITELA_ERR_INVALID_ARGUMENT, "events must point to 3 CUDA events");
+  return litela::run_oproj(qkv, w_o, bias, static_cast<__nv_bfloat16*>(y), B, N, H, d, C_out, eps, tokens_per_block,
+                           stream, events);
+}
+
+litela_status lite_la_out_proj(const void* x, const void* w_o, const float* bias, void* y, int B, int N, int C_in,
+                               int C_out, cudaStream_t stream) {
+  return litela::run_linear(x, w_o, bias, static_cast<__nv_bfloat16*>(y), B, N, C_in, C_out, stream);
 }
 
 litela_status lite_la_elu1_fwd(const void* qkv, void* out, int B, int N, int H, int d, float clamp_min,

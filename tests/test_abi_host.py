@@ -199,3 +199,33 @@ def test_autograd_entry_point_rejects_host_tensors():
     qkv = torch.zeros((1, 4, 96), dtype=torch.bfloat16)
     with pytest.raises(TypeError):
         ll.lite_la(qkv, 1)
+
+
+def test_output_projection_entry_points_validate_on_the_host(lib):
+    """lite_la_fwd_oproj and lite_la_out_proj check every buffer and size before any CUDA call:
+    C_in and C_out multiples of 8 (16-byte rows), 16-byte aligned weight and output, a 4-byte
+    aligned bias (or none), no output overlapping an input, a block size that is a multiple of
+    128 tokens for the block-causal form; empty problems are no-ops."""
+    a, w, y, b = (ctypes.c_void_p(1 << k) for k in (20, 24, 30, 34))
+    f, lin = lib.lite_la_fwd_oproj, lib.lite_la_out_proj
+    for B, N, H, d, eps, want in BAD_ARGS:
+        assert f(a, w, None, y, B, N, H, d, 64, eps, 0, None) == want
+    assert f(a, w, None, y, 1, 4, 1, 32, 36, 1e-15, 0, None) == 1                    # C_out % 8
+    assert f(a, w, None, y, 1, 4, 1, 32, -8, 1e-15, 0, None) == 1
+    assert f(a, ctypes.c_void_p((1 << 24) + 8), None, y, 1, 4, 1, 32, 64, 1e-15, 0, None) == 1
+    assert f(a, w, ctypes.c_void_p((1 << 34) + 2), y, 1, 4, 1, 32, 64, 1e-15, 0, None) == 1
+    assert f(a, None, None, y, 1, 4, 1, 32, 64, 1e-15, 0, None) == 1
+    assert f(a, w, None, ctypes.c_void_p((1 << 20) + 256), 1, 4, 1, 32, 64, 1e-15, 0, None) == 1
+    assert "overlap" in lib.lite_la_last_error().decode()
+    assert f(a, w, None, y, 1, 300, 1, 32, 64, 1e-15, 100, None) == 2              # block of 100 tokens
+    assert f(a, w, None, y, 1, 4, 1, 64, 64, 1e-15, 0, None) == 2                   # d != 32
+    assert f(None, None, None, None, 0, 4, 1, 32, 64, 1e-15, 0, None) == 0          # empty
+    assert f(a, None, None, y, 1, 4, 1, 32, 0, 1e-15, 0, None) == 0                 # C_out = 0
+    null = (ctypes.c_void_p * 3)(None, None, None)
+    assert lib.lite_la_fwd_oproj_events(a, w, None, y, 1, 4, 1, 32, 64, 1e-15, 0, None, null) == 1
+    assert lin(a, w, None, y, 1, 4, 60, 64, None) == 1                              # C_in % 8
+    assert lin(ctypes.c_void_p((1 << 20) + 8), w, None, y, 1, 4, 64, 64, None) == 1
+    assert lin(None, w, None, y, 1, 4, 64, 64, None) == 1
+    assert lin(a, w, None, ctypes.c_void_p((1 << 20) + 64), 1, 4, 64, 64, None) == 1
+    assert lin(a, w, None, y, -1, 4, 64, 64, None) == 1
+    assert lin(None, None, None, None, 0, 4, 64, 64, None) == 0
