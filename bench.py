@@ -939,7 +939,8 @@ def main_oproj(args):
     k_flops = gemm_flops + apply_flops
     achieved = k_flops / (ph_us["litela_oproj_tc"] * 1e-6) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": bf16_sust, "unit": "TFLOP/s",
-                "frac": achieved / bf16_sust, "traffic": None, "kernel": "litela_oproj_tc",
+                "frac": achieved / bf16_sust, "traffic": load_traffic("litela_oproj_tc", B, N, H, T, "oproj"),
+                "kernel": "litela_oproj_tc",
                 "kernel_us": ph_us["litela_oproj_tc"], "alg_flops_per_launch": k_flops,
                 "alg_bytes_per_launch": 2 * E + 2 * C * C + 2 * B * N * C,
                 "peak_source": "%s sustained dense bf16 (cuBLAS) throughput" % bf16_src, "kernel_us_all": ph_us,
@@ -1056,6 +1057,7 @@ KERNEL_SOURCES = {
     "fwd": ["litela_abi.cu", "litela_fused.cuh", "litela_plan.h", "litela_tc.cuh", "sm100_ptx.cuh"],
     "elu1_fwd": ["litela_abi.cu", "litela_plan.h", "litela_tc.cuh", "sm100_ptx.cuh"],
     "bwd": ["litela_abi.cu", "litela_bwd.cuh", "litela_plan.h", "litela_tc.cuh", "sm100_ptx.cuh"],
+    "oproj": ["litela_abi.cu", "litela_oproj.cuh", "litela_plan.h", "litela_tc.cuh", "sm100_ptx.cuh"],
 }
 
 
