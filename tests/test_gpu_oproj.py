@@ -153,6 +153,20 @@ def test_fused_agrees_with_the_unfused_chain_and_is_deterministic():
     check(dec(y1), yud, 2.0 ** -7 * (np.abs(xd) @ np.abs(wd).T) + 2.0 ** -8 * np.abs(yud) + 1e-6, "fused vs unfused")
 
 
+def test_fused_1024px_every_element():
+    """The Sana-1600M 1024px shape (B = 2 CFG pair, N = 32 x 32, H = 70, C_out = 2240), every
+    output element, with bias."""
+    B, N, H, C_out = 2, 1024, 70, 2240
+    qkv = make_qkv(B, N, H, D, seed=1001, device="cuda")
+    w, b = make_weight(C_out, H * D, seed=1024)
+    y = run_fused(qkv, H, w.cuda(), b.cuda())
+    y2 = run_fused(qkv, H, w.cuda(), b.cuda())
+    assert torch.equal(y, y2)
+    x = attention(qkv, H)
+    y_ref = oracle.linear(x, to_bits(w), C_out, H * D, b.numpy())
+    check(dec(y), y_ref, fused_tol(x, dec(w), y_ref), "fused 1024px vs oracle")
+
+
 def test_fused_full_size_4096px_sampled_rows():
     B, N, H, C_out = 2, 16384, 70, 2240
     qkv = make_qkv(B, N, H, D, seed=4000, device="cuda")
