@@ -597,7 +597,8 @@ def main():
             e.record(stream)
     torch.cuda.synchronize(dev)
     ev_handles = [(ctypes.c_void_p * nev)(*[ctypes.c_void_p(e.cuda_event) for e in trip]) for trip in evs]
-    nk = 5 if bwd else (3 if args.variant == "elu1" else int(lib.lite_la_kernels_per_call(B, N, H, D, T)))
+    # the ELU + 1 variant's block-causal form always takes the three-kernel path
+    nk = 5 if bwd else (3 if args.variant == "elu1" and T else int(lib.lite_la_kernels_per_call(B, N, H, D, T)))
     phases = PATHS[nk]["phases"]
     kern_ms = {k: 0.0 for k in phases}
     nlaunch = 0
@@ -1055,7 +1056,7 @@ def load_traffic(kernel, B, N, H, T, call="fwd"):
 # the kernel sources each profiled kernel is built from (the ABI file sets its launch shape)
 KERNEL_SOURCES = {
     "fwd": ["litela_abi.cu", "litela_fused.cuh", "litela_plan.h", "litela_tc.cuh", "sm100_ptx.cuh"],
-    "elu1_fwd": ["litela_abi.cu", "litela_plan.h", "litela_tc.cuh", "sm100_ptx.cuh"],
+    "elu1_fwd": ["litela_abi.cu", "litela_fused.cuh", "litela_plan.h", "litela_tc.cuh", "sm100_ptx.cuh"],
     "bwd": ["litela_abi.cu", "litela_bwd.cuh", "litela_plan.h", "litela_tc.cuh", "sm100_ptx.cuh"],
     "oproj": ["litela_abi.cu", "litela_oproj.cuh", "litela_plan.h", "litela_tc.cuh", "sm100_ptx.cuh"],
 }

@@ -237,7 +237,8 @@ size_t lite_la_workspace_bytes(int B, int N, int H, int d, int tokens_per_block)
  * when it takes the fused single kernel (B * ceil(H/4) <= SM count; block-causal calls also need
  * a block size that is a multiple of 128 tokens and at most two blocks per CTA), 3 otherwise
  * (state reduction, prefix scan, apply); 0 for an empty or invalid problem.  The streaming-carry
- * and ELU+1 forms always take the three-kernel path. */
+ * form always takes the three-kernel path, and so does the ELU+1 variant's block-causal form (its
+ * non-causal form takes the fused kernel under the same condition as LiteLA's). */
 int lite_la_kernels_per_call(int B, int N, int H, int d, int tokens_per_block);
 
 /* ---- LiteLA with the output projection fused ---------------------------------------------

@@ -87,6 +87,10 @@ litela_status device_setup(int* num_sms) {
                                   (int)FusedCfg<__nv_bfloat16, true>::kSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_fused_tc<float, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)FusedCfg<float, true>::kSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_fused_tc<__nv_bfloat16, false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)FusedCfg<__nv_bfloat16, false, 1>::kSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_fused_tc<float, false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)FusedCfg<float, false, 1>::kSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_bwd_q_tc<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kBqSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_bwd_q_tc<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -338,7 +342,8 @@ litela_status launch_scan(const Plan& plan, const float* partials, uint8_t* imag
 
 // Launches the fused single kernel (non-causal path) for `plan` with the given scratch; phase
 // events, if requested, bracket it (events[1] is recorded with events[2], after the kernel).
-template <typename OutT>
+// kMap 1: the ELU + 1 variant (non-causal plans only).
+template <typename OutT, int kMap = 0>
 litela_status launch_fused(const Plan& plan, const void* qkv, OutT* out, float eps, float* partials, int* ctl,
                            size_t ctl_words, cudaStream_t stream,
                            cudaEvent_t* events, float* states = nullptr) {
@@ -360,12 +365,19 @@ litela_status launch_fused(const Plan& plan, const void* qkv, OutT* out, float e
                      plan.fused_bpc, totals};
   const unsigned grid = (unsigned)(plan.B * plan.nquads * plan.fused_cpb);
   unsigned* counters = reinterpret_cast<unsigned*>(ctl + kCounterBase);
-  if (plan.fused_causal)
-    e = launch_ex(litela_fused_tc<OutT, true>, dim3(grid), dim3(kFuThreads), FusedCfg<OutT, true>::kSmemBytes, stream,
-                  events == nullptr, map_kv, map_q, map_out, partials, counters, out, ctl, fp);
-  else
-    e = launch_ex(litela_fused_tc<OutT, false>, dim3(grid), dim3(kFuThreads), FusedCfg<OutT>::kSmemBytes, stream,
-                  events == nullptr, map_kv, map_q, map_out, partials, counters, out, ctl, fp);
+  if (kMap != 0) {
+    if (plan.fused_causal) return fail(LITELA_ERR_UNSUPPORTED, "the ELU + 1 variant's fused form is non-causal");
+    e = launch_ex(litela_fused_tc<OutT, false, 1>, dim3(grid), dim3(FusedCfg<OutT, false, 1>::kThreads),
+                  FusedCfg<OutT, false, 1>::kSmemBytes, stream, events == nullptr, map_kv, map_q, map_out, partials,
+                  counters, out, ctl, fp);
+  } else if (plan.fused_causal) {
+    e = launch_ex(litela_fused_tc<OutT, true>, dim3(grid), dim3(FusedCfg<OutT, true>::kThreads),
+                  FusedCfg<OutT, true>::kSmemBytes, stream, events == nullptr, map_kv, map_q, map_out, partials,
+                  counters, out, ctl, fp);
+  } else {
+    e = launch_ex(litela_fused_tc<OutT, false>, dim3(grid), dim3(FusedCfg<OutT>::kThreads), FusedCfg<OutT>::kSmemBytes,
+                  stream, events == nullptr, map_kv, map_q, map_out, partials, counters, out, ctl, fp);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "launch litela_fused_tc");
   if (events && ((e = cudaEventRecord(events[1], stream)) != cudaSuccess ||
                  (e = cudaEventRecord(events[2], stream)) != cudaSuccess))
@@ -460,7 +472,9 @@ litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float 
   if (s != LITELA_OK) return s;
   Plan plan;
   make_plan(B, N, H, causal ? tokens_per_block : 0, num_sms, &plan);
-  if (carry || kMap != 0) {   // the carried state enters through the scan: the three-kernel path
+  // the carried state enters through the scan, and the ELU + 1 variant's block-causal form has
+  // no fused kernel: the three-kernel path
+  if (carry || (kMap != 0 && plan.fused_causal)) {
     plan.fused = plan.fused_causal = false;
     plan.counters = 0;
   }
@@ -484,8 +498,8 @@ litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float 
                            reinterpret_cast<uint8_t*>(base + plan.off_images), ws->err, num_sms, stream, events,
                            state_in, state_out);
   else if (plan.fused)
-    s = launch_fused(plan, qkv, out, eps, reinterpret_cast<float*>(base), ws->err, ws->ctl_words, stream,
-                     events, save_states);
+    s = launch_fused<OutT, kMap>(plan, qkv, out, eps, reinterpret_cast<float*>(base), ws->err, ws->ctl_words, stream,
+                                 events, save_states);
   else
     s = launch<OutT, kMap>(plan, qkv, out, eps, reinterpret_cast<float*>(base),
                            reinterpret_cast<uint8_t*>(base + plan.off_images), ws->err, num_sms, stream, events,

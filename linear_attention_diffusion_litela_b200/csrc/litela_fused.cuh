@@ -52,18 +52,30 @@ struct FusedPlan {
 
 enum : int { kErrFusedSibling = 0x410, kErrFusedMerge = 0x420, kErrFusedP1 = 0x430, kErrFusedTicket = 0x440 };
 
-constexpr int kFuThreads = 256;     // w0 TMA, w1 MMA, w2..5 phase-1 ReLU/epilogue; phase 2: w2..3 ReLU,
-                                    // w4..7 merge then epilogue
-constexpr int kFuStages1 = 6;       // phase-1 ring of k|v stages (32 KB each)
 constexpr uint32_t kFuTmemCols = 512;
 
-template <typename OutT, bool kCausal = false>
+// kMap 0: LiteLA (ReLU, + eps).  kMap 1: the ELU + 1 variant (non-causal form only): phi formed
+// in fp32 and entered as bf16 hi + lo (phase 1: phi(k) lo boxes after each stage's k|v boxes;
+// phase 2: phi(q) / sqrt(d) lo boxes after each q stage's hi boxes), 8 feature-map warps in
+// each phase, the denominator clamped from below instead of + eps.
+template <typename OutT, bool kCausal = false, int kMap = 0>
 struct FusedCfg {
-  using A = ApplyCfg<OutT>;
+  using A = ApplyCfg<OutT, kMap>;
+  // warps: 0 TMA, 1 MMA; phase 1: 2 .. 2 + kMapWarps1 feature map (warps 2..5 also read the
+  // accumulators); phase 2: 2 .. kEpiWarp0 feature map, then 4 merge / epilogue warps
+  static constexpr int kMapWarps1 = kMap ? 8 : 4;
+  static constexpr int kMapWarps2 = kMap ? 8 : 2;
+  static constexpr int kEpiWarp0 = 2 + kMapWarps2;
+  static constexpr int kThreads = 32 * (kEpiWarp0 + 4);
+  // launch bound: with 448 threads it keeps ptxas at 128 registers (4 warps share an SM
+  // sub-partition's 16K registers)
+  static constexpr int kLaunchBound = kMap ? 512 : 256;
+  static constexpr uint32_t kStage1Bytes = (kMap ? 6 : 4) * kRedBoxBytes;       // k | v (| phi(k) lo)
+  static constexpr int kStages1 = kMap ? 4 : 6;                                  // phase-1 ring
   // the block-causal form keeps two state images (its blocks) and, for bf16 output, one q stage less
   static constexpr int kQStages = (kCausal && sizeof(OutT) == 2) ? A::kQStages - 1 : A::kQStages;
   static constexpr int kSBufs = kCausal ? 2 : 1;
-  static constexpr uint32_t kPhase1Bytes = kFuStages1 * kRedStageBytes + 512;   // + the ones tile
+  static constexpr uint32_t kPhase1Bytes = kStages1 * kStage1Bytes + 512;   // + the ones tile
   static constexpr uint32_t kPhase2Bytes =
       kQStages * A::kQStageBytes + A::kOutSlots * A::kOutSlotBytes + kSBufs * kApSbufBytes;
   static constexpr uint32_t kBodyBytes = kPhase1Bytes > kPhase2Bytes ? kPhase1Bytes : kPhase2Bytes;
@@ -74,22 +86,27 @@ struct FusedCfg {
   static constexpr int kMergeBatch = (int)(kMergeBufBytes / (kRedHeads * kStateFloats * 4));
 };
 
-template <typename OutT, bool kCausal = false>
-__global__ void __launch_bounds__(kFuThreads, 1)
+template <typename OutT, bool kCausal = false, int kMap = 0>
+__global__ void __launch_bounds__(FusedCfg<OutT, kCausal, kMap>::kLaunchBound, 1)
 litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant__ CUtensorMap tmap_q,
                 const __grid_constant__ CUtensorMap tmap_out, float* __restrict__ partials,
                 unsigned* __restrict__ counters, OutT* __restrict__ out, int* __restrict__ err, FusedPlan p) {
   using namespace sm100;
-  using Cfg = FusedCfg<OutT, kCausal>;
+  using Cfg = FusedCfg<OutT, kCausal, kMap>;
+  static_assert(!(kMap && kCausal), "the ELU + 1 variant's fused form is non-causal");
   using A = typename Cfg::A;
   constexpr int kQStages = Cfg::kQStages;
+  constexpr int kFuStages1 = Cfg::kStages1;
+  constexpr uint32_t kStage1Bytes = Cfg::kStage1Bytes;
+  constexpr int kFuThreads = Cfg::kThreads;
+  constexpr int kEpiWarp0 = Cfg::kEpiWarp0;
   constexpr int kChunksPerHead = kD * (int)sizeof(OutT) / 16;
   constexpr uint32_t kPartBytes = kRedHeads * kStateFloats * 4;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   // phase 1 layout
   uint8_t* stages = smem;
-  uint8_t* ones = smem + kFuStages1 * kRedStageBytes;
+  uint8_t* ones = smem + kFuStages1 * kStage1Bytes;
   // phase 2 layout (reuses the same bytes once phase 1 is over)
   uint8_t* qst = smem;
   uint8_t* obuf = qst + kQStages * A::kQStageBytes;
@@ -127,13 +144,13 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
     const unsigned tk = atomicAdd(&my_counters[p.counter_words - 1], 1u);
     for (int s = 0; s < kFuStages1; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&relu_done[s], 128);
+      mbar_init(&relu_done[s], 32 * Cfg::kMapWarps1);
       mbar_init(&empty[s], 1);
     }
     mbar_init(done, 1);
     for (int s = 0; s < kQStages; ++s) {
       mbar_init(&qfull[s], 1);
-      mbar_init(&qrelu[s], kApReluThreads);
+      mbar_init(&qrelu[s], 32 * Cfg::kMapWarps2);
       mbar_init(&qempty[s], 1);
     }
     mbar_init(sfull, 1);
@@ -222,7 +239,7 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
         if (i >= kFuStages1 &&
             !mbar_wait(&empty[s], ((i / kFuStages1) - 1) & 1, abort_flag, err, kErrFusedP1 | s))
           break;
-        uint8_t* st = stages + s * kRedStageBytes;
+        uint8_t* st = stages + s * kStage1Bytes;
         const int y = n0 + i * kRedTile;
         mbar_arrive_expect_tx(&full[s], kRedStageBytes);
         tma_load_3d(st, &tmap_kv, &full[s], kx, y, b);
@@ -246,7 +263,7 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
         const int s = i % kFuStages1;
         if (!mbar_wait(&relu_done[s], (i / kFuStages1) & 1, abort_flag, err, kErrFusedP1 | 8 | s)) break;
         tc_fence_after_sync();
-        const uint32_t kbase = smem_u32(stages + s * kRedStageBytes);
+        const uint32_t kbase = smem_u32(stages + s * kStage1Bytes);
         const uint32_t vbase = kbase + 2 * kRedBoxBytes;
         // block-causal: local block i / tpb accumulates in its own 256-column TMEM region
         const uint32_t dacc = tmem + (kCausal ? (uint32_t)(i / tpb) * 256u : 0u);
@@ -258,26 +275,39 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
           const uint32_t acc = (!first || ks != 0) ? 1u : 0u;
           umma_bf16(dacc, a, bv, idesc_num, acc);
           umma_bf16(dacc + 128, a, ones_desc, idesc_den, acc);
+          if (kMap) {   // the lo halves of phi(k)
+            const uint64_t al = smem_desc(kbase + 4 * kRedBoxBytes + ks * 2048, kRedBoxBytes, 1024, kSwizzle128B);
+            umma_bf16(dacc, al, bv, idesc_num, 1u);
+            umma_bf16(dacc + 128, al, ones_desc, idesc_den, 1u);
+          }
         }
         umma_commit(&empty[s]);
       }
       umma_commit(done);
     }
-  } else if (warp < 6) {
-    const int t = threadIdx.x - 64;   // 0..127
+  } else if (warp < 2 + Cfg::kMapWarps1) {
+    constexpr int kMapThreads = 32 * Cfg::kMapWarps1;
+    const int t = threadIdx.x - 64;
     for (int i = 0; i < ntiles1; ++i) {
       const int s = i % kFuStages1;
       if (!mbar_wait(&full[s], (i / kFuStages1) & 1, abort_flag, err, kErrFusedP1 | 12)) break;
-      uint8_t* st = stages + s * kRedStageBytes;
+      uint8_t* st = stages + s * kStage1Bytes;
       const int valid = min(kRedTile, n1 - (n0 + i * kRedTile));
 #pragma unroll 4
-      for (int j = t; j < 1024; j += 128) {
+      for (int j = t; j < 1024; j += kMapThreads) {
         uint4* c = reinterpret_cast<uint4*>(st + j * 16);
         const int row = (j >> 3) & (kRedTile - 1);
-        *c = row < valid ? relu_bf16x8(*c) : make_uint4(0u, 0u, 0u, 0u);
+        if (kMap == 0) {
+          *c = row < valid ? relu_bf16x8(*c) : make_uint4(0u, 0u, 0u, 0u);
+        } else {   // phi(k) = ELU + 1 as bf16 hi (in place) + lo (two boxes after v)
+          uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
+          if (row < valid) phi_elu1_hilo(*c, 1.0f, hi, lo);
+          *c = hi;
+          *reinterpret_cast<uint4*>(st + 4 * kRedBoxBytes + j * 16) = lo;
+        }
       }
       if (valid < kRedTile) {
-        for (int j = t; j < 1024; j += 128) {
+        for (int j = t; j < 1024; j += kMapThreads) {
           const int row = (j >> 3) & (kRedTile - 1);
           if (row >= valid) *reinterpret_cast<uint4*>(st + 2 * kRedBoxBytes + j * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
@@ -285,6 +315,7 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
       fence_proxy_async_smem();
       mbar_arrive(&relu_done[s]);
     }
+    if (warp < 6) {   // warps 2..5 read the accumulators (warp quarter = TMEM lane quarter)
     const int hq = warp & 3;
     float sv[kRows], tot[kRows];
 #pragma unroll
@@ -320,6 +351,7 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
       float* dst = p.totals + (((int64_t)cidx * p.cpb + r) * kRedHeads + hq) * kStateFloats;
 #pragma unroll
       for (int j = 0; j < kRows; ++j) dst[j * kD + lane] = tot[j];
+    }
     }
   }
   // phase 1 is over for this CTA: every MMA completed (the epilogue waited for `done`), every
@@ -390,6 +422,11 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
               const uint64_t ad = smem_desc(qaddr + h * kQBoxBytes + j * 64 + ks * 32, 16, 1024, kSwizzle128B);
               const uint64_t bd = smem_desc(iaddr + (h * kApHeads + j) * kImageBytes + ks * 256, 128, 512, kSwizzleNone);
               umma_bf16(tmem + a * kApAccCols + j * kImageRows, ad, bd, idesc, ks);
+              if (kMap) {   // the lo halves of phi(q)
+                const uint64_t al =
+                    smem_desc(qaddr + 2 * kQBoxBytes + h * kQBoxBytes + j * 64 + ks * 32, 16, 1024, kSwizzle128B);
+                umma_bf16(tmem + a * kApAccCols + j * kImageRows, al, bd, idesc, 1u);
+              }
             }
           }
           umma_commit(&tfull[a]);
@@ -399,23 +436,30 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
         umma_commit(&qempty[s]);
       }
     }
-  } else if (warp < 4) {
-    const int t = threadIdx.x - 64;   // 0..63
+  } else if (warp < kEpiWarp0) {
+    const int t = threadIdx.x - 64;
     const int nchunks = (pair_heads_h(p.H, q, 1) > 0 ? 2 : 1) * (int)(kQBoxBytes / 16);
     for (int lu = 0; lu < nunits; ++lu) {
       const int s = lu % kQStages;
       if (!mbar_wait(&qfull[s], (lu / kQStages) & 1, abort_flag, err, kErrApplyRelu | s)) break;
       uint8_t* st = qst + s * A::kQStageBytes;
 #pragma unroll 4
-      for (int j = t; j < nchunks; j += kApReluThreads) {
+      for (int j = t; j < nchunks; j += 32 * Cfg::kMapWarps2) {
         uint4* c = reinterpret_cast<uint4*>(st + j * 16);
-        *c = relu_bf16x8(*c);
+        if (kMap == 0) {
+          *c = relu_bf16x8(*c);
+        } else {   // phi(q) / sqrt(d): hi in place, lo two boxes further
+          uint4 hi, lo;
+          phi_elu1_hilo(*c, kInvSqrtD, hi, lo);
+          *c = hi;
+          *reinterpret_cast<uint4*>(st + 2 * kQBoxBytes + j * 16) = lo;
+        }
       }
       fence_proxy_async_smem();
       mbar_arrive(&qrelu[s]);
     }
-  } else if (warp < 8) {
-    const int et = threadIdx.x - 128;   // 0..127
+  } else if (warp < kEpiWarp0 + 4) {
+    const int et = threadIdx.x - 32 * kEpiWarp0;   // 0..127
     const bool leader = (et == 0);
     // ---- merge: wait for the siblings, sum their partials in fixed order, build the B operand.
     // Non-causal: all cpb siblings' partials, then one image.  Block-causal: the totals of
@@ -549,7 +593,9 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
             tc_fence_before_sync();
             mbar_arrive(&tempty[a]);
           }
-          const float den = (__uint_as_float(v[kD]) + __uint_as_float(v[kImageLoRow + kD])) + p.eps;
+          // LiteLA adds eps to the denominator; the ELU + 1 variant clamps it from below (p.eps)
+          const float y_d = __uint_as_float(v[kD]) + __uint_as_float(v[kImageLoRow + kD]);
+          const float den = kMap ? fmaxf(y_d, p.eps) : y_d + p.eps;
           const float inv = 1.0f / den;
           float o[kD];
 #pragma unroll

@@ -88,3 +88,14 @@ def test_elu1_is_deterministic_and_differs_from_litela():
     c = ll.lite_la_fwd(qkv, H)
     torch.cuda.synchronize()
     assert torch.equal(a, b) and not torch.equal(a, c)
+
+
+def test_elu1_more_head_quads_than_sms_takes_the_three_kernel_path():
+    """Non-causal ELU + 1 calls take the fused single kernel while B * ceil(H/4) fits the SMs;
+    with 160 head quads they take the reduction, the scan and the apply: both match the oracle."""
+    B, N, H = 8, 512, 80
+    assert ll.lib().lite_la_kernels_per_call(B, N, H, D, 0) == 3
+    assert ll.lib().lite_la_kernels_per_call(2, 4096, 70, D, 0) == 1
+    qkv = make_qkv(B, N, H, D, seed=8300, device="cuda")
+    want = oracle.elu1_fwd(to_bits(qkv), B, N, H, D, 1e-6)
+    check(run(qkv, H, None, "bf16"), want, "bf16")
