@@ -70,7 +70,11 @@ struct FusedCfg {
   // launch bound: with 448 threads it keeps ptxas at 128 registers (4 warps share an SM
   // sub-partition's 16K registers)
   static constexpr int kLaunchBound = kMap ? 512 : 256;
-  static constexpr uint32_t kStage1Bytes = (kMap ? 6 : 4) * kRedBoxBytes;       // k | v (| phi(k) lo)
+  // phase-1 stage: k | v boxes; for ELU + 1 also a box of ones right after v (so that one
+  // N = 144 product gives the numerator and the denominator: the tensor core pays per
+  // instruction, and phi's hi + lo halves would otherwise double four products per 16 tokens)
+  // and the phi(k) lo boxes
+  static constexpr uint32_t kStage1Bytes = (kMap ? 7 : 4) * kRedBoxBytes;
   static constexpr int kStages1 = kMap ? 4 : 6;                                  // phase-1 ring
   // the block-causal form keeps two state images (its blocks) and, for bf16 output, one q stage less
   static constexpr int kQStages = (kCausal && sizeof(OutT) == 2) ? A::kQStages - 1 : A::kQStages;
@@ -169,6 +173,10 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
     fence_mbar_init();
   }
   for (int i = threadIdx.x; i < 128; i += kFuThreads) reinterpret_cast<uint32_t*>(ones)[i] = 0x3F803F80u;
+  if (kMap)   // the ones box of every phase-1 stage (the loads and the map never write it)
+    for (int i = threadIdx.x; i < kFuStages1 * (int)(kRedBoxBytes / 4); i += kFuThreads)
+      reinterpret_cast<uint32_t*>(stages + (i / (kRedBoxBytes / 4)) * kStage1Bytes + 4 * kRedBoxBytes)[i % (kRedBoxBytes / 4)] =
+          0x3F803F80u;
   fence_proxy_async_smem();
   if (warp == 1) {
     tmem_alloc(tmem_holder, kFuTmemCols);
@@ -273,12 +281,14 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
           const uint64_t a = smem_desc(kbase + ks * 2048, kRedBoxBytes, 1024, kSwizzle128B);
           const uint64_t bv = smem_desc(vbase + ks * 2048, kRedBoxBytes, 1024, kSwizzle128B);
           const uint32_t acc = (!first || ks != 0) ? 1u : 0u;
-          umma_bf16(dacc, a, bv, idesc_num, acc);
-          umma_bf16(dacc + 128, a, ones_desc, idesc_den, acc);
-          if (kMap) {   // the lo halves of phi(k)
-            const uint64_t al = smem_desc(kbase + 4 * kRedBoxBytes + ks * 2048, kRedBoxBytes, 1024, kSwizzle128B);
-            umma_bf16(dacc, al, bv, idesc_num, 1u);
-            umma_bf16(dacc + 128, al, ones_desc, idesc_den, 1u);
+          if (kMap == 0) {
+            umma_bf16(dacc, a, bv, idesc_num, acc);
+            umma_bf16(dacc + 128, a, ones_desc, idesc_den, acc);
+          } else {   // [v | ones] as one N = 144 operand, for phi(k) hi then lo
+            constexpr uint32_t idesc_nd = idesc_bf16_f32(128, 144, true, true);
+            const uint64_t al = smem_desc(kbase + 5 * kRedBoxBytes + ks * 2048, kRedBoxBytes, 1024, kSwizzle128B);
+            umma_bf16(dacc, a, bv, idesc_nd, acc);
+            umma_bf16(dacc, al, bv, idesc_nd, 1u);
           }
         }
         umma_commit(&empty[s]);
@@ -299,11 +309,11 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
         const int row = (j >> 3) & (kRedTile - 1);
         if (kMap == 0) {
           *c = row < valid ? relu_bf16x8(*c) : make_uint4(0u, 0u, 0u, 0u);
-        } else {   // phi(k) = ELU + 1 as bf16 hi (in place) + lo (two boxes after v)
+        } else {   // phi(k) = ELU + 1 as bf16 hi (in place) + lo (after v and the ones box)
           uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
           if (row < valid) phi_elu1_hilo(*c, 1.0f, hi, lo);
           *c = hi;
-          *reinterpret_cast<uint4*>(st + 4 * kRedBoxBytes + j * 16) = lo;
+          *reinterpret_cast<uint4*>(st + 5 * kRedBoxBytes + j * 16) = lo;
         }
       }
       if (valid < kRedTile) {
