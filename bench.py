@@ -452,6 +452,10 @@ def main():
     ap.add_argument("--variant", choices=["litela", "elu1", "fused_oproj"], default="litela",
                     help="elu1 times the ELU+1 feature-map variant of the forward (clamp 1e-6); fused_oproj "
                          "LiteLA with the output projection fused (and the unfused chain beside it)")
+    ap.add_argument("--shard-heads", action="store_true",
+                    help="strong scaling: the ranks split the workload's heads (each rank runs its own head shard "
+                         "of every call, as after a tensor-parallel qkv projection) instead of each running the "
+                         "whole workload")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the `workloads` record (the other configs, timed after the headline)")
     args = ap.parse_args()
@@ -495,14 +499,20 @@ def main():
 
     lib = ll.lib()
     B, N, H, calls, seed0, T = WORKLOADS_BENCH[args.workload]
+    H_total = H
+    if args.shard_heads:   # this rank's heads of every call (strong scaling)
+        from linear_attention_diffusion_litela_b200.dist import shard_heads
+        h0, h1 = shard_heads(H, world, rank)
+        H = h1 - h0
     bwd = args.direction == "bwd"
     qkv_bytes, out_bytes = B * N * 3 * H * D * 2, B * N * H * D * 2
     free, _ = torch.cuda.mem_get_info(dev)
     need = calls * (qkv_bytes + out_bytes + (qkv_bytes if bwd else 0)) + (2 << 30)
     if free < need:
         raise SystemExit("not enough free GPU memory: need %.1f GB, free %.1f GB" % (need / 1e9, free / 1e9))
-    seeds = rank_seeds(workload_seeds(args.workload, calls), rank)
-    ins = [make_qkv(B, N, H, D, seed=s, device=dev, qk_shift=QK_SHIFT.get(args.workload, 0.0)) for s in seeds]
+    seeds = rank_seeds(workload_seeds(args.workload, calls), 0 if args.shard_heads else rank)
+    ins = [make_qkv(B, N, H, D, seed=s + (7919 * rank if args.shard_heads else 0), device=dev,
+                    qk_shift=QK_SHIFT.get(args.workload, 0.0)) for s in seeds]
     outs = [torch.empty((B, N, H * D), dtype=torch.bfloat16, device=dev) for _ in range(calls)]
     if bwd:   # the backward reads an incoming gradient (in `outs`) and writes dqkv
         outs = [make_dout(B, N, H, s + 500, dev) for s in seeds]
@@ -586,7 +596,9 @@ def main():
     ms_total = max_over_ranks(ms_total)
     ms_step = ms_total / args.steps
     us_call = 1e3 * ms_step / calls
-    value = aggregate_rate(B * N * H * calls * args.steps, world, ms_total)
+    # weak scaling: every rank processes the whole workload; strong: the ranks share its heads
+    value = (B * N * H_total * calls * args.steps / (ms_total / 1e3) if args.shard_heads else
+             aggregate_rate(B * N * H * calls * args.steps, world, ms_total))
 
     # per-kernel durations: the same calls through the phase-timed entry points (3 events per
     # forward call, 4 per backward call)
@@ -714,7 +726,8 @@ def main():
         torch.cuda.synchronize(dev)
         e2e_ms, _ = timed(e2e_step, args.e2e_steps)
         e2e_ms = max_over_ranks(e2e_ms)
-        e2e = {"value": aggregate_rate(B * N * H * calls * args.e2e_steps, world, e2e_ms), "unit": UNIT,
+        e2e = {"value": (B * N * H_total * calls * args.e2e_steps / (e2e_ms / 1e3) if args.shard_heads else
+                         aggregate_rate(B * N * H * calls * args.e2e_steps, world, e2e_ms)), "unit": UNIT,
                "h2d_bytes_per_step": calls * (qkv_bytes + (out_bytes if bwd else 0)),
                "d2h_bytes_per_step": calls * (qkv_bytes if bwd else out_bytes),
                "ms_per_step": e2e_ms / args.e2e_steps, "steps": args.e2e_steps,
@@ -765,6 +778,12 @@ def main():
                 "clocks": clocks, "gpu": torch.cuda.get_device_name(dev)}
         if world > 1:
             line["config"]["parallelism"] = "dp%d (independent calls per rank, no collective)" % world
+        if args.shard_heads:
+            from linear_attention_diffusion_litela_b200.dist import shard_heads
+            line["scaling"] = "strong"
+            line["config"]["parallelism"] = ("tp%d over heads: rank r runs heads shard_heads(%d, %d, r) of every call "
+                                             "(no collective)" % (world, H_total, world))
+            line["config"]["heads_per_rank"] = [shard_heads(H_total, world, r) for r in range(world)]
         if rejected is not None:
             line["clocks_rejected_first_run"] = rejected
         if records is not None:

@@ -9,7 +9,7 @@ from __future__ import annotations
 
 import os
 
-__all__ = ["world_info", "rank_seeds", "shard_heads", "max_over_ranks", "aggregate_rate"]
+__all__ = ["world_info", "rank_seeds", "shard_heads", "pack_head_shard", "max_over_ranks", "aggregate_rate"]
 
 
 def world_info():
@@ -32,6 +32,16 @@ def shard_heads(H: int, world: int, rank: int):
     h0 = H * rank // world
     h1 = H * (rank + 1) // world
     return h0, h1
+
+
+def pack_head_shard(qkv, H: int, h0: int, h1: int, d: int = 32):
+    """The packed qkv [B, N, 3*(h1-h0)*d] of heads [h0, h1) of a packed qkv [B, N, 3*H*d] (q, k
+    and v of those heads, each head-major): the input a rank gets when a tensor-parallel qkv
+    projection produces only its own heads.  Data movement only (a strided copy)."""
+    B, N = qkv.shape[0], qkv.shape[1]
+    if not 0 <= h0 < h1 <= H or qkv.shape[2] != 3 * H * d:
+        raise ValueError("bad head range or qkv shape")
+    return qkv.view(B, N, 3, H, d)[:, :, :, h0:h1].reshape(B, N, 3 * (h1 - h0) * d).contiguous()
 
 
 def max_over_ranks(value: float, device=None) -> float:

@@ -428,3 +428,20 @@ def test_fused_call_replayed_from_a_captured_graph(T):
         ll.lite_la_device_status(s)
         assert torch.equal(og, ref) and torch.equal(oe, ref)
     del g
+
+
+def test_head_shards_of_one_problem_match_the_full_call():
+    """Tensor-parallel use: each of 3 ranks gets its heads' packed qkv (pack_head_shard) and calls
+    lite_la_fwd with its own head count; the shards' outputs are the full call's heads, to the
+    oracle's bf16 tolerance (heads are independent; the shards group heads into other quads)."""
+    from linear_attention_diffusion_litela_b200.dist import pack_head_shard, shard_heads
+    B, N, H = 2, 700, 70
+    qkv = make_qkv(B, N, H, 32, seed=7070, device="cuda")
+    want = oracle_run(qkv, H)
+    full = gpu_run(qkv, H)
+    assert_close(full, want, "bf16")
+    for rank in range(3):
+        h0, h1 = shard_heads(H, 3, rank)
+        sub = pack_head_shard(qkv, H, h0, h1)
+        got = gpu_run(sub, h1 - h0)
+        assert_close(got, want[:, :, h0:h1], "bf16")

@@ -71,3 +71,26 @@ def test_shard_heads_covers_every_head_once(H, world):
     assert covered == list(range(H))
     sizes = [b - a for a, b in spans]
     assert max(sizes) - min(sizes) <= 1
+
+
+def test_head_shards_cover_every_head_once_and_pack_their_columns():
+    """shard_heads splits H heads into contiguous ranges that cover each head once (sizes differ
+    by at most one); pack_head_shard takes exactly those heads' q, k and v columns."""
+    for H in (1, 5, 36, 70):
+        for world in (1, 2, 3, 4, 8):
+            if world > H:
+                continue
+            spans = [shard_heads(H, world, r) for r in range(world)]
+            assert spans[0][0] == 0 and spans[-1][1] == H
+            assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
+            sizes = [h1 - h0 for h0, h1 in spans]
+            assert max(sizes) - min(sizes) <= 1
+    from linear_attention_diffusion_litela_b200.dist import pack_head_shard
+    B, N, H, d = 2, 3, 5, 4
+    x = torch.arange(B * N * 3 * H * d, dtype=torch.float32).reshape(B, N, 3 * H * d)
+    sub = pack_head_shard(x, H, 1, 3, d)
+    assert sub.shape == (B, N, 3 * 2 * d)
+    full = x.view(B, N, 3, H, d)
+    assert torch.equal(sub.view(B, N, 3, 2, d), full[:, :, :, 1:3])
+    with pytest.raises(ValueError):
+        pack_head_shard(x, H, 3, 3, d)
