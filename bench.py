@@ -58,6 +58,7 @@ UNIT = "tokens·heads/s"
 FP32_LANES_PER_SM = 128          # B200: 4 SM sub-partitions x 32 fp32 lanes
 NUM_SMS = 148
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
+FORM_FUSED_PAIRED = 2            # lite_la_forward_form: the fused kernel's paired form
 # The library runs a non-causal call as one fused kernel when B * ceil(H/4) fits the SMs
 # (lite_la_kernels_per_call == 1), else as three (reduction, scan, apply); lite_la_fwd_events
 # brackets the phases.  Per path: the timed phases and their algorithmic bytes (in units of
@@ -69,6 +70,8 @@ PATHS = {
         "alg_bytes_E": {"litela_reduce_tc+litela_state_scan": 4, "litela_bwd_q_tc": 6,
                         "litela_state_scan+litela_bwd_kv_tc": 8}},
     1: {"phases": ("litela_fused_tc",), "alg_bytes_E": {"litela_fused_tc": 8}},
+    # the fused kernel's paired form (lite_la_forward_form == LITELA_FORM_FUSED_PAIRED)
+    "paired": {"phases": ("litela_paired_tc",), "alg_bytes_E": {"litela_paired_tc": 8}},
     3: {"phases": ("litela_reduce_tc+litela_state_scan", "litela_apply_tc"),
         "alg_bytes_E": {"litela_reduce_tc+litela_state_scan": 4, "litela_apply_tc": 4}},
 }
@@ -313,6 +316,7 @@ def time_record_workload(ll, lib, dev, stream, wl, peaks, ffma_tflops=None, reps
            "qk_shift": QK_SHIFT.get(wl), "calls_per_step": calls, "steps_per_rep": K, "reps": reps,
            "us_per_call": us_call, "us_per_call_reps": us, "tokens_heads_per_s": B * N * H / (us_call * 1e-6),
            "kernels_per_call": int(lib.lite_la_kernels_per_call(B, N, H, D, T)),
+           "form": ll.FORMS.get(int(lib.lite_la_forward_form(B, N, H, D, T))),
            "t_hbm_us": t_hbm, "hbm_frac": t_hbm / us_call, "t_fma_us": t_fma,
            "t_roof_us": max(t_hbm, t_fma), "roof_frac": max(t_hbm, t_fma) / us_call,
            "l2": l2_note(B, N, H, calls), "clocks": clocks}
@@ -611,7 +615,10 @@ def main():
     ev_handles = [(ctypes.c_void_p * nev)(*[ctypes.c_void_p(e.cuda_event) for e in trip]) for trip in evs]
     # the ELU + 1 variant's block-causal form always takes the three-kernel path
     nk = 5 if bwd else (3 if args.variant == "elu1" and T else int(lib.lite_la_kernels_per_call(B, N, H, D, T)))
-    phases = PATHS[nk]["phases"]
+    # the ELU + 1 variant never takes the paired form
+    path = PATHS["paired"] if (nk == 1 and args.variant == "litela" and
+                               int(lib.lite_la_forward_form(B, N, H, D, T)) == FORM_FUSED_PAIRED) else PATHS[nk]
+    phases = path["phases"]
     kern_ms = {k: 0.0 for k in phases}
     nlaunch = 0
     for _ in range(args.steps):
@@ -643,7 +650,7 @@ def main():
     # element), 14 bytes per element instead of 18
     call_bytes_E = (14 if args.bwd_from_state else 18) if bwd else 8
     call_flops = flops_per_call - (2 * E * (D + 1) if bwd and args.bwd_from_state else 0)
-    alg_bytes = {k: PATHS[nk]["alg_bytes_E"][k] * E for k in phases}
+    alg_bytes = {k: path["alg_bytes_E"][k] * E for k in phases}
     peaks = load_peaks()
     dom = max(kern_us, key=kern_us.get)
     traffic = load_traffic(dom, B, N, H, T, "bwd" if bwd else ("elu1_fwd" if args.variant == "elu1" else "fwd"))
@@ -1074,7 +1081,8 @@ def load_traffic(kernel, B, N, H, T, call="fwd"):
 
 # the kernel sources each profiled kernel is built from (the ABI file sets its launch shape)
 KERNEL_SOURCES = {
-    "fwd": ["litela_abi.cu", "litela_fused.cuh", "litela_plan.h", "litela_tc.cuh", "sm100_ptx.cuh"],
+    "fwd": ["litela_abi.cu", "litela_fused.cuh", "litela_paired.cuh", "litela_plan.h", "litela_tc.cuh",
+            "sm100_ptx.cuh"],
     "elu1_fwd": ["litela_abi.cu", "litela_fused.cuh", "litela_plan.h", "litela_tc.cuh", "sm100_ptx.cuh"],
     "bwd": ["litela_abi.cu", "litela_bwd.cuh", "litela_plan.h", "litela_tc.cuh", "sm100_ptx.cuh"],
     "oproj": ["litela_abi.cu", "litela_oproj.cuh", "litela_plan.h", "litela_tc.cuh", "sm100_ptx.cuh"],

@@ -241,6 +241,29 @@ size_t lite_la_workspace_bytes(int B, int N, int H, int d, int tokens_per_block)
  * non-causal form takes the fused kernel under the same condition as LiteLA's). */
 int lite_la_kernels_per_call(int B, int N, int H, int d, int tokens_per_block);
 
+/* Which form a LiteLA forward call (lite_la_fwd, lite_la_block_causal_fwd and their _f32out
+ * forms) with these arguments takes on the current device: LITELA_FORM_THREE_KERNEL (state
+ * reduction, prefix scan, apply), LITELA_FORM_FUSED (one kernel: a CTA reduces a chunk of one
+ * head quad's tokens, the quad's sibling CTAs merge their partial states, then apply the state to
+ * a share of the quad's queries), LITELA_FORM_FUSED_PAIRED (the same work, but every CTA owns a
+ * chunk of two head quads, so that one quad's merge runs while the CTA streams the other quad's
+ * tokens; taken when a chunk has at least the paired minimum of tokens, see
+ * lite_la_set_paired_min_chunk) or LITELA_FORM_FUSED_CAUSAL (the fused kernel's block-causal
+ * form); -1 for an empty or invalid problem.  The ELU+1 variant never takes the paired form. */
+#define LITELA_FORM_THREE_KERNEL 0
+#define LITELA_FORM_FUSED 1
+#define LITELA_FORM_FUSED_PAIRED 2
+#define LITELA_FORM_FUSED_CAUSAL 3
+int lite_la_forward_form(int B, int N, int H, int d, int tokens_per_block);
+
+/* Sets the chunk length (tokens per sibling CTA and head quad) from which non-causal LiteLA calls
+ * take the paired fused form, for every device and thread of the process; tokens <= 0 restores
+ * the default, 1024 (measured on B200: with shorter chunks one quad's state reduction is too
+ * short to hide the other's merge, and the plain fused form is faster).  Returns the previous
+ * value.  Calls already enqueued are not affected; the result of a call does not depend on the
+ * form up to the order of its fp32 partial-state sums. */
+int lite_la_set_paired_min_chunk(int tokens);
+
 /* ---- LiteLA with the output projection fused ---------------------------------------------
  *
  * In Sana's block, LiteLA's output feeds the attention's output projection (Sana explainer,
@@ -286,11 +309,11 @@ litela_status lite_la_out_proj(const void* x, const void* w_o, const float* bias
  * GPU that loads the library holds it until the process exits.  A problem whose scratch does
  * not fit (lite_la_workspace_bytes() plus a few hundred bytes of control words above the limit)
  * is rejected with LITELA_ERR_INVALID_ARGUMENT and a message before anything is launched.  The
- * 4096px Sana call (B=2, N=16384, H=70) takes the single fused kernel and needs about 2.4 MB
- * (its sibling partial states); calls with more than 148 head quads (B * ceil(H/4)) take the
- * three-kernel path, whose partial states and state images need more (B=8, N=512, H=80: about
- * 6 MB).  The first call on a device looks
- * up that device's address of the array (once per device); make that first call before any
+ * 4096px Sana call (B=2, N=16384, H=70) takes the paired fused kernel and needs about 4.9 MB
+ * (the partial states of 8 siblings per head quad; 2.4 MB in the plain fused form of the 1024px
+ * and 2048px calls); calls with more than 148 head quads (B * ceil(H/4)) take the three-kernel
+ * path, whose partial states and state images need more (B=8, N=512, H=80: about 6 MB).  The
+ * first call on a device looks up that device's address of the array (once per device); make that first call before any
  * stream capture.  The call never calls cudaMalloc or cudaFree; it clears the counters it needs
  * with cudaMemsetAsync on `stream`.  All calls on a device share the one array and it keeps the
  * last call's contents, so calls that can overlap on the GPU (different streams without an

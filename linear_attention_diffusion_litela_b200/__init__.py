@@ -17,7 +17,8 @@ import threading
 __all__ = [
     "LiteLAError", "lib", "lib_path", "lite_la_fwd", "lite_la_block_causal_fwd", "lite_la_bwd",
     "lite_la_fwd_oproj", "lite_la_out_proj",
-    "lite_la_workspace_bytes", "lite_la_release_workspace", "STATUS", "EXPORTED_SYMBOLS",
+    "lite_la_workspace_bytes", "lite_la_release_workspace", "lite_la_forward_form",
+    "lite_la_set_paired_min_chunk", "STATUS", "EXPORTED_SYMBOLS",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -53,6 +54,8 @@ _SIGNATURES = {
     "lite_la_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "lite_la_fwd_noalloc": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp]),
     "lite_la_kernels_per_call": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "lite_la_forward_form": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "lite_la_set_paired_min_chunk": (_c_int, [_c_int]),
     "lite_la_elu1_fwd": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
     "lite_la_elu1_fwd_f32out": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),
     "lite_la_elu1_fwd_events": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp, _vp]),
@@ -329,6 +332,24 @@ def lite_la(qkv, H: int, tokens_per_block: int = 0, d: int = 32, eps: float = 1e
 
 def lite_la_workspace_bytes(B: int, N: int, H: int, d: int = 32, tokens_per_block: int = 0) -> int:
     return int(lib().lite_la_workspace_bytes(B, N, H, d, tokens_per_block))
+
+
+# forms of a forward call (lite_la_forward_form)
+FORMS = {0: "three_kernel", 1: "fused", 2: "fused_paired", 3: "fused_causal"}
+
+
+def lite_la_forward_form(B: int, N: int, H: int, d: int = 32, tokens_per_block: int = 0) -> str:
+    """Which kernel form a forward call with these arguments takes on the current device."""
+    f = int(lib().lite_la_forward_form(B, N, H, d, tokens_per_block))
+    if f < 0:
+        raise ValueError("empty or invalid problem")
+    return FORMS[f]
+
+
+def lite_la_set_paired_min_chunk(tokens: int) -> int:
+    """Sets the chunk length from which non-causal calls take the paired fused form (tokens <= 0:
+    the default); returns the previous value."""
+    return int(lib().lite_la_set_paired_min_chunk(int(tokens)))
 
 
 def _check_weight(w, bias, C_in, device):

@@ -11,6 +11,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <string>
@@ -21,6 +22,7 @@
 #include "litela_bwd.cuh"
 #include "litela_fused.cuh"
 #include "litela_oproj.cuh"
+#include "litela_paired.cuh"
 #include "litela_tc.cuh"
 
 namespace litela {
@@ -91,6 +93,10 @@ litela_status device_setup(int* num_sms) {
                                   (int)FusedCfg<__nv_bfloat16, false, 1>::kSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_fused_tc<float, false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)FusedCfg<float, false, 1>::kSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_paired_tc<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)PairedCfg<__nv_bfloat16>::kSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_paired_tc<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)PairedCfg<float>::kSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_bwd_q_tc<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kBqSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_bwd_q_tc<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -195,7 +201,12 @@ struct Workspace {
 };
 
 // bytes of partial-state workspace a call with `plan` uses
-size_t work_bytes(const Plan& plan) { return plan.fused ? plan.fused_bytes : plan.bytes; }
+size_t work_bytes(const Plan& plan) {
+  return plan.fused ? (plan.fused_paired ? plan.paired_bytes : plan.fused_bytes) : plan.bytes;
+}
+
+// chunk length (tokens) from which the non-causal fused path takes its paired form
+std::atomic<int> g_paired_min_chunk{kPairedMinChunk};
 
 std::mutex g_ws_mutex;
 std::map<std::pair<int, uintptr_t>, Workspace> g_ws;
@@ -365,7 +376,14 @@ litela_status launch_fused(const Plan& plan, const void* qkv, OutT* out, float e
                      plan.fused_bpc, totals};
   const unsigned grid = (unsigned)(plan.B * plan.nquads * plan.fused_cpb);
   unsigned* counters = reinterpret_cast<unsigned*>(ctl + kCounterBase);
-  if (kMap != 0) {
+  if (kMap == 0 && plan.fused_paired) {
+    FusedPlan pp = fp;
+    pp.cpb = plan.paired_cpb;
+    pp.chunk = plan.paired_chunk;
+    const unsigned pgrid = (unsigned)((plan.B * plan.nquads + 1) / 2 * plan.paired_cpb);
+    e = launch_ex(litela_paired_tc<OutT>, dim3(pgrid), dim3(PairedCfg<OutT>::kThreads), PairedCfg<OutT>::kSmemBytes,
+                  stream, events == nullptr, map_kv, map_q, map_out, partials, counters, ctl, pp);
+  } else if (kMap != 0) {
     if (plan.fused_causal) return fail(LITELA_ERR_UNSUPPORTED, "the ELU + 1 variant's fused form is non-causal");
     e = launch_ex(litela_fused_tc<OutT, false, 1>, dim3(grid), dim3(FusedCfg<OutT, false, 1>::kThreads),
                   FusedCfg<OutT, false, 1>::kSmemBytes, stream, events == nullptr, map_kv, map_q, map_out, partials,
@@ -471,13 +489,14 @@ litela_status run(const void* qkv, OutT* out, int B, int N, int H, int d, float 
   s = device_setup(&num_sms);
   if (s != LITELA_OK) return s;
   Plan plan;
-  make_plan(B, N, H, causal ? tokens_per_block : 0, num_sms, &plan);
+  make_plan(B, N, H, causal ? tokens_per_block : 0, num_sms, &plan, g_paired_min_chunk.load());
   // the carried state enters through the scan, and the ELU + 1 variant's block-causal form has
   // no fused kernel: the three-kernel path
   if (carry || (kMap != 0 && plan.fused_causal)) {
-    plan.fused = plan.fused_causal = false;
+    plan.fused = plan.fused_causal = plan.fused_paired = false;
     plan.counters = 0;
   }
+  if (kMap != 0) plan.fused_paired = false;   // the paired form is built for ReLU only
   if (carry) {
     const size_t sbytes = (size_t)B * H * kStateFloats * sizeof(float);
     const size_t qkv_bytes = (size_t)B * N * 3 * H * d * sizeof(__nv_bfloat16);
@@ -660,7 +679,7 @@ litela_status run_oproj(const void* qkv, const void* w, const float* bias, __nv_
   if (s != LITELA_OK) return s;
   Plan plan;
   make_plan(B, N, H, causal ? tokens_per_block : 0, num_sms, &plan);
-  plan.fused = plan.fused_causal = false;   // the state images go through the workspace
+  plan.fused = plan.fused_causal = plan.fused_paired = false;   // the state images go through the workspace
   plan.counters = 0;
   Workspace* ws = nullptr;
   s = get_workspace(plan, stream, &ws, plan.bytes);
@@ -757,7 +776,7 @@ litela_status run_noalloc(const void* qkv, __nv_bfloat16* out, int B, int N, int
   s = device_setup(&num_sms);
   if (s != LITELA_OK) return s;
   Plan plan;
-  make_plan(B, N, H, 0, num_sms, &plan);
+  make_plan(B, N, H, 0, num_sms, &plan, g_paired_min_chunk.load());
   const size_t err_bytes = align_up((kCounterBase + plan.counters) * sizeof(int), 256);
   const size_t need = err_bytes + work_bytes(plan);
   if (need > LITELA_NOALLOC_SCRATCH_BYTES)
@@ -946,7 +965,7 @@ int lite_la_kernels_per_call(int B, int N, int H, int d, int tokens_per_block) {
     sms = 148;
   }
   litela::Plan p;
-  litela::make_plan(B, N, H, tokens_per_block, sms, &p);
+  litela::make_plan(B, N, H, tokens_per_block, sms, &p, litela::g_paired_min_chunk.load());
   return p.fused ? 1 : 3;
 }
 
@@ -1043,8 +1062,26 @@ litela_status lite_la_release_workspace(void) {
 size_t lite_la_workspace_bytes(int B, int N, int H, int d, int tokens_per_block) {
   if (B < 0 || N < 0 || H < 0 || d != litela::kD) return 0;
   litela::Plan p;
-  if (!litela::make_plan(B, N, H, tokens_per_block, 148, &p)) return 0;
+  if (!litela::make_plan(B, N, H, tokens_per_block, 148, &p, litela::g_paired_min_chunk.load())) return 0;
   return litela::work_bytes(p) + (litela::kCounterBase + p.counters) * sizeof(int);
+}
+
+int lite_la_forward_form(int B, int N, int H, int d, int tokens_per_block) {
+  if (B <= 0 || N <= 0 || H <= 0 || d != litela::kD) return -1;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  litela::Plan p;
+  litela::make_plan(B, N, H, tokens_per_block, sms, &p, litela::g_paired_min_chunk.load());
+  if (!p.fused) return LITELA_FORM_THREE_KERNEL;
+  if (p.fused_causal) return LITELA_FORM_FUSED_CAUSAL;
+  return p.fused_paired ? LITELA_FORM_FUSED_PAIRED : LITELA_FORM_FUSED;
+}
+
+int lite_la_set_paired_min_chunk(int tokens) {
+  return litela::g_paired_min_chunk.exchange(tokens > 0 ? tokens : litela::kPairedMinChunk);
 }
 
 }  // extern "C"

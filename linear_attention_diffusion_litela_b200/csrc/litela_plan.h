@@ -34,6 +34,9 @@ constexpr int kImageTBytes = kImageTRows * kD * 2;
 // small zero-initialised control buffer: word 0 is the kernels' error word (a bounded wait that
 // timed out); the fused kernel's sibling counters start at word kCounterBase
 constexpr int kErrWords = 64;
+// the paired form of the fused path is taken when a sibling's chunk has at least this many
+// tokens: with shorter chunks one quad's reduction is too short to hide the other's merge
+constexpr int kPairedMinChunk = 1024;
 constexpr int kCounterBase = kErrWords;
 
 struct Plan {
@@ -56,6 +59,13 @@ struct Plan {
   bool fused = false;
   int fused_cpb = 0, fused_chunk = 0, fused_ntiles = 0;
   size_t fused_bytes = 0, counters = 0;
+  // its paired form (fused_paired, ReLU only): CTA r of sibling group g works on quads g and
+  // g + ceil(B * nquads / 2) (index b * nquads + q), paired_cpb siblings per quad of
+  // paired_chunk tokens each;
+  // workspace = partials [B * nquads][paired_cpb][4][33][32]; the same control words
+  bool fused_paired = false;
+  int paired_cpb = 0, paired_chunk = 0;
+  size_t paired_bytes = 0;
   // block-causal fused path (fused_causal): CTA (b, quad, r) owns blocks [r * fused_bpc, ...),
   // at most 2; workspace = block states [B][nquads][nblk][4][33][32], then the CTA totals
   // [B][nquads][fused_cpb][4][33][32] at fused_off_totals; control words: an arrival flag per
@@ -76,8 +86,10 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // tokens_per_block <= 0 or >= N selects the non-causal form.  Returns false for an empty
 // problem (B, N or H == 0); sizes must already be validated as non-negative.  num_sms is the
-// device's SM count (148 on B200).
-inline bool make_plan(int B, int N, int H, int tokens_per_block, int num_sms, Plan* p) {
+// device's SM count (148 on B200); paired_min_chunk the chunk length (tokens) from which the
+// non-causal fused path takes its paired form.
+inline bool make_plan(int B, int N, int H, int tokens_per_block, int num_sms, Plan* p,
+                      int paired_min_chunk = kPairedMinChunk) {
   *p = Plan{};
   if (B <= 0 || N <= 0 || H <= 0) return false;
   p->B = B; p->N = N; p->H = H;
@@ -114,6 +126,19 @@ inline bool make_plan(int B, int N, int H, int tokens_per_block, int num_sms, Pl
     p->fused_chunk = (int)chunk;
     p->fused_bytes = align_up((size_t)B * p->nquads * cpb * kRedHeads * kStateFloats * sizeof(float), 256);
     p->counters = (size_t)B * p->nquads + 2;   // an arrival counter per quad; finish, ticket
+    const int64_t nq = (int64_t)B * p->nquads;
+    const int64_t groups = (nq + 1) / 2;
+    int64_t S = sms / groups;
+    if (S > p->fused_ntiles) S = p->fused_ntiles;
+    if (S < 1) S = 1;
+    int64_t ch = ((int64_t)N + S - 1) / S;
+    ch = (ch + kRedTile - 1) / kRedTile * kRedTile;
+    if (nq >= 2 && ch >= paired_min_chunk) {
+      p->fused_paired = true;
+      p->paired_chunk = (int)ch;
+      p->paired_cpb = (int)(((int64_t)N + ch - 1) / ch);
+      p->paired_bytes = align_up((size_t)nq * p->paired_cpb * kRedHeads * kStateFloats * sizeof(float), 256);
+    }
   } else if (p->nblk > 1 && p->T % kApTile == 0 && (int64_t)B * p->nquads <= sms) {
     int cpb = sms / (B * p->nquads);
     if (cpb > p->nblk) cpb = p->nblk;

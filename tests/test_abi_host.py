@@ -229,3 +229,25 @@ def test_output_projection_entry_points_validate_on_the_host(lib):
     assert lin(a, w, None, ctypes.c_void_p((1 << 20) + 64), 1, 4, 64, 64, None) == 1
     assert lin(a, w, None, y, -1, 4, 64, 64, None) == 1
     assert lin(None, None, None, None, 0, 4, 64, 64, None) == 0
+
+
+def test_forward_form_and_the_paired_minimum(lib):
+    """The form query needs no GPU; the paired minimum is process-wide, returns the previous
+    value and falls back to its default (1024 tokens) for values <= 0."""
+    assert lib.lite_la_forward_form(0, 16, 1, 32, 0) == -1
+    assert lib.lite_la_forward_form(1, 16, 1, 64, 0) == -1
+    assert ll.lite_la_forward_form(2, 16384, 70) == "fused_paired"       # chunks of 2048 tokens
+    assert ll.lite_la_forward_form(2, 4096, 70) == "fused"               # chunks of 512
+    assert ll.lite_la_forward_form(1, 16384, 70, 32, 1024) == "fused_causal"
+    assert ll.lite_la_forward_form(8, 512, 80) == "three_kernel"         # 160 head quads
+    prev = ll.lite_la_set_paired_min_chunk(512)
+    try:
+        assert prev == 1024
+        assert ll.lite_la_forward_form(2, 4096, 70) == "fused_paired"
+        assert ll.lite_la_forward_form(1, 4096, 4) == "fused"            # one quad: nothing to pair
+        assert ll.lite_la_set_paired_min_chunk(-5) == 512
+        assert ll.lite_la_set_paired_min_chunk(0) == 1024
+    finally:
+        ll.lite_la_set_paired_min_chunk(prev)
+    # the workspace query follows the form: 8 siblings' partial states per quad when paired
+    assert ll.lite_la_workspace_bytes(2, 16384, 70) >= 36 * 8 * 4 * 33 * 32 * 4

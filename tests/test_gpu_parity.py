@@ -76,6 +76,37 @@ def test_small_shapes_every_element(B, N, H, mode):
     assert_close(gpu_run(qkv, H, mode=mode), oracle_run(qkv, H), mode)
 
 
+PAIRED = [  # the paired fused form (N >= 2048, two or more head quads; each CTA of a sibling
+            # group works on two quads): an odd quad count (a group with one quad), quads of 1 to
+            # 3 heads, a ragged last chunk, quads whose head pair count changes between a CTA's
+            # two quads, many siblings of one 64-token tile each
+    (1, 2048, 8), (1, 2100, 5), (2, 2048, 7), (1, 4097, 12), (2, 3000, 9), (4, 2500, 36), (3, 2048, 10),
+]
+
+
+@pytest.mark.parametrize("mode", ["bf16", "f32"])
+@pytest.mark.parametrize("B,N,H", PAIRED)
+def test_paired_fused_shapes_every_element(B, N, H, mode, paired_min_chunk):
+    paired_min_chunk(64)   # chunks of 64 tokens and more take the paired form
+    assert ll.lite_la_forward_form(B, N, H) == "fused_paired"
+    qkv = make_qkv(B, N, H, 32, seed=B * 7919 + N * 13 + H, device="cuda")
+    assert_close(gpu_run(qkv, H, mode=mode), oracle_run(qkv, H), mode)
+
+
+def test_paired_and_plain_fused_forms_agree_and_are_deterministic(paired_min_chunk):
+    """Both fused forms of the 2048px call: each bitwise repeatable, the two within the bf16
+    rounding of each other (their fp32 partial states are summed over different chunks)."""
+    w = WORKLOADS["sana1600m_2048px"]
+    qkv = make_qkv(w["B"], w["N"], w["H"], 32, seed=2222, device="cuda")
+    assert ll.lite_la_forward_form(w["B"], w["N"], w["H"]) == "fused"
+    plain = [gpu_run(qkv, w["H"]) for _ in range(2)]
+    paired_min_chunk(64)
+    assert ll.lite_la_forward_form(w["B"], w["N"], w["H"]) == "fused_paired"
+    paired = [gpu_run(qkv, w["H"]) for _ in range(2)]
+    assert np.array_equal(plain[0], plain[1]) and np.array_equal(paired[0], paired[1])
+    assert np.all(np.abs(paired[0] - plain[0]) <= 2.0 ** -7 * np.abs(plain[0]) + 1e-6)
+
+
 @pytest.mark.parametrize("mode", ["bf16", "f32"])
 @pytest.mark.parametrize("B,N,H,T", [(1, 7, 2, 1), (2, 40, 3, 1), (1, 100, 2, 7), (2, 300, 3, 128),
                                      (1, 1000, 4, 256), (1, 1000, 2, 300), (1, 513, 3, 512),
@@ -117,6 +148,7 @@ def test_2048px_sampled(shift, mode):
 @pytest.mark.parametrize("mode", ["bf16", "f32"])
 def test_4096px_sampled(mode):
     w = WORKLOADS["sana4800m_4096px"]
+    assert ll.lite_la_forward_form(w["B"], w["N"], w["H"]) == "fused_paired"
     qkv = make_qkv(w["B"], w["N"], w["H"], 32, seed=4000, device="cuda")
     rows = sample_rows(w["N"], k=96, seed=4)
     got = gpu_run(qkv, w["H"], mode=mode)[:, rows]

@@ -1,0 +1,98 @@
+"""Host-side checks of the forward's partition (litela_plan.h compiled with g++; no GPU).
+
+The paired fused form (fused_paired: every CTA of a sibling group works on two head quads) must
+reduce every (quad, token) exactly once and apply every (quad, 128-token tile) exactly once,
+with at most one CTA per SM; the index arithmetic below restates the kernel's role decode
+(ticket -> sibling r of group g, units g and g + ceil(nq / 2), token chunk r, tiles
+[r*nt/S, (r+1)*nt/S)).
+"""
+import json
+import os
+import shutil
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "linear_attention_diffusion_litela_b200", "csrc")
+
+SHAPES = [(2, 16384, 70), (2, 4096, 70), (2, 1024, 70), (1, 256, 36), (1, 2048, 8), (1, 2100, 5),
+          (2, 2048, 7), (3, 4096, 6), (1, 4097, 12), (2, 3000, 9), (4, 2500, 36), (1, 8192, 140),
+          (1, 2049, 2), (1, 5000, 4), (40, 2048, 32)]
+
+DRIVER = r"""
+#include <cstdio>
+#include "litela_plan.h"
+int main(int argc, char** argv) {
+  const int min_chunk = atoi(argv[1]);
+  for (int i = 2; i + 2 < argc; i += 3) {
+    litela::Plan p;
+    litela::make_plan(atoi(argv[i]), atoi(argv[i + 1]), atoi(argv[i + 2]), 0, 148, &p, min_chunk);
+    printf("{\"fused\": %d, \"paired\": %d, \"nquads\": %d, \"ntiles\": %d, \"S\": %d, \"chunk\": %d, "
+           "\"bytes\": %zu, \"counters\": %zu, \"cpb\": %d}\n", p.fused, p.fused_paired, p.nquads,
+           p.fused_ntiles, p.paired_cpb, p.paired_chunk, p.paired_bytes, p.counters, p.fused_cpb);
+  }
+  return 0;
+}
+"""
+
+
+@pytest.fixture(scope="module", params=[1024, 64], ids=["default_min_chunk", "min_chunk_64"])
+def plans(tmp_path_factory, request):
+    gxx = shutil.which("g++")
+    if gxx is None:
+        pytest.skip("g++ not available")
+    d = tmp_path_factory.mktemp("plan")
+    src = d / "plan_driver.cpp"
+    src.write_text("#include <cstdlib>\n" + DRIVER)
+    exe = d / "plan_driver"
+    subprocess.run([gxx, "-std=c++17", "-O1", "-I", CSRC, str(src), "-o", str(exe)], check=True)
+    args = [str(x) for s in SHAPES for x in s]
+    out = subprocess.run([str(exe), str(request.param), *args], check=True, capture_output=True, text=True).stdout
+    return request.param, dict(zip(SHAPES, (json.loads(l) for l in out.splitlines())))
+
+
+def test_paired_form_is_chosen_for_chunks_of_the_paired_minimum(plans):
+    min_chunk, plans = plans
+    for (B, N, H), p in plans.items():
+        nq = B * ((H + 3) // 4)
+        assert p["fused"] == (nq <= 148)
+        # the paired form's chunk: 148 // ceil(nq / 2) siblings per quad (at most one per apply
+        # tile), tokens split evenly and rounded up to 64
+        S = max(1, min(148 // ((nq + 1) // 2), -(-N // 128)))
+        chunk = -(-(-(-N // S)) // 64) * 64
+        assert p["paired"] == (p["fused"] == 1 and nq >= 2 and chunk >= min_chunk), (B, N, H, p)
+        if p["paired"]:
+            assert p["chunk"] == chunk
+    # the Sana 4096px call: 18 sibling groups of 8 CTAs (144 CTAs), chunks of 2048 tokens; the
+    # 2048px call (chunks of 512) takes the plain fused form unless the minimum is lowered
+    p = plans[(2, 16384, 70)]
+    assert p["paired"] and p["S"] == 8 and p["chunk"] == 2048
+    assert plans[(2, 4096, 70)]["paired"] == (min_chunk <= 512)
+
+
+@pytest.mark.parametrize("shape", [s for s in SHAPES])
+def test_paired_partition_covers_every_token_and_tile_once(plans, shape):
+    B, N, H = shape
+    p = plans[1][shape]
+    if not p["paired"]:
+        return
+    nq = B * p["nquads"]
+    S, chunk, nt = p["S"], p["chunk"], p["ntiles"]
+    grid = (nq + 1) // 2 * S
+    assert grid <= 148 and chunk % 64 == 0 and (S - 1) * chunk < N <= S * chunk
+    assert p["bytes"] >= nq * S * 4 * 33 * 32 * 4 and p["counters"] == nq + 2
+    red = [[0] * N for _ in range(nq)]
+    app = [[0] * nt for _ in range(nq)]
+    for ticket in range(grid):
+        r, g = ticket % S, ticket // S
+        units = [c for c in (g, g + (nq + 1) // 2) if c < nq]
+        n0, n1 = r * chunk, min(r * chunk + chunk, N)
+        t0, t1 = r * nt // S, (r + 1) * nt // S
+        for c in units:
+            for t in range(n0, n1):
+                red[c][t] += 1
+            for tl in range(t0, t1):
+                app[c][tl] += 1
+    assert all(x == 1 for row in red for x in row)
+    assert all(x == 1 for row in app for x in row)

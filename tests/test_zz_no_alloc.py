@@ -13,8 +13,9 @@ check each result three ways:
     order, so any difference would come from the scratch (a stale value, a wrong offset);
   * through lite_la_device_status, which reads the array's error word (a bounded wait that
     timed out would otherwise show only as wrong output).
-Both of the entry point's paths are covered: the single fused kernel (B * ceil(H/4) <= 148)
-and the three-kernel path (more head quads than SMs).  A problem too large for the array is
+All of the entry point's paths are covered: the single fused kernel (B * ceil(H/4) <= 148), its
+paired form (chunks of at least the paired minimum: the 4096px call) and the three-kernel path
+(more head quads than SMs).  A problem too large for the array is
 refused before anything runs.  This file is named to be collected last.
 """
 import ctypes
@@ -82,6 +83,7 @@ def test_noalloc_matches_the_oracle_and_lite_la_fwd_on_two_calls_in_a_row(lib):
 
 def test_noalloc_full_size_4096px_call(lib):
     B, N, H = 2, 16384, 70
+    assert ll.lite_la_forward_form(B, N, H) == "fused_paired"
     qkv = make_qkv(B, N, H, 32, seed=4000, device="cuda")
     got = noalloc(lib, qkv, H)
     ll.lite_la_device_status()
