@@ -88,6 +88,8 @@ struct FusedCfg {
   // are contiguous and idle until the state is ready (the last stage's first q load waits)
   static constexpr uint32_t kMergeBufBytes = A::kQStageBytes + A::kOutSlots * A::kOutSlotBytes;
   static constexpr int kMergeBatch = (int)(kMergeBufBytes / (kRedHeads * kStateFloats * 4));
+  // 32 KB stages of the CTA's input prefetched into L2 before the programmatic-launch wait
+  static constexpr int kPrefetchStages = 12;
 };
 
 template <typename OutT, bool kCausal = false, int kMap = 0>
@@ -214,6 +216,37 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
       tmem_dealloc(tmem, kFuTmemCols);
     }
   };
+  if (warp == 0 && lane == 0) {
+    // while the previous call drains: warm L2 with this CTA's first tiles, its k|v tiles then
+    // (short chunks) its q tiles, up to kPrefetchStages stages of 32 KB (the ticket fixes the
+    // CTA's role before the wait; a prefetch reads nothing into the CTA).  Measured back to
+    // back, without / with 12 stages: 2048px 40.2 / 37.4 us, 1024px 18.1 / 16.8 us, 512px
+    // 11.3 / 10.7 us, block-causal 16 x 1024 72.9 / 67.7 us (6 stages: 38.6 and 69.3 us; 24
+    // stages: 42.0 and 70.9 us, the prefetches then evict more of what the previous call uses)
+    const int tk = *ticket_slot;
+    if (tk >= 0 && tk < (int)gridDim.x) {
+      const int rr = tk % p.cpb, qb = tk / p.cpb;
+      const int qq = qb % p.nquads, bb = qb / p.nquads;
+      const int b0k = kCausal ? rr * p.bpc : 0;
+      const int nb = kCausal ? max(0, min(b0k + p.bpc, p.nblk) - b0k) : 1;
+      const int y0 = kCausal ? b0k * p.T : rr * p.chunk;
+      const int y1 = kCausal ? min((b0k + nb) * p.T, p.N) : min(y0 + p.chunk, p.N);
+      const int kx = p.H * kD + qq * (kRedHeads * kD), vx = 2 * p.H * kD + qq * (kRedHeads * kD);
+      int left = Cfg::kPrefetchStages;
+      for (int y = y0; y < y1 && left > 0; y += kRedTile, --left) {
+        tma_prefetch_3d(&tmap_kv, kx, y, bb);
+        tma_prefetch_3d(&tmap_kv, kx + 64, y, bb);
+        tma_prefetch_3d(&tmap_kv, vx, y, bb);
+        tma_prefetch_3d(&tmap_kv, vx + 64, y, bb);
+      }
+      const int u0 = kCausal ? y0 / kApTile : (int)((long long)rr * p.ntiles / p.cpb);
+      const int u1 = kCausal ? (y1 + kApTile - 1) / kApTile : (int)((long long)(rr + 1) * p.ntiles / p.cpb);
+      const int np = pair_heads_h(p.H, qq, 1) > 0 ? 2 : 1;
+      for (int u = u0; u < u1 && left > 0; ++u, --left)
+        for (int h = 0; h < np; ++h)
+          tma_prefetch_3d(&tmap_q, qq * kApUnitHeads * kD + h * kApHeads * kD, u * kApTile, bb);
+    }
+  }
   pdl_wait_primary();
   const int ticket = *ticket_slot;
   if (ticket < 0 || ticket >= (int)gridDim.x) {   // control words not clean: record it, do nothing

@@ -70,6 +70,8 @@ struct PairedCfg {
   static constexpr uint32_t kBarBytes = 512;
   static constexpr uint32_t kSmemBytes = kStages1 * kStageBytes + kApSbufBytes + 512 + kBarBytes + 1024;
   static constexpr uint32_t kAcc1Col = 2 * kApAccCols;
+  // k|v tiles of unit 0 prefetched into L2 before the programmatic-launch wait
+  static constexpr int kPrefetchTiles = 12;
 };
 static_assert(kRedStageBytes == 2 * kQBoxBytes, "a k|v stage and a q stage take the same ring slot");
 static_assert(kApSbufBytes <= kRedStageBytes, "unit 1's image fits one stage");
@@ -165,6 +167,26 @@ litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
       tmem_dealloc(tmem, kFuTmemCols);
     }
   };
+  if (warp == 0 && lane == 0) {
+    // while the previous call drains: warm L2 with this CTA's first k|v tiles (its ticket fixes
+    // its units before the wait; a prefetch reads nothing into the CTA).  Measured at 4096px,
+    // back to back: 119.8 us without, 114.1 us with 12 tiles (6 and 18: 116.2, 114.4; 24: 116.3,
+    // the prefetches then evict more of what the previous call still uses)
+    const int tk = *ticket_slot;
+    if (tk >= 0 && tk < (int)gridDim.x) {
+      const int rr = tk % p.cpb, c = tk / p.cpb;
+      const int bb = c / p.nquads, qq = c - bb * p.nquads;
+      const int y0 = rr * p.chunk, y1 = min(y0 + p.chunk, p.N);
+      const int kx = p.H * kD + qq * (kRedHeads * kD), vx = 2 * p.H * kD + qq * (kRedHeads * kD);
+      for (int i = 0; i < Cfg::kPrefetchTiles && y0 + i * kRedTile < y1; ++i) {
+        const int y = y0 + i * kRedTile;
+        tma_prefetch_3d(&tmap_kv, kx, y, bb);
+        tma_prefetch_3d(&tmap_kv, kx + 64, y, bb);
+        tma_prefetch_3d(&tmap_kv, vx, y, bb);
+        tma_prefetch_3d(&tmap_kv, vx + 64, y, bb);
+      }
+    }
+  }
   pdl_wait_primary();
   const int ticket = *ticket_slot;
   if (ticket < 0 || ticket >= (int)gridDim.x) {   // control words not clean: record it, do nothing
