@@ -5,14 +5,17 @@
 //
 // Method: see litela_tc.cuh.  The nq quads are indexed c = b * nquads + q.  A sibling group g
 // of S CTAs (S consecutive tickets) owns quads g and g + ceil(nq / 2) (its units 0 and 1; the
-// last group may own one); sibling r takes token chunk r of both quads for the reduction and apply tiles
-// [r * ntiles / S, (r + 1) * ntiles / S) of both.  One ring of 32 KB stages carries, in order,
+// last group may own one); sibling r takes token chunk r of both quads for the reduction and
+// apply tiles [r * ntiles / S, (r + 1) * ntiles / S) of both.  One ring of 32 KB stages
+// carries, in order,
 //   unit 0's k|v tiles (64 tokens x 4 heads of k and of v), unit 1's k|v tiles   (6 stages),
-//   unit 0's q tiles (128 tokens x 4 heads), unit 1's q tiles            (the first 4 stages),
+//   unit 0's q tiles (128 tokens x 4 heads), unit 1's q tiles       (the first 4 stages),
 // so the TMA producer streams without a break between the phases; once the reductions are
-// over, the stages after the q stages hold the output staging and unit 1's state image.  Four
-// ReLU warps clamp every stage in place (k of a k|v stage, all of a q stage).  One thread
-// issues the MMAs in the same order: per 16 tokens of unit u's k|v, D_u[0:128, 0:128] += phi(K)^T . V and
+// over, the stages after the q stages hold the output staging and unit 1's state image.
+// Before the programmatic-launch wait the producer prefetches its first k|v tiles into L2, so
+// that the start of a call overlaps the end of the previous one.  Four ReLU warps clamp every
+// stage in place (k of a k|v stage, all of a q stage).  One thread issues the MMAs in the same
+// order: per 16 tokens of unit u's k|v, D_u[0:128, 0:128] += phi(K)^T . V and
 // D_u[0:128, 128:144] += phi(K)^T . 1 into TMEM accumulator u; then, once unit 0's merged state
 // is in shared memory, y = phi(Q) . [S_hi ; S_lo]^T per head of unit 0's q tiles (M = 128
 // tokens, N = 80, one head pair per TMEM slot, three slots), then the same for unit 1.
