@@ -58,7 +58,7 @@ UNIT = "tokens·heads/s"
 FP32_LANES_PER_SM = 128          # B200: 4 SM sub-partitions x 32 fp32 lanes
 NUM_SMS = 148
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0}
-FORM_FUSED_PAIRED = 2            # lite_la_forward_form: the fused kernel's paired form
+FORMS_PAIRED = (2, 4)            # lite_la_forward_form: the paired fused forms (non-causal, block-causal)
 # The library runs a non-causal call as one fused kernel when B * ceil(H/4) fits the SMs
 # (lite_la_kernels_per_call == 1), else as three (reduction, scan, apply); lite_la_fwd_events
 # brackets the phases.  Per path: the timed phases and their algorithmic bytes (in units of
@@ -617,7 +617,7 @@ def main():
     nk = 5 if bwd else (3 if args.variant == "elu1" and T else int(lib.lite_la_kernels_per_call(B, N, H, D, T)))
     # the ELU + 1 variant never takes the paired form
     path = PATHS["paired"] if (nk == 1 and args.variant == "litela" and
-                               int(lib.lite_la_forward_form(B, N, H, D, T)) == FORM_FUSED_PAIRED) else PATHS[nk]
+                               int(lib.lite_la_forward_form(B, N, H, D, T)) in FORMS_PAIRED) else PATHS[nk]
     phases = path["phases"]
     kern_ms = {k: 0.0 for k in phases}
     nlaunch = 0

@@ -248,16 +248,21 @@ int lite_la_kernels_per_call(int B, int N, int H, int d, int tokens_per_block);
  * a share of the quad's queries), LITELA_FORM_FUSED_PAIRED (the same work, but every CTA owns a
  * chunk of two head quads, so that one quad's merge runs while the CTA streams the other quad's
  * tokens; taken when a chunk has at least the paired minimum of tokens, see
- * lite_la_set_paired_min_chunk) or LITELA_FORM_FUSED_CAUSAL (the fused kernel's block-causal
- * form); -1 for an empty or invalid problem.  The ELU+1 variant never takes the paired form. */
+ * lite_la_set_paired_min_chunk), LITELA_FORM_FUSED_CAUSAL (the fused kernel's block-causal form:
+ * a CTA owns one or two consecutive causal blocks of one quad) or LITELA_FORM_FUSED_PAIRED_CAUSAL
+ * (the paired kernel's block-causal form: a CTA owns blocks r and r + ceil(nblk/2) of one quad,
+ * so that the prefix of its first block is merged while it reduces the second; taken where
+ * the plain form would give each CTA two blocks and blocks have at least the paired minimum of
+ * tokens); -1 for an empty or invalid problem.  The ELU+1 variant never takes a paired form. */
 #define LITELA_FORM_THREE_KERNEL 0
 #define LITELA_FORM_FUSED 1
 #define LITELA_FORM_FUSED_PAIRED 2
 #define LITELA_FORM_FUSED_CAUSAL 3
+#define LITELA_FORM_FUSED_PAIRED_CAUSAL 4
 int lite_la_forward_form(int B, int N, int H, int d, int tokens_per_block);
 
-/* Sets the chunk length (tokens per sibling CTA and head quad) from which non-causal LiteLA calls
- * take the paired fused form, for every device and thread of the process; tokens <= 0 restores
+/* Sets the chunk length (tokens per sibling CTA and head quad; the block size for block-causal
+ * calls) from which LiteLA calls take a paired fused form, for every device and thread of the process; tokens <= 0 restores
  * the default, 1024 (measured on B200: with shorter chunks one quad's state reduction is too
  * short to hide the other's merge, and the plain fused form is faster).  Returns the previous
  * value.  Calls already enqueued are not affected; the result of a call does not depend on the

@@ -335,7 +335,7 @@ def lite_la_workspace_bytes(B: int, N: int, H: int, d: int = 32, tokens_per_bloc
 
 
 # forms of a forward call (lite_la_forward_form)
-FORMS = {0: "three_kernel", 1: "fused", 2: "fused_paired", 3: "fused_causal"}
+FORMS = {0: "three_kernel", 1: "fused", 2: "fused_paired", 3: "fused_causal", 4: "fused_paired_causal"}
 
 
 def lite_la_forward_form(B: int, N: int, H: int, d: int = 32, tokens_per_block: int = 0) -> str:
@@ -347,8 +347,8 @@ def lite_la_forward_form(B: int, N: int, H: int, d: int = 32, tokens_per_block: 
 
 
 def lite_la_set_paired_min_chunk(tokens: int) -> int:
-    """Sets the chunk length from which non-causal calls take the paired fused form (tokens <= 0:
-    the default); returns the previous value."""
+    """Sets the chunk length (the block size of block-causal calls) from which calls take a paired
+    fused form (tokens <= 0: the default); returns the previous value."""
     return int(lib().lite_la_set_paired_min_chunk(int(tokens)))
 
 

@@ -97,6 +97,10 @@ litela_status device_setup(int* num_sms) {
                                   (int)PairedCfg<__nv_bfloat16>::kSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_paired_tc<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)PairedCfg<float>::kSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_paired_tc<__nv_bfloat16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)PairedCfg<__nv_bfloat16>::kSmemBytes)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(litela_paired_tc<float, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)PairedCfg<float>::kSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_bwd_q_tc<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kBqSmemBytes)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(litela_bwd_q_tc<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -380,9 +384,16 @@ litela_status launch_fused(const Plan& plan, const void* qkv, OutT* out, float e
     FusedPlan pp = fp;
     pp.cpb = plan.paired_cpb;
     pp.chunk = plan.paired_chunk;
-    const unsigned pgrid = (unsigned)((plan.B * plan.nquads + 1) / 2 * plan.paired_cpb);
-    e = launch_ex(litela_paired_tc<OutT>, dim3(pgrid), dim3(PairedCfg<OutT>::kThreads), PairedCfg<OutT>::kSmemBytes,
-                  stream, events == nullptr, map_kv, map_q, map_out, partials, counters, ctl, pp);
+    // non-causal: ceil(nq / 2) sibling groups of two quads; block-causal: a group per quad
+    const int nq = plan.B * plan.nquads;
+    const unsigned pgrid = (unsigned)((plan.fused_causal ? nq : (nq + 1) / 2) * plan.paired_cpb);
+    if (plan.fused_causal)
+      e = launch_ex(litela_paired_tc<OutT, true>, dim3(pgrid), dim3(PairedCfg<OutT>::kThreads),
+                    PairedCfg<OutT>::kSmemBytes, stream, events == nullptr, map_kv, map_q, map_out, partials, counters,
+                    ctl, pp);
+    else
+      e = launch_ex(litela_paired_tc<OutT>, dim3(pgrid), dim3(PairedCfg<OutT>::kThreads), PairedCfg<OutT>::kSmemBytes,
+                    stream, events == nullptr, map_kv, map_q, map_out, partials, counters, ctl, pp);
   } else if (kMap != 0) {
     if (plan.fused_causal) return fail(LITELA_ERR_UNSUPPORTED, "the ELU + 1 variant's fused form is non-causal");
     e = launch_ex(litela_fused_tc<OutT, false, 1>, dim3(grid), dim3(FusedCfg<OutT, false, 1>::kThreads),
@@ -1076,7 +1087,7 @@ int lite_la_forward_form(int B, int N, int H, int d, int tokens_per_block) {
   litela::Plan p;
   litela::make_plan(B, N, H, tokens_per_block, sms, &p, litela::g_paired_min_chunk.load());
   if (!p.fused) return LITELA_FORM_THREE_KERNEL;
-  if (p.fused_causal) return LITELA_FORM_FUSED_CAUSAL;
+  if (p.fused_causal) return p.fused_paired ? LITELA_FORM_FUSED_PAIRED_CAUSAL : LITELA_FORM_FUSED_CAUSAL;
   return p.fused_paired ? LITELA_FORM_FUSED_PAIRED : LITELA_FORM_FUSED;
 }
 

@@ -26,6 +26,13 @@
 // during unit 0's apply.  Four epilogue warps read the apply's accumulators (thread = token),
 // form y[r] / (y[d] + eps) and stage each head pair's output box, which is stored with TMA as
 // soon as it is staged.
+// Block-causal form (kCausal, blocks of T tokens, T a multiple of 128): group g is quad g alone
+// and sibling r owns its blocks r and r + S (units 0 and 1; S = ceil(nblk / 2)).  Each sibling
+// publishes its two block states, each with a flag of its own.  Block r's prefix (the sum of
+// the states of blocks 0..r, in that order) needs only first-half blocks, which the siblings
+// publish halfway through their reductions, so its merge runs during block r + S's reduction;
+// block r + S's prefix continues the same running sum over blocks r + 1..r + S, during block r's
+// apply.
 // TMEM (512 columns): accumulator 0 in columns 0..143, under apply slot 0, which the MMAs use
 // only after unit 0's merge (it follows the read-out); accumulator 1 in columns 320..463,
 // under apply slot 2, which they use only after the merge warps release it.
@@ -80,7 +87,7 @@ static_assert(kRedStageBytes == 2 * kQBoxBytes, "a k|v stage and a q stage take 
 static_assert(kApSbufBytes <= kRedStageBytes, "unit 1's image fits one stage");
 static_assert(PairedCfg<__nv_bfloat16>::kAcc1Col + 144 <= kFuTmemCols, "TMEM columns");
 
-template <typename OutT>
+template <typename OutT, bool kCausal = false>
 __global__ void __launch_bounds__(PairedCfg<OutT>::kLaunchBound, 1)
 litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant__ CUtensorMap tmap_q,
                  const __grid_constant__ CUtensorMap tmap_out, float* __restrict__ partials,
@@ -202,21 +209,37 @@ litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
   }
   const int S = p.cpb;
   const int r = ticket % S, g = ticket / S;
-  // units g and g + G of the nq quads (G = ceil(nq / 2) groups): at any time the CTAs stream the
-  // quads of one contiguous range, so every DRAM page of a token row is read in one pass
+  // non-causal: units g and g + G of the nq quads (G = ceil(nq / 2) groups): at any time the CTAs
+  // stream the quads of one contiguous range, so every DRAM page of a token row is read in one
+  // pass; block-causal: blocks r and r + S of quad g
   const int nq = p.B * p.nquads, G = (nq + 1) / 2;
-  const int c0 = g, c1 = g + G;
-  const int nu = c1 < nq ? 2 : 1;
+  const int c0 = g, c1 = kCausal ? g : g + G;
+  const int blk0 = r, blk1 = r + S;   // block-causal
+  const int nu = kCausal ? (blk1 < p.nblk ? 2 : 1) : (c1 < nq ? 2 : 1);
   const int b0 = c0 / p.nquads, q0 = c0 - b0 * p.nquads;
   const int b1 = c1 / p.nquads, q1 = c1 - b1 * p.nquads;
-  // this sibling's share of both quads: reduction tiles of 64 tokens in [n0, n1), apply tiles
-  // of 128 tokens [t0, t1)
-  const int n0 = r * p.chunk, n1 = min(n0 + p.chunk, p.N);
-  const int P = n1 > n0 ? (n1 - n0 + kRedTile - 1) / kRedTile : 0;
-  const int t0 = (int)((long long)r * p.ntiles / S), t1 = (int)((long long)(r + 1) * p.ntiles / S);
-  const int Q = t1 - t0;
-  const int nitems = nu * (P + Q);
-  const int nP = nu * P;
+  // unit u's tokens: reduction tiles of 64 tokens in [n0_u, n1_u), apply tiles of 128 tokens
+  // [t0_u, t1_u) (non-causal: chunk r of the quad and tiles [r * ntiles / S, (r + 1) * ntiles / S);
+  // block-causal: the block and its tiles)
+  const int n0a = kCausal ? blk0 * p.T : r * p.chunk;
+  const int n1a = min(n0a + p.chunk, p.N);
+  const int n0b = kCausal ? blk1 * p.T : n0a;
+  const int n1b = nu == 2 ? min(n0b + p.chunk, p.N) : n0b;
+  const int Pa = n1a > n0a ? (n1a - n0a + kRedTile - 1) / kRedTile : 0;
+  const int Pb = n1b > n0b ? (n1b - n0b + kRedTile - 1) / kRedTile : 0;
+  const int t0a = kCausal ? n0a / kApTile : (int)((long long)r * p.ntiles / S);
+  const int t1a = kCausal ? (n1a + kApTile - 1) / kApTile : (int)((long long)(r + 1) * p.ntiles / S);
+  const int t0b = kCausal ? n0b / kApTile : t0a;
+  const int t1b = kCausal ? (n1b + kApTile - 1) / kApTile : (nu == 2 ? t1a : t0a);
+  const int Qa = t1a - t0a, Qb = t1b - t0b;
+  const int nP = Pa + Pb;
+  const int nitems = nP + Qa + Qb;
+  // per unit u: first reduction token, reduction end, reduction tiles, first apply tile, apply tiles
+  auto N0 = [&](int u) { return u ? n0b : n0a; };
+  auto N1 = [&](int u) { return u ? n1b : n1a; };
+  auto P_ = [&](int u) { return u ? Pb : Pa; };
+  auto T0 = [&](int u) { return u ? t0b : t0a; };
+  auto Q_ = [&](int u) { return u ? Qb : Qa; };
   // item i's ring stage and how many earlier items used it: the reductions' items cycle
   // through R stages, the applies' through the first R2
   auto slot = [&](int i, int& s, int& use) {
@@ -229,9 +252,10 @@ litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
       use = (nP - s + R - 1) / R + k / R2;
     }
   };
-  // the ring's items in order: (phase, unit, index within the unit's phase)
+  // the ring's items in order: (phase, unit, index within the unit's phase); a phase in which
+  // the units have no items (a sibling past the end of the tokens) is skipped whole
   auto advance = [&](int& u, int& j, bool& ph2) {
-    if (++j == (ph2 ? Q : P)) {
+    if (++j == (ph2 ? Q_(u) : P_(u))) {
       j = 0;
       if (++u == nu) {
         u = 0;
@@ -244,7 +268,7 @@ litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int u = 0, j = 0, issued = 0;
-      bool ph2 = P == 0;
+      bool ph2 = nP == 0;
       for (int i = 0; i < nitems; ++i) {
         int s, use;
         slot(i, s, use);
@@ -253,7 +277,7 @@ litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
         const int b = u ? b1 : b0, q = u ? q1 : q0;
         if (!ph2) {
           const int kx = p.H * kD + q * (kRedHeads * kD), vx = 2 * p.H * kD + q * (kRedHeads * kD);
-          const int y = n0 + j * kRedTile;
+          const int y = N0(u) + j * kRedTile;
           mbar_arrive_expect_tx(&full[s], kRedStageBytes);
           tma_load_3d(st, &tmap_kv, &full[s], kx, y, b);
           tma_load_3d(st + kRedBoxBytes, &tmap_kv, &full[s], kx + 64, y, b);
@@ -264,7 +288,7 @@ litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
           mbar_arrive_expect_tx(&full[s], np * kQBoxBytes);
           for (int h = 0; h < np; ++h)
             tma_load_3d(st + h * kQBoxBytes, &tmap_q, &full[s], q * kApUnitHeads * kD + h * kApHeads * kD,
-                        (t0 + j) * kApTile, b);
+                        (T0(u) + j) * kApTile, b);
         }
         issued = i + 1;
         advance(u, j, ph2);
@@ -285,7 +309,7 @@ litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
       constexpr uint32_t idesc_ap = idesc_bf16_f32(128, kImageRows, false, false);
       const uint64_t ones_desc = smem_desc(smem_u32(ones), 128, 256, kSwizzleNone);
       int u = 0, j = 0, pn = 0;
-      bool ph2 = P == 0, stop = false;
+      bool ph2 = nP == 0, stop = false;
       for (int i = 0; i < nitems && !stop; ++i) {
         int s, use;
         slot(i, s, use);
@@ -304,7 +328,7 @@ litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
             umma_bf16(dacc + 128, a, ones_desc, idesc_den, acc);
           }
           umma_commit(&empty[s]);
-          if (j == P - 1) umma_commit(&done[u]);
+          if (j == P_(u) - 1) umma_commit(&done[u]);
         } else {
           const int q = u ? q1 : q0;
           const uint32_t saddr = smem_u32(u ? sbuf1 : sbuf);
@@ -346,7 +370,7 @@ litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
     // ------------------------------------------------------------------ ReLU of every stage
     const int t = threadIdx.x - 64;   // 0..127
     int u = 0, j = 0;
-    bool ph2 = P == 0;
+    bool ph2 = nP == 0;
     for (int i = 0; i < nitems; ++i) {
       int s, use;
       slot(i, s, use);
@@ -354,7 +378,7 @@ litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
       uint8_t* st = ring + s * kStageBytes;
       if (!ph2) {
         // k boxes in place; rows of tokens past the chunk are zeroed in k and v
-        const int valid = min(kRedTile, n1 - (n0 + j * kRedTile));
+        const int valid = min(kRedTile, N1(u) - (N0(u) + j * kRedTile));
 #pragma unroll 4
         for (int c = t; c < 1024; c += 128) {
           uint4* w = reinterpret_cast<uint4*>(st + c * 16);
@@ -395,10 +419,17 @@ litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
     }
     bool ok = true;
     if (nu == 1 && leader) mbar_arrive(acc1_free);   // no second accumulator
+    // the running sums (block-causal: unit 1 continues unit 0's prefix)
+    float sum[kUPT][8];
+#pragma unroll
+    for (int m = 0; m < kUPT; ++m)
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sum[m][k] = 0.f;
     for (int u = 0; u < nu; ++u) {
       const int c = u ? c1 : c0, b = u ? b1 : b0, q = u ? q1 : q0;
+      const int blk = u ? blk1 : blk0;   // block-causal
       // (1) accumulator u -> this sibling's partial of quad c
-      bool got = ok && P > 0;
+      bool got = ok && P_(u) > 0;
       if (got) got = mbar_wait_long(&done[u], 0, abort_flag, err, kErrPairMerge | u);
       got = __all_sync(0xffffffffu, got);
       float sv[kRows];
@@ -417,10 +448,12 @@ litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
         for (int k = 0; k < kRows; ++k) sv[k] = 0.f;
       }
       tc_fence_before_sync();
-      float* dst = partials + ((int64_t)c * S + r) * kPartFloats + hq * kStateFloats;
+      // non-causal: partial r of quad c, [nq][S]; block-causal: the state of block blk, [nq][nblk]
+      float* dst = partials + ((int64_t)c * (kCausal ? p.nblk : S) + (kCausal ? blk : r)) * kPartFloats +
+                   hq * kStateFloats;
 #pragma unroll
       for (int k = 0; k < kRows; ++k) dst[k * kD + lane] = sv[k];
-      if (bar_any(3, 128, ok && P > 0 && !got)) ok = false;
+      if (bar_any(3, 128, ok && P_(u) > 0 && !got)) ok = false;
       if (leader) {
         if (u == 1) mbar_arrive(acc1_free);
         // the arrival: the barrier orders the group's partial writes before the leader's fence,
@@ -428,35 +461,43 @@ litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
         // the streaming load a fence waits several microseconds for the stores to land)
         if (ok) {
           __threadfence();
-          atomicAdd(&counters[c], 1u);
+          if (kCausal) atomicExch(&counters[c * p.nblk + blk], 1u);   // the block's flag
+          else atomicAdd(&counters[c], 1u);
         }
       }
-      // (2) wait for the quad's siblings
+      // (2) wait for what this unit sums: non-causal, all S partials of quad c; block-causal,
+      // the states of blocks [k0, k1) (unit 0: 0..r; unit 1: r + 1..r + S)
+      const int k0 = kCausal && u ? r + 1 : 0;
+      const int k1 = kCausal ? (u ? r + S + 1 : r + 1) : S;
       if (leader && ok) {
         const uint64_t tstart = globaltimer_ns();
-        volatile unsigned* arr = counters + c;
-        while (*arr < (unsigned)S) {
-          if (*abort_flag) { ok = false; break; }
-          if (globaltimer_ns() - tstart > kWaitLimitNs) {
-            *abort_flag = 1;
-            atomicCAS(err, 0, kErrPairSibling | u);
-            ok = false;
-            break;
+        for (int w = (kCausal ? k0 : 0); ok && w < (kCausal ? k1 : 1); ++w) {
+          volatile unsigned* arr = counters + (kCausal ? c * p.nblk + w : c);
+          while (kCausal ? *arr == 0u : *arr < (unsigned)S) {
+            if (*abort_flag) { ok = false; break; }
+            if (globaltimer_ns() - tstart > kWaitLimitNs) {
+              *abort_flag = 1;
+              atomicCAS(err, 0, kErrPairSibling | u);
+              ok = false;
+              break;
+            }
+            __nanosleep(256);
           }
-          __nanosleep(256);
         }
         __threadfence();   // acquire: the siblings' partial writes precede their arrivals
       }
       if (bar_any(3, 128, !ok)) ok = false;
       if (!ok) break;
-      // (3) the sum of the S partials in fixed order
-      float sum[kUPT][8];
+      // (3) the sum in fixed order: non-causal, partials 0..S-1; block-causal, block states
+      // k0..k1-1 added to the running prefix
+      if (!kCausal && u == 1) {
 #pragma unroll
-      for (int m = 0; m < kUPT; ++m)
+        for (int m = 0; m < kUPT; ++m)
 #pragma unroll
-        for (int k = 0; k < 8; ++k) sum[m][k] = 0.f;
-      const float* src = partials + (int64_t)c * S * kPartFloats;
-      for (int k = 0; k < S; ++k, src += kPartFloats) {
+          for (int k = 0; k < 8; ++k) sum[m][k] = 0.f;
+      }
+      const float* src = partials + ((int64_t)c * (kCausal ? p.nblk : S) + k0) * kPartFloats;
+      for (int k = k0; k < k1; ++k, src += kPartFloats) {
         float4 x[kUPT][2];
 #pragma unroll
         for (int m = 0; m < kUPT; ++m)
@@ -481,7 +522,7 @@ litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
         const int un = et + m * 128;
         if (un >= kUnits) break;
         const int hl = un / (kRows * 4), rcc = un - hl * (kRows * 4), rr = rcc >> 2, cc = rcc & 3;
-        if (Q > 0) {
+        if (Q_(u) > 0) {
           float hi[8], lo[8];
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
@@ -493,14 +534,15 @@ litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
           *reinterpret_cast<uint4*>(img + image_offset(rr, cc * 8)) = pack_bf16x8(hi);
           *reinterpret_cast<uint4*>(img + image_offset(kImageLoRow + rr, cc * 8)) = pack_bf16x8(lo);
         }
-        if (p.states != nullptr && r == 0 && hl < heads) {
-          float4* d4 = reinterpret_cast<float4*>(p.states + ((int64_t)b * p.H + q * kApUnitHeads + hl) * kStateFloats +
-                                                 rr * kD + cc * 8);
+        if (p.states != nullptr && (kCausal || r == 0) && hl < heads) {
+          // the states the queries use, [B][H][nblk][33][32] (non-causal: nblk = 1)
+          const int64_t st = ((int64_t)b * p.H + q * kApUnitHeads + hl) * (kCausal ? p.nblk : 1) + (kCausal ? blk : 0);
+          float4* d4 = reinterpret_cast<float4*>(p.states + st * kStateFloats + rr * kD + cc * 8);
           d4[0] = make_float4(sum[m][0], sum[m][1], sum[m][2], sum[m][3]);
           d4[1] = make_float4(sum[m][4], sum[m][5], sum[m][6], sum[m][7]);
         }
       }
-      if (Q > 0)
+      if (Q_(u) > 0)
         for (int i = et; i < kRedHeads * 14 * 4; i += 128) {   // zero rows 33..39, 73..79
           const int hl = i / 56, k = i - hl * 56, zr = k >> 2, cc = k & 3;
           const int nrow = zr < 7 ? kRows + zr : kImageLoRow + kRows + (zr - 7);
@@ -526,8 +568,8 @@ litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
     for (int u = 0; ok && u < nu; ++u) {
       const int b = u ? b1 : b0, q = u ? q1 : q0;
       const int np = pair_heads_h(p.H, q, 1) > 0 ? 2 : 1;
-      for (int lu = 0; ok && lu < Q; ++lu) {
-        const int tok0 = (t0 + lu) * kApTile;   // the last tile is clipped to N by the TMA store
+      for (int lu = 0; ok && lu < Q_(u); ++lu) {
+        const int tok0 = (T0(u) + lu) * kApTile;   // the last tile is clipped to N by the TMA store
         for (int h = 0; h < np; ++h) {
           const int nh = pair_heads_h(p.H, q, h);
           const int a = pn % kApAccSlots;

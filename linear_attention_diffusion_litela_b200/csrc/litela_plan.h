@@ -154,6 +154,21 @@ inline bool make_plan(int B, int N, int H, int tokens_per_block, int num_sms, Pl
       p->fused_bytes = p->fused_off_totals + align_up((size_t)B * p->nquads * cpb * part, 256);
       p->counters = (size_t)B * p->nquads * cpb + 2;   // an arrival flag per CTA; finish, ticket
     }
+    // paired block-causal form, where the plain form gives each CTA two consecutive blocks: the
+    // same CTAs, but sibling r of quad c owns its blocks r and r + S (S = ceil(nblk / 2)), so that
+    // block r's prefix is merged while the CTA reduces block r + S; workspace = block states
+    // [B * nquads][nblk][4][33][32]; control words: a flag per (quad, block), the finish and
+    // ticket counters
+    const int64_t nq = (int64_t)B * p->nquads, S = (p->nblk + 1) / 2;
+    if (bpc == 2 && p->T >= paired_min_chunk) {
+      const size_t part = (size_t)kRedHeads * kStateFloats * sizeof(float);
+      p->fused = p->fused_causal = p->fused_paired = true;
+      p->fused_ntiles = (N + kApTile - 1) / kApTile;
+      p->paired_cpb = (int)S;
+      p->paired_chunk = p->T;
+      p->paired_bytes = align_up((size_t)nq * p->nblk * part, 256);
+      p->counters = (size_t)nq * p->nblk + 2;
+    }
   }
   return true;
 }

@@ -238,7 +238,9 @@ def test_forward_form_and_the_paired_minimum(lib):
     assert lib.lite_la_forward_form(1, 16, 1, 64, 0) == -1
     assert ll.lite_la_forward_form(2, 16384, 70) == "fused_paired"       # chunks of 2048 tokens
     assert ll.lite_la_forward_form(2, 4096, 70) == "fused"               # chunks of 512
-    assert ll.lite_la_forward_form(1, 16384, 70, 32, 1024) == "fused_causal"
+    assert ll.lite_la_forward_form(1, 16384, 70, 32, 1024) == "fused_paired_causal"   # 18 quads x 8 block pairs
+    assert ll.lite_la_forward_form(2, 16384, 70, 32, 1024) == "three_kernel"          # 36 x 8 > 148, 4 blocks a CTA
+    assert ll.lite_la_forward_form(1, 4096, 70, 32, 512) == "fused_causal"            # blocks < 1024 tokens
     assert ll.lite_la_forward_form(8, 512, 80) == "three_kernel"         # 160 head quads
     prev = ll.lite_la_set_paired_min_chunk(512)
     try:

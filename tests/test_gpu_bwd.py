@@ -230,15 +230,15 @@ def test_zz_report_worst_errors():
 
 
 @pytest.mark.parametrize("B,N,H,T,min_chunk", [(2, 1500, 9, 0, 0), (1, 700, 600, 0, 0), (1, 2000, 5, 256, 0),
-                                               (2, 300, 3, 1, 0), (2, 2100, 7, 0, 64)])
+                                               (2, 300, 3, 1, 0), (2, 2100, 7, 0, 64), (1, 1300, 60, 128, 64)])
 def test_forward_saves_the_state_and_the_backward_uses_it(B, N, H, T, min_chunk, paired_min_chunk):
     """lite_la_fwd_save_state: bitwise the plain forward's output, states equal to their
     definition; lite_la_bwd_from_state: the backward within tolerance of the oracle.  The last
-    case takes the paired fused form, which writes the states from its merge warps."""
+    two cases take the paired fused forms, which write the states from their merge warps."""
     from tests.test_gpu_parity import state_reference
     if min_chunk:
         paired_min_chunk(min_chunk)
-        assert ll.lite_la_forward_form(B, N, H) == "fused_paired"
+        assert ll.lite_la_forward_form(B, N, H, D, T) == ("fused_paired_causal" if T else "fused_paired")
     qkv = make_qkv(B, N, H, D, seed=7950 + N + H + T, device="cuda")
     dout = make_dout(B, N, H, seed=7951 + N)
     out, states = ll.lite_la_fwd_save_state(qkv, H, tokens_per_block=T, eps=EPS)

@@ -93,6 +93,22 @@ def test_paired_fused_shapes_every_element(B, N, H, mode, paired_min_chunk):
     assert_close(gpu_run(qkv, H, mode=mode), oracle_run(qkv, H), mode)
 
 
+PAIRED_CAUSAL = [  # the paired block-causal form (sibling r owns blocks r and r + ceil(nblk/2) of a
+                   # quad; taken where the plain form gives a CTA two blocks): an odd block count
+                   # (the last sibling has one block), a ragged last block, quads of 2 heads
+    (1, 2048, 40, 128), (1, 2100, 40, 128), (3, 1024, 30, 128), (2, 700, 70, 128), (2, 640, 66, 128),
+]
+
+
+@pytest.mark.parametrize("mode", ["bf16", "f32"])
+@pytest.mark.parametrize("B,N,H,T", PAIRED_CAUSAL)
+def test_paired_block_causal_shapes_every_element(B, N, H, T, mode, paired_min_chunk):
+    paired_min_chunk(128)
+    assert ll.lite_la_forward_form(B, N, H, 32, T) == "fused_paired_causal"
+    qkv = make_qkv(B, N, H, 32, seed=B * 31337 + N + H * 7 + T, device="cuda")
+    assert_close(gpu_run(qkv, H, T=T, mode=mode), oracle_run(qkv, H, T=T), mode)
+
+
 def test_paired_and_plain_fused_forms_agree_and_are_deterministic(paired_min_chunk):
     """Both fused forms of the 2048px call: each bitwise repeatable, the two within the bf16
     rounding of each other (their fp32 partial states are summed over different chunks)."""
@@ -159,6 +175,7 @@ def test_4096px_sampled(mode):
 def test_block_causal_workload_sampled(mode):
     w = WORKLOADS["block_causal_16x1024"]
     T = w["tokens_per_block"]
+    assert ll.lite_la_forward_form(w["B"], w["N"], w["H"], 32, T) == "fused_paired_causal"
     qkv = make_qkv(w["B"], w["N"], w["H"], 32, seed=1004, device="cuda")
     rows = sample_rows(w["N"], T=T, k=64, seed=5)
     got = gpu_run(qkv, w["H"], T=T, mode=mode)[:, rows]
