@@ -419,12 +419,18 @@ def test_phase_timed_calls_give_the_plain_calls_result(B, N, H, T):
     assert lib.lite_la_fwd_events(qkv.data_ptr(), out.data_ptr(), B, N, H, 32, EPS, sh, null) == 1
 
 
-@pytest.mark.parametrize("T", [0, 1024])
-def test_concurrent_fused_calls_on_two_streams(T):
+# one shape per fused form: paired, plain, paired block-causal, plain block-causal
+FUSED_FORMS = [((2, 8192, 70, 0), "fused_paired"), ((2, 4096, 70, 0), "fused"),
+               ((1, 16384, 70, 1024), "fused_paired_causal"), ((1, 8192, 70, 1024), "fused_causal")]
+
+
+@pytest.mark.parametrize("shape,form", FUSED_FORMS)
+def test_concurrent_fused_calls_on_two_streams(shape, form):
     """Two fused calls at once on two streams: each grid alone fills the SMs, so only part of
     each can be resident; CTAs take their roles by ticket in arrival order, so both complete.
     The results equal the single-stream ones bitwise and no wait times out."""
-    B, N, H = (2, 8192, 70) if T == 0 else (1, 16384, 70)
+    B, N, H, T = shape
+    assert ll.lite_la_forward_form(B, N, H, 32, T) == form
     xa = make_qkv(B, N, H, 32, seed=6100 + T, device="cuda")
     xb = make_qkv(B, N, H, 32, seed=6200 + T, device="cuda")
     run = (lambda x, **kw: ll.lite_la_fwd(x, H, eps=EPS, **kw)) if T == 0 else \
@@ -444,12 +450,13 @@ def test_concurrent_fused_calls_on_two_streams(T):
         assert torch.equal(oa, ra) and torch.equal(ob, rb)
 
 
-@pytest.mark.parametrize("T", [0, 1024])
-def test_fused_call_replayed_from_a_captured_graph(T):
+@pytest.mark.parametrize("shape,form", FUSED_FORMS)
+def test_fused_call_replayed_from_a_captured_graph(shape, form):
     """One fused call captured into a CUDA graph and replayed several times, interleaved with
     eager calls on the same stream: the kernel's control words are left clean by the last CTA
     of every call, so each replay and each eager call gives the eager result bitwise."""
-    B, N, H = (2, 8192, 70) if T == 0 else (1, 16384, 70)
+    B, N, H, T = shape
+    assert ll.lite_la_forward_form(B, N, H, 32, T) == form
     x = make_qkv(B, N, H, 32, seed=6300 + T, device="cuda")
     run = (lambda **kw: ll.lite_la_fwd(x, H, eps=EPS, **kw)) if T == 0 else \
         (lambda **kw: ll.lite_la_block_causal_fwd(x, H, T, eps=EPS, **kw))
