@@ -66,10 +66,15 @@ struct FusedCfg {
   static constexpr int kMapWarps1 = kMap ? 8 : 4;
   static constexpr int kMapWarps2 = kMap ? 8 : 2;
   static constexpr int kEpiWarp0 = 2 + kMapWarps2;
-  static constexpr int kThreads = 32 * (kEpiWarp0 + 4);
+  // apply epilogue: groups of 4 warps, group g taking head pair g of every tile.  Two groups
+  // measured faster for the non-causal form (2048px 36.9 -> 36.1 us, 1024px 16.9 -> 16.5 us,
+  // 512px 10.7 -> 10.5 us) and slightly slower for the block-causal one (39.1 -> 39.3 us at
+  // N = 8192, T = 1024); the ELU + 1 form's feature-map warps leave no registers for a second
+  static constexpr int kEpiGroups = (kMap || kCausal) ? 1 : 2;
+  static constexpr int kThreads = 32 * (kEpiWarp0 + 4 * kEpiGroups);
   // launch bound: with 448 threads it keeps ptxas at 128 registers (4 warps share an SM
-  // sub-partition's 16K registers)
-  static constexpr int kLaunchBound = kMap ? 512 : 256;
+  // sub-partition's 16K registers); with 384, at 168
+  static constexpr int kLaunchBound = kMap ? 512 : (kEpiGroups == 2 ? 384 : 256);
   // phase-1 stage: k | v boxes; for ELU + 1 also a box of ones right after v (so that one
   // N = 144 product gives the numerator and the denominator: the tensor core pays per
   // instruction, and phi's hi + lo halves would otherwise double four products per 16 tokens)
@@ -501,13 +506,15 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
       fence_proxy_async_smem();
       mbar_arrive(&qrelu[s]);
     }
-  } else if (warp < kEpiWarp0 + 4) {
-    const int et = threadIdx.x - 32 * kEpiWarp0;   // 0..127
+  } else {
+    const int egrp = (warp - kEpiWarp0) >> 2;       // epilogue group (group 0 also merges)
+    const int et = threadIdx.x - 32 * (kEpiWarp0 + 4 * egrp);   // 0..127
     const bool leader = (et == 0);
+    bool ok = true;
+    if (egrp == 0) {
     // ---- merge: wait for the siblings, sum their partials in fixed order, build the B operand.
     // Non-causal: all cpb siblings' partials, then one image.  Block-causal: the totals of
     // siblings 0..r-1, then this CTA's block states one by one, an image after each.
-    bool ok = true;
     if (leader) {
       const uint64_t tstart = globaltimer_ns();
       for (int w = 0; ok && w < (kCausal ? r : 1); ++w) {
@@ -605,23 +612,28 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
     if (ok) fence_proxy_async_smem();
     bar_sync(2, 128);
     if (leader && ok) mbar_arrive(sfull);
-    // ---- epilogue (as litela_apply_tc; the merge buffer overlapped the output staging region)
+    }
+    // ---- epilogue (as litela_apply_tc; the merge buffer overlapped the output staging region,
+    // which group 1 first writes after the apply's first result, i.e. after the merge).  With two
+    // groups, group g takes head pair g of every tile and stores that pair's boxes itself.
     const int hq = warp & 3;
     const int row = hq * 32 + lane;
-    int nstaged = 0, pn = 0;
-    for (int lu = 0; ok && lu < nunits; ++lu) {
+    const int bar_a = 1 + 2 * egrp, bar_b = 2 + 2 * egrp;   // the group's named barriers
+    const int npairs = pair_heads_h(p.H, q, 1) > 0 ? 2 : 1;
+    constexpr int kBoxesPerPair = A::kOutBoxes / 2;
+    for (int lu = 0; ok && lu < nunits && (Cfg::kEpiGroups == 1 || egrp < npairs); ++lu) {
       const int tok0 = (t0 + lu) * kApTile;   // the last tile is clipped to N by the TMA store
-      uint8_t* slot = obuf + (nstaged % A::kOutSlots) * A::kOutSlotBytes;
+      uint8_t* slot = obuf + (lu % A::kOutSlots) * A::kOutSlotBytes;
       if (leader) bulk_wait_group_read<A::kOutSlots - 1>();
-      bar_sync(2, 128);
-      ++nstaged;
+      bar_sync(bar_b, 128);
       bool stop = false;
-      for (int h = 0; h < 2; ++h) {
+      for (int h = (Cfg::kEpiGroups == 1 ? 0 : egrp); h < 2; h += Cfg::kEpiGroups) {
         const int nh = pair_heads_h(p.H, q, h);
         if (nh == 0) break;
+        const int pn = lu * npairs + h;   // the MMAs' running pair count
         const int a = pn % kApAccSlots;
         const bool okw = mbar_wait(&tfull[a], (pn / kApAccSlots) & 1, abort_flag, err, kErrApplyEpi | a);
-        if (bar_any(1, 128, !okw)) {
+        if (bar_any(bar_a, 128, !okw)) {
           stop = true;
           break;
         }
@@ -654,15 +666,16 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
             *reinterpret_cast<uint4*>(box + row * 128 + (((ck & 7) ^ (row & 7)) << 4)) = w[k];
           }
         }
-        ++pn;
       }
       if (stop) break;
       fence_proxy_async_smem();
-      bar_sync(2, 128);
+      bar_sync(bar_b, 128);
       if (leader) {
         const int x0 = q * kApUnitHeads * kD;
-#pragma unroll
-        for (int bx = 0; bx < A::kOutBoxes; ++bx)
+        // one group: every box of the tile; two: the boxes of the group's pair
+        const int bx0 = Cfg::kEpiGroups == 1 ? 0 : egrp * kBoxesPerPair;
+        const int bx1 = Cfg::kEpiGroups == 1 ? A::kOutBoxes : bx0 + kBoxesPerPair;
+        for (int bx = bx0; bx < bx1; ++bx)
           if (x0 + bx * A::kBoxChannels < p.H * kD)
             tma_store_3d(&tmap_out, slot + bx * kOutBoxBytes, x0 + bx * A::kBoxChannels, tok0, b);
         bulk_commit_group();
