@@ -507,7 +507,8 @@ litela_fused_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_consta
       mbar_arrive(&qrelu[s]);
     }
   } else {
-    const int egrp = (warp - kEpiWarp0) >> 2;       // epilogue group (group 0 also merges)
+    // epilogue group (group 0 also merges); a compile-time 0 with one group
+    const int egrp = Cfg::kEpiGroups == 1 ? 0 : (warp - kEpiWarp0) >> 2;
     const int et = threadIdx.x - 32 * (kEpiWarp0 + 4 * egrp);   // 0..127
     const bool leader = (et == 0);
     bool ok = true;
