@@ -234,8 +234,9 @@ litela_status lite_la_release_workspace(void);
 size_t lite_la_workspace_bytes(int B, int N, int H, int d, int tokens_per_block);
 
 /* Number of kernels one forward call with these arguments launches on the current device: 1
- * when it takes the fused single kernel (B * ceil(H/4) <= SM count; block-causal calls also need
- * a block size that is a multiple of 128 tokens and at most two blocks per CTA), 3 otherwise
+ * when it takes a fused single kernel, plain or paired (B * ceil(H/4) <= SM count; block-causal
+ * calls also need a block size that is a multiple of 128 tokens and at most two blocks per CTA;
+ * lite_la_forward_form says which), 3 otherwise
  * (state reduction, prefix scan, apply); 0 for an empty or invalid problem.  The streaming-carry
  * form always takes the three-kernel path, and so does the ELU+1 variant's block-causal form (its
  * non-causal form takes the fused kernel under the same condition as LiteLA's). */
@@ -262,11 +263,11 @@ int lite_la_kernels_per_call(int B, int N, int H, int d, int tokens_per_block);
 int lite_la_forward_form(int B, int N, int H, int d, int tokens_per_block);
 
 /* Sets the chunk length (tokens per sibling CTA and head quad; the block size for block-causal
- * calls) from which LiteLA calls take a paired fused form, for every device and thread of the process; tokens <= 0 restores
- * the default, 1024 (measured on B200: with shorter chunks one quad's state reduction is too
- * short to hide the other's merge, and the plain fused form is faster).  Returns the previous
- * value.  Calls already enqueued are not affected; the result of a call does not depend on the
- * form up to the order of its fp32 partial-state sums. */
+ * calls) from which LiteLA calls take a paired fused form, for every device and thread of the
+ * process; tokens <= 0 restores the default, 1024 (measured on B200: with shorter chunks one
+ * quad's state reduction is too short to hide the other's merge, and the plain fused form is
+ * faster).  Returns the previous value.  Calls already enqueued are not affected; the result of
+ * a call does not depend on the form up to the order of its fp32 partial-state sums. */
 int lite_la_set_paired_min_chunk(int tokens);
 
 /* ---- LiteLA with the output projection fused ---------------------------------------------
