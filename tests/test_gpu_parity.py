@@ -501,3 +501,50 @@ def test_head_shards_of_one_problem_match_the_full_call():
         sub = pack_head_shard(qkv, H, h0, h1)
         got = gpu_run(sub, h1 - h0)
         assert_close(got, want[:, :, h0:h1], "bf16")
+
+
+@pytest.mark.parametrize("shape,form", FUSED_FORMS + [((2, 300, 600, 0), "three_kernel")])
+def test_input_rewritten_by_the_previous_kernel_is_the_one_read(shape, form):
+    """Every fused form prefetches its CTA's first input tiles into L2 before it waits for the
+    previous kernel in the stream (programmatic dependent launch).  Here that previous kernel
+    rewrites the very qkv buffer in place; the call must see the new values, bitwise as a call
+    on a fresh buffer, in both directions of the rewrite and back to back."""
+    B, N, H, T = shape
+    assert ll.lite_la_forward_form(B, N, H, 32, T) == form
+    xa = make_qkv(B, N, H, 32, seed=7100 + N, device="cuda")
+    xb = make_qkv(B, N, H, 32, seed=7200 + N, device="cuda")
+    run = (lambda x: ll.lite_la_fwd(x, H, eps=EPS)) if T == 0 else \
+        (lambda x: ll.lite_la_block_causal_fwd(x, H, T, eps=EPS))
+    ra, rb = run(xa), run(xb)
+    torch.cuda.synchronize()
+    buf = xa.clone()
+    outs = []
+    for i in range(6):
+        outs.append(run(buf))
+        src = xb if i % 2 == 0 else xa
+        torch.mul(src, 1.0, out=buf)   # an elementwise kernel rewrites the input in place
+    torch.cuda.synchronize()
+    ll.lite_la_device_status()
+    for i, o in enumerate(outs):
+        assert torch.equal(o, ra if i % 2 == 0 else rb), i
+
+
+def test_backward_input_rewritten_by_the_previous_kernel_is_the_one_read():
+    """The backward's state reduction prefetches k and v before its dependency wait: a qkv
+    rewritten in place by the kernel just before must be the one the backward reads."""
+    B, N, H = 2, 2048, 70
+    xa = make_qkv(B, N, H, 32, seed=7300, device="cuda")
+    xb = make_qkv(B, N, H, 32, seed=7301, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(7302)
+    dout = torch.randn((B, N, H * 32), generator=g, device="cuda").to(torch.bfloat16)
+    ra, rb = ll.lite_la_bwd(xa, dout, H, eps=EPS), ll.lite_la_bwd(xb, dout, H, eps=EPS)
+    torch.cuda.synchronize()
+    buf = xa.clone()
+    outs = []
+    for i in range(4):
+        outs.append(ll.lite_la_bwd(buf, dout, H, eps=EPS))
+        torch.mul(xb if i % 2 == 0 else xa, 1.0, out=buf)
+    torch.cuda.synchronize()
+    ll.lite_la_device_status()
+    for i, o in enumerate(outs):
+        assert torch.equal(o, ra if i % 2 == 0 else rb), i
