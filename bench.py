@@ -439,7 +439,7 @@ def l2_note(B, N, H, calls, direction="fwd"):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)   # 50 x 60 calls: ~0.33 s timed at 4096px
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=list(WORKLOADS_BENCH), default="sana4800m_4096px_x60")
