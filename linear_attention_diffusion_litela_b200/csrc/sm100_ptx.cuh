@@ -1,6 +1,6 @@
 // Thin inline-PTX layer for sm_100a: mbarriers with bounded waits, TMA tile loads and bulk
-// copies (no cluster multicast anywhere), tcgen05 tensor-memory allocation, MMA, commit and
-// loads.  Everything here is written from the PTX ISA's instruction descriptions.
+// copies (each into the issuing CTA's own shared memory only), tcgen05 tensor-memory allocation,
+// MMA, commit and loads.  Everything here is written from the PTX ISA's instruction descriptions.
 #pragma once
 
 #include <cuda.h>
@@ -150,7 +150,7 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
 
 // ---------------------------------------------------------------------------------------
 // TMA (tensor tile) loads and plain bulk copies, global -> shared, completing on an mbarrier.
-// The destination operand is this CTA's own shared memory; no multicast is used.
+// The destination operand is this CTA's own shared memory, and no other CTA's.
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
