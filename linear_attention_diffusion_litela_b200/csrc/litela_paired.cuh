@@ -267,6 +267,9 @@ litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      // every input byte is read once: its L2 lines go first, ahead of the outputs still being
+      // written back and of the next call's prefetched tiles
+      const uint64_t pol = l2_policy_evict_first();
       int u = 0, j = 0, issued = 0;
       bool ph2 = nP == 0;
       for (int i = 0; i < nitems; ++i) {
@@ -279,16 +282,16 @@ litela_paired_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
           const int kx = p.H * kD + q * (kRedHeads * kD), vx = 2 * p.H * kD + q * (kRedHeads * kD);
           const int y = N0(u) + j * kRedTile;
           mbar_arrive_expect_tx(&full[s], kRedStageBytes);
-          tma_load_3d(st, &tmap_kv, &full[s], kx, y, b);
-          tma_load_3d(st + kRedBoxBytes, &tmap_kv, &full[s], kx + 64, y, b);
-          tma_load_3d(st + 2 * kRedBoxBytes, &tmap_kv, &full[s], vx, y, b);
-          tma_load_3d(st + 3 * kRedBoxBytes, &tmap_kv, &full[s], vx + 64, y, b);
+          tma_load_3d(st, &tmap_kv, &full[s], kx, y, b, pol);
+          tma_load_3d(st + kRedBoxBytes, &tmap_kv, &full[s], kx + 64, y, b, pol);
+          tma_load_3d(st + 2 * kRedBoxBytes, &tmap_kv, &full[s], vx, y, b, pol);
+          tma_load_3d(st + 3 * kRedBoxBytes, &tmap_kv, &full[s], vx + 64, y, b, pol);
         } else {
           const int np = pair_heads_h(p.H, q, 1) > 0 ? 2 : 1;
           mbar_arrive_expect_tx(&full[s], np * kQBoxBytes);
           for (int h = 0; h < np; ++h)
             tma_load_3d(st + h * kQBoxBytes, &tmap_q, &full[s], q * kApUnitHeads * kD + h * kApHeads * kD,
-                        (T0(u) + j) * kApTile, b);
+                        (T0(u) + j) * kApTile, b, pol);
         }
         issued = i + 1;
         advance(u, j, ph2);
