@@ -230,6 +230,15 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
 
   if (warp == 0) {
     if (lane == 0) {
+      // k and v are read once: with the ReLU map their L2 lines go first (measured faster for
+      // the three-kernel forward; the ELU + 1 map keeps the default policy)
+      const uint64_t pol = l2_policy_evict_first();
+      auto load = [&](void* dst, uint64_t* bar, int x, int y) {
+        if (kMap == 0)
+          tma_load_3d(dst, &tmap, bar, x, y, b, pol);
+        else
+          tma_load_3d(dst, &tmap, bar, x, y, b);
+      };
       int issued = 0;
       for (int i = 0; i < ntiles; ++i) {
         const int s = i % kStages;
@@ -239,10 +248,10 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
         uint8_t* st = stages + s * kStageBytes;
         const int y = n0 + i * kRedTile;
         mbar_arrive_expect_tx(&full[s], kRedStageBytes);
-        tma_load_3d(st, &tmap, &full[s], kx, y, b);
-        tma_load_3d(st + kRedBoxBytes, &tmap, &full[s], kx + 64, y, b);
-        tma_load_3d(st + 2 * kRedBoxBytes, &tmap, &full[s], vx, y, b);
-        tma_load_3d(st + 3 * kRedBoxBytes, &tmap, &full[s], vx + 64, y, b);
+        load(st, &full[s], kx, y);
+        load(st + kRedBoxBytes, &full[s], kx + 64, y);
+        load(st + 2 * kRedBoxBytes, &full[s], vx, y);
+        load(st + 3 * kRedBoxBytes, &full[s], vx + 64, y);
         issued = i + 1;
       }
       if (*abort_flag) {   // let the copies still in flight land before the CTA exits (bounded)
