@@ -189,11 +189,12 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
 }
 
 // L2 prefetch of a tile (no shared-memory destination, no completion): a hint that changes no
-// memory contents, so it may be issued before the programmatic-launch wait
+// memory contents, so it may be issued before the programmatic-launch wait.  The tiles are
+// inputs that the kernel reads once: their lines are marked evict-first.
 __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int c0, int c1, int c2) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile.L2::cache_hint [%0, {%1, %2, %3}], %4;" ::"l"(
                    reinterpret_cast<uint64_t>(map)),
-               "r"(c0), "r"(c1), "r"(c2)
+               "r"(c0), "r"(c1), "r"(c2), "l"(l2_policy_evict_first())
                : "memory");
 }
 
