@@ -69,6 +69,10 @@ PATHS = {
     5: {"phases": ("litela_reduce_tc+litela_state_scan", "litela_bwd_q_tc", "litela_state_scan+litela_bwd_kv_tc"),
         "alg_bytes_E": {"litela_reduce_tc+litela_state_scan": 4, "litela_bwd_q_tc": 6,
                         "litela_state_scan+litela_bwd_kv_tc": 8}},
+    # the backward with one block per sequence (lite_la_bwd_kernels_per_call == 3): the dq and
+    # dk/dv kernels sum the partial states into their images themselves, no scan launches
+    "bwd3": {"phases": ("litela_reduce_tc", "litela_bwd_q_tc", "litela_bwd_kv_tc"),
+             "alg_bytes_E": {"litela_reduce_tc": 4, "litela_bwd_q_tc": 6, "litela_bwd_kv_tc": 8}},
     1: {"phases": ("litela_fused_tc",), "alg_bytes_E": {"litela_fused_tc": 8}},
     # the fused kernel's paired form (lite_la_forward_form == LITELA_FORM_FUSED_PAIRED)
     "paired": {"phases": ("litela_paired_tc",), "alg_bytes_E": {"litela_paired_tc": 8}},
@@ -615,9 +619,15 @@ def main():
     ev_handles = [(ctypes.c_void_p * nev)(*[ctypes.c_void_p(e.cuda_event) for e in trip]) for trip in evs]
     # the ELU + 1 variant's block-causal form always takes the three-kernel path
     nk = 5 if bwd else (3 if args.variant == "elu1" and T else int(lib.lite_la_kernels_per_call(B, N, H, D, T)))
+    # kernels per timed call (the saved-state backward: its own count)
+    launches_per_call = (int(lib.lite_la_bwd_kernels_per_call(B, N, H, D, T, 1 if args.bwd_from_state else 0))
+                         if bwd else nk)
     # the ELU + 1 variant never takes the paired form
-    path = PATHS["paired"] if (nk == 1 and args.variant == "litela" and
-                               int(lib.lite_la_forward_form(B, N, H, D, T)) in FORMS_PAIRED) else PATHS[nk]
+    if bwd:   # the phases are timed on the recomputing backward
+        path = PATHS["bwd3"] if int(lib.lite_la_bwd_kernels_per_call(B, N, H, D, T, 0)) == 3 else PATHS[5]
+    else:
+        path = PATHS["paired"] if (nk == 1 and args.variant == "litela" and
+                                   int(lib.lite_la_forward_form(B, N, H, D, T)) in FORMS_PAIRED) else PATHS[nk]
     phases = path["phases"]
     kern_ms = {k: 0.0 for k in phases}
     nlaunch = 0
@@ -779,9 +789,9 @@ def main():
                 "roofline": roofline,
                 "call_roofline": call_roof,
                 "cpu_baseline": cpu, "e2e": e2e,
-                # kernels the timed calls launch: the saved-state backward runs the state images,
-                # the dq kernel, the reverse scan and the dk/dv kernel (4), not the 5 of `nk`
-                "gpu_launches": (4 if bwd and args.bwd_from_state else nk) * calls * args.steps,
+                # kernels the timed calls launch (lite_la_kernels_per_call,
+                # lite_la_bwd_kernels_per_call)
+                "gpu_launches": launches_per_call * calls * args.steps,
                 "clocks": clocks, "gpu": torch.cuda.get_device_name(dev)}
         if world > 1:
             line["config"]["parallelism"] = "dp%d (independent calls per rank, no collective)" % world

@@ -242,6 +242,14 @@ size_t lite_la_workspace_bytes(int B, int N, int H, int d, int tokens_per_block)
  * non-causal form takes the fused kernel under the same condition as LiteLA's). */
 int lite_la_kernels_per_call(int B, int N, int H, int d, int tokens_per_block);
 
+/* Number of kernels one backward call launches (lite_la_bwd, lite_la_block_causal_bwd when
+ * from_state is 0; lite_la_bwd_from_state when it is 1): 3 when the call has one block per
+ * sequence (non-causal, or tokens_per_block >= N): the state (the reduction, or the images of
+ * the saved states), dq, and dk/dv, the last two summing the partial states into their own
+ * images; otherwise 5 (reduction, prefix scan, dq, reverse scan, dk/dv), 4 from saved states.
+ * 0 for an empty or invalid problem. */
+int lite_la_bwd_kernels_per_call(int B, int N, int H, int d, int tokens_per_block, int from_state);
+
 /* Which form a LiteLA forward call (lite_la_fwd, lite_la_block_causal_fwd and their _f32out
  * forms) with these arguments takes on the current device: LITELA_FORM_THREE_KERNEL (state
  * reduction, prefix scan, apply), LITELA_FORM_FUSED (one kernel: a CTA reduces a chunk of one

@@ -54,6 +54,7 @@ _SIGNATURES = {
     "lite_la_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "lite_la_fwd_noalloc": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _vp]),
     "lite_la_kernels_per_call": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "lite_la_bwd_kernels_per_call": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int]),
     "lite_la_forward_form": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "lite_la_set_paired_min_chunk": (_c_int, [_c_int]),
     "lite_la_elu1_fwd": (_c_int, [_vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_float, _c_int, _vp]),

@@ -601,15 +601,21 @@ litela_status run_bwd(const void* qkv, const void* dout, OutT* dqkv, int B, int 
     if (s != LITELA_OK) return s;
   }
   const bool pdl = events == nullptr;
-  const BwdPlan bp{B, N, H, plan.T, plan.nblk, plan.nquads, plan.bwd_cpb, plan.bwd_chunk, eps};
+  // one block per quad: the dq and dk/dv kernels sum the partial states into their images
+  // themselves (in the scans' order), and the two scan launches are left out
+  const int fold_fwd = (plan.nblk == 1 && states_in == nullptr) ? tc_plan(plan, 0.f).cpb : 0;
+  const int fold_bwd = plan.nblk == 1 ? plan.bwd_cpb : 0;
+  const BwdPlan bp{B, N, H, plan.T, plan.nblk, plan.nquads, plan.bwd_cpb, plan.bwd_chunk, eps, fold_fwd, fold_bwd};
   const dim3 grid((unsigned)(plan.nblk * plan.bwd_cpb), (unsigned)plan.nquads, (unsigned)B);
   cudaError_t e;
   if (events && (e = cudaEventRecord(events[0], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   if (states_in == nullptr) {
     s = launch_reduce(plan, qkv, partials, ws->err, stream, pdl);
     if (s != LITELA_OK) return s;
-    s = launch_scan(plan, partials, images, nullptr, num_sms, stream, pdl, nullptr, nullptr, images_t, false);
-    if (s != LITELA_OK) return s;
+    if (fold_fwd == 0) {
+      s = launch_scan(plan, partials, images, nullptr, num_sms, stream, pdl, nullptr, nullptr, images_t, false);
+      if (s != LITELA_OK) return s;
+    }
   } else {
     const long long nst = (long long)B * H * plan.nblk;
     long long grid = (nst * kStateFloats + kScanThreads - 1) / kScanThreads;
@@ -620,16 +626,18 @@ litela_status run_bwd(const void* qkv, const void* dout, OutT* dqkv, int B, int 
   }
   if (events && (e = cudaEventRecord(events[1], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   e = launch_ex(litela_bwd_q_tc<OutT>, grid, dim3(kBwThreads), kBqSmemBytes, stream, pdl, map_qkv, map_g, map_dq,
-                static_cast<const uint8_t*>(images), static_cast<const uint8_t*>(images_t), dpartials, dqkv, ws->err,
-                bp);
+                static_cast<const uint8_t*>(images), static_cast<const uint8_t*>(images_t),
+                static_cast<const float*>(partials), dpartials, dqkv, ws->err, bp);
   if (e != cudaSuccess) return cuda_fail(e, "launch litela_bwd_q_tc");
   if (events && (e = cudaEventRecord(events[2], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-  s = launch_scan(plan, dpartials, dimages, nullptr, num_sms, stream, pdl, nullptr, nullptr, dimages_t, true,
-                  plan.bwd_cpb, true, dzrows);
-  if (s != LITELA_OK) return s;
+  if (fold_bwd == 0) {
+    s = launch_scan(plan, dpartials, dimages, nullptr, num_sms, stream, pdl, nullptr, nullptr, dimages_t, true,
+                    plan.bwd_cpb, true, dzrows);
+    if (s != LITELA_OK) return s;
+  }
   e = launch_ex(litela_bwd_kv_tc<OutT>, grid, dim3(kBwThreads), kBkSmemBytes, stream, pdl, map_qkv, map_dqkv,
                 static_cast<const uint8_t*>(dimages), static_cast<const uint8_t*>(dimages_t),
-                static_cast<const float*>(dzrows), dqkv, ws->err, bp);
+                static_cast<const float*>(dzrows), static_cast<const float*>(dpartials), dqkv, ws->err, bp);
   if (e != cudaSuccess) return cuda_fail(e, "launch litela_bwd_kv_tc");
   if (events && (e = cudaEventRecord(events[3], stream)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
   g_last_error.clear();
@@ -978,6 +986,15 @@ int lite_la_kernels_per_call(int B, int N, int H, int d, int tokens_per_block) {
   litela::Plan p;
   litela::make_plan(B, N, H, tokens_per_block, sms, &p, litela::g_paired_min_chunk.load());
   return p.fused ? 1 : 3;
+}
+
+int lite_la_bwd_kernels_per_call(int B, int N, int H, int d, int tokens_per_block, int from_state) {
+  if (B <= 0 || N <= 0 || H <= 0 || d != litela::kD) return 0;
+  const bool one_block = tokens_per_block <= 0 || tokens_per_block >= N;
+  // the state (reduction, or the saved states' images) + its scan + dq + the reverse scan + dk/dv;
+  // with one block per quad the dq and dk/dv kernels do the scans themselves
+  if (one_block) return 3;
+  return from_state ? 4 : 5;
 }
 
 litela_status lite_la_selftest_timeout(cudaStream_t stream) {

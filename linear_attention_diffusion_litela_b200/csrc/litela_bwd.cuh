@@ -15,7 +15,9 @@
 //   dv    = dS[0:d] k~
 // relu'(0) = 0, as in PyTorch's ReLU backward.
 //
-// A call runs five kernels chained with programmatic dependent launch:
+// A call runs five kernels chained with programmatic dependent launch (three with one block per
+// sequence: the dq and dk/dv kernels then sum the partial states into their images themselves,
+// in the scans' order, and the two scans are not launched):
 //   litela_reduce_tc, litela_state_scan   S (as in the forward) as B-operand images: S (rows r)
 //                                         and S[0:d]^T (rows c), bf16 hi + lo
 //   litela_bwd_q_tc                        per 128-token tile and head: y = q~ . S^T and
@@ -48,7 +50,61 @@ namespace litela {
 struct BwdPlan {
   int B, N, H, T, nblk, nquads, cpb, chunk;   // cpb CTAs of `chunk` tokens per (batch, quad, block)
   float eps;
+  // fold_fwd > 0: the dq kernel forms its S images itself from the reduction's fold_fwd partial
+  // states per quad (one block only), instead of loading a scan's images; fold_bwd > 0: the
+  // dk/dv kernel forms its dS images from the dq kernel's fold_bwd partials per quad
+  int fold_fwd, fold_bwd;
 };
+
+// The states of one block as a scan over that block's partials forms them (one block: the plain
+// sum of its parts, visited first to last, or last to first for the reverse scan), for the
+// nh * 33 * 32 elements (head j, element e) of this quad's partials at `base` (part k of element
+// (j, e) at base + (k * 4 + j) * 33 * 32 + e).  Threads t = 0..nthreads-1 share the elements, 4
+// at a time with 8 parts each in flight; write(j, r, c, sum, hi, lo) stores one element (row r,
+// column c) with its bf16 hi + lo rounding.
+template <typename Write>
+__device__ __forceinline__ void fold_states(const float* __restrict__ base, int nh, int nparts, bool reverse, int t,
+                                            int nthreads, Write write) {
+  constexpr int kF = 4;
+  constexpr int64_t kStride = (int64_t)kRedHeads * kStateFloats;
+  const int total = nh * kStateFloats;
+  for (int i0 = t; i0 < total; i0 += kF * nthreads) {
+    const float* src[kF];
+    bool ok[kF];
+    float sum[kF];
+#pragma unroll
+    for (int f = 0; f < kF; ++f) {
+      const int i = i0 + f * nthreads;
+      ok[f] = i < total;
+      src[f] = base + (ok[f] ? i : 0);   // (j, e) at j * 33 * 32 + e = i
+      sum[f] = 0.f;
+    }
+    for (int k0 = 0; k0 < nparts; k0 += 8) {
+      float v[kF][8];
+#pragma unroll
+      for (int f = 0; f < kF; ++f)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int k = reverse ? nparts - 1 - (k0 + q) : k0 + q;
+          v[f][q] = (ok[f] && k0 + q < nparts) ? __ldcg(src[f] + k * kStride) : 0.f;
+        }
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (k0 + q < nparts) {
+#pragma unroll
+          for (int f = 0; f < kF; ++f) sum[f] += v[f][q];
+        }
+    }
+#pragma unroll
+    for (int f = 0; f < kF; ++f) {
+      if (!ok[f]) continue;
+      const int i = i0 + f * nthreads, j = i / kStateFloats, e = i - j * kStateFloats;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(sum[f]);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(sum[f] - __bfloat162float(hi));
+      write(j, e >> 5, e & 31, sum[f], hi, lo);
+    }
+  }
+}
 
 enum : int {
   kErrBwdQProducer = 0x510, kErrBwdQMma = 0x520, kErrBwdQRelu = 0x530, kErrBwdQEpi = 0x540,
@@ -177,7 +233,7 @@ template <typename OutT>
 __global__ void __launch_bounds__(kBwThreads, 1)
 litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_g,
                 const __grid_constant__ CUtensorMap tmap_dq, const uint8_t* __restrict__ images,
-                const uint8_t* __restrict__ images_t,
+                const uint8_t* __restrict__ images_t, const float* __restrict__ fold_src,
                 float* __restrict__ dpartials, OutT* __restrict__ dqkv, int* __restrict__ err, BwdPlan p) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
@@ -212,7 +268,7 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       mbar_init(&qrelu[2 * s + 1], kApReluThreads);
       mbar_init(&qempty[s], 1);
     }
-    mbar_init(sfull, 1);
+    mbar_init(sfull, p.fold_fwd > 0 ? kBwEpiThreads : 1);   // the images: the epilogue's fold, or bulk copies
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 128);
@@ -286,7 +342,7 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
       int issued = pre;
       bool images_loaded = false;
       pdl_wait_primary();   // the S images come from the preceding scan
-      if (sp.ntiles > 0) {
+      if (sp.ntiles > 0 && p.fold_fwd == 0) {
         mbar_arrive_expect_tx(sfull, sp.nh * (kImageBytes + kImageTBytes));
         for (int j = 0; j < sp.nh; ++j) {
           const int64_t im = ((int64_t)b * p.H + quad * kApUnitHeads + j) * p.nblk + sp.blk;
@@ -383,6 +439,31 @@ litela_bwd_q_tc(const __grid_constant__ CUtensorMap tmap_q, const __grid_constan
     // stored with TMA by the group's first thread; otherwise each thread stores its row
     uint8_t* dqbuf = smem + kBqOffDq + g * kDqBoxBytes;
     const bool storer = lane == 0 && wq == 0;
+    if (p.fold_fwd > 0 && sp.ntiles > 0) {
+      // the S and S^T images of the quad's heads from the reduction's partial states
+      pdl_wait_primary();
+      const int et = threadIdx.x - 128;
+      fold_states(fold_src + ((int64_t)b * p.nquads + quad) * p.fold_fwd * kRedHeads * kStateFloats, sp.nh,
+                  p.fold_fwd, false, et, kBwEpiThreads,
+                  [&](int j, int r, int c, float, __nv_bfloat16 hi, __nv_bfloat16 lo) {
+                    uint8_t* img = simg + j * kImageBytes;
+                    *reinterpret_cast<__nv_bfloat16*>(img + image_offset(r, c)) = hi;
+                    *reinterpret_cast<__nv_bfloat16*>(img + image_offset(kImageLoRow + r, c)) = lo;
+                    if (r < kD) {
+                      uint8_t* imt = stimg + j * kImageTBytes;
+                      *reinterpret_cast<__nv_bfloat16*>(imt + image_offset(c, r)) = hi;
+                      *reinterpret_cast<__nv_bfloat16*>(imt + image_offset(kD + c, r)) = lo;
+                    }
+                  });
+      for (int i = et; i < sp.nh * (kImageRows - 2 * kRows) * kD; i += kBwEpiThreads) {   // the zero rows
+        const int j = i / ((kImageRows - 2 * kRows) * kD), k = i - j * ((kImageRows - 2 * kRows) * kD);
+        const int zr = k >> 5, c = k & 31, half = kImageLoRow - kRows;
+        const int nrow = zr < half ? kRows + zr : kImageLoRow + kRows + (zr - half);
+        *reinterpret_cast<__nv_bfloat16*>(simg + j * kImageBytes + image_offset(nrow, c)) = __float2bfloat16_rn(0.f);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(sfull);
+    }
     bool ok = sp.ntiles > 0 && mbar_wait(sfull, 0, abort_flag, err, kErrBwdQEpi | 8);
     if (ok && threadIdx.x < 256) ones_rows_fp32(simg, sp.nh, zf, threadIdx.x - 128);
     bar_sync(2, kBwEpiThreads);
@@ -563,7 +644,8 @@ template <typename OutT>
 __global__ void __launch_bounds__(kBwThreads, 1)
 litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_constant__ CUtensorMap tmap_dqkv,
                  const uint8_t* __restrict__ dimages, const uint8_t* __restrict__ dimages_t,
-                 const float* __restrict__ dzrows, OutT* __restrict__ dqkv, int* __restrict__ err, BwdPlan p) {
+                 const float* __restrict__ dzrows, const float* __restrict__ fold_src, OutT* __restrict__ dqkv,
+                 int* __restrict__ err, BwdPlan p) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -593,7 +675,7 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
       mbar_init(&krelu[2 * s + 1], kApReluThreads);
       mbar_init(&kvempty[s], 2);
     }
-    mbar_init(sfull, 1);
+    mbar_init(sfull, p.fold_bwd > 0 ? kBwEpiThreads : 1);   // the images: the epilogue's fold, or bulk copies
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 128);
@@ -631,7 +713,7 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
       int issued = pre;
       bool images_loaded = false;
       pdl_wait_primary();   // the dS images come from the preceding scan
-      if (sp.ntiles > 0) {
+      if (sp.ntiles > 0 && p.fold_bwd == 0) {
         mbar_arrive_expect_tx(sfull, sp.nh * (2 * kImageTBytes + kD * 4));
         for (int j = 0; j < sp.nh; ++j) {
           const int64_t im = ((int64_t)b * p.H + quad * kApUnitHeads + j) * p.nblk + sp.blk;
@@ -712,6 +794,27 @@ litela_bwd_kv_tc(const __grid_constant__ CUtensorMap tmap_kv, const __grid_const
     // epilogue: group g takes heads g, g + 2 through TMEM slot g; thread = token row (TMEM lane)
     const int g = (warp - 4) >> 2, wq = warp & 3, row = wq * 32 + lane;
     const int gbar = 1 + 2 * g;
+    if (p.fold_bwd > 0 && sp.ntiles > 0) {
+      // the dS images (rows 0..d-1 and their transposes) and dS[d] of the quad's heads from the
+      // dq kernel's partials, summed last to first as the reverse scan does
+      pdl_wait_primary();
+      fold_states(fold_src + ((int64_t)b * p.nquads + quad) * p.fold_bwd * kRedHeads * kStateFloats, sp.nh,
+                  p.fold_bwd, true, threadIdx.x - 128, kBwEpiThreads,
+                  [&](int j, int r, int c, float sum, __nv_bfloat16 hi, __nv_bfloat16 lo) {
+                    if (r < kD) {
+                      uint8_t* img = dimg + j * kImageTBytes;
+                      *reinterpret_cast<__nv_bfloat16*>(img + image_offset(r, c)) = hi;
+                      *reinterpret_cast<__nv_bfloat16*>(img + image_offset(kD + r, c)) = lo;
+                      uint8_t* imt = dtimg + j * kImageTBytes;
+                      *reinterpret_cast<__nv_bfloat16*>(imt + image_offset(c, r)) = hi;
+                      *reinterpret_cast<__nv_bfloat16*>(imt + image_offset(kD + c, r)) = lo;
+                    } else {
+                      zf[j * kD + c] = sum;
+                    }
+                  });
+      fence_proxy_async_smem();
+      mbar_arrive(sfull);
+    }
     bool ok = sp.ntiles > 0 && mbar_wait(sfull, 0, abort_flag, err, kErrBwdKvEpi | 8);
     // bf16 results of a whole tile are written over the k and v tiles they came from (each
     // head's columns once its products are done and its mask is read) and stored with TMA:

@@ -253,3 +253,14 @@ def test_forward_form_and_the_paired_minimum(lib):
         ll.lite_la_set_paired_min_chunk(prev)
     # the workspace query follows the form: 8 siblings' partial states per quad when paired
     assert ll.lite_la_workspace_bytes(2, 16384, 70) >= 36 * 8 * 4 * 33 * 32 * 4
+
+
+def test_backward_kernel_count(lib):
+    """With one block per sequence the backward is three kernels (the dq and dk/dv kernels sum
+    the partial states into their images themselves); with more blocks it keeps the two scans
+    (one of them from saved states).  The query needs no GPU."""
+    f = lib.lite_la_bwd_kernels_per_call
+    assert f(2, 16384, 70, 32, 0, 0) == 3 and f(2, 16384, 70, 32, 0, 1) == 3
+    assert f(1, 3000, 9, 32, 3000, 0) == 3 and f(1, 3000, 9, 32, 5000, 1) == 3   # T >= N: one block
+    assert f(1, 16384, 70, 32, 1024, 0) == 5 and f(1, 16384, 70, 32, 1024, 1) == 4
+    assert f(0, 16, 1, 32, 0, 0) == 0 and f(1, 16, 1, 64, 0, 0) == 0
