@@ -346,7 +346,7 @@ litela_status launch_scan(const Plan& plan, const float* partials, uint8_t* imag
                           int chunks_per_block = 0, bool rows64 = false, float* zrows = nullptr) {
   const int64_t work = ((int64_t)plan.B * plan.H * kStateFloats + kScanElems - 1) / kScanElems;
   int64_t grid = (work + kScanThreads - 1) / kScanThreads;
-  if (grid > num_sms) grid = num_sms;
+  if (grid > kScanCtasPerSm * num_sms) grid = kScanCtasPerSm * num_sms;
   TcPlan tp = tc_plan(plan, 0.f);
   if (chunks_per_block > 0) tp.cpb = chunks_per_block;   // partials of another chunking (the backward's)
   cudaError_t e = launch_ex(litela_state_scan, dim3((unsigned)grid), dim3(kScanThreads), 0, stream, pdl,

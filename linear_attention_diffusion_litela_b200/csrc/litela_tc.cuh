@@ -372,13 +372,15 @@ __device__ __forceinline__ const float* partial_ptr(const float* partials, const
 // the images hold only rows 0..31 (hi rows 0..31, lo rows 32..63: kImageTBytes each, no zero
 // rows) and row 32 goes to `zrows` in fp32 ([B][H][nblk][32]).  `state_in` (fp32 [B][H][33][32], may be
 // null) is a state carried from earlier chunks of the sequence and starts every prefix;
-// `state_out` (may be null, may alias state_in) receives the final prefix.  Grid-stride over the state elements
-// with at most one small CTA per SM: its CTAs launch early as a programmatic dependent of the
-// reduction and must leave registers on each SM for the apply's CTAs to land while they wait.
-// Each thread keeps 2 elements x 8 partial loads in flight per round.
+// `state_out` (may be null, may alias state_in) receives the final prefix.  Grid-stride over the state elements,
+// one per thread, with at most kScanCtasPerSm CTAs per SM; each thread keeps 8 partial loads in
+// flight per round.  A thread's work is one long chain (a conversion and stores at every block
+// end), so the scan needs many warps per SM: with one CTA per SM and 2 elements a thread,
+// block-causal calls with many blocks took 3-11 % longer.
 constexpr int kScanThreads = 256;
+constexpr int kScanCtasPerSm = 4;
 constexpr int kScanZeros = 14 * kD;   // zero elements of one image
-constexpr int kScanElems = 2;         // state elements per thread and round
+constexpr int kScanElems = 1;         // state elements per thread and round
 
 __global__ void __launch_bounds__(kScanThreads)
 litela_state_scan(const float* __restrict__ partials, uint8_t* __restrict__ images, uint8_t* __restrict__ images_t,
