@@ -82,7 +82,9 @@ struct FusedCfg {
   static constexpr uint32_t kStage1Bytes = (kMap ? 7 : 4) * kRedBoxBytes;
   static constexpr int kStages1 = kMap ? 4 : 6;                                  // phase-1 ring
   // the block-causal form keeps two state images (its blocks) and, for bf16 output, one q stage less
-  static constexpr int kQStages = (kCausal && sizeof(OutT) == 2) ? A::kQStages - 1 : A::kQStages;
+  // q stages: bf16 output 4 (3 beside the block-causal form's second state buffer), fp32 output
+  // and the ELU + 1 map 2
+  static constexpr int kQStages = kMap ? 2 : (sizeof(OutT) == 2 ? (kCausal ? 3 : 4) : 2);
   static constexpr int kSBufs = kCausal ? 2 : 1;
   static constexpr uint32_t kPhase1Bytes = kStages1 * kStage1Bytes + 512;   // + the ones tile
   static constexpr uint32_t kPhase2Bytes =
