@@ -64,7 +64,8 @@ FORMS_PAIRED = (2, 4)            # lite_la_forward_form: the paired fused forms 
 # brackets the phases.  Per path: the timed phases and their algorithmic bytes (in units of
 # E = B*N*H*d elements).
 PATHS = {
-    # backward (--direction bwd): five kernels in three timed phases; 18 bytes per element
+    # backward (--direction bwd) with more than one block per sequence: five kernels in three
+    # timed phases; 18 bytes per element
     # (k, v read for the state; q, dout read and dq written; k, v read and dk, dv written)
     5: {"phases": ("litela_reduce_tc+litela_state_scan", "litela_bwd_q_tc", "litela_state_scan+litela_bwd_kv_tc"),
         "alg_bytes_E": {"litela_reduce_tc+litela_state_scan": 4, "litela_bwd_q_tc": 6,
