@@ -305,7 +305,7 @@ litela_status validate(const void* qkv, const void* out, size_t out_elem, int B,
 
 TcPlan tc_plan(const Plan& plan, float eps) {
   return TcPlan{plan.B,     plan.N,      plan.H,     plan.T, plan.nblk, plan.ngroups, plan.chunks_per_block,
-                plan.chunk, plan.nquads, plan.tiles_per_block, (long long)plan.units, eps};
+                plan.chunk, plan.nquads, plan.tiles_per_block, (long long)plan.units, eps, plan.red_bpc};
 }
 
 
@@ -333,7 +333,8 @@ litela_status launch_reduce(const Plan& plan, const void* qkv, float* partials, 
   CUtensorMap map;
   litela_status s = encode_qkv_map(qkv, plan.B, plan.N, plan.H, kRedTile, &map);
   if (s != LITELA_OK) return s;
-  cudaError_t e = launch_ex(litela_reduce_tc<kMap>, dim3(plan.nblk * plan.chunks_per_block, plan.ngroups, plan.B),
+  const int xs = plan.red_bpc > 1 ? (plan.nblk + plan.red_bpc - 1) / plan.red_bpc : plan.nblk * plan.chunks_per_block;
+  cudaError_t e = launch_ex(litela_reduce_tc<kMap>, dim3(xs, plan.ngroups, plan.B),
                             dim3(RedCfg<kMap>::kThreads), RedCfg<kMap>::kSmemBytes, stream, pdl, map, partials, err,
                             tc_plan(plan, 0.f));
   if (e != cudaSuccess) return cuda_fail(e, "launch litela_reduce_tc");

@@ -46,6 +46,7 @@ struct Plan {
   int ngroups = 0;           // reduce head groups, ceil(H / 4)
   int chunks_per_block = 0;  // reduce CTAs per (batch, group, block)
   int chunk = 0;             // tokens per reduce CTA (a multiple of kRedTile)
+  int red_bpc = 1;           // consecutive blocks per reduce CTA (> 1 only with one chunk per block)
   int nquads = 0;            // apply head quads, ceil(H / 4)
   int tiles_per_block = 0;   // apply tiles per (batch, quad, block)
   int64_t units = 0;         // apply work units
@@ -106,6 +107,11 @@ inline bool make_plan(int B, int N, int H, int tokens_per_block, int num_sms, Pl
   chunk = (chunk + kRedTile - 1) / kRedTile * kRedTile;
   p->chunk = (int)chunk;
   p->chunks_per_block = (int)((p->T + chunk - 1) / chunk);
+  // one chunk per block and more blocks than the target number of CTAs: a reduction CTA walks
+  // several consecutive blocks (one partial state each) instead of launching a CTA per block
+  const int64_t ctas_per_group = target / ((int64_t)B * p->ngroups) > 0 ? target / ((int64_t)B * p->ngroups) : 1;
+  if (p->chunks_per_block == 1 && p->nblk > ctas_per_group)
+    p->red_bpc = (int)((p->nblk + ctas_per_group - 1) / ctas_per_group);
   p->nquads = (H + kApUnitHeads - 1) / kApUnitHeads;
   p->tiles_per_block = (p->T + kApTile - 1) / kApTile;
   p->units = (int64_t)B * p->nquads * p->nblk * p->tiles_per_block;

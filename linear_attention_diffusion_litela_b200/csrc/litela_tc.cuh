@@ -58,6 +58,7 @@ struct TcPlan {
   int B, N, H, T, nblk, ngroups, cpb, chunk, nquads, tpb;
   long long units;
   float eps;
+  int bpc;   // consecutive blocks per reduction CTA (> 1 only with cpb == 1)
 };
 
 // error codes written to the workspace error word: 0x100 | role << 4 | stage
@@ -171,17 +172,25 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
   uint64_t* full = reinterpret_cast<uint64_t*>(ones + 512);
   uint64_t* relu_done = full + kStages;
   uint64_t* empty = relu_done + kStages;
-  uint64_t* done = empty + kStages;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* done = empty + kStages;      // a block's products are done (one phase per block)
+  uint64_t* tfree = done + 1;            // the epilogue has read a block's accumulator
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tfree + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int x = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int blk = x / p.cpb, ch = x - blk * p.cpb;
-  const int blk_end = min((blk + 1) * p.T, p.N);
-  const int n0 = blk * p.T + ch * p.chunk;
-  const int n1 = min(n0 + p.chunk, blk_end);
-  const int ntiles = n1 > n0 ? (n1 - n0 + kRedTile - 1) / kRedTile : 0;
+  // this CTA's blocks [bb0, bb1) (several only with one chunk per block), its chunk ch of each;
+  // block k's tokens [n0, n1) and 64-token tiles
+  const int bb0 = p.bpc > 1 ? x * p.bpc : x / p.cpb;
+  const int bb1 = p.bpc > 1 ? min(bb0 + p.bpc, p.nblk) : bb0 + 1;
+  const int ch = p.bpc > 1 ? 0 : x - bb0 * p.cpb;
+  auto span = [&](int k, int& n0, int& n1) {
+    n0 = k * p.T + ch * p.chunk;
+    n1 = min(n0 + p.chunk, min((k + 1) * p.T, p.N));
+    return n1 > n0 ? (n1 - n0 + kRedTile - 1) / kRedTile : 0;
+  };
+  int n0, n1;
+  const int ntiles = span(bb0, n0, n1);   // the first block's (the L2 prefetch covers it)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -190,6 +199,7 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
       mbar_init(&empty[s], 1);
     }
     mbar_init(done, 1);
+    mbar_init(tfree, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -239,20 +249,27 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
         else
           tma_load_3d(dst, &tmap, bar, x, y, b);
       };
-      int issued = 0;
-      for (int i = 0; i < ntiles; ++i) {
-        const int s = i % kStages;
-        if (i >= kStages &&
-            !mbar_wait(&empty[s], ((i / kStages) - 1) & 1, abort_flag, err, kErrReduceProducer | s))
-          break;
-        uint8_t* st = stages + s * kStageBytes;
-        const int y = n0 + i * kRedTile;
-        mbar_arrive_expect_tx(&full[s], kRedStageBytes);
-        load(st, &full[s], kx, y);
-        load(st + kRedBoxBytes, &full[s], kx + 64, y);
-        load(st + 2 * kRedBoxBytes, &full[s], vx, y);
-        load(st + 3 * kRedBoxBytes, &full[s], vx + 64, y);
-        issued = i + 1;
+      int issued = 0, i = 0;
+      bool stop = false;
+      for (int k = bb0; k < bb1 && !stop; ++k) {
+        int a0, a1;
+        const int nt = span(k, a0, a1);
+        for (int j = 0; j < nt; ++j, ++i) {
+          const int s = i % kStages;
+          if (i >= kStages &&
+              !mbar_wait(&empty[s], ((i / kStages) - 1) & 1, abort_flag, err, kErrReduceProducer | s)) {
+            stop = true;
+            break;
+          }
+          uint8_t* st = stages + s * kStageBytes;
+          const int y = a0 + j * kRedTile;
+          mbar_arrive_expect_tx(&full[s], kRedStageBytes);
+          load(st, &full[s], kx, y);
+          load(st + kRedBoxBytes, &full[s], kx + 64, y);
+          load(st + 2 * kRedBoxBytes, &full[s], vx, y);
+          load(st + 3 * kRedBoxBytes, &full[s], vx + 64, y);
+          issued = i + 1;
+        }
       }
       if (*abort_flag) {   // let the copies still in flight land before the CTA exits (bounded)
         for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
@@ -264,85 +281,111 @@ litela_reduce_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ p
       constexpr uint32_t idesc_num = idesc_bf16_f32(128, 128, true, true);
       constexpr uint32_t idesc_den = idesc_bf16_f32(128, 16, true, false);
       const uint64_t ones_desc = smem_desc(smem_u32(ones), 128, 256, kSwizzleNone);
-      for (int i = 0; i < ntiles; ++i) {
-        const int s = i % kStages;
-        if (!mbar_wait(&relu_done[s], (i / kStages) & 1, abort_flag, err, kErrReduceMma | s)) break;
-        tc_fence_after_sync();
-        const uint32_t kbase = smem_u32(stages + s * kStageBytes);
-        const uint32_t vbase = kbase + 2 * kRedBoxBytes;
-#pragma unroll
-        for (int ks = 0; ks < kRedTile / 16; ++ks) {
-          // MN-major, 128B swizzle: 8-token row groups 1024 B apart, 64-channel blocks one box apart
-          const uint64_t a = smem_desc(kbase + ks * 2048, kRedBoxBytes, 1024, kSwizzle128B);
-          const uint64_t bv = smem_desc(vbase + ks * 2048, kRedBoxBytes, 1024, kSwizzle128B);
-          const uint32_t acc = (i | ks) != 0;
-          umma_bf16(tmem, a, bv, idesc_num, acc);
-          umma_bf16(tmem + 128, a, ones_desc, idesc_den, acc);
-          if (kMap) {   // the lo halves of phi(k)
-            const uint64_t al = smem_desc(kbase + 4 * kRedBoxBytes + ks * 2048, kRedBoxBytes, 1024, kSwizzle128B);
-            umma_bf16(tmem, al, bv, idesc_num, 1u);
-            umma_bf16(tmem + 128, al, ones_desc, idesc_den, 1u);
+      int i = 0;
+      bool stop = false;
+      for (int k = bb0; k < bb1 && !stop; ++k) {
+        int a0, a1;
+        const int nt = span(k, a0, a1);
+        // the accumulator is overwritten by this block's first product: the epilogue has read
+        // the previous block's
+        if (k > bb0 && !mbar_wait(tfree, (k - bb0 - 1) & 1, abort_flag, err, kErrReduceMma | 8)) break;
+        for (int j = 0; j < nt; ++j, ++i) {
+          const int s = i % kStages;
+          if (!mbar_wait(&relu_done[s], (i / kStages) & 1, abort_flag, err, kErrReduceMma | s)) {
+            stop = true;
+            break;
           }
+          tc_fence_after_sync();
+          const uint32_t kbase = smem_u32(stages + s * kStageBytes);
+          const uint32_t vbase = kbase + 2 * kRedBoxBytes;
+#pragma unroll
+          for (int ks = 0; ks < kRedTile / 16; ++ks) {
+            // MN-major, 128B swizzle: 8-token row groups 1024 B apart, 64-channel blocks one box apart
+            const uint64_t a = smem_desc(kbase + ks * 2048, kRedBoxBytes, 1024, kSwizzle128B);
+            const uint64_t bv = smem_desc(vbase + ks * 2048, kRedBoxBytes, 1024, kSwizzle128B);
+            const uint32_t acc = (j | ks) != 0;
+            umma_bf16(tmem, a, bv, idesc_num, acc);
+            umma_bf16(tmem + 128, a, ones_desc, idesc_den, acc);
+            if (kMap) {   // the lo halves of phi(k)
+              const uint64_t al = smem_desc(kbase + 4 * kRedBoxBytes + ks * 2048, kRedBoxBytes, 1024, kSwizzle128B);
+              umma_bf16(tmem, al, bv, idesc_num, 1u);
+              umma_bf16(tmem + 128, al, ones_desc, idesc_den, 1u);
+            }
+          }
+          umma_commit(&empty[s]);
         }
-        umma_commit(&empty[s]);
+        if (!stop) umma_commit(done);
       }
-      umma_commit(done);
     }
   } else {
     constexpr int kMapThreads = 32 * RedCfg<kMap>::kMapWarps;
     const int t = threadIdx.x - 64;
-    for (int i = 0; i < ntiles; ++i) {
-      const int s = i % kStages;
-      if (!mbar_wait(&full[s], (i / kStages) & 1, abort_flag, err, kErrReduceRelu | s)) break;
-      uint8_t* st = stages + s * kStageBytes;
-      const int valid = min(kRedTile, n1 - (n0 + i * kRedTile));   // tokens of this chunk in the tile
-#pragma unroll 4
-      for (int j = t; j < 1024; j += kMapThreads) {   // k: 2 boxes x 64 rows x 8 chunks of 16 B
-        uint4* c = reinterpret_cast<uint4*>(st + j * 16);
-        const int row = (j >> 3) & (kRedTile - 1);
-        if (kMap == 0) {
-          *c = row < valid ? relu_bf16x8(*c) : make_uint4(0u, 0u, 0u, 0u);
-        } else {
-          uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
-          if (row < valid) phi_elu1_hilo(*c, 1.0f, hi, lo);
-          *c = hi;
-          *reinterpret_cast<uint4*>(st + 4 * kRedBoxBytes + j * 16) = lo;
-        }
-      }
-      if (valid < kRedTile) {
-        for (int j = t; j < 1024; j += kMapThreads) {
-          const int row = (j >> 3) & (kRedTile - 1);
-          if (row >= valid) *reinterpret_cast<uint4*>(st + 2 * kRedBoxBytes + j * 16) = make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&relu_done[s]);
-    }
-    // epilogue (warps 2..5): warp quarter q reads TMEM lanes 32q..32q+31 = head q's key channels c
-    if (warp < 6) {
-    const int q = warp & 3;
-    float sv[kRows];
-    bool ok = ntiles > 0;
-    if (ok) ok = mbar_wait(done, 0, abort_flag, err, kErrReduceEpi);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
-      tc_fence_after_sync();
-      uint32_t r[32], zr;
-      const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16);
-      tmem_ld_x32(ta + q * 32, r);
-      tmem_ld_x1(ta + 128, zr);
-      tmem_wait_ld();
-#pragma unroll
-      for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(r[j]);
-      sv[32] = __uint_as_float(zr);
-    } else {
-#pragma unroll
-      for (int j = 0; j < kRows; ++j) sv[j] = 0.f;
-    }
     const int64_t nparts = (int64_t)p.nblk * p.cpb;
-    float* dst = partials + ((((int64_t)b * p.ngroups + g) * nparts + x) * kRedHeads + q) * kStateFloats;
+    int i = 0;
+    bool ok = true;
+    for (int k = bb0; k < bb1; ++k) {
+      int a0, a1;
+      const int nt = span(k, a0, a1);
+      for (int j = 0; ok && j < nt; ++j, ++i) {
+        const int s = i % kStages;
+        if (!mbar_wait(&full[s], (i / kStages) & 1, abort_flag, err, kErrReduceRelu | s)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = stages + s * kStageBytes;
+        const int valid = min(kRedTile, a1 - (a0 + j * kRedTile));   // tokens of this chunk in the tile
+#pragma unroll 4
+        for (int w = t; w < 1024; w += kMapThreads) {   // k: 2 boxes x 64 rows x 8 chunks of 16 B
+          uint4* c = reinterpret_cast<uint4*>(st + w * 16);
+          const int row = (w >> 3) & (kRedTile - 1);
+          if (kMap == 0) {
+            *c = row < valid ? relu_bf16x8(*c) : make_uint4(0u, 0u, 0u, 0u);
+          } else {
+            uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
+            if (row < valid) phi_elu1_hilo(*c, 1.0f, hi, lo);
+            *c = hi;
+            *reinterpret_cast<uint4*>(st + 4 * kRedBoxBytes + w * 16) = lo;
+          }
+        }
+        if (valid < kRedTile) {
+          for (int w = t; w < 1024; w += kMapThreads) {
+            const int row = (w >> 3) & (kRedTile - 1);
+            if (row >= valid) *reinterpret_cast<uint4*>(st + 2 * kRedBoxBytes + w * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&relu_done[s]);
+      }
+      // epilogue (warps 2..5): block k's partial state; warp quarter q reads TMEM lanes
+      // 32q..32q+31 = head q's key channels c, then frees the accumulator for the next block
+      if (warp < 6) {
+        const int q = warp & 3;
+        float sv[kRows];
+        bool got = ok && nt > 0;
+        if (got) got = mbar_wait(done, (k - bb0) & 1, abort_flag, err, kErrReduceEpi);
+        got = __all_sync(0xffffffffu, got);
+        if (got) {
+          tc_fence_after_sync();
+          uint32_t r[32], zr;
+          const uint32_t ta = tmem + (static_cast<uint32_t>(q * 32) << 16);
+          tmem_ld_x32(ta + q * 32, r);
+          tmem_ld_x1(ta + 128, zr);
+          tmem_wait_ld();
 #pragma unroll
-    for (int j = 0; j < kRows; ++j) dst[j * kD + lane] = sv[j];   // S[r = j][c = lane]
+          for (int jj = 0; jj < 32; ++jj) sv[jj] = __uint_as_float(r[jj]);
+          sv[32] = __uint_as_float(zr);
+        } else {
+#pragma unroll
+          for (int jj = 0; jj < kRows; ++jj) sv[jj] = 0.f;
+        }
+        tc_fence_before_sync();
+        mbar_arrive(tfree);
+        float* dst = partials + ((((int64_t)b * p.ngroups + g) * nparts + (int64_t)k * p.cpb + ch) * kRedHeads + q) *
+                                    kStateFloats;
+#pragma unroll
+        for (int jj = 0; jj < kRows; ++jj) dst[jj * kD + lane] = sv[jj];   // S[r = jj][c = lane]
+      }
+      if (!ok) break;
     }
   }
 
