@@ -182,6 +182,20 @@ def test_block_causal_workload_sampled(mode):
     assert_close(got, oracle_run(qkv, w["H"], T=T, rows=rows), mode)
 
 
+@pytest.mark.parametrize("T", [512, 256])
+@pytest.mark.parametrize("mode", ["bf16", "f32"])
+def test_block_causal_short_blocks_sampled(T, mode):
+    """Short blocks at the 4096px token count (N = 16384, H = 70): more blocks than the
+    reduction has CTAs, so each reduction CTA walks several consecutive blocks (three-kernel
+    path); sampled rows, block edges among them, against the oracle."""
+    B, N, H = 1, 16384, 70
+    assert ll.lite_la_forward_form(B, N, H, 32, T) == "three_kernel"
+    qkv = make_qkv(B, N, H, 32, seed=1005 + T, device="cuda")
+    rows = sample_rows(N, T=T, k=48, seed=7)
+    got = gpu_run(qkv, H, T=T, mode=mode)[:, rows]
+    assert_close(got, oracle_run(qkv, H, T=T, rows=rows), mode)
+
+
 def test_hand_worked_example_padded_to_d32():
     """The golden d=2 example embedded in channels 0..1 of a d=32 head (other channels 0)."""
     from tests.test_golden import as_float, load_golden

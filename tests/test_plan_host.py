@@ -22,7 +22,7 @@ SHAPES = [(2, 16384, 70), (2, 4096, 70), (2, 1024, 70), (1, 256, 36), (1, 2048, 
 # block-causal (B, N, H, T)
 CAUSAL = [(1, 16384, 70, 1024), (2, 16384, 70, 1024), (1, 8192, 70, 1024), (1, 2048, 40, 128), (1, 2100, 40, 128),
           (3, 1024, 30, 128), (2, 700, 70, 128), (2, 640, 66, 128), (1, 1000, 8, 128), (1, 16384, 70, 512),
-          (1, 4096, 70, 512), (1, 300, 8, 100), (2, 8192, 36, 1024)]
+          (1, 4096, 70, 512), (1, 300, 8, 100), (2, 8192, 36, 1024), (1, 16384, 70, 256), (1, 300, 5, 1)]
 
 DRIVER = r"""
 #include <cstdio>
@@ -33,9 +33,10 @@ int main(int argc, char** argv) {
     litela::Plan p;
     litela::make_plan(atoi(argv[i]), atoi(argv[i + 1]), atoi(argv[i + 2]), atoi(argv[i + 3]), 148, &p, min_chunk);
     printf("{\"fused\": %d, \"paired\": %d, \"causal\": %d, \"nquads\": %d, \"ntiles\": %d, \"S\": %d, "
-           "\"chunk\": %d, \"bytes\": %zu, \"counters\": %zu, \"cpb\": %d, \"bpc\": %d, \"nblk\": %d}\n",
+           "\"chunk\": %d, \"bytes\": %zu, \"counters\": %zu, \"cpb\": %d, \"bpc\": %d, \"nblk\": %d, "
+           "\"red_cpb\": %d, \"red_bpc\": %d, \"ngroups\": %d}\n",
            p.fused, p.fused_paired, p.fused_causal, p.nquads, p.fused_ntiles, p.paired_cpb, p.paired_chunk,
-           p.paired_bytes, p.counters, p.fused_cpb, p.fused_bpc, p.nblk);
+           p.paired_bytes, p.counters, p.fused_cpb, p.fused_bpc, p.nblk, p.chunks_per_block, p.red_bpc, p.ngroups);
   }
   return 0;
 }
@@ -143,3 +144,26 @@ def test_paired_block_causal_form_and_its_partition(plans):
         assert all(x == 1 for row in red for x in row)
         assert all(x == 1 for row in app for x in row)
     assert causal[(1, 16384, 70, 1024)]["paired"]   # the 16 x 1024 workload: 18 quads x 8 siblings
+
+
+def test_reduction_walks_several_blocks_per_cta_when_blocks_are_short(plans):
+    """With one chunk per block and more (batch, group, block) units than two CTAs per SM, a
+    reduction CTA walks red_bpc consecutive blocks: the grid is at most one wave and covers
+    every block of every (batch, group) once."""
+    _, _, causal = plans
+    seen_multi = False
+    for (B, N, H, T), p in causal.items():
+        units = B * p["ngroups"] * p["nblk"]
+        if p["red_bpc"] == 1:
+            assert p["red_cpb"] > 1 or units <= 2 * 148 or p["nblk"] <= (2 * 148) // (B * p["ngroups"])
+            continue
+        seen_multi = True
+        assert p["red_cpb"] == 1
+        per_group = -(-p["nblk"] // p["red_bpc"])
+        assert B * p["ngroups"] * per_group <= 2 * 148
+        cover = [0] * p["nblk"]
+        for x in range(per_group):
+            for k in range(x * p["red_bpc"], min((x + 1) * p["red_bpc"], p["nblk"])):
+                cover[k] += 1
+        assert all(c == 1 for c in cover), (B, N, H, T)
+    assert seen_multi
