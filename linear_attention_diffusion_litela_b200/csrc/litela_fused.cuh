@@ -56,15 +56,17 @@ constexpr uint32_t kFuTmemCols = 512;
 
 // kMap 0: LiteLA (ReLU, + eps).  kMap 1: the ELU + 1 variant (non-causal form only): phi formed
 // in fp32 and entered as bf16 hi + lo (phase 1: phi(k) lo boxes after each stage's k|v boxes;
-// phase 2: phi(q) / sqrt(d) lo boxes after each q stage's hi boxes), 8 feature-map warps in
+// phase 2: phi(q) / sqrt(d) lo boxes after each q stage's hi boxes), 12 feature-map warps in
 // each phase, the denominator clamped from below instead of + eps.
 template <typename OutT, bool kCausal = false, int kMap = 0>
 struct FusedCfg {
   using A = ApplyCfg<OutT, kMap>;
   // warps: 0 TMA, 1 MMA; phase 1: 2 .. 2 + kMapWarps1 feature map (warps 2..5 also read the
   // accumulators); phase 2: 2 .. kEpiWarp0 feature map, then 4 merge / epilogue warps
-  static constexpr int kMapWarps1 = kMap ? 8 : 4;
-  static constexpr int kMapWarps2 = kMap ? 8 : 2;
+  // the ELU + 1 map is latency-bound per warp: 12 warps measured faster than 8 (4096px 183.3 ->
+  // 176.2 us, 2048px 55.1 -> 53.8 us), 10 and 16 no faster
+  static constexpr int kMapWarps1 = kMap ? 12 : 4;
+  static constexpr int kMapWarps2 = kMap ? 12 : 2;
   static constexpr int kEpiWarp0 = 2 + kMapWarps2;
   // apply epilogue: groups of 4 warps, group g taking head pair g of every tile.  Two groups
   // measured faster for the non-causal form (2048px 36.9 -> 36.1 us, 1024px 16.9 -> 16.5 us,
@@ -72,9 +74,9 @@ struct FusedCfg {
   // N = 8192, T = 1024); the ELU + 1 form's feature-map warps leave no registers for a second
   static constexpr int kEpiGroups = (kMap || kCausal) ? 1 : 2;
   static constexpr int kThreads = 32 * (kEpiWarp0 + 4 * kEpiGroups);
-  // launch bound: with 448 threads it keeps ptxas at 128 registers (4 warps share an SM
-  // sub-partition's 16K registers); with 384, at 168
-  static constexpr int kLaunchBound = kMap ? 512 : (kEpiGroups == 2 ? 384 : 256);
+  // launch bound: the ELU + 1 form's 576 threads (ptxas: 96 registers, a few spilled); the
+  // ReLU form's 384 threads with two epilogue groups (at most 168 registers), else 256
+  static constexpr int kLaunchBound = kMap ? 576 : (kEpiGroups == 2 ? 384 : 256);
   // phase-1 stage: k | v boxes; for ELU + 1 also a box of ones right after v (so that one
   // N = 144 product gives the numerator and the denominator: the tensor core pays per
   // instruction, and phi's hi + lo halves would otherwise double four products per 16 tokens)
