@@ -63,10 +63,11 @@ struct FusedCfg {
   using A = ApplyCfg<OutT, kMap>;
   // warps: 0 TMA, 1 MMA; phase 1: 2 .. 2 + kMapWarps1 feature map (warps 2..5 also read the
   // accumulators); phase 2: 2 .. kEpiWarp0 feature map, then 4 merge / epilogue warps
-  // the ELU + 1 map is latency-bound per warp: 12 warps measured faster than 8 (4096px 183.3 ->
-  // 176.2 us, 2048px 55.1 -> 53.8 us), 10 and 16 no faster
-  static constexpr int kMapWarps1 = kMap ? 12 : 4;
-  static constexpr int kMapWarps2 = kMap ? 12 : 2;
+  // the feature maps are latency-bound per warp: the ELU + 1 map with 12 warps against 8
+  // (4096px 183.3 -> 176.2 us, 2048px 55.1 -> 53.8 us; 10 and 16 no faster), ReLU with 8 warps
+  // in phase 1 and 4 in phase 2 against 4 and 2 (2048px 35.0 -> 32.1 us, 1024px 16.1 -> 15.9 us)
+  static constexpr int kMapWarps1 = kMap ? 12 : 8;
+  static constexpr int kMapWarps2 = kMap ? 12 : 4;
   static constexpr int kEpiWarp0 = 2 + kMapWarps2;
   // apply epilogue: groups of 4 warps, group g taking head pair g of every tile.  Two groups
   // measured faster for the non-causal form (2048px 36.9 -> 36.1 us, 1024px 16.9 -> 16.5 us,
@@ -75,8 +76,11 @@ struct FusedCfg {
   static constexpr int kEpiGroups = (kMap || kCausal) ? 1 : 2;
   static constexpr int kThreads = 32 * (kEpiWarp0 + 4 * kEpiGroups);
   // launch bound: the ELU + 1 form's 576 threads (ptxas: 96 registers, a few spilled); the
-  // ReLU form's 384 threads with two epilogue groups (at most 168 registers), else 256
-  static constexpr int kLaunchBound = kMap ? 576 : (kEpiGroups == 2 ? 384 : 256);
+  // ReLU form's 448 threads with two epilogue groups, else 320
+  static constexpr int kLaunchBound = kMap ? 576 : (kEpiGroups == 2 ? 448 : 320);
+  // the phase-1 map warps 2 .. 2 + kMapWarps1 - 1 are warps of the block (a form with fewer
+  // threads would leave the map's barrier short of arrivals)
+  static_assert(2 + kMapWarps1 <= kThreads / 32 && kThreads <= kLaunchBound, "phase-1 map warps");
   // phase-1 stage: k | v boxes; for ELU + 1 also a box of ones right after v (so that one
   // N = 144 product gives the numerator and the denominator: the tensor core pays per
   // instruction, and phi's hi + lo halves would otherwise double four products per 16 tokens)
