@@ -85,6 +85,11 @@ struct PairedCfg {
   static constexpr int kPrefetchTiles = 8;
 };
 static_assert(kRedStageBytes == 2 * kQBoxBytes, "a k|v stage and a q stage take the same ring slot");
+// the ReLU role is warps 2..5 (128 threads: its loops and its barrier count), then 4 merge and 4
+// epilogue warps (any 4 consecutive warps cover the four TMEM lane quarters)
+static_assert(PairedCfg<__nv_bfloat16>::kMergeWarp0 == 6 && PairedCfg<__nv_bfloat16>::kEpiWarp0 == 10 &&
+                  PairedCfg<__nv_bfloat16>::kThreads == 32 * 14 && PairedCfg<float>::kThreads == 32 * 14,
+              "paired kernel warp roles");
 static_assert(kApSbufBytes <= kRedStageBytes, "unit 1's image fits one stage");
 static_assert(PairedCfg<__nv_bfloat16>::kAcc1Col + 144 <= kFuTmemCols, "TMEM columns");
 

@@ -133,6 +133,8 @@ struct RedCfg {
   // accumulators at the end
   static constexpr int kMapWarps = kMap ? 8 : 4;
   static constexpr int kThreads = 32 * (2 + kMapWarps);
+  // the read-out warps 2..5 cover the four TMEM lane quarters and are all map warps
+  static_assert(kMapWarps >= 4, "reduction read-out warps");
 };
 
 // exp by the hardware approximation (__expf, ~2^-21 relative error here): far inside the
